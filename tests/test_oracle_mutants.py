@@ -1,0 +1,115 @@
+"""The pins must catch plausible mistakes in the oracle.
+
+Each case plants one mistake in a copy of gdn_oracle.c (on the CPU, in a
+temporary directory), loads the mutant in place of the real oracle and runs
+every pin of test_oracle_pins.py against it.  At least one pin must fail.
+"""
+import ctypes
+import inspect
+import os
+import subprocess
+
+import pytest
+
+from oracle import oracle as O
+import tests.test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(O.__file__), "gdn_oracle.c")
+
+# (name, original text, mutated text)
+MUTANTS = [
+    ("decay_after_read",  # the read uses the undecayed state
+     "  for (size_t x = 0; x < (size_t)dk * dv; ++x) S[x] *= alpha;\n  for (int j = 0; j < dv; ++j) kv[j] = 0.0;\n  for (int i = 0; i < dk; ++i)\n    for (int j = 0; j < dv; ++j) kv[j] += S[(size_t)i * dv + j] * k[i];\n",
+     "  for (int j = 0; j < dv; ++j) kv[j] = 0.0;\n  for (int i = 0; i < dk; ++i)\n    for (int j = 0; j < dv; ++j) kv[j] += S[(size_t)i * dv + j] * k[i];\n  for (size_t x = 0; x < (size_t)dk * dv; ++x) S[x] *= alpha;\n"),
+    ("readout_transposed",  # o_i = sum_j S_ij q_j on a square state
+     "    for (int j = 0; j < dv; ++j) o[j] += S[(size_t)i * dv + j] * q[i];",
+     "    for (int j = 0; j < dv; ++j) o[j] += S[(size_t)j * dv + i] * q[j < dk ? j : 0];"),
+    ("beta_dropped",
+     "kv[j] = beta * (v[j] - kv[j]);", "kv[j] = (v[j] - kv[j]);"),
+    ("delta_sign",
+     "kv[j] = beta * (v[j] - kv[j]);", "kv[j] = beta * (v[j] + kv[j]);"),
+    ("readout_before_write",  # o uses S' instead of S_t
+     "  for (int j = 0; j < dv; ++j) kv[j] = beta * (v[j] - kv[j]);\n  for (int i = 0; i < dk; ++i)\n    for (int j = 0; j < dv; ++j) S[(size_t)i * dv + j] += k[i] * kv[j];\n  for (int j = 0; j < dv; ++j) o[j] = 0.0;\n  for (int i = 0; i < dk; ++i)\n    for (int j = 0; j < dv; ++j) o[j] += S[(size_t)i * dv + j] * q[i];\n",
+     "  for (int j = 0; j < dv; ++j) kv[j] = beta * (v[j] - kv[j]);\n  for (int j = 0; j < dv; ++j) o[j] = 0.0;\n  for (int i = 0; i < dk; ++i)\n    for (int j = 0; j < dv; ++j) o[j] += S[(size_t)i * dv + j] * q[i];\n  for (int i = 0; i < dk; ++i)\n    for (int j = 0; j < dv; ++j) S[(size_t)i * dv + j] += k[i] * kv[j];\n"),
+    ("gate_sign", "*g = -exp(A_log) * softplus(a + dt_bias);",
+     "*g = exp(A_log) * softplus(a + dt_bias);"),
+    ("gate_no_exp", "*g = -exp(A_log) * softplus(a + dt_bias);",
+     "*g = -A_log * softplus(a + dt_bias);"),
+    ("softplus_threshold", "  if (x > 0.0) return x + log1p(exp(-x));",
+     "  if (x > 20.0) return x;\n  if (x > 0.0) return x + log1p(exp(-x));"),
+    ("beta_sigmoid_sign", "static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }",
+     "static double sigmoid(double x) { return 1.0 / (1.0 + exp(x)); }"),
+    ("norm_no_eps", "double inv = 1.0 / sqrt(ss + 1e-6);", "double inv = 1.0 / sqrt(ss);"),
+    ("scale_on_k", "load_vec(k, in_f64, (row * Hk + hk) * dk, dk, l2norm, 1.0, kt);",
+     "load_vec(k, in_f64, (row * Hk + hk) * dk, dk, l2norm, scale, kt);"),
+    ("gqa_modulo", "hk = hv / group;\n    double* S", "hk = hv % Hk;\n    double* S"),
+    ("conv_taps_reversed",
+     "    double acc = ld(conv_w, in_f64, (size_t)c * 4 + 0) * cs[c * 3 + 0] +",
+     "    double acc = ld(conv_w, in_f64, (size_t)c * 4 + 3) * cs[c * 3 + 0] +"),
+    ("conv_no_shift", "    cs[c * 3 + 0] = cs[c * 3 + 1];\n", "\n"),
+    ("gdn2_decay_value_side",
+     "        for (int j = 0; j < dv; ++j) S[(size_t)i * dv + j] *= dec[i];",
+     "        for (int j = 0; j < dv; ++j) S[(size_t)i * dv + j] *= dec[j < dk ? j : 0];"),
+    ("gdn2_erase_unscaled", "        et[i] = bi_ * kt[i];", "        et[i] = kt[i];"),
+    ("gdn2_write_ungated", "        zt[j] = wj * vt[j];", "        zt[j] = vt[j];"),
+]
+
+PIN_TESTS = [(n, f) for n, f in inspect.getmembers(pins, inspect.isfunction)
+             if n.startswith("test_")]
+
+
+def _build_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    mutated = src.replace(old, new)
+    c = tmp_path / f"{name}.c"
+    so = tmp_path / f"lib{name}.so"
+    c.write_text(mutated)
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-w", "-o",
+                    str(so), str(c), "-lm"], check=True)
+    return str(so)
+
+
+def _run_pins_against(lib_path):
+    """Run every pin with the oracle's library swapped for lib_path; count failures."""
+    real = O._load()
+    mutant = ctypes.CDLL(lib_path)
+    for fname in ("oracle_gdn_fwd", "oracle_gate_prep", "oracle_conv_step",
+                  "oracle_gdn_decode_step", "oracle_gdn2_fwd"):
+        getattr(mutant, fname).argtypes = getattr(real, fname).argtypes
+        getattr(mutant, fname).restype = ctypes.c_int
+    mutant.oracle_max_threads.restype = ctypes.c_int
+    failed = []
+    O._lib = mutant
+    try:
+        for n, f in PIN_TESTS:
+            params = inspect.signature(f).parameters
+            marks = getattr(f, "pytestmark", [])
+            argsets = [{}]
+            for m in marks:
+                if m.name == "parametrize":
+                    names = [s.strip() for s in m.args[0].split(",")]
+                    argsets = [dict(zip(names, v if isinstance(v, tuple) else (v,)))
+                               for v in m.args[1]]
+            assert all(set(a) == set(params) for a in argsets), n
+            for a in argsets:
+                try:
+                    f(**a)
+                except Exception:  # noqa: BLE001 - any failure counts as caught
+                    failed.append(n)
+                    break
+    finally:
+        O._lib = real
+    return failed
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, old, new):
+    lib = _build_mutant(tmp_path, name, old, new)
+    failed = _run_pins_against(lib)
+    assert failed, f"no pin caught the planted mistake '{name}'"
+
+
+def test_unmutated_copy_passes_all_pins(tmp_path):
+    lib = _build_mutant(tmp_path, "identity", "#include <math.h>", "#include <math.h>")
+    assert _run_pins_against(lib) == []

@@ -1,0 +1,358 @@
+"""Pins of the fp64 oracle against facts the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a hand-worked
+example, a closed form, an invariant, a special case that reduces to a textbook
+computation or a library routine, or an independent formulation of the same
+recurrence.  Together they are chosen so that a dropped term, a wrong sign, a
+transposed operand, a misplaced decay or a wrong head mapping fails at least one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(12345)
+
+
+def _rand(*shape):
+    return rng.standard_normal(shape)
+
+
+# --------------------------------------------------------------------------
+# Worked examples (derived by hand, derivations stored beside the values)
+# --------------------------------------------------------------------------
+
+def test_worked_example_gdn_2x2():
+    """Qwen3.5 page, GDN详解 five-step recurrence, three tokens by hand."""
+    f = json.load(open(os.path.join(GOLDEN, "gdn_worked_2x2.json")))
+    T = len(f["g"])
+    q = np.array(f["q"]).reshape(1, T, 1, 2)
+    k = np.array(f["k"]).reshape(1, T, 1, 2)
+    v = np.array(f["v"]).reshape(1, T, 1, 2)
+    g = np.array(f["g"]).reshape(1, T, 1)
+    beta = np.array(f["beta"]).reshape(1, T, 1)
+    h0 = np.array(f["h0"]).reshape(1, 1, 2, 2)
+    o, ht = O.gdn_fwd(q, k, v, g, beta, h0=h0, scale=1.0, l2norm=False, gates_given=True)
+    np.testing.assert_allclose(o[0, :, 0], np.array(f["o"]), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(ht[0, 0], np.array(f["ht"]), rtol=0, atol=1e-14)
+
+
+def test_worked_example_gdn2_2x2():
+    """Gated DeltaNet-2 page, 新更新公式, two tokens by hand."""
+    f = json.load(open(os.path.join(GOLDEN, "gdn2_worked_2x2.json")))
+    T = len(f["g"])
+    sh = (1, T, 1, 2)
+    q, k, v = (np.array(f[n]).reshape(sh) for n in ("q", "k", "v"))
+    g, b, w = (np.array(f[n]).reshape(sh) for n in ("g", "b", "w"))
+    h0 = np.array(f["h0"]).reshape(1, 1, 2, 2)
+    o, ht = O.gdn2_fwd(q, k, v, g, b, w, h0=h0, scale=1.0, l2norm=False, gates_given=True)
+    np.testing.assert_allclose(o[0, :, 0], np.array(f["o"]), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(ht[0, 0], np.array(f["ht"]), rtol=0, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Special cases that reduce to textbook computations
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dk,dv,T", [(4, 3, 9), (16, 8, 33)])
+def test_linear_attention_bruteforce(dk, dv, T):
+    """No decay, no erase, full write: S_t = S_{t-1} + k_t v_t^T and o_t = S_t^T q_t,
+    which equals causal (Q K^T (.) M) V with M lower-triangular including the
+    diagonal ("从 Full Attention 到 Gated DeltaNet" sections 2-3; "Qwen3.5" GDN演进 1)."""
+    q, k, v = _rand(1, T, 1, dk), _rand(1, T, 1, dk), _rand(1, T, 1, dv)
+    zeros_k = np.zeros((1, T, 1, dk))
+    ones_v = np.ones((1, T, 1, dv))
+    o, ht = O.gdn2_fwd(q, k, v, zeros_k, zeros_k, ones_v, scale=1.0, l2norm=False,
+                       gates_given=True)
+    Q, K, V = q[0, :, 0], k[0, :, 0], v[0, :, 0]
+    ref = (np.tril(Q @ K.T)) @ V
+    np.testing.assert_allclose(o[0, :, 0], ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ht[0, 0], K.T @ V, rtol=1e-12, atol=1e-12)
+    # the same special case reached through the logit parameterisation with
+    # IEEE infinities: D = exp(-exp(-inf)*softplus(.)) = 1, sigmoid(-inf) = 0,
+    # sigmoid(+inf) = 1.
+    A_log = np.full((1, dk), -np.inf)
+    dt_bias = np.zeros((1, dk))
+    o2, ht2 = O.gdn2_fwd(q, k, v, _rand(1, T, 1, dk), np.full((1, T, 1, dk), -np.inf),
+                         np.full((1, T, 1, dv), np.inf), A_log, dt_bias, scale=1.0,
+                         l2norm=False)
+    np.testing.assert_allclose(o2[0, :, 0], ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ht2[0, 0], K.T @ V, rtol=1e-12, atol=1e-12)
+
+
+def test_delta_overwrite_orthonormal_keys():
+    """alpha = 1, beta = 1, orthonormal keys: rewriting a key returns exactly the
+    new value and leaves the other key's value alone ("从 Full Attention 到 Gated
+    DeltaNet" section 5 exact retrieval, section 7 overwrite when beta|k|^2 = 1)."""
+    d = 8
+    Qm, _ = np.linalg.qr(_rand(d, d))
+    k1, k2 = Qm[0], Qm[1]
+    v1, v2, v1n = _rand(d), _rand(d), _rand(d)
+    ks = np.stack([k1, k2, k1, k1, k2])
+    vs = np.stack([v1, v2, v1n, _rand(d), _rand(d)])
+    qs = np.stack([k2, k1, k1, k2, k1])
+    beta = np.array([1.0, 1.0, 1.0, 0.0, 0.0])
+    g = np.zeros(5)
+    o, ht = O.gdn_fwd(qs[None, :, None], ks[None, :, None], vs[None, :, None],
+                      g[None, :, None], beta[None, :, None], scale=1.0, l2norm=False,
+                      gates_given=True)
+    o = o[0, :, 0]
+    np.testing.assert_allclose(o[0], np.zeros(d), atol=1e-12)  # k2 not written yet
+    np.testing.assert_allclose(o[1], v1, atol=1e-12)
+    np.testing.assert_allclose(o[2], v1n, atol=1e-12)           # overwritten
+    np.testing.assert_allclose(o[3], v2, atol=1e-12)            # untouched
+    np.testing.assert_allclose(o[4], v1n, atol=1e-12)
+
+
+def test_overwrite_identity_each_step():
+    """S_t^T k_t = (1 - beta|k|^2) (alpha S_{t-1})^T k_t + beta |k|^2 v_t for any
+    inputs ("从 Full Attention 到 Gated DeltaNet" section 7, with the decay applied
+    before the read as in "Qwen3.5" GDN详解).  Checked one token at a time."""
+    dk, dv, T = 6, 5, 12
+    S = _rand(1, 1, dk, dv)
+    for _ in range(T):
+        q, k, v = _rand(1, 1, 1, dk), _rand(1, 1, 1, dk), _rand(1, 1, 1, dv)
+        g = np.array([[[-rng.uniform(0.05, 2.0)]]])
+        beta = np.array([[[rng.uniform(0.05, 1.0)]]])
+        _, S_new = O.gdn_fwd(q, k, v, g, beta, h0=S, scale=1.0, l2norm=False,
+                             gates_given=True)
+        kk = k[0, 0, 0]
+        n2 = kk @ kk
+        lhs = S_new[0, 0].T @ kk
+        rhs = (1 - beta.item() * n2) * (math.exp(g.item()) * S[0, 0]).T @ kk \
+            + beta.item() * n2 * v[0, 0, 0]
+        np.testing.assert_allclose(lhs, rhs, rtol=1e-11, atol=1e-11)
+        S = S_new
+
+
+def test_pure_decay_closed_form():
+    """beta = 0: S_t = (prod alpha) S_0 and o_t = (prod_{i<=t} alpha_i) S_0^T q_t
+    ("从 Full Attention 到 Gated DeltaNet" section 9, S_t = alpha^n S_{t-n})."""
+    dk, dv, T = 6, 4, 10
+    q, k, v = _rand(1, T, 1, dk), _rand(1, T, 1, dk), _rand(1, T, 1, dv)
+    g = -rng.uniform(0.0, 0.7, size=(1, T, 1))
+    beta = np.zeros((1, T, 1))
+    h0 = _rand(1, 1, dk, dv)
+    o, ht = O.gdn_fwd(q, k, v, g, beta, h0=h0, scale=1.0, l2norm=False, gates_given=True)
+    cum = np.exp(np.cumsum(g[0, :, 0]))
+    ref = cum[:, None] * (q[0, :, 0] @ h0[0, 0])
+    np.testing.assert_allclose(o[0, :, 0], ref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(ht[0, 0], cum[-1] * h0[0, 0], rtol=1e-12)
+
+
+def test_matrix_form_recurrence():
+    """The pages' matrix form, M_t = alpha_t M_{t-1} (I - beta_t k_t k_t^T)
+    + beta_t v_t k_t^T, o_t = M_t q_t (M = S^T; "Qwen3.5" GDN详解 整体公式),
+    computed with explicit matrix products, equals the five-step oracle."""
+    dk, dv, T = 5, 3, 7
+    q, k, v = _rand(1, T, 1, dk), _rand(1, T, 1, dk), _rand(1, T, 1, dv)
+    g = -rng.uniform(0.0, 1.0, size=(1, T, 1))
+    beta = rng.uniform(0.0, 1.0, size=(1, T, 1))
+    h0 = _rand(1, 1, dk, dv)
+    o, ht = O.gdn_fwd(q, k, v, g, beta, h0=h0, scale=1.0, l2norm=False, gates_given=True)
+    M = h0[0, 0].T.copy()
+    for t in range(T):
+        kt, vt, qt = k[0, t, 0], v[0, t, 0], q[0, t, 0]
+        a_t, b_t = math.exp(g[0, t, 0]), beta[0, t, 0]
+        M = a_t * M @ (np.eye(dk) - b_t * np.outer(kt, kt)) + b_t * np.outer(vt, kt)
+        np.testing.assert_allclose(o[0, t, 0], M @ qt, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ht[0, 0], M.T, rtol=1e-12, atol=1e-12)
+
+
+def test_gdn2_matrix_form():
+    """Gated DeltaNet-2 matrix form S_t = (I - k_t e_t^T) D_t S_{t-1} + k_t z_t^T
+    ("Gated DeltaNet-2", 新更新公式) with explicit matrices, random channel decay."""
+    dk, dv, T = 5, 4, 6
+    q, k, v = _rand(1, T, 1, dk), _rand(1, T, 1, dk), _rand(1, T, 1, dv)
+    g = -rng.uniform(0.0, 1.5, size=(1, T, 1, dk))
+    b = rng.uniform(0.0, 1.0, size=(1, T, 1, dk))
+    w = rng.uniform(0.0, 1.0, size=(1, T, 1, dv))
+    h0 = _rand(1, 1, dk, dv)
+    o, ht = O.gdn2_fwd(q, k, v, g, b, w, h0=h0, scale=1.0, l2norm=False, gates_given=True)
+    S = h0[0, 0].copy()
+    for t in range(T):
+        kt, qt = k[0, t, 0], q[0, t, 0]
+        e = b[0, t, 0] * kt
+        z = w[0, t, 0] * v[0, t, 0]
+        D = np.diag(np.exp(g[0, t, 0]))
+        S = (np.eye(dk) - np.outer(kt, e)) @ D @ S + np.outer(kt, z)
+        np.testing.assert_allclose(o[0, t, 0], S.T @ qt, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ht[0, 0], S, rtol=1e-12, atol=1e-12)
+
+
+def test_gdn2_reduces_to_gdn():
+    """b_t = beta_t 1, w_t = beta_t 1 and scalar decay rows turn Gated DeltaNet-2
+    into Gated DeltaNet ("Gated DeltaNet-2", 退化兼容性), through the full gate path."""
+    B, T, H, d = 2, 11, 3, 8
+    q, k, v = _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d)
+    a, b = _rand(B, T, H), _rand(B, T, H)
+    A_log = rng.uniform(0, math.log(16), size=H)
+    dt_bias = rng.uniform(-4, -1, size=H)
+    h0 = 0.02 * _rand(B, H, d, d)
+    o1, ht1 = O.gdn_fwd(q, k, v, a, b, A_log, dt_bias, h0)
+    rep = lambda x: np.repeat(x[..., None], d, axis=-1)
+    o2, ht2 = O.gdn2_fwd(q, k, v, rep(a), rep(b), rep(b), rep(A_log), rep(dt_bias), h0)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(ht2, ht1, rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# Gates and normalisation: closed forms
+# --------------------------------------------------------------------------
+
+def test_gate_closed_forms():
+    """g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b) ("Qwen3.5" module
+    skeleton; softplus(x) = log(1 + e^x), "从 Full Attention 到 Gated DeltaNet" s.9)."""
+    # column h: (a, b, A_log, dt_bias) -> expected (g, beta)
+    a = np.array([[[0.5, math.log(math.e - 1) + 1.0, 800.0, -50.0, 0.0, 22.0]]])
+    b = np.array([[[0.0, math.log(3.0), -math.log(3.0), 40.0, -800.0, 0.0]]])
+    A_log = np.array([0.0, math.log(2.0), 0.0, 0.0, math.log(16.0), 0.0])
+    dt_bias = np.array([-0.5, -1.0, -1.0, 0.0, 0.0, -1.0])
+    g_exp = np.array([-math.log(2.0),        # softplus(0) = ln 2
+                      -2.0,                  # 2 * softplus(ln(e-1)) = 2 * 1
+                      -799.0,                # softplus(799) = 799 (to 1e-300)
+                      -math.log1p(math.exp(-50.0)),
+                      -16.0 * math.log(2.0),
+                      # log(1 + e^21) as the page prints it: exact here to
+                      # ~1e-16 and 7.6e-10 above 21 (no large-x cut-off)
+                      -math.log(1.0 + math.exp(21.0))])
+    beta_exp = np.array([0.5, 0.75, 0.25, 1.0 / (1.0 + math.exp(-40.0)), 0.0, 0.5])
+    q = np.ones((1, 1, 1, 4))
+    _, _, g, beta = O.gate_prep(q, q, a, b, A_log, dt_bias)
+    np.testing.assert_allclose(g[0, 0], g_exp, rtol=1e-14, atol=1e-300)
+    np.testing.assert_allclose(beta[0, 0], beta_exp, rtol=1e-14, atol=1e-300)
+    assert np.all(np.isfinite(g))
+
+
+def test_l2norm_closed_form():
+    """q_hat = scale * q / sqrt(|q|^2 + eps), k_hat = k / sqrt(|k|^2 + eps) with the
+    build's reading eps = 1e-6 and scale = 1/sqrt(d_k) (a 3-4-5 vector)."""
+    d = 16
+    q = np.zeros((1, 1, 1, d)); q[0, 0, 0, :2] = [3.0, 4.0]
+    k = np.zeros((1, 1, 1, d)); k[0, 0, 0, 5] = -2.0
+    a = np.zeros((1, 1, 1)); b = np.zeros((1, 1, 1))
+    qh, kh, _, _ = O.gate_prep(q, k, a, b, np.zeros(1), np.zeros(1))
+    den = math.sqrt(25.0 + 1e-6)
+    np.testing.assert_allclose(qh[0, 0, 0, :2], np.array([3.0, 4.0]) / den / 4.0, rtol=1e-15)
+    np.testing.assert_allclose(kh[0, 0, 0, 5], -2.0 / math.sqrt(4.0 + 1e-6), rtol=1e-15)
+    assert np.count_nonzero(qh) == 2 and np.count_nonzero(kh) == 1
+
+
+# --------------------------------------------------------------------------
+# Head mapping, streaming, decode
+# --------------------------------------------------------------------------
+
+def test_gqa_contiguous_groups():
+    """Value head hv reads key head hv // (Hv/Hk): running each value head alone
+    with its key head gives the same result as the grouped call."""
+    B, T, Hk, Hv, d = 1, 9, 2, 6, 8
+    q, k, v = _rand(B, T, Hk, d), _rand(B, T, Hk, d), _rand(B, T, Hv, d)
+    a, b = _rand(B, T, Hv), _rand(B, T, Hv)
+    A_log = rng.uniform(0, math.log(16), size=Hv)
+    dt_bias = rng.uniform(-4, -1, size=Hv)
+    o, ht = O.gdn_fwd(q, k, v, a, b, A_log, dt_bias)
+    for hv in range(Hv):
+        hk = hv // (Hv // Hk)
+        o1, ht1 = O.gdn_fwd(q[:, :, hk:hk + 1], k[:, :, hk:hk + 1], v[:, :, hv:hv + 1],
+                            a[:, :, hv:hv + 1], b[:, :, hv:hv + 1], A_log[hv:hv + 1],
+                            dt_bias[hv:hv + 1])
+        np.testing.assert_array_equal(o[:, :, hv], o1[:, :, 0])
+        np.testing.assert_array_equal(ht[:, hv], ht1[:, 0])
+    # and the selection interface returns the same rows
+    sel = [4, 1]
+    os_, hts = O.gdn_fwd(q, k, v, a, b, A_log, dt_bias, heads=sel)
+    for i, hv in enumerate(sel):
+        np.testing.assert_array_equal(os_[i], o[0, :, hv])
+        np.testing.assert_array_equal(hts[i], ht[0, hv])
+
+
+@pytest.mark.parametrize("split", [1, 7, 16])
+def test_streaming_split(split):
+    """S_t = f(S_{t-1}, x_t): running [0, T1) then [T1, T) from the carried state
+    equals one pass ("从 Full Attention 到 Gated DeltaNet" section 12)."""
+    B, T, Hk, Hv, d = 1, 23, 1, 2, 8
+    x = dict(q=_rand(B, T, Hk, d), k=_rand(B, T, Hk, d), v=_rand(B, T, Hv, d),
+             a=_rand(B, T, Hv), b=_rand(B, T, Hv))
+    A_log = rng.uniform(0, math.log(16), size=Hv)
+    dt_bias = rng.uniform(-4, -1, size=Hv)
+    h0 = 0.02 * _rand(B, Hv, d, d)
+    o, ht = O.gdn_fwd(x["q"], x["k"], x["v"], x["a"], x["b"], A_log, dt_bias, h0)
+    p1 = {n: t[:, :split] for n, t in x.items()}
+    p2 = {n: t[:, split:] for n, t in x.items()}
+    oa, hta = O.gdn_fwd(p1["q"], p1["k"], p1["v"], p1["a"], p1["b"], A_log, dt_bias, h0)
+    ob, htb = O.gdn_fwd(p2["q"], p2["k"], p2["v"], p2["a"], p2["b"], A_log, dt_bias, hta)
+    np.testing.assert_allclose(np.concatenate([oa, ob], 1), o, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(htb, ht, rtol=1e-13, atol=1e-14)
+
+
+def test_conv_step_matches_library_conv1d():
+    """Causal depthwise conv1d (kernel 4) + SiLU, one token at a time from a cached
+    window, equals torch's grouped conv1d over the concatenated stream followed by
+    SiLU ("从 Full Attention 到 Gated DeltaNet" s.10; "gated-deltanet-qwen3.5" conv)."""
+    N, Cc, steps = 3, 10, 6
+    w = rng.uniform(-0.5, 0.5, size=(Cc, 4))
+    cs0 = _rand(N, Cc, 3)
+    xs = _rand(steps, N, Cc)
+    cs = cs0.copy()
+    ys = [O.conv_step(xs[t], w, cs) for t in range(steps)]
+    stream = torch.cat([torch.from_numpy(cs0), torch.from_numpy(xs).permute(1, 2, 0)], dim=2)
+    ref = torch.nn.functional.silu(
+        torch.nn.functional.conv1d(stream, torch.from_numpy(w)[:, None, :], groups=Cc))
+    np.testing.assert_allclose(np.stack(ys, 0), ref.permute(2, 0, 1).numpy(), rtol=1e-13,
+                               atol=1e-14)
+    np.testing.assert_array_equal(cs, np.concatenate([cs0, xs.transpose(1, 2, 0)], 2)[:, :, -3:])
+
+
+def test_decode_steps_equal_prefill_on_conv_stream():
+    """A run of decode steps (conv fused) equals the conv step followed by the
+    prefill oracle over the resulting q, k, v stream, with the state carried."""
+    N, Hk, Hv, d, steps = 2, 1, 2, 8, 5
+    Cc = 2 * Hk * d + Hv * d
+    xs = _rand(steps, N, Cc)
+    w = rng.uniform(-0.5, 0.5, size=(Cc, 4))
+    a, b = _rand(steps, N, Hv), _rand(steps, N, Hv)
+    A_log = rng.uniform(0, math.log(16), size=Hv)
+    dt_bias = rng.uniform(-4, -1, size=Hv)
+    S0 = 0.02 * _rand(N, Hv, d, d)
+    cs0 = _rand(N, Cc, 3)
+    cs, S = cs0.copy(), S0.copy()
+    outs = [O.decode_step(xs[t], w, a[t], b[t], A_log, dt_bias, cs, S, Hk=Hk, Hv=Hv, dk=d,
+                          dv=d) for t in range(steps)]
+    cs2 = cs0.copy()
+    ys = np.stack([O.conv_step(xs[t], w, cs2) for t in range(steps)], 1)  # [N, steps, Cc]
+    q = ys[:, :, :Hk * d].reshape(N, steps, Hk, d)
+    k = ys[:, :, Hk * d:2 * Hk * d].reshape(N, steps, Hk, d)
+    v = ys[:, :, 2 * Hk * d:].reshape(N, steps, Hv, d)
+    o, ht = O.gdn_fwd(q, k, v, a.transpose(1, 0, 2), b.transpose(1, 0, 2), A_log, dt_bias, S0)
+    np.testing.assert_allclose(np.stack(outs, 1), o, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S, ht, rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(cs, cs2)
+    # selection interface: one sequence alone gives the same numbers
+    cs3, S3 = cs0[1:2].copy(), S0[1:2].copy()
+    for t in range(steps):
+        o1 = O.decode_step(xs[t], w, a[t], b[t], A_log, dt_bias, cs3, S3, Hk=Hk, Hv=Hv,
+                           dk=d, dv=d, seqs=[1])
+        np.testing.assert_allclose(o1[0], outs[t][1], rtol=1e-13, atol=1e-14)
+
+
+def test_float32_inputs_match_float64_inputs():
+    """Inputs given as float32 (how the GPU's bf16/fp32 values are handed over)
+    are widened exactly: the result equals the float64 call on the same values."""
+    B, T, Hk, Hv, d = 1, 7, 1, 2, 8
+    q = _rand(B, T, Hk, d).astype(np.float32)
+    k = _rand(B, T, Hk, d).astype(np.float32)
+    v = _rand(B, T, Hv, d).astype(np.float32)
+    a = _rand(B, T, Hv).astype(np.float32)
+    b = _rand(B, T, Hv).astype(np.float32)
+    A_log = rng.uniform(0, 2, size=Hv).astype(np.float32)
+    dt_bias = rng.uniform(-4, -1, size=Hv).astype(np.float32)
+    o32, h32 = O.gdn_fwd(q, k, v, a, b, A_log, dt_bias)
+    o64, h64 = O.gdn_fwd(*(x.astype(np.float64) for x in (q, k, v, a, b, A_log, dt_bias)))
+    np.testing.assert_array_equal(o32, o64)
+    np.testing.assert_array_equal(h32, h64)
