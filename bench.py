@@ -1,0 +1,460 @@
+"""Benchmark of the GDN hot path on B200: prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline (`value`): GDN chunkwise prefill tokens/s on the Qwen3.5-shaped layer
+(B=1, T=8192, 16 key heads, 64 value heads, d=128, bf16 inputs, fp32 state);
+one step = one gdn_chunk_fwd call (gates, L2 norm, WY chunk solve, output and
+inter-chunk state scan in one kernel) over that batch.  The decode step
+(256 sequences, fused conv1d, state GB/s), the long-context prefill and the
+Gated DeltaNet-2 forward are measured in the same run and reported under
+"extra".  Multi-GPU runs are independent replicas (every (batch, head) scan is
+independent; no collective on the data path): weak scaling, time = max over
+ranks.  `--impl reference` times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
+
+from gdn_synth import WORKLOADS, workload_inputs  # noqa: E402
+
+CHUNK_FLOP_PER_TOKEN_HEAD = 180_224  # dense GEMM FLOPs of the chunk form at C=64, d=128
+HEADLINE = "prefill_8k"
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "src": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self._t.join(timeout=2)
+        rows = [l for (t, l) in self.lines if t0 - 0.06 <= t <= t1 + 0.06] or \
+            [l for (_, l) in self.lines[-3:]]
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in rows:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def flush_l2(buf):
+    buf.add_(1.0)
+
+
+def rank_info():
+    if "WORLD_SIZE" in os.environ and int(os.environ["WORLD_SIZE"]) > 1:
+        return int(os.environ["RANK"]), int(os.environ["LOCAL_RANK"]), int(os.environ["WORLD_SIZE"])
+    return 0, 0, 1
+
+
+def kernel_traffic(name):
+    """dram bytes per launch from a committed ncu summary, if its kernel source
+    hash still matches the current source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{name}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    h = re.search(r"source_sha256:\s*([0-9a-f]{16,64})", txt)
+    if not m or not h:
+        return None
+    return float(m.group(1)) if h.group(1) == source_hash()[:len(h.group(1))] else None
+
+
+def source_hash():
+    d = os.path.join(ROOT, "gated_deltanet_sequence_gdn_b200", "csrc")
+    hs = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            hs.update(open(os.path.join(d, f), "rb").read())
+    return hs.hexdigest()
+
+
+# ----------------------------------------------------------------------------- our arm
+def time_steps(fn, steps, warmup, stream, flush=None, sync_group=False):
+    """CUDA-event time of `steps` calls of fn on `stream`, after `warmup` calls.
+    Returns (total_ms, per-launch ms list)."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            fn()
+    torch.cuda.synchronize()
+    if sync_group:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(steps):
+            if flush is not None:
+                flush()
+            evs[i][0].record(stream)
+            fn()
+            evs[i][1].record(stream)
+        end.record(stream)
+    torch.cuda.synchronize()
+    if sync_group:
+        dist.barrier()
+    per = [a.elapsed_time(b) for a, b in evs]
+    return start.elapsed_time(end), per
+
+
+def run_ours(args, rank, local_rank, world):
+    import gated_deltanet_sequence_gdn_b200 as G
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    pk = peaks()
+    w = WORKLOADS[HEADLINE]
+    x = workload_inputs(w, dev)
+    o = torch.empty((w.B, w.T, w.Hv, w.d), device=dev, dtype=w.dtype)
+    ht = torch.empty((w.B, w.Hv, w.d, w.d), device=dev, dtype=torch.float32)
+
+    def step():
+        G.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                        x["h0"], o=o, ht=ht, stream=stream)
+
+    clocks = ClockSampler(local_rank).start()
+    time.sleep(0.3)
+    t0 = time.time()
+    total_ms, per = time_steps(step, args.steps, args.warmup, stream, sync_group=world > 1)
+    t1 = time.time()
+    clk = clocks.stop(t0, t1)
+    G.gdn_check_status(stream)
+    ms = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    ms_step = ms.item() / args.steps
+    tokens = w.B * w.T
+    value = world * tokens / (ms_step / 1e3)
+    flop = CHUNK_FLOP_PER_TOKEN_HEAD * w.T * w.Hv * w.B
+    launch_ms = sum(per) / len(per)
+    achieved = flop / (launch_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2),
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_tflops"], 4),
+                "traffic": kernel_traffic("chunk_prefill_8k"),
+                "kernel": "gdn_chunk_fwd (one launch per step)",
+                "flop_per_launch": flop, "peak_src": pk["src"] + " burst bf16"}
+
+    # ---- end to end through the public call, host buffers, copies inside the timed region
+    e2e = measure_e2e(G, x, w, dev, stream, args, world)
+
+    extra = {}
+    if not args.headline_only:
+        extra["decode_256"] = measure_decode(G, dev, stream, pk, args)
+        extra["gdn2_b4_4k"] = measure_gdn2(G, dev, stream, pk, args)
+        extra["prefill_128k"] = measure_prefill(G, "prefill_128k", dev, stream, pk, args)
+
+    launches = args.steps  # one gdn_chunk_fwd kernel per step
+    line = {
+        "metric": "GDN prefill tokens/s (chunk_gated_delta_rule) on 1 B200, % of roofline",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": HEADLINE, "B": w.B, "T": w.T, "Hk": w.Hk, "Hv": w.Hv,
+                   "d": w.d, "chunk": 64, "state": "fp32", "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (q,k,v,o ~340 MB per step > 126 MB)"},
+        "roofline": roofline, "e2e": e2e, "clocks": clk, "gpu_launches": launches,
+        "extra": extra,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, x)
+    return line
+
+
+def measure_e2e(G, x, w, dev, stream, args, world):
+    host = {n: (t.cpu().pin_memory() if t is not None else None) for n, t in x.items()}
+    o_h = torch.empty((w.B, w.T, w.Hv, w.d), dtype=w.dtype).pin_memory()
+    ht_h = torch.empty((w.B, w.Hv, w.d, w.d), dtype=torch.float32).pin_memory()
+    dev_in = {n: (torch.empty_like(t, device=dev) if t is not None else None)
+              for n, t in host.items()}
+    o = torch.empty((w.B, w.T, w.Hv, w.d), device=dev, dtype=w.dtype)
+    ht = torch.empty((w.B, w.Hv, w.d, w.d), device=dev, dtype=torch.float32)
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    d2h = o_h.numel() * o_h.element_size() + ht_h.numel() * ht_h.element_size()
+
+    def step():
+        for n, t in host.items():
+            if t is not None:
+                dev_in[n].copy_(t, non_blocking=True)
+        G.gdn_chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["a"], dev_in["b"],
+                        dev_in["A_log"], dev_in["dt_bias"], dev_in["h0"], o=o, ht=ht,
+                        stream=stream)
+        o_h.copy_(o, non_blocking=True)
+        ht_h.copy_(ht, non_blocking=True)
+
+    steps = max(3, min(args.steps, 20))
+    total_ms, _ = time_steps(step, steps, 2, stream, sync_group=world > 1)
+    ms = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    ms_step = ms.item() / steps
+    return {"value": round(world * w.B * w.T / (ms_step / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms_step, 4), "steps": steps,
+            "path": "pinned host -> gdn_chunk_fwd (C ABI) -> pinned host"}
+
+
+def measure_prefill(G, name, dev, stream, pk, args):
+    w = WORKLOADS[name]
+    x = workload_inputs(w, dev)
+    o = torch.empty((w.B, w.T, w.Hv, w.d), device=dev, dtype=w.dtype)
+    ht = torch.empty((w.B, w.Hv, w.d, w.d), device=dev, dtype=torch.float32)
+
+    def step():
+        G.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                        x["h0"], o=o, ht=ht, stream=stream)
+
+    total, per = time_steps(step, 3, 1, stream)
+    ms = total / 3
+    flop = CHUNK_FLOP_PER_TOKEN_HEAD * w.T * w.Hv * w.B
+    ach = flop / (ms / 1e3) / 1e12
+    del x, o, ht
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+            "B": w.B, "T": w.T, "achieved_tflops": round(ach, 2),
+            "frac_of_bf16_peak": round(ach / pk["bf16_tflops"], 4)}
+
+
+def measure_decode(G, dev, stream, pk, args):
+    w = WORKLOADS["decode_256"]
+    x = workload_inputs(w, dev)
+    cs, S = x["conv_state"], x["state"]
+    o = torch.empty((w.B, w.Hv, w.d), device=dev, dtype=w.dtype)
+    it = [0]
+
+    def step():
+        t = it[0] % w.steps
+        it[0] += 1
+        G.gdn_recurrent_step(x["x"][t], x["conv_w"], cs, x["a"][t], x["b"][t], x["A_log"],
+                             x["dt_bias"], S, Hk=w.Hk, Hv=w.Hv, dk=w.d, dv=w.d, o=o,
+                             stream=stream)
+
+    total, per = time_steps(step, w.steps, 3, stream)
+    ms = total / w.steps
+    state_bytes = 2 * w.B * w.Hv * w.d * w.d * 4
+    Cc = 2 * w.Hk * w.d + w.Hv * w.d
+    other = w.B * Cc * 2 + 2 * w.B * Cc * 3 * 2 + Cc * 16 + w.B * w.Hv * (4 + w.d * 2)
+    gbs = state_bytes / (ms / 1e3) / 1e9
+    del x, cs, S
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(w.B / (ms / 1e3), 1), "ms_per_step": round(ms, 5),
+            "state_gb_per_s": round(gbs, 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                         "algorithmic_bytes_per_launch": state_bytes,
+                         "other_bytes_per_launch": other,
+                         "traffic": kernel_traffic("decode_256")},
+            "steps": w.steps}
+
+
+def measure_gdn2(G, dev, stream, pk, args):
+    w = WORKLOADS["gdn2_b4_4k"]
+    x = workload_inputs(w, dev)
+    o = torch.empty((w.B, w.T, w.Hv, w.d), device=dev, dtype=w.dtype)
+    ht = torch.empty((w.B, w.Hv, w.d, w.d), device=dev, dtype=torch.float32)
+
+    def step():
+        G.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["a"], x["b_logit"], x["w_logit"],
+                         x["A_log"], x["dt_bias"], x["h0"], o=o, ht=ht, stream=stream)
+
+    total, per = time_steps(step, 5, 2, stream)
+    ms = total / 5
+    flop = CHUNK_FLOP_PER_TOKEN_HEAD * w.T * w.Hv * w.B
+    ach = flop / (ms / 1e3) / 1e12
+    del x, o, ht
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+            "achieved_tflops": round(ach, 2),
+            "frac_of_bf16_peak": round(ach / pk["bf16_tflops"], 4)}
+
+
+def run_only(args, local_rank):
+    import gated_deltanet_sequence_gdn_b200 as G
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    pk = peaks()
+    if args.only == "decode_256":
+        r = measure_decode(G, dev, stream, pk, args)
+    elif args.only == "gdn2_b4_4k":
+        r = measure_gdn2(G, dev, stream, pk, args)
+    else:
+        r = measure_prefill(G, args.only, dev, stream, pk, args)
+    G.gdn_check_status(stream)
+    return {"workload": args.only, **r}
+
+
+# ----------------------------------------------------------------------------- oracle
+def _oracle_prefix(w, x_cpu, T_prefix, threads):
+    from oracle import oracle as O
+    sl = lambda t: t[:, :T_prefix]
+    t0 = time.perf_counter()
+    O.gdn_fwd(sl(x_cpu["q"]), sl(x_cpu["k"]), sl(x_cpu["v"]), sl(x_cpu["a"]), sl(x_cpu["b"]),
+              x_cpu["A_log"], x_cpu["dt_bias"], x_cpu["h0"], want_o=True, want_ht=True,
+              threads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, x, target_s=10.0):
+    """The fp64 oracle, as it stands, on the host cores: a T-prefix of the same
+    workload (all heads), sized for ~target_s seconds."""
+    from oracle import oracle as O
+    cores = O.max_threads()
+    x_cpu = {n: (t.cpu() if t is not None else None) for n, t in x.items()}
+    probe_T = 64
+    dt = _oracle_prefix(w, x_cpu, probe_T, cores)
+    T_pre = int(min(w.T, max(probe_T, probe_T * target_s / max(dt, 1e-6))))
+    T_pre = max(64, (T_pre // 64) * 64)
+    dt = _oracle_prefix(w, x_cpu, T_pre, cores)
+    return {"value": round(w.B * T_pre / dt, 1), "unit": "tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{HEADLINE} first {T_pre} of {w.T} tokens, all {w.B * w.Hv} heads, "
+                      f"{dt:.1f} s wall"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 oracle on the host cores (rank 0 only)."""
+    from oracle import oracle as O
+    if rank != 0:
+        return None
+    w = WORKLOADS[HEADLINE]
+    x = workload_inputs(w, "cpu")
+    cores = O.max_threads()
+    # size one step for ~3 s of wall time
+    dt = _oracle_prefix(w, x, 64, cores)
+    T_pre = max(64, int(min(w.T, 64 * 3.0 / max(dt, 1e-6))) // 64 * 64)
+    for _ in range(args.warmup):
+        _oracle_prefix(w, x, T_pre, cores)
+    times = [_oracle_prefix(w, x, T_pre, cores) for _ in range(args.steps)]
+    s = sum(times) / len(times)
+    value = w.B * T_pre / s
+    sample = f"{HEADLINE} first {T_pre} of {w.T} tokens per step, all {w.B * w.Hv} heads"
+    return {"impl": "reference",
+            "metric": "GDN prefill tokens/s (chunk_gated_delta_rule) on 1 B200, % of roofline",
+            "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(s * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": HEADLINE, "B": w.B, "T": w.T, "Hk": w.Hk, "Hv": w.Hv,
+                       "d": w.d, "chunk": 64},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the decode / GDN-2 / long-prefill extras")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["decode_256", "gdn2_b4_4k", "prefill_128k",
+                                       "prefill_b8_16k"], default=None,
+                    help="measure one secondary workload alone (profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, local_rank, world = rank_info()
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        if args.only:
+            line = run_only(args, local_rank)
+        else:
+            line = run_ours(args, rank, local_rank, world)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,210 @@
+"""Python binding of libgdn.so, the B200 (sm_100a) Gated DeltaNet hot path.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libgdn.so, called through its C ABI (include/gdn.h) with ctypes.
+PyTorch provides device memory and the current stream.  There is no CPU or
+Python fallback: importing this module fails if the library is not built, and
+every call raises if the library reports an error.
+
+Entry points (same names as the C ABI):
+    gdn_gate_prep, gdn_chunk_fwd, gdn_recurrent_step, gdn2_chunk_fwd,
+    gdn_check_status
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_recurrent_step", "gdn2_chunk_fwd",
+           "gdn_check_status", "GDNError", "LIB_PATH", "lib", "F32", "BF16",
+           "QK_L2NORM", "GATES_PRECOMPUTED", "OUT_F32"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m gated_deltanet_sequence_gdn_b200.build`"
+        " (nvcc, sm_100a). There is no fallback implementation.")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+F32, BF16 = 0, 1
+QK_L2NORM, GATES_PRECOMPUTED, OUT_F32 = 1, 2, 4
+_STATUS = {0: "GDN_OK", -1: "GDN_ERR_INVALID_ARG", -2: "GDN_ERR_UNSUPPORTED",
+           -3: "GDN_ERR_CUDA", -4: "GDN_ERR_TIMEOUT", -5: "GDN_ERR_WORKSPACE"}
+
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+lib.gdn_gate_prep.argtypes = [_vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f,
+                              _vp, _vp, _vp, _vp, _vp]
+lib.gdn_chunk_fwd.argtypes = [_vp] * 8 + [_i] * 7 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
+lib.gdn2_chunk_fwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
+lib.gdn_recurrent_step.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _vp]
+lib.gdn_chunk_workspace_bytes.argtypes = [_i] * 7
+lib.gdn2_chunk_workspace_bytes.argtypes = [_i] * 6
+lib.gdn_chunk_workspace_bytes.restype = _sz
+lib.gdn2_chunk_workspace_bytes.restype = _sz
+lib.gdn_check_status.argtypes = [_vp]
+lib.gdn_status_string.argtypes = [_i]
+lib.gdn_status_string.restype = ctypes.c_char_p
+lib.gdn_version.argtypes = []
+for _fn in (lib.gdn_gate_prep, lib.gdn_chunk_fwd, lib.gdn2_chunk_fwd, lib.gdn_recurrent_step,
+            lib.gdn_check_status, lib.gdn_version):
+    _fn.restype = _i
+
+
+class GDNError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS.get(status, status)}")
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise GDNError(status, where)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return BF16
+    if t == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t}; expected bfloat16 or float32")
+
+
+def _p(t):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def gdn_gate_prep(q, k, a, b, A_log, dt_bias, *, scale=None, q_out=None, k_out=None,
+                  g_out=None, beta_out=None, stream=None):
+    """Gate + L2-norm prologue. Returns (q_hat, k_hat, g, beta)."""
+    B, T, Hk, d = q.shape
+    Hv = a.shape[2]
+    dt = q.dtype
+    scale = d ** -0.5 if scale is None else scale
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    g_out = torch.empty((B, T, Hv), device=q.device, dtype=torch.float32) if g_out is None else g_out
+    beta_out = torch.empty_like(g_out) if beta_out is None else beta_out
+    _need(k, dt, q.shape, "k")
+    _need(a, dt, (B, T, Hv), "a")
+    _need(b, dt, (B, T, Hv), "b")
+    _check(lib.gdn_gate_prep(_p(q), _p(k), _dtype_code(dt), _p(a), _p(b), _p(A_log),
+                             _p(dt_bias), B, T, Hk, Hv, d, float(scale), _p(q_out), _p(k_out),
+                             _p(g_out), _p(beta_out), _stream(stream)), "gdn_gate_prep")
+    return q_out, k_out, g_out, beta_out
+
+
+def gdn_chunk_fwd(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, scale=None,
+                  l2norm=True, gates_precomputed=False, out_f32=False, o=None, ht=None,
+                  want_ht=True, stream=None):
+    """Chunkwise GDN prefill. q, k [B,T,Hk,dk]; v [B,T,Hv,dv]; a, b [B,T,Hv]
+    (float32 g, beta with gates_precomputed); A_log, dt_bias [Hv] float32;
+    h0 [B,Hv,dk,dv] float32 or None.  Returns (o [B,T,Hv,dv], ht or None);
+    o has the input dtype, or float32 with out_f32."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dt = q.dtype
+    scale = dk ** -0.5 if scale is None else scale
+    _need(k, dt, q.shape, "k")
+    _need(v, dt, (B, T, Hv, dv), "v")
+    gdt = torch.float32 if gates_precomputed else dt
+    _need(a, gdt, (B, T, Hv), "a")
+    _need(b, gdt, (B, T, Hv), "b")
+    if h0 is not None:
+        _need(h0, torch.float32, (B, Hv, dk, dv), "h0")
+    odt = torch.float32 if out_f32 else dt
+    o = torch.empty((B, T, Hv, dv), device=q.device, dtype=odt) if o is None else o
+    _need(o, odt, (B, T, Hv, dv), "o")
+    if ht is None and want_ht:
+        ht = torch.empty((B, Hv, dk, dv), device=q.device, dtype=torch.float32)
+    flags = ((QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
+             | (OUT_F32 if out_f32 else 0))
+    _check(lib.gdn_chunk_fwd(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(dt_bias), _p(h0),
+                             B, T, Hk, Hv, dk, dv, _dtype_code(dt), float(scale), flags, _p(o),
+                             _p(ht), None, 0, _stream(stream)), "gdn_chunk_fwd")
+    return o, ht
+
+
+def gdn2_chunk_fwd(q, k, v, a, b_logit, w_logit, A_log=None, dt_bias=None, h0=None, *,
+                   scale=None, l2norm=True, gates_precomputed=False, out_f32=False, o=None,
+                   ht=None, want_ht=True, stream=None):
+    """Chunkwise Gated DeltaNet-2 forward. q, k, a, b_logit [B,T,H,dk]; v, w_logit
+    [B,T,H,dv]; A_log, dt_bias [H,dk] float32; h0 [B,H,dk,dv] or None."""
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    dt = q.dtype
+    scale = dk ** -0.5 if scale is None else scale
+    gdt = torch.float32 if gates_precomputed else dt
+    _need(k, dt, q.shape, "k")
+    _need(v, dt, (B, T, H, dv), "v")
+    _need(a, gdt, (B, T, H, dk), "a")
+    _need(b_logit, gdt, (B, T, H, dk), "b_logit")
+    _need(w_logit, gdt, (B, T, H, dv), "w_logit")
+    if h0 is not None:
+        _need(h0, torch.float32, (B, H, dk, dv), "h0")
+    odt = torch.float32 if out_f32 else dt
+    o = torch.empty((B, T, H, dv), device=q.device, dtype=odt) if o is None else o
+    _need(o, odt, (B, T, H, dv), "o")
+    if ht is None and want_ht:
+        ht = torch.empty((B, H, dk, dv), device=q.device, dtype=torch.float32)
+    flags = ((QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
+             | (OUT_F32 if out_f32 else 0))
+    _check(lib.gdn2_chunk_fwd(_p(q), _p(k), _p(v), _p(a), _p(b_logit), _p(w_logit), _p(A_log),
+                              _p(dt_bias), _p(h0), B, T, H, dk, dv, _dtype_code(dt),
+                              float(scale), flags, _p(o), _p(ht), None, 0, _stream(stream)),
+           "gdn2_chunk_fwd")
+    return o, ht
+
+
+def gdn_recurrent_step(x, conv_w, conv_state, a, b, A_log, dt_bias, state, *, Hk, Hv, dk,
+                       dv, scale=None, out_f32=False, o=None, stream=None):
+    """One fused conv1d + GDN decode step for N sequences; conv_state and state
+    are updated in place.  x [N, 2*Hk*dk + Hv*dv]; returns o [N, Hv, dv]."""
+    N = x.shape[0]
+    dt = x.dtype
+    scale = dk ** -0.5 if scale is None else scale
+    _need(x, dt, (N, 2 * Hk * dk + Hv * dv), "x")
+    _need(a, dt, (N, Hv), "a")
+    _need(b, dt, (N, Hv), "b")
+    _need(state, torch.float32, (N, Hv, dk, dv), "state")
+    if conv_w is not None:
+        _need(conv_w, torch.float32, (x.shape[1], 4), "conv_w")
+        _need(conv_state, dt, (N, x.shape[1], 3), "conv_state")
+    odt = torch.float32 if out_f32 else dt
+    o = torch.empty((N, Hv, dv), device=x.device, dtype=odt) if o is None else o
+    _need(o, odt, (N, Hv, dv), "o")
+    _check(lib.gdn_recurrent_step(_p(x), _p(conv_w), _p(conv_state), _p(a), _p(b), _p(A_log),
+                                  _p(dt_bias), _p(state), _p(o), N, Hk, Hv, dk, dv,
+                                  _dtype_code(dt), float(scale), OUT_F32 if out_f32 else 0,
+                                  _stream(stream)),
+           "gdn_recurrent_step")
+    return o
+
+
+def gdn_check_status(stream=None):
+    """Synchronise the stream and raise if a bounded device wait expired."""
+    _check(lib.gdn_check_status(_stream(stream)), "gdn_check_status")

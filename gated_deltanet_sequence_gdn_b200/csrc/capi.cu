@@ -1,0 +1,178 @@
+// capi.cu -- the extern "C" entry points of libgdn.so declared in include/gdn.h:
+// host-side argument validation, dispatch to the kernels, status reporting.
+#include <stdint.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace gdn {
+
+// One status word per device; kernels with bounded waits get its address.
+__device__ int g_gdn_status = 0;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
+// element-aligned pointers (read with scalar loads): gates, decode inputs
+bool ok_elem(const void* p, size_t elem) {
+  return p != nullptr && (reinterpret_cast<uintptr_t>(p) % elem) == 0;
+}
+size_t elem_size(int dtype) { return dtype == GDN_BF16 ? 2 : 4; }
+bool ok_head_dim(int d) { return d == 64 || d == 128; }
+bool ok_dtype(int t) { return t == GDN_F32 || t == GDN_BF16; }
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+__global__ void copy_or_zero_kernel(const float* __restrict__ src, float* dst, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = src ? src[i] : 0.f;
+}
+
+}  // namespace
+
+int* status_word() {
+  static int* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gdn_status) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
+cudaError_t launch_copy_state(const float* h0, float* ht, size_t n, cudaStream_t s) {
+  if (n == 0 || ht == nullptr || h0 == ht) return cudaSuccess;
+  const unsigned grid = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  copy_or_zero_kernel<<<grid, 256, 0, s>>>(h0, ht, n);
+  return cudaGetLastError();
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+int gdn_version(void) { return 100; }  // 0.1.0
+
+const char* gdn_status_string(int status) {
+  switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+    default: return "GDN_ERR_UNKNOWN";
+  }
+}
+
+int gdn_gate_prep(const void* q, const void* k, int dtype, const void* a, const void* b,
+                  const float* A_log, const float* dt_bias, int B, int T, int Hk, int Hv,
+                  int d, float scale, void* q_out, void* k_out, float* g_out,
+                  float* beta_out, gdn_stream_t stream) {
+  if (B < 0 || T < 0 || Hk <= 0 || Hv <= 0 || !ok_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  if (!ok_head_dim(d) || Hv % Hk != 0) return GDN_ERR_UNSUPPORTED;
+  if ((long)B * T == 0) return GDN_OK;
+  const size_t es = elem_size(dtype);
+  if (!ok_ptr(q) || !ok_ptr(k) || !ok_elem(a, es) || !ok_elem(b, es) || !ok_elem(A_log, 4) ||
+      !ok_elem(dt_bias, 4) || !ok_ptr(q_out) || !ok_ptr(k_out) || !ok_elem(g_out, 4) ||
+      !ok_elem(beta_out, 4))
+    return GDN_ERR_INVALID_ARG;
+  return from_cuda(launch_gate_prep(q, k, dtype, a, b, A_log, dt_bias, B, T, Hk, Hv, d, scale,
+                                    q_out, k_out, g_out, beta_out, (cudaStream_t)stream));
+}
+
+size_t gdn_chunk_workspace_bytes(int, int, int, int, int, int, int) { return 0; }
+size_t gdn2_chunk_workspace_bytes(int, int, int, int, int, int) { return 0; }
+
+static int validate_chunk(const ChunkArgs& c, bool gdn2) {
+  if (c.B < 0 || c.T < 0 || c.Hk <= 0 || c.Hv <= 0 || !ok_dtype(c.dtype))
+    return GDN_ERR_INVALID_ARG;
+  if (c.flags & ~(GDN_QK_L2NORM | GDN_GATES_PRECOMPUTED | GDN_OUT_F32))
+    return GDN_ERR_INVALID_ARG;
+  if (!ok_head_dim(c.dk) || !ok_head_dim(c.dv) || c.Hv % c.Hk != 0) return GDN_ERR_UNSUPPORTED;
+  if (!ok_opt(c.h0) || !ok_opt(c.ht)) return GDN_ERR_INVALID_ARG;
+  if ((long)c.B * c.T == 0) return GDN_OK;
+  const size_t ges = (c.flags & GDN_GATES_PRECOMPUTED) ? 4 : elem_size(c.dtype);
+  if (!ok_ptr(c.q) || !ok_ptr(c.k) || !ok_ptr(c.v) || !ok_elem(c.a, ges) ||
+      !ok_elem(c.b, ges) || !ok_ptr(c.o))
+    return GDN_ERR_INVALID_ARG;
+  if (gdn2 && !ok_elem(c.w, ges)) return GDN_ERR_INVALID_ARG;
+  if (!(c.flags & GDN_GATES_PRECOMPUTED) && (!ok_elem(c.A_log, 4) || !ok_elem(c.dt_bias, 4)))
+    return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+static int run_chunk(const ChunkArgs& c, bool gdn2, cudaStream_t s) {
+  const size_t state_elems = (size_t)c.B * c.Hv * c.dk * c.dv;
+  if (c.T == 0 || c.B == 0) return from_cuda(launch_copy_state(c.h0, c.ht, state_elems, s));
+  if (!gdn2 && c.dtype == GDN_BF16 && chunk_tc_supported(c))
+    return from_cuda(launch_chunk_tc(c, s));
+  return from_cuda(launch_chunk_simt(c, gdn2, s));
+}
+
+int gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* a, const void* b,
+                  const float* A_log, const float* dt_bias, const float* h0, int B, int T,
+                  int Hk, int Hv, int dk, int dv, int dtype, float scale, int flags, void* o,
+                  float* ht, void* workspace, size_t ws_bytes, gdn_stream_t stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  ChunkArgs c{q, k, v, a, b, nullptr, A_log, dt_bias, h0, B, T, Hk, Hv, dk, dv, dtype,
+              scale, flags, o, ht};
+  int st = validate_chunk(c, false);
+  if (st != GDN_OK) return st;
+  return run_chunk(c, false, (cudaStream_t)stream);
+}
+
+int gdn2_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
+                   const void* b_logit, const void* w_logit, const float* A_log,
+                   const float* dt_bias, const float* h0, int B, int T, int H, int dk, int dv,
+                   int dtype, float scale, int flags, void* o, float* ht, void* workspace,
+                   size_t ws_bytes, gdn_stream_t stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  ChunkArgs c{q, k, v, a, b_logit, w_logit, A_log, dt_bias, h0, B, T, H, H, dk, dv, dtype,
+              scale, flags, o, ht};
+  int st = validate_chunk(c, true);
+  if (st != GDN_OK) return st;
+  return run_chunk(c, true, (cudaStream_t)stream);
+}
+
+int gdn_recurrent_step(const void* x_qkv, const float* conv_w, void* conv_state, const void* a,
+                       const void* b, const float* A_log, const float* dt_bias, float* state,
+                       void* o, int N, int Hk, int Hv, int dk, int dv, int dtype, float scale,
+                       int flags, gdn_stream_t stream) {
+  if (N < 0 || Hk <= 0 || Hv <= 0 || !ok_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  if (flags & ~GDN_OUT_F32) return GDN_ERR_INVALID_ARG;
+  if (!ok_head_dim(dk) || !ok_head_dim(dv) || Hv % Hk != 0) return GDN_ERR_UNSUPPORTED;
+  if (N == 0) return GDN_OK;
+  const size_t es = elem_size(dtype);
+  if (!ok_elem(x_qkv, es) || !ok_elem(a, es) || !ok_elem(b, es) || !ok_elem(A_log, 4) ||
+      !ok_elem(dt_bias, 4) || !ok_ptr(state) || !ok_elem(o, (flags & GDN_OUT_F32) ? 4 : es) ||
+      !ok_opt(conv_w))
+    return GDN_ERR_INVALID_ARG;
+  if (conv_w != nullptr && !ok_elem(conv_state, es)) return GDN_ERR_INVALID_ARG;
+  return from_cuda(launch_recurrent_step(x_qkv, conv_w, conv_state, a, b, A_log, dt_bias,
+                                         state, o, N, Hk, Hv, dk, dv, dtype, scale,
+                                         (flags & GDN_OUT_F32) != 0, (cudaStream_t)stream));
+}
+
+int gdn_check_status(gdn_stream_t stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDN_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_gdn_status, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_gdn_status, &zero, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+    return GDN_ERR_TIMEOUT;
+  }
+  return GDN_OK;
+}
+
+}  // extern "C"

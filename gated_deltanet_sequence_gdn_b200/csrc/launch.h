@@ -1,0 +1,43 @@
+// launch.h -- internal launchers behind the C ABI (host side, C++).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace gdn {
+
+struct ChunkArgs {
+  const void* q; const void* k; const void* v; const void* a; const void* b;
+  const void* w;  // GDN-2 write-gate logits, else NULL
+  const float* A_log; const float* dt_bias; const float* h0;
+  int B, T, Hk, Hv, dk, dv, dtype;
+  float scale;
+  int flags;
+  void* o; float* ht;
+};
+
+cudaError_t launch_gate_prep(const void* q, const void* k, int dtype, const void* a,
+                             const void* b, const float* A_log, const float* dt_bias,
+                             int B, int T, int Hk, int Hv, int d, float scale,
+                             void* q_out, void* k_out, float* g_out, float* beta_out,
+                             cudaStream_t s);
+
+cudaError_t launch_recurrent_step(const void* x, const float* conv_w, void* conv_state,
+                                  const void* a, const void* b, const float* A_log,
+                                  const float* dt_bias, float* state, void* o, int N,
+                                  int Hk, int Hv, int dk, int dv, int dtype, float scale,
+                                  bool out_f32, cudaStream_t s);
+
+// float32 CUDA-core chunk path (GDN and, with gdn2 = true, Gated DeltaNet-2).
+cudaError_t launch_chunk_simt(const ChunkArgs& a, bool gdn2, cudaStream_t s);
+
+// bf16 tcgen05 chunk path (GDN).
+cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s);
+bool chunk_tc_supported(const ChunkArgs& a);
+
+// Device address of this device's status word (set up once per device).
+int* status_word();
+
+cudaError_t launch_copy_state(const float* h0, float* ht, size_t n, cudaStream_t s);
+
+}  // namespace gdn

@@ -1,0 +1,193 @@
+/*
+ * gdn.h -- C ABI of libgdn.so, the B200 (sm_100a) Gated DeltaNet hot path.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor pointer is a DEVICE pointer into memory the caller owns
+ *    (allocated by any means: cudaMalloc, a PyTorch tensor, a pool).  The
+ *    library never allocates, frees or synchronises; each call only enqueues
+ *    kernels on `stream` and returns.  NULL stream = the legacy default stream.
+ *  - Layouts are dense, row-major, token-major, with no padding:
+ *      q, k        [B, T, Hk, dk]
+ *      v, o        [B, T, Hv, dv]
+ *      a, b        [B, T, Hv]              (GDN gate inputs, one per value head)
+ *      A_log,
+ *      dt_bias     [Hv] float32
+ *      h0, ht      [B, Hv, dk, dv] float32 (state S, key index first; o = S^T q)
+ *    Value head hv reads key/query head hv / (Hv / Hk) (contiguous groups).
+ *  - `dtype` selects the element type of q, k, v, a, b, x, o and the conv
+ *    state: GDN_F32 (float) or GDN_BF16 (__nv_bfloat16).  States, A_log,
+ *    dt_bias and conv weights are always float32; arithmetic is float32 with
+ *    float32 accumulation.
+ *  - Tensors moved in 16-byte pieces must be 16-byte aligned: q, k, v, o and
+ *    q_out/k_out of the chunk and gate-prep calls, h0, ht, the decode state and
+ *    conv_w.  The other pointers (gates a, b, w, A_log, dt_bias, g/beta outputs,
+ *    the decode x, o and conv_state) need only their element alignment.  Head
+ *    dims dk, dv must be 64 or 128 (heads are tiled in 64-column blocks); Hv
+ *    must be a multiple of Hk.
+ *  - Return value: GDN_OK or a negative gdn_status.  Argument errors are
+ *    detected on the host before anything is enqueued.  GDN_ERR_CUDA reports a
+ *    launch failure (the CUDA error is left for cudaGetLastError).  Kernels
+ *    whose waits on the tensor-memory / TMA pipeline are bounded record an
+ *    expired wait in a device status word instead of hanging; the host reads
+ *    it with gdn_check_status().
+ *
+ * Method (pages: "Qwen3.5" rainlin-net, section GDN详解; "从 Full Attention 到
+ * Gated DeltaNet" sections 9-10; "gated-deltanet-qwen3.5" architecture diagram;
+ * "Gated DeltaNet-2" zhichai, sections 新更新公式 and 高效训练):
+ *    g_t = -exp(A_log) * softplus(a_t + dt_bias),  alpha_t = e^{g_t},
+ *    beta_t = sigmoid(b_t),
+ *    S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,
+ *    o_t = S_t^T q_t.
+ */
+#ifndef GDN_B200_GDN_H_
+#define GDN_B200_GDN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* gdn_stream_t;
+
+typedef enum gdn_status {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = -1, /* null / misaligned pointer, negative size, bad dtype */
+  GDN_ERR_UNSUPPORTED = -2, /* head dim not 64/128, Hv % Hk != 0, ...           */
+  GDN_ERR_CUDA = -3,        /* a kernel launch or driver call failed            */
+  GDN_ERR_TIMEOUT = -4,     /* a bounded device-side wait expired               */
+  GDN_ERR_WORKSPACE = -5    /* workspace smaller than gdn_*_workspace_bytes()   */
+} gdn_status;
+
+typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* Flags of the chunk and decode entry points. */
+enum {
+  GDN_QK_L2NORM = 1,         /* normalise q and k per head: x / sqrt(|x|^2 + 1e-6)
+                                (chunk entry points; decode always normalises)   */
+  GDN_GATES_PRECOMPUTED = 2, /* a holds g (float32), b holds beta (float32);
+                                A_log and dt_bias are ignored and may be NULL
+                                (chunk entry points)                             */
+  GDN_OUT_F32 = 4            /* o is written as float32 whatever `dtype` is      */
+};
+
+/*
+ * gdn_gate_prep -- the gate and L2-norm prologue as one elementwise kernel.
+ * ("Qwen3.5", module skeleton: beta = sigmoid(b), g = -exp(A_log) *
+ *  softplus(a + dt_bias) in float32; L2 norm and the 1/sqrt(dk) query scale
+ *  are this library's reading of the pages, applied after the norm.)
+ *   q, k       [B,T,Hk,d]  dtype, read
+ *   a, b       [B,T,Hv]    dtype, read
+ *   A_log,
+ *   dt_bias    [Hv]        float32, read
+ *   q_out,
+ *   k_out      [B,T,Hk,d]  dtype, written: scale*q/|q|, k/|k| (may alias q, k)
+ *   g_out,
+ *   beta_out   [B,T,Hv]    float32, written
+ */
+int gdn_gate_prep(const void* q, const void* k, int dtype, const void* a,
+                  const void* b, const float* A_log, const float* dt_bias,
+                  int B, int T, int Hk, int Hv, int d, float scale, void* q_out,
+                  void* k_out, float* g_out, float* beta_out,
+                  gdn_stream_t stream);
+
+/*
+ * gdn_chunk_fwd -- chunkwise-parallel GDN prefill (chunk_gated_delta_rule;
+ * "gated-deltanet-qwen3.5" training/prefill branch).  Each 64-token chunk is
+ * solved in WY form: A = (I + tril(diag(beta) K K^T (.) Gamma, -1))^-1 by
+ * forward substitution, W = A diag(beta gamma) K, U = A diag(beta) V,
+ * U~ = U - W S, O = diag(gamma) Q S + tril(Q K^T (.) Gamma) U~,
+ * S <- gamma_C S + (diag(gamma_C/gamma) K)^T U~  ("Gated DeltaNet-2",
+ * 高效训练, with scalar decay).  The float32 state stays on chip across the
+ * chunks of one (batch, value head).  bf16 runs on the tcgen05 tensor cores;
+ * float32 runs a float32 CUDA-core path.
+ *   q, k [B,T,Hk,dk], v [B,T,Hv,dv], a, b [B,T,Hv]: dtype, read
+ *     (with GDN_GATES_PRECOMPUTED: a = g, b = beta, float32)
+ *   A_log, dt_bias [Hv] float32, read (unused with GDN_GATES_PRECOMPUTED)
+ *   h0 [B,Hv,dk,dv] float32, read; NULL = zero initial state
+ *   o  [B,T,Hv,dv] dtype (float32 with GDN_OUT_F32), written
+ *   ht [B,Hv,dk,dv] float32, written; NULL = not stored; may alias h0
+ *   flags: GDN_QK_L2NORM | GDN_GATES_PRECOMPUTED | GDN_OUT_F32; scale
+ *     multiplies q after the norm (pass 1/sqrt(dk) for the usual scaling).
+ *   workspace / ws_bytes: unused by the current kernels (may be NULL / 0);
+ *     gdn_chunk_workspace_bytes() returns the size a call needs.
+ *   T may be any value >= 0 (a partial last chunk is masked); T = 0 copies h0
+ *   to ht (or zeros).
+ */
+int gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
+                  const void* b, const float* A_log, const float* dt_bias,
+                  const float* h0, int B, int T, int Hk, int Hv, int dk, int dv,
+                  int dtype, float scale, int flags, void* o, float* ht,
+                  void* workspace, size_t ws_bytes, gdn_stream_t stream);
+
+size_t gdn_chunk_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv,
+                                 int dtype);
+
+/*
+ * gdn_recurrent_step -- one-token decode step for N independent sequences
+ * (recurrent_gated_delta_rule; "gated-deltanet-qwen3.5" inference branch,
+ * conv_states and recurrent_states updated in place), fused with the causal
+ * depthwise conv1d (kernel 4) + SiLU over the mixed [q | k | v] stream
+ * ("从 Full Attention 到 Gated DeltaNet" section 10).
+ *   x_qkv      [N, Cc] dtype, Cc = 2*Hk*dk + Hv*dv, channel order q | k | v;
+ *              pre-conv input when conv_w != NULL, else already post-conv
+ *   conv_w     [Cc, 4] float32 or NULL; tap 3 multiplies the newest input
+ *   conv_state [N, Cc, 3] dtype, read and updated in place (index 2 newest);
+ *              ignored when conv_w == NULL
+ *   a, b       [N, Hv] dtype; A_log, dt_bias [Hv] float32
+ *   state      [N, Hv, dk, dv] float32, read and updated in place
+ *   o          [N, Hv, dv] dtype (float32 with GDN_OUT_F32), written
+ *   q and k are L2-normalised per head; q is multiplied by scale after that.
+ *   flags: 0 or GDN_OUT_F32.
+ */
+int gdn_recurrent_step(const void* x_qkv, const float* conv_w, void* conv_state,
+                       const void* a, const void* b, const float* A_log,
+                       const float* dt_bias, float* state, void* o, int N,
+                       int Hk, int Hv, int dk, int dv, int dtype, float scale,
+                       int flags, gdn_stream_t stream);
+
+/*
+ * gdn2_chunk_fwd -- chunkwise Gated DeltaNet-2 forward ("Gated DeltaNet-2",
+ * 新更新公式 and 高效训练): channel-wise decay
+ * D_t = diag(exp(-exp(A_log) (.) softplus(a_t + dt_bias))), erase gate
+ * b_t = sigmoid(b_logit_t), write gate w_t = sigmoid(w_logit_t),
+ * S_t = (I - k_t (b_t (.) k_t)^T) D_t S_{t-1} + k_t (w_t (.) v_t)^T,
+ * o_t = S_t^T q_t.  One key head per value head (H heads).
+ *   q, k    [B,T,H,dk]  dtype      v  [B,T,H,dv] dtype
+ *   a,
+ *   b_logit [B,T,H,dk]  dtype      w_logit [B,T,H,dv] dtype
+ *     (with GDN_GATES_PRECOMPUTED: a = per-channel log-decay g, b_logit = b,
+ *      w_logit = w, all float32)
+ *   A_log, dt_bias [H,dk] float32 (unused with GDN_GATES_PRECOMPUTED)
+ *   h0, ht [B,H,dk,dv] float32 (NULL allowed; ht may alias h0)
+ *   o [B,T,H,dv] dtype (float32 with GDN_OUT_F32), written
+ */
+int gdn2_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
+                   const void* b_logit, const void* w_logit, const float* A_log,
+                   const float* dt_bias, const float* h0, int B, int T, int H,
+                   int dk, int dv, int dtype, float scale, int flags, void* o,
+                   float* ht, void* workspace, size_t ws_bytes,
+                   gdn_stream_t stream);
+
+size_t gdn2_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
+
+/*
+ * gdn_check_status -- waits for `stream`, then reads and clears the device
+ * status word of the current device.  Returns GDN_OK, GDN_ERR_TIMEOUT if a
+ * bounded wait in a kernel expired since the last check, or GDN_ERR_CUDA.
+ */
+int gdn_check_status(gdn_stream_t stream);
+
+/* Human-readable name of a gdn_status value (static string). */
+const char* gdn_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_B200_GDN_H_ */

@@ -1,0 +1,109 @@
+"""The C-ABI library loads, exports every entry point include/gdn.h declares,
+and rejects bad arguments on the host before touching a GPU (no CUDA call is
+made on these paths, so they run without a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+import gated_deltanet_sequence_gdn_b200 as G  # noqa: E402
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced on the host paths tested
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(gdn2?_\w+)\s*\(", src,
+                                 flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("gdn_gate_prep", "gdn_chunk_fwd", "gdn_recurrent_step", "gdn2_chunk_fwd",
+              "gdn_check_status", "gdn_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(G.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in gdn.h but not exported"
+
+
+def test_only_declared_symbols_are_exported():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", G.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = sorted(l.split()[-1] for l in out.splitlines() if l.strip())
+    assert exported == declared_functions()
+
+
+def test_status_strings_and_version():
+    assert G.lib.gdn_status_string(0) == b"GDN_OK"
+    assert G.lib.gdn_status_string(-1) == b"GDN_ERR_INVALID_ARG"
+    assert G.lib.gdn_status_string(-4) == b"GDN_ERR_TIMEOUT"
+    assert G.lib.gdn_status_string(12345) == b"GDN_ERR_UNKNOWN"
+    assert G.lib.gdn_version() >= 100
+
+
+def test_no_workspace_needed():
+    assert G.lib.gdn_chunk_workspace_bytes(1, 8192, 16, 64, 128, 128, 1) == 0
+    assert G.lib.gdn2_chunk_workspace_bytes(4, 4096, 16, 128, 128, 1) == 0
+
+
+def _chunk(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, a=FAKE, b=FAKE, A_log=FAKE, dt_bias=FAKE, h0=None,
+                B=1, T=64, Hk=2, Hv=4, dk=128, dv=128, dtype=1, scale=0.1, flags=1, o=FAKE,
+                ht=None)
+    args.update(kw)
+    return G.lib.gdn_chunk_fwd(args["q"], args["k"], args["v"], args["a"], args["b"],
+                               args["A_log"], args["dt_bias"], args["h0"], args["B"],
+                               args["T"], args["Hk"], args["Hv"], args["dk"], args["dv"],
+                               args["dtype"], args["scale"], args["flags"], args["o"],
+                               args["ht"], None, 0, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), -1), (dict(o=None), -1), (dict(a=None), -1),
+    (dict(q=FAKE + 2), -1), (dict(h0=FAKE + 8), -1), (dict(ht=FAKE + 4), -1),
+    (dict(dtype=7), -1), (dict(B=-1), -1), (dict(T=-5), -1), (dict(flags=8), -1),
+    (dict(flags=16), -1),
+    (dict(A_log=None), -1), (dict(Hk=0), -1),
+    (dict(dk=96), -2), (dict(dv=32), -2), (dict(Hk=3, Hv=4), -2),
+])
+def test_chunk_rejects_bad_arguments(kw, expect):
+    assert _chunk(**kw) == expect
+
+
+def test_gdn2_and_decode_reject_bad_arguments():
+    L = G.lib
+    assert L.gdn2_chunk_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, 1, 64, 2,
+                            128, 128, 1, 0.1, 1, FAKE, None, None, 0, None) == -1
+    assert L.gdn2_chunk_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 64, 2,
+                            100, 128, 1, 0.1, 1, FAKE, None, None, 0, None) == -2
+    # decode: conv weights given but no conv state
+    assert L.gdn_recurrent_step(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 4,
+                                128, 128, 1, 0.1, 0, None) == -1
+    assert L.gdn_recurrent_step(FAKE, None, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 4, 6,
+                                128, 128, 1, 0.1, 0, None) == -2
+    assert L.gdn_recurrent_step(FAKE, None, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 4,
+                                128, 128, 1, 0.1, 1, None) == -1
+    assert L.gdn_gate_prep(FAKE, FAKE, 1, FAKE, FAKE, FAKE, FAKE, 1, 8, 2, 4, 80, 0.1, FAKE,
+                           FAKE, FAKE, FAKE, None) == -2
+    assert L.gdn_gate_prep(FAKE, None, 1, FAKE, FAKE, FAKE, FAKE, 1, 8, 2, 4, 128, 0.1, FAKE,
+                           FAKE, FAKE, FAKE, None) == -1
+
+
+def test_empty_calls_are_no_ops():
+    # zero tokens / zero sequences return before any launch (no state pointers)
+    assert _chunk(T=0) == 0
+    assert _chunk(B=0) == 0
+    assert G.lib.gdn_recurrent_step(FAKE, None, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2,
+                                    4, 128, 128, 1, 0.1, 0, None) == 0
+    assert G.lib.gdn_gate_prep(FAKE, FAKE, 1, FAKE, FAKE, FAKE, FAKE, 1, 0, 2, 4, 128, 0.1,
+                               FAKE, FAKE, FAKE, FAKE, None) == 0
