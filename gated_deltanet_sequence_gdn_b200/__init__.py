@@ -17,7 +17,8 @@ import os
 
 import torch
 
-__all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_recurrent_step", "gdn2_chunk_fwd",
+__all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_chunk_workspace_bytes", "gdn_recurrent_step",
+           "gdn2_chunk_fwd",
            "gdn_check_status", "GDNError", "LIB_PATH", "lib", "F32", "BF16",
            "QK_L2NORM", "GATES_PRECOMPUTED", "OUT_F32"]
 
@@ -118,13 +119,20 @@ def gdn_gate_prep(q, k, a, b, A_log, dt_bias, *, scale=None, q_out=None, k_out=N
     return q_out, k_out, g_out, beta_out
 
 
+def gdn_chunk_workspace_bytes(B, T, Hk, Hv, dk, dv, dtype) -> int:
+    """Bytes of device workspace gdn_chunk_fwd needs for these sizes (0 = none)."""
+    return int(lib.gdn_chunk_workspace_bytes(B, T, Hk, Hv, dk, dv, _dtype_code(dtype)))
+
+
 def gdn_chunk_fwd(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, scale=None,
                   l2norm=True, gates_precomputed=False, out_f32=False, o=None, ht=None,
-                  want_ht=True, stream=None):
+                  want_ht=True, workspace=None, stream=None):
     """Chunkwise GDN prefill. q, k [B,T,Hk,dk]; v [B,T,Hv,dv]; a, b [B,T,Hv]
     (float32 g, beta with gates_precomputed); A_log, dt_bias [Hv] float32;
     h0 [B,Hv,dk,dv] float32 or None.  Returns (o [B,T,Hv,dv], ht or None);
-    o has the input dtype, or float32 with out_f32."""
+    o has the input dtype, or float32 with out_f32.  workspace: a uint8 CUDA
+    tensor of at least gdn_chunk_workspace_bytes(...) bytes, allocated here
+    when None."""
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     dt = q.dtype
@@ -143,9 +151,13 @@ def gdn_chunk_fwd(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, scale=Non
         ht = torch.empty((B, Hv, dk, dv), device=q.device, dtype=torch.float32)
     flags = ((QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
              | (OUT_F32 if out_f32 else 0))
+    ws_need = gdn_chunk_workspace_bytes(B, T, Hk, Hv, dk, dv, dt)
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.gdn_chunk_fwd(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(dt_bias), _p(h0),
                              B, T, Hk, Hv, dk, dv, _dtype_code(dt), float(scale), flags, _p(o),
-                             _p(ht), None, 0, _stream(stream)), "gdn_chunk_fwd")
+                             _p(ht), _p(workspace), ws_bytes, _stream(stream)), "gdn_chunk_fwd")
     return o, ht
 
 

@@ -88,7 +88,12 @@ int gdn_gate_prep(const void* q, const void* k, int dtype, const void* a, const 
                                     q_out, k_out, g_out, beta_out, (cudaStream_t)stream));
 }
 
-size_t gdn_chunk_workspace_bytes(int, int, int, int, int, int, int) { return 0; }
+size_t gdn_chunk_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int dtype) {
+  if (B <= 0 || T <= 0 || Hk <= 0 || Hv <= 0 || Hv % Hk != 0) return 0;
+  ChunkArgs c{};
+  c.B = B; c.T = T; c.Hk = Hk; c.Hv = Hv; c.dk = dk; c.dv = dv; c.dtype = dtype;
+  return chunk_mma_supported(c) ? chunk_mma_workspace_bytes(B, T, Hv) : 0;
+}
 size_t gdn2_chunk_workspace_bytes(int, int, int, int, int, int) { return 0; }
 
 static int validate_chunk(const ChunkArgs& c, bool gdn2) {
@@ -109,11 +114,16 @@ static int validate_chunk(const ChunkArgs& c, bool gdn2) {
   return GDN_OK;
 }
 
-static int run_chunk(const ChunkArgs& c, bool gdn2, cudaStream_t s) {
+static int run_chunk(const ChunkArgs& c, bool gdn2, void* ws, size_t ws_bytes,
+                     cudaStream_t s) {
   const size_t state_elems = (size_t)c.B * c.Hv * c.dk * c.dv;
   if (c.T == 0 || c.B == 0) return from_cuda(launch_copy_state(c.h0, c.ht, state_elems, s));
-  if (!gdn2 && c.dtype == GDN_BF16 && chunk_tc_supported(c))
-    return from_cuda(launch_chunk_tc(c, s));
+  if (!gdn2 && chunk_mma_supported(c)) {
+    if (ws == nullptr || !aligned16(ws) ||
+        ws_bytes < chunk_mma_workspace_bytes(c.B, c.T, c.Hv))
+      return GDN_ERR_WORKSPACE;
+    return from_cuda(launch_chunk_mma(c, ws, s));
+  }
   return from_cuda(launch_chunk_simt(c, gdn2, s));
 }
 
@@ -121,13 +131,11 @@ int gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* a, co
                   const float* A_log, const float* dt_bias, const float* h0, int B, int T,
                   int Hk, int Hv, int dk, int dv, int dtype, float scale, int flags, void* o,
                   float* ht, void* workspace, size_t ws_bytes, gdn_stream_t stream) {
-  (void)workspace;
-  (void)ws_bytes;
   ChunkArgs c{q, k, v, a, b, nullptr, A_log, dt_bias, h0, B, T, Hk, Hv, dk, dv, dtype,
               scale, flags, o, ht};
   int st = validate_chunk(c, false);
   if (st != GDN_OK) return st;
-  return run_chunk(c, false, (cudaStream_t)stream);
+  return run_chunk(c, false, workspace, ws_bytes, (cudaStream_t)stream);
 }
 
 int gdn2_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
@@ -135,13 +143,11 @@ int gdn2_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
                    const float* dt_bias, const float* h0, int B, int T, int H, int dk, int dv,
                    int dtype, float scale, int flags, void* o, float* ht, void* workspace,
                    size_t ws_bytes, gdn_stream_t stream) {
-  (void)workspace;
-  (void)ws_bytes;
   ChunkArgs c{q, k, v, a, b_logit, w_logit, A_log, dt_bias, h0, B, T, H, H, dk, dv, dtype,
               scale, flags, o, ht};
   int st = validate_chunk(c, true);
   if (st != GDN_OK) return st;
-  return run_chunk(c, true, (cudaStream_t)stream);
+  return run_chunk(c, true, workspace, ws_bytes, (cudaStream_t)stream);
 }
 
 int gdn_recurrent_step(const void* x_qkv, const float* conv_w, void* conv_state, const void* a,

@@ -1,0 +1,81 @@
+// warp_mma.cuh -- warp-level tensor-core building blocks in inline PTX:
+// ldmatrix (plain and transposed), mma.sync m16n8k16 bf16 -> fp32, and
+// cp.async 16-byte copies with zero fill and group waits.
+//
+// Fragment layouts (PTX ISA, "Matrix fragments for mma.m16n8k16"), with
+// g = lane / 4 and t = lane % 4:
+//   A 16x16 (row-major): a0 = (g, 2t..2t+1), a1 = (g+8, 2t..), a2 = (g, 2t+8..),
+//                        a3 = (g+8, 2t+8..)
+//   B 16x8  (k x n):     b0 = (k 2t..2t+1, n g), b1 = (k 2t+8.., n g)
+//   C 16x8  (fp32):      c0,c1 = (g, 2t..2t+1), c2,c3 = (g+8, 2t..2t+1)
+#pragma once
+
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace gdn {
+namespace wm {
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Four 8x8 b16 matrices; lane l supplies the row address of matrix l / 8.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+
+// D = A B + D, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Per-lane offsets of the ldmatrix row addresses (in elements):
+//  tile_a : A operand from a row-major [m][k] tile, also the B operand (two n8
+//           tiles) from a row-major [k][n] tile with ldsm_x4_t;
+//           row += (l % 8) + 8 * ((l / 8) % 2), col += 8 * (l / 16).
+//  tile_bn: B operand (two n8 tiles) from an [n][k] tile (k contiguous) with
+//           ldsm_x4; row(n) += (l % 8) + 8 * (l / 16), col(k) += 8 * ((l / 8) % 2).
+//  tile_at: A operand from a [k][m] tile (m contiguous) with ldsm_x4_t;
+//           row(k) += (l % 8) + 8 * (l / 16), col(m) += 8 * ((l / 8) % 2).
+__device__ __forceinline__ int lrow_a(int l) { return (l & 7) + ((l >> 3) & 1) * 8; }
+__device__ __forceinline__ int lcol_a(int l) { return (l >> 4) * 8; }
+__device__ __forceinline__ int lrow_b(int l) { return (l & 7) + (l >> 4) * 8; }
+__device__ __forceinline__ int lcol_b(int l) { return ((l >> 3) & 1) * 8; }
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack2(uint32_t u) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+}
+
+// 16-byte global -> shared copy; src_bytes = 0 fills the 16 bytes with zeros
+// (src must still be a valid address).
+__device__ __forceinline__ void cp16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+}  // namespace wm
+}  // namespace gdn

@@ -101,8 +101,11 @@ int gdn_gate_prep(const void* q, const void* k, int dtype, const void* a,
  * U~ = U - W S, O = diag(gamma) Q S + tril(Q K^T (.) Gamma) U~,
  * S <- gamma_C S + (diag(gamma_C/gamma) K)^T U~  ("Gated DeltaNet-2",
  * 高效训练, with scalar decay).  The float32 state stays on chip across the
- * chunks of one (batch, value head).  bf16 runs on the tcgen05 tensor cores;
- * float32 runs a float32 CUDA-core path.
+ * chunks of one (batch, value head, 64 value columns).  bf16 with
+ * dk = dv = 128 runs on the tensor cores in two kernels (a chunk-parallel WY
+ * prep that writes W, U, A_qk and per-row factors to the workspace, then a
+ * scan over the chunks that keeps the state in registers); other shapes and
+ * float32 run a float32 CUDA-core path with no workspace.
  *   q, k [B,T,Hk,dk], v [B,T,Hv,dv], a, b [B,T,Hv]: dtype, read
  *     (with GDN_GATES_PRECOMPUTED: a = g, b = beta, float32)
  *   A_log, dt_bias [Hv] float32, read (unused with GDN_GATES_PRECOMPUTED)
@@ -111,8 +114,10 @@ int gdn_gate_prep(const void* q, const void* k, int dtype, const void* a,
  *   ht [B,Hv,dk,dv] float32, written; NULL = not stored; may alias h0
  *   flags: GDN_QK_L2NORM | GDN_GATES_PRECOMPUTED | GDN_OUT_F32; scale
  *     multiplies q after the norm (pass 1/sqrt(dk) for the usual scaling).
- *   workspace / ws_bytes: unused by the current kernels (may be NULL / 0);
- *     gdn_chunk_workspace_bytes() returns the size a call needs.
+ *   workspace / ws_bytes: device scratch owned by the caller, 16-byte aligned,
+ *     at least gdn_chunk_workspace_bytes() bytes (may be NULL / 0 when that
+ *     returns 0); its contents are overwritten and need no initialisation.
+ *     Too small or misaligned -> GDN_ERR_WORKSPACE, nothing launched.
  *   T may be any value >= 0 (a partial last chunk is masked); T = 0 copies h0
  *   to ht (or zeros).
  */
@@ -122,6 +127,11 @@ int gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
                   int dtype, float scale, int flags, void* o, float* ht,
                   void* workspace, size_t ws_bytes, gdn_stream_t stream);
 
+/* Workspace bytes gdn_chunk_fwd needs for these sizes: for the tensor-core
+ * path (bf16, dk = dv = 128) B*Hv*(Tp*1024 + (Tp/64)*528) with Tp = T rounded
+ * up to a multiple of 64 (per padded token and value head: a W row of 128 bf16,
+ * a U row of 128 float32, A_qk rows of 64 bf16 in two parts; 528 B of factors
+ * per chunk); 0 for every other case and for B*T = 0. */
 size_t gdn_chunk_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv,
                                  int dtype);
 

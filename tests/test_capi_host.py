@@ -51,21 +51,41 @@ def test_status_strings_and_version():
     assert G.lib.gdn_version() >= 100
 
 
-def test_no_workspace_needed():
-    assert G.lib.gdn_chunk_workspace_bytes(1, 8192, 16, 64, 128, 128, 1) == 0
+def test_workspace_sizes():
+    """Tensor-core path (bf16, d = 128): per padded token and value head a W row
+    (256 B), a float32 U row (512 B) and two A_qk rows (2 x 128 B); 528 B of
+    factors per chunk and value head."""
+    ws = G.lib.gdn_chunk_workspace_bytes
+    assert ws(1, 8192, 16, 64, 128, 128, 1) == 64 * (8192 * 1024 + 128 * 528)
+    assert ws(2, 100, 2, 4, 128, 128, 1) == 2 * 4 * (128 * 1024 + 2 * 528)
+    assert ws(1, 64, 1, 1, 128, 128, 1) == 1024 * 64 + 528
+    # no workspace: float32, other head sizes, empty inputs, Gated DeltaNet-2
+    assert ws(1, 8192, 16, 64, 128, 128, 0) == 0
+    assert ws(1, 256, 2, 2, 64, 64, 1) == 0
+    assert ws(0, 256, 2, 2, 128, 128, 1) == 0
+    assert ws(1, 0, 2, 2, 128, 128, 1) == 0
     assert G.lib.gdn2_chunk_workspace_bytes(4, 4096, 16, 128, 128, 1) == 0
+
+
+def test_missing_workspace_rejected():
+    """A bf16 d = 128 call without (enough) workspace is refused before any launch."""
+    assert _chunk() == -5
+    need = 4 * (1024 * 64 + 528)  # B=1, T=64, Hv=4
+    assert _chunk(ws=FAKE, ws_bytes=need - 1) == -5
+    assert _chunk(ws=FAKE + 8, ws_bytes=1 << 20) == -5  # misaligned
+    assert _chunk(ws=FAKE, ws_bytes=need, flags=9) == -1  # a bad flag is reported first
 
 
 def _chunk(**kw):
     args = dict(q=FAKE, k=FAKE, v=FAKE, a=FAKE, b=FAKE, A_log=FAKE, dt_bias=FAKE, h0=None,
                 B=1, T=64, Hk=2, Hv=4, dk=128, dv=128, dtype=1, scale=0.1, flags=1, o=FAKE,
-                ht=None)
+                ht=None, ws=None, ws_bytes=0)
     args.update(kw)
     return G.lib.gdn_chunk_fwd(args["q"], args["k"], args["v"], args["a"], args["b"],
                                args["A_log"], args["dt_bias"], args["h0"], args["B"],
                                args["T"], args["Hk"], args["Hv"], args["dk"], args["dv"],
                                args["dtype"], args["scale"], args["flags"], args["o"],
-                               args["ht"], None, 0, None)
+                               args["ht"], args["ws"], args["ws_bytes"], None)
 
 
 @pytest.mark.parametrize("kw,expect", [

@@ -64,7 +64,8 @@ def test_chunk_tiny_fp32_workload():
 
 SHAPES = [  # B, T, Hk, Hv, d
     (1, 1, 1, 1, 128), (1, 63, 1, 2, 128), (2, 64, 2, 2, 64), (1, 65, 2, 4, 128),
-    (2, 100, 1, 4, 64), (1, 200, 2, 8, 128), (1, 384, 16, 64, 128),
+    (2, 100, 1, 4, 64), (1, 200, 2, 8, 128), (1, 384, 16, 64, 128), (3, 130, 2, 4, 128),
+    (2, 1000, 2, 2, 128),
 ]
 
 
@@ -97,6 +98,22 @@ def test_chunk_zero_initial_state_and_in_place_state(dtype):
     ro2, rht2 = _oracle_gdn(x)
     assert ht2.data_ptr() == h.data_ptr()
     assert rel_err(o2, ro2) <= TOL[dtype] and rel_err(h, rht2) <= TOL[dtype]
+
+
+def test_chunk_workspace_reuse_and_size_check():
+    """The workspace carries nothing from call to call: one NaN-filled buffer
+    serves two different problems; a workspace one chunk-row short is refused."""
+    shape = (2, 190, 2, 4, 128)
+    need = G.gdn_chunk_workspace_bytes(*shape, 128, torch.bfloat16)
+    assert need > 0
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=DEV)  # bf16 0xFFFF = NaN
+    for seed in (21, 22):
+        x = gdn_inputs(*shape, torch.bfloat16, seed=seed, device=DEV)
+        o, ht = _gpu_gdn(x, workspace=ws)
+        ro, rht = _oracle_gdn(x)
+        assert rel_err(o, ro) <= 2e-2 and rel_err(ht, rht) <= 2e-2
+    with pytest.raises(G.GDNError):
+        _gpu_gdn(x, workspace=ws[: need - 16])
 
 
 def test_chunk_empty_sequence_copies_state():
