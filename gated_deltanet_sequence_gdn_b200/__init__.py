@@ -7,8 +7,8 @@ Python fallback: importing this module fails if the library is not built, and
 every call raises if the library reports an error.
 
 Entry points (same names as the C ABI):
-    gdn_gate_prep, gdn_chunk_fwd, gdn_recurrent_step, gdn2_chunk_fwd,
-    gdn_check_status
+    gdn_gate_prep, gdn_chunk_fwd, gdn_chunk_workspace_bytes, gdn_chunk_fwd_noalloc,
+    gdn_recurrent_step, gdn2_chunk_fwd, gdn_check_status
 """
 from __future__ import annotations
 
@@ -18,7 +18,7 @@ import os
 import torch
 
 __all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_chunk_workspace_bytes", "gdn_recurrent_step",
-           "gdn2_chunk_fwd",
+           "gdn2_chunk_fwd", "gdn_chunk_fwd_noalloc",
            "gdn_check_status", "GDNError", "LIB_PATH", "lib", "F32", "BF16",
            "QK_L2NORM", "GATES_PRECOMPUTED", "OUT_F32"]
 
@@ -42,6 +42,7 @@ lib.gdn_gate_prep.argtypes = [_vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, 
                               _vp, _vp, _vp, _vp, _vp]
 lib.gdn_chunk_fwd.argtypes = [_vp] * 8 + [_i] * 7 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
 lib.gdn2_chunk_fwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
+lib.gdn_chunk_fwd_noalloc.argtypes = [_vp] * 8 + [_i] * 7 + [_f, _i, _vp, _vp, _vp]
 lib.gdn_recurrent_step.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _vp]
 lib.gdn_chunk_workspace_bytes.argtypes = [_i] * 7
 lib.gdn2_chunk_workspace_bytes.argtypes = [_i] * 6
@@ -51,8 +52,8 @@ lib.gdn_check_status.argtypes = [_vp]
 lib.gdn_status_string.argtypes = [_i]
 lib.gdn_status_string.restype = ctypes.c_char_p
 lib.gdn_version.argtypes = []
-for _fn in (lib.gdn_gate_prep, lib.gdn_chunk_fwd, lib.gdn2_chunk_fwd, lib.gdn_recurrent_step,
-            lib.gdn_check_status, lib.gdn_version):
+for _fn in (lib.gdn_gate_prep, lib.gdn_chunk_fwd, lib.gdn_chunk_fwd_noalloc, lib.gdn2_chunk_fwd,
+            lib.gdn_recurrent_step, lib.gdn_check_status, lib.gdn_version):
     _fn.restype = _i
 
 
@@ -158,6 +159,36 @@ def gdn_chunk_fwd(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, scale=Non
     _check(lib.gdn_chunk_fwd(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(dt_bias), _p(h0),
                              B, T, Hk, Hv, dk, dv, _dtype_code(dt), float(scale), flags, _p(o),
                              _p(ht), _p(workspace), ws_bytes, _stream(stream)), "gdn_chunk_fwd")
+    return o, ht
+
+
+def gdn_chunk_fwd_noalloc(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, scale=None,
+                          l2norm=True, gates_precomputed=False, out_f32=False, o=None, ht=None,
+                          want_ht=True, stream=None):
+    """gdn_chunk_fwd with the library's fixed 64 MiB device scratch instead of a
+    workspace (raises GDNError(GDN_ERR_WORKSPACE) when the sizes need more)."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dt = q.dtype
+    scale = dk ** -0.5 if scale is None else scale
+    _need(k, dt, q.shape, "k")
+    _need(v, dt, (B, T, Hv, dv), "v")
+    gdt = torch.float32 if gates_precomputed else dt
+    _need(a, gdt, (B, T, Hv), "a")
+    _need(b, gdt, (B, T, Hv), "b")
+    if h0 is not None:
+        _need(h0, torch.float32, (B, Hv, dk, dv), "h0")
+    odt = torch.float32 if out_f32 else dt
+    o = torch.empty((B, T, Hv, dv), device=q.device, dtype=odt) if o is None else o
+    _need(o, odt, (B, T, Hv, dv), "o")
+    if ht is None and want_ht:
+        ht = torch.empty((B, Hv, dk, dv), device=q.device, dtype=torch.float32)
+    flags = ((QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
+             | (OUT_F32 if out_f32 else 0))
+    _check(lib.gdn_chunk_fwd_noalloc(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(dt_bias),
+                                     _p(h0), B, T, Hk, Hv, dk, dv, _dtype_code(dt), float(scale),
+                                     flags, _p(o), _p(ht), _stream(stream)),
+           "gdn_chunk_fwd_noalloc")
     return o, ht
 
 

@@ -136,6 +136,25 @@ size_t gdn_chunk_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv,
                                  int dtype);
 
 /*
+ * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd without a caller workspace.  The pages
+ * have no counterpart: this is a convenience of this library for callers that
+ * cannot hand out device memory.  The scratch is a fixed 64 MiB device array
+ * inside the library (one per device, reserved when this function is first
+ * used on that device); the call allocates nothing.
+ *   Arguments, layouts and results are those of gdn_chunk_fwd.
+ *   Capacity: calls with gdn_chunk_workspace_bytes(...) > 64 MiB return
+ *     GDN_ERR_WORKSPACE and launch nothing (argument errors are reported
+ *     first); calls that need no workspace run as gdn_chunk_fwd does.
+ *   The array is shared by every call on a device: calls on different
+ *     streams must not run concurrently (calls on one stream are ordered).
+ */
+int gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                          const void* a, const void* b, const float* A_log,
+                          const float* dt_bias, const float* h0, int B, int T,
+                          int Hk, int Hv, int dk, int dv, int dtype, float scale,
+                          int flags, void* o, float* ht, gdn_stream_t stream);
+
+/*
  * gdn_recurrent_step -- one-token decode step for N independent sequences
  * (recurrent_gated_delta_rule; "gated-deltanet-qwen3.5" inference branch,
  * conv_states and recurrent_states updated in place), fused with the causal
