@@ -117,6 +117,20 @@ def rank_info():
     return 0, 0, 1
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest of the ranks' values (the job's time is its slowest rank's)."""
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_rate(units_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes units_per_rank per step (weak
+    scaling, independent replicas), the step takes the slowest rank's time."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 def kernel_traffic(name):
     """dram bytes per launch from a committed ncu summary, if its kernel source
     hash still matches the current source (else None)."""
@@ -194,12 +208,9 @@ def run_ours(args, rank, local_rank, world):
     t1 = time.time()
     clk = clocks.stop(t0, t1)
     G.gdn_check_status(stream)
-    ms = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    ms_step = ms.item() / args.steps
+    ms_step = max_over_ranks(total_ms, dev) / args.steps
     tokens = w.B * w.T
-    value = world * tokens / (ms_step / 1e3)
+    value = job_rate(tokens, world, ms_step)
     flop = CHUNK_FLOP_PER_TOKEN_HEAD * w.T * w.Hv * w.B
     launch_ms = sum(per) / len(per)
     achieved = flop / (launch_ms / 1e3) / 1e12
@@ -264,11 +275,8 @@ def measure_e2e(G, x, w, dev, stream, args, world):
 
     steps = max(3, min(args.steps, 20))
     total_ms, _ = time_steps(step, steps, 2, stream, sync_group=world > 1)
-    ms = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    ms_step = ms.item() / steps
-    return {"value": round(world * w.B * w.T / (ms_step / 1e3), 1), "unit": "tokens/s",
+    ms_step = max_over_ranks(total_ms, dev) / steps
+    return {"value": round(job_rate(w.B * w.T, world, ms_step), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms_step, 4), "steps": steps,
             "path": "pinned host -> gdn_chunk_fwd (C ABI) -> pinned host"}
@@ -434,7 +442,7 @@ def main():
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the decode / GDN-2 / long-prefill extras")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["decode_256", "gdn2_b4_4k", "prefill_128k",
+    ap.add_argument("--only", choices=["prefill_8k", "decode_256", "gdn2_b4_4k", "prefill_128k",
                                        "prefill_b8_16k"], default=None,
                     help="measure one secondary workload alone (profiling runs)")
     args = ap.parse_args()

@@ -1,10 +1,11 @@
 // chunk_mma.cu -- bf16 chunkwise GDN forward (dk = dv = 128, chunk C = 64) on
 // the tensor cores, in two kernels:
 //
-//  wy_prep_kernel  : one CTA per (chunk, key head), parallel over the whole
-//      sequence.  Forms the raw Gram matrices K K^T and Q K^T once per key head
-//      (bf16 mma, fp32 accumulation) and, for each value head of the GQA group,
-//      the gates and their in-chunk prefix sums G_r, the strictly lower
+//  wy_prep_kernel  : one CTA per (chunk, value head), parallel over the whole
+//      sequence; the CTAs of one GQA group are launched next to each other so
+//      their shared K / Q tiles come from L2.  Forms the Gram matrices K K^T and
+//      Q K^T (bf16 mma, fp32 accumulation) with the gates applied in registers:
+//      the in-chunk prefix sums G_r of the log-decays, the strictly lower
 //      L = diag(beta) (K^ K^^T o Gamma), X = (I + L)^-1 by blocked forward
 //      substitution in fp32, W = X diag(beta gamma) K^, U = X diag(beta) V and
 //      A_qk = tril(Q^ K^^T o Gamma) (diagonal included), written to the
@@ -68,33 +69,19 @@ __device__ __forceinline__ void split2(float x, float y, uint32_t& hi, uint32_t&
 }
 
 // ---------------------------------------------------------------- prep kernel
-constexpr int P_KT = 0;                     // K tile  [64][LDT] bf16
-constexpr int P_QT = P_KT + kC * LDT * 2;   // Q tile
-constexpr int P_VT = P_QT + kC * LDT * 2;   // V tile of one value head
-constexpr int P_ST = P_VT + kC * LDT * 2;   // staging of W / U for coalesced stores
-constexpr int P_KK = P_ST + kC * LDT * 2;   // raw K K^T [64][LDF] f32
-constexpr int P_QK = P_KK + kC * LDF * 4;   // raw Q K^T
-constexpr int P_L = P_QK + kC * LDF * 4;    // L
-constexpr int P_X = P_L + kC * LDF * 4;     // X = (I + L)^-1
-constexpr int P_T = P_X + kC * LDF * 4;     // block products [3][16][17] f32
-constexpr int P_A1 = P_T + 3 * 16 * 17 * 4; // X diag(beta gamma rk) [64][LDH] bf16
-constexpr int P_A2 = P_A1 + kC * LDH * 2;   // X diag(beta), hi part
-constexpr int P_A2L = P_A2 + kC * LDH * 2;  // X diag(beta), lo part
-constexpr int P_VEC = P_A2L + kC * LDH * 2; // rk, sq, G, beta [64] + misc
-constexpr int P_BYTES = P_VEC + 5 * 64 * 4;
-
-__device__ __forceinline__ void st16_bf16(bf16* dst, const float* v) {
-  uint4 p0, p1;
-  p0.x = pack2(v[0], v[1]);   p0.y = pack2(v[2], v[3]);
-  p0.z = pack2(v[4], v[5]);   p0.w = pack2(v[6], v[7]);
-  p1.x = pack2(v[8], v[9]);   p1.y = pack2(v[10], v[11]);
-  p1.z = pack2(v[12], v[13]); p1.w = pack2(v[14], v[15]);
-  reinterpret_cast<uint4*>(dst)[0] = p0;
-  reinterpret_cast<uint4*>(dst)[1] = p1;
-}
+constexpr int LDX = 64 + 8;                  // f32 row stride of L and X (conflict-free float2)
+constexpr int P_KT = 0;                      // K tile  [64][LDT] bf16 (key head)
+constexpr int P_QT = P_KT + kC * LDT * 2;    // Q tile  (key head)
+constexpr int P_VT = P_QT + kC * LDT * 2;    // V tile  (value head)
+constexpr int P_L = P_VT + kC * LDT * 2;     // L [64][LDX] f32
+constexpr int P_X = P_L + kC * LDX * 4;      // X = (I + L)^-1
+constexpr int P_T = P_X + kC * LDX * 4;      // block products [3][16][17] f32
+constexpr int P_VEC = P_T + 3 * 16 * 17 * 4; // rk, sq, G, beta, c1 [64] + misc
+constexpr int P_BYTES = P_VEC + 6 * 64 * 4;
+static_assert(2 * (P_BYTES + 1024) <= 228 * 1024, "two prep CTAs per SM");
 
 template <bool PRE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                const void* __restrict__ ga, const void* __restrict__ gb,
                const float* __restrict__ A_log, const float* __restrict__ dt_bias, int T, int Hk,
@@ -103,39 +90,67 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
   bf16* Kt = reinterpret_cast<bf16*>(sm + P_KT);
   bf16* Qt = reinterpret_cast<bf16*>(sm + P_QT);
   bf16* Vt = reinterpret_cast<bf16*>(sm + P_VT);
-  bf16* St = reinterpret_cast<bf16*>(sm + P_ST);
-  float* KK = reinterpret_cast<float*>(sm + P_KK);
-  float* QK = reinterpret_cast<float*>(sm + P_QK);
   float* Lm = reinterpret_cast<float*>(sm + P_L);
   float* Xm = reinterpret_cast<float*>(sm + P_X);
   float* Tm = reinterpret_cast<float*>(sm + P_T);
-  bf16* A1 = reinterpret_cast<bf16*>(sm + P_A1);
-  bf16* A2 = reinterpret_cast<bf16*>(sm + P_A2);
-  bf16* A2l = reinterpret_cast<bf16*>(sm + P_A2L);
   float* rk = reinterpret_cast<float*>(sm + P_VEC);
   float* sq = rk + 64;
   float* Gs = sq + 64;
   float* bet = Gs + 64;
-  float* misc = bet + 64;
+  float* c1 = bet + 64;
+  float* misc = c1 + 64;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
-  const int n = blockIdx.x, Nc = gridDim.x, Tp = Nc * kC;
-  const int b = blockIdx.y / Hk, hk = blockIdx.y % Hk, G = Hv / Hk;
+  const int G = Hv / Hk;
+  const int n = blockIdx.y, Nc = gridDim.y, Tp = Nc * kC;
+  const int b = blockIdx.z / Hk, hk = blockIdx.z % Hk, hv = hk * G + blockIdx.x;
+  const size_t head = (size_t)b * Hv + hv;
   const int t0 = n * kC, nv = min(kC, T - t0);
 
-  // 1. raw K and Q tiles of the chunk (rows past the end of the sequence are zeros)
-  for (int i = tid; i < 2 * kC * 16; i += kThreads) {
+  // 1. raw K, Q tiles of the key head and the V tile of this value head (rows
+  //    past the end of the sequence are zeros)
+  for (int i = tid; i < 3 * kC * 16; i += kThreads) {
     const int which = i >> 10, r = (i >> 4) & 63, c16 = i & 15;
     const bool ok = r < nv;
-    const size_t off = ok ? ((((size_t)b * T + t0 + r) * Hk + hk) * kD + c16 * 8) : 0;
-    cp16((which ? Qt : Kt) + r * LDT + c16 * 8, (which ? q : k) + off, ok ? 16 : 0);
+    size_t off = 0;
+    if (ok)
+      off = which < 2 ? ((((size_t)b * T + t0 + r) * Hk + hk) * kD + c16 * 8)
+                      : ((((size_t)b * T + t0 + r) * Hv + hv) * kD + c16 * 8);
+    bf16* dst = (which == 0 ? Kt : (which == 1 ? Qt : Vt)) + r * LDT + c16 * 8;
+    cp16(dst, (which == 0 ? k : (which == 1 ? q : v)) + off, ok ? 16 : 0);
   }
   cp_commit();
+
+  // 2. gates (zero past the end of the sequence) and their in-chunk prefix sums,
+  //    while the tiles land
+  if (tid < kC) {
+    float g = 0.f, be = 0.f;
+    if (tid < nv) {
+      const size_t idx = ((size_t)b * T + t0 + tid) * Hv + hv;
+      if (PRE) {
+        g = reinterpret_cast<const float*>(ga)[idx];
+        be = reinterpret_cast<const float*>(gb)[idx];
+      } else {
+        g = gdn_log_decay(__bfloat162float(reinterpret_cast<const bf16*>(ga)[idx]), A_log[hv],
+                          dt_bias[hv]);
+        be = sigmoid_f(__bfloat162float(reinterpret_cast<const bf16*>(gb)[idx]));
+      }
+    }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, g, off);
+      if (lane >= off) g += y;
+    }
+    if (tid == 31) misc[0] = g;
+    Gs[tid] = g;
+    bet[tid] = be;
+  }
   cp_wait<0>();
   __syncthreads();
+  if (tid >= 32 && tid < kC) Gs[tid] += misc[0];
 
-  // 2. L2 norms: rk = 1 / |k|, sq = scale / |q| (two threads per row)
+  //    L2 norms: rk = 1 / |k|, sq = scale / |q| (two threads per row)
   {
     const int which = tid >> 7, r = (tid & 127) >> 1, h = tid & 1;
     const bf16* row = (which ? Qt : Kt) + r * LDT + h * 64;
@@ -154,12 +169,17 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
       else rk[r] = inv;
     }
   }
+  __syncthreads();
+  if (tid < kC) c1[tid] = bet[tid] * __expf(Gs[tid]) * rk[tid];  // column factor of W
 
-  // 3. raw Gram matrices: warps 0-3 K K^T, warps 4-7 Q K^T (rows 16 * (warp % 4))
+  // 3. Gram matrices on the tensor cores with the gates applied in registers:
+  //    warps 0-3: L = strictly lower (beta_r rk_r rk_c e^(G_r - G_c) k_r.k_c) -> smem
+  //    warps 4-7: A_qk = lower incl. diagonal (sq_r rk_c e^(G_r - G_c) q_r.k_c),
+  //               stored to the workspace as bf16 hi + lo
   {
     const int mt = warp & 3;
-    const bf16* At = warp < 4 ? Kt : Qt;
-    float* dst = warp < 4 ? KK : QK;
+    const bool isq = warp >= 4;
+    const bf16* At = isq ? Qt : Kt;
     float acc[8][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -173,212 +193,147 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
         mma_bf16(acc[2 * np + 1], a, bb[2], bb[3]);
       }
     }
+    const int ra = 16 * mt + g8, rb = ra + 8;
+    const float Ga = Gs[ra], Gb = Gs[rb];
+    const float fa = isq ? sq[ra] : bet[ra] * rk[ra];
+    const float fb = isq ? sq[rb] : bet[rb] * rk[rb];
+    bf16* ahg = reinterpret_cast<bf16*>(ws + L.ah) + (head * Tp + t0) * kC;
+    bf16* alg = reinterpret_cast<bf16*>(ws + L.al) + (head * Tp + t0) * kC;
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
-      const int r0 = 16 * mt + g8, c = 8 * nt + 2 * t4;
-      dst[r0 * LDF + c] = acc[nt][0];
-      dst[r0 * LDF + c + 1] = acc[nt][1];
-      dst[(r0 + 8) * LDF + c] = acc[nt][2];
-      dst[(r0 + 8) * LDF + c + 1] = acc[nt][3];
+      const int c = 8 * nt + 2 * t4;
+      const float k0 = rk[c] * __expf(fminf(Ga - Gs[c], 0.f));
+      const float k1 = rk[c + 1] * __expf(fminf(Ga - Gs[c + 1], 0.f));
+      const float k2 = rk[c] * __expf(fminf(Gb - Gs[c], 0.f));
+      const float k3 = rk[c + 1] * __expf(fminf(Gb - Gs[c + 1], 0.f));
+      if (!isq) {
+        *reinterpret_cast<float2*>(Lm + ra * LDX + c) =
+            make_float2(c < ra ? fa * k0 * acc[nt][0] : 0.f, c + 1 < ra ? fa * k1 * acc[nt][1] : 0.f);
+        *reinterpret_cast<float2*>(Lm + rb * LDX + c) =
+            make_float2(c < rb ? fb * k2 * acc[nt][2] : 0.f, c + 1 < rb ? fb * k3 * acc[nt][3] : 0.f);
+      } else {
+        uint32_t h, l;
+        split2(c <= ra ? fa * k0 * acc[nt][0] : 0.f, c + 1 <= ra ? fa * k1 * acc[nt][1] : 0.f, h, l);
+        *reinterpret_cast<uint32_t*>(ahg + ra * kC + c) = h;
+        *reinterpret_cast<uint32_t*>(alg + ra * kC + c) = l;
+        split2(c <= rb ? fb * k2 * acc[nt][2] : 0.f, c + 1 <= rb ? fb * k3 * acc[nt][3] : 0.f, h, l);
+        *reinterpret_cast<uint32_t*>(ahg + rb * kC + c) = h;
+        *reinterpret_cast<uint32_t*>(alg + rb * kC + c) = l;
+      }
     }
   }
   __syncthreads();
 
-  for (int j = 0; j < G; ++j) {
-    const int hv = hk * G + j;
-    const size_t head = (size_t)b * Hv + hv;
-
-    // V tile of this value head; lands while the gates and the inverse are computed
-    for (int i = tid; i < kC * 16; i += kThreads) {
-      const int r = i >> 4, c16 = i & 15;
-      const bool ok = r < nv;
-      const size_t off = ok ? ((((size_t)b * T + t0 + r) * Hv + hv) * kD + c16 * 8) : 0;
-      cp16(Vt + r * LDT + c16 * 8, v + off, ok ? 16 : 0);
+  // 4. X = (I + L)^-1: the four 16 x 16 diagonal blocks by forward substitution
+  //    (thread = one column of one block), zeros above the diagonal blocks
+  if (tid < kC) {
+    const int base = 16 * (tid >> 4), cc = tid & 15;
+    float x[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float s = 0.f;
+#pragma unroll
+      for (int jj = 0; jj < r; ++jj) s = fmaf(Lm[(base + r) * LDX + base + jj], x[jj], s);
+      x[r] = r == cc ? 1.f : -s;  // rows above cc come out as zero
     }
-    cp_commit();
-
-    // 4. gates (zero past the end of the sequence) and in-chunk prefix sums
-    if (tid < kC) {
-      float g = 0.f, be = 0.f;
-      if (tid < nv) {
-        const size_t idx = ((size_t)b * T + t0 + tid) * Hv + hv;
-        if (PRE) {
-          g = reinterpret_cast<const float*>(ga)[idx];
-          be = reinterpret_cast<const float*>(gb)[idx];
-        } else {
-          g = gdn_log_decay(__bfloat162float(reinterpret_cast<const bf16*>(ga)[idx]), A_log[hv],
-                            dt_bias[hv]);
-          be = sigmoid_f(__bfloat162float(reinterpret_cast<const bf16*>(gb)[idx]));
-        }
-      }
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, g, off);
-        if (lane >= off) g += y;
-      }
-      if (tid == 31) misc[0] = g;
-      Gs[tid] = g;
-      bet[tid] = be;
+    for (int r = 0; r < 16; ++r) Xm[(base + r) * LDX + base + cc] = x[r];
+  } else {
+    for (int i = tid - kC; i < 6 * 256; i += kThreads - kC) {
+      const int blk = i >> 8, e = i & 255;  // blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+      const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+      const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+      Xm[(16 * bi + (e >> 4)) * LDX + 16 * bj + (e & 15)] = 0.f;
     }
-    __syncthreads();
-    if (tid >= 32 && tid < kC) Gs[tid] += misc[0];
-    __syncthreads();
-
-    // 5. L (strictly lower) and A_qk (lower with diagonal, stored to the workspace)
-    {
-      const int r = tid >> 2, cb = (tid & 3) * 16;
-      const float Gr = Gs[r], br = bet[r] * rk[r], sr = sq[r];
-      float aq[16], al[16];
-#pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        const int c = cb + cc;
-        const float e = __expf(fminf(Gr - Gs[c], 0.f));
-        Lm[r * LDF + c] = c < r ? br * rk[c] * KK[r * LDF + c] * e : 0.f;
-        aq[cc] = c <= r ? sr * rk[c] * QK[r * LDF + c] * e : 0.f;
-        al[cc] = aq[cc] - __bfloat162float(__float2bfloat16_rn(aq[cc]));
-      }
-      const size_t ro = (head * Tp + t0 + r) * kC + cb;
-      st16_bf16(reinterpret_cast<bf16*>(ws + L.ah) + ro, aq);
-      st16_bf16(reinterpret_cast<bf16*>(ws + L.al) + ro, al);
-    }
-    __syncthreads();
-
-    // 6. X = (I + L)^-1: the four 16 x 16 diagonal blocks by forward substitution
-    //    (thread = one column of one block), zeros above the diagonal blocks
-    if (tid < kC) {
-      const int base = 16 * (tid >> 4), cc = tid & 15;
-      float x[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        float s = 0.f;
-#pragma unroll
-        for (int jj = 0; jj < r; ++jj) s = fmaf(Lm[(base + r) * LDF + base + jj], x[jj], s);
-        x[r] = r == cc ? 1.f : -s;  // rows above cc come out as zero
-      }
-#pragma unroll
-      for (int r = 0; r < 16; ++r) Xm[(base + r) * LDF + base + cc] = x[r];
-    } else {
-      for (int i = tid - kC; i < 6 * 256; i += kThreads - kC) {
-        const int blk = i >> 8, e = i & 255;  // blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
-        const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-        const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-        Xm[(16 * bi + (e >> 4)) * LDF + 16 * bj + (e & 15)] = 0.f;
-      }
-    }
-    __syncthreads();
-    //    then block row by block row: X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj
-    for (int bi = 1; bi < 4; ++bi) {
-      for (int e = tid; e < bi * 256; e += kThreads) {
-        const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-        float s = 0.f;
-        for (int kb = bj; kb < bi; ++kb) {
-#pragma unroll
-          for (int qq = 0; qq < 16; ++qq)
-            s = fmaf(Lm[(16 * bi + rr) * LDF + 16 * kb + qq], Xm[(16 * kb + qq) * LDF + 16 * bj + cc],
-                     s);
-        }
-        Tm[(bj * 16 + rr) * 17 + cc] = s;
-      }
-      __syncthreads();
-      for (int e = tid; e < bi * 256; e += kThreads) {
-        const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-        float s = 0.f;
+  }
+  __syncthreads();
+  //    then block row by block row: X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj
+  for (int bi = 1; bi < 4; ++bi) {
+    for (int e = tid; e < bi * 256; e += kThreads) {
+      const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+      float s = 0.f;
+      for (int kb = bj; kb < bi; ++kb) {
 #pragma unroll
         for (int qq = 0; qq < 16; ++qq)
-          s = fmaf(Xm[(16 * bi + rr) * LDF + 16 * bi + qq], Tm[(bj * 16 + qq) * 17 + cc], s);
-        Xm[(16 * bi + rr) * LDF + 16 * bj + cc] = -s;
+          s = fmaf(Lm[(16 * bi + rr) * LDX + 16 * kb + qq], Xm[(16 * kb + qq) * LDX + 16 * bj + cc],
+                   s);
       }
-      __syncthreads();
+      Tm[(bj * 16 + rr) * 17 + cc] = s;
     }
-
-    // 7. A1 = X diag(beta gamma rk) in bf16, A2 = X diag(beta) as bf16 hi + lo
-    {
-      const int r = tid >> 2, cb = (tid & 3) * 16;
-      float a1[16], a2[16], a2l[16];
-#pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        const int c = cb + cc;
-        const float x = Xm[r * LDF + c] * bet[c];
-        a2[cc] = x;
-        a2l[cc] = x - __bfloat162float(__float2bfloat16_rn(x));
-        a1[cc] = x * __expf(Gs[c]) * rk[c];
-      }
-      st16_bf16(A1 + r * LDH + cb, a1);
-      st16_bf16(A2 + r * LDH + cb, a2);
-      st16_bf16(A2l + r * LDH + cb, a2l);
-    }
-    cp_wait<0>();
     __syncthreads();
+    for (int e = tid; e < bi * 256; e += kThreads) {
+      const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+      float s = 0.f;
+#pragma unroll
+      for (int qq = 0; qq < 16; ++qq)
+        s = fmaf(Xm[(16 * bi + rr) * LDX + 16 * bi + qq], Tm[(bj * 16 + qq) * 17 + cc], s);
+      Xm[(16 * bi + rr) * LDX + 16 * bj + cc] = -s;
+    }
+    __syncthreads();
+  }
 
-    // 8. W = A1 K (bf16, staged for coalesced stores) and U = (A2 + A2lo) V (fp32);
-    //    warp -> rows 16 (warp % 4), cols 64 (warp / 4)
-    {
-      const int mt = warp & 3, nb = 64 * (warp >> 2);
-      float acc[8][4] = {};
+  // 5. W = X diag(c1) K (bf16) and U = X diag(beta) V (fp32, X diag(beta) as bf16
+  //    hi + lo); the A fragments are formed from X in registers.
+  //    warp -> rows 16 (warp % 4), cols 64 (warp / 4)
+  const int mt = warp & 3, nb = 64 * (warp >> 2);
+  const int ra = 16 * mt + g8;
+#pragma unroll 1
+  for (int which = 0; which < 2; ++which) {
+    float acc[8][4] = {};
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        uint32_t a[4];
-        ldsm_x4(a, A1 + (16 * mt + lrow_a(lane)) * LDH + 16 * ks + lcol_a(lane));
+    for (int ks = 0; ks < 4; ++ks) {
+      const int ca = 16 * ks + 2 * t4;
+      const float2 x00 = *reinterpret_cast<const float2*>(Xm + ra * LDX + ca);
+      const float2 x10 = *reinterpret_cast<const float2*>(Xm + (ra + 8) * LDX + ca);
+      const float2 x01 = *reinterpret_cast<const float2*>(Xm + ra * LDX + ca + 8);
+      const float2 x11 = *reinterpret_cast<const float2*>(Xm + (ra + 8) * LDX + ca + 8);
+      const float* f = which ? bet : c1;
+      const float f0 = f[ca], f1 = f[ca + 1], f2 = f[ca + 8], f3 = f[ca + 9];
+      uint32_t ah[4], al[4];
+      split2(x00.x * f0, x00.y * f1, ah[0], al[0]);
+      split2(x10.x * f0, x10.y * f1, ah[1], al[1]);
+      split2(x01.x * f2, x01.y * f3, ah[2], al[2]);
+      split2(x11.x * f2, x11.y * f3, ah[3], al[3]);
+      const bf16* Bm = which ? Vt : Kt;
 #pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t bb[4];
-          ldsm_x4_t(bb, Kt + (16 * ks + lrow_a(lane)) * LDT + nb + 16 * np + lcol_a(lane));
-          mma_bf16(acc[2 * np], a, bb[0], bb[1]);
-          mma_bf16(acc[2 * np + 1], a, bb[2], bb[3]);
-        }
-      }
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const int r0 = 16 * mt + g8, c = nb + 8 * nt + 2 * t4;
-        *reinterpret_cast<uint32_t*>(St + r0 * LDT + c) = pack2(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<uint32_t*>(St + (r0 + 8) * LDT + c) = pack2(acc[nt][2], acc[nt][3]);
-      }
-      __syncthreads();
-      bf16* dst = reinterpret_cast<bf16*>(ws + L.w) + (head * Tp + t0) * kD;
-      for (int i = tid; i < kC * 16; i += kThreads) {
-        const int r = i >> 4, c16 = i & 15;
-        *reinterpret_cast<uint4*>(dst + (size_t)r * kD + c16 * 8) =
-            *reinterpret_cast<const uint4*>(St + r * LDT + c16 * 8);
-      }
-
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        uint32_t ah[4], al[4];
-        ldsm_x4(ah, A2 + (16 * mt + lrow_a(lane)) * LDH + 16 * ks + lcol_a(lane));
-        ldsm_x4(al, A2l + (16 * mt + lrow_a(lane)) * LDH + 16 * ks + lcol_a(lane));
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t bb[4];
-          ldsm_x4_t(bb, Vt + (16 * ks + lrow_a(lane)) * LDT + nb + 16 * np + lcol_a(lane));
-          mma_bf16(acc[2 * np], ah, bb[0], bb[1]);
-          mma_bf16(acc[2 * np + 1], ah, bb[2], bb[3]);
+      for (int np = 0; np < 4; ++np) {
+        uint32_t bb[4];
+        ldsm_x4_t(bb, Bm + (16 * ks + lrow_a(lane)) * LDT + nb + 16 * np + lcol_a(lane));
+        mma_bf16(acc[2 * np], ah, bb[0], bb[1]);
+        mma_bf16(acc[2 * np + 1], ah, bb[2], bb[3]);
+        if (which) {
           mma_bf16(acc[2 * np], al, bb[0], bb[1]);
           mma_bf16(acc[2 * np + 1], al, bb[2], bb[3]);
         }
       }
+    }
+    if (which == 0) {
+      bf16* dw = reinterpret_cast<bf16*>(ws + L.w) + (head * Tp + t0) * kD;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const int c = nb + 8 * nt + 2 * t4;
+        *reinterpret_cast<uint32_t*>(dw + (size_t)ra * kD + c) = pack2(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<uint32_t*>(dw + (size_t)(ra + 8) * kD + c) = pack2(acc[nt][2], acc[nt][3]);
+      }
+    } else {
       float* du = reinterpret_cast<float*>(ws + L.u) + (head * Tp + t0) * kD;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
-        const int r0 = 16 * mt + g8, c = nb + 8 * nt + 2 * t4;
-        *reinterpret_cast<float2*>(du + (size_t)r0 * kD + c) = make_float2(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<float2*>(du + (size_t)(r0 + 8) * kD + c) =
+        const int c = nb + 8 * nt + 2 * t4;
+        *reinterpret_cast<float2*>(du + (size_t)ra * kD + c) = make_float2(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<float2*>(du + (size_t)(ra + 8) * kD + c) =
             make_float2(acc[nt][2], acc[nt][3]);
       }
     }
+  }
 
-    // 9. per-row factors of the scan: fo = gamma sq, fs = rk gamma_C / gamma, gamma_C
-    if (tid < kC) {
-      float* sc = reinterpret_cast<float*>(ws + L.scal) + (head * Nc + n) * kScal;
-      const float GC = Gs[kC - 1];
-      sc[tid] = __expf(Gs[tid]) * sq[tid];
-      sc[kC + tid] = tid < nv ? rk[tid] * __expf(GC - Gs[tid]) : 0.f;
-      if (tid < 4) sc[2 * kC + tid] = tid == 0 ? __expf(GC) : 0.f;
-    }
-    __syncthreads();
+  // 6. per-row factors of the scan: fo = gamma sq, fs = rk gamma_C / gamma, gamma_C
+  if (tid < kC) {
+    float* sc = reinterpret_cast<float*>(ws + L.scal) + (head * Nc + n) * kScal;
+    const float GC = Gs[kC - 1];
+    sc[tid] = __expf(Gs[tid]) * sq[tid];
+    sc[kC + tid] = tid < nv ? rk[tid] * __expf(GC - Gs[tid]) : 0.f;
+    if (tid < 4) sc[2 * kC + tid] = tid == 0 ? __expf(GC) : 0.f;
   }
 }
 
@@ -649,7 +604,7 @@ cudaError_t launch_t(const ChunkArgs& a, uint8_t* ws, const WsLayout& L, cudaStr
   if (e != cudaSuccess) return e;
   const bf16* q = static_cast<const bf16*>(a.q);
   const bf16* k = static_cast<const bf16*>(a.k);
-  prep<<<dim3(Nc, a.B * a.Hk), kThreads, P_BYTES, s>>>(
+  prep<<<dim3(a.Hv / a.Hk, Nc, a.B * a.Hk), kThreads, P_BYTES, s>>>(
       q, k, static_cast<const bf16*>(a.v), a.a, a.b, a.A_log, a.dt_bias, a.T, a.Hk, a.Hv,
       a.scale, (a.flags & GDN_QK_L2NORM) ? 1 : 0, ws, L);
   e = cudaGetLastError();
@@ -663,7 +618,7 @@ cudaError_t launch_t(const ChunkArgs& a, uint8_t* ws, const WsLayout& L, cudaStr
 
 bool chunk_mma_supported(const ChunkArgs& a) {
   return a.dtype == GDN_BF16 && a.dk == kD && a.dv == kD && (long)a.B * a.Hv <= 65535 &&
-         (long)a.B * a.Hk <= 65535;
+         (long)a.B * a.Hk <= 65535 && ((long)a.T + kC - 1) / kC <= 65535;
 }
 
 size_t chunk_mma_workspace_bytes(int B, int T, int Hv) {
