@@ -35,7 +35,8 @@ lib = ctypes.CDLL(LIB_PATH)
 F32, BF16 = 0, 1
 QK_L2NORM, GATES_PRECOMPUTED, OUT_F32 = 1, 2, 4
 _STATUS = {0: "GDN_OK", -1: "GDN_ERR_INVALID_ARG", -2: "GDN_ERR_UNSUPPORTED",
-           -3: "GDN_ERR_CUDA", -4: "GDN_ERR_TIMEOUT", -5: "GDN_ERR_WORKSPACE"}
+           -3: "GDN_ERR_CUDA", -4: "GDN_ERR_TIMEOUT", -5: "GDN_ERR_WORKSPACE",
+           -6: "GDN_ERR_RANGE"}
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 lib.gdn_gate_prep.argtypes = [_vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f,

@@ -68,6 +68,7 @@ const char* gdn_status_string(int status) {
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
     case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
     case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+    case GDN_ERR_RANGE: return "GDN_ERR_RANGE";
     default: return "GDN_ERR_UNKNOWN";
   }
 }
@@ -92,7 +93,7 @@ size_t gdn_chunk_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, i
   if (B <= 0 || T <= 0 || Hk <= 0 || Hv <= 0 || Hv % Hk != 0) return 0;
   ChunkArgs c{};
   c.B = B; c.T = T; c.Hk = Hk; c.Hv = Hv; c.dk = dk; c.dv = dv; c.dtype = dtype;
-  return chunk_mma_supported(c) ? chunk_mma_workspace_bytes(B, T, Hv) : 0;
+  return chunk_mma_supported(c) ? chunk_mma_workspace_bytes(B, T, Hk, Hv) : 0;
 }
 size_t gdn2_chunk_workspace_bytes(int, int, int, int, int, int) { return 0; }
 
@@ -120,7 +121,7 @@ static int run_chunk(const ChunkArgs& c, bool gdn2, void* ws, size_t ws_bytes,
   if (c.T == 0 || c.B == 0) return from_cuda(launch_copy_state(c.h0, c.ht, state_elems, s));
   if (!gdn2 && chunk_mma_supported(c)) {
     if (ws == nullptr || !aligned16(ws) ||
-        ws_bytes < chunk_mma_workspace_bytes(c.B, c.T, c.Hv))
+        ws_bytes < chunk_mma_workspace_bytes(c.B, c.T, c.Hk, c.Hv))
       return GDN_ERR_WORKSPACE;
     return from_cuda(launch_chunk_mma(c, ws, s));
   }
@@ -176,7 +177,7 @@ int gdn_check_status(gdn_stream_t stream) {
   if (h != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_gdn_status, &zero, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
-    return GDN_ERR_TIMEOUT;
+    return (h & kStatusRange) ? GDN_ERR_RANGE : GDN_ERR_TIMEOUT;
   }
   return GDN_OK;
 }

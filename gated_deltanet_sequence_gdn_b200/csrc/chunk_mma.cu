@@ -9,24 +9,33 @@
 //      L = diag(beta) (K^ K^^T o Gamma), X = (I + L)^-1 by blocked forward
 //      substitution in fp32, W = X diag(beta gamma) K^, U = X diag(beta) V and
 //      A_qk = tril(Q^ K^^T o Gamma) (diagonal included), written to the
-//      workspace with the per-row factors of the second kernel.
+//      workspace with the per-row factors of the second kernel, together with
+//      fp16 copies of the raw Q and K tiles.
 //  state_scan_kernel : one CTA per (value head, 64-column half of d_v),
 //      sequential over the chunks with the fp32 state slice held in mma
 //      accumulator registers:  U~ = U - W S,  o = diag(gamma sq) Q S + A_qk U~,
 //      S <- gamma_C S + K^T diag(rk gamma_C / gamma) U~.  The next chunk's tiles
 //      are fetched with cp.async while the current one is computed.
 //
-// Precision: bf16 operands, fp32 accumulation and state.  Where one bf16
-// rounding of an operand would cost more than the 2e-2 (max |err| / RMS)
-// budget, the operand is carried as an unevaluated sum hi + lo of two bf16
-// numbers (hi = rn(x), lo = rn(x - hi), about 16 significant bits) and the
-// product takes one mma per term: X diag(beta) in U, U~ and A_qk in the
-// output, U~ diag(fs) in the state update, and the state in Q S.  U is kept
-// in fp32.  W S uses the state's hi part only.
-//
 // The algebra is the WY / UT chunk form of the delta rule ("Gated DeltaNet-2",
 // section on the chunkwise algorithm; GDN is its scalar-decay special case):
 // Gamma_rj = exp(G_r - G_j) only for j <= r, so every exponent is <= 0.
+//
+// Precision: fp32 accumulation and state.  The prep's products take bf16
+// operands (the inputs are bf16; X diag(beta) is carried as bf16 hi + lo, one
+// mma per part, and U is stored in fp32).  The scan's products take fp16
+// operands (11 significant bits): W, A_qk, the state, U~ and U~ diag(fs), and
+// the raw Q / K rows.  fp16 has a narrow range, so every fp16 operand is kept in
+// range by an exact power-of-2 scale folded into a factor applied in fp32:
+//   - each raw Q / K row r is stored as q_r 2^-e_r with its largest entry in
+//     [1, 2); 2^e_r is folded into fo_r / fs_r;
+//   - the scan multiplies U, the state and the output of one CTA by one
+//     sigma = 2^-e chosen from the largest |U| of its head and |h0| of its
+//     slice, so that both are below 2^8 (the delta rule keeps |S| of the
+//     order of |v|); the output and the final state are divided by sigma;
+//   - W and A_qk are bounded by construction for unit-norm keys.
+// A value that still leaves the fp16 range sets the range bit of the status
+// word (read by gdn_check_status); nothing is clamped silently.
 #include "common.cuh"
 #include "launch.h"
 #include "warp_mma.cuh"
@@ -40,24 +49,26 @@ using bf16 = __nv_bfloat16;
 constexpr int kC = 64;         // chunk length
 constexpr int kD = 128;        // dk = dv
 constexpr int kThreads = 256;  // 8 warps
-constexpr int LDT = kD + 8;    // bf16 row stride of 128-wide tiles (272 B: ldmatrix conflict-free)
-constexpr int LDH = 64 + 8;    // bf16 row stride of 64-wide tiles (144 B)
-constexpr int LDF = 65;        // fp32 row stride of 64 x 64 matrices
-constexpr int kScal = 132;     // floats per (head, chunk): fo[64], fs[64], gamma_C, pad
+constexpr int LDT = kD + 8;    // 16-bit row stride of 128-wide tiles (272 B: ldmatrix conflict-free)
+constexpr int LDH = 64 + 8;    // 16-bit row stride of 64-wide tiles (144 B)
+constexpr int kScal = 132;     // floats per (head, chunk): fo[64], fs[64], gamma_C, max|U|, pad
+constexpr float kF16Max = 65000.f;  // largest magnitude accepted for an fp16 operand
 
 // ---------------------------------------------------------------- workspace
 struct WsLayout {
-  size_t w, u, ah, al, scal, total;
+  size_t w, u, a, qh, kh, scal, total;
 };
-WsLayout ws_layout(int B, int T, int Hv) {
-  const size_t Nc = ((size_t)T + kC - 1) / kC, Tp = Nc * kC, heads = (size_t)B * Hv;
+WsLayout ws_layout(int B, int T, int Hk, int Hv) {
+  const size_t Nc = ((size_t)T + kC - 1) / kC, Tp = Nc * kC;
+  const size_t hv = (size_t)B * Hv, hk = (size_t)B * Hk;
   WsLayout L;
-  L.w = 0;                                  // W        [B*Hv][Tp][128] bf16
-  L.u = L.w + heads * Tp * kD * 2;          // U        [B*Hv][Tp][128] f32
-  L.ah = L.u + heads * Tp * kD * 4;         // A_qk hi  [B*Hv][Tp][64]  bf16
-  L.al = L.ah + heads * Tp * kC * 2;        // A_qk lo  [B*Hv][Tp][64]  bf16
-  L.scal = L.al + heads * Tp * kC * 2;      // scalars  [B*Hv][Nc][132] f32
-  L.total = L.scal + heads * Nc * kScal * 4;
+  L.w = 0;                                  // W      [B*Hv][Tp][128] f16
+  L.u = L.w + hv * Tp * kD * 2;             // U      [B*Hv][Tp][128] f32
+  L.a = L.u + hv * Tp * kD * 4;             // A_qk   [B*Hv][Tp][64]  f16
+  L.qh = L.a + hv * Tp * kC * 2;            // Q rows [B*Hk][Tp][128] f16 (row-scaled)
+  L.kh = L.qh + hk * Tp * kD * 2;           // K rows [B*Hk][Tp][128] f16 (row-scaled)
+  L.scal = L.kh + hk * Tp * kD * 2;         // scalars [B*Hv][Nc][132] f32
+  L.total = L.scal + hv * Nc * kScal * 4;
   return L;
 }
 
@@ -68,6 +79,9 @@ __device__ __forceinline__ void split2(float x, float y, uint32_t& hi, uint32_t&
   lo = pack2(x - h.x, y - h.y);
 }
 
+// Exponent e with (max |row|) * 2^-e in [1, 2) (e = 0 for a zero row).
+__device__ __forceinline__ int row_exponent(float m) { return m > 0.f ? ilogbf(m) : 0; }
+
 // ---------------------------------------------------------------- prep kernel
 constexpr int LDX = 64 + 8;                  // f32 row stride of L and X (conflict-free float2)
 constexpr int P_KT = 0;                      // K tile  [64][LDT] bf16 (key head)
@@ -76,8 +90,8 @@ constexpr int P_VT = P_QT + kC * LDT * 2;    // V tile  (value head)
 constexpr int P_L = P_VT + kC * LDT * 2;     // L [64][LDX] f32
 constexpr int P_X = P_L + kC * LDX * 4;      // X = (I + L)^-1
 constexpr int P_T = P_X + kC * LDX * 4;      // block products [3][16][17] f32
-constexpr int P_VEC = P_T + 3 * 16 * 17 * 4; // rk, sq, G, beta, c1 [64] + misc
-constexpr int P_BYTES = P_VEC + 6 * 64 * 4;
+constexpr int P_VEC = P_T + 3 * 16 * 17 * 4; // rk, sq, G, beta, c1, 2^eq, 2^ek [64], misc
+constexpr int P_BYTES = P_VEC + 8 * 64 * 4;
 static_assert(2 * (P_BYTES + 1024) <= 228 * 1024, "two prep CTAs per SM");
 
 template <bool PRE>
@@ -85,7 +99,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                const void* __restrict__ ga, const void* __restrict__ gb,
                const float* __restrict__ A_log, const float* __restrict__ dt_bias, int T, int Hk,
-               int Hv, float scale, int l2, uint8_t* __restrict__ ws, WsLayout L) {
+               int Hv, float scale, int l2, uint8_t* __restrict__ ws, WsLayout L, int* status) {
   extern __shared__ __align__(16) uint8_t sm[];
   bf16* Kt = reinterpret_cast<bf16*>(sm + P_KT);
   bf16* Qt = reinterpret_cast<bf16*>(sm + P_QT);
@@ -98,7 +112,9 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
   float* Gs = sq + 64;
   float* bet = Gs + 64;
   float* c1 = bet + 64;
-  float* misc = c1 + 64;
+  float* pq = c1 + 64;   // 2^e of the stored Q row
+  float* pk = pq + 64;   // 2^e of the stored K row
+  float* misc = pk + 64; // [0] prefix carry, [8..15] per-warp max |U|
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
@@ -107,6 +123,7 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
   const int b = blockIdx.z / Hk, hk = blockIdx.z % Hk, hv = hk * G + blockIdx.x;
   const size_t head = (size_t)b * Hv + hv;
   const int t0 = n * kC, nv = min(kC, T - t0);
+  float range = 0.f;  // largest magnitude this thread converted to fp16
 
   // 1. raw K, Q tiles of the key head and the V tile of this value head (rows
   //    past the end of the sequence are zeros)
@@ -150,23 +167,49 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
   __syncthreads();
   if (tid >= 32 && tid < kC) Gs[tid] += misc[0];
 
-  //    L2 norms: rk = 1 / |k|, sq = scale / |q| (two threads per row)
+  //    L2 norms: rk = 1 / |k|, sq = scale / |q|, and the row exponents of the
+  //    fp16 copies (two threads per row)
   {
     const int which = tid >> 7, r = (tid & 127) >> 1, h = tid & 1;
     const bf16* row = (which ? Qt : Kt) + r * LDT + h * 64;
-    float ss = 0.f;
+    float ss = 0.f, mx = 0.f;
 #pragma unroll
     for (int c = 0; c < 64; c += 8) {
       const uint4 u = *reinterpret_cast<const uint4*>(row + c);
       const float2 f0 = unpack2(u.x), f1 = unpack2(u.y), f2 = unpack2(u.z), f3 = unpack2(u.w);
       ss += f0.x * f0.x + f0.y * f0.y + f1.x * f1.x + f1.y * f1.y + f2.x * f2.x + f2.y * f2.y +
             f3.x * f3.x + f3.y * f3.y;
+      mx = fmaxf(mx, fmaxf(fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y))),
+                           fmaxf(fmaxf(fabsf(f2.x), fabsf(f2.y)), fmaxf(fabsf(f3.x), fabsf(f3.y)))));
     }
     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    const int e = row_exponent(mx);
     if (h == 0) {
       const float inv = l2 ? rsqrtf(ss + 1e-6f) : 1.f;
-      if (which) sq[r] = inv * scale;
-      else rk[r] = inv;
+      if (which) {
+        sq[r] = inv * scale;
+        pq[r] = ldexpf(1.f, e);
+      } else {
+        rk[r] = inv;
+        pk[r] = ldexpf(1.f, e);
+      }
+    }
+    // fp16 copies of the raw rows, row-scaled by 2^-e (written once per key head)
+    if (blockIdx.x == 0) {
+      __half* dst = reinterpret_cast<__half*>(ws + (which ? L.qh : L.kh)) +
+                    ((size_t)blockIdx.z * Tp + t0 + r) * kD + h * 64;
+#pragma unroll
+      for (int c = 0; c < 64; c += 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(row + c);
+        const float2 f0 = unpack2(u.x), f1 = unpack2(u.y), f2 = unpack2(u.z), f3 = unpack2(u.w);
+        uint4 o;
+        o.x = pack2h(ldexpf(f0.x, -e), ldexpf(f0.y, -e));
+        o.y = pack2h(ldexpf(f1.x, -e), ldexpf(f1.y, -e));
+        o.z = pack2h(ldexpf(f2.x, -e), ldexpf(f2.y, -e));
+        o.w = pack2h(ldexpf(f3.x, -e), ldexpf(f3.y, -e));
+        *reinterpret_cast<uint4*>(dst + c) = o;
+      }
     }
   }
   __syncthreads();
@@ -175,7 +218,7 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
   // 3. Gram matrices on the tensor cores with the gates applied in registers:
   //    warps 0-3: L = strictly lower (beta_r rk_r rk_c e^(G_r - G_c) k_r.k_c) -> smem
   //    warps 4-7: A_qk = lower incl. diagonal (sq_r rk_c e^(G_r - G_c) q_r.k_c),
-  //               stored to the workspace as bf16 hi + lo
+  //               stored to the workspace in fp16 (|A_qk| <= scale for unit rows)
   {
     const int mt = warp & 3;
     const bool isq = warp >= 4;
@@ -197,8 +240,7 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
     const float Ga = Gs[ra], Gb = Gs[rb];
     const float fa = isq ? sq[ra] : bet[ra] * rk[ra];
     const float fb = isq ? sq[rb] : bet[rb] * rk[rb];
-    bf16* ahg = reinterpret_cast<bf16*>(ws + L.ah) + (head * Tp + t0) * kC;
-    bf16* alg = reinterpret_cast<bf16*>(ws + L.al) + (head * Tp + t0) * kC;
+    __half* ag = reinterpret_cast<__half*>(ws + L.a) + (head * Tp + t0) * kC;
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
       const int c = 8 * nt + 2 * t4;
@@ -212,13 +254,13 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
         *reinterpret_cast<float2*>(Lm + rb * LDX + c) =
             make_float2(c < rb ? fb * k2 * acc[nt][2] : 0.f, c + 1 < rb ? fb * k3 * acc[nt][3] : 0.f);
       } else {
-        uint32_t h, l;
-        split2(c <= ra ? fa * k0 * acc[nt][0] : 0.f, c + 1 <= ra ? fa * k1 * acc[nt][1] : 0.f, h, l);
-        *reinterpret_cast<uint32_t*>(ahg + ra * kC + c) = h;
-        *reinterpret_cast<uint32_t*>(alg + ra * kC + c) = l;
-        split2(c <= rb ? fb * k2 * acc[nt][2] : 0.f, c + 1 <= rb ? fb * k3 * acc[nt][3] : 0.f, h, l);
-        *reinterpret_cast<uint32_t*>(ahg + rb * kC + c) = h;
-        *reinterpret_cast<uint32_t*>(alg + rb * kC + c) = l;
+        const float x0 = c <= ra ? fa * k0 * acc[nt][0] : 0.f;
+        const float x1 = c + 1 <= ra ? fa * k1 * acc[nt][1] : 0.f;
+        const float x2 = c <= rb ? fb * k2 * acc[nt][2] : 0.f;
+        const float x3 = c + 1 <= rb ? fb * k3 * acc[nt][3] : 0.f;
+        range = fmaxf(range, fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3))));
+        *reinterpret_cast<uint32_t*>(ag + ra * kC + c) = pack2h(x0, x1);
+        *reinterpret_cast<uint32_t*>(ag + rb * kC + c) = pack2h(x2, x3);
       }
     }
   }
@@ -272,11 +314,12 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
     __syncthreads();
   }
 
-  // 5. W = X diag(c1) K (bf16) and U = X diag(beta) V (fp32, X diag(beta) as bf16
-  //    hi + lo); the A fragments are formed from X in registers.
+  // 5. W = X diag(c1) K (stored in fp16) and U = X diag(beta) V (fp32, X diag(beta)
+  //    as bf16 hi + lo); the A fragments are formed from X in registers.
   //    warp -> rows 16 (warp % 4), cols 64 (warp / 4)
   const int mt = warp & 3, nb = 64 * (warp >> 2);
   const int ra = 16 * mt + g8;
+  float umax = 0.f;
 #pragma unroll 1
   for (int which = 0; which < 2; ++which) {
     float acc[8][4] = {};
@@ -308,55 +351,68 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
       }
     }
     if (which == 0) {
-      bf16* dw = reinterpret_cast<bf16*>(ws + L.w) + (head * Tp + t0) * kD;
+      __half* dw = reinterpret_cast<__half*>(ws + L.w) + (head * Tp + t0) * kD;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         const int c = nb + 8 * nt + 2 * t4;
-        *reinterpret_cast<uint32_t*>(dw + (size_t)ra * kD + c) = pack2(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<uint32_t*>(dw + (size_t)(ra + 8) * kD + c) = pack2(acc[nt][2], acc[nt][3]);
+        range = fmaxf(range, fmaxf(fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][1])),
+                                   fmaxf(fabsf(acc[nt][2]), fabsf(acc[nt][3]))));
+        *reinterpret_cast<uint32_t*>(dw + (size_t)ra * kD + c) = pack2h(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<uint32_t*>(dw + (size_t)(ra + 8) * kD + c) =
+            pack2h(acc[nt][2], acc[nt][3]);
       }
     } else {
       float* du = reinterpret_cast<float*>(ws + L.u) + (head * Tp + t0) * kD;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         const int c = nb + 8 * nt + 2 * t4;
+        umax = fmaxf(umax, fmaxf(fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][1])),
+                                 fmaxf(fabsf(acc[nt][2]), fabsf(acc[nt][3]))));
         *reinterpret_cast<float2*>(du + (size_t)ra * kD + c) = make_float2(acc[nt][0], acc[nt][1]);
         *reinterpret_cast<float2*>(du + (size_t)(ra + 8) * kD + c) =
             make_float2(acc[nt][2], acc[nt][3]);
       }
     }
   }
+  if (!(range <= kF16Max)) report_range(status);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) umax = fmaxf(umax, __shfl_xor_sync(0xffffffffu, umax, o));
+  if (lane == 0) misc[8 + warp] = umax;
+  __syncthreads();
 
-  // 6. per-row factors of the scan: fo = gamma sq, fs = rk gamma_C / gamma, gamma_C
+  // 6. per-row factors of the scan: fo = gamma sq 2^eq, fs = rk 2^ek gamma_C / gamma,
+  //    gamma_C, and the largest |U| of the chunk
   if (tid < kC) {
     float* sc = reinterpret_cast<float*>(ws + L.scal) + (head * Nc + n) * kScal;
     const float GC = Gs[kC - 1];
-    sc[tid] = __expf(Gs[tid]) * sq[tid];
-    sc[kC + tid] = tid < nv ? rk[tid] * __expf(GC - Gs[tid]) : 0.f;
-    if (tid < 4) sc[2 * kC + tid] = tid == 0 ? __expf(GC) : 0.f;
+    sc[tid] = __expf(Gs[tid]) * sq[tid] * pq[tid];
+    sc[kC + tid] = tid < nv ? rk[tid] * pk[tid] * __expf(GC - Gs[tid]) : 0.f;
+    if (tid < 4) {
+      float m = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) m = fmaxf(m, misc[8 + w]);
+      sc[2 * kC + tid] = tid == 0 ? __expf(GC) : (tid == 1 ? m : 0.f);
+    }
   }
 }
 
 // ---------------------------------------------------------------- scan kernel
 constexpr int LDU = 64 + 8;                 // f32 row stride of the U tile (conflict-free float2)
 // double-buffered, fetched one chunk ahead
-constexpr int S_W = 0;                      // W tile   [64][LDT] bf16
-constexpr int S_Q = S_W + kC * LDT * 2;     // raw Q tile
+constexpr int S_W = 0;                      // W tile     [64][LDT] f16
+constexpr int S_Q = S_W + kC * LDT * 2;     // Q rows     [64][LDT] f16
 constexpr int S_U = S_Q + kC * LDT * 2;     // U columns of this CTA [64][LDU] f32
 constexpr int S_SC = S_U + kC * LDU * 4;    // scalars (132 f32)
 constexpr int STAGE = S_SC + kScal * 4;
 // single-buffered, fetched at the start of the chunk that uses them
-constexpr int S_K = 2 * STAGE;              // raw K tile [64][LDT] bf16
-constexpr int S_AH = S_K + kC * LDT * 2;    // A_qk hi [64][LDH] bf16
-constexpr int S_AL = S_AH + kC * LDH * 2;   // A_qk lo
+constexpr int S_K = 2 * STAGE;              // K rows [64][LDT] f16
+constexpr int S_A = S_K + kC * LDT * 2;     // A_qk   [64][LDH] f16
 // on-chip operands
-constexpr int S_SBH = S_AL + kC * LDH * 2;  // state slice, bf16 hi [128][LDH]
-constexpr int S_SBL = S_SBH + kD * LDH * 2; // state slice, bf16 lo
-constexpr int S_UTH = S_SBL + kD * LDH * 2; // U~ hi [64][LDH]
-constexpr int S_UTL = S_UTH + kC * LDH * 2; // U~ lo
-constexpr int S_USH = S_UTL + kC * LDH * 2; // U~ diag(fs) hi
-constexpr int S_USL = S_USH + kC * LDH * 2; // U~ diag(fs) lo
-constexpr int S_BYTES = S_USL + kC * LDH * 2;
+constexpr int S_SB = S_A + kC * LDH * 2;    // state slice (scaled) [128][LDH] f16
+constexpr int S_UT = S_SB + kD * LDH * 2;   // U~ (scaled)          [64][LDH] f16
+constexpr int S_US = S_UT + kC * LDH * 2;   // U~ diag(fs)          [64][LDH] f16
+constexpr int S_RED = S_US + kC * LDH * 2;  // 8 floats for the CTA max
+constexpr int S_BYTES = S_RED + 64;
 static_assert(STAGE % 16 == 0, "stage buffers must stay 16-byte aligned");
 static_assert(S_BYTES <= 227 * 1024, "shared memory of the scan kernel");
 
@@ -373,77 +429,57 @@ __device__ __forceinline__ void store2<bf16>(bf16* p, float x, float y) {
 
 template <typename TO>
 __global__ void __launch_bounds__(kThreads, 1)
-state_scan_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
-                  const uint8_t* __restrict__ ws, WsLayout L, const float* h0, int T, int Hk,
-                  int Hv, TO* __restrict__ o, float* ht) {
+state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, int T, int Hk,
+                  int Hv, TO* __restrict__ o, float* ht, int* status) {
   extern __shared__ __align__(16) uint8_t sm[];
-  bf16* Kt = reinterpret_cast<bf16*>(sm + S_K);
-  bf16* Ah = reinterpret_cast<bf16*>(sm + S_AH);
-  bf16* Al = reinterpret_cast<bf16*>(sm + S_AL);
-  bf16* Sbh = reinterpret_cast<bf16*>(sm + S_SBH);
-  bf16* Sbl = reinterpret_cast<bf16*>(sm + S_SBL);
-  bf16* Uth = reinterpret_cast<bf16*>(sm + S_UTH);
-  bf16* Utl = reinterpret_cast<bf16*>(sm + S_UTL);
-  bf16* Ush = reinterpret_cast<bf16*>(sm + S_USH);
-  bf16* Usl = reinterpret_cast<bf16*>(sm + S_USL);
+  __half* Kt = reinterpret_cast<__half*>(sm + S_K);
+  __half* At = reinterpret_cast<__half*>(sm + S_A);
+  __half* Sb = reinterpret_cast<__half*>(sm + S_SB);
+  __half* Ut = reinterpret_cast<__half*>(sm + S_UT);
+  __half* Us = reinterpret_cast<__half*>(sm + S_US);
+  float* red = reinterpret_cast<float*>(sm + S_RED);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
   const int c0 = 64 * blockIdx.x;
   const int head = blockIdx.y, b = head / Hv, hv = head % Hv, hk = hv / (Hv / Hk);
   const int Nc = (T + kC - 1) / kC, Tp = Nc * kC;
-  const bf16* Wg = reinterpret_cast<const bf16*>(ws + L.w) + (size_t)head * Tp * kD;
+  const size_t khead = (size_t)b * Hk + hk;
+  const __half* Wg = reinterpret_cast<const __half*>(ws + L.w) + (size_t)head * Tp * kD;
   const float* Ug = reinterpret_cast<const float*>(ws + L.u) + (size_t)head * Tp * kD + c0;
-  const bf16* Ahg = reinterpret_cast<const bf16*>(ws + L.ah) + (size_t)head * Tp * kC;
-  const bf16* Alg = reinterpret_cast<const bf16*>(ws + L.al) + (size_t)head * Tp * kC;
+  const __half* Ag = reinterpret_cast<const __half*>(ws + L.a) + (size_t)head * Tp * kC;
+  const __half* Qg = reinterpret_cast<const __half*>(ws + L.qh) + khead * Tp * kD;
+  const __half* Kg = reinterpret_cast<const __half*>(ws + L.kh) + khead * Tp * kD;
   const float* Sg = reinterpret_cast<const float*>(ws + L.scal) + (size_t)head * Nc * kScal;
 
   // W, Q, U and the scalars of chunk n into stage n % 2
   auto issue_stage = [&](int n) {
     uint8_t* st = sm + (n & 1) * STAGE;
-    const int t0 = n * kC, nv = min(kC, T - t0);
+    const size_t r0 = (size_t)n * kC;
     for (int i = tid; i < kC * 16; i += kThreads) {
       const int r = i >> 4, c16 = i & 15;
-      cp16(st + S_W + (r * LDT + c16 * 8) * 2, Wg + (size_t)(t0 + r) * kD + c16 * 8, 16);
-      const bool ok = r < nv;
-      const size_t off = ok ? ((((size_t)b * T + t0 + r) * Hk + hk) * kD + c16 * 8) : 0;
-      cp16(st + S_Q + (r * LDT + c16 * 8) * 2, q + off, ok ? 16 : 0);
-      cp16(st + S_U + (r * LDU + c16 * 4) * 4, Ug + (size_t)(t0 + r) * kD + c16 * 4, 16);
+      cp16(st + S_W + (r * LDT + c16 * 8) * 2, Wg + (r0 + r) * kD + c16 * 8, 16);
+      cp16(st + S_Q + (r * LDT + c16 * 8) * 2, Qg + (r0 + r) * kD + c16 * 8, 16);
+      cp16(st + S_U + (r * LDU + c16 * 4) * 4, Ug + (r0 + r) * kD + c16 * 4, 16);
     }
     if (tid < kScal / 4) cp16(st + S_SC + tid * 16, Sg + (size_t)n * kScal + tid * 4, 16);
     cp_commit();
   };
-  // K and A_qk of chunk n
+  // K rows and A_qk of chunk n
   auto issue_ka = [&](int n) {
-    const int t0 = n * kC, nv = min(kC, T - t0);
+    const size_t r0 = (size_t)n * kC;
     for (int i = tid; i < kC * 16; i += kThreads) {
       const int r = i >> 4, c16 = i & 15;
-      const bool ok = r < nv;
-      const size_t off = ok ? ((((size_t)b * T + t0 + r) * Hk + hk) * kD + c16 * 8) : 0;
-      cp16(Kt + r * LDT + c16 * 8, k + off, ok ? 16 : 0);
-      if (c16 < 8) {
-        cp16(Ah + r * LDH + c16 * 8, Ahg + (size_t)(t0 + r) * kC + c16 * 8, 16);
-        cp16(Al + r * LDH + c16 * 8, Alg + (size_t)(t0 + r) * kC + c16 * 8, 16);
-      }
+      cp16(Kt + r * LDT + c16 * 8, Kg + (r0 + r) * kD + c16 * 8, 16);
+      if (c16 < 8) cp16(At + r * LDH + c16 * 8, Ag + (r0 + r) * kC + c16 * 8, 16);
     }
     cp_commit();
   };
+  issue_stage(0);
 
   // state slice: warp w holds rows 16 w .. 16 w + 15, all 64 columns, as 8 C fragments
   float S[8][4];
   const int s0 = 16 * warp + g8;
-  auto store_state_bf16 = [&]() {
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int c = 8 * nt + 2 * t4;
-      uint32_t h, l;
-      split2(S[nt][0], S[nt][1], h, l);
-      *reinterpret_cast<uint32_t*>(Sbh + s0 * LDH + c) = h;
-      *reinterpret_cast<uint32_t*>(Sbl + s0 * LDH + c) = l;
-      split2(S[nt][2], S[nt][3], h, l);
-      *reinterpret_cast<uint32_t*>(Sbh + (s0 + 8) * LDH + c) = h;
-      *reinterpret_cast<uint32_t*>(Sbl + (s0 + 8) * LDH + c) = l;
-    }
-  };
+  float mx = 0.f;
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt) {
     float2 x0 = make_float2(0.f, 0.f), x1 = x0;
@@ -453,9 +489,36 @@ state_scan_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       x1 = *reinterpret_cast<const float2*>(src + 8 * kD);
     }
     S[nt][0] = x0.x; S[nt][1] = x0.y; S[nt][2] = x1.x; S[nt][3] = x1.y;
+    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x0.x), fabsf(x0.y)), fmaxf(fabsf(x1.x), fabsf(x1.y))));
   }
-  store_state_bf16();
-  issue_stage(0);
+  // sigma = 2^-e: the largest |U| of the head and |h0| of this slice land below 2^8
+  for (int n = tid; n < Nc; n += kThreads) mx = fmaxf(mx, Sg[(size_t)n * kScal + 2 * kC + 1]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  mx = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) mx = fmaxf(mx, red[w]);
+  const int e = mx > 0.f ? min(max(ilogbf(mx) - 7, -100), 100) : 0;
+  const float sigma = ldexpf(1.f, -e), inv_sigma = ldexpf(1.f, e);
+  float range = 0.f;
+
+  auto store_state = [&]() {
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      const int c = 8 * nt + 2 * t4;
+      range = fmaxf(range, fmaxf(fmaxf(fabsf(S[nt][0]), fabsf(S[nt][1])),
+                                 fmaxf(fabsf(S[nt][2]), fabsf(S[nt][3]))));
+      *reinterpret_cast<uint32_t*>(Sb + s0 * LDH + c) = pack2h(S[nt][0], S[nt][1]);
+      *reinterpret_cast<uint32_t*>(Sb + (s0 + 8) * LDH + c) = pack2h(S[nt][2], S[nt][3]);
+    }
+  };
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) S[nt][i] *= sigma;
+  store_state();
 
   const int mt = warp & 3, nb = 32 * (warp >> 2);  // output tile of this warp: 16 rows x 32 cols
   const int r0 = 16 * mt + g8, r1 = r0 + 8;
@@ -466,13 +529,13 @@ state_scan_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     const bool more = n + 1 < Nc;
     if (more) issue_stage(n + 1);
     const uint8_t* st = sm + (n & 1) * STAGE;
-    const bf16* Wt = reinterpret_cast<const bf16*>(st + S_W);
-    const bf16* Qt = reinterpret_cast<const bf16*>(st + S_Q);
+    const __half* Wt = reinterpret_cast<const __half*>(st + S_W);
+    const __half* Qt = reinterpret_cast<const __half*>(st + S_Q);
     const float* Uc = reinterpret_cast<const float*>(st + S_U);
     const float* sc = reinterpret_cast<const float*>(st + S_SC);
     const int t0 = n * kC;
 
-    // P = W S_hi and OQ = Q (S_hi + S_lo) for this warp's tile
+    // P = W S and OQ = Q S for this warp's tile (S scaled by sigma)
     float P[4][4] = {}, OQ[4][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -481,19 +544,15 @@ state_scan_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       ldsm_x4(aq, Qt + (16 * mt + lrow_a(lane)) * LDT + 16 * ks + lcol_a(lane));
 #pragma unroll
       for (int np = 0; np < 2; ++np) {
-        uint32_t bh[4], bl[4];
-        const int so = (16 * ks + lrow_a(lane)) * LDH + nb + 16 * np + lcol_a(lane);
-        ldsm_x4_t(bh, Sbh + so);
-        ldsm_x4_t(bl, Sbl + so);
-        mma_bf16(P[2 * np], aw, bh[0], bh[1]);
-        mma_bf16(P[2 * np + 1], aw, bh[2], bh[3]);
-        mma_bf16(OQ[2 * np], aq, bh[0], bh[1]);
-        mma_bf16(OQ[2 * np + 1], aq, bh[2], bh[3]);
-        mma_bf16(OQ[2 * np], aq, bl[0], bl[1]);
-        mma_bf16(OQ[2 * np + 1], aq, bl[2], bl[3]);
+        uint32_t bb[4];
+        ldsm_x4_t(bb, Sb + (16 * ks + lrow_a(lane)) * LDH + nb + 16 * np + lcol_a(lane));
+        mma_f16(P[2 * np], aw, bb[0], bb[1]);
+        mma_f16(P[2 * np + 1], aw, bb[2], bb[3]);
+        mma_f16(OQ[2 * np], aq, bb[0], bb[1]);
+        mma_f16(OQ[2 * np + 1], aq, bb[2], bb[3]);
       }
     }
-    // U~ = U - P, and U~ diag(fs) for the state update, both as bf16 hi + lo
+    // U~ = sigma U - P, and U~ diag(fs) for the state update, in fp16
     {
       const float fs0 = sc[kC + r0], fs1 = sc[kC + r1];
 #pragma unroll
@@ -501,47 +560,32 @@ state_scan_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
         const int c = nb + 8 * nt + 2 * t4;
         const float2 u0 = *reinterpret_cast<const float2*>(Uc + r0 * LDU + c);
         const float2 u1 = *reinterpret_cast<const float2*>(Uc + r1 * LDU + c);
-        const float x0 = u0.x - P[nt][0], x1 = u0.y - P[nt][1];
-        const float x2 = u1.x - P[nt][2], x3 = u1.y - P[nt][3];
-        uint32_t h, l;
-        split2(x0, x1, h, l);
-        *reinterpret_cast<uint32_t*>(Uth + r0 * LDH + c) = h;
-        *reinterpret_cast<uint32_t*>(Utl + r0 * LDH + c) = l;
-        split2(x2, x3, h, l);
-        *reinterpret_cast<uint32_t*>(Uth + r1 * LDH + c) = h;
-        *reinterpret_cast<uint32_t*>(Utl + r1 * LDH + c) = l;
-        split2(x0 * fs0, x1 * fs0, h, l);
-        *reinterpret_cast<uint32_t*>(Ush + r0 * LDH + c) = h;
-        *reinterpret_cast<uint32_t*>(Usl + r0 * LDH + c) = l;
-        split2(x2 * fs1, x3 * fs1, h, l);
-        *reinterpret_cast<uint32_t*>(Ush + r1 * LDH + c) = h;
-        *reinterpret_cast<uint32_t*>(Usl + r1 * LDH + c) = l;
+        const float x0 = fmaf(sigma, u0.x, -P[nt][0]), x1 = fmaf(sigma, u0.y, -P[nt][1]);
+        const float x2 = fmaf(sigma, u1.x, -P[nt][2]), x3 = fmaf(sigma, u1.y, -P[nt][3]);
+        range = fmaxf(range, fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3))));
+        *reinterpret_cast<uint32_t*>(Ut + r0 * LDH + c) = pack2h(x0, x1);
+        *reinterpret_cast<uint32_t*>(Ut + r1 * LDH + c) = pack2h(x2, x3);
+        *reinterpret_cast<uint32_t*>(Us + r0 * LDH + c) = pack2h(x0 * fs0, x1 * fs0);
+        *reinterpret_cast<uint32_t*>(Us + r1 * LDH + c) = pack2h(x2 * fs1, x3 * fs1);
       }
     }
-    if (more) cp_wait<1>();  // K and A_qk of chunk n (the next stage may still be in flight)
+    if (more) cp_wait<1>();  // K rows and A_qk of chunk n (the next stage may still be in flight)
     else cp_wait<0>();
     __syncthreads();
 
-    // o = fo (Q S) + (A_hi + A_lo)(U~_hi + U~_lo), the lo x lo term dropped
+    // o = (fo (Q S) + A_qk U~) / sigma
     {
       float OA[4][4] = {};
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        uint32_t ah[4], al[4];
-        ldsm_x4(ah, Ah + (16 * mt + lrow_a(lane)) * LDH + 16 * ks + lcol_a(lane));
-        ldsm_x4(al, Al + (16 * mt + lrow_a(lane)) * LDH + 16 * ks + lcol_a(lane));
+        uint32_t a[4];
+        ldsm_x4(a, At + (16 * mt + lrow_a(lane)) * LDH + 16 * ks + lcol_a(lane));
 #pragma unroll
         for (int np = 0; np < 2; ++np) {
-          uint32_t bh[4], bl[4];
-          const int uo = (16 * ks + lrow_a(lane)) * LDH + nb + 16 * np + lcol_a(lane);
-          ldsm_x4_t(bh, Uth + uo);
-          ldsm_x4_t(bl, Utl + uo);
-          mma_bf16(OA[2 * np], ah, bh[0], bh[1]);
-          mma_bf16(OA[2 * np + 1], ah, bh[2], bh[3]);
-          mma_bf16(OA[2 * np], ah, bl[0], bl[1]);
-          mma_bf16(OA[2 * np + 1], ah, bl[2], bl[3]);
-          mma_bf16(OA[2 * np], al, bh[0], bh[1]);
-          mma_bf16(OA[2 * np + 1], al, bh[2], bh[3]);
+          uint32_t bb[4];
+          ldsm_x4_t(bb, Ut + (16 * ks + lrow_a(lane)) * LDH + nb + 16 * np + lcol_a(lane));
+          mma_f16(OA[2 * np], a, bb[0], bb[1]);
+          mma_f16(OA[2 * np + 1], a, bb[2], bb[3]);
         }
       }
       const float fo0 = sc[r0], fo1 = sc[r1];
@@ -550,44 +594,46 @@ state_scan_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       const bool w0 = t0 + r0 < T, w1 = t0 + r1 < T;
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) {
-        if (w0) store2<TO>(o0 + 8 * nt, fo0 * OQ[nt][0] + OA[nt][0], fo0 * OQ[nt][1] + OA[nt][1]);
-        if (w1) store2<TO>(o1 + 8 * nt, fo1 * OQ[nt][2] + OA[nt][2], fo1 * OQ[nt][3] + OA[nt][3]);
+        if (w0)
+          store2<TO>(o0 + 8 * nt, (fo0 * OQ[nt][0] + OA[nt][0]) * inv_sigma,
+                     (fo0 * OQ[nt][1] + OA[nt][1]) * inv_sigma);
+        if (w1)
+          store2<TO>(o1 + 8 * nt, (fo1 * OQ[nt][2] + OA[nt][2]) * inv_sigma,
+                     (fo1 * OQ[nt][3] + OA[nt][3]) * inv_sigma);
       }
     }
 
-    // S <- gamma_C S + K^T (U~s_hi + U~s_lo)  (this warp's 16 state rows)
+    // S <- gamma_C S + K^T U~s  (this warp's 16 state rows)
     {
       const float gC = sc[2 * kC];
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) S[nt][e] *= gC;
+        for (int i = 0; i < 4; ++i) S[nt][i] *= gC;
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
         uint32_t a[4];
         ldsm_x4_t(a, Kt + (16 * ks + lrow_b(lane)) * LDT + 16 * warp + lcol_b(lane));
 #pragma unroll
         for (int np = 0; np < 4; ++np) {
-          uint32_t bh[4], bl[4];
-          const int uo = (16 * ks + lrow_a(lane)) * LDH + 16 * np + lcol_a(lane);
-          ldsm_x4_t(bh, Ush + uo);
-          ldsm_x4_t(bl, Usl + uo);
-          mma_bf16(S[2 * np], a, bh[0], bh[1]);
-          mma_bf16(S[2 * np + 1], a, bh[2], bh[3]);
-          mma_bf16(S[2 * np], a, bl[0], bl[1]);
-          mma_bf16(S[2 * np + 1], a, bl[2], bl[3]);
+          uint32_t bb[4];
+          ldsm_x4_t(bb, Us + (16 * ks + lrow_a(lane)) * LDH + 16 * np + lcol_a(lane));
+          mma_f16(S[2 * np], a, bb[0], bb[1]);
+          mma_f16(S[2 * np + 1], a, bb[2], bb[3]);
         }
       }
-      store_state_bf16();
+      store_state();
     }
   }
+  if (!(range <= kF16Max)) report_range(status);
 
   if (ht != nullptr) {
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
       float* dst = ht + ((size_t)head * kD + s0) * kD + c0 + 8 * nt + 2 * t4;
-      *reinterpret_cast<float2*>(dst) = make_float2(S[nt][0], S[nt][1]);
-      *reinterpret_cast<float2*>(dst + 8 * kD) = make_float2(S[nt][2], S[nt][3]);
+      *reinterpret_cast<float2*>(dst) = make_float2(S[nt][0] * inv_sigma, S[nt][1] * inv_sigma);
+      *reinterpret_cast<float2*>(dst + 8 * kD) =
+          make_float2(S[nt][2] * inv_sigma, S[nt][3] * inv_sigma);
     }
   }
 }
@@ -596,21 +642,22 @@ template <typename TO>
 cudaError_t launch_t(const ChunkArgs& a, uint8_t* ws, const WsLayout& L, cudaStream_t s) {
   const int Nc = (a.T + kC - 1) / kC;
   const bool pre = (a.flags & GDN_GATES_PRECOMPUTED) != 0;
+  int* status = status_word();
+  if (status == nullptr) return cudaErrorUnknown;
   auto prep = pre ? wy_prep_kernel<true> : wy_prep_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_BYTES);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(state_scan_kernel<TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            S_BYTES);
   if (e != cudaSuccess) return e;
-  const bf16* q = static_cast<const bf16*>(a.q);
-  const bf16* k = static_cast<const bf16*>(a.k);
   prep<<<dim3(a.Hv / a.Hk, Nc, a.B * a.Hk), kThreads, P_BYTES, s>>>(
-      q, k, static_cast<const bf16*>(a.v), a.a, a.b, a.A_log, a.dt_bias, a.T, a.Hk, a.Hv,
-      a.scale, (a.flags & GDN_QK_L2NORM) ? 1 : 0, ws, L);
+      static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
+      static_cast<const bf16*>(a.v), a.a, a.b, a.A_log, a.dt_bias, a.T, a.Hk, a.Hv, a.scale,
+      (a.flags & GDN_QK_L2NORM) ? 1 : 0, ws, L, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   state_scan_kernel<TO><<<dim3(2, a.B * a.Hv), kThreads, S_BYTES, s>>>(
-      q, k, ws, L, a.h0, a.T, a.Hk, a.Hv, static_cast<TO*>(a.o), a.ht);
+      ws, L, a.h0, a.T, a.Hk, a.Hv, static_cast<TO*>(a.o), a.ht, status);
   return cudaGetLastError();
 }
 
@@ -621,13 +668,13 @@ bool chunk_mma_supported(const ChunkArgs& a) {
          (long)a.B * a.Hk <= 65535 && ((long)a.T + kC - 1) / kC <= 65535;
 }
 
-size_t chunk_mma_workspace_bytes(int B, int T, int Hv) {
+size_t chunk_mma_workspace_bytes(int B, int T, int Hk, int Hv) {
   if (B <= 0 || T <= 0) return 0;
-  return ws_layout(B, T, Hv).total;
+  return ws_layout(B, T, Hk, Hv).total;
 }
 
 cudaError_t launch_chunk_mma(const ChunkArgs& a, void* ws, cudaStream_t s) {
-  const WsLayout L = ws_layout(a.B, a.T, a.Hv);
+  const WsLayout L = ws_layout(a.B, a.T, a.Hk, a.Hv);
   uint8_t* w = static_cast<uint8_t*>(ws);
   if (a.flags & GDN_OUT_F32) return launch_t<float>(a, w, L, s);
   return launch_t<bf16>(a, w, L, s);

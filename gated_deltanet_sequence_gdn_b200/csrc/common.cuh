@@ -41,5 +41,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ void report_timeout(int* status, int where) {
   atomicCAS(status, 0, where);
 }
+// Bit of the status word set when an intermediate left the range of its
+// reduced-precision operand format (the outputs of that call are not valid).
+constexpr int kStatusRange = 1 << 30;
+__device__ __forceinline__ void report_range(int* status) {
+  if (status) atomicOr(status, kStatusRange);
+}
 
 }  // namespace gdn

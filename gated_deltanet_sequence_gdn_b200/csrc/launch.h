@@ -34,7 +34,7 @@ cudaError_t launch_chunk_simt(const ChunkArgs& a, bool gdn2, cudaStream_t s);
 // bf16 tensor-core chunk path (GDN, dk = dv = 128): WY prep + state scan,
 // with its intermediates in a caller-provided workspace.
 bool chunk_mma_supported(const ChunkArgs& a);
-size_t chunk_mma_workspace_bytes(int B, int T, int Hv);
+size_t chunk_mma_workspace_bytes(int B, int T, int Hk, int Hv);
 cudaError_t launch_chunk_mma(const ChunkArgs& a, void* workspace, cudaStream_t s);
 
 // Device address of this device's status word (set up once per device).

@@ -1,5 +1,5 @@
 // warp_mma.cuh -- warp-level tensor-core building blocks in inline PTX:
-// ldmatrix (plain and transposed), mma.sync m16n8k16 bf16 -> fp32, and
+// ldmatrix (plain and transposed), mma.sync m16n8k16 bf16 / fp16 -> fp32, and
 // cp.async 16-byte copies with zero fill and group waits.
 //
 // Fragment layouts (PTX ISA, "Matrix fragments for mma.m16n8k16"), with
@@ -11,6 +11,8 @@
 #pragma once
 
 #include <stdint.h>
+
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 
@@ -43,6 +45,16 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D = A B + D, fp16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                        uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // Per-lane offsets of the ldmatrix row addresses (in elements):
 //  tile_a : A operand from a row-major [m][k] tile, also the B operand (two n8
 //           tiles) from a row-major [k][n] tile with ldsm_x4_t;
@@ -62,6 +74,10 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 }
 __device__ __forceinline__ float2 unpack2(uint32_t u) {
   return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+}
+__device__ __forceinline__ uint32_t pack2h(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 // 16-byte global -> shared copy; src_bytes = 0 fills the 16 bytes with zeros

@@ -58,7 +58,9 @@ typedef enum gdn_status {
   GDN_ERR_UNSUPPORTED = -2, /* head dim not 64/128, Hv % Hk != 0, ...           */
   GDN_ERR_CUDA = -3,        /* a kernel launch or driver call failed            */
   GDN_ERR_TIMEOUT = -4,     /* a bounded device-side wait expired               */
-  GDN_ERR_WORKSPACE = -5    /* workspace smaller than gdn_*_workspace_bytes()   */
+  GDN_ERR_WORKSPACE = -5,   /* workspace smaller than gdn_*_workspace_bytes()   */
+  GDN_ERR_RANGE = -6        /* an intermediate left the range of its fp16      */
+                            /* operand format; that call's outputs are invalid  */
 } gdn_status;
 
 typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
@@ -128,10 +130,11 @@ int gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
                   void* workspace, size_t ws_bytes, gdn_stream_t stream);
 
 /* Workspace bytes gdn_chunk_fwd needs for these sizes: for the tensor-core
- * path (bf16, dk = dv = 128) B*Hv*(Tp*1024 + (Tp/64)*528) with Tp = T rounded
- * up to a multiple of 64 (per padded token and value head: a W row of 128 bf16,
- * a U row of 128 float32, A_qk rows of 64 bf16 in two parts; 528 B of factors
- * per chunk); 0 for every other case and for B*T = 0. */
+ * path (bf16, dk = dv = 128) B*Hv*(Tp*896 + (Tp/64)*528) + B*Hk*Tp*512 with
+ * Tp = T rounded up to a multiple of 64 (per padded token and value head: a W
+ * row of 128 fp16, a U row of 128 float32 and an A_qk row of 64 fp16; per
+ * padded token and key head: fp16 copies of the q and k rows; 528 B of factors
+ * per chunk and value head); 0 for every other case and for B*T = 0. */
 size_t gdn_chunk_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv,
                                  int dtype);
 
@@ -204,8 +207,11 @@ size_t gdn2_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype
 
 /*
  * gdn_check_status -- waits for `stream`, then reads and clears the device
- * status word of the current device.  Returns GDN_OK, GDN_ERR_TIMEOUT if a
- * bounded wait in a kernel expired since the last check, or GDN_ERR_CUDA.
+ * status word of the current device.  Returns GDN_OK, GDN_ERR_RANGE if an
+ * intermediate of the tensor-core chunk path left the fp16 operand range since
+ * the last check (inputs far outside the method's domain, e.g. keys of norm
+ * >> 1 with GDN_QK_L2NORM off), GDN_ERR_TIMEOUT if a bounded wait in a kernel
+ * expired, or GDN_ERR_CUDA.
  */
 int gdn_check_status(gdn_stream_t stream);
 
