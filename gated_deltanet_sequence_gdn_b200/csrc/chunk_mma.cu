@@ -11,11 +11,11 @@
 //      A_qk = tril(Q^ K^^T o Gamma) (diagonal included), written to the
 //      workspace with the per-row factors of the second kernel, together with
 //      fp16 copies of the raw Q and K tiles.
-//  state_scan_kernel : one CTA per (value head, 64-column half of d_v),
-//      sequential over the chunks with the fp32 state slice held in mma
-//      accumulator registers:  U~ = U - W S,  o = diag(gamma sq) Q S + A_qk U~,
-//      S <- gamma_C S + K^T diag(rk gamma_C / gamma) U~.  The next chunk's tiles
-//      are fetched with cp.async while the current one is computed.
+//  state_scan_kernel : one CTA (16 warps) per (value head, 64-column half of
+//      d_v), sequential over the chunks with the fp32 state slice held in mma
+//      accumulator registers (16 x 32 per warp):  U~ = U - W S,  o = diag(gamma sq) Q S + A_qk U~,
+//      S <- gamma_C S + K^T diag(rk gamma_C / gamma) U~.  All tiles of the next
+//      chunk are fetched with cp.async while the current one is computed.
 //
 // The algebra is the WY / UT chunk form of the delta rule ("Gated DeltaNet-2",
 // section on the chunkwise algorithm; GDN is its scalar-decay special case):
@@ -79,6 +79,35 @@ __device__ __forceinline__ void split2(float x, float y, uint32_t& hi, uint32_t&
   lo = pack2(x - h.x, y - h.y);
 }
 
+// A fragment (16 x 16, row-major) of an fp32 matrix M (row stride ld) at
+// (r0, c0), as bf16 hi + lo parts.
+__device__ __forceinline__ void frag_a_split(const float* M, int ld, int r0, int c0, int g8, int t4,
+                                             uint32_t (&hi)[4], uint32_t (&lo)[4]) {
+  const float2 x00 = *reinterpret_cast<const float2*>(M + (r0 + g8) * ld + c0 + 2 * t4);
+  const float2 x10 = *reinterpret_cast<const float2*>(M + (r0 + g8 + 8) * ld + c0 + 2 * t4);
+  const float2 x01 = *reinterpret_cast<const float2*>(M + (r0 + g8) * ld + c0 + 2 * t4 + 8);
+  const float2 x11 = *reinterpret_cast<const float2*>(M + (r0 + g8 + 8) * ld + c0 + 2 * t4 + 8);
+  split2(x00.x, x00.y, hi[0], lo[0]);
+  split2(x10.x, x10.y, hi[1], lo[1]);
+  split2(x01.x, x01.y, hi[2], lo[2]);
+  split2(x11.x, x11.y, hi[3], lo[3]);
+}
+// B fragment (16 x 8, k x n) of an fp32 matrix M (row = k) at (k0, n0), split.
+__device__ __forceinline__ void frag_b_split(const float* M, int ld, int k0, int n0, int g8, int t4,
+                                             uint32_t (&hi)[2], uint32_t (&lo)[2]) {
+  const float* p = M + (k0 + 2 * t4) * ld + n0 + g8;
+  split2(p[0], p[ld], hi[0], lo[0]);
+  split2(p[8 * ld], p[9 * ld], hi[1], lo[1]);
+}
+// D += A B for split operands, the lo x lo term dropped (about 2^-16 relative).
+__device__ __forceinline__ void mma_split3(float (&d)[4], const uint32_t (&ah)[4],
+                                           const uint32_t (&al)[4], const uint32_t (&bh)[2],
+                                           const uint32_t (&bl)[2]) {
+  mma_bf16(d, ah, bh[0], bh[1]);
+  mma_bf16(d, ah, bl[0], bl[1]);
+  mma_bf16(d, al, bh[0], bh[1]);
+}
+
 // Exponent e with (max |row|) * 2^-e in [1, 2) (e = 0 for a zero row).
 __device__ __forceinline__ int row_exponent(float m) { return m > 0.f ? ilogbf(m) : 0; }
 
@@ -89,8 +118,9 @@ constexpr int P_QT = P_KT + kC * LDT * 2;    // Q tile  (key head)
 constexpr int P_VT = P_QT + kC * LDT * 2;    // V tile  (value head)
 constexpr int P_L = P_VT + kC * LDT * 2;     // L [64][LDX] f32
 constexpr int P_X = P_L + kC * LDX * 4;      // X = (I + L)^-1
-constexpr int P_T = P_X + kC * LDX * 4;      // block products [3][16][17] f32
-constexpr int P_VEC = P_T + 3 * 16 * 17 * 4; // rk, sq, G, beta, c1, 2^eq, 2^ek [64], misc
+constexpr int LDB = 20;                      // f32 row stride of a 16 x 16 block product
+constexpr int P_T = P_X + kC * LDX * 4;      // block products, one [16][LDB] f32 per warp 0-2
+constexpr int P_VEC = P_T + 3 * 16 * LDB * 4; // rk, sq, G, beta, c1, 2^eq, 2^ek [64], misc
 constexpr int P_BYTES = P_VEC + 8 * 64 * 4;
 static_assert(2 * (P_BYTES + 1024) <= 228 * 1024, "two prep CTAs per SM");
 
@@ -171,10 +201,10 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
   //    fp16 copies (two threads per row)
   {
     const int which = tid >> 7, r = (tid & 127) >> 1, h = tid & 1;
-    const bf16* row = (which ? Qt : Kt) + r * LDT + h * 64;
+    const bf16* row = (which ? Qt : Kt) + r * LDT + h * 8;  // 16-byte chunks h, h + 2, ...
     float ss = 0.f, mx = 0.f;
 #pragma unroll
-    for (int c = 0; c < 64; c += 8) {
+    for (int c = 0; c < 128; c += 16) {
       const uint4 u = *reinterpret_cast<const uint4*>(row + c);
       const float2 f0 = unpack2(u.x), f1 = unpack2(u.y), f2 = unpack2(u.z), f3 = unpack2(u.w);
       ss += f0.x * f0.x + f0.y * f0.y + f1.x * f1.x + f1.y * f1.y + f2.x * f2.x + f2.y * f2.y +
@@ -185,29 +215,30 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     const int e = row_exponent(mx);
+    const float up = ldexpf(1.f, e), down = ldexpf(1.f, -e);  // exact powers of 2
     if (h == 0) {
       const float inv = l2 ? rsqrtf(ss + 1e-6f) : 1.f;
       if (which) {
         sq[r] = inv * scale;
-        pq[r] = ldexpf(1.f, e);
+        pq[r] = up;
       } else {
         rk[r] = inv;
-        pk[r] = ldexpf(1.f, e);
+        pk[r] = up;
       }
     }
     // fp16 copies of the raw rows, row-scaled by 2^-e (written once per key head)
     if (blockIdx.x == 0) {
       __half* dst = reinterpret_cast<__half*>(ws + (which ? L.qh : L.kh)) +
-                    ((size_t)blockIdx.z * Tp + t0 + r) * kD + h * 64;
+                    ((size_t)blockIdx.z * Tp + t0 + r) * kD + h * 8;
 #pragma unroll
-      for (int c = 0; c < 64; c += 8) {
+      for (int c = 0; c < 128; c += 16) {
         const uint4 u = *reinterpret_cast<const uint4*>(row + c);
         const float2 f0 = unpack2(u.x), f1 = unpack2(u.y), f2 = unpack2(u.z), f3 = unpack2(u.w);
         uint4 o;
-        o.x = pack2h(ldexpf(f0.x, -e), ldexpf(f0.y, -e));
-        o.y = pack2h(ldexpf(f1.x, -e), ldexpf(f1.y, -e));
-        o.z = pack2h(ldexpf(f2.x, -e), ldexpf(f2.y, -e));
-        o.w = pack2h(ldexpf(f3.x, -e), ldexpf(f3.y, -e));
+        o.x = pack2h(f0.x * down, f0.y * down);
+        o.y = pack2h(f1.x * down, f1.y * down);
+        o.z = pack2h(f2.x * down, f2.y * down);
+        o.w = pack2h(f3.x * down, f3.y * down);
         *reinterpret_cast<uint4*>(dst + c) = o;
       }
     }
@@ -289,27 +320,47 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
     }
   }
   __syncthreads();
-  //    then block row by block row: X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj
+  //    then block row by block row, on the tensor cores (fp32 operands as bf16
+  //    hi + lo): warp j < i computes T = sum_{k=j}^{i-1} L_ik X_kj and
+  //    X_ij = -X_ii T for its block (j = warp)
   for (int bi = 1; bi < 4; ++bi) {
-    for (int e = tid; e < bi * 256; e += kThreads) {
-      const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-      float s = 0.f;
+    if (warp < bi) {
+      const int bj = warp;
+      float* Tw = Tm + warp * 16 * LDB;
+      float t[2][4] = {};
       for (int kb = bj; kb < bi; ++kb) {
+        uint32_t ah[4], al[4];
+        frag_a_split(Lm, LDX, 16 * bi, 16 * kb, g8, t4, ah, al);
 #pragma unroll
-        for (int qq = 0; qq < 16; ++qq)
-          s = fmaf(Lm[(16 * bi + rr) * LDX + 16 * kb + qq], Xm[(16 * kb + qq) * LDX + 16 * bj + cc],
-                   s);
+        for (int nt = 0; nt < 2; ++nt) {
+          uint32_t bh[2], bl[2];
+          frag_b_split(Xm, LDX, 16 * kb, 16 * bj + 8 * nt, g8, t4, bh, bl);
+          mma_split3(t[nt], ah, al, bh, bl);
+        }
       }
-      Tm[(bj * 16 + rr) * 17 + cc] = s;
-    }
-    __syncthreads();
-    for (int e = tid; e < bi * 256; e += kThreads) {
-      const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-      float s = 0.f;
 #pragma unroll
-      for (int qq = 0; qq < 16; ++qq)
-        s = fmaf(Xm[(16 * bi + rr) * LDX + 16 * bi + qq], Tm[(bj * 16 + qq) * 17 + cc], s);
-      Xm[(16 * bi + rr) * LDX + 16 * bj + cc] = -s;
+      for (int nt = 0; nt < 2; ++nt) {
+        *reinterpret_cast<float2*>(Tw + g8 * LDB + 8 * nt + 2 * t4) = make_float2(t[nt][0], t[nt][1]);
+        *reinterpret_cast<float2*>(Tw + (g8 + 8) * LDB + 8 * nt + 2 * t4) =
+            make_float2(t[nt][2], t[nt][3]);
+      }
+      __syncwarp();
+      float x[2][4] = {};
+      uint32_t ah[4], al[4];
+      frag_a_split(Xm, LDX, 16 * bi, 16 * bi, g8, t4, ah, al);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t bh[2], bl[2];
+        frag_b_split(Tw, LDB, 0, 8 * nt, g8, t4, bh, bl);
+        mma_split3(x[nt], ah, al, bh, bl);
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int c = 16 * bj + 8 * nt + 2 * t4;
+        *reinterpret_cast<float2*>(Xm + (16 * bi + g8) * LDX + c) = make_float2(-x[nt][0], -x[nt][1]);
+        *reinterpret_cast<float2*>(Xm + (16 * bi + g8 + 8) * LDX + c) =
+            make_float2(-x[nt][2], -x[nt][3]);
+      }
     }
     __syncthreads();
   }
@@ -397,21 +448,21 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
 }
 
 // ---------------------------------------------------------------- scan kernel
+constexpr int kScanThreads = 512;           // 16 warps
 constexpr int LDU = 64 + 8;                 // f32 row stride of the U tile (conflict-free float2)
 // double-buffered, fetched one chunk ahead
 constexpr int S_W = 0;                      // W tile     [64][LDT] f16
 constexpr int S_Q = S_W + kC * LDT * 2;     // Q rows     [64][LDT] f16
-constexpr int S_U = S_Q + kC * LDT * 2;     // U columns of this CTA [64][LDU] f32
+constexpr int S_K = S_Q + kC * LDT * 2;     // K rows     [64][LDT] f16
+constexpr int S_A = S_K + kC * LDT * 2;     // A_qk       [64][LDH] f16
+constexpr int S_U = S_A + kC * LDH * 2;     // U columns of this CTA [64][LDU] f32
 constexpr int S_SC = S_U + kC * LDU * 4;    // scalars (132 f32)
 constexpr int STAGE = S_SC + kScal * 4;
-// single-buffered, fetched at the start of the chunk that uses them
-constexpr int S_K = 2 * STAGE;              // K rows [64][LDT] f16
-constexpr int S_A = S_K + kC * LDT * 2;     // A_qk   [64][LDH] f16
 // on-chip operands
-constexpr int S_SB = S_A + kC * LDH * 2;    // state slice (scaled) [128][LDH] f16
+constexpr int S_SB = 2 * STAGE;             // state slice (scaled) [128][LDH] f16
 constexpr int S_UT = S_SB + kD * LDH * 2;   // U~ (scaled)          [64][LDH] f16
 constexpr int S_US = S_UT + kC * LDH * 2;   // U~ diag(fs)          [64][LDH] f16
-constexpr int S_RED = S_US + kC * LDH * 2;  // 8 floats for the CTA max
+constexpr int S_RED = S_US + kC * LDH * 2;  // 16 floats for the CTA max
 constexpr int S_BYTES = S_RED + 64;
 static_assert(STAGE % 16 == 0, "stage buffers must stay 16-byte aligned");
 static_assert(S_BYTES <= 227 * 1024, "shared memory of the scan kernel");
@@ -428,12 +479,10 @@ __device__ __forceinline__ void store2<bf16>(bf16* p, float x, float y) {
 }
 
 template <typename TO>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kScanThreads, 1)
 state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, int T, int Hk,
                   int Hv, TO* __restrict__ o, float* ht, int* status) {
   extern __shared__ __align__(16) uint8_t sm[];
-  __half* Kt = reinterpret_cast<__half*>(sm + S_K);
-  __half* At = reinterpret_cast<__half*>(sm + S_A);
   __half* Sb = reinterpret_cast<__half*>(sm + S_SB);
   __half* Ut = reinterpret_cast<__half*>(sm + S_UT);
   __half* Us = reinterpret_cast<__half*>(sm + S_US);
@@ -451,40 +500,33 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
   const __half* Kg = reinterpret_cast<const __half*>(ws + L.kh) + khead * Tp * kD;
   const float* Sg = reinterpret_cast<const float*>(ws + L.scal) + (size_t)head * Nc * kScal;
 
-  // W, Q, U and the scalars of chunk n into stage n % 2
+  // every tile of chunk n into stage n % 2
   auto issue_stage = [&](int n) {
     uint8_t* st = sm + (n & 1) * STAGE;
     const size_t r0 = (size_t)n * kC;
-    for (int i = tid; i < kC * 16; i += kThreads) {
+    for (int i = tid; i < kC * 16; i += kScanThreads) {
       const int r = i >> 4, c16 = i & 15;
       cp16(st + S_W + (r * LDT + c16 * 8) * 2, Wg + (r0 + r) * kD + c16 * 8, 16);
       cp16(st + S_Q + (r * LDT + c16 * 8) * 2, Qg + (r0 + r) * kD + c16 * 8, 16);
+      cp16(st + S_K + (r * LDT + c16 * 8) * 2, Kg + (r0 + r) * kD + c16 * 8, 16);
       cp16(st + S_U + (r * LDU + c16 * 4) * 4, Ug + (r0 + r) * kD + c16 * 4, 16);
+      if (c16 < 8) cp16(st + S_A + (r * LDH + c16 * 8) * 2, Ag + (r0 + r) * kC + c16 * 8, 16);
     }
     if (tid < kScal / 4) cp16(st + S_SC + tid * 16, Sg + (size_t)n * kScal + tid * 4, 16);
     cp_commit();
   };
-  // K rows and A_qk of chunk n
-  auto issue_ka = [&](int n) {
-    const size_t r0 = (size_t)n * kC;
-    for (int i = tid; i < kC * 16; i += kThreads) {
-      const int r = i >> 4, c16 = i & 15;
-      cp16(Kt + r * LDT + c16 * 8, Kg + (r0 + r) * kD + c16 * 8, 16);
-      if (c16 < 8) cp16(At + r * LDH + c16 * 8, Ag + (r0 + r) * kC + c16 * 8, 16);
-    }
-    cp_commit();
-  };
   issue_stage(0);
 
-  // state slice: warp w holds rows 16 w .. 16 w + 15, all 64 columns, as 8 C fragments
-  float S[8][4];
-  const int s0 = 16 * warp + g8;
+  // state slice: warp w holds rows 16 (w % 8) .. + 15 and columns 32 (w / 8) .. + 31
+  // of the CTA's 128 x 64 slice, as 4 C fragments
+  const int sr = 16 * (warp & 7) + g8, scb = 32 * (warp >> 3);
+  float S[4][4];
   float mx = 0.f;
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
+  for (int nt = 0; nt < 4; ++nt) {
     float2 x0 = make_float2(0.f, 0.f), x1 = x0;
     if (h0) {
-      const float* src = h0 + ((size_t)head * kD + s0) * kD + c0 + 8 * nt + 2 * t4;
+      const float* src = h0 + ((size_t)head * kD + sr) * kD + c0 + scb + 8 * nt + 2 * t4;
       x0 = *reinterpret_cast<const float2*>(src);
       x1 = *reinterpret_cast<const float2*>(src + 8 * kD);
     }
@@ -492,71 +534,68 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
     mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x0.x), fabsf(x0.y)), fmaxf(fabsf(x1.x), fabsf(x1.y))));
   }
   // sigma = 2^-e: the largest |U| of the head and |h0| of this slice land below 2^8
-  for (int n = tid; n < Nc; n += kThreads) mx = fmaxf(mx, Sg[(size_t)n * kScal + 2 * kC + 1]);
+  for (int n = tid; n < Nc; n += kScanThreads) mx = fmaxf(mx, Sg[(size_t)n * kScal + 2 * kC + 1]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   if (lane == 0) red[warp] = mx;
   __syncthreads();
   mx = red[0];
 #pragma unroll
-  for (int w = 1; w < 8; ++w) mx = fmaxf(mx, red[w]);
+  for (int w = 1; w < 16; ++w) mx = fmaxf(mx, red[w]);
   const int e = mx > 0.f ? min(max(ilogbf(mx) - 7, -100), 100) : 0;
   const float sigma = ldexpf(1.f, -e), inv_sigma = ldexpf(1.f, e);
   float range = 0.f;
 
   auto store_state = [&]() {
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int c = 8 * nt + 2 * t4;
+    for (int nt = 0; nt < 4; ++nt) {
+      const int c = scb + 8 * nt + 2 * t4;
       range = fmaxf(range, fmaxf(fmaxf(fabsf(S[nt][0]), fabsf(S[nt][1])),
                                  fmaxf(fabsf(S[nt][2]), fabsf(S[nt][3]))));
-      *reinterpret_cast<uint32_t*>(Sb + s0 * LDH + c) = pack2h(S[nt][0], S[nt][1]);
-      *reinterpret_cast<uint32_t*>(Sb + (s0 + 8) * LDH + c) = pack2h(S[nt][2], S[nt][3]);
+      *reinterpret_cast<uint32_t*>(Sb + sr * LDH + c) = pack2h(S[nt][0], S[nt][1]);
+      *reinterpret_cast<uint32_t*>(Sb + (sr + 8) * LDH + c) = pack2h(S[nt][2], S[nt][3]);
     }
   };
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
+  for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) S[nt][i] *= sigma;
   store_state();
 
-  const int mt = warp & 3, nb = 32 * (warp >> 2);  // output tile of this warp: 16 rows x 32 cols
+  // output tile of this warp: rows 16 (w % 4) .. + 15, columns 16 (w / 4) .. + 15
+  const int mt = warp & 3, nb = 16 * (warp >> 2);
   const int r0 = 16 * mt + g8, r1 = r0 + 8;
   for (int n = 0; n < Nc; ++n) {
     cp_wait<0>();
-    __syncthreads();  // stage n landed; the previous chunk's reads and state stores are done
-    issue_ka(n);
-    const bool more = n + 1 < Nc;
-    if (more) issue_stage(n + 1);
+    __syncthreads();  // chunk n landed; the previous chunk's reads and state stores are done
+    if (n + 1 < Nc) issue_stage(n + 1);
     const uint8_t* st = sm + (n & 1) * STAGE;
     const __half* Wt = reinterpret_cast<const __half*>(st + S_W);
     const __half* Qt = reinterpret_cast<const __half*>(st + S_Q);
+    const __half* Kt = reinterpret_cast<const __half*>(st + S_K);
+    const __half* At = reinterpret_cast<const __half*>(st + S_A);
     const float* Uc = reinterpret_cast<const float*>(st + S_U);
     const float* sc = reinterpret_cast<const float*>(st + S_SC);
     const int t0 = n * kC;
 
     // P = W S and OQ = Q S for this warp's tile (S scaled by sigma)
-    float P[4][4] = {}, OQ[4][4] = {};
+    float P[2][4] = {}, OQ[2][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      uint32_t aw[4], aq[4];
+      uint32_t aw[4], aq[4], bb[4];
       ldsm_x4(aw, Wt + (16 * mt + lrow_a(lane)) * LDT + 16 * ks + lcol_a(lane));
       ldsm_x4(aq, Qt + (16 * mt + lrow_a(lane)) * LDT + 16 * ks + lcol_a(lane));
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        uint32_t bb[4];
-        ldsm_x4_t(bb, Sb + (16 * ks + lrow_a(lane)) * LDH + nb + 16 * np + lcol_a(lane));
-        mma_f16(P[2 * np], aw, bb[0], bb[1]);
-        mma_f16(P[2 * np + 1], aw, bb[2], bb[3]);
-        mma_f16(OQ[2 * np], aq, bb[0], bb[1]);
-        mma_f16(OQ[2 * np + 1], aq, bb[2], bb[3]);
-      }
+      ldsm_x4_t(bb, Sb + (16 * ks + lrow_a(lane)) * LDH + nb + lcol_a(lane));
+      mma_f16(P[0], aw, bb[0], bb[1]);
+      mma_f16(P[1], aw, bb[2], bb[3]);
+      mma_f16(OQ[0], aq, bb[0], bb[1]);
+      mma_f16(OQ[1], aq, bb[2], bb[3]);
     }
     // U~ = sigma U - P, and U~ diag(fs) for the state update, in fp16
     {
       const float fs0 = sc[kC + r0], fs1 = sc[kC + r1];
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
+      for (int nt = 0; nt < 2; ++nt) {
         const int c = nb + 8 * nt + 2 * t4;
         const float2 u0 = *reinterpret_cast<const float2*>(Uc + r0 * LDU + c);
         const float2 u1 = *reinterpret_cast<const float2*>(Uc + r1 * LDU + c);
@@ -569,31 +608,25 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
         *reinterpret_cast<uint32_t*>(Us + r1 * LDH + c) = pack2h(x2 * fs1, x3 * fs1);
       }
     }
-    if (more) cp_wait<1>();  // K rows and A_qk of chunk n (the next stage may still be in flight)
-    else cp_wait<0>();
     __syncthreads();
 
     // o = (fo (Q S) + A_qk U~) / sigma
     {
-      float OA[4][4] = {};
+      float OA[2][4] = {};
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        uint32_t a[4];
+        uint32_t a[4], bb[4];
         ldsm_x4(a, At + (16 * mt + lrow_a(lane)) * LDH + 16 * ks + lcol_a(lane));
-#pragma unroll
-        for (int np = 0; np < 2; ++np) {
-          uint32_t bb[4];
-          ldsm_x4_t(bb, Ut + (16 * ks + lrow_a(lane)) * LDH + nb + 16 * np + lcol_a(lane));
-          mma_f16(OA[2 * np], a, bb[0], bb[1]);
-          mma_f16(OA[2 * np + 1], a, bb[2], bb[3]);
-        }
+        ldsm_x4_t(bb, Ut + (16 * ks + lrow_a(lane)) * LDH + nb + lcol_a(lane));
+        mma_f16(OA[0], a, bb[0], bb[1]);
+        mma_f16(OA[1], a, bb[2], bb[3]);
       }
       const float fo0 = sc[r0], fo1 = sc[r1];
       TO* o0 = o + (((size_t)b * T + t0 + r0) * Hv + hv) * kD + c0 + nb + 2 * t4;
       TO* o1 = o0 + (size_t)8 * Hv * kD;
       const bool w0 = t0 + r0 < T, w1 = t0 + r1 < T;
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
+      for (int nt = 0; nt < 2; ++nt) {
         if (w0)
           store2<TO>(o0 + 8 * nt, (fo0 * OQ[nt][0] + OA[nt][0]) * inv_sigma,
                      (fo0 * OQ[nt][1] + OA[nt][1]) * inv_sigma);
@@ -603,21 +636,21 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
       }
     }
 
-    // S <- gamma_C S + K^T U~s  (this warp's 16 state rows)
+    // S <- gamma_C S + K^T U~s  (this warp's 16 x 32 block of the state slice)
     {
       const float gC = sc[2 * kC];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
+      for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) S[nt][i] *= gC;
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
         uint32_t a[4];
-        ldsm_x4_t(a, Kt + (16 * ks + lrow_b(lane)) * LDT + 16 * warp + lcol_b(lane));
+        ldsm_x4_t(a, Kt + (16 * ks + lrow_b(lane)) * LDT + 16 * (warp & 7) + lcol_b(lane));
 #pragma unroll
-        for (int np = 0; np < 4; ++np) {
+        for (int np = 0; np < 2; ++np) {
           uint32_t bb[4];
-          ldsm_x4_t(bb, Us + (16 * ks + lrow_a(lane)) * LDH + 16 * np + lcol_a(lane));
+          ldsm_x4_t(bb, Us + (16 * ks + lrow_a(lane)) * LDH + scb + 16 * np + lcol_a(lane));
           mma_f16(S[2 * np], a, bb[0], bb[1]);
           mma_f16(S[2 * np + 1], a, bb[2], bb[3]);
         }
@@ -629,8 +662,8 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
 
   if (ht != nullptr) {
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      float* dst = ht + ((size_t)head * kD + s0) * kD + c0 + 8 * nt + 2 * t4;
+    for (int nt = 0; nt < 4; ++nt) {
+      float* dst = ht + ((size_t)head * kD + sr) * kD + c0 + scb + 8 * nt + 2 * t4;
       *reinterpret_cast<float2*>(dst) = make_float2(S[nt][0] * inv_sigma, S[nt][1] * inv_sigma);
       *reinterpret_cast<float2*>(dst + 8 * kD) =
           make_float2(S[nt][2] * inv_sigma, S[nt][3] * inv_sigma);
@@ -656,7 +689,7 @@ cudaError_t launch_t(const ChunkArgs& a, uint8_t* ws, const WsLayout& L, cudaStr
       (a.flags & GDN_QK_L2NORM) ? 1 : 0, ws, L, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  state_scan_kernel<TO><<<dim3(2, a.B * a.Hv), kThreads, S_BYTES, s>>>(
+  state_scan_kernel<TO><<<dim3(2, a.B * a.Hv), kScanThreads, S_BYTES, s>>>(
       ws, L, a.h0, a.T, a.Hk, a.Hv, static_cast<TO*>(a.o), a.ht, status);
   return cudaGetLastError();
 }
