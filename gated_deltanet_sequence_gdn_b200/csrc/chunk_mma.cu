@@ -11,9 +11,9 @@
 //      A_qk = tril(Q^ K^^T o Gamma) (diagonal included), written to the
 //      workspace with the per-row factors of the second kernel, together with
 //      fp16 copies of the raw Q and K tiles.
-//  state_scan_kernel : one CTA (16 warps) per (value head, 64-column half of
+//  state_scan_kernel : one CTA (8 warps) per (value head, 64-column half of
 //      d_v), sequential over the chunks with the fp32 state slice held in mma
-//      accumulator registers (16 x 32 per warp):  U~ = U - W S,  o = diag(gamma sq) Q S + A_qk U~,
+//      accumulator registers (16 x 64 per warp):  U~ = U - W S,  o = diag(gamma sq) Q S + A_qk U~,
 //      S <- gamma_C S + K^T diag(rk gamma_C / gamma) U~.  All tiles of the next
 //      chunk are fetched with cp.async while the current one is computed.
 //
@@ -448,7 +448,7 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
 }
 
 // ---------------------------------------------------------------- scan kernel
-constexpr int kScanThreads = 512;           // 16 warps
+constexpr int kScanThreads = 256;           // 8 warps
 constexpr int LDU = 64 + 8;                 // f32 row stride of the U tile (conflict-free float2)
 // double-buffered, fetched one chunk ahead
 constexpr int S_W = 0;                      // W tile     [64][LDT] f16
@@ -462,7 +462,7 @@ constexpr int STAGE = S_SC + kScal * 4;
 constexpr int S_SB = 2 * STAGE;             // state slice (scaled) [128][LDH] f16
 constexpr int S_UT = S_SB + kD * LDH * 2;   // U~ (scaled)          [64][LDH] f16
 constexpr int S_US = S_UT + kC * LDH * 2;   // U~ diag(fs)          [64][LDH] f16
-constexpr int S_RED = S_US + kC * LDH * 2;  // 16 floats for the CTA max
+constexpr int S_RED = S_US + kC * LDH * 2;  // 8 floats for the CTA max
 constexpr int S_BYTES = S_RED + 64;
 static_assert(STAGE % 16 == 0, "stage buffers must stay 16-byte aligned");
 static_assert(S_BYTES <= 227 * 1024, "shared memory of the scan kernel");
@@ -517,16 +517,16 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
   };
   issue_stage(0);
 
-  // state slice: warp w holds rows 16 (w % 8) .. + 15 and columns 32 (w / 8) .. + 31
-  // of the CTA's 128 x 64 slice, as 4 C fragments
-  const int sr = 16 * (warp & 7) + g8, scb = 32 * (warp >> 3);
-  float S[4][4];
+  // state slice: warp w holds rows 16 w .. + 15 and all 64 columns of the CTA's
+  // 128 x 64 slice, as 8 C fragments
+  const int sr = 16 * warp + g8;
+  float S[8][4];
   float mx = 0.f;
 #pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
+  for (int nt = 0; nt < 8; ++nt) {
     float2 x0 = make_float2(0.f, 0.f), x1 = x0;
     if (h0) {
-      const float* src = h0 + ((size_t)head * kD + sr) * kD + c0 + scb + 8 * nt + 2 * t4;
+      const float* src = h0 + ((size_t)head * kD + sr) * kD + c0 + 8 * nt + 2 * t4;
       x0 = *reinterpret_cast<const float2*>(src);
       x1 = *reinterpret_cast<const float2*>(src + 8 * kD);
     }
@@ -541,15 +541,15 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
   __syncthreads();
   mx = red[0];
 #pragma unroll
-  for (int w = 1; w < 16; ++w) mx = fmaxf(mx, red[w]);
+  for (int w = 1; w < 8; ++w) mx = fmaxf(mx, red[w]);
   const int e = mx > 0.f ? min(max(ilogbf(mx) - 7, -100), 100) : 0;
   const float sigma = ldexpf(1.f, -e), inv_sigma = ldexpf(1.f, e);
   float range = 0.f;
 
   auto store_state = [&]() {
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const int c = scb + 8 * nt + 2 * t4;
+    for (int nt = 0; nt < 8; ++nt) {
+      const int c = 8 * nt + 2 * t4;
       range = fmaxf(range, fmaxf(fmaxf(fabsf(S[nt][0]), fabsf(S[nt][1])),
                                  fmaxf(fabsf(S[nt][2]), fabsf(S[nt][3]))));
       *reinterpret_cast<uint32_t*>(Sb + sr * LDH + c) = pack2h(S[nt][0], S[nt][1]);
@@ -557,13 +557,13 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
     }
   };
 #pragma unroll
-  for (int nt = 0; nt < 4; ++nt)
+  for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) S[nt][i] *= sigma;
   store_state();
 
-  // output tile of this warp: rows 16 (w % 4) .. + 15, columns 16 (w / 4) .. + 15
-  const int mt = warp & 3, nb = 16 * (warp >> 2);
+  // output tile of this warp: rows 16 (w % 4) .. + 15, columns 32 (w / 4) .. + 31
+  const int mt = warp & 3, nb = 32 * (warp >> 2);
   const int r0 = 16 * mt + g8, r1 = r0 + 8;
   for (int n = 0; n < Nc; ++n) {
     cp_wait<0>();
@@ -579,23 +579,27 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
     const int t0 = n * kC;
 
     // P = W S and OQ = Q S for this warp's tile (S scaled by sigma)
-    float P[2][4] = {}, OQ[2][4] = {};
+    float P[4][4] = {}, OQ[4][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      uint32_t aw[4], aq[4], bb[4];
+      uint32_t aw[4], aq[4];
       ldsm_x4(aw, Wt + (16 * mt + lrow_a(lane)) * LDT + 16 * ks + lcol_a(lane));
       ldsm_x4(aq, Qt + (16 * mt + lrow_a(lane)) * LDT + 16 * ks + lcol_a(lane));
-      ldsm_x4_t(bb, Sb + (16 * ks + lrow_a(lane)) * LDH + nb + lcol_a(lane));
-      mma_f16(P[0], aw, bb[0], bb[1]);
-      mma_f16(P[1], aw, bb[2], bb[3]);
-      mma_f16(OQ[0], aq, bb[0], bb[1]);
-      mma_f16(OQ[1], aq, bb[2], bb[3]);
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        uint32_t bb[4];
+        ldsm_x4_t(bb, Sb + (16 * ks + lrow_a(lane)) * LDH + nb + 16 * np + lcol_a(lane));
+        mma_f16(P[2 * np], aw, bb[0], bb[1]);
+        mma_f16(P[2 * np + 1], aw, bb[2], bb[3]);
+        mma_f16(OQ[2 * np], aq, bb[0], bb[1]);
+        mma_f16(OQ[2 * np + 1], aq, bb[2], bb[3]);
+      }
     }
     // U~ = sigma U - P, and U~ diag(fs) for the state update, in fp16
     {
       const float fs0 = sc[kC + r0], fs1 = sc[kC + r1];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
+      for (int nt = 0; nt < 4; ++nt) {
         const int c = nb + 8 * nt + 2 * t4;
         const float2 u0 = *reinterpret_cast<const float2*>(Uc + r0 * LDU + c);
         const float2 u1 = *reinterpret_cast<const float2*>(Uc + r1 * LDU + c);
@@ -612,21 +616,25 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
 
     // o = (fo (Q S) + A_qk U~) / sigma
     {
-      float OA[2][4] = {};
+      float OA[4][4] = {};
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        uint32_t a[4], bb[4];
+        uint32_t a[4];
         ldsm_x4(a, At + (16 * mt + lrow_a(lane)) * LDH + 16 * ks + lcol_a(lane));
-        ldsm_x4_t(bb, Ut + (16 * ks + lrow_a(lane)) * LDH + nb + lcol_a(lane));
-        mma_f16(OA[0], a, bb[0], bb[1]);
-        mma_f16(OA[1], a, bb[2], bb[3]);
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+          uint32_t bb[4];
+          ldsm_x4_t(bb, Ut + (16 * ks + lrow_a(lane)) * LDH + nb + 16 * np + lcol_a(lane));
+          mma_f16(OA[2 * np], a, bb[0], bb[1]);
+          mma_f16(OA[2 * np + 1], a, bb[2], bb[3]);
+        }
       }
       const float fo0 = sc[r0], fo1 = sc[r1];
       TO* o0 = o + (((size_t)b * T + t0 + r0) * Hv + hv) * kD + c0 + nb + 2 * t4;
       TO* o1 = o0 + (size_t)8 * Hv * kD;
       const bool w0 = t0 + r0 < T, w1 = t0 + r1 < T;
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
+      for (int nt = 0; nt < 4; ++nt) {
         if (w0)
           store2<TO>(o0 + 8 * nt, (fo0 * OQ[nt][0] + OA[nt][0]) * inv_sigma,
                      (fo0 * OQ[nt][1] + OA[nt][1]) * inv_sigma);
@@ -636,21 +644,21 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
       }
     }
 
-    // S <- gamma_C S + K^T U~s  (this warp's 16 x 32 block of the state slice)
+    // S <- gamma_C S + K^T U~s  (this warp's 16 state rows)
     {
       const float gC = sc[2 * kC];
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
+      for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) S[nt][i] *= gC;
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
         uint32_t a[4];
-        ldsm_x4_t(a, Kt + (16 * ks + lrow_b(lane)) * LDT + 16 * (warp & 7) + lcol_b(lane));
+        ldsm_x4_t(a, Kt + (16 * ks + lrow_b(lane)) * LDT + 16 * warp + lcol_b(lane));
 #pragma unroll
-        for (int np = 0; np < 2; ++np) {
+        for (int np = 0; np < 4; ++np) {
           uint32_t bb[4];
-          ldsm_x4_t(bb, Us + (16 * ks + lrow_a(lane)) * LDH + scb + 16 * np + lcol_a(lane));
+          ldsm_x4_t(bb, Us + (16 * ks + lrow_a(lane)) * LDH + 16 * np + lcol_a(lane));
           mma_f16(S[2 * np], a, bb[0], bb[1]);
           mma_f16(S[2 * np + 1], a, bb[2], bb[3]);
         }
@@ -662,8 +670,8 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
 
   if (ht != nullptr) {
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      float* dst = ht + ((size_t)head * kD + sr) * kD + c0 + scb + 8 * nt + 2 * t4;
+    for (int nt = 0; nt < 8; ++nt) {
+      float* dst = ht + ((size_t)head * kD + sr) * kD + c0 + 8 * nt + 2 * t4;
       *reinterpret_cast<float2*>(dst) = make_float2(S[nt][0] * inv_sigma, S[nt][1] * inv_sigma);
       *reinterpret_cast<float2*>(dst + 8 * kD) =
           make_float2(S[nt][2] * inv_sigma, S[nt][3] * inv_sigma);
