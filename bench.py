@@ -341,16 +341,19 @@ def measure_gdn2(G, dev, stream, pk, args):
     x = workload_inputs(w, dev)
     o = torch.empty((w.B, w.T, w.Hv, w.d), device=dev, dtype=w.dtype)
     ht = torch.empty((w.B, w.Hv, w.d, w.d), device=dev, dtype=torch.float32)
+    n_ws = G.gdn2_chunk_workspace_bytes(w.B, w.T, w.Hv, w.d, w.d, w.dtype)
+    ws = torch.empty(n_ws, device=dev, dtype=torch.uint8) if n_ws else None
 
     def step():
         G.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["a"], x["b_logit"], x["w_logit"],
-                         x["A_log"], x["dt_bias"], x["h0"], o=o, ht=ht, stream=stream)
+                         x["A_log"], x["dt_bias"], x["h0"], o=o, ht=ht, workspace=ws,
+                         stream=stream)
 
     total, per = time_steps(step, 5, 2, stream)
     ms = total / 5
     flop = CHUNK_FLOP_PER_TOKEN_HEAD * w.T * w.Hv * w.B
     ach = flop / (ms / 1e3) / 1e12
-    del x, o, ht
+    del x, o, ht, ws
     torch.cuda.empty_cache()
     return {"tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
             "achieved_tflops": round(ach, 2),

@@ -18,7 +18,7 @@ import os
 import torch
 
 __all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_chunk_workspace_bytes", "gdn_recurrent_step",
-           "gdn2_chunk_fwd", "gdn_chunk_fwd_noalloc",
+           "gdn2_chunk_fwd", "gdn2_chunk_workspace_bytes", "gdn_chunk_fwd_noalloc",
            "gdn_check_status", "GDNError", "LIB_PATH", "lib", "F32", "BF16",
            "QK_L2NORM", "GATES_PRECOMPUTED", "OUT_F32"]
 
@@ -193,11 +193,18 @@ def gdn_chunk_fwd_noalloc(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, s
     return o, ht
 
 
+def gdn2_chunk_workspace_bytes(B, T, H, dk, dv, dtype) -> int:
+    """Bytes of device workspace gdn2_chunk_fwd needs for these sizes (0 = none)."""
+    return int(lib.gdn2_chunk_workspace_bytes(B, T, H, dk, dv, _dtype_code(dtype)))
+
+
 def gdn2_chunk_fwd(q, k, v, a, b_logit, w_logit, A_log=None, dt_bias=None, h0=None, *,
                    scale=None, l2norm=True, gates_precomputed=False, out_f32=False, o=None,
-                   ht=None, want_ht=True, stream=None):
+                   ht=None, want_ht=True, workspace=None, stream=None):
     """Chunkwise Gated DeltaNet-2 forward. q, k, a, b_logit [B,T,H,dk]; v, w_logit
-    [B,T,H,dv]; A_log, dt_bias [H,dk] float32; h0 [B,H,dk,dv] or None."""
+    [B,T,H,dv]; A_log, dt_bias [H,dk] float32; h0 [B,H,dk,dv] or None.  With
+    gates_precomputed, a is the per-channel log-decay and b_logit / w_logit are
+    the gate values (float32).  workspace as for gdn_chunk_fwd."""
     B, T, H, dk = q.shape
     dv = v.shape[3]
     dt = q.dtype
@@ -217,9 +224,14 @@ def gdn2_chunk_fwd(q, k, v, a, b_logit, w_logit, A_log=None, dt_bias=None, h0=No
         ht = torch.empty((B, H, dk, dv), device=q.device, dtype=torch.float32)
     flags = ((QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
              | (OUT_F32 if out_f32 else 0))
+    ws_need = gdn2_chunk_workspace_bytes(B, T, H, dk, dv, dt)
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.gdn2_chunk_fwd(_p(q), _p(k), _p(v), _p(a), _p(b_logit), _p(w_logit), _p(A_log),
                               _p(dt_bias), _p(h0), B, T, H, dk, dv, _dtype_code(dt),
-                              float(scale), flags, _p(o), _p(ht), None, 0, _stream(stream)),
+                              float(scale), flags, _p(o), _p(ht), _p(workspace), ws_bytes,
+                              _stream(stream)),
            "gdn2_chunk_fwd")
     return o, ht
 

@@ -95,7 +95,9 @@ size_t gdn_chunk_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, i
   c.B = B; c.T = T; c.Hk = Hk; c.Hv = Hv; c.dk = dk; c.dv = dv; c.dtype = dtype;
   return chunk_mma_supported(c) ? chunk_mma_workspace_bytes(B, T, Hk, Hv) : 0;
 }
-size_t gdn2_chunk_workspace_bytes(int, int, int, int, int, int) { return 0; }
+size_t gdn2_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
+  return gdn_chunk_workspace_bytes(B, T, H, H, dk, dv, dtype);
+}
 
 static int validate_chunk(const ChunkArgs& c, bool gdn2) {
   if (c.B < 0 || c.T < 0 || c.Hk <= 0 || c.Hv <= 0 || !ok_dtype(c.dtype))
@@ -119,11 +121,11 @@ static int run_chunk(const ChunkArgs& c, bool gdn2, void* ws, size_t ws_bytes,
                      cudaStream_t s) {
   const size_t state_elems = (size_t)c.B * c.Hv * c.dk * c.dv;
   if (c.T == 0 || c.B == 0) return from_cuda(launch_copy_state(c.h0, c.ht, state_elems, s));
-  if (!gdn2 && chunk_mma_supported(c)) {
+  if (chunk_mma_supported(c)) {
     if (ws == nullptr || !aligned16(ws) ||
         ws_bytes < chunk_mma_workspace_bytes(c.B, c.T, c.Hk, c.Hv))
       return GDN_ERR_WORKSPACE;
-    return from_cuda(launch_chunk_mma(c, ws, s));
+    return from_cuda(launch_chunk_mma(c, gdn2, ws, s));
   }
   return from_cuda(launch_chunk_simt(c, gdn2, s));
 }

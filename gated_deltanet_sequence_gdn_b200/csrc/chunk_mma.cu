@@ -51,7 +51,10 @@ constexpr int kD = 128;        // dk = dv
 constexpr int kThreads = 256;  // 8 warps
 constexpr int LDT = kD + 8;    // 16-bit row stride of 128-wide tiles (272 B: ldmatrix conflict-free)
 constexpr int LDH = 64 + 8;    // 16-bit row stride of 64-wide tiles (144 B)
-constexpr int kScal = 132;     // floats per (head, chunk): fo[64], fs[64], gamma_C, max|U|, pad
+constexpr int kScal = 260;     // floats per (head, chunk): fo[64], fs[64], gamma_C[128] (per state
+                               // row), max|U|, pad
+constexpr int kScGC = 2 * 64;  // offset of gamma_C in the scalar block
+constexpr int kScMaxU = kScGC + 128;
 constexpr float kF16Max = 65000.f;  // largest magnitude accepted for an fp16 operand
 
 // ---------------------------------------------------------------- workspace
@@ -67,7 +70,7 @@ WsLayout ws_layout(int B, int T, int Hk, int Hv) {
   L.a = L.u + hv * Tp * kD * 4;             // A_qk   [B*Hv][Tp][64]  f16
   L.qh = L.a + hv * Tp * kC * 2;            // Q rows [B*Hk][Tp][128] f16 (row-scaled)
   L.kh = L.qh + hk * Tp * kD * 2;           // K rows [B*Hk][Tp][128] f16 (row-scaled)
-  L.scal = L.kh + hk * Tp * kD * 2;         // scalars [B*Hv][Nc][132] f32
+  L.scal = L.kh + hk * Tp * kD * 2;         // scalars [B*Hv][Nc][260] f32
   L.total = L.scal + hv * Nc * kScal * 4;
   return L;
 }
@@ -123,6 +126,77 @@ constexpr int P_T = P_X + kC * LDX * 4;      // block products, one [16][LDB] f3
 constexpr int P_VEC = P_T + 3 * 16 * LDB * 4; // rk, sq, G, beta, c1, 2^eq, 2^ek [64], misc
 constexpr int P_BYTES = P_VEC + 8 * 64 * 4;
 static_assert(2 * (P_BYTES + 1024) <= 228 * 1024, "two prep CTAs per SM");
+
+// X = (I + L)^-1 for a strictly lower 64 x 64 fp32 L (row stride LDX) in shared
+// memory, by the whole CTA: the four 16 x 16 diagonal blocks by forward
+// substitution (thread = one column of one block), then block row by block row
+// on the tensor cores with the fp32 operands as bf16 hi + lo: warp j < i
+// computes T = sum_{k=j}^{i-1} L_ik X_kj and X_ij = -X_ii T.  Ends with a barrier.
+__device__ void invert_unit_lower(const float* Lm, float* Xm, float* Tm, int tid, int warp, int g8,
+                                  int t4) {
+  if (tid < kC) {
+    const int base = 16 * (tid >> 4), cc = tid & 15;
+    float x[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float s = 0.f;
+#pragma unroll
+      for (int jj = 0; jj < r; ++jj) s = fmaf(Lm[(base + r) * LDX + base + jj], x[jj], s);
+      x[r] = r == cc ? 1.f : -s;  // rows above cc come out as zero
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) Xm[(base + r) * LDX + base + cc] = x[r];
+  } else {
+    for (int i = tid - kC; i < 6 * 256; i += kThreads - kC) {
+      const int blk = i >> 8, e = i & 255;  // blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+      const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+      const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+      Xm[(16 * bi + (e >> 4)) * LDX + 16 * bj + (e & 15)] = 0.f;
+    }
+  }
+  __syncthreads();
+  for (int bi = 1; bi < 4; ++bi) {
+    if (warp < bi) {
+      const int bj = warp;
+      float* Tw = Tm + warp * 16 * LDB;
+      float t[2][4] = {};
+      for (int kb = bj; kb < bi; ++kb) {
+        uint32_t ah[4], al[4];
+        frag_a_split(Lm, LDX, 16 * bi, 16 * kb, g8, t4, ah, al);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          uint32_t bh[2], bl[2];
+          frag_b_split(Xm, LDX, 16 * kb, 16 * bj + 8 * nt, g8, t4, bh, bl);
+          mma_split3(t[nt], ah, al, bh, bl);
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        *reinterpret_cast<float2*>(Tw + g8 * LDB + 8 * nt + 2 * t4) = make_float2(t[nt][0], t[nt][1]);
+        *reinterpret_cast<float2*>(Tw + (g8 + 8) * LDB + 8 * nt + 2 * t4) =
+            make_float2(t[nt][2], t[nt][3]);
+      }
+      __syncwarp();
+      float x[2][4] = {};
+      uint32_t ah[4], al[4];
+      frag_a_split(Xm, LDX, 16 * bi, 16 * bi, g8, t4, ah, al);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t bh[2], bl[2];
+        frag_b_split(Tw, LDB, 0, 8 * nt, g8, t4, bh, bl);
+        mma_split3(x[nt], ah, al, bh, bl);
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int c = 16 * bj + 8 * nt + 2 * t4;
+        *reinterpret_cast<float2*>(Xm + (16 * bi + g8) * LDX + c) = make_float2(-x[nt][0], -x[nt][1]);
+        *reinterpret_cast<float2*>(Xm + (16 * bi + g8 + 8) * LDX + c) =
+            make_float2(-x[nt][2], -x[nt][3]);
+      }
+    }
+    __syncthreads();
+  }
+}
 
 template <bool PRE>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -297,73 +371,8 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
   }
   __syncthreads();
 
-  // 4. X = (I + L)^-1: the four 16 x 16 diagonal blocks by forward substitution
-  //    (thread = one column of one block), zeros above the diagonal blocks
-  if (tid < kC) {
-    const int base = 16 * (tid >> 4), cc = tid & 15;
-    float x[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float s = 0.f;
-#pragma unroll
-      for (int jj = 0; jj < r; ++jj) s = fmaf(Lm[(base + r) * LDX + base + jj], x[jj], s);
-      x[r] = r == cc ? 1.f : -s;  // rows above cc come out as zero
-    }
-#pragma unroll
-    for (int r = 0; r < 16; ++r) Xm[(base + r) * LDX + base + cc] = x[r];
-  } else {
-    for (int i = tid - kC; i < 6 * 256; i += kThreads - kC) {
-      const int blk = i >> 8, e = i & 255;  // blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
-      const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-      const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-      Xm[(16 * bi + (e >> 4)) * LDX + 16 * bj + (e & 15)] = 0.f;
-    }
-  }
-  __syncthreads();
-  //    then block row by block row, on the tensor cores (fp32 operands as bf16
-  //    hi + lo): warp j < i computes T = sum_{k=j}^{i-1} L_ik X_kj and
-  //    X_ij = -X_ii T for its block (j = warp)
-  for (int bi = 1; bi < 4; ++bi) {
-    if (warp < bi) {
-      const int bj = warp;
-      float* Tw = Tm + warp * 16 * LDB;
-      float t[2][4] = {};
-      for (int kb = bj; kb < bi; ++kb) {
-        uint32_t ah[4], al[4];
-        frag_a_split(Lm, LDX, 16 * bi, 16 * kb, g8, t4, ah, al);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          uint32_t bh[2], bl[2];
-          frag_b_split(Xm, LDX, 16 * kb, 16 * bj + 8 * nt, g8, t4, bh, bl);
-          mma_split3(t[nt], ah, al, bh, bl);
-        }
-      }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        *reinterpret_cast<float2*>(Tw + g8 * LDB + 8 * nt + 2 * t4) = make_float2(t[nt][0], t[nt][1]);
-        *reinterpret_cast<float2*>(Tw + (g8 + 8) * LDB + 8 * nt + 2 * t4) =
-            make_float2(t[nt][2], t[nt][3]);
-      }
-      __syncwarp();
-      float x[2][4] = {};
-      uint32_t ah[4], al[4];
-      frag_a_split(Xm, LDX, 16 * bi, 16 * bi, g8, t4, ah, al);
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        uint32_t bh[2], bl[2];
-        frag_b_split(Tw, LDB, 0, 8 * nt, g8, t4, bh, bl);
-        mma_split3(x[nt], ah, al, bh, bl);
-      }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int c = 16 * bj + 8 * nt + 2 * t4;
-        *reinterpret_cast<float2*>(Xm + (16 * bi + g8) * LDX + c) = make_float2(-x[nt][0], -x[nt][1]);
-        *reinterpret_cast<float2*>(Xm + (16 * bi + g8 + 8) * LDX + c) =
-            make_float2(-x[nt][2], -x[nt][3]);
-      }
-    }
-    __syncthreads();
-  }
+  // 4. X = (I + L)^-1
+  invert_unit_lower(Lm, Xm, Tm, tid, warp, g8, t4);
 
   // 5. W = X diag(c1) K (stored in fp16) and U = X diag(beta) V (fp32, X diag(beta)
   //    as bf16 hi + lo); the A fragments are formed from X in registers.
@@ -432,17 +441,378 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
   __syncthreads();
 
   // 6. per-row factors of the scan: fo = gamma sq 2^eq, fs = rk 2^ek gamma_C / gamma,
-  //    gamma_C, and the largest |U| of the chunk
-  if (tid < kC) {
+  //    gamma_C for every state row, and the largest |U| of the chunk
+  if (tid < 128) {
     float* sc = reinterpret_cast<float*>(ws + L.scal) + (head * Nc + n) * kScal;
     const float GC = Gs[kC - 1];
-    sc[tid] = __expf(Gs[tid]) * sq[tid] * pq[tid];
-    sc[kC + tid] = tid < nv ? rk[tid] * pk[tid] * __expf(GC - Gs[tid]) : 0.f;
+    if (tid < kC) {
+      sc[tid] = __expf(Gs[tid]) * sq[tid] * pq[tid];
+      sc[kC + tid] = tid < nv ? rk[tid] * pk[tid] * __expf(GC - Gs[tid]) : 0.f;
+    }
+    sc[kScGC + tid] = __expf(GC);  // one decay for every state row
     if (tid < 4) {
       float m = 0.f;
 #pragma unroll
       for (int w = 0; w < 8; ++w) m = fmaxf(m, misc[8 + w]);
-      sc[2 * kC + tid] = tid == 0 ? __expf(GC) : (tid == 1 ? m : 0.f);
+      sc[kScMaxU + tid] = tid == 0 ? m : 0.f;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- GDN-2 prep kernel
+// Gated DeltaNet-2: per-channel decay d_t = exp(g_t) (g_t in R^dk), erase
+// direction e_t = b_t (.) k^_t, written value z_t = w_t (.) v_t.  With G the
+// in-chunk prefix sum of g (per channel) the chunk form is
+//   L_ji   = sum_c e_jc k^_ic exp(G_jc - G_ic)       (i < j)
+//   A_tj   = sum_c q^_tc k^_jc exp(G_tc - G_jc)      (j <= t)
+//   X = (I + L)^-1,  W = X (exp(G) (.) E),  U = X Z
+//   o = (exp(G) (.) Q^) S + A (U - W S),   S <- diag(exp(G_C)) S + K_tail^T (U - W S)
+// with K_tail rows exp(G_C - G_j) (.) k^_j ("Gated DeltaNet-2", 通道级衰减的吸收技巧
+// and WY 形式).  The exponents differ per channel, so the 16 x 16 diagonal blocks
+// of L and A are summed element by element, and each off-diagonal block row I is
+// a product of operands scaled about its first row r = 16 I:
+//   L_ji = sum_c [e_jc exp(G_jc - G_rc)] [k^_ic exp(G_rc - G_ic)]   (i < r <= j)
+// where both exponents are <= 0, so every operand stays within its input's size.
+constexpr int LDG = kD + 4;                    // f32 row stride of [64][128] channel tiles
+constexpr int Q2_KT = 0;                       // raw K tile [64][LDT] bf16
+constexpr int Q2_QT = Q2_KT + kC * LDT * 2;    // raw Q tile
+constexpr int Q2_ZH = Q2_QT + kC * LDT * 2;    // raw V tile, then z = w (.) v (bf16 hi part)
+constexpr int Q2_ZL = Q2_ZH + kC * LDT * 2;    // z lo part
+constexpr int Q2_G = Q2_ZL + kC * LDT * 2;     // G [64][LDG] f32 (first: g, or the raw g tile)
+constexpr int Q2_E = Q2_G + kC * LDG * 4;      // e [64][LDG] f32 (first: the raw b tile)
+constexpr int Q2_L = Q2_E + kC * LDG * 4;      // L [64][LDX] f32
+constexpr int Q2_X = Q2_L + kC * LDX * 4;      // A staging (f32), then X
+constexpr int Q2_T = Q2_X + kC * LDX * 4;      // block products
+constexpr int Q2_OP = Q2_T + 3 * 16 * LDB * 4; // raw gate tiles, then fp16 operands, then E-bar
+constexpr int Q2_OPB = 192 * LDT * 2;
+constexpr int Q2_VEC = Q2_OP + Q2_OPB;         // rk, sq [64], carry [128], misc [64]
+constexpr int Q2_BYTES = Q2_VEC + 320 * 4;
+static_assert(Q2_BYTES <= 227 * 1024, "shared memory of the GDN-2 prep kernel");
+static_assert(kC * LDG * 4 <= Q2_OPB, "raw float32 w tile fits the operand scratch");
+
+template <bool PRE>
+__global__ void __launch_bounds__(kThreads, 1)
+wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
+                const void* __restrict__ ga, const void* __restrict__ gb,
+                const void* __restrict__ gw, const float* __restrict__ A_log,
+                const float* __restrict__ dt_bias, int T, int H, float scale, int l2,
+                uint8_t* __restrict__ ws, WsLayout L, int* status) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  bf16* Kt = reinterpret_cast<bf16*>(sm + Q2_KT);
+  bf16* Qt = reinterpret_cast<bf16*>(sm + Q2_QT);
+  bf16* Zh = reinterpret_cast<bf16*>(sm + Q2_ZH);
+  bf16* Zl = reinterpret_cast<bf16*>(sm + Q2_ZL);
+  float* Gm = reinterpret_cast<float*>(sm + Q2_G);
+  float* Em = reinterpret_cast<float*>(sm + Q2_E);
+  float* Lm = reinterpret_cast<float*>(sm + Q2_L);
+  float* Xm = reinterpret_cast<float*>(sm + Q2_X);
+  float* Tm = reinterpret_cast<float*>(sm + Q2_T);
+  uint8_t* op = sm + Q2_OP;
+  float* rk = reinterpret_cast<float*>(sm + Q2_VEC);
+  float* sq = rk + 64;
+  float* carry = sq + 64;
+  float* misc = carry + 128;  // [8..15] per-warp max |U|
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g8 = lane >> 2, t4 = lane & 3;
+  const int n = blockIdx.y, Nc = gridDim.y, Tp = Nc * kC;
+  const int b = blockIdx.z / H, h = blockIdx.z % H;
+  const size_t head = blockIdx.z;  // one key head per value head
+  const int t0 = n * kC, nv = min(kC, T - t0);
+  float range = 0.f;
+
+  // 1. raw q, k, v tiles and the gate tiles (rows past the end of the sequence are zeros)
+  for (int i = tid; i < 3 * kC * 16; i += kThreads) {
+    const int which = i >> 10, r = (i >> 4) & 63, c16 = i & 15;
+    const bool ok = r < nv;
+    const size_t off = ok ? ((((size_t)b * T + t0 + r) * H + h) * kD + c16 * 8) : 0;
+    bf16* dst = (which == 0 ? Kt : (which == 1 ? Qt : Zh)) + r * LDT + c16 * 8;
+    cp16(dst, (which == 0 ? k : (which == 1 ? q : v)) + off, ok ? 16 : 0);
+    if (!PRE) {  // a, b, w logits in bf16
+      const bf16* src = reinterpret_cast<const bf16*>(which == 0 ? ga : (which == 1 ? gb : gw));
+      cp16(reinterpret_cast<bf16*>(op + which * kC * LDT * 2) + r * LDT + c16 * 8, src + off,
+           ok ? 16 : 0);
+    }
+  }
+  if (PRE) {  // g, b, w values in float32
+    for (int i = tid; i < 3 * kC * 32; i += kThreads) {
+      const int which = i / (kC * 32), r = (i >> 5) & 63, c32 = i & 31;
+      const bool ok = r < nv;
+      const size_t off = ok ? ((((size_t)b * T + t0 + r) * H + h) * kD + c32 * 4) : 0;
+      const float* src = reinterpret_cast<const float*>(which == 0 ? ga : (which == 1 ? gb : gw));
+      float* dst = (which == 0 ? Gm : (which == 1 ? Em : reinterpret_cast<float*>(op))) + r * LDG;
+      cp16(dst + c32 * 4, src + off, ok ? 16 : 0);
+    }
+  }
+  cp_commit();
+  for (int i = tid; i < kC * LDX; i += kThreads) Xm[i] = 0.f;  // A staging starts at zero
+  cp_wait<0>();
+  __syncthreads();
+
+  // 2. L2 norms: rk = 1 / |k|, sq = scale / |q| (two threads per row)
+  {
+    const int which = tid >> 7, r = (tid & 127) >> 1, hh = tid & 1;
+    const bf16* row = (which ? Qt : Kt) + r * LDT + hh * 8;
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < 128; c += 16) {
+      const uint4 u = *reinterpret_cast<const uint4*>(row + c);
+      const float2 f0 = unpack2(u.x), f1 = unpack2(u.y), f2 = unpack2(u.z), f3 = unpack2(u.w);
+      ss += f0.x * f0.x + f0.y * f0.y + f1.x * f1.x + f1.y * f1.y + f2.x * f2.x + f2.y * f2.y +
+            f3.x * f3.x + f3.y * f3.y;
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    if (hh == 0) {
+      const float inv = l2 ? rsqrtf(ss + 1e-6f) : 1.f;
+      if (which) sq[r] = inv * scale;
+      else rk[r] = inv;
+    }
+  }
+  __syncthreads();
+
+  // 3. per (token, channel): g, the in-chunk prefix sums G (two threads per channel,
+  //    32 tokens each), e = b (.) k^ and z = w (.) v (as bf16 hi + lo)
+  const int ch = tid & 127, half = tid >> 7;
+  {
+    float nal = 0.f, dtb = 0.f;
+    if (!PRE) {
+      nal = -expf(A_log[(size_t)h * kD + ch]);
+      dtb = dt_bias[(size_t)h * kD + ch];
+    }
+    const bf16* at = reinterpret_cast<const bf16*>(op);
+    const bf16* bt = at + kC * LDT;
+    const bf16* wt = bt + kC * LDT;
+    const float* wf = reinterpret_cast<const float*>(op);
+    float run = 0.f;
+    for (int tt = 0; tt < 32; ++tt) {
+      const int r = 32 * half + tt;
+      float g, bv, wv;
+      if (PRE) {
+        g = Gm[r * LDG + ch];
+        bv = Em[r * LDG + ch];
+        wv = wf[r * LDG + ch];
+      } else {
+        g = r < nv ? nal * softplus_f(__bfloat162float(at[r * LDT + ch]) + dtb) : 0.f;
+        bv = sigmoid_f(__bfloat162float(bt[r * LDT + ch]));
+        wv = sigmoid_f(__bfloat162float(wt[r * LDT + ch]));
+      }
+      run += g;
+      Gm[r * LDG + ch] = run;
+      Em[r * LDG + ch] = bv * __bfloat162float(Kt[r * LDT + ch]) * rk[r];
+      const float z = wv * __bfloat162float(Zh[r * LDT + ch]);
+      const bf16 zh = __float2bfloat16_rn(z);
+      Zh[r * LDT + ch] = zh;
+      Zl[r * LDT + ch] = __float2bfloat16_rn(z - __bfloat162float(zh));
+    }
+    if (half == 0) carry[ch] = run;
+  }
+  __syncthreads();
+  if (half == 1)
+    for (int r = 32; r < kC; ++r) Gm[r * LDG + ch] += carry[ch];
+  __syncthreads();
+
+  // 4. diagonal 16 x 16 blocks of L and A, element by element: warp per (j, i)
+  //    pair, lanes over channels (4 each); exp(G_j - G_i) <= 1 for i <= j
+  for (int p = warp; p < 4 * 136; p += 8) {
+    const int blk = p / 136;
+    int rem = p - blk * 136, jj = 0;
+    while (rem > jj) {
+      rem -= jj + 1;
+      ++jj;
+    }
+    const int j = 16 * blk + jj, i = 16 * blk + rem;  // i <= j
+    const float4 gj = *reinterpret_cast<const float4*>(Gm + j * LDG + 4 * lane);
+    const float4 gi = *reinterpret_cast<const float4*>(Gm + i * LDG + 4 * lane);
+    const float4 ej = *reinterpret_cast<const float4*>(Em + j * LDG + 4 * lane);
+    const uint2 qj = *reinterpret_cast<const uint2*>(Qt + j * LDT + 4 * lane);
+    const uint2 ki = *reinterpret_cast<const uint2*>(Kt + i * LDT + 4 * lane);
+    const float2 q01 = unpack2(qj.x), q23 = unpack2(qj.y);
+    const float2 k01 = unpack2(ki.x), k23 = unpack2(ki.y);
+    const float x0 = __expf(gj.x - gi.x) * k01.x, x1 = __expf(gj.y - gi.y) * k01.y;
+    const float x2 = __expf(gj.z - gi.z) * k23.x, x3 = __expf(gj.w - gi.w) * k23.y;
+    float sl = ej.x * x0 + ej.y * x1 + ej.z * x2 + ej.w * x3;
+    float sa = q01.x * x0 + q01.y * x1 + q23.x * x2 + q23.y * x3;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sl += __shfl_xor_sync(0xffffffffu, sl, o);
+      sa += __shfl_xor_sync(0xffffffffu, sa, o);
+    }
+    if (lane == 0) {
+      Lm[j * LDX + i] = i < j ? sl * rk[i] : 0.f;
+      Xm[j * LDX + i] = sa * sq[j] * rk[i];
+    }
+  }
+
+  // 5. off-diagonal blocks on the tensor cores: fp16 operands scaled about the
+  //    reference row r = 16 I of block row I (I = 1..3).  Rows of the operand
+  //    scratch: [0,48) e rows of blocks 1-3, [48,96) q^ rows, [96,192) k^ rows
+  //    0..16 I - 1 for I = 1, 2, 3 (at 96, 112, 144).
+  __half* Op = reinterpret_cast<__half*>(op);
+  for (int e = tid; e < 192 * kD; e += kThreads) {
+    const int row = e >> 7, c = e & 127;
+    float val;
+    if (row < 96) {
+      const int I = 1 + ((row % 48) >> 4), j = 16 * I + (row & 15);
+      const float sc = __expf(Gm[j * LDG + c] - Gm[16 * I * LDG + c]);
+      val = row < 48 ? Em[j * LDG + c] * sc : __bfloat162float(Qt[j * LDT + c]) * sq[j] * sc;
+    } else {
+      const int kr = row - 96;
+      const int I = kr < 16 ? 1 : (kr < 48 ? 2 : 3);
+      const int i = kr - (I == 1 ? 0 : (I == 2 ? 16 : 48));
+      val = __bfloat162float(Kt[i * LDT + c]) * rk[i] *
+            __expf(Gm[16 * I * LDG + c] - Gm[i * LDG + c]);
+    }
+    Op[row * LDT + c] = __float2half_rn(val);
+  }
+  __syncthreads();
+  //    tasks (matrix, I, column pair np < I): 6 for L, 6 for A
+  for (int task = warp; task < 12; task += 8) {
+    const bool isa = task >= 6;
+    const int tk = isa ? task - 6 : task;
+    const int I = tk < 1 ? 1 : (tk < 3 ? 2 : 3);
+    const int np = tk - (I == 1 ? 0 : (I == 2 ? 1 : 3));
+    const __half* Arows = Op + ((isa ? 48 : 0) + 16 * (I - 1)) * LDT;
+    const __half* Brows = Op + (96 + (I == 1 ? 0 : (I == 2 ? 16 : 48))) * LDT;
+    float acc[2][4] = {};
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t a[4], bb[4];
+      ldsm_x4(a, Arows + lrow_a(lane) * LDT + 16 * ks + lcol_a(lane));
+      ldsm_x4(bb, Brows + (16 * np + lrow_b(lane)) * LDT + 16 * ks + lcol_b(lane));
+      mma_f16(acc[0], a, bb[0], bb[1]);
+      mma_f16(acc[1], a, bb[2], bb[3]);
+    }
+    float* dst = isa ? Xm : Lm;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int r = 16 * I + g8, c = 16 * np + 8 * nt + 2 * t4;
+      *reinterpret_cast<float2*>(dst + r * LDX + c) = make_float2(acc[nt][0], acc[nt][1]);
+      *reinterpret_cast<float2*>(dst + (r + 8) * LDX + c) = make_float2(acc[nt][2], acc[nt][3]);
+    }
+  }
+  __syncthreads();
+  //    A to the workspace (fp16, zeros above the diagonal)
+  {
+    __half* ag = reinterpret_cast<__half*>(ws + L.a) + (head * Tp + t0) * kC;
+    for (int i = tid; i < kC * 8; i += kThreads) {
+      const int r = i >> 3, c8 = (i & 7) * 8;
+      uint4 o;
+      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c8 + 2 * u;
+        ow[u] = pack2h(c <= r ? Xm[r * LDX + c] : 0.f, c + 1 <= r ? Xm[r * LDX + c + 1] : 0.f);
+      }
+      *reinterpret_cast<uint4*>(ag + (size_t)r * kC + c8) = o;
+    }
+  }
+  __syncthreads();
+
+  // 6. X = (I + L)^-1
+  invert_unit_lower(Lm, Xm, Tm, tid, warp, g8, t4);
+
+  // 7. E-bar = exp(G) (.) e in bf16 (the B operand of W), in the operand scratch
+  bf16* Eb = reinterpret_cast<bf16*>(op);
+  for (int e = tid; e < kC * kD; e += kThreads) {
+    const int r = e >> 7, c = e & 127;
+    Eb[r * LDT + c] = __float2bfloat16_rn(__expf(Gm[r * LDG + c]) * Em[r * LDG + c]);
+  }
+  __syncthreads();
+
+  //    W = X E-bar (fp16 out) and U = X Z (fp32 out, X and Z both as hi + lo);
+  //    warp -> rows 16 (warp % 4), cols 64 (warp / 4)
+  const int mt = warp & 3, nb = 64 * (warp >> 2);
+  const int ra = 16 * mt + g8;
+  float umax = 0.f;
+#pragma unroll 1
+  for (int which = 0; which < 2; ++which) {
+    float acc[8][4] = {};
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t ah[4], al[4];
+      frag_a_split(Xm, LDX, 16 * mt, 16 * ks, g8, t4, ah, al);
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        const int bo = (16 * ks + lrow_a(lane)) * LDT + nb + 16 * np + lcol_a(lane);
+        uint32_t bh[4];
+        ldsm_x4_t(bh, (which ? Zh : Eb) + bo);
+        mma_bf16(acc[2 * np], ah, bh[0], bh[1]);
+        mma_bf16(acc[2 * np + 1], ah, bh[2], bh[3]);
+        if (which) {
+          uint32_t bl[4];
+          ldsm_x4_t(bl, Zl + bo);
+          mma_bf16(acc[2 * np], ah, bl[0], bl[1]);
+          mma_bf16(acc[2 * np + 1], ah, bl[2], bl[3]);
+          mma_bf16(acc[2 * np], al, bh[0], bh[1]);
+          mma_bf16(acc[2 * np + 1], al, bh[2], bh[3]);
+        }
+      }
+    }
+    if (which == 0) {
+      __half* dw = reinterpret_cast<__half*>(ws + L.w) + (head * Tp + t0) * kD;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const int c = nb + 8 * nt + 2 * t4;
+        range = fmaxf(range, fmaxf(fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][1])),
+                                   fmaxf(fabsf(acc[nt][2]), fabsf(acc[nt][3]))));
+        *reinterpret_cast<uint32_t*>(dw + (size_t)ra * kD + c) = pack2h(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<uint32_t*>(dw + (size_t)(ra + 8) * kD + c) =
+            pack2h(acc[nt][2], acc[nt][3]);
+      }
+    } else {
+      float* du = reinterpret_cast<float*>(ws + L.u) + (head * Tp + t0) * kD;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const int c = nb + 8 * nt + 2 * t4;
+        umax = fmaxf(umax, fmaxf(fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][1])),
+                                 fmaxf(fabsf(acc[nt][2]), fabsf(acc[nt][3]))));
+        *reinterpret_cast<float2*>(du + (size_t)ra * kD + c) = make_float2(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<float2*>(du + (size_t)(ra + 8) * kD + c) =
+            make_float2(acc[nt][2], acc[nt][3]);
+      }
+    }
+  }
+  if (!(range <= kF16Max)) report_range(status);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) umax = fmaxf(umax, __shfl_xor_sync(0xffffffffu, umax, o));
+  if (lane == 0) misc[8 + warp] = umax;
+
+  // 8. the scan's Q and K rows in fp16: exp(G) (.) q^ and exp(G_C - G) (.) k^ (both
+  //    at most their unit-norm inputs), and the per-chunk factors
+  {
+    __half* qd = reinterpret_cast<__half*>(ws + L.qh) + (head * Tp + t0) * kD;
+    __half* kd = reinterpret_cast<__half*>(ws + L.kh) + (head * Tp + t0) * kD;
+    for (int i = tid; i < kC * 16; i += kThreads) {
+      const int r = i >> 4, c8 = (i & 15) * 8;
+      uint4 oq, ok;
+      uint32_t* wq = reinterpret_cast<uint32_t*>(&oq);
+      uint32_t* wk = reinterpret_cast<uint32_t*>(&ok);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c8 + 2 * u;
+        const float2 qq = unpack2(*reinterpret_cast<const uint32_t*>(Qt + r * LDT + c));
+        const float2 kk = unpack2(*reinterpret_cast<const uint32_t*>(Kt + r * LDT + c));
+        wq[u] = pack2h(qq.x * sq[r] * __expf(Gm[r * LDG + c]), qq.y * sq[r] * __expf(Gm[r * LDG + c + 1]));
+        wk[u] = pack2h(kk.x * rk[r] * __expf(Gm[(kC - 1) * LDG + c] - Gm[r * LDG + c]),
+                       kk.y * rk[r] * __expf(Gm[(kC - 1) * LDG + c + 1] - Gm[r * LDG + c + 1]));
+      }
+      *reinterpret_cast<uint4*>(qd + (size_t)r * kD + c8) = oq;
+      *reinterpret_cast<uint4*>(kd + (size_t)r * kD + c8) = ok;
+    }
+  }
+  __syncthreads();
+  if (tid < 128) {
+    float* sc = reinterpret_cast<float*>(ws + L.scal) + (head * Nc + n) * kScal;
+    if (tid < kC) {
+      sc[tid] = 1.f;
+      sc[kC + tid] = tid < nv ? 1.f : 0.f;
+    }
+    sc[kScGC + tid] = __expf(Gm[(kC - 1) * LDG + tid]);
+    if (tid < 4) {
+      float m = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) m = fmaxf(m, misc[8 + w]);
+      sc[kScMaxU + tid] = tid == 0 ? m : 0.f;
     }
   }
 }
@@ -534,7 +904,7 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
     mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x0.x), fabsf(x0.y)), fmaxf(fabsf(x1.x), fabsf(x1.y))));
   }
   // sigma = 2^-e: the largest |U| of the head and |h0| of this slice land below 2^8
-  for (int n = tid; n < Nc; n += kScanThreads) mx = fmaxf(mx, Sg[(size_t)n * kScal + 2 * kC + 1]);
+  for (int n = tid; n < Nc; n += kScanThreads) mx = fmaxf(mx, Sg[(size_t)n * kScal + kScMaxU]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   if (lane == 0) red[warp] = mx;
@@ -644,13 +1014,13 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
       }
     }
 
-    // S <- gamma_C S + K^T U~s  (this warp's 16 state rows)
+    // S <- diag(gamma_C) S + K^T U~s  (this warp's 16 state rows)
     {
-      const float gC = sc[2 * kC];
+      const float gA = sc[kScGC + sr], gB = sc[kScGC + sr + 8];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) S[nt][i] *= gC;
+      for (int nt = 0; nt < 8; ++nt) {
+        S[nt][0] *= gA; S[nt][1] *= gA; S[nt][2] *= gB; S[nt][3] *= gB;
+      }
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
         uint32_t a[4];
@@ -680,22 +1050,35 @@ state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, i
 }
 
 template <typename TO>
-cudaError_t launch_t(const ChunkArgs& a, uint8_t* ws, const WsLayout& L, cudaStream_t s) {
+cudaError_t launch_t(const ChunkArgs& a, bool gdn2, uint8_t* ws, const WsLayout& L,
+                     cudaStream_t s) {
   const int Nc = (a.T + kC - 1) / kC;
   const bool pre = (a.flags & GDN_GATES_PRECOMPUTED) != 0;
+  const int l2 = (a.flags & GDN_QK_L2NORM) ? 1 : 0;
   int* status = status_word();
   if (status == nullptr) return cudaErrorUnknown;
-  auto prep = pre ? wy_prep_kernel<true> : wy_prep_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_BYTES);
+  cudaError_t e;
+  if (gdn2) {
+    auto prep = pre ? wy_prep2_kernel<true> : wy_prep2_kernel<false>;
+    e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, Q2_BYTES);
+    if (e != cudaSuccess) return e;
+    prep<<<dim3(1, Nc, a.B * a.Hv), kThreads, Q2_BYTES, s>>>(
+        static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
+        static_cast<const bf16*>(a.v), a.a, a.b, a.w, a.A_log, a.dt_bias, a.T, a.Hv, a.scale, l2,
+        ws, L, status);
+  } else {
+    auto prep = pre ? wy_prep_kernel<true> : wy_prep_kernel<false>;
+    e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_BYTES);
+    if (e != cudaSuccess) return e;
+    prep<<<dim3(a.Hv / a.Hk, Nc, a.B * a.Hk), kThreads, P_BYTES, s>>>(
+        static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
+        static_cast<const bf16*>(a.v), a.a, a.b, a.A_log, a.dt_bias, a.T, a.Hk, a.Hv, a.scale, l2,
+        ws, L, status);
+  }
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(state_scan_kernel<TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            S_BYTES);
-  if (e != cudaSuccess) return e;
-  prep<<<dim3(a.Hv / a.Hk, Nc, a.B * a.Hk), kThreads, P_BYTES, s>>>(
-      static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
-      static_cast<const bf16*>(a.v), a.a, a.b, a.A_log, a.dt_bias, a.T, a.Hk, a.Hv, a.scale,
-      (a.flags & GDN_QK_L2NORM) ? 1 : 0, ws, L, status);
-  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   state_scan_kernel<TO><<<dim3(2, a.B * a.Hv), kScanThreads, S_BYTES, s>>>(
       ws, L, a.h0, a.T, a.Hk, a.Hv, static_cast<TO*>(a.o), a.ht, status);
@@ -714,11 +1097,11 @@ size_t chunk_mma_workspace_bytes(int B, int T, int Hk, int Hv) {
   return ws_layout(B, T, Hk, Hv).total;
 }
 
-cudaError_t launch_chunk_mma(const ChunkArgs& a, void* ws, cudaStream_t s) {
+cudaError_t launch_chunk_mma(const ChunkArgs& a, bool gdn2, void* ws, cudaStream_t s) {
   const WsLayout L = ws_layout(a.B, a.T, a.Hk, a.Hv);
   uint8_t* w = static_cast<uint8_t*>(ws);
-  if (a.flags & GDN_OUT_F32) return launch_t<float>(a, w, L, s);
-  return launch_t<bf16>(a, w, L, s);
+  if (a.flags & GDN_OUT_F32) return launch_t<float>(a, gdn2, w, L, s);
+  return launch_t<bf16>(a, gdn2, w, L, s);
 }
 
 }  // namespace gdn

@@ -31,11 +31,12 @@ cudaError_t launch_recurrent_step(const void* x, const float* conv_w, void* conv
 // float32 CUDA-core chunk path (GDN and, with gdn2 = true, Gated DeltaNet-2).
 cudaError_t launch_chunk_simt(const ChunkArgs& a, bool gdn2, cudaStream_t s);
 
-// bf16 tensor-core chunk path (GDN, dk = dv = 128): WY prep + state scan,
-// with its intermediates in a caller-provided workspace.
+// bf16 tensor-core chunk path (GDN and, with gdn2 = true, Gated DeltaNet-2;
+// dk = dv = 128): WY prep + state scan, with its intermediates in a
+// caller-provided workspace.
 bool chunk_mma_supported(const ChunkArgs& a);
 size_t chunk_mma_workspace_bytes(int B, int T, int Hk, int Hv);
-cudaError_t launch_chunk_mma(const ChunkArgs& a, void* workspace, cudaStream_t s);
+cudaError_t launch_chunk_mma(const ChunkArgs& a, bool gdn2, void* workspace, cudaStream_t s);
 
 // Device address of this device's status word (set up once per device).
 int* status_word();

@@ -130,11 +130,12 @@ int gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
                   void* workspace, size_t ws_bytes, gdn_stream_t stream);
 
 /* Workspace bytes gdn_chunk_fwd needs for these sizes: for the tensor-core
- * path (bf16, dk = dv = 128) B*Hv*(Tp*896 + (Tp/64)*528) + B*Hk*Tp*512 with
+ * path (bf16, dk = dv = 128) B*Hv*(Tp*896 + (Tp/64)*1040) + B*Hk*Tp*512 with
  * Tp = T rounded up to a multiple of 64 (per padded token and value head: a W
  * row of 128 fp16, a U row of 128 float32 and an A_qk row of 64 fp16; per
- * padded token and key head: fp16 copies of the q and k rows; 528 B of factors
- * per chunk and value head); 0 for every other case and for B*T = 0. */
+ * padded token and key head: fp16 copies of the scan's q and k rows; 1040 B of
+ * per-row factors per chunk and value head); 0 for every other case and for
+ * B*T = 0.  gdn2_chunk_workspace_bytes is the same with Hk = Hv = H. */
 size_t gdn_chunk_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv,
                                  int dtype);
 
@@ -195,6 +196,9 @@ int gdn_recurrent_step(const void* x_qkv, const float* conv_w, void* conv_state,
  *   A_log, dt_bias [H,dk] float32 (unused with GDN_GATES_PRECOMPUTED)
  *   h0, ht [B,H,dk,dv] float32 (NULL allowed; ht may alias h0)
  *   o [B,T,H,dv] dtype (float32 with GDN_OUT_F32), written
+ *   workspace / ws_bytes: as for gdn_chunk_fwd, sized by
+ *     gdn2_chunk_workspace_bytes (bf16 with dk = dv = 128 runs on the tensor
+ *     cores and needs it; other cases run a float32 CUDA-core path without).
  */
 int gdn2_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
                    const void* b_logit, const void* w_logit, const float* A_log,

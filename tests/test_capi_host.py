@@ -55,24 +55,27 @@ def test_status_strings_and_version():
 def test_workspace_sizes():
     """Tensor-core path (bf16, d = 128): per padded token and value head an fp16
     W row (256 B), a float32 U row (512 B) and an fp16 A_qk row (128 B); per
-    padded token and key head fp16 q and k rows (512 B); 528 B of factors per
+    padded token and key head fp16 q and k rows (512 B); 1040 B of factors per
     chunk and value head."""
     ws = G.lib.gdn_chunk_workspace_bytes
-    assert ws(1, 8192, 16, 64, 128, 128, 1) == 64 * (8192 * 896 + 128 * 528) + 16 * 8192 * 512
-    assert ws(2, 100, 2, 4, 128, 128, 1) == 2 * 4 * (128 * 896 + 2 * 528) + 2 * 2 * 128 * 512
-    assert ws(1, 64, 1, 1, 128, 128, 1) == 64 * 896 + 528 + 64 * 512
+    assert ws(1, 8192, 16, 64, 128, 128, 1) == 64 * (8192 * 896 + 128 * 1040) + 16 * 8192 * 512
+    assert ws(2, 100, 2, 4, 128, 128, 1) == 2 * 4 * (128 * 896 + 2 * 1040) + 2 * 2 * 128 * 512
+    assert ws(1, 64, 1, 1, 128, 128, 1) == 64 * 896 + 1040 + 64 * 512
     # no workspace: float32, other head sizes, empty inputs, Gated DeltaNet-2
     assert ws(1, 8192, 16, 64, 128, 128, 0) == 0
     assert ws(1, 256, 2, 2, 64, 64, 1) == 0
     assert ws(0, 256, 2, 2, 128, 128, 1) == 0
     assert ws(1, 0, 2, 2, 128, 128, 1) == 0
-    assert G.lib.gdn2_chunk_workspace_bytes(4, 4096, 16, 128, 128, 1) == 0
+    # Gated DeltaNet-2 (bf16, d = 128): the same layout with one key head per head
+    assert G.lib.gdn2_chunk_workspace_bytes(4, 4096, 16, 128, 128, 1) == \
+        4 * 16 * (4096 * 896 + 64 * 1040) + 4 * 16 * 4096 * 512
+    assert G.lib.gdn2_chunk_workspace_bytes(4, 4096, 16, 128, 128, 0) == 0
 
 
 def test_missing_workspace_rejected():
     """A bf16 d = 128 call without (enough) workspace is refused before any launch."""
     assert _chunk() == -5
-    need = 4 * (896 * 64 + 528) + 2 * 64 * 512  # B=1, T=64, Hk=2, Hv=4
+    need = 4 * (896 * 64 + 1040) + 2 * 64 * 512  # B=1, T=64, Hk=2, Hv=4
     assert _chunk(ws=FAKE, ws_bytes=need - 1) == -5
     assert _chunk(ws=FAKE + 8, ws_bytes=1 << 20) == -5  # misaligned
     assert _chunk(ws=FAKE, ws_bytes=need, flags=9) == -1  # a bad flag is reported first

@@ -250,8 +250,9 @@ def _gpu_gdn2(x, **kw):
 
 @pytest.mark.parametrize("out_f32", [False, True])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("shape", [(1, 1, 1, 128), (1, 70, 2, 128), (2, 129, 2, 64),
-                                   (1, 256, 4, 128)])
+@pytest.mark.parametrize("shape", [(1, 1, 1, 128), (1, 63, 1, 128), (1, 70, 2, 128),
+                                   (2, 129, 2, 64), (1, 256, 4, 128), (3, 200, 2, 128),
+                                   (1, 1000, 1, 128)])
 def test_gdn2_shapes(shape, dtype, out_f32):
     B, T, H, d = shape
     if dtype == torch.float32 and out_f32:
@@ -261,6 +262,55 @@ def test_gdn2_shapes(shape, dtype, out_f32):
     ro, rht = _oracle_gdn2(x)
     assert rel_err(o, ro) <= TOL[dtype], rel_err(o, ro)
     assert rel_err(ht, rht) <= TOL[dtype], rel_err(ht, rht)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_gdn2_zero_and_in_place_state(dtype):
+    x = gdn2_inputs(1, 150, 2, 128, dtype, seed=41, device=DEV)
+    x0 = dict(x, h0=None)
+    o, ht = _gpu_gdn2(x0)
+    ro, rht = _oracle_gdn2(x0)
+    assert rel_err(o, ro) <= TOL[dtype] and rel_err(ht, rht) <= TOL[dtype]
+    h = x["h0"].clone()
+    o2, ht2 = _gpu_gdn2(dict(x, h0=h), ht=h)
+    ro2, rht2 = _oracle_gdn2(x)
+    assert ht2.data_ptr() == h.data_ptr()
+    assert rel_err(o2, ro2) <= TOL[dtype] and rel_err(h, rht2) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_gdn2_precomputed_gates_and_no_norm(dtype):
+    """GDN_GATES_PRECOMPUTED: a = per-channel log-decay, b / w = gate values (float32);
+    GDN_QK_L2NORM off with unit-norm q, k from the caller."""
+    x = gdn2_inputs(2, 140, 2, 128, dtype, seed=42, device=DEV)
+    q = torch.nn.functional.normalize(x["q"].float(), dim=-1).to(dtype)
+    k = torch.nn.functional.normalize(x["k"].float(), dim=-1).to(dtype)
+    a = cpu(x["a"]).double()
+    g = -torch.exp(cpu(x["A_log"]).double()) * torch.nn.functional.softplus(
+        a + cpu(x["dt_bias"]).double())
+    bg = torch.sigmoid(cpu(x["b_logit"]).double())
+    wg = torch.sigmoid(cpu(x["w_logit"]).double())
+    g32, b32, w32 = (t.float().to(DEV) for t in (g, bg, wg))
+    scale = 128 ** -0.5
+    o, ht = G.gdn2_chunk_fwd(q, k, x["v"], g32, b32, w32, None, None, x["h0"], scale=scale,
+                             l2norm=False, gates_precomputed=True)
+    ro, rht = O.gdn2_fwd(cpu(q), cpu(k), cpu(x["v"]), cpu(g32), cpu(b32), cpu(w32),
+                         h0=cpu(x["h0"]), scale=scale, l2norm=False, gates_given=True)
+    assert rel_err(o, ro) <= TOL[dtype] and rel_err(ht, rht) <= TOL[dtype]
+
+
+def test_gdn2_workspace_reuse_and_size_check():
+    shape = (2, 190, 2, 128)
+    need = G.gdn2_chunk_workspace_bytes(*shape, 128, torch.bfloat16)
+    assert need > 0
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=DEV)  # fp16 / f32 NaN patterns
+    for seed in (43, 44):
+        x = gdn2_inputs(*shape, torch.bfloat16, seed=seed, device=DEV)
+        o, ht = _gpu_gdn2(x, workspace=ws)
+        ro, rht = _oracle_gdn2(x)
+        assert rel_err(o, ro) <= 2e-2 and rel_err(ht, rht) <= 2e-2
+    with pytest.raises(G.GDNError):
+        _gpu_gdn2(x, workspace=ws[: need - 16])
 
 
 def test_gdn2_full_size_sampled_heads():
