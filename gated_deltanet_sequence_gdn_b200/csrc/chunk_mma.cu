@@ -11,11 +11,10 @@
 //      A_qk = tril(Q^ K^^T o Gamma) (diagonal included), written to the
 //      workspace with the per-row factors of the second kernel, together with
 //      fp16 copies of the raw Q and K tiles.
-//  state_scan_kernel : one CTA (8 warps) per (value head, 64-column half of
-//      d_v), sequential over the chunks with the fp32 state slice held in mma
-//      accumulator registers (16 x 64 per warp):  U~ = U - W S,  o = diag(gamma sq) Q S + A_qk U~,
-//      S <- gamma_C S + K^T diag(rk gamma_C / gamma) U~.  All tiles of the next
-//      chunk are fetched with cp.async while the current one is computed.
+//  the state scan (scan_tc.cu, tcgen05): one CTA per (value head, 64-column
+//      half of d_v), sequential over the chunks with the fp32 state held in
+//      registers:  U~ = U - W S,  o = diag(gamma sq) Q S + A_qk U~,
+//      S <- gamma_C S + K^T diag(rk gamma_C / gamma) U~.
 //
 // The algebra is the WY / UT chunk form of the delta rule ("Gated DeltaNet-2",
 // section on the chunkwise algorithm; GDN is its scalar-decay special case):
@@ -38,6 +37,7 @@
 // word (read by gdn_check_status); nothing is clamped silently.
 #include "common.cuh"
 #include "launch.h"
+#include "chunk_layout.cuh"
 #include "warp_mma.cuh"
 
 namespace gdn {
@@ -46,34 +46,9 @@ namespace {
 using namespace wm;
 using bf16 = __nv_bfloat16;
 
-constexpr int kC = 64;         // chunk length
-constexpr int kD = 128;        // dk = dv
 constexpr int kThreads = 256;  // 8 warps
 constexpr int LDT = kD + 8;    // 16-bit row stride of 128-wide tiles (272 B: ldmatrix conflict-free)
 constexpr int LDH = 64 + 8;    // 16-bit row stride of 64-wide tiles (144 B)
-constexpr int kScal = 260;     // floats per (head, chunk): fo[64], fs[64], gamma_C[128] (per state
-                               // row), max|U|, pad
-constexpr int kScGC = 2 * 64;  // offset of gamma_C in the scalar block
-constexpr int kScMaxU = kScGC + 128;
-constexpr float kF16Max = 65000.f;  // largest magnitude accepted for an fp16 operand
-
-// ---------------------------------------------------------------- workspace
-struct WsLayout {
-  size_t w, u, a, qh, kh, scal, total;
-};
-WsLayout ws_layout(int B, int T, int Hk, int Hv) {
-  const size_t Nc = ((size_t)T + kC - 1) / kC, Tp = Nc * kC;
-  const size_t hv = (size_t)B * Hv, hk = (size_t)B * Hk;
-  WsLayout L;
-  L.w = 0;                                  // W      [B*Hv][Tp][128] f16
-  L.u = L.w + hv * Tp * kD * 2;             // U      [B*Hv][Tp][128] f32
-  L.a = L.u + hv * Tp * kD * 4;             // A_qk   [B*Hv][Tp][64]  f16
-  L.qh = L.a + hv * Tp * kC * 2;            // Q rows [B*Hk][Tp][128] f16 (row-scaled)
-  L.kh = L.qh + hk * Tp * kD * 2;           // K rows [B*Hk][Tp][128] f16 (row-scaled)
-  L.scal = L.kh + hk * Tp * kD * 2;         // scalars [B*Hv][Nc][260] f32
-  L.total = L.scal + hv * Nc * kScal * 4;
-  return L;
-}
 
 // x = hi + lo with hi = rn_bf16(x), lo = rn_bf16(x - hi), for a pair of values.
 __device__ __forceinline__ void split2(float x, float y, uint32_t& hi, uint32_t& lo) {
@@ -460,6 +435,29 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
 }
 
 // ---------------------------------------------------------------- GDN-2 prep kernel
+// Gate arithmetic of the tensor-core GDN-2 path with the hardware exp2/log2
+// approximations (relative error ~1e-6, far below the bf16 path's budget):
+// softplus(x) = max(x, 0) + log(1 + e^-|x|), sigmoid(x) = 1 / (1 + e^-x).
+__device__ __forceinline__ float softplus_fast(float x) {
+  return fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x)));
+}
+__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+// (jj, ii) with ii <= jj < 16, in row order: the 136 lower pairs of a 16 x 16 block
+struct PairTable {
+  unsigned char jj[136], ii[136];
+};
+__constant__ PairTable c_pairs = {
+    {0,1,1,2,2,2,3,3,3,3,4,4,4,4,4,5,5,5,5,5,5,6,6,6,6,6,6,6,7,7,7,7,7,7,7,7,
+     8,8,8,8,8,8,8,8,8,9,9,9,9,9,9,9,9,9,9,10,10,10,10,10,10,10,10,10,10,10,
+     11,11,11,11,11,11,11,11,11,11,11,11,12,12,12,12,12,12,12,12,12,12,12,12,12,
+     13,13,13,13,13,13,13,13,13,13,13,13,13,13,14,14,14,14,14,14,14,14,14,14,14,
+     14,14,14,14,15,15,15,15,15,15,15,15,15,15,15,15,15,15,15,15},
+    {0,0,1,0,1,2,0,1,2,3,0,1,2,3,4,0,1,2,3,4,5,0,1,2,3,4,5,6,0,1,2,3,4,5,6,7,
+     0,1,2,3,4,5,6,7,8,0,1,2,3,4,5,6,7,8,9,0,1,2,3,4,5,6,7,8,9,10,
+     0,1,2,3,4,5,6,7,8,9,10,11,0,1,2,3,4,5,6,7,8,9,10,11,12,
+     0,1,2,3,4,5,6,7,8,9,10,11,12,13,0,1,2,3,4,5,6,7,8,9,10,
+     11,12,13,14,0,1,2,3,4,5,6,7,8,9,10,11,12,13,14,15}
+};
 // Gated DeltaNet-2: per-channel decay d_t = exp(g_t) (g_t in R^dk), erase
 // direction e_t = b_t (.) k^_t, written value z_t = w_t (.) v_t.  With G the
 // in-chunk prefix sum of g (per channel) the chunk form is
@@ -570,8 +568,9 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   }
   __syncthreads();
 
-  // 3. per (token, channel): g, the in-chunk prefix sums G (two threads per channel,
-  //    32 tokens each), e = b (.) k^ and z = w (.) v (as bf16 hi + lo)
+  // 3. per (token, channel): g, e = b (.) k^ and z = w (.) v (as bf16 hi + lo), all
+  //    independent; then the in-chunk prefix sums G down each channel (two threads
+  //    per channel, 32 tokens each)
   const int ch = tid & 127, half = tid >> 7;
   {
     float nal = 0.f, dtb = 0.f;
@@ -583,7 +582,7 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     const bf16* bt = at + kC * LDT;
     const bf16* wt = bt + kC * LDT;
     const float* wf = reinterpret_cast<const float*>(op);
-    float run = 0.f;
+#pragma unroll 8
     for (int tt = 0; tt < 32; ++tt) {
       const int r = 32 * half + tt;
       float g, bv, wv;
@@ -592,55 +591,64 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         bv = Em[r * LDG + ch];
         wv = wf[r * LDG + ch];
       } else {
-        g = r < nv ? nal * softplus_f(__bfloat162float(at[r * LDT + ch]) + dtb) : 0.f;
-        bv = sigmoid_f(__bfloat162float(bt[r * LDT + ch]));
-        wv = sigmoid_f(__bfloat162float(wt[r * LDT + ch]));
+        g = r < nv ? nal * softplus_fast(__bfloat162float(at[r * LDT + ch]) + dtb) : 0.f;
+        bv = sigmoid_fast(__bfloat162float(bt[r * LDT + ch]));
+        wv = sigmoid_fast(__bfloat162float(wt[r * LDT + ch]));
       }
-      run += g;
-      Gm[r * LDG + ch] = run;
+      Gm[r * LDG + ch] = g;
       Em[r * LDG + ch] = bv * __bfloat162float(Kt[r * LDT + ch]) * rk[r];
       const float z = wv * __bfloat162float(Zh[r * LDT + ch]);
       const bf16 zh = __float2bfloat16_rn(z);
       Zh[r * LDT + ch] = zh;
       Zl[r * LDT + ch] = __float2bfloat16_rn(z - __bfloat162float(zh));
     }
+    float run = 0.f;
+#pragma unroll 8
+    for (int tt = 0; tt < 32; ++tt) {
+      const int r = 32 * half + tt;
+      run += Gm[r * LDG + ch];
+      Gm[r * LDG + ch] = run;
+    }
     if (half == 0) carry[ch] = run;
   }
   __syncthreads();
-  if (half == 1)
-    for (int r = 32; r < kC; ++r) Gm[r * LDG + ch] += carry[ch];
+  if (half == 1) {
+    const float cy = carry[ch];
+#pragma unroll 8
+    for (int r = 32; r < kC; ++r) Gm[r * LDG + ch] += cy;
+  }
   __syncthreads();
 
-  // 4. diagonal 16 x 16 blocks of L and A, element by element: warp per (j, i)
-  //    pair, lanes over channels (4 each); exp(G_j - G_i) <= 1 for i <= j
-  for (int p = warp; p < 4 * 136; p += 8) {
-    const int blk = p / 136;
-    int rem = p - blk * 136, jj = 0;
-    while (rem > jj) {
-      rem -= jj + 1;
-      ++jj;
+  // 4. diagonal 16 x 16 blocks of L and A, element by element: one thread per
+  //    lower pair (j, i) of a block (544 pairs), summing over the 128 channels
+  //    (exp(G_j - G_i) <= 1 for i <= j)
+#pragma unroll 1
+  for (int p = tid; p < 4 * 136; p += kThreads) {
+    const int blk = p / 136, pi = p - blk * 136;
+    const int jj = c_pairs.jj[pi], ii = c_pairs.ii[pi];
+    const int j = 16 * blk + jj, i = 16 * blk + ii;
+    const float* gj = Gm + j * LDG;
+    const float* gi = Gm + i * LDG;
+    const float* ej = Em + j * LDG;
+    const bf16* qj = Qt + j * LDT;
+    const bf16* ki = Kt + i * LDT;
+    float sl = 0.f, sa = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < kD; c += 4) {
+      const float4 a4 = *reinterpret_cast<const float4*>(gj + c);
+      const float4 b4 = *reinterpret_cast<const float4*>(gi + c);
+      const float4 e4 = *reinterpret_cast<const float4*>(ej + c);
+      const uint2 qq = *reinterpret_cast<const uint2*>(qj + c);
+      const uint2 kk = *reinterpret_cast<const uint2*>(ki + c);
+      const float2 q01 = unpack2(qq.x), q23 = unpack2(qq.y);
+      const float2 k01 = unpack2(kk.x), k23 = unpack2(kk.y);
+      const float x0 = __expf(a4.x - b4.x) * k01.x, x1 = __expf(a4.y - b4.y) * k01.y;
+      const float x2 = __expf(a4.z - b4.z) * k23.x, x3 = __expf(a4.w - b4.w) * k23.y;
+      sl = fmaf(e4.x, x0, fmaf(e4.y, x1, fmaf(e4.z, x2, fmaf(e4.w, x3, sl))));
+      sa = fmaf(q01.x, x0, fmaf(q01.y, x1, fmaf(q23.x, x2, fmaf(q23.y, x3, sa))));
     }
-    const int j = 16 * blk + jj, i = 16 * blk + rem;  // i <= j
-    const float4 gj = *reinterpret_cast<const float4*>(Gm + j * LDG + 4 * lane);
-    const float4 gi = *reinterpret_cast<const float4*>(Gm + i * LDG + 4 * lane);
-    const float4 ej = *reinterpret_cast<const float4*>(Em + j * LDG + 4 * lane);
-    const uint2 qj = *reinterpret_cast<const uint2*>(Qt + j * LDT + 4 * lane);
-    const uint2 ki = *reinterpret_cast<const uint2*>(Kt + i * LDT + 4 * lane);
-    const float2 q01 = unpack2(qj.x), q23 = unpack2(qj.y);
-    const float2 k01 = unpack2(ki.x), k23 = unpack2(ki.y);
-    const float x0 = __expf(gj.x - gi.x) * k01.x, x1 = __expf(gj.y - gi.y) * k01.y;
-    const float x2 = __expf(gj.z - gi.z) * k23.x, x3 = __expf(gj.w - gi.w) * k23.y;
-    float sl = ej.x * x0 + ej.y * x1 + ej.z * x2 + ej.w * x3;
-    float sa = q01.x * x0 + q01.y * x1 + q23.x * x2 + q23.y * x3;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      sl += __shfl_xor_sync(0xffffffffu, sl, o);
-      sa += __shfl_xor_sync(0xffffffffu, sa, o);
-    }
-    if (lane == 0) {
-      Lm[j * LDX + i] = i < j ? sl * rk[i] : 0.f;
-      Xm[j * LDX + i] = sa * sq[j] * rk[i];
-    }
+    Lm[j * LDX + i] = ii < jj ? sl * rk[i] : 0.f;
+    Xm[j * LDX + i] = sa * sq[j] * rk[i];
   }
 
   // 5. off-diagonal blocks on the tensor cores: fp16 operands scaled about the
@@ -648,21 +656,42 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   //    scratch: [0,48) e rows of blocks 1-3, [48,96) q^ rows, [96,192) k^ rows
   //    0..16 I - 1 for I = 1, 2, 3 (at 96, 112, 144).
   __half* Op = reinterpret_cast<__half*>(op);
-  for (int e = tid; e < 192 * kD; e += kThreads) {
-    const int row = e >> 7, c = e & 127;
-    float val;
+  for (int row = warp; row < 192; row += 8) {
+    const int c = 4 * lane;
+    int j, I;
+    const float* src;  // row of e, or of raw q / k (bf16) below
+    float f = 1.f;
+    float4 sc;
     if (row < 96) {
-      const int I = 1 + ((row % 48) >> 4), j = 16 * I + (row & 15);
-      const float sc = __expf(Gm[j * LDG + c] - Gm[16 * I * LDG + c]);
-      val = row < 48 ? Em[j * LDG + c] * sc : __bfloat162float(Qt[j * LDT + c]) * sq[j] * sc;
+      I = 1 + ((row < 48 ? row : row - 48) >> 4);
+      j = 16 * I + (row & 15);
+      const float4 gj = *reinterpret_cast<const float4*>(Gm + j * LDG + c);
+      const float4 gr = *reinterpret_cast<const float4*>(Gm + 16 * I * LDG + c);
+      sc = make_float4(__expf(gj.x - gr.x), __expf(gj.y - gr.y), __expf(gj.z - gr.z),
+                       __expf(gj.w - gr.w));
     } else {
       const int kr = row - 96;
-      const int I = kr < 16 ? 1 : (kr < 48 ? 2 : 3);
-      const int i = kr - (I == 1 ? 0 : (I == 2 ? 16 : 48));
-      val = __bfloat162float(Kt[i * LDT + c]) * rk[i] *
-            __expf(Gm[16 * I * LDG + c] - Gm[i * LDG + c]);
+      I = kr < 16 ? 1 : (kr < 48 ? 2 : 3);
+      j = kr - (I == 1 ? 0 : (I == 2 ? 16 : 48));
+      const float4 gj = *reinterpret_cast<const float4*>(Gm + j * LDG + c);
+      const float4 gr = *reinterpret_cast<const float4*>(Gm + 16 * I * LDG + c);
+      sc = make_float4(__expf(gr.x - gj.x), __expf(gr.y - gj.y), __expf(gr.z - gj.z),
+                       __expf(gr.w - gj.w));
     }
-    Op[row * LDT + c] = __float2half_rn(val);
+    float4 val;
+    if (row < 48) {
+      src = Em + j * LDG;
+      val = *reinterpret_cast<const float4*>(src + c);
+    } else {
+      const uint2 raw = *reinterpret_cast<const uint2*>((row < 96 ? Qt : Kt) + j * LDT + c);
+      const float2 v01 = unpack2(raw.x), v23 = unpack2(raw.y);
+      f = row < 96 ? sq[j] : rk[j];
+      val = make_float4(v01.x, v01.y, v23.x, v23.y);
+    }
+    uint2 o;
+    o.x = pack2h(val.x * f * sc.x, val.y * f * sc.y);
+    o.y = pack2h(val.z * f * sc.z, val.w * f * sc.w);
+    *reinterpret_cast<uint2*>(Op + row * LDT + c) = o;
   }
   __syncthreads();
   //    tasks (matrix, I, column pair np < I): 6 for L, 6 for A
@@ -817,238 +846,6 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   }
 }
 
-// ---------------------------------------------------------------- scan kernel
-constexpr int kScanThreads = 256;           // 8 warps
-constexpr int LDU = 64 + 8;                 // f32 row stride of the U tile (conflict-free float2)
-// double-buffered, fetched one chunk ahead
-constexpr int S_W = 0;                      // W tile     [64][LDT] f16
-constexpr int S_Q = S_W + kC * LDT * 2;     // Q rows     [64][LDT] f16
-constexpr int S_K = S_Q + kC * LDT * 2;     // K rows     [64][LDT] f16
-constexpr int S_A = S_K + kC * LDT * 2;     // A_qk       [64][LDH] f16
-constexpr int S_U = S_A + kC * LDH * 2;     // U columns of this CTA [64][LDU] f32
-constexpr int S_SC = S_U + kC * LDU * 4;    // scalars (132 f32)
-constexpr int STAGE = S_SC + kScal * 4;
-// on-chip operands
-constexpr int S_SB = 2 * STAGE;             // state slice (scaled) [128][LDH] f16
-constexpr int S_UT = S_SB + kD * LDH * 2;   // U~ (scaled)          [64][LDH] f16
-constexpr int S_US = S_UT + kC * LDH * 2;   // U~ diag(fs)          [64][LDH] f16
-constexpr int S_RED = S_US + kC * LDH * 2;  // 8 floats for the CTA max
-constexpr int S_BYTES = S_RED + 64;
-static_assert(STAGE % 16 == 0, "stage buffers must stay 16-byte aligned");
-static_assert(S_BYTES <= 227 * 1024, "shared memory of the scan kernel");
-
-template <typename TO>
-__device__ __forceinline__ void store2(TO* p, float x, float y);
-template <>
-__device__ __forceinline__ void store2<float>(float* p, float x, float y) {
-  *reinterpret_cast<float2*>(p) = make_float2(x, y);
-}
-template <>
-__device__ __forceinline__ void store2<bf16>(bf16* p, float x, float y) {
-  *reinterpret_cast<uint32_t*>(p) = pack2(x, y);
-}
-
-template <typename TO>
-__global__ void __launch_bounds__(kScanThreads, 1)
-state_scan_kernel(const uint8_t* __restrict__ ws, WsLayout L, const float* h0, int T, int Hk,
-                  int Hv, TO* __restrict__ o, float* ht, int* status) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  __half* Sb = reinterpret_cast<__half*>(sm + S_SB);
-  __half* Ut = reinterpret_cast<__half*>(sm + S_UT);
-  __half* Us = reinterpret_cast<__half*>(sm + S_US);
-  float* red = reinterpret_cast<float*>(sm + S_RED);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g8 = lane >> 2, t4 = lane & 3;
-  const int c0 = 64 * blockIdx.x;
-  const int head = blockIdx.y, b = head / Hv, hv = head % Hv, hk = hv / (Hv / Hk);
-  const int Nc = (T + kC - 1) / kC, Tp = Nc * kC;
-  const size_t khead = (size_t)b * Hk + hk;
-  const __half* Wg = reinterpret_cast<const __half*>(ws + L.w) + (size_t)head * Tp * kD;
-  const float* Ug = reinterpret_cast<const float*>(ws + L.u) + (size_t)head * Tp * kD + c0;
-  const __half* Ag = reinterpret_cast<const __half*>(ws + L.a) + (size_t)head * Tp * kC;
-  const __half* Qg = reinterpret_cast<const __half*>(ws + L.qh) + khead * Tp * kD;
-  const __half* Kg = reinterpret_cast<const __half*>(ws + L.kh) + khead * Tp * kD;
-  const float* Sg = reinterpret_cast<const float*>(ws + L.scal) + (size_t)head * Nc * kScal;
-
-  // every tile of chunk n into stage n % 2
-  auto issue_stage = [&](int n) {
-    uint8_t* st = sm + (n & 1) * STAGE;
-    const size_t r0 = (size_t)n * kC;
-    for (int i = tid; i < kC * 16; i += kScanThreads) {
-      const int r = i >> 4, c16 = i & 15;
-      cp16(st + S_W + (r * LDT + c16 * 8) * 2, Wg + (r0 + r) * kD + c16 * 8, 16);
-      cp16(st + S_Q + (r * LDT + c16 * 8) * 2, Qg + (r0 + r) * kD + c16 * 8, 16);
-      cp16(st + S_K + (r * LDT + c16 * 8) * 2, Kg + (r0 + r) * kD + c16 * 8, 16);
-      cp16(st + S_U + (r * LDU + c16 * 4) * 4, Ug + (r0 + r) * kD + c16 * 4, 16);
-      if (c16 < 8) cp16(st + S_A + (r * LDH + c16 * 8) * 2, Ag + (r0 + r) * kC + c16 * 8, 16);
-    }
-    if (tid < kScal / 4) cp16(st + S_SC + tid * 16, Sg + (size_t)n * kScal + tid * 4, 16);
-    cp_commit();
-  };
-  issue_stage(0);
-
-  // state slice: warp w holds rows 16 w .. + 15 and all 64 columns of the CTA's
-  // 128 x 64 slice, as 8 C fragments
-  const int sr = 16 * warp + g8;
-  float S[8][4];
-  float mx = 0.f;
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    float2 x0 = make_float2(0.f, 0.f), x1 = x0;
-    if (h0) {
-      const float* src = h0 + ((size_t)head * kD + sr) * kD + c0 + 8 * nt + 2 * t4;
-      x0 = *reinterpret_cast<const float2*>(src);
-      x1 = *reinterpret_cast<const float2*>(src + 8 * kD);
-    }
-    S[nt][0] = x0.x; S[nt][1] = x0.y; S[nt][2] = x1.x; S[nt][3] = x1.y;
-    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x0.x), fabsf(x0.y)), fmaxf(fabsf(x1.x), fabsf(x1.y))));
-  }
-  // sigma = 2^-e: the largest |U| of the head and |h0| of this slice land below 2^8
-  for (int n = tid; n < Nc; n += kScanThreads) mx = fmaxf(mx, Sg[(size_t)n * kScal + kScMaxU]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  if (lane == 0) red[warp] = mx;
-  __syncthreads();
-  mx = red[0];
-#pragma unroll
-  for (int w = 1; w < 8; ++w) mx = fmaxf(mx, red[w]);
-  const int e = mx > 0.f ? min(max(ilogbf(mx) - 7, -100), 100) : 0;
-  const float sigma = ldexpf(1.f, -e), inv_sigma = ldexpf(1.f, e);
-  float range = 0.f;
-
-  auto store_state = [&]() {
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int c = 8 * nt + 2 * t4;
-      range = fmaxf(range, fmaxf(fmaxf(fabsf(S[nt][0]), fabsf(S[nt][1])),
-                                 fmaxf(fabsf(S[nt][2]), fabsf(S[nt][3]))));
-      *reinterpret_cast<uint32_t*>(Sb + sr * LDH + c) = pack2h(S[nt][0], S[nt][1]);
-      *reinterpret_cast<uint32_t*>(Sb + (sr + 8) * LDH + c) = pack2h(S[nt][2], S[nt][3]);
-    }
-  };
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) S[nt][i] *= sigma;
-  store_state();
-
-  // output tile of this warp: rows 16 (w % 4) .. + 15, columns 32 (w / 4) .. + 31
-  const int mt = warp & 3, nb = 32 * (warp >> 2);
-  const int r0 = 16 * mt + g8, r1 = r0 + 8;
-  for (int n = 0; n < Nc; ++n) {
-    cp_wait<0>();
-    __syncthreads();  // chunk n landed; the previous chunk's reads and state stores are done
-    if (n + 1 < Nc) issue_stage(n + 1);
-    const uint8_t* st = sm + (n & 1) * STAGE;
-    const __half* Wt = reinterpret_cast<const __half*>(st + S_W);
-    const __half* Qt = reinterpret_cast<const __half*>(st + S_Q);
-    const __half* Kt = reinterpret_cast<const __half*>(st + S_K);
-    const __half* At = reinterpret_cast<const __half*>(st + S_A);
-    const float* Uc = reinterpret_cast<const float*>(st + S_U);
-    const float* sc = reinterpret_cast<const float*>(st + S_SC);
-    const int t0 = n * kC;
-
-    // P = W S and OQ = Q S for this warp's tile (S scaled by sigma)
-    float P[4][4] = {}, OQ[4][4] = {};
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      uint32_t aw[4], aq[4];
-      ldsm_x4(aw, Wt + (16 * mt + lrow_a(lane)) * LDT + 16 * ks + lcol_a(lane));
-      ldsm_x4(aq, Qt + (16 * mt + lrow_a(lane)) * LDT + 16 * ks + lcol_a(lane));
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        uint32_t bb[4];
-        ldsm_x4_t(bb, Sb + (16 * ks + lrow_a(lane)) * LDH + nb + 16 * np + lcol_a(lane));
-        mma_f16(P[2 * np], aw, bb[0], bb[1]);
-        mma_f16(P[2 * np + 1], aw, bb[2], bb[3]);
-        mma_f16(OQ[2 * np], aq, bb[0], bb[1]);
-        mma_f16(OQ[2 * np + 1], aq, bb[2], bb[3]);
-      }
-    }
-    // U~ = sigma U - P, and U~ diag(fs) for the state update, in fp16
-    {
-      const float fs0 = sc[kC + r0], fs1 = sc[kC + r1];
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        const int c = nb + 8 * nt + 2 * t4;
-        const float2 u0 = *reinterpret_cast<const float2*>(Uc + r0 * LDU + c);
-        const float2 u1 = *reinterpret_cast<const float2*>(Uc + r1 * LDU + c);
-        const float x0 = fmaf(sigma, u0.x, -P[nt][0]), x1 = fmaf(sigma, u0.y, -P[nt][1]);
-        const float x2 = fmaf(sigma, u1.x, -P[nt][2]), x3 = fmaf(sigma, u1.y, -P[nt][3]);
-        range = fmaxf(range, fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3))));
-        *reinterpret_cast<uint32_t*>(Ut + r0 * LDH + c) = pack2h(x0, x1);
-        *reinterpret_cast<uint32_t*>(Ut + r1 * LDH + c) = pack2h(x2, x3);
-        *reinterpret_cast<uint32_t*>(Us + r0 * LDH + c) = pack2h(x0 * fs0, x1 * fs0);
-        *reinterpret_cast<uint32_t*>(Us + r1 * LDH + c) = pack2h(x2 * fs1, x3 * fs1);
-      }
-    }
-    __syncthreads();
-
-    // o = (fo (Q S) + A_qk U~) / sigma
-    {
-      float OA[4][4] = {};
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        uint32_t a[4];
-        ldsm_x4(a, At + (16 * mt + lrow_a(lane)) * LDH + 16 * ks + lcol_a(lane));
-#pragma unroll
-        for (int np = 0; np < 2; ++np) {
-          uint32_t bb[4];
-          ldsm_x4_t(bb, Ut + (16 * ks + lrow_a(lane)) * LDH + nb + 16 * np + lcol_a(lane));
-          mma_f16(OA[2 * np], a, bb[0], bb[1]);
-          mma_f16(OA[2 * np + 1], a, bb[2], bb[3]);
-        }
-      }
-      const float fo0 = sc[r0], fo1 = sc[r1];
-      TO* o0 = o + (((size_t)b * T + t0 + r0) * Hv + hv) * kD + c0 + nb + 2 * t4;
-      TO* o1 = o0 + (size_t)8 * Hv * kD;
-      const bool w0 = t0 + r0 < T, w1 = t0 + r1 < T;
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        if (w0)
-          store2<TO>(o0 + 8 * nt, (fo0 * OQ[nt][0] + OA[nt][0]) * inv_sigma,
-                     (fo0 * OQ[nt][1] + OA[nt][1]) * inv_sigma);
-        if (w1)
-          store2<TO>(o1 + 8 * nt, (fo1 * OQ[nt][2] + OA[nt][2]) * inv_sigma,
-                     (fo1 * OQ[nt][3] + OA[nt][3]) * inv_sigma);
-      }
-    }
-
-    // S <- diag(gamma_C) S + K^T U~s  (this warp's 16 state rows)
-    {
-      const float gA = sc[kScGC + sr], gB = sc[kScGC + sr + 8];
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        S[nt][0] *= gA; S[nt][1] *= gA; S[nt][2] *= gB; S[nt][3] *= gB;
-      }
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        uint32_t a[4];
-        ldsm_x4_t(a, Kt + (16 * ks + lrow_b(lane)) * LDT + 16 * warp + lcol_b(lane));
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t bb[4];
-          ldsm_x4_t(bb, Us + (16 * ks + lrow_a(lane)) * LDH + 16 * np + lcol_a(lane));
-          mma_f16(S[2 * np], a, bb[0], bb[1]);
-          mma_f16(S[2 * np + 1], a, bb[2], bb[3]);
-        }
-      }
-      store_state();
-    }
-  }
-  if (!(range <= kF16Max)) report_range(status);
-
-  if (ht != nullptr) {
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      float* dst = ht + ((size_t)head * kD + sr) * kD + c0 + 8 * nt + 2 * t4;
-      *reinterpret_cast<float2*>(dst) = make_float2(S[nt][0] * inv_sigma, S[nt][1] * inv_sigma);
-      *reinterpret_cast<float2*>(dst + 8 * kD) =
-          make_float2(S[nt][2] * inv_sigma, S[nt][3] * inv_sigma);
-    }
-  }
-}
-
 template <typename TO>
 cudaError_t launch_t(const ChunkArgs& a, bool gdn2, uint8_t* ws, const WsLayout& L,
                      cudaStream_t s) {
@@ -1077,12 +874,7 @@ cudaError_t launch_t(const ChunkArgs& a, bool gdn2, uint8_t* ws, const WsLayout&
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(state_scan_kernel<TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           S_BYTES);
-  if (e != cudaSuccess) return e;
-  state_scan_kernel<TO><<<dim3(2, a.B * a.Hv), kScanThreads, S_BYTES, s>>>(
-      ws, L, a.h0, a.T, a.Hk, a.Hv, static_cast<TO*>(a.o), a.ht, status);
-  return cudaGetLastError();
+  return launch_scan_tc(a, ws, status, s);
 }
 
 }  // namespace

@@ -1,0 +1,451 @@
+// scan_tc.cu -- the sequential state scan of the bf16 chunk paths on the tcgen05
+// tensor cores (sm_100a): one CTA per (batch, value head, 64-column half of d_v),
+// over the chunks of the sequence, with
+//   [O_q; P] = [Q; W] S          (M = 128: Q rows in TMEM lanes 0-63, W rows in 64-127)
+//   U~ = sigma U - P,  U~s = U~ diag(fs)
+//   O_a = A_qk U~                (M = 128; lanes 64-127 of the result are unused)
+//   DS = K^T U~s                 (M = 128 over the d_k rows of the state)
+//   o = (fo O_q + O_a) / sigma,  S <- diag(gamma_C) S + DS
+// The operands come from the workspace written by the prep kernels (fp16 W, A_qk,
+// scan Q / K rows; fp32 U; per-chunk factors), see chunk_mma.cu for the algebra,
+// the precision design and the range scale sigma.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: every tile of chunk n into stage n % 2 (10 bulk copies)
+//   warp 1      TMEM allocation and the tcgen05.mma issue (one thread)
+//   warps 2-5   epilogue: one state row (d_k row = TMEM lane) per thread in fp32
+//               registers; TMEM loads of the accumulators, U~ / U~s / the state
+//               written back to shared memory as fp16 operands, o stored.
+// Hand-offs go through mbarriers; every wait is bounded and an expired wait ends
+// the kernel through the status word (GDN_ERR_TIMEOUT) after its copies and
+// tensor-core work in flight have drained.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "chunk_layout.cuh"
+#include "common.cuh"
+#include "launch.h"
+#include "tc_ptx.cuh"
+
+namespace gdn {
+namespace {
+
+using namespace tc;
+using bf16 = __nv_bfloat16;
+
+constexpr int kScanTcThreads = 192;
+// shared memory map (offsets from a 1024-byte aligned base); 128-byte swizzled
+// fp16 tiles are stored as 64-column halves of [64 rows][128 bytes]
+constexpr uint32_t ST_QW = 0;        // [Q; W] K-major: half h at h * 16384 (Q rows, then W rows)
+constexpr uint32_t ST_K = 32768;     // K rows: half h (d_k columns 64 h ..) at + h * 8192
+constexpr uint32_t ST_A = 49152;     // A_qk [64][64]
+constexpr uint32_t ST_U = 57344;     // U (fp32) columns c0 .. c0 + 63: two [64][32] boxes
+constexpr uint32_t ST_SC = 73728;    // per-chunk factors (kScal floats)
+constexpr uint32_t STAGE_BYTES = 75776;
+constexpr uint32_t TX_BYTES = 32768 + 16384 + 8192 + 16384 + kScal * 4;
+constexpr uint32_t OFF_SB = 2 * STAGE_BYTES;  // state (scaled) fp16, MN-major B: [128][64]
+constexpr uint32_t OFF_UT = OFF_SB + 16384;   // U~ fp16 [64][64]
+constexpr uint32_t OFF_US = OFF_UT + 8192;    // U~s fp16 [64][64]
+constexpr uint32_t OFF_RED = OFF_US + 8192;   // CTA max reduction (4 floats)
+constexpr uint32_t OFF_BAR = OFF_RED + 64;    // mbarriers + TMEM address
+constexpr uint32_t SCAN_TC_SMEM = OFF_BAR + 128 + 1024;
+static_assert(ST_SC + kScal * 4 <= STAGE_BYTES, "stage layout");
+static_assert(SCAN_TC_SMEM <= 227 * 1024, "shared memory of the tcgen05 scan");
+
+// TMEM columns of the accumulators (M = 128, N = 64 each)
+constexpr uint32_t TM_QP = 0, TM_OA = 64, TM_DS = 128, TM_COLS = 256;
+
+// barrier indices
+enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_QP, B_UT, B_DS, B_OA, B_S, B_COUNT };
+
+// Byte offset of 16-byte chunk c16 of row r in a 128-byte swizzled tile.
+__device__ __forceinline__ uint32_t swz(int r, int c16) {
+  return (uint32_t)(r * 128 + ((c16 ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t pack2h(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// 64 fp32 values as one fp16 row of a 128-byte swizzled tile.
+__device__ __forceinline__ void store_row_f16(uint8_t* tile, int r, const float* v) {
+#pragma unroll
+  for (int c16 = 0; c16 < 8; ++c16) {
+    uint4 p;
+    p.x = pack2h(v[8 * c16 + 0], v[8 * c16 + 1]);
+    p.y = pack2h(v[8 * c16 + 2], v[8 * c16 + 3]);
+    p.z = pack2h(v[8 * c16 + 4], v[8 * c16 + 5]);
+    p.w = pack2h(v[8 * c16 + 6], v[8 * c16 + 7]);
+    *reinterpret_cast<uint4*>(tile + swz(r, c16)) = p;
+  }
+}
+
+// Bounded wait that also gives up as soon as another role of the CTA has given up.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status,
+                                              int where, volatile int* abort_flag) {
+  for (uint32_t i = 0; i < (1u << 24); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 255u && *abort_flag) return false;
+  }
+  report_timeout(status, where);
+  *abort_flag = 1;
+  return false;
+}
+
+// 64 output values of one row with 16-byte stores.
+template <typename TO>
+__device__ __forceinline__ void store_row(TO* dst, const float* v);
+template <>
+__device__ __forceinline__ void store_row<float>(float* dst, const float* v) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 4)
+    *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+}
+template <>
+__device__ __forceinline__ void store_row<bf16>(bf16* dst, const float* v) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 8) {
+    uint4 p;
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[c], v[c + 1]);
+    __nv_bfloat162 h1 = __floats2bfloat162_rn(v[c + 2], v[c + 3]);
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[c + 4], v[c + 5]);
+    __nv_bfloat162 h3 = __floats2bfloat162_rn(v[c + 6], v[c + 7]);
+    p.x = *reinterpret_cast<uint32_t*>(&h0);
+    p.y = *reinterpret_cast<uint32_t*>(&h1);
+    p.z = *reinterpret_cast<uint32_t*>(&h2);
+    p.w = *reinterpret_cast<uint32_t*>(&h3);
+    *reinterpret_cast<uint4*>(dst + c) = p;
+  }
+}
+
+struct ScanMaps {
+  CUtensorMap q, w, k, a, u;
+};
+
+template <typename TO>
+__global__ void __launch_bounds__(kScanTcThreads, 1)
+state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __restrict__ ws,
+                     WsLayout L, const float* h0, int T, int Hk, int Hv, TO* __restrict__ o,
+                     float* ht, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(sm + OFF_RED);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c0 = 64 * blockIdx.x;
+  const int head = blockIdx.y, b = head / Hv, hv = head % Hv, hk = hv / (Hv / Hk);
+  const int Nc = (T + kC - 1) / kC, Tp = Nc * kC;
+  const int khead = b * Hk + hk;
+  const float* Sg = reinterpret_cast<const float*>(ws + L.scal) + (size_t)head * Nc * kScal;
+  const uint32_t sbase = smem_u32(sm);
+
+  if (warp == 1) tmem_alloc(tmem_slot, TM_COLS);
+  if (tid == 0) {
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], (i == B_EMPTY0 || i == B_EMPTY1) ? 2 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&maps.q);
+    prefetch_tmap(&maps.w);
+    prefetch_tmap(&maps.k);
+    prefetch_tmap(&maps.a);
+    prefetch_tmap(&maps.u);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      for (int n = 0; n < Nc; ++n) {
+        const int s = n & 1;
+        if (n >= 2 &&
+            !wait_or_abort(&bar[B_EMPTY0 + s], ((n >> 1) - 1) & 1, status, 101, abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        uint8_t* st = sm + s * STAGE_BYTES;
+        uint64_t* full = &bar[B_FULL0 + s];
+        mbar_arrive_expect_tx(full, TX_BYTES);
+        const int rq = khead * Tp + n * kC, rw = head * Tp + n * kC;
+        tma_load_2d(st + ST_QW + 0, &maps.q, full, 0, rq);
+        tma_load_2d(st + ST_QW + 16384, &maps.q, full, 64, rq);
+        tma_load_2d(st + ST_QW + 8192, &maps.w, full, 0, rw);
+        tma_load_2d(st + ST_QW + 24576, &maps.w, full, 64, rw);
+        tma_load_2d(st + ST_K + 0, &maps.k, full, 0, rq);
+        tma_load_2d(st + ST_K + 8192, &maps.k, full, 64, rq);
+        tma_load_2d(st + ST_A, &maps.a, full, 0, rw);
+        tma_load_2d(st + ST_U + 0, &maps.u, full, c0, rw);
+        tma_load_2d(st + ST_U + 8192, &maps.u, full, c0 + 32, rw);
+        bulk_load(st + ST_SC, Sg + (size_t)n * kScal, kScal * 4, full);
+      }
+      // drain: every stage armed must have landed before the CTA may exit
+      for (int n = (Nc >= 2 ? Nc - 2 : 0); n < Nc; ++n)
+        mbar_wait(&bar[B_FULL0 + (n & 1)], (n >> 1) & 1, nullptr, 0, 1u << 20);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t id_qw = idesc_f16(128, 64, false, true);
+      const uint32_t id_a = idesc_f16(128, 64, false, true);
+      const uint32_t id_k = idesc_f16(128, 64, true, true);
+      uint32_t qp_phases = 0;  // phases of B_QP completed by our commits
+      for (int n = 0; n < Nc; ++n) {
+        const int s = n & 1;
+        const uint32_t st = sbase + s * STAGE_BYTES;
+        if (!wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 102, abort_flag) ||
+            !wait_or_abort(&bar[B_S], n & 1, status, 103, abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        // [O_q; P] = [Q; W] S   (K = d_k = 128: two 64-column halves of 4 steps)
+        for (int k16 = 0; k16 < 8; ++k16) {
+          const uint32_t aoff = (uint32_t)(k16 >> 2) * 16384u + (uint32_t)(k16 & 3) * 32u;
+          mma_bf16(tmem + TM_QP, sw128_desc(st + ST_QW + aoff, 16, 1024),
+                   sw128_desc(sbase + OFF_SB + k16 * 2048, 8192, 1024), id_qw, k16 > 0);
+        }
+        mma_commit(&bar[B_QP]);
+        ++qp_phases;
+        if (!wait_or_abort(&bar[B_UT], n & 1, status, 104, abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        // DS = K^T U~s first (the state update waits for it), then O_a = A_qk U~
+        // (K = 64 tokens: 4 steps each)
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_bf16(tmem + TM_DS, sw128_desc(st + ST_K + k16 * 2048, 8192, 1024),
+                   sw128_desc(sbase + OFF_US + k16 * 2048, 8192, 1024), id_k, k16 > 0);
+        mma_commit(&bar[B_DS]);
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_bf16(tmem + TM_OA, sw128_desc(st + ST_A + k16 * 32, 16, 1024),
+                   sw128_desc(sbase + OFF_UT + k16 * 2048, 8192, 1024), id_a, k16 > 0);
+        mma_commit(&bar[B_OA]);
+        mma_commit(&bar[B_EMPTY0 + s]);  // the stage's operands have been read
+      }
+      // drain: nothing of ours may still run on the tensor cores at teardown (the
+      // commit below completes phase qp_phases of B_QP once all our MMAs are done)
+      mma_commit(&bar[B_QP]);
+      mbar_wait(&bar[B_QP], qp_phases & 1, nullptr, 0, 1u << 20);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = tid - 64;                       // 0..127
+    const int row = 32 * (warp & 3) + lane;       // TMEM lane = d_k row of the state
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    const bool p_rows = row >= 64;                // lanes 64-127: rows of P (token row - 64)
+    float S[64];
+    float mx = 0.f;
+    {
+      const float* src = h0 ? h0 + ((size_t)head * kD + row) * kD + c0 : nullptr;
+#pragma unroll
+      for (int c = 0; c < 64; c += 4) {
+        const float4 t = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0, 0, 0, 0);
+        S[c] = t.x; S[c + 1] = t.y; S[c + 2] = t.z; S[c + 3] = t.w;
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(t.x), fabsf(t.y)), fmaxf(fabsf(t.z), fabsf(t.w))));
+      }
+    }
+    for (int n = e; n < Nc; n += 128) mx = fmaxf(mx, Sg[(size_t)n * kScal + kScMaxU]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) red[warp - 2] = mx;
+    named_barrier(1, 128);
+    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const int ex = mx > 0.f ? min(max(ilogbf(mx) - 7, -100), 100) : 0;
+    const float sigma = ldexpf(1.f, -ex), inv_sigma = ldexpf(1.f, ex);
+    float range = 0.f;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) {
+      S[c] *= sigma;
+      range = fmaxf(range, fabsf(S[c]));
+    }
+    store_row_f16(sm + OFF_SB, row, S);
+    fence_proxy_async_smem();
+    named_barrier(1, 128);
+    if (e == 0) mbar_arrive(&bar[B_S]);
+
+    float OQ[64];
+    for (int n = 0; n < Nc; ++n) {
+      const int s = n & 1;
+      const uint8_t* st = sm + s * STAGE_BYTES;
+      const float* sc = reinterpret_cast<const float*>(st + ST_SC);
+      {  // every epilogue thread takes the same decision (no thread is left at a barrier)
+        const bool ok = wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 105, abort_flag) &&
+                        wait_or_abort(&bar[B_QP], n & 1, status, 106, abort_flag);
+        if (named_barrier_or(1, 128, !ok)) {
+          *abort_flag = 1;
+          break;
+        }
+      }
+      tc_fence_after();
+      float fo = 0.f;
+      if (p_rows) {
+        // U~ = sigma U - P and U~s = U~ fs for token r, written as fp16 operand rows
+        const int r = row - 64;
+        const float fs = sc[kC + r];
+        float P[64];
+        tmem_ld64(tl + TM_QP, P);
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const int box = c4 >> 3, ch = c4 & 7;  // 32 fp32 columns per swizzled box
+          const float4 u = *reinterpret_cast<const float4*>(st + ST_U + box * 8192 + swz(r, ch));
+          P[4 * c4 + 0] = fmaf(sigma, u.x, -P[4 * c4 + 0]);
+          P[4 * c4 + 1] = fmaf(sigma, u.y, -P[4 * c4 + 1]);
+          P[4 * c4 + 2] = fmaf(sigma, u.z, -P[4 * c4 + 2]);
+          P[4 * c4 + 3] = fmaf(sigma, u.w, -P[4 * c4 + 3]);
+        }
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) {
+          const float* v = P + 8 * c16;
+          uint4 pu, ps;
+          pu.x = pack2h(v[0], v[1]);
+          pu.y = pack2h(v[2], v[3]);
+          pu.z = pack2h(v[4], v[5]);
+          pu.w = pack2h(v[6], v[7]);
+          ps.x = pack2h(v[0] * fs, v[1] * fs);
+          ps.y = pack2h(v[2] * fs, v[3] * fs);
+          ps.z = pack2h(v[4] * fs, v[5] * fs);
+          ps.w = pack2h(v[6] * fs, v[7] * fs);
+          const uint32_t off = swz(r, c16);
+          *reinterpret_cast<uint4*>(sm + OFF_UT + off) = pu;
+          *reinterpret_cast<uint4*>(sm + OFF_US + off) = ps;
+        }
+#pragma unroll
+        for (int c = 0; c < 64; ++c) range = fmaxf(range, fabsf(P[c]));
+      } else {
+        tmem_ld64(tl + TM_QP, OQ);  // O_q of token row
+        fo = sc[row];
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_barrier(1, 128);
+      if (e == 0) mbar_arrive(&bar[B_UT]);
+
+      // the state update first: it is what the next chunk waits for
+      {
+        const bool ok = wait_or_abort(&bar[B_DS], n & 1, status, 107, abort_flag);
+        if (named_barrier_or(1, 128, !ok)) {
+          *abort_flag = 1;
+          break;
+        }
+      }
+      tc_fence_after();
+      {
+        float D[64];
+        tmem_ld64(tl + TM_DS, D);
+        const float gc = sc[kScGC + row];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          S[c] = fmaf(gc, S[c], D[c]);
+          range = fmaxf(range, fabsf(S[c]));
+        }
+      }
+      store_row_f16(sm + OFF_SB, row, S);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_barrier(1, 128);
+      if (e == 0) {
+        mbar_arrive(&bar[B_S]);
+        mbar_arrive(&bar[B_EMPTY0 + s]);  // U and the factors of the stage are read
+      }
+
+      // then the output rows (lanes 0-63), overlapping the next chunk's products
+      if (!p_rows) {
+        if (!wait_or_abort(&bar[B_OA], n & 1, status, 108, abort_flag)) continue;
+        tc_fence_after();
+        float OA[64];
+        tmem_ld64(tl + TM_OA, OA);
+        tc_fence_before();
+        const int t = n * kC + row;
+        if (t < T) {
+          TO* dst = o + (((size_t)b * T + t) * Hv + hv) * kD + c0;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) OA[c] = (fo * OQ[c] + OA[c]) * inv_sigma;
+          store_row<TO>(dst, OA);
+        }
+      }
+    }
+    if (!(range <= kF16Max)) report_range(status);
+    if (ht != nullptr && !*abort_flag) {
+      float* dst = ht + ((size_t)head * kD + row) * kD + c0;
+#pragma unroll
+      for (int c = 0; c < 64; c += 4)
+        *reinterpret_cast<float4*>(dst + c) = make_float4(S[c] * inv_sigma, S[c + 1] * inv_sigma,
+                                                          S[c + 2] * inv_sigma, S[c + 3] * inv_sigma);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a [rows][cols] row-major region, boxes of [64 rows][128 bytes], 128-byte swizzle.
+bool make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base,
+              CUtensorMapDataType dt, int elem_bytes, uint64_t cols, uint64_t rows) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * elem_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), 64};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <typename TO>
+cudaError_t launch_t(const ChunkArgs& a, const WsLayout& L, const uint8_t* ws, int* status,
+                     cudaStream_t s) {
+  auto enc = encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  const uint64_t Tp = (uint64_t)((a.T + kC - 1) / kC) * kC;
+  const uint64_t rv = (uint64_t)a.B * a.Hv * Tp, rk = (uint64_t)a.B * a.Hk * Tp;
+  ScanMaps m;
+  if (!make_map(enc, &m.q, ws + L.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rk) ||
+      !make_map(enc, &m.w, ws + L.w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rv) ||
+      !make_map(enc, &m.k, ws + L.kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rk) ||
+      !make_map(enc, &m.a, ws + L.a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kC, rv) ||
+      !make_map(enc, &m.u, ws + L.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kD, rv))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(state_scan_tc_kernel<TO>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_TC_SMEM);
+  if (e != cudaSuccess) return e;
+  state_scan_tc_kernel<TO><<<dim3(2, a.B * a.Hv), kScanTcThreads, SCAN_TC_SMEM, s>>>(
+      m, ws, L, a.h0, a.T, a.Hk, a.Hv, static_cast<TO*>(a.o), a.ht, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_scan_tc(const ChunkArgs& a, const void* ws, int* status, cudaStream_t s) {
+  const WsLayout L = ws_layout(a.B, a.T, a.Hk, a.Hv);
+  const uint8_t* w = static_cast<const uint8_t*>(ws);
+  if (a.flags & GDN_OUT_F32) return launch_t<float>(a, L, w, status, s);
+  return launch_t<bf16>(a, L, w, status, s);
+}
+
+}  // namespace gdn
