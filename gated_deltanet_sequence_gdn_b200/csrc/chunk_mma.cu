@@ -48,7 +48,6 @@ using bf16 = __nv_bfloat16;
 
 constexpr int kThreads = 256;  // 8 warps
 constexpr int LDT = kD + 8;    // 16-bit row stride of 128-wide tiles (272 B: ldmatrix conflict-free)
-constexpr int LDH = 64 + 8;    // 16-bit row stride of 64-wide tiles (144 B)
 
 // x = hi + lo with hi = rn_bf16(x), lo = rn_bf16(x - hi), for a pair of values.
 __device__ __forceinline__ void split2(float x, float y, uint32_t& hi, uint32_t& lo) {
