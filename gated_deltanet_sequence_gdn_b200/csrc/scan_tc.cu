@@ -10,12 +10,14 @@
 // scan Q / K rows; fp32 U; per-chunk factors), see chunk_mma.cu for the algebra,
 // the precision design and the range scale sigma.
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0      TMA producer: every tile of chunk n into stage n % 2 (10 bulk copies)
 //   warp 1      TMEM allocation and the tcgen05.mma issue (one thread)
-//   warps 2-5   epilogue: one state row (d_k row = TMEM lane) per thread in fp32
-//               registers; TMEM loads of the accumulators, U~ / U~s / the state
-//               written back to shared memory as fp16 operands, o stored.
+//   warps 2-9   epilogue, two warps per TMEM lane quarter (warps w and w + 4 take
+//               columns 0-31 and 32-63): 32 columns of one state row (d_k row =
+//               TMEM lane) per thread in fp32 registers; TMEM loads of the
+//               accumulators, U~ / U~s / the state written back to shared memory
+//               as fp16 operands, o stored.
 // Hand-offs go through mbarriers; every wait is bounded and an expired wait ends
 // the kernel through the status word (GDN_ERR_TIMEOUT) after its copies and
 // tensor-core work in flight have drained.
@@ -33,7 +35,8 @@ namespace {
 using namespace tc;
 using bf16 = __nv_bfloat16;
 
-constexpr int kScanTcThreads = 192;
+constexpr int kScanTcThreads = 320;
+constexpr int kEpi = 256;  // epilogue threads
 // shared memory map (offsets from a 1024-byte aligned base); 128-byte swizzled
 // fp16 tiles are stored as 64-column halves of [64 rows][128 bytes]
 constexpr uint32_t ST_QW = 0;        // [Q; W] K-major: half h at h * 16384 (Q rows, then W rows)
@@ -46,7 +49,7 @@ constexpr uint32_t TX_BYTES = 32768 + 16384 + 8192 + 16384 + kScal * 4;
 constexpr uint32_t OFF_SB = 2 * STAGE_BYTES;  // state (scaled) fp16, MN-major B: [128][64]
 constexpr uint32_t OFF_UT = OFF_SB + 16384;   // U~ fp16 [64][64]
 constexpr uint32_t OFF_US = OFF_UT + 8192;    // U~s fp16 [64][64]
-constexpr uint32_t OFF_RED = OFF_US + 8192;   // CTA max reduction (4 floats)
+constexpr uint32_t OFF_RED = OFF_US + 8192;   // CTA max reduction (8 floats)
 constexpr uint32_t OFF_BAR = OFF_RED + 64;    // mbarriers + TMEM address
 constexpr uint32_t SCAN_TC_SMEM = OFF_BAR + 128 + 1024;
 static_assert(ST_SC + kScal * 4 <= STAGE_BYTES, "stage layout");
@@ -68,16 +71,16 @@ __device__ __forceinline__ uint32_t pack2h(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// 64 fp32 values as one fp16 row of a 128-byte swizzled tile.
-__device__ __forceinline__ void store_row_f16(uint8_t* tile, int r, const float* v) {
+// 32 fp32 values as 16-byte chunks c0 .. c0 + 3 of row r of a 128-byte swizzled fp16 tile.
+__device__ __forceinline__ void store_half_row_f16(uint8_t* tile, int r, int c0, const float* v) {
 #pragma unroll
-  for (int c16 = 0; c16 < 8; ++c16) {
+  for (int j = 0; j < 4; ++j) {
     uint4 p;
-    p.x = pack2h(v[8 * c16 + 0], v[8 * c16 + 1]);
-    p.y = pack2h(v[8 * c16 + 2], v[8 * c16 + 3]);
-    p.z = pack2h(v[8 * c16 + 4], v[8 * c16 + 5]);
-    p.w = pack2h(v[8 * c16 + 6], v[8 * c16 + 7]);
-    *reinterpret_cast<uint4*>(tile + swz(r, c16)) = p;
+    p.x = pack2h(v[8 * j + 0], v[8 * j + 1]);
+    p.y = pack2h(v[8 * j + 2], v[8 * j + 3]);
+    p.z = pack2h(v[8 * j + 4], v[8 * j + 5]);
+    p.w = pack2h(v[8 * j + 6], v[8 * j + 7]);
+    *reinterpret_cast<uint4*>(tile + swz(r, c0 + j)) = p;
   }
 }
 
@@ -93,19 +96,19 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, in
   return false;
 }
 
-// 64 output values of one row with 16-byte stores.
+// 32 output values of one row with 16-byte stores.
 template <typename TO>
 __device__ __forceinline__ void store_row(TO* dst, const float* v);
 template <>
 __device__ __forceinline__ void store_row<float>(float* dst, const float* v) {
 #pragma unroll
-  for (int c = 0; c < 64; c += 4)
+  for (int c = 0; c < 32; c += 4)
     *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
 }
 template <>
 __device__ __forceinline__ void store_row<bf16>(bf16* dst, const float* v) {
 #pragma unroll
-  for (int c = 0; c < 64; c += 8) {
+  for (int c = 0; c < 32; c += 8) {
     uint4 p;
     __nv_bfloat162 h0 = __floats2bfloat162_rn(v[c], v[c + 1]);
     __nv_bfloat162 h1 = __floats2bfloat162_rn(v[c + 2], v[c + 3]);
@@ -237,41 +240,45 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = tid - 64;                       // 0..127
+    const int e = tid - 64;                       // 0..255
     const int row = 32 * (warp & 3) + lane;       // TMEM lane = d_k row of the state
-    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    const int half = (warp - 2) >> 2;             // columns 32 half .. 32 half + 31
+    const int cb = 32 * half;
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)cb;
     const bool p_rows = row >= 64;                // lanes 64-127: rows of P (token row - 64)
-    float S[64];
+    float S[32];
     float mx = 0.f;
     {
-      const float* src = h0 ? h0 + ((size_t)head * kD + row) * kD + c0 : nullptr;
+      const float* src = h0 ? h0 + ((size_t)head * kD + row) * kD + c0 + cb : nullptr;
 #pragma unroll
-      for (int c = 0; c < 64; c += 4) {
+      for (int c = 0; c < 32; c += 4) {
         const float4 t = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0, 0, 0, 0);
         S[c] = t.x; S[c + 1] = t.y; S[c + 2] = t.z; S[c + 3] = t.w;
         mx = fmaxf(mx, fmaxf(fmaxf(fabsf(t.x), fabsf(t.y)), fmaxf(fabsf(t.z), fabsf(t.w))));
       }
     }
-    for (int n = e; n < Nc; n += 128) mx = fmaxf(mx, Sg[(size_t)n * kScal + kScMaxU]);
+    for (int n = e; n < Nc; n += kEpi) mx = fmaxf(mx, Sg[(size_t)n * kScal + kScMaxU]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     if (lane == 0) red[warp - 2] = mx;
-    named_barrier(1, 128);
-    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    named_barrier(1, kEpi);
+    mx = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) mx = fmaxf(mx, red[w]);
     const int ex = mx > 0.f ? min(max(ilogbf(mx) - 7, -100), 100) : 0;
     const float sigma = ldexpf(1.f, -ex), inv_sigma = ldexpf(1.f, ex);
     float range = 0.f;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) {
+    for (int c = 0; c < 32; ++c) {
       S[c] *= sigma;
       range = fmaxf(range, fabsf(S[c]));
     }
-    store_row_f16(sm + OFF_SB, row, S);
+    store_half_row_f16(sm + OFF_SB, row, 4 * half, S);
     fence_proxy_async_smem();
-    named_barrier(1, 128);
+    named_barrier(1, kEpi);
     if (e == 0) mbar_arrive(&bar[B_S]);
 
-    float OQ[64];
+    float OQ[32];
     for (int n = 0; n < Nc; ++n) {
       const int s = n & 1;
       const uint8_t* st = sm + s * STAGE_BYTES;
@@ -279,7 +286,7 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       {  // every epilogue thread takes the same decision (no thread is left at a barrier)
         const bool ok = wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 105, abort_flag) &&
                         wait_or_abort(&bar[B_QP], n & 1, status, 106, abort_flag);
-        if (named_barrier_or(1, 128, !ok)) {
+        if (named_barrier_or(1, kEpi, !ok)) {
           *abort_flag = 1;
           break;
         }
@@ -287,23 +294,23 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       tc_fence_after();
       float fo = 0.f;
       if (p_rows) {
-        // U~ = sigma U - P and U~s = U~ fs for token r, written as fp16 operand rows
+        // U~ = sigma U - P and U~s = U~ fs for token r and this thread's 32 columns,
+        // written as fp16 operand rows
         const int r = row - 64;
         const float fs = sc[kC + r];
-        float P[64];
-        tmem_ld64(tl + TM_QP, P);
+        float P[32];
+        tmem_ld32(tl + TM_QP, P);
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const int box = c4 >> 3, ch = c4 & 7;  // 32 fp32 columns per swizzled box
-          const float4 u = *reinterpret_cast<const float4*>(st + ST_U + box * 8192 + swz(r, ch));
-          P[4 * c4 + 0] = fmaf(sigma, u.x, -P[4 * c4 + 0]);
-          P[4 * c4 + 1] = fmaf(sigma, u.y, -P[4 * c4 + 1]);
-          P[4 * c4 + 2] = fmaf(sigma, u.z, -P[4 * c4 + 2]);
-          P[4 * c4 + 3] = fmaf(sigma, u.w, -P[4 * c4 + 3]);
+        for (int ch = 0; ch < 8; ++ch) {  // U box `half` holds columns cb .. cb + 31
+          const float4 u = *reinterpret_cast<const float4*>(st + ST_U + half * 8192 + swz(r, ch));
+          P[4 * ch + 0] = fmaf(sigma, u.x, -P[4 * ch + 0]);
+          P[4 * ch + 1] = fmaf(sigma, u.y, -P[4 * ch + 1]);
+          P[4 * ch + 2] = fmaf(sigma, u.z, -P[4 * ch + 2]);
+          P[4 * ch + 3] = fmaf(sigma, u.w, -P[4 * ch + 3]);
         }
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
-          const float* v = P + 8 * c16;
+        for (int j = 0; j < 4; ++j) {
+          const float* v = P + 8 * j;
           uint4 pu, ps;
           pu.x = pack2h(v[0], v[1]);
           pu.y = pack2h(v[2], v[3]);
@@ -313,44 +320,44 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
           ps.y = pack2h(v[2] * fs, v[3] * fs);
           ps.z = pack2h(v[4] * fs, v[5] * fs);
           ps.w = pack2h(v[6] * fs, v[7] * fs);
-          const uint32_t off = swz(r, c16);
+          const uint32_t off = swz(r, 4 * half + j);
           *reinterpret_cast<uint4*>(sm + OFF_UT + off) = pu;
           *reinterpret_cast<uint4*>(sm + OFF_US + off) = ps;
         }
 #pragma unroll
-        for (int c = 0; c < 64; ++c) range = fmaxf(range, fabsf(P[c]));
+        for (int c = 0; c < 32; ++c) range = fmaxf(range, fabsf(P[c]));
       } else {
-        tmem_ld64(tl + TM_QP, OQ);  // O_q of token row
+        tmem_ld32(tl + TM_QP, OQ);  // O_q of token row, this thread's 32 columns
         fo = sc[row];
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_barrier(1, 128);
+      named_barrier(1, kEpi);
       if (e == 0) mbar_arrive(&bar[B_UT]);
 
       // the state update first: it is what the next chunk waits for
       {
         const bool ok = wait_or_abort(&bar[B_DS], n & 1, status, 107, abort_flag);
-        if (named_barrier_or(1, 128, !ok)) {
+        if (named_barrier_or(1, kEpi, !ok)) {
           *abort_flag = 1;
           break;
         }
       }
       tc_fence_after();
       {
-        float D[64];
-        tmem_ld64(tl + TM_DS, D);
+        float D[32];
+        tmem_ld32(tl + TM_DS, D);
         const float gc = sc[kScGC + row];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < 32; ++c) {
           S[c] = fmaf(gc, S[c], D[c]);
           range = fmaxf(range, fabsf(S[c]));
         }
       }
-      store_row_f16(sm + OFF_SB, row, S);
+      store_half_row_f16(sm + OFF_SB, row, 4 * half, S);
       fence_proxy_async_smem();
       tc_fence_before();
-      named_barrier(1, 128);
+      named_barrier(1, kEpi);
       if (e == 0) {
         mbar_arrive(&bar[B_S]);
         mbar_arrive(&bar[B_EMPTY0 + s]);  // U and the factors of the stage are read
@@ -360,23 +367,23 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       if (!p_rows) {
         if (!wait_or_abort(&bar[B_OA], n & 1, status, 108, abort_flag)) continue;
         tc_fence_after();
-        float OA[64];
-        tmem_ld64(tl + TM_OA, OA);
+        float OA[32];
+        tmem_ld32(tl + TM_OA, OA);
         tc_fence_before();
         const int t = n * kC + row;
         if (t < T) {
-          TO* dst = o + (((size_t)b * T + t) * Hv + hv) * kD + c0;
+          TO* dst = o + (((size_t)b * T + t) * Hv + hv) * kD + c0 + cb;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) OA[c] = (fo * OQ[c] + OA[c]) * inv_sigma;
+          for (int c = 0; c < 32; ++c) OA[c] = (fo * OQ[c] + OA[c]) * inv_sigma;
           store_row<TO>(dst, OA);
         }
       }
     }
     if (!(range <= kF16Max)) report_range(status);
     if (ht != nullptr && !*abort_flag) {
-      float* dst = ht + ((size_t)head * kD + row) * kD + c0;
+      float* dst = ht + ((size_t)head * kD + row) * kD + c0 + cb;
 #pragma unroll
-      for (int c = 0; c < 64; c += 4)
+      for (int c = 0; c < 32; c += 4)
         *reinterpret_cast<float4*>(dst + c) = make_float4(S[c] * inv_sigma, S[c + 1] * inv_sigma,
                                                           S[c + 2] * inv_sigma, S[c + 3] * inv_sigma);
     }
