@@ -38,6 +38,8 @@
 #include "common.cuh"
 #include "launch.h"
 #include "chunk_layout.cuh"
+#include "tc_ptx.cuh"
+#include "tmap.cuh"
 #include "warp_mma.cuh"
 
 namespace gdn {
@@ -90,16 +92,31 @@ __device__ __forceinline__ int row_exponent(float m) { return m > 0.f ? ilogbf(m
 
 // ---------------------------------------------------------------- prep kernel
 constexpr int LDX = 64 + 8;                  // f32 row stride of L and X (conflict-free float2)
-constexpr int P_KT = 0;                      // K tile  [64][LDT] bf16 (key head)
-constexpr int P_QT = P_KT + kC * LDT * 2;    // Q tile  (key head)
-constexpr int P_VT = P_QT + kC * LDT * 2;    // V tile  (value head)
-constexpr int P_L = P_VT + kC * LDT * 2;     // L [64][LDX] f32
+// K, Q, V tiles: [2 column halves][64 rows][128 B] bf16, 128-byte swizzled (TMA)
+constexpr int P_KT = 0;                      // K tile (key head)
+constexpr int P_QT = P_KT + 16384;           // Q tile (key head)
+constexpr int P_VT = P_QT + 16384;           // V tile (value head)
+constexpr int P_L = P_VT + 16384;            // L [64][LDX] f32
 constexpr int P_X = P_L + kC * LDX * 4;      // X = (I + L)^-1
 constexpr int LDB = 20;                      // f32 row stride of a 16 x 16 block product
 constexpr int P_T = P_X + kC * LDX * 4;      // block products, one [16][LDB] f32 per warp 0-2
 constexpr int P_VEC = P_T + 3 * 16 * LDB * 4; // rk, sq, G, beta, c1, 2^eq, 2^ek [64], misc
-constexpr int P_BYTES = P_VEC + 8 * 64 * 4;
+constexpr int P_BAR = P_VEC + 8 * 64 * 4;    // two mbarriers
+constexpr int P_BYTES = P_BAR + 16 + 1024;   // + alignment slack of the 1024-byte base
 static_assert(2 * (P_BYTES + 1024) <= 228 * 1024, "two prep CTAs per SM");
+
+// Byte offset of the 16-byte chunk j (0..15, columns 8j..8j+7) of row r in a
+// K / Q / V tile: column half j / 8 is a [64 rows][128 B] box written by TMA with
+// the 128-byte swizzle, which stores the 16-byte unit u of row r at u ^ (r % 8).
+__device__ __forceinline__ int swz(int r, int j) {
+  return ((j >> 3) << 13) + (r << 7) + (((j & 7) ^ (r & 7)) << 4);
+}
+
+// 4-D tensor maps over the bf16 inputs [B][T][H][128], boxes of 64 columns x 64
+// time steps of one head (rows past T read as zeros).
+struct PrepMaps {
+  CUtensorMap q, k, v;
+};
 
 // X = (I + L)^-1 for a strictly lower 64 x 64 fp32 L (row stride LDX) in shared
 // memory, by the whole CTA: the four 16 x 16 diagonal blocks by forward
@@ -174,14 +191,17 @@ __device__ void invert_unit_lower(const float* Lm, float* Xm, float* Tm, int tid
 
 template <bool PRE>
 __global__ void __launch_bounds__(kThreads, 2)
-wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
+wy_prep_kernel(const __grid_constant__ PrepMaps maps,
                const void* __restrict__ ga, const void* __restrict__ gb,
                const float* __restrict__ A_log, const float* __restrict__ dt_bias, int T, int Hk,
                int Hv, float scale, int l2, uint8_t* __restrict__ ws, WsLayout L, int* status) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  bf16* Kt = reinterpret_cast<bf16*>(sm + P_KT);
-  bf16* Qt = reinterpret_cast<bf16*>(sm + P_QT);
-  bf16* Vt = reinterpret_cast<bf16*>(sm + P_VT);
+  extern __shared__ __align__(1024) uint8_t sm_raw[];
+  // the swizzled tiles need a 1024-byte aligned base
+  uint8_t* sm = sm_raw + ((1024u - (tc::smem_u32(sm_raw) & 1023u)) & 1023u);
+  const uint8_t* Kt = sm + P_KT;
+  const uint8_t* Qt = sm + P_QT;
+  const uint8_t* Vt = sm + P_VT;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + P_BAR);  // [0] K and Q, [1] V
   float* Lm = reinterpret_cast<float*>(sm + P_L);
   float* Xm = reinterpret_cast<float*>(sm + P_X);
   float* Tm = reinterpret_cast<float*>(sm + P_T);
@@ -203,19 +223,25 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
   const int t0 = n * kC, nv = min(kC, T - t0);
   float range = 0.f;  // largest magnitude this thread converted to fp16
 
-  // 1. raw K, Q tiles of the key head and the V tile of this value head (rows
-  //    past the end of the sequence are zeros)
-  for (int i = tid; i < 3 * kC * 16; i += kThreads) {
-    const int which = i >> 10, r = (i >> 4) & 63, c16 = i & 15;
-    const bool ok = r < nv;
-    size_t off = 0;
-    if (ok)
-      off = which < 2 ? ((((size_t)b * T + t0 + r) * Hk + hk) * kD + c16 * 8)
-                      : ((((size_t)b * T + t0 + r) * Hv + hv) * kD + c16 * 8);
-    bf16* dst = (which == 0 ? Kt : (which == 1 ? Qt : Vt)) + r * LDT + c16 * 8;
-    cp16(dst, (which == 0 ? k : (which == 1 ? q : v)) + off, ok ? 16 : 0);
+  // 1. raw K, Q tiles of the key head (barrier 0), then the V tile of this value
+  //    head (barrier 1, only waited for before U), by TMA; rows past the end of
+  //    the sequence read as zeros
+  if (tid == 0) {
+    tc::mbar_init(&bar[0], 1);
+    tc::mbar_init(&bar[1], 1);
+    tc::fence_mbar_init();
+    tc::mbar_arrive_expect_tx(&bar[0], 4 * 8192);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      tc::tma_load_4d(sm + P_KT + h * 8192, &maps.k, &bar[0], 64 * h, hk, t0, b);
+      tc::tma_load_4d(sm + P_QT + h * 8192, &maps.q, &bar[0], 64 * h, hk, t0, b);
+    }
+    tc::mbar_arrive_expect_tx(&bar[1], 2 * 8192);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      tc::tma_load_4d(sm + P_VT + h * 8192, &maps.v, &bar[1], 64 * h, hv, t0, b);
   }
-  cp_commit();
+  __syncthreads();  // the barriers are initialised
 
   // 2. gates (zero past the end of the sequence) and their in-chunk prefix sums,
   //    while the tiles land
@@ -241,19 +267,25 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
     Gs[tid] = g;
     bet[tid] = be;
   }
-  cp_wait<0>();
-  __syncthreads();
+  // bounded wait for K and Q; all threads leave together if any wait expired
+  // (after the V copy has landed, so no copy is left writing this CTA's memory)
+  if (__syncthreads_or(!tc::mbar_wait(&bar[0], 0, status, 111))) {
+    tc::mbar_wait(&bar[1], 0, nullptr, 0, 1u << 20);
+    return;
+  }
   if (tid >= 32 && tid < kC) Gs[tid] += misc[0];
 
   //    L2 norms: rk = 1 / |k|, sq = scale / |q|, and the row exponents of the
-  //    fp16 copies (two threads per row)
+  //    fp16 copies (two threads per row, thread h on column half h; its m-th
+  //    read is chunk m ^ 4h of the half, so the 8 lanes of one 16-byte load
+  //    phase touch 8 distinct bank groups)
   {
     const int which = tid >> 7, r = (tid & 127) >> 1, h = tid & 1;
-    const bf16* row = (which ? Qt : Kt) + r * LDT + h * 8;  // 16-byte chunks h, h + 2, ...
+    const uint8_t* tile = which ? Qt : Kt;
     float ss = 0.f, mx = 0.f;
 #pragma unroll
-    for (int c = 0; c < 128; c += 16) {
-      const uint4 u = *reinterpret_cast<const uint4*>(row + c);
+    for (int m = 0; m < 8; ++m) {
+      const uint4 u = *reinterpret_cast<const uint4*>(tile + swz(r, 8 * h + (m ^ (4 * h))));
       const float2 f0 = unpack2(u.x), f1 = unpack2(u.y), f2 = unpack2(u.z), f3 = unpack2(u.w);
       ss += f0.x * f0.x + f0.y * f0.y + f1.x * f1.x + f1.y * f1.y + f2.x * f2.x + f2.y * f2.y +
             f3.x * f3.x + f3.y * f3.y;
@@ -277,17 +309,18 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
     // fp16 copies of the raw rows, row-scaled by 2^-e (written once per key head)
     if (blockIdx.x == 0) {
       __half* dst = reinterpret_cast<__half*>(ws + (which ? L.qh : L.kh)) +
-                    ((size_t)blockIdx.z * Tp + t0 + r) * kD + h * 8;
+                    ((size_t)blockIdx.z * Tp + t0 + r) * kD;
 #pragma unroll
-      for (int c = 0; c < 128; c += 16) {
-        const uint4 u = *reinterpret_cast<const uint4*>(row + c);
+      for (int m = 0; m < 8; ++m) {
+        const int j = 8 * h + (m ^ (4 * h));
+        const uint4 u = *reinterpret_cast<const uint4*>(tile + swz(r, j));
         const float2 f0 = unpack2(u.x), f1 = unpack2(u.y), f2 = unpack2(u.z), f3 = unpack2(u.w);
         uint4 o;
         o.x = pack2h(f0.x * down, f0.y * down);
         o.y = pack2h(f1.x * down, f1.y * down);
         o.z = pack2h(f2.x * down, f2.y * down);
         o.w = pack2h(f3.x * down, f3.y * down);
-        *reinterpret_cast<uint4*>(dst + c) = o;
+        *reinterpret_cast<uint4*>(dst + 8 * j) = o;
       }
     }
   }
@@ -301,16 +334,16 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
   {
     const int mt = warp & 3;
     const bool isq = warp >= 4;
-    const bf16* At = isq ? Qt : Kt;
+    const uint8_t* At = isq ? Qt : Kt;
     float acc[8][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       uint32_t a[4];
-      ldsm_x4(a, At + (16 * mt + lrow_a(lane)) * LDT + 16 * ks + lcol_a(lane));
+      ldsm_x4(a, At + swz(16 * mt + lrow_a(lane), 2 * ks + (lcol_a(lane) >> 3)));
 #pragma unroll
       for (int np = 0; np < 4; ++np) {
         uint32_t bb[4];
-        ldsm_x4(bb, Kt + (16 * np + lrow_b(lane)) * LDT + 16 * ks + lcol_b(lane));
+        ldsm_x4(bb, Kt + swz(16 * np + lrow_b(lane), 2 * ks + (lcol_b(lane) >> 3)));
         mma_bf16(acc[2 * np], a, bb[0], bb[1]);
         mma_bf16(acc[2 * np + 1], a, bb[2], bb[3]);
       }
@@ -343,7 +376,8 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
       }
     }
   }
-  __syncthreads();
+  // bounded wait for V (landed long ago in the normal case), uniform exit
+  if (__syncthreads_or(!tc::mbar_wait(&bar[1], 0, status, 112))) return;
 
   // 4. X = (I + L)^-1
   invert_unit_lower(Lm, Xm, Tm, tid, warp, g8, t4);
@@ -371,11 +405,11 @@ wy_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf1
       split2(x10.x * f0, x10.y * f1, ah[1], al[1]);
       split2(x01.x * f2, x01.y * f3, ah[2], al[2]);
       split2(x11.x * f2, x11.y * f3, ah[3], al[3]);
-      const bf16* Bm = which ? Vt : Kt;
+      const uint8_t* Bm = which ? Vt : Kt;
 #pragma unroll
       for (int np = 0; np < 4; ++np) {
         uint32_t bb[4];
-        ldsm_x4_t(bb, Bm + (16 * ks + lrow_a(lane)) * LDT + nb + 16 * np + lcol_a(lane));
+        ldsm_x4_t(bb, Bm + swz(16 * ks + lrow_a(lane), (nb >> 3) + 2 * np + (lcol_a(lane) >> 3)));
         mma_bf16(acc[2 * np], ah, bb[0], bb[1]);
         mma_bf16(acc[2 * np + 1], ah, bb[2], bb[3]);
         if (which) {
@@ -863,13 +897,15 @@ cudaError_t launch_t(const ChunkArgs& a, bool gdn2, uint8_t* ws, const WsLayout&
         static_cast<const bf16*>(a.v), a.a, a.b, a.w, a.A_log, a.dt_bias, a.T, a.Hv, a.scale, l2,
         ws, L, status);
   } else {
+    PrepMaps m;
+    if (!make_map_bthd(&m.q, a.q, a.B, a.T, a.Hk) || !make_map_bthd(&m.k, a.k, a.B, a.T, a.Hk) ||
+        !make_map_bthd(&m.v, a.v, a.B, a.T, a.Hv))
+      return cudaErrorInvalidValue;
     auto prep = pre ? wy_prep_kernel<true> : wy_prep_kernel<false>;
     e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_BYTES);
     if (e != cudaSuccess) return e;
     prep<<<dim3(a.Hv / a.Hk, Nc, a.B * a.Hk), kThreads, P_BYTES, s>>>(
-        static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
-        static_cast<const bf16*>(a.v), a.a, a.b, a.A_log, a.dt_bias, a.T, a.Hk, a.Hv, a.scale, l2,
-        ws, L, status);
+        m, a.a, a.b, a.A_log, a.dt_bias, a.T, a.Hk, a.Hv, a.scale, l2, ws, L, status);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -21,13 +21,11 @@
 // Hand-offs go through mbarriers; every wait is bounded and an expired wait ends
 // the kernel through the status word (GDN_ERR_TIMEOUT) after its copies and
 // tensor-core work in flight have drained.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include "chunk_layout.cuh"
 #include "common.cuh"
 #include "launch.h"
 #include "tc_ptx.cuh"
+#include "tmap.cuh"
 
 namespace gdn {
 namespace {
@@ -398,45 +396,18 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 2-D map over a [rows][cols] row-major region, boxes of [64 rows][128 bytes], 128-byte swizzle.
-bool make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base,
-              CUtensorMapDataType dt, int elem_bytes, uint64_t cols, uint64_t rows) {
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * elem_bytes};
-  const cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), 64};
-  const cuuint32_t es[2] = {1, 1};
-  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
 template <typename TO>
 cudaError_t launch_t(const ChunkArgs& a, const WsLayout& L, const uint8_t* ws, int* status,
                      cudaStream_t s) {
-  auto enc = encode_fn();
-  if (enc == nullptr) return cudaErrorNotSupported;
+  if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
   const uint64_t Tp = (uint64_t)((a.T + kC - 1) / kC) * kC;
   const uint64_t rv = (uint64_t)a.B * a.Hv * Tp, rk = (uint64_t)a.B * a.Hk * Tp;
   ScanMaps m;
-  if (!make_map(enc, &m.q, ws + L.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rk) ||
-      !make_map(enc, &m.w, ws + L.w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rv) ||
-      !make_map(enc, &m.k, ws + L.kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rk) ||
-      !make_map(enc, &m.a, ws + L.a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kC, rv) ||
-      !make_map(enc, &m.u, ws + L.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kD, rv))
+  if (!make_map_rows(&m.q, ws + L.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rk) ||
+      !make_map_rows(&m.w, ws + L.w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rv) ||
+      !make_map_rows(&m.k, ws + L.kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rk) ||
+      !make_map_rows(&m.a, ws + L.a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kC, rv) ||
+      !make_map_rows(&m.u, ws + L.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kD, rv))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(state_scan_tc_kernel<TO>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_TC_SMEM);
