@@ -38,85 +38,18 @@
 #include "common.cuh"
 #include "launch.h"
 #include "chunk_layout.cuh"
-#include "tc_ptx.cuh"
-#include "tmap.cuh"
 #include "warp_mma.cuh"
+#include "wy_common.cuh"
 
 namespace gdn {
 namespace {
 
 using namespace wm;
+using namespace wy;
 using bf16 = __nv_bfloat16;
 
 constexpr int kThreads = 256;  // 8 warps
 constexpr int LDT = kD + 8;    // 16-bit row stride of 128-wide tiles (272 B: ldmatrix conflict-free)
-
-// x = hi + lo with hi = rn_bf16(x), lo = rn_bf16(x - hi), for a pair of values.
-__device__ __forceinline__ void split2(float x, float y, uint32_t& hi, uint32_t& lo) {
-  hi = pack2(x, y);
-  const float2 h = unpack2(hi);
-  lo = pack2(x - h.x, y - h.y);
-}
-
-// A fragment (16 x 16, row-major) of an fp32 matrix M (row stride ld) at
-// (r0, c0), as bf16 hi + lo parts.
-__device__ __forceinline__ void frag_a_split(const float* M, int ld, int r0, int c0, int g8, int t4,
-                                             uint32_t (&hi)[4], uint32_t (&lo)[4]) {
-  const float2 x00 = *reinterpret_cast<const float2*>(M + (r0 + g8) * ld + c0 + 2 * t4);
-  const float2 x10 = *reinterpret_cast<const float2*>(M + (r0 + g8 + 8) * ld + c0 + 2 * t4);
-  const float2 x01 = *reinterpret_cast<const float2*>(M + (r0 + g8) * ld + c0 + 2 * t4 + 8);
-  const float2 x11 = *reinterpret_cast<const float2*>(M + (r0 + g8 + 8) * ld + c0 + 2 * t4 + 8);
-  split2(x00.x, x00.y, hi[0], lo[0]);
-  split2(x10.x, x10.y, hi[1], lo[1]);
-  split2(x01.x, x01.y, hi[2], lo[2]);
-  split2(x11.x, x11.y, hi[3], lo[3]);
-}
-// B fragment (16 x 8, k x n) of an fp32 matrix M (row = k) at (k0, n0), split.
-__device__ __forceinline__ void frag_b_split(const float* M, int ld, int k0, int n0, int g8, int t4,
-                                             uint32_t (&hi)[2], uint32_t (&lo)[2]) {
-  const float* p = M + (k0 + 2 * t4) * ld + n0 + g8;
-  split2(p[0], p[ld], hi[0], lo[0]);
-  split2(p[8 * ld], p[9 * ld], hi[1], lo[1]);
-}
-// D += A B for split operands, the lo x lo term dropped (about 2^-16 relative).
-__device__ __forceinline__ void mma_split3(float (&d)[4], const uint32_t (&ah)[4],
-                                           const uint32_t (&al)[4], const uint32_t (&bh)[2],
-                                           const uint32_t (&bl)[2]) {
-  mma_bf16(d, ah, bh[0], bh[1]);
-  mma_bf16(d, ah, bl[0], bl[1]);
-  mma_bf16(d, al, bh[0], bh[1]);
-}
-
-// Exponent e with (max |row|) * 2^-e in [1, 2) (e = 0 for a zero row).
-__device__ __forceinline__ int row_exponent(float m) { return m > 0.f ? ilogbf(m) : 0; }
-
-// ---------------------------------------------------------------- prep kernel
-constexpr int LDX = 64 + 8;                  // f32 row stride of L and X (conflict-free float2)
-// K, Q, V tiles: [2 column halves][64 rows][128 B] bf16, 128-byte swizzled (TMA)
-constexpr int P_KT = 0;                      // K tile (key head)
-constexpr int P_QT = P_KT + 16384;           // Q tile (key head)
-constexpr int P_VT = P_QT + 16384;           // V tile (value head)
-constexpr int P_L = P_VT + 16384;            // L [64][LDX] f32
-constexpr int P_X = P_L + kC * LDX * 4;      // X = (I + L)^-1
-constexpr int LDB = 20;                      // f32 row stride of a 16 x 16 block product
-constexpr int P_T = P_X + kC * LDX * 4;      // block products, one [16][LDB] f32 per warp 0-2
-constexpr int P_VEC = P_T + 3 * 16 * LDB * 4; // rk, sq, G, beta, c1, 2^eq, 2^ek [64], misc
-constexpr int P_BAR = P_VEC + 8 * 64 * 4;    // two mbarriers
-constexpr int P_BYTES = P_BAR + 16 + 1024;   // + alignment slack of the 1024-byte base
-static_assert(2 * (P_BYTES + 1024) <= 228 * 1024, "two prep CTAs per SM");
-
-// Byte offset of the 16-byte chunk j (0..15, columns 8j..8j+7) of row r in a
-// K / Q / V tile: column half j / 8 is a [64 rows][128 B] box written by TMA with
-// the 128-byte swizzle, which stores the 16-byte unit u of row r at u ^ (r % 8).
-__device__ __forceinline__ int swz(int r, int j) {
-  return ((j >> 3) << 13) + (r << 7) + (((j & 7) ^ (r & 7)) << 4);
-}
-
-// 4-D tensor maps over the bf16 inputs [B][T][H][128], boxes of 64 columns x 64
-// time steps of one head (rows past T read as zeros).
-struct PrepMaps {
-  CUtensorMap q, k, v;
-};
 
 // X = (I + L)^-1 for a strictly lower 64 x 64 fp32 L (row stride LDX) in shared
 // memory, by the whole CTA: the four 16 x 16 diagonal blocks by forward
@@ -186,284 +119,6 @@ __device__ void invert_unit_lower(const float* Lm, float* Xm, float* Tm, int tid
       }
     }
     __syncthreads();
-  }
-}
-
-template <bool PRE>
-__global__ void __launch_bounds__(kThreads, 2)
-wy_prep_kernel(const __grid_constant__ PrepMaps maps,
-               const void* __restrict__ ga, const void* __restrict__ gb,
-               const float* __restrict__ A_log, const float* __restrict__ dt_bias, int T, int Hk,
-               int Hv, float scale, int l2, uint8_t* __restrict__ ws, WsLayout L, int* status) {
-  extern __shared__ __align__(1024) uint8_t sm_raw[];
-  // the swizzled tiles need a 1024-byte aligned base
-  uint8_t* sm = sm_raw + ((1024u - (tc::smem_u32(sm_raw) & 1023u)) & 1023u);
-  const uint8_t* Kt = sm + P_KT;
-  const uint8_t* Qt = sm + P_QT;
-  const uint8_t* Vt = sm + P_VT;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + P_BAR);  // [0] K and Q, [1] V
-  float* Lm = reinterpret_cast<float*>(sm + P_L);
-  float* Xm = reinterpret_cast<float*>(sm + P_X);
-  float* Tm = reinterpret_cast<float*>(sm + P_T);
-  float* rk = reinterpret_cast<float*>(sm + P_VEC);
-  float* sq = rk + 64;
-  float* Gs = sq + 64;
-  float* bet = Gs + 64;
-  float* c1 = bet + 64;
-  float* pq = c1 + 64;   // 2^e of the stored Q row
-  float* pk = pq + 64;   // 2^e of the stored K row
-  float* misc = pk + 64; // [0] prefix carry, [8..15] per-warp max |U|
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g8 = lane >> 2, t4 = lane & 3;
-  const int G = Hv / Hk;
-  const int n = blockIdx.y, Nc = gridDim.y, Tp = Nc * kC;
-  const int b = blockIdx.z / Hk, hk = blockIdx.z % Hk, hv = hk * G + blockIdx.x;
-  const size_t head = (size_t)b * Hv + hv;
-  const int t0 = n * kC, nv = min(kC, T - t0);
-  float range = 0.f;  // largest magnitude this thread converted to fp16
-
-  // 1. raw K, Q tiles of the key head (barrier 0), then the V tile of this value
-  //    head (barrier 1, only waited for before U), by TMA; rows past the end of
-  //    the sequence read as zeros
-  if (tid == 0) {
-    tc::mbar_init(&bar[0], 1);
-    tc::mbar_init(&bar[1], 1);
-    tc::fence_mbar_init();
-    tc::mbar_arrive_expect_tx(&bar[0], 4 * 8192);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      tc::tma_load_4d(sm + P_KT + h * 8192, &maps.k, &bar[0], 64 * h, hk, t0, b);
-      tc::tma_load_4d(sm + P_QT + h * 8192, &maps.q, &bar[0], 64 * h, hk, t0, b);
-    }
-    tc::mbar_arrive_expect_tx(&bar[1], 2 * 8192);
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-      tc::tma_load_4d(sm + P_VT + h * 8192, &maps.v, &bar[1], 64 * h, hv, t0, b);
-  }
-  __syncthreads();  // the barriers are initialised
-
-  // 2. gates (zero past the end of the sequence) and their in-chunk prefix sums,
-  //    while the tiles land
-  if (tid < kC) {
-    float g = 0.f, be = 0.f;
-    if (tid < nv) {
-      const size_t idx = ((size_t)b * T + t0 + tid) * Hv + hv;
-      if (PRE) {
-        g = reinterpret_cast<const float*>(ga)[idx];
-        be = reinterpret_cast<const float*>(gb)[idx];
-      } else {
-        g = gdn_log_decay(__bfloat162float(reinterpret_cast<const bf16*>(ga)[idx]), A_log[hv],
-                          dt_bias[hv]);
-        be = sigmoid_f(__bfloat162float(reinterpret_cast<const bf16*>(gb)[idx]));
-      }
-    }
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, g, off);
-      if (lane >= off) g += y;
-    }
-    if (tid == 31) misc[0] = g;
-    Gs[tid] = g;
-    bet[tid] = be;
-  }
-  // bounded wait for K and Q; all threads leave together if any wait expired
-  // (after the V copy has landed, so no copy is left writing this CTA's memory)
-  if (__syncthreads_or(!tc::mbar_wait(&bar[0], 0, status, 111))) {
-    tc::mbar_wait(&bar[1], 0, nullptr, 0, 1u << 20);
-    return;
-  }
-  if (tid >= 32 && tid < kC) Gs[tid] += misc[0];
-
-  //    L2 norms: rk = 1 / |k|, sq = scale / |q|, and the row exponents of the
-  //    fp16 copies (two threads per row, thread h on column half h; its m-th
-  //    read is chunk m ^ 4h of the half, so the 8 lanes of one 16-byte load
-  //    phase touch 8 distinct bank groups)
-  {
-    const int which = tid >> 7, r = (tid & 127) >> 1, h = tid & 1;
-    const uint8_t* tile = which ? Qt : Kt;
-    float ss = 0.f, mx = 0.f;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const uint4 u = *reinterpret_cast<const uint4*>(tile + swz(r, 8 * h + (m ^ (4 * h))));
-      const float2 f0 = unpack2(u.x), f1 = unpack2(u.y), f2 = unpack2(u.z), f3 = unpack2(u.w);
-      ss += f0.x * f0.x + f0.y * f0.y + f1.x * f1.x + f1.y * f1.y + f2.x * f2.x + f2.y * f2.y +
-            f3.x * f3.x + f3.y * f3.y;
-      mx = fmaxf(mx, fmaxf(fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y))),
-                           fmaxf(fmaxf(fabsf(f2.x), fabsf(f2.y)), fmaxf(fabsf(f3.x), fabsf(f3.y)))));
-    }
-    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    const int e = row_exponent(mx);
-    const float up = ldexpf(1.f, e), down = ldexpf(1.f, -e);  // exact powers of 2
-    if (h == 0) {
-      const float inv = l2 ? rsqrtf(ss + 1e-6f) : 1.f;
-      if (which) {
-        sq[r] = inv * scale;
-        pq[r] = up;
-      } else {
-        rk[r] = inv;
-        pk[r] = up;
-      }
-    }
-    // fp16 copies of the raw rows, row-scaled by 2^-e (written once per key head)
-    if (blockIdx.x == 0) {
-      __half* dst = reinterpret_cast<__half*>(ws + (which ? L.qh : L.kh)) +
-                    ((size_t)blockIdx.z * Tp + t0 + r) * kD;
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int j = 8 * h + (m ^ (4 * h));
-        const uint4 u = *reinterpret_cast<const uint4*>(tile + swz(r, j));
-        const float2 f0 = unpack2(u.x), f1 = unpack2(u.y), f2 = unpack2(u.z), f3 = unpack2(u.w);
-        uint4 o;
-        o.x = pack2h(f0.x * down, f0.y * down);
-        o.y = pack2h(f1.x * down, f1.y * down);
-        o.z = pack2h(f2.x * down, f2.y * down);
-        o.w = pack2h(f3.x * down, f3.y * down);
-        *reinterpret_cast<uint4*>(dst + 8 * j) = o;
-      }
-    }
-  }
-  __syncthreads();
-  if (tid < kC) c1[tid] = bet[tid] * __expf(Gs[tid]) * rk[tid];  // column factor of W
-
-  // 3. Gram matrices on the tensor cores with the gates applied in registers:
-  //    warps 0-3: L = strictly lower (beta_r rk_r rk_c e^(G_r - G_c) k_r.k_c) -> smem
-  //    warps 4-7: A_qk = lower incl. diagonal (sq_r rk_c e^(G_r - G_c) q_r.k_c),
-  //               stored to the workspace in fp16 (|A_qk| <= scale for unit rows)
-  {
-    const int mt = warp & 3;
-    const bool isq = warp >= 4;
-    const uint8_t* At = isq ? Qt : Kt;
-    float acc[8][4] = {};
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      uint32_t a[4];
-      ldsm_x4(a, At + swz(16 * mt + lrow_a(lane), 2 * ks + (lcol_a(lane) >> 3)));
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t bb[4];
-        ldsm_x4(bb, Kt + swz(16 * np + lrow_b(lane), 2 * ks + (lcol_b(lane) >> 3)));
-        mma_bf16(acc[2 * np], a, bb[0], bb[1]);
-        mma_bf16(acc[2 * np + 1], a, bb[2], bb[3]);
-      }
-    }
-    const int ra = 16 * mt + g8, rb = ra + 8;
-    const float Ga = Gs[ra], Gb = Gs[rb];
-    const float fa = isq ? sq[ra] : bet[ra] * rk[ra];
-    const float fb = isq ? sq[rb] : bet[rb] * rk[rb];
-    __half* ag = reinterpret_cast<__half*>(ws + L.a) + (head * Tp + t0) * kC;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int c = 8 * nt + 2 * t4;
-      const float k0 = rk[c] * __expf(fminf(Ga - Gs[c], 0.f));
-      const float k1 = rk[c + 1] * __expf(fminf(Ga - Gs[c + 1], 0.f));
-      const float k2 = rk[c] * __expf(fminf(Gb - Gs[c], 0.f));
-      const float k3 = rk[c + 1] * __expf(fminf(Gb - Gs[c + 1], 0.f));
-      if (!isq) {
-        *reinterpret_cast<float2*>(Lm + ra * LDX + c) =
-            make_float2(c < ra ? fa * k0 * acc[nt][0] : 0.f, c + 1 < ra ? fa * k1 * acc[nt][1] : 0.f);
-        *reinterpret_cast<float2*>(Lm + rb * LDX + c) =
-            make_float2(c < rb ? fb * k2 * acc[nt][2] : 0.f, c + 1 < rb ? fb * k3 * acc[nt][3] : 0.f);
-      } else {
-        const float x0 = c <= ra ? fa * k0 * acc[nt][0] : 0.f;
-        const float x1 = c + 1 <= ra ? fa * k1 * acc[nt][1] : 0.f;
-        const float x2 = c <= rb ? fb * k2 * acc[nt][2] : 0.f;
-        const float x3 = c + 1 <= rb ? fb * k3 * acc[nt][3] : 0.f;
-        range = fmaxf(range, fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3))));
-        *reinterpret_cast<uint32_t*>(ag + ra * kC + c) = pack2h(x0, x1);
-        *reinterpret_cast<uint32_t*>(ag + rb * kC + c) = pack2h(x2, x3);
-      }
-    }
-  }
-  // bounded wait for V (landed long ago in the normal case), uniform exit
-  if (__syncthreads_or(!tc::mbar_wait(&bar[1], 0, status, 112))) return;
-
-  // 4. X = (I + L)^-1
-  invert_unit_lower(Lm, Xm, Tm, tid, warp, g8, t4);
-
-  // 5. W = X diag(c1) K (stored in fp16) and U = X diag(beta) V (fp32, X diag(beta)
-  //    as bf16 hi + lo); the A fragments are formed from X in registers.
-  //    warp -> rows 16 (warp % 4), cols 64 (warp / 4)
-  const int mt = warp & 3, nb = 64 * (warp >> 2);
-  const int ra = 16 * mt + g8;
-  float umax = 0.f;
-#pragma unroll 1
-  for (int which = 0; which < 2; ++which) {
-    float acc[8][4] = {};
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const int ca = 16 * ks + 2 * t4;
-      const float2 x00 = *reinterpret_cast<const float2*>(Xm + ra * LDX + ca);
-      const float2 x10 = *reinterpret_cast<const float2*>(Xm + (ra + 8) * LDX + ca);
-      const float2 x01 = *reinterpret_cast<const float2*>(Xm + ra * LDX + ca + 8);
-      const float2 x11 = *reinterpret_cast<const float2*>(Xm + (ra + 8) * LDX + ca + 8);
-      const float* f = which ? bet : c1;
-      const float f0 = f[ca], f1 = f[ca + 1], f2 = f[ca + 8], f3 = f[ca + 9];
-      uint32_t ah[4], al[4];
-      split2(x00.x * f0, x00.y * f1, ah[0], al[0]);
-      split2(x10.x * f0, x10.y * f1, ah[1], al[1]);
-      split2(x01.x * f2, x01.y * f3, ah[2], al[2]);
-      split2(x11.x * f2, x11.y * f3, ah[3], al[3]);
-      const uint8_t* Bm = which ? Vt : Kt;
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t bb[4];
-        ldsm_x4_t(bb, Bm + swz(16 * ks + lrow_a(lane), (nb >> 3) + 2 * np + (lcol_a(lane) >> 3)));
-        mma_bf16(acc[2 * np], ah, bb[0], bb[1]);
-        mma_bf16(acc[2 * np + 1], ah, bb[2], bb[3]);
-        if (which) {
-          mma_bf16(acc[2 * np], al, bb[0], bb[1]);
-          mma_bf16(acc[2 * np + 1], al, bb[2], bb[3]);
-        }
-      }
-    }
-    if (which == 0) {
-      __half* dw = reinterpret_cast<__half*>(ws + L.w) + (head * Tp + t0) * kD;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const int c = nb + 8 * nt + 2 * t4;
-        range = fmaxf(range, fmaxf(fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][1])),
-                                   fmaxf(fabsf(acc[nt][2]), fabsf(acc[nt][3]))));
-        *reinterpret_cast<uint32_t*>(dw + (size_t)ra * kD + c) = pack2h(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<uint32_t*>(dw + (size_t)(ra + 8) * kD + c) =
-            pack2h(acc[nt][2], acc[nt][3]);
-      }
-    } else {
-      float* du = reinterpret_cast<float*>(ws + L.u) + (head * Tp + t0) * kD;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const int c = nb + 8 * nt + 2 * t4;
-        umax = fmaxf(umax, fmaxf(fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][1])),
-                                 fmaxf(fabsf(acc[nt][2]), fabsf(acc[nt][3]))));
-        *reinterpret_cast<float2*>(du + (size_t)ra * kD + c) = make_float2(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<float2*>(du + (size_t)(ra + 8) * kD + c) =
-            make_float2(acc[nt][2], acc[nt][3]);
-      }
-    }
-  }
-  if (!(range <= kF16Max)) report_range(status);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) umax = fmaxf(umax, __shfl_xor_sync(0xffffffffu, umax, o));
-  if (lane == 0) misc[8 + warp] = umax;
-  __syncthreads();
-
-  // 6. per-row factors of the scan: fo = gamma sq 2^eq, fs = rk 2^ek gamma_C / gamma,
-  //    gamma_C for every state row, and the largest |U| of the chunk
-  if (tid < 128) {
-    float* sc = reinterpret_cast<float*>(ws + L.scal) + (head * Nc + n) * kScal;
-    const float GC = Gs[kC - 1];
-    if (tid < kC) {
-      sc[tid] = __expf(Gs[tid]) * sq[tid] * pq[tid];
-      sc[kC + tid] = tid < nv ? rk[tid] * pk[tid] * __expf(GC - Gs[tid]) : 0.f;
-    }
-    sc[kScGC + tid] = __expf(GC);  // one decay for every state row
-    if (tid < 4) {
-      float m = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) m = fmaxf(m, misc[8 + w]);
-      sc[kScMaxU + tid] = tid == 0 ? m : 0.f;
-    }
   }
 }
 
@@ -896,19 +551,12 @@ cudaError_t launch_t(const ChunkArgs& a, bool gdn2, uint8_t* ws, const WsLayout&
         static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
         static_cast<const bf16*>(a.v), a.a, a.b, a.w, a.A_log, a.dt_bias, a.T, a.Hv, a.scale, l2,
         ws, L, status);
-  } else {
-    PrepMaps m;
-    if (!make_map_bthd(&m.q, a.q, a.B, a.T, a.Hk) || !make_map_bthd(&m.k, a.k, a.B, a.T, a.Hk) ||
-        !make_map_bthd(&m.v, a.v, a.B, a.T, a.Hv))
-      return cudaErrorInvalidValue;
-    auto prep = pre ? wy_prep_kernel<true> : wy_prep_kernel<false>;
-    e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_BYTES);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    prep<<<dim3(a.Hv / a.Hk, Nc, a.B * a.Hk), kThreads, P_BYTES, s>>>(
-        m, a.a, a.b, a.A_log, a.dt_bias, a.T, a.Hk, a.Hv, a.scale, l2, ws, L, status);
+  } else {
+    e = launch_prep_tc(a, ws, status, s);
+    if (e != cudaSuccess) return e;
   }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   return launch_scan_tc(a, ws, status, s);
 }
 

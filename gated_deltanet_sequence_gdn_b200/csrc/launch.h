@@ -37,6 +37,9 @@ cudaError_t launch_chunk_simt(const ChunkArgs& a, bool gdn2, cudaStream_t s);
 bool chunk_mma_supported(const ChunkArgs& a);
 size_t chunk_mma_workspace_bytes(int B, int T, int Hk, int Hv);
 cudaError_t launch_chunk_mma(const ChunkArgs& a, bool gdn2, void* workspace, cudaStream_t s);
+// The GDN prep of that path on the tcgen05 tensor cores (one CTA per chunk and
+// key head; writes the workspace the scan reads).
+cudaError_t launch_prep_tc(const ChunkArgs& a, void* workspace, int* status, cudaStream_t s);
 // The state scan of those paths on the tcgen05 tensor cores (reads the workspace
 // the prep kernel wrote on the same stream).
 cudaError_t launch_scan_tc(const ChunkArgs& a, const void* workspace, int* status, cudaStream_t s);
