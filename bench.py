@@ -218,7 +218,7 @@ def run_ours(args, rank, local_rank, world):
                 "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(achieved / pk["bf16_tflops"], 4),
                 "traffic": kernel_traffic("chunk_prefill_8k"),
-                "kernel": "gdn_chunk_fwd = wy_prep_kernel + state_scan_kernel (timed together)",
+                "kernel": "gdn_chunk_fwd = wy_prep_tc_kernel + state_scan_tc_kernel (timed together)",
                 "flop_per_launch": flop, "peak_src": pk["src"] + " burst bf16"}
 
     # ---- end to end through the public call, host buffers, copies inside the timed region
@@ -230,7 +230,7 @@ def run_ours(args, rank, local_rank, world):
         extra["gdn2_b4_4k"] = measure_gdn2(G, dev, stream, pk, args)
         extra["prefill_128k"] = measure_prefill(G, "prefill_128k", dev, stream, pk, args)
 
-    launches = 2 * args.steps  # wy_prep_kernel + state_scan_kernel per step
+    launches = 2 * args.steps  # wy_prep_tc_kernel + state_scan_tc_kernel per step
     line = {
         "metric": "GDN prefill tokens/s (chunk_gated_delta_rule) on 1 B200, % of roofline",
         "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

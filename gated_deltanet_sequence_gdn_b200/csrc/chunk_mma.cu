@@ -1,16 +1,15 @@
-// chunk_mma.cu -- bf16 chunkwise GDN forward (dk = dv = 128, chunk C = 64) on
-// the tensor cores, in two kernels:
+// chunk_mma.cu -- bf16 chunkwise GDN / Gated DeltaNet-2 forward (dk = dv = 128,
+// chunk C = 64) on the tensor cores, in two kernels per call:
 //
-//  wy_prep_kernel  : one CTA per (chunk, value head), parallel over the whole
-//      sequence; the CTAs of one GQA group are launched next to each other so
-//      their shared K / Q tiles come from L2.  Forms the Gram matrices K K^T and
-//      Q K^T (bf16 mma, fp32 accumulation) with the gates applied in registers:
-//      the in-chunk prefix sums G_r of the log-decays, the strictly lower
-//      L = diag(beta) (K^ K^^T o Gamma), X = (I + L)^-1 by blocked forward
-//      substitution in fp32, W = X diag(beta gamma) K^, U = X diag(beta) V and
-//      A_qk = tril(Q^ K^^T o Gamma) (diagonal included), written to the
-//      workspace with the per-row factors of the second kernel, together with
-//      fp16 copies of the raw Q and K tiles.
+//  the prep, parallel over the whole sequence:
+//    GDN   : wy_prep_tc_kernel (prep_tc.cu, tcgen05), one CTA per (chunk, key
+//            head) serving the value heads of its GQA group;
+//    GDN-2 : wy_prep2_kernel (this file), one CTA per (chunk, value head).
+//    Both form the in-chunk prefix sums G_r of the log-decays, the strictly
+//    lower L = diag(beta) (K^ K^^T o Gamma), X = (I + L)^-1 by blocked forward
+//    substitution in fp32, W = X diag(beta gamma) K^, U = X diag(beta) V and
+//    A_qk = tril(Q^ K^^T o Gamma) (diagonal included), written to the workspace
+//    with the per-row factors of the scan and fp16 copies of the raw Q and K rows.
 //  the state scan (scan_tc.cu, tcgen05): one CTA per (value head, 64-column
 //      half of d_v), sequential over the chunks with the fp32 state held in
 //      registers:  U~ = U - W S,  o = diag(gamma sq) Q S + A_qk U~,
