@@ -48,14 +48,14 @@ constexpr int S_V = S_KQ + 32768;   // 2 slots of V: [2 d-halves][64 rows][128 B
 constexpr int S_R = S_V + 32768;    // region, used in turn as:
 //   before the first head: fp16 q / k rows to store, [K, Q][2 d-halves][64][128 B]
 constexpr int S_XW = S_R;           //   W operand [64 rows][64 columns] bf16 (during the
-                                    //   inverse: its block products [3][16][LDB] f32)
+                                    //   inverse: its block products [4][16][LDB] f32)
 constexpr int S_XH = S_R + 8192;    //   U operand, bf16 hi part
 constexpr int S_XL = S_R + 16384;   //   U operand, bf16 lo part (before: A_qk to store,
                                     //   [64 rows][128 B] fp16)
 constexpr int S_LX = S_R + 24576;   //   L, then X in place: [64][LDX] f32
 constexpr int S_VEC = S_LX + kC * LDX * 4;
 static_assert(S_VEC >= S_R + 32768, "q / k staging");
-static_assert(3 * 16 * LDB * 4 <= 8192, "block products");
+static_assert(4 * 16 * LDB * 4 <= 8192, "block products");
 // rk, sq, 2^eq, 2^ek [64] (key head); G, beta [4 heads][64]; c1, lc, lk, lq [64]; misc [32]
 constexpr int S_BAR = S_VEC + (4 * 64 + 8 * 64 + 4 * 64 + 32) * 4;
 constexpr int PT_SMEM = S_BAR + 64 + 1024;  // 4 mbarriers + TMEM address; alignment slack
@@ -84,12 +84,35 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// One 16 x 8 tile (columns n0 .. n0 + 7) of sum_i A_i B_i over nk pairs of 16 x 16
+// fp32 blocks, A_i at (ar, ac[i]) of A (row stride lda) and B_i at (br[i], n0) of
+// B (row stride ldb), on the warp tensor cores with the operands as bf16 hi + lo.
+__device__ __forceinline__ void block_prod(const float* A, int lda, int ar, const int* ac,
+                                           const float* Bm, int ldb, const int* br, int nk, int n0,
+                                           int g8, int t4, float (&d)[4]) {
+  for (int i = 0; i < nk; ++i) {
+    uint32_t ah[4], al[4], bh[2], bl[2];
+    frag_a_split(A, lda, ar, ac[i], g8, t4, ah, al);
+    frag_b_split(Bm, ldb, br[i], n0, g8, t4, bh, bl);
+    mma_split3(d, ah, al, bh, bl);
+  }
+}
+// The 16 x 8 tile d to rows r0 .. r0 + 15, columns c0 .. c0 + 7 of M (row stride ld), scaled by s.
+__device__ __forceinline__ void store_tile(float* M, int ld, int r0, int c0, int g8, int t4,
+                                           const float (&d)[4], float s) {
+  *reinterpret_cast<float2*>(M + (r0 + g8) * ld + c0 + 2 * t4) = make_float2(s * d[0], s * d[1]);
+  *reinterpret_cast<float2*>(M + (r0 + g8 + 8) * ld + c0 + 2 * t4) = make_float2(s * d[2], s * d[3]);
+}
+
 // X = (I + L)^-1 in place for a strictly lower 64 x 64 fp32 L (row stride LDX,
-// zero upper triangle), by the whole CTA: the four 16 x 16 diagonal blocks by
-// forward substitution (thread = one column of one block), then block row by
-// block row on the warp tensor cores with the fp32 operands as bf16 hi + lo:
-// warp j < i forms T = sum_{k=j}^{i-1} L_ik X_kj and X_ij = -X_ii T.  Each write
-// waits at a barrier until every read of the L block it replaces is done.
+// zero upper triangle), by the whole CTA (8 warps), by recursive doubling over
+// 16 x 16 blocks (L_ij, X_ij):
+//   X_ii       : forward substitution, one thread per column of a diagonal block;
+//   32 x 32    : X_10 = -X_11 (L_10 X_00),  X_32 = -X_33 (L_32 X_22);
+//   64 x 64    : X_[2:4][0:2] = -X_[2:4][2:4] (L_[2:4][0:2] X_[0:2][0:2]),
+// each product stage one 16 x 8 output tile per warp, the intermediate products in Tm
+// (four [16][LDB] fp32 tiles).  Every write of a block waits at a barrier until the
+// reads of the L block it replaces are done.
 __device__ void invert_in_place(float* M, float* Tm, int tid, int warp, int g8, int t4) {
   float x[16];
   const int base = 16 * (tid >> 4), cc = tid & 15;
@@ -108,49 +131,43 @@ __device__ void invert_in_place(float* M, float* Tm, int tid, int warp, int g8, 
     for (int r = 0; r < 16; ++r) M[(base + r) * LDX + base + cc] = x[r];
   }
   __syncthreads();
-  for (int bi = 1; bi < 4; ++bi) {
-    const int bj = warp;
-    float* Tw = Tm + warp * 16 * LDB;
-    if (warp < bi) {
-      float t[2][4] = {};
-      for (int kb = bj; kb < bi; ++kb) {
-        uint32_t ah[4], al[4];
-        frag_a_split(M, LDX, 16 * bi, 16 * kb, g8, t4, ah, al);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          uint32_t bh[2], bl[2];
-          frag_b_split(M, LDX, 16 * kb, 16 * bj + 8 * nt, g8, t4, bh, bl);
-          mma_split3(t[nt], ah, al, bh, bl);
-        }
-      }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        *reinterpret_cast<float2*>(Tw + g8 * LDB + 8 * nt + 2 * t4) = make_float2(t[nt][0], t[nt][1]);
-        *reinterpret_cast<float2*>(Tw + (g8 + 8) * LDB + 8 * nt + 2 * t4) =
-            make_float2(t[nt][2], t[nt][3]);
-      }
-    }
-    __syncthreads();  // block row bi of L is read; T is visible
-    if (warp < bi) {
-      float xo[2][4] = {};
-      uint32_t ah[4], al[4];
-      frag_a_split(M, LDX, 16 * bi, 16 * bi, g8, t4, ah, al);
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        uint32_t bh[2], bl[2];
-        frag_b_split(Tw, LDB, 0, 8 * nt, g8, t4, bh, bl);
-        mma_split3(xo[nt], ah, al, bh, bl);
-      }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int c = 16 * bj + 8 * nt + 2 * t4;
-        *reinterpret_cast<float2*>(M + (16 * bi + g8) * LDX + c) = make_float2(-xo[nt][0], -xo[nt][1]);
-        *reinterpret_cast<float2*>(M + (16 * bi + g8 + 8) * LDX + c) =
-            make_float2(-xo[nt][2], -xo[nt][3]);
-      }
-    }
-    __syncthreads();
+  const int nt = warp & 1, n8 = 8 * nt;
+  // 32 x 32 blocks: T_0 = L_10 X_00, T_1 = L_32 X_22 (warps 0-3), then X_10, X_32
+  if (warp < 4) {
+    const int b = warp >> 1, o = 32 * b;  // block pair (0, 1) or (2, 3)
+    float d[4] = {};
+    const int ac[1] = {o}, br[1] = {o};
+    block_prod(M, LDX, o + 16, ac, M, LDX, br, 1, o + n8, g8, t4, d);
+    store_tile(Tm + b * 16 * LDB, LDB, 0, n8, g8, t4, d, 1.f);
   }
+  __syncthreads();
+  if (warp < 4) {
+    const int b = warp >> 1, o = 32 * b;
+    float d[4] = {};
+    const int ac[1] = {o + 16}, br[1] = {0};
+    block_prod(M, LDX, o + 16, ac, Tm + b * 16 * LDB, LDB, br, 1, n8, g8, t4, d);
+    store_tile(M, LDX, o + 16, o + n8, g8, t4, d, -1.f);
+  }
+  __syncthreads();
+  // 64 x 64: T_(ri, cj) = sum_{k=cj}^{1} L_(ri, k) X_(k, cj) for ri = 2, 3 and cj = 0, 1
+  const int t = warp >> 1, ri = 2 + (t >> 1), cj = t & 1;
+  {
+    float d[4] = {};
+    const int ac[2] = {16 * cj, 16}, br[2] = {16 * cj, 16};
+    block_prod(M, LDX, 16 * ri, ac, M, LDX, br, 2 - cj, 16 * cj + n8, g8, t4, d);
+    store_tile(Tm + t * 16 * LDB, LDB, 0, n8, g8, t4, d, 1.f);
+  }
+  __syncthreads();
+  //         X_(ri, cj) = -sum_{k=2}^{ri} X_(ri, k) T_(k, cj)
+  {
+    float d[4] = {};
+    for (int k = 2; k <= ri; ++k) {
+      const int ac[1] = {16 * k}, br[1] = {0};
+      block_prod(M, LDX, 16 * ri, ac, Tm + (2 * (k - 2) + cj) * 16 * LDB, LDB, br, 1, n8, g8, t4, d);
+    }
+    store_tile(M, LDX, 16 * ri, 16 * cj + n8, g8, t4, d, -1.f);
+  }
+  __syncthreads();
 }
 
 template <bool PRE>
