@@ -44,6 +44,9 @@ lib.gdn_gate_prep.argtypes = [_vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, 
 lib.gdn_chunk_fwd.argtypes = [_vp] * 8 + [_i] * 7 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
 lib.gdn2_chunk_fwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
 lib.gdn_chunk_fwd_noalloc.argtypes = [_vp] * 8 + [_i] * 7 + [_f, _i, _vp, _vp, _vp]
+lib.gdn_chunk_fwd_host.argtypes = [_vp] * 8 + [_i] * 7 + [_f, _i, _vp, _vp, _i, _vp, _sz, _vp]
+lib.gdn_chunk_fwd_host_workspace_bytes.argtypes = [_i] * 9
+lib.gdn_chunk_fwd_host_workspace_bytes.restype = _sz
 lib.gdn_recurrent_step.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _vp]
 lib.gdn_chunk_workspace_bytes.argtypes = [_i] * 7
 lib.gdn2_chunk_workspace_bytes.argtypes = [_i] * 6
@@ -53,7 +56,8 @@ lib.gdn_check_status.argtypes = [_vp]
 lib.gdn_status_string.argtypes = [_i]
 lib.gdn_status_string.restype = ctypes.c_char_p
 lib.gdn_version.argtypes = []
-for _fn in (lib.gdn_gate_prep, lib.gdn_chunk_fwd, lib.gdn_chunk_fwd_noalloc, lib.gdn2_chunk_fwd,
+for _fn in (lib.gdn_gate_prep, lib.gdn_chunk_fwd, lib.gdn_chunk_fwd_noalloc, lib.gdn_chunk_fwd_host,
+            lib.gdn2_chunk_fwd,
             lib.gdn_recurrent_step, lib.gdn_check_status, lib.gdn_version):
     _fn.restype = _i
 
@@ -83,6 +87,18 @@ def _p(t):
         return None
     if not t.is_cuda:
         raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _ph(t):
+    """Host pointer of a contiguous CPU tensor (None -> NULL); page-locked memory
+    (tensor.pin_memory()) gives asynchronous copies."""
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("tensor must live in host memory")
     if not t.is_contiguous():
         raise ValueError("tensor must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
@@ -190,6 +206,59 @@ def gdn_chunk_fwd_noalloc(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, s
                                      _p(h0), B, T, Hk, Hv, dk, dv, _dtype_code(dt), float(scale),
                                      flags, _p(o), _p(ht), _stream(stream)),
            "gdn_chunk_fwd_noalloc")
+    return o, ht
+
+
+def gdn_chunk_fwd_host_workspace_bytes(B, T, Hk, Hv, dk, dv, dtype, *, l2norm=True,
+                                       gates_precomputed=False, out_f32=False,
+                                       piece_tokens=0) -> int:
+    """Bytes of device scratch gdn_chunk_fwd_host needs for these sizes."""
+    flags = ((QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
+             | (OUT_F32 if out_f32 else 0))
+    return int(lib.gdn_chunk_fwd_host_workspace_bytes(B, T, Hk, Hv, dk, dv, _dtype_code(dtype),
+                                                      flags, piece_tokens))
+
+
+def gdn_chunk_fwd_host(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, scale=None,
+                       l2norm=True, gates_precomputed=False, out_f32=False, o=None, ht=None,
+                       want_ht=True, piece_tokens=0, dev_workspace=None, device=None,
+                       stream=None):
+    """gdn_chunk_fwd for host (CPU) tensors: the library copies the sequence to the
+    device piece by piece, overlapping the copies in, the compute and the copies
+    out.  Arguments as gdn_chunk_fwd, all CPU tensors (pin_memory() for
+    asynchronous copies); o / ht are CPU tensors (page-locked when allocated
+    here).  dev_workspace: a uint8 CUDA tensor of at least
+    gdn_chunk_fwd_host_workspace_bytes(...) bytes, allocated here when None.
+    Returns (o, ht) once the stream has completed."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dt = q.dtype
+    scale = dk ** -0.5 if scale is None else scale
+    _need(k, dt, q.shape, "k")
+    _need(v, dt, (B, T, Hv, dv), "v")
+    gdt = torch.float32 if gates_precomputed else dt
+    _need(a, gdt, (B, T, Hv), "a")
+    _need(b, gdt, (B, T, Hv), "b")
+    if h0 is not None:
+        _need(h0, torch.float32, (B, Hv, dk, dv), "h0")
+    odt = torch.float32 if out_f32 else dt
+    o = torch.empty((B, T, Hv, dv), dtype=odt).pin_memory() if o is None else o
+    _need(o, odt, (B, T, Hv, dv), "o")
+    if ht is None and want_ht:
+        ht = torch.empty((B, Hv, dk, dv), dtype=torch.float32).pin_memory()
+    flags = ((QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
+             | (OUT_F32 if out_f32 else 0))
+    need = lib.gdn_chunk_fwd_host_workspace_bytes(B, T, Hk, Hv, dk, dv, _dtype_code(dt), flags,
+                                                  piece_tokens)
+    if dev_workspace is None and need > 0:
+        dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        dev_workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    ws_bytes = 0 if dev_workspace is None else dev_workspace.numel() * dev_workspace.element_size()
+    st = _stream(stream)
+    _check(lib.gdn_chunk_fwd_host(_ph(q), _ph(k), _ph(v), _ph(a), _ph(b), _ph(A_log),
+                                  _ph(dt_bias), _ph(h0), B, T, Hk, Hv, dk, dv, _dtype_code(dt),
+                                  float(scale), flags, _ph(o), _ph(ht), int(piece_tokens),
+                                  _p(dev_workspace), ws_bytes, st), "gdn_chunk_fwd_host")
     return o, ht
 
 

@@ -159,6 +159,41 @@ int gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
                           int flags, void* o, float* ht, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_fwd_host -- gdn_chunk_fwd for inputs and outputs in host memory.
+ * The pages have no counterpart: this is this library's pipeline for data that
+ * starts and ends on the host.  The sequence is cut into pieces of
+ * piece_tokens tokens (a multiple of the 64-token chunk; <= 0 picks about
+ * T / 8); the inputs of one piece are copied to the device while the previous
+ * piece is computed and the output of the one before is copied back, on two
+ * copy streams of the library; the state is carried from piece to piece on the
+ * device, so the result is that of one gdn_chunk_fwd call (the pieces' chunk
+ * boundaries are the call's).
+ *   q, k, v, a, b, A_log, dt_bias, h0: host pointers, layouts and meaning as
+ *     for gdn_chunk_fwd (page-locked memory gives asynchronous copies; other
+ *     host memory is copied synchronously by the runtime).
+ *   o, ht: host pointers, written.
+ *   dev_ws / dev_ws_bytes: device scratch owned by the caller, 256-byte aligned,
+ *     at least gdn_chunk_fwd_host_workspace_bytes() bytes (two sets of piece
+ *     buffers, the state, the piece's chunk workspace) -> else GDN_ERR_WORKSPACE.
+ *   stream: the pieces are computed on it, and it completes only after every
+ *     copy of the call; the host buffers must stay valid until then.
+ *   Returns the first error of gdn_chunk_fwd for a piece (what was already
+ *   enqueued still completes on the stream), GDN_ERR_CUDA if a stream or event
+ *   of the pipeline could not be made.  T = 0 copies h0 to ht (or zeros) after
+ *   synchronising the stream.
+ */
+int gdn_chunk_fwd_host(const void* q, const void* k, const void* v, const void* a,
+                       const void* b, const float* A_log, const float* dt_bias,
+                       const float* h0, int B, int T, int Hk, int Hv, int dk, int dv,
+                       int dtype, float scale, int flags, void* o, float* ht,
+                       int piece_tokens, void* dev_ws, size_t dev_ws_bytes,
+                       gdn_stream_t stream);
+
+/* Device scratch bytes gdn_chunk_fwd_host needs (0 for invalid sizes). */
+size_t gdn_chunk_fwd_host_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv,
+                                          int dtype, int flags, int piece_tokens);
+
+/*
  * gdn_recurrent_step -- one-token decode step for N independent sequences
  * (recurrent_gated_delta_rule; "gated-deltanet-qwen3.5" inference branch,
  * conv_states and recurrent_states updated in place), fused with the causal
