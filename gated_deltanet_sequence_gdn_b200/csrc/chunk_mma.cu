@@ -50,77 +50,6 @@ using bf16 = __nv_bfloat16;
 constexpr int kThreads = 256;  // 8 warps
 constexpr int LDT = kD + 8;    // 16-bit row stride of 128-wide tiles (272 B: ldmatrix conflict-free)
 
-// X = (I + L)^-1 for a strictly lower 64 x 64 fp32 L (row stride LDX) in shared
-// memory, by the whole CTA: the four 16 x 16 diagonal blocks by forward
-// substitution (thread = one column of one block), then block row by block row
-// on the tensor cores with the fp32 operands as bf16 hi + lo: warp j < i
-// computes T = sum_{k=j}^{i-1} L_ik X_kj and X_ij = -X_ii T.  Ends with a barrier.
-__device__ void invert_unit_lower(const float* Lm, float* Xm, float* Tm, int tid, int warp, int g8,
-                                  int t4) {
-  if (tid < kC) {
-    const int base = 16 * (tid >> 4), cc = tid & 15;
-    float x[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float s = 0.f;
-#pragma unroll
-      for (int jj = 0; jj < r; ++jj) s = fmaf(Lm[(base + r) * LDX + base + jj], x[jj], s);
-      x[r] = r == cc ? 1.f : -s;  // rows above cc come out as zero
-    }
-#pragma unroll
-    for (int r = 0; r < 16; ++r) Xm[(base + r) * LDX + base + cc] = x[r];
-  } else {
-    for (int i = tid - kC; i < 6 * 256; i += kThreads - kC) {
-      const int blk = i >> 8, e = i & 255;  // blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
-      const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-      const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-      Xm[(16 * bi + (e >> 4)) * LDX + 16 * bj + (e & 15)] = 0.f;
-    }
-  }
-  __syncthreads();
-  for (int bi = 1; bi < 4; ++bi) {
-    if (warp < bi) {
-      const int bj = warp;
-      float* Tw = Tm + warp * 16 * LDB;
-      float t[2][4] = {};
-      for (int kb = bj; kb < bi; ++kb) {
-        uint32_t ah[4], al[4];
-        frag_a_split(Lm, LDX, 16 * bi, 16 * kb, g8, t4, ah, al);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          uint32_t bh[2], bl[2];
-          frag_b_split(Xm, LDX, 16 * kb, 16 * bj + 8 * nt, g8, t4, bh, bl);
-          mma_split3(t[nt], ah, al, bh, bl);
-        }
-      }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        *reinterpret_cast<float2*>(Tw + g8 * LDB + 8 * nt + 2 * t4) = make_float2(t[nt][0], t[nt][1]);
-        *reinterpret_cast<float2*>(Tw + (g8 + 8) * LDB + 8 * nt + 2 * t4) =
-            make_float2(t[nt][2], t[nt][3]);
-      }
-      __syncwarp();
-      float x[2][4] = {};
-      uint32_t ah[4], al[4];
-      frag_a_split(Xm, LDX, 16 * bi, 16 * bi, g8, t4, ah, al);
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        uint32_t bh[2], bl[2];
-        frag_b_split(Tw, LDB, 0, 8 * nt, g8, t4, bh, bl);
-        mma_split3(x[nt], ah, al, bh, bl);
-      }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int c = 16 * bj + 8 * nt + 2 * t4;
-        *reinterpret_cast<float2*>(Xm + (16 * bi + g8) * LDX + c) = make_float2(-x[nt][0], -x[nt][1]);
-        *reinterpret_cast<float2*>(Xm + (16 * bi + g8 + 8) * LDX + c) =
-            make_float2(-x[nt][2], -x[nt][3]);
-      }
-    }
-    __syncthreads();
-  }
-}
-
 // ---------------------------------------------------------------- GDN-2 prep kernel
 // Gate arithmetic of the tensor-core GDN-2 path with the hardware exp2/log2
 // approximations (relative error ~1e-6, far below the bf16 path's budget):
@@ -165,10 +94,9 @@ constexpr int Q2_ZH = Q2_QT + kC * LDT * 2;    // raw V tile, then z = w (.) v (
 constexpr int Q2_ZL = Q2_ZH + kC * LDT * 2;    // z lo part
 constexpr int Q2_G = Q2_ZL + kC * LDT * 2;     // G [64][LDG] f32 (first: g, or the raw g tile)
 constexpr int Q2_E = Q2_G + kC * LDG * 4;      // e [64][LDG] f32 (first: the raw b tile)
-constexpr int Q2_L = Q2_E + kC * LDG * 4;      // L [64][LDX] f32
-constexpr int Q2_X = Q2_L + kC * LDX * 4;      // A staging (f32), then X
-constexpr int Q2_T = Q2_X + kC * LDX * 4;      // block products
-constexpr int Q2_OP = Q2_T + 3 * 16 * LDB * 4; // raw gate tiles, then fp16 operands, then E-bar
+constexpr int Q2_L = Q2_E + kC * LDG * 4;      // L [64][LDX] f32, then X in place
+constexpr int Q2_X = Q2_L + kC * LDX * 4;      // A staging (f32), then the inverse's block products
+constexpr int Q2_OP = Q2_X + kC * LDX * 4;     // raw gate tiles, then fp16 operands, then E-bar
 constexpr int Q2_OPB = 192 * LDT * 2;
 constexpr int Q2_VEC = Q2_OP + Q2_OPB;         // rk, sq [64], carry [128], misc [64]
 constexpr int Q2_BYTES = Q2_VEC + 320 * 4;
@@ -191,7 +119,6 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   float* Em = reinterpret_cast<float*>(sm + Q2_E);
   float* Lm = reinterpret_cast<float*>(sm + Q2_L);
   float* Xm = reinterpret_cast<float*>(sm + Q2_X);
-  float* Tm = reinterpret_cast<float*>(sm + Q2_T);
   uint8_t* op = sm + Q2_OP;
   float* rk = reinterpret_cast<float*>(sm + Q2_VEC);
   float* sq = rk + 64;
@@ -424,8 +351,16 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   }
   __syncthreads();
 
-  // 6. X = (I + L)^-1
-  invert_unit_lower(Lm, Xm, Tm, tid, warp, g8, t4);
+  // 6. X = (I + L)^-1 in place of L (the A staging is free now and takes the
+  //    block products); the blocks above the diagonal, never written, are zeroed
+  for (int i = tid; i < 6 * 256; i += kThreads) {
+    const int blk = i >> 8, e = i & 255;  // blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+    const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+    const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+    Lm[(16 * bi + (e >> 4)) * LDX + 16 * bj + (e & 15)] = 0.f;
+  }
+  invert_in_place(Lm, Xm, tid, warp, g8, t4);
+  float* Xi = Lm;  // X
 
   // 7. E-bar = exp(G) (.) e in bf16 (the B operand of W), in the operand scratch
   bf16* Eb = reinterpret_cast<bf16*>(op);
@@ -446,7 +381,7 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
       uint32_t ah[4], al[4];
-      frag_a_split(Xm, LDX, 16 * mt, 16 * ks, g8, t4, ah, al);
+      frag_a_split(Xi, LDX, 16 * mt, 16 * ks, g8, t4, ah, al);
 #pragma unroll
       for (int np = 0; np < 4; ++np) {
         const int bo = (16 * ks + lrow_a(lane)) * LDT + nb + 16 * np + lcol_a(lane);
