@@ -132,25 +132,31 @@ def job_rate(units_per_rank: float, world: int, ms_per_step: float) -> float:
 
 
 def kernel_traffic(name):
-    """dram bytes per launch from a committed ncu summary, if its kernel source
-    hash still matches the current source (else None)."""
+    """dram bytes per launch from a committed ncu summary, if the kernel sources it
+    lists (`source_files:`, relative to the package's csrc/; every source when the
+    line is absent) still hash to its `source_sha256` (else None)."""
     path = os.path.join(ROOT, "profiles", f"{name}.md")
     if not os.path.exists(path):
         return None
     txt = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     h = re.search(r"source_sha256:\s*([0-9a-f]{16,64})", txt)
+    f = re.search(r"source_files:\s*(.+)", txt)
     if not m or not h:
         return None
-    return float(m.group(1)) if h.group(1) == source_hash()[:len(h.group(1))] else None
+    files = f.group(1).split() if f else None
+    return float(m.group(1)) if h.group(1) == source_hash(files)[:len(h.group(1))] else None
 
 
-def source_hash():
+def source_hash(files=None):
+    """sha256 over the given kernel sources (names in csrc/, in the given order), or
+    over every .cu / .cuh / .h of csrc/ in name order."""
     d = os.path.join(ROOT, "gated_deltanet_sequence_gdn_b200", "csrc")
+    if files is None:
+        files = sorted(f for f in os.listdir(d) if f.endswith((".cu", ".cuh", ".h")))
     hs = hashlib.sha256()
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            hs.update(open(os.path.join(d, f), "rb").read())
+    for f in files:
+        hs.update(open(os.path.join(d, f), "rb").read())
     return hs.hexdigest()
 
 
