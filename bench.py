@@ -235,6 +235,7 @@ def run_ours(args, rank, local_rank, world):
         extra["decode_256"] = measure_decode(G, dev, stream, pk, args)
         extra["gdn2_b4_4k"] = measure_gdn2(G, dev, stream, pk, args)
         extra["prefill_128k"] = measure_prefill(G, "prefill_128k", dev, stream, pk, args)
+        extra["prefill_b8_16k"] = measure_prefill(G, "prefill_b8_16k", dev, stream, pk, args)
 
     launches = 2 * args.steps  # wy_prep_tc_kernel + state_scan_tc_kernel per step
     line = {

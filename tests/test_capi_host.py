@@ -132,3 +132,41 @@ def test_empty_calls_are_no_ops():
                                     4, 128, 128, 1, 0.1, 0, None) == 0
     assert G.lib.gdn_gate_prep(FAKE, FAKE, 1, FAKE, FAKE, FAKE, FAKE, 1, 0, 2, 4, 128, 0.1,
                                FAKE, FAKE, FAKE, FAKE, None) == 0
+
+
+def test_host_pipeline_workspace_bytes():
+    """gdn_chunk_fwd_host's device scratch: two sets of piece buffers (q, k, v, a, b),
+    two output pieces, the state, A_log and dt_bias, and the piece's chunk workspace,
+    each rounded up to 256 bytes."""
+    up = lambda x: (x + 255) // 256 * 256
+    B, T, Hk, Hv, d, Tc = 1, 8192, 16, 64, 128, 1024
+    rows = [Hk * d * 2, Hk * d * 2, Hv * d * 2, Hv * 2, Hv * 2]
+    want = 2 * sum(up(B * Tc * r) for r in rows) + 2 * up(B * Tc * Hv * d * 2)
+    want += up(B * Hv * d * d * 4) + 2 * up(Hv * 4)
+    want += up(G.lib.gdn_chunk_workspace_bytes(B, Tc, Hk, Hv, d, d, 1))
+    fn = G.lib.gdn_chunk_fwd_host_workspace_bytes
+    assert fn(B, T, Hk, Hv, d, d, 1, 1, 0) == want          # default: about T / 8 per piece
+    assert fn(B, T, Hk, Hv, d, d, 1, 1, 1000) == want       # rounded up to whole chunks
+    # float32 outputs and precomputed (float32) gates widen the rows
+    assert fn(B, T, Hk, Hv, d, d, 1, 1 | 4, 1024) > want
+    assert fn(B, T, Hk, Hv, d, d, 1, 1 | 2, 1024) > want
+    assert fn(0, T, Hk, Hv, d, d, 1, 1, 0) == 0 and fn(B, 0, Hk, Hv, d, d, 1, 1, 0) == 0
+    assert fn(B, T, Hk, Hv, d, d, 9, 1, 0) == 0
+
+
+def test_host_pipeline_rejects_bad_arguments():
+    """Refusals before any CUDA call: null inputs or outputs, negative sizes, a
+    missing or too small device scratch; B = 0 does nothing."""
+    f = G.lib.gdn_chunk_fwd_host
+    args = [FAKE] * 7 + [None, 1, 64, 2, 4, 128, 128, 1, 0.1, 1, FAKE, None, 64, None, 0, None]
+    assert f(*args) == -5                                    # no device scratch
+    bad = list(args); bad[0] = None
+    assert f(*bad) == -1                                     # q missing
+    bad = list(args); bad[17] = None
+    assert f(*bad) == -1                                     # o missing
+    bad = list(args); bad[9] = -1
+    assert f(*bad) == -1                                     # negative T
+    bad = list(args); bad[8] = 0
+    assert f(*bad) == 0                                      # B = 0: nothing to do
+    bad = list(args); bad[20] = FAKE; bad[21] = 1024
+    assert f(*bad) == -5                                     # scratch too small
