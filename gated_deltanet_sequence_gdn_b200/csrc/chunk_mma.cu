@@ -58,22 +58,6 @@ __device__ __forceinline__ float softplus_fast(float x) {
   return fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x)));
 }
 __device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
-// (jj, ii) with ii <= jj < 16, in row order: the 136 lower pairs of a 16 x 16 block
-struct PairTable {
-  unsigned char jj[136], ii[136];
-};
-__constant__ PairTable c_pairs = {
-    {0,1,1,2,2,2,3,3,3,3,4,4,4,4,4,5,5,5,5,5,5,6,6,6,6,6,6,6,7,7,7,7,7,7,7,7,
-     8,8,8,8,8,8,8,8,8,9,9,9,9,9,9,9,9,9,9,10,10,10,10,10,10,10,10,10,10,10,
-     11,11,11,11,11,11,11,11,11,11,11,11,12,12,12,12,12,12,12,12,12,12,12,12,12,
-     13,13,13,13,13,13,13,13,13,13,13,13,13,13,14,14,14,14,14,14,14,14,14,14,14,
-     14,14,14,14,15,15,15,15,15,15,15,15,15,15,15,15,15,15,15,15},
-    {0,0,1,0,1,2,0,1,2,3,0,1,2,3,4,0,1,2,3,4,5,0,1,2,3,4,5,6,0,1,2,3,4,5,6,7,
-     0,1,2,3,4,5,6,7,8,0,1,2,3,4,5,6,7,8,9,0,1,2,3,4,5,6,7,8,9,10,
-     0,1,2,3,4,5,6,7,8,9,10,11,0,1,2,3,4,5,6,7,8,9,10,11,12,
-     0,1,2,3,4,5,6,7,8,9,10,11,12,13,0,1,2,3,4,5,6,7,8,9,10,
-     11,12,13,14,0,1,2,3,4,5,6,7,8,9,10,11,12,13,14,15}
-};
 // Gated DeltaNet-2: per-channel decay d_t = exp(g_t) (g_t in R^dk), erase
 // direction e_t = b_t (.) k^_t, written value z_t = w_t (.) v_t.  With G the
 // in-chunk prefix sum of g (per channel) the chunk form is
@@ -83,8 +67,9 @@ __constant__ PairTable c_pairs = {
 //   o = (exp(G) (.) Q^) S + A (U - W S),   S <- diag(exp(G_C)) S + K_tail^T (U - W S)
 // with K_tail rows exp(G_C - G_j) (.) k^_j ("Gated DeltaNet-2", 通道级衰减的吸收技巧
 // and WY 形式).  The exponents differ per channel, so the 16 x 16 diagonal blocks
-// of L and A are summed element by element, and each off-diagonal block row I is
-// a product of operands scaled about its first row r = 16 I:
+// of L and A are summed element by element (exp(G_j - G_i) there is the product of
+// the per-token decays d = exp(g) of rows i+1..j), and each off-diagonal block row
+// I is a product of operands scaled about its first row r = 16 I:
 //   L_ji = sum_c [e_jc exp(G_jc - G_rc)] [k^_ic exp(G_rc - G_ic)]   (i < r <= j)
 // where both exponents are <= 0, so every operand stays within its input's size.
 constexpr int LDG = kD + 4;                    // f32 row stride of [64][128] channel tiles
@@ -96,12 +81,12 @@ constexpr int Q2_G = Q2_ZL + kC * LDT * 2;     // G [64][LDG] f32 (first: g, or 
 constexpr int Q2_E = Q2_G + kC * LDG * 4;      // e [64][LDG] f32 (first: the raw b tile)
 constexpr int Q2_L = Q2_E + kC * LDG * 4;      // L [64][LDX] f32, then X in place
 constexpr int Q2_X = Q2_L + kC * LDX * 4;      // A staging (f32), then the inverse's block products
-constexpr int Q2_OP = Q2_X + kC * LDX * 4;     // raw gate tiles, then fp16 operands, then E-bar
+constexpr int Q2_OP = Q2_X + kC * LDX * 4;     // raw gate tiles, decays d, fp16 operands, E-bar
 constexpr int Q2_OPB = 192 * LDT * 2;
 constexpr int Q2_VEC = Q2_OP + Q2_OPB;         // rk, sq [64], carry [128], misc [64]
 constexpr int Q2_BYTES = Q2_VEC + 320 * 4;
 static_assert(Q2_BYTES <= 227 * 1024, "shared memory of the GDN-2 prep kernel");
-static_assert(kC * LDG * 4 <= Q2_OPB, "raw float32 w tile fits the operand scratch");
+static_assert(kC * LDG * 4 <= Q2_OPB, "a float32 [64][LDG] tile (raw w, the decays) fits the operand scratch");
 
 template <bool PRE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -182,45 +167,100 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   }
   __syncthreads();
 
-  // 3. per (token, channel): g, e = b (.) k^ and z = w (.) v (as bf16 hi + lo), all
-  //    independent; then the in-chunk prefix sums G down each channel (two threads
-  //    per channel, 32 tokens each)
-  const int ch = tid & 127, half = tid >> 7;
+  // 3. per (token, channel), all independent: g, e = b (.) k^ and z = w (.) v (as
+  //    bf16 hi + lo); a thread takes 8 channels of a row at a time (its channels
+  //    c8 .. c8 + 7 are the same in every row); then the in-chunk prefix sums G down
+  //    each channel (two threads per channel, 32 tokens each)
   {
-    float nal = 0.f, dtb = 0.f;
-    if (!PRE) {
-      nal = -expf(A_log[(size_t)h * kD + ch]);
-      dtb = dt_bias[(size_t)h * kD + ch];
+    const int c8 = (tid & 15) * 8;
+    float nal[8], dtb[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      nal[u] = PRE ? 0.f : -expf(A_log[(size_t)h * kD + c8 + u]);
+      dtb[u] = PRE ? 0.f : dt_bias[(size_t)h * kD + c8 + u];
     }
     const bf16* at = reinterpret_cast<const bf16*>(op);
     const bf16* bt = at + kC * LDT;
     const bf16* wt = bt + kC * LDT;
     const float* wf = reinterpret_cast<const float*>(op);
-#pragma unroll 8
-    for (int tt = 0; tt < 32; ++tt) {
-      const int r = 32 * half + tt;
-      float g, bv, wv;
+#pragma unroll 1
+    for (int it = tid; it < kC * 16; it += kThreads) {
+      const int r = it >> 4;
+      float g[8], bv[8], wv[8], kr[8], vr[8];
       if (PRE) {
-        g = Gm[r * LDG + ch];
-        bv = Em[r * LDG + ch];
-        wv = wf[r * LDG + ch];
+#pragma unroll
+        for (int h4 = 0; h4 < 2; ++h4) {
+          const float4 g4 = *reinterpret_cast<const float4*>(Gm + r * LDG + c8 + 4 * h4);
+          const float4 b4 = *reinterpret_cast<const float4*>(Em + r * LDG + c8 + 4 * h4);
+          const float4 w4 = *reinterpret_cast<const float4*>(wf + r * LDG + c8 + 4 * h4);
+          g[4 * h4] = g4.x, g[4 * h4 + 1] = g4.y, g[4 * h4 + 2] = g4.z, g[4 * h4 + 3] = g4.w;
+          bv[4 * h4] = b4.x, bv[4 * h4 + 1] = b4.y, bv[4 * h4 + 2] = b4.z, bv[4 * h4 + 3] = b4.w;
+          wv[4 * h4] = w4.x, wv[4 * h4 + 1] = w4.y, wv[4 * h4 + 2] = w4.z, wv[4 * h4 + 3] = w4.w;
+        }
       } else {
-        g = r < nv ? nal * softplus_fast(__bfloat162float(at[r * LDT + ch]) + dtb) : 0.f;
-        bv = sigmoid_fast(__bfloat162float(bt[r * LDT + ch]));
-        wv = sigmoid_fast(__bfloat162float(wt[r * LDT + ch]));
+        const uint4 ua = *reinterpret_cast<const uint4*>(at + r * LDT + c8);
+        const uint4 ub = *reinterpret_cast<const uint4*>(bt + r * LDT + c8);
+        const uint4 uw = *reinterpret_cast<const uint4*>(wt + r * LDT + c8);
+        const uint32_t* pa = reinterpret_cast<const uint32_t*>(&ua);
+        const uint32_t* pb = reinterpret_cast<const uint32_t*>(&ub);
+        const uint32_t* pw = reinterpret_cast<const uint32_t*>(&uw);
+#pragma unroll
+        for (int u2 = 0; u2 < 4; ++u2) {
+          const float2 a2 = unpack2(pa[u2]), b2 = unpack2(pb[u2]), w2 = unpack2(pw[u2]);
+          g[2 * u2] = r < nv ? nal[2 * u2] * softplus_fast(a2.x + dtb[2 * u2]) : 0.f;
+          g[2 * u2 + 1] = r < nv ? nal[2 * u2 + 1] * softplus_fast(a2.y + dtb[2 * u2 + 1]) : 0.f;
+          bv[2 * u2] = sigmoid_fast(b2.x), bv[2 * u2 + 1] = sigmoid_fast(b2.y);
+          wv[2 * u2] = sigmoid_fast(w2.x), wv[2 * u2 + 1] = sigmoid_fast(w2.y);
+        }
       }
-      Gm[r * LDG + ch] = g;
-      Em[r * LDG + ch] = bv * __bfloat162float(Kt[r * LDT + ch]) * rk[r];
-      const float z = wv * __bfloat162float(Zh[r * LDT + ch]);
-      const bf16 zh = __float2bfloat16_rn(z);
-      Zh[r * LDT + ch] = zh;
-      Zl[r * LDT + ch] = __float2bfloat16_rn(z - __bfloat162float(zh));
+      {
+        const uint4 uk = *reinterpret_cast<const uint4*>(Kt + r * LDT + c8);
+        const uint4 uv = *reinterpret_cast<const uint4*>(Zh + r * LDT + c8);
+        const uint32_t* pk = reinterpret_cast<const uint32_t*>(&uk);
+        const uint32_t* pv = reinterpret_cast<const uint32_t*>(&uv);
+#pragma unroll
+        for (int u2 = 0; u2 < 4; ++u2) {
+          const float2 k2 = unpack2(pk[u2]), v2 = unpack2(pv[u2]);
+          kr[2 * u2] = k2.x, kr[2 * u2 + 1] = k2.y, vr[2 * u2] = v2.x, vr[2 * u2 + 1] = v2.y;
+        }
+      }
+      const float rkr = rk[r];
+      uint4 zh4, zl4;
+      uint32_t* ph = reinterpret_cast<uint32_t*>(&zh4);
+      uint32_t* pl = reinterpret_cast<uint32_t*>(&zl4);
+#pragma unroll
+      for (int u2 = 0; u2 < 4; ++u2) {
+        const float z0 = wv[2 * u2] * vr[2 * u2], z1 = wv[2 * u2 + 1] * vr[2 * u2 + 1];
+        ph[u2] = pack2(z0, z1);
+        const float2 zr = unpack2(ph[u2]);
+        pl[u2] = pack2(z0 - zr.x, z1 - zr.y);
+      }
+      *reinterpret_cast<uint4*>(Zh + r * LDT + c8) = zh4;
+      *reinterpret_cast<uint4*>(Zl + r * LDT + c8) = zl4;
+#pragma unroll
+      for (int h4 = 0; h4 < 2; ++h4) {
+        const int u = 4 * h4;
+        *reinterpret_cast<float4*>(Gm + r * LDG + c8 + u) =
+            make_float4(g[u], g[u + 1], g[u + 2], g[u + 3]);
+        *reinterpret_cast<float4*>(Em + r * LDG + c8 + u) =
+            make_float4(bv[u] * kr[u] * rkr, bv[u + 1] * kr[u + 1] * rkr,
+                        bv[u + 2] * kr[u + 2] * rkr, bv[u + 3] * kr[u + 3] * rkr);
+      }
     }
+  }
+  const int ch = tid & 127, half = tid >> 7;
+  __syncthreads();
+  //    the raw gate tiles are consumed: the per-token decays d = exp(g) go to the
+  //    operand scratch (for the diagonal blocks below), then g becomes G in place
+  float* Dm = reinterpret_cast<float*>(op);
+  {
     float run = 0.f;
 #pragma unroll 8
     for (int tt = 0; tt < 32; ++tt) {
       const int r = 32 * half + tt;
-      run += Gm[r * LDG + ch];
+      const float g = Gm[r * LDG + ch];
+      Dm[r * LDG + ch] = __expf(g);
+      run += g;
       Gm[r * LDG + ch] = run;
     }
     if (half == 0) carry[ch] = run;
@@ -233,37 +273,60 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   }
   __syncthreads();
 
-  // 4. diagonal 16 x 16 blocks of L and A, element by element: one thread per
-  //    lower pair (j, i) of a block (544 pairs), summing over the 128 channels
-  //    (exp(G_j - G_i) <= 1 for i <= j)
+  // 4. diagonal 16 x 16 blocks of L and A, element by element.  Inside a block
+  //    exp(G_j - G_i) = d_{i+1} ... d_j (each factor <= 1), so column i is one
+  //    running product P = k_i d_{i+1} ... d_j per channel, walked down the rows
+  //    j = i..15.  Lane: block bl = lane / 8 and the 16 channels 4 cg + 32 s + u
+  //    (cg = lane % 8, s, u < 4); warp w takes the columns w and 15 - w of all four
+  //    blocks (17 rows in all, the same for every warp).  The eight lanes of a block
+  //    then sum their partial L and A over the 128 channels.
+  {
+    const int bl = lane >> 3, cg = lane & 7;
+    const bool odd = (cg & 1) != 0;
 #pragma unroll 1
-  for (int p = tid; p < 4 * 136; p += kThreads) {
-    const int blk = p / 136, pi = p - blk * 136;
-    const int jj = c_pairs.jj[pi], ii = c_pairs.ii[pi];
-    const int j = 16 * blk + jj, i = 16 * blk + ii;
-    const float* gj = Gm + j * LDG;
-    const float* gi = Gm + i * LDG;
-    const float* ej = Em + j * LDG;
-    const bf16* qj = Qt + j * LDT;
-    const bf16* ki = Kt + i * LDT;
-    float sl = 0.f, sa = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < kD; c += 4) {
-      const float4 a4 = *reinterpret_cast<const float4*>(gj + c);
-      const float4 b4 = *reinterpret_cast<const float4*>(gi + c);
-      const float4 e4 = *reinterpret_cast<const float4*>(ej + c);
-      const uint2 qq = *reinterpret_cast<const uint2*>(qj + c);
-      const uint2 kk = *reinterpret_cast<const uint2*>(ki + c);
-      const float2 q01 = unpack2(qq.x), q23 = unpack2(qq.y);
-      const float2 k01 = unpack2(kk.x), k23 = unpack2(kk.y);
-      const float x0 = __expf(a4.x - b4.x) * k01.x, x1 = __expf(a4.y - b4.y) * k01.y;
-      const float x2 = __expf(a4.z - b4.z) * k23.x, x3 = __expf(a4.w - b4.w) * k23.y;
-      sl = fmaf(e4.x, x0, fmaf(e4.y, x1, fmaf(e4.z, x2, fmaf(e4.w, x3, sl))));
-      sa = fmaf(q01.x, x0, fmaf(q01.y, x1, fmaf(q23.x, x2, fmaf(q23.y, x3, sa))));
+    for (int pass = 0; pass < 2; ++pass) {
+      const int ic = pass ? 15 - warp : warp;  // column within the block (warp-uniform)
+      const int ci = 16 * bl + ic;
+      float2 P[8];
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const uint2 kk = *reinterpret_cast<const uint2*>(Kt + ci * LDT + 4 * cg + 32 * s);
+        P[2 * s] = unpack2(kk.x);
+        P[2 * s + 1] = unpack2(kk.y);
+      }
+      const float rki = rk[ci];
+#pragma unroll 1
+      for (int jr = ic; jr < 16; ++jr) {
+        const int rj = 16 * bl + jr;
+        if (jr > ic) {
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            const float4 d4 = *reinterpret_cast<const float4*>(Dm + rj * LDG + 4 * cg + 32 * s);
+            P[2 * s] = fmul2(P[2 * s], make_float2(d4.x, d4.y));
+            P[2 * s + 1] = fmul2(P[2 * s + 1], make_float2(d4.z, d4.w));
+          }
+        }
+        float2 sl2 = make_float2(0.f, 0.f), sa2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const float4 e4 = *reinterpret_cast<const float4*>(Em + rj * LDG + 4 * cg + 32 * s);
+          const uint2 qq = *reinterpret_cast<const uint2*>(Qt + rj * LDT + 4 * cg + 32 * s);
+          sl2 = ffma2(make_float2(e4.x, e4.y), P[2 * s], sl2);
+          sl2 = ffma2(make_float2(e4.z, e4.w), P[2 * s + 1], sl2);
+          sa2 = ffma2(unpack2(qq.x), P[2 * s], sa2);
+          sa2 = ffma2(unpack2(qq.y), P[2 * s + 1], sa2);
+        }
+        const float sl = sl2.x + sl2.y, sa = sa2.x + sa2.y;
+        // even lanes go on with L, odd lanes with A, each summing over all eight
+        float acc = (odd ? sa : sl) + __shfl_xor_sync(0xffffffffu, odd ? sl : sa, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        if (cg == 0) Lm[rj * LDX + ci] = jr > ic ? acc * rki : 0.f;
+        if (cg == 1) Xm[rj * LDX + ci] = acc * sq[rj] * rki;
+      }
     }
-    Lm[j * LDX + i] = ii < jj ? sl * rk[i] : 0.f;
-    Xm[j * LDX + i] = sa * sq[j] * rk[i];
   }
+  __syncthreads();  // the decays in the operand scratch are read
 
   // 5. off-diagonal blocks on the tensor cores: fp16 operands scaled about the
   //    reference row r = 16 I of block row I (I = 1..3).  Rows of the operand
@@ -364,9 +427,18 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
 
   // 7. E-bar = exp(G) (.) e in bf16 (the B operand of W), in the operand scratch
   bf16* Eb = reinterpret_cast<bf16*>(op);
-  for (int e = tid; e < kC * kD; e += kThreads) {
-    const int r = e >> 7, c = e & 127;
-    Eb[r * LDT + c] = __float2bfloat16_rn(__expf(Gm[r * LDG + c]) * Em[r * LDG + c]);
+  for (int i = tid; i < kC * 16; i += kThreads) {
+    const int r = i >> 4, c8 = (i & 15) * 8;
+    uint4 o;
+    uint32_t* po = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int h4 = 0; h4 < 2; ++h4) {
+      const float4 g4 = *reinterpret_cast<const float4*>(Gm + r * LDG + c8 + 4 * h4);
+      const float4 e4 = *reinterpret_cast<const float4*>(Em + r * LDG + c8 + 4 * h4);
+      po[2 * h4] = pack2(__expf(g4.x) * e4.x, __expf(g4.y) * e4.y);
+      po[2 * h4 + 1] = pack2(__expf(g4.z) * e4.z, __expf(g4.w) * e4.w);
+    }
+    *reinterpret_cast<uint4*>(Eb + r * LDT + c8) = o;
   }
   __syncthreads();
 
@@ -435,17 +507,28 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     __half* kd = reinterpret_cast<__half*>(ws + L.kh) + (head * Tp + t0) * kD;
     for (int i = tid; i < kC * 16; i += kThreads) {
       const int r = i >> 4, c8 = (i & 15) * 8;
+      const uint4 uq = *reinterpret_cast<const uint4*>(Qt + r * LDT + c8);
+      const uint4 uk = *reinterpret_cast<const uint4*>(Kt + r * LDT + c8);
+      const uint32_t* pq = reinterpret_cast<const uint32_t*>(&uq);
+      const uint32_t* pk = reinterpret_cast<const uint32_t*>(&uk);
+      float gr[8], gc[8];
+#pragma unroll
+      for (int h4 = 0; h4 < 2; ++h4) {
+        const float4 a4 = *reinterpret_cast<const float4*>(Gm + r * LDG + c8 + 4 * h4);
+        const float4 b4 = *reinterpret_cast<const float4*>(Gm + (kC - 1) * LDG + c8 + 4 * h4);
+        gr[4 * h4] = a4.x, gr[4 * h4 + 1] = a4.y, gr[4 * h4 + 2] = a4.z, gr[4 * h4 + 3] = a4.w;
+        gc[4 * h4] = b4.x, gc[4 * h4 + 1] = b4.y, gc[4 * h4 + 2] = b4.z, gc[4 * h4 + 3] = b4.w;
+      }
+      const float sqr = sq[r], rkr = rk[r];
       uint4 oq, ok;
       uint32_t* wq = reinterpret_cast<uint32_t*>(&oq);
       uint32_t* wk = reinterpret_cast<uint32_t*>(&ok);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int c = c8 + 2 * u;
-        const float2 qq = unpack2(*reinterpret_cast<const uint32_t*>(Qt + r * LDT + c));
-        const float2 kk = unpack2(*reinterpret_cast<const uint32_t*>(Kt + r * LDT + c));
-        wq[u] = pack2h(qq.x * sq[r] * __expf(Gm[r * LDG + c]), qq.y * sq[r] * __expf(Gm[r * LDG + c + 1]));
-        wk[u] = pack2h(kk.x * rk[r] * __expf(Gm[(kC - 1) * LDG + c] - Gm[r * LDG + c]),
-                       kk.y * rk[r] * __expf(Gm[(kC - 1) * LDG + c + 1] - Gm[r * LDG + c + 1]));
+        const float2 qq = unpack2(pq[u]), kk = unpack2(pk[u]);
+        wq[u] = pack2h(qq.x * sqr * __expf(gr[2 * u]), qq.y * sqr * __expf(gr[2 * u + 1]));
+        wk[u] = pack2h(kk.x * rkr * __expf(gc[2 * u] - gr[2 * u]),
+                       kk.y * rkr * __expf(gc[2 * u + 1] - gr[2 * u + 1]));
       }
       *reinterpret_cast<uint4*>(qd + (size_t)r * kD + c8) = oq;
       *reinterpret_cast<uint4*>(kd + (size_t)r * kD + c8) = ok;
