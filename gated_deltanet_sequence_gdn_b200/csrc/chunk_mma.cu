@@ -47,7 +47,7 @@ using namespace wm;
 using namespace wy;
 using bf16 = __nv_bfloat16;
 
-constexpr int kThreads = 256;  // 8 warps
+constexpr int kThreads = 512;  // 16 warps
 constexpr int LDT = kD + 8;    // 16-bit row stride of 128-wide tiles (272 B: ldmatrix conflict-free)
 
 // ---------------------------------------------------------------- GDN-2 prep kernel
@@ -83,8 +83,8 @@ constexpr int Q2_L = Q2_E + kC * LDG * 4;      // L [64][LDX] f32, then X in pla
 constexpr int Q2_X = Q2_L + kC * LDX * 4;      // A staging (f32), then the inverse's block products
 constexpr int Q2_OP = Q2_X + kC * LDX * 4;     // raw gate tiles, decays d, fp16 operands, E-bar
 constexpr int Q2_OPB = 192 * LDT * 2;
-constexpr int Q2_VEC = Q2_OP + Q2_OPB;         // rk, sq [64], carry [128], misc [64]
-constexpr int Q2_BYTES = Q2_VEC + 320 * 4;
+constexpr int Q2_VEC = Q2_OP + Q2_OPB;         // rk, sq [64], carry [3][128], misc [64]
+constexpr int Q2_BYTES = Q2_VEC + 576 * 4;
 static_assert(Q2_BYTES <= 227 * 1024, "shared memory of the GDN-2 prep kernel");
 static_assert(kC * LDG * 4 <= Q2_OPB, "a float32 [64][LDG] tile (raw w, the decays) fits the operand scratch");
 
@@ -107,8 +107,8 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   uint8_t* op = sm + Q2_OP;
   float* rk = reinterpret_cast<float*>(sm + Q2_VEC);
   float* sq = rk + 64;
-  float* carry = sq + 64;
-  float* misc = carry + 128;  // [8..15] per-warp max |U|
+  float* carry = sq + 64;     // [3][128] prefix sums of the first three quarters
+  float* misc = carry + 384;  // [8..23] per-warp max |U|
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
@@ -142,23 +142,23 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     }
   }
   cp_commit();
-  for (int i = tid; i < kC * LDX; i += kThreads) Xm[i] = 0.f;  // A staging starts at zero
   cp_wait<0>();
   __syncthreads();
 
-  // 2. L2 norms: rk = 1 / |k|, sq = scale / |q| (two threads per row)
+  // 2. L2 norms: rk = 1 / |k|, sq = scale / |q| (four threads per row)
   {
-    const int which = tid >> 7, r = (tid & 127) >> 1, hh = tid & 1;
+    const int which = tid >> 8, r = (tid & 255) >> 2, hh = tid & 3;
     const bf16* row = (which ? Qt : Kt) + r * LDT + hh * 8;
     float ss = 0.f;
 #pragma unroll
-    for (int c = 0; c < 128; c += 16) {
+    for (int c = 0; c < 128; c += 32) {
       const uint4 u = *reinterpret_cast<const uint4*>(row + c);
       const float2 f0 = unpack2(u.x), f1 = unpack2(u.y), f2 = unpack2(u.z), f3 = unpack2(u.w);
       ss += f0.x * f0.x + f0.y * f0.y + f1.x * f1.x + f1.y * f1.y + f2.x * f2.x + f2.y * f2.y +
             f3.x * f3.x + f3.y * f3.y;
     }
     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
     if (hh == 0) {
       const float inv = l2 ? rsqrtf(ss + 1e-6f) : 1.f;
       if (which) sq[r] = inv * scale;
@@ -170,7 +170,7 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   // 3. per (token, channel), all independent: g, e = b (.) k^ and z = w (.) v (as
   //    bf16 hi + lo); a thread takes 8 channels of a row at a time (its channels
   //    c8 .. c8 + 7 are the same in every row); then the in-chunk prefix sums G down
-  //    each channel (two threads per channel, 32 tokens each)
+  //    each channel (four threads per channel, 16 tokens each)
   {
     const int c8 = (tid & 15) * 8;
     float nal[8], dtb[8];
@@ -248,7 +248,7 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
       }
     }
   }
-  const int ch = tid & 127, half = tid >> 7;
+  const int ch = tid & 127, qtr = tid >> 7;
   __syncthreads();
   //    the raw gate tiles are consumed: the per-token decays d = exp(g) go to the
   //    operand scratch (for the diagonal blocks below), then g becomes G in place
@@ -256,20 +256,22 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   {
     float run = 0.f;
 #pragma unroll 8
-    for (int tt = 0; tt < 32; ++tt) {
-      const int r = 32 * half + tt;
+    for (int tt = 0; tt < 16; ++tt) {
+      const int r = 16 * qtr + tt;
       const float g = Gm[r * LDG + ch];
       Dm[r * LDG + ch] = __expf(g);
       run += g;
       Gm[r * LDG + ch] = run;
     }
-    if (half == 0) carry[ch] = run;
+    if (qtr < 3) carry[qtr * 128 + ch] = run;
   }
   __syncthreads();
-  if (half == 1) {
-    const float cy = carry[ch];
+  if (qtr > 0) {
+    float cy = carry[ch];
+    if (qtr > 1) cy += carry[128 + ch];
+    if (qtr > 2) cy += carry[256 + ch];
 #pragma unroll 8
-    for (int r = 32; r < kC; ++r) Gm[r * LDG + ch] += cy;
+    for (int tt = 0; tt < 16; ++tt) Gm[(16 * qtr + tt) * LDG + ch] += cy;
   }
   __syncthreads();
 
@@ -277,15 +279,15 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   //    exp(G_j - G_i) = d_{i+1} ... d_j (each factor <= 1), so column i is one
   //    running product P = k_i d_{i+1} ... d_j per channel, walked down the rows
   //    j = i..15.  Lane: block bl = lane / 8 and the 16 channels 4 cg + 32 s + u
-  //    (cg = lane % 8, s, u < 4); warp w takes the columns w and 15 - w of all four
-  //    blocks (17 rows in all, the same for every warp).  The eight lanes of a block
-  //    then sum their partial L and A over the 128 channels.
+  //    (cg = lane % 8, s, u < 4); warp w takes column w (w < 8) or 23 - w of all
+  //    four blocks, so that the four warps w = s, s + 4, s + 8, s + 12 of one
+  //    scheduler walk 34 rows in all.  The eight lanes of a block then sum their
+  //    partial L and A over the 128 channels.
   {
     const int bl = lane >> 3, cg = lane & 7;
     const bool odd = (cg & 1) != 0;
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-      const int ic = pass ? 15 - warp : warp;  // column within the block (warp-uniform)
+    {
+      const int ic = warp < 8 ? warp : 23 - warp;  // column within the block (warp-uniform)
       const int ci = 16 * bl + ic;
       float2 P[8];
 #pragma unroll
@@ -333,7 +335,7 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   //    scratch: [0,48) e rows of blocks 1-3, [48,96) q^ rows, [96,192) k^ rows
   //    0..16 I - 1 for I = 1, 2, 3 (at 96, 112, 144).
   __half* Op = reinterpret_cast<__half*>(op);
-  for (int row = warp; row < 192; row += 8) {
+  for (int row = warp; row < 192; row += kThreads / 32) {
     const int c = 4 * lane;
     int j, I;
     const float* src;  // row of e, or of raw q / k (bf16) below
@@ -372,7 +374,8 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   }
   __syncthreads();
   //    tasks (matrix, I, column pair np < I): 6 for L, 6 for A
-  for (int task = warp; task < 12; task += 8) {
+  if (warp < 12) {
+    const int task = warp;
     const bool isa = task >= 6;
     const int tk = isa ? task - 6 : task;
     const int I = tk < 1 ? 1 : (tk < 3 ? 2 : 3);
@@ -443,19 +446,19 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   __syncthreads();
 
   //    W = X E-bar (fp16 out) and U = X Z (fp32 out, X and Z both as hi + lo);
-  //    warp -> rows 16 (warp % 4), cols 64 (warp / 4)
-  const int mt = warp & 3, nb = 64 * (warp >> 2);
+  //    warp -> rows 16 (warp % 4), cols 32 (warp / 4)
+  const int mt = warp & 3, nb = 32 * (warp >> 2);
   const int ra = 16 * mt + g8;
   float umax = 0.f;
 #pragma unroll 1
   for (int which = 0; which < 2; ++which) {
-    float acc[8][4] = {};
+    float acc[4][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
       uint32_t ah[4], al[4];
       frag_a_split(Xi, LDX, 16 * mt, 16 * ks, g8, t4, ah, al);
 #pragma unroll
-      for (int np = 0; np < 4; ++np) {
+      for (int np = 0; np < 2; ++np) {
         const int bo = (16 * ks + lrow_a(lane)) * LDT + nb + 16 * np + lcol_a(lane);
         uint32_t bh[4];
         ldsm_x4_t(bh, (which ? Zh : Eb) + bo);
@@ -474,7 +477,7 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     if (which == 0) {
       __half* dw = reinterpret_cast<__half*>(ws + L.w) + (head * Tp + t0) * kD;
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
+      for (int nt = 0; nt < 4; ++nt) {
         const int c = nb + 8 * nt + 2 * t4;
         range = fmaxf(range, fmaxf(fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][1])),
                                    fmaxf(fabsf(acc[nt][2]), fabsf(acc[nt][3]))));
@@ -485,7 +488,7 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     } else {
       float* du = reinterpret_cast<float*>(ws + L.u) + (head * Tp + t0) * kD;
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
+      for (int nt = 0; nt < 4; ++nt) {
         const int c = nb + 8 * nt + 2 * t4;
         umax = fmaxf(umax, fmaxf(fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][1])),
                                  fmaxf(fabsf(acc[nt][2]), fabsf(acc[nt][3]))));
@@ -545,7 +548,7 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     if (tid < 4) {
       float m = 0.f;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) m = fmaxf(m, misc[8 + w]);
+      for (int w = 0; w < kThreads / 32; ++w) m = fmaxf(m, misc[8 + w]);
       sc[kScMaxU + tid] = tid == 0 ? m : 0.f;
     }
   }

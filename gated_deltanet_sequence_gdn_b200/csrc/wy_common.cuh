@@ -75,8 +75,8 @@ __device__ __forceinline__ void store_tile(float* M, int ld, int r0, int c0, int
 }
 
 // X = (I + L)^-1 in place for a strictly lower 64 x 64 fp32 L (row stride LDX,
-// zero upper triangle), by the whole CTA (8 warps), by recursive doubling over
-// 16 x 16 blocks (L_ij, X_ij):
+// zero upper triangle), by the whole CTA (products on warps 0-7, every warp at the
+// barriers), by recursive doubling over 16 x 16 blocks (L_ij, X_ij):
 //   X_ii       : forward substitution, one thread per column of a diagonal block;
 //   32 x 32    : X_10 = -X_11 (L_10 X_00),  X_32 = -X_33 (L_32 X_22);
 //   64 x 64    : X_[2:4][0:2] = -X_[2:4][2:4] (L_[2:4][0:2] X_[0:2][0:2]),
@@ -120,8 +120,9 @@ __device__ inline void invert_in_place(float* M, float* Tm, int tid, int warp, i
   }
   __syncthreads();
   // 64 x 64: T_(ri, cj) = sum_{k=cj}^{1} L_(ri, k) X_(k, cj) for ri = 2, 3 and cj = 0, 1
+  // (warps 0-7; the warps past them only keep the barriers)
   const int t = warp >> 1, ri = 2 + (t >> 1), cj = t & 1;
-  {
+  if (warp < 8) {
     float d[4] = {};
     const int ac[2] = {16 * cj, 16}, br[2] = {16 * cj, 16};
     block_prod(M, LDX, 16 * ri, ac, M, LDX, br, 2 - cj, 16 * cj + n8, g8, t4, d);
@@ -129,7 +130,7 @@ __device__ inline void invert_in_place(float* M, float* Tm, int tid, int warp, i
   }
   __syncthreads();
   //         X_(ri, cj) = -sum_{k=2}^{ri} X_(ri, k) T_(k, cj)
-  {
+  if (warp < 8) {
     float d[4] = {};
     for (int k = 2; k <= ri; ++k) {
       const int ac[1] = {16 * k}, br[1] = {0};
