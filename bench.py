@@ -234,6 +234,7 @@ def run_ours(args, rank, local_rank, world):
     if not args.headline_only:
         extra["decode_256"] = measure_decode(G, dev, stream, pk, args)
         extra["gdn2_b4_4k"] = measure_gdn2(G, dev, stream, pk, args)
+        extra["conv_prefill_8k"] = measure_conv(G, dev, stream, pk, args)
         extra["prefill_128k"] = measure_prefill(G, "prefill_128k", dev, stream, pk, args)
         extra["prefill_b8_16k"] = measure_prefill(G, "prefill_b8_16k", dev, stream, pk, args)
 
@@ -365,6 +366,39 @@ def measure_gdn2(G, dev, stream, pk, args):
             "frac_of_bf16_peak": round(ach / pk["bf16_tflops"], 4)}
 
 
+def measure_conv(G, dev, stream, pk, args):
+    """gdn_conv_prefill over the mixed stream of the prefill_8k layer: HBM-bound,
+    reported against the measured copy bandwidth.  Algorithmic bytes per launch:
+    the input stream read once, q, k, v written once, the taps and the window read
+    and written (inputs of 201 MB, larger than L2, so no flush between launches)."""
+    w = WORKLOADS["conv_prefill_8k"]
+    x = workload_inputs(w, dev)
+    Cc = 2 * w.Hk * w.d + w.Hv * w.d
+    cs = x["conv_state"]
+    q = torch.empty((w.B, w.T, w.Hk, w.d), device=dev, dtype=w.dtype)
+    k = torch.empty_like(q)
+    v = torch.empty((w.B, w.T, w.Hv, w.d), device=dev, dtype=w.dtype)
+
+    def step():
+        G.gdn_conv_prefill(x["x"], x["conv_w"], cs, Hk=w.Hk, Hv=w.Hv, dk=w.d, dv=w.d, q=q, k=k,
+                           v=v, stream=stream)
+
+    steps = 20
+    total, per = time_steps(step, steps, 3, stream)
+    ms = sum(per) / len(per)
+    es = 2  # bf16
+    nbytes = 2 * w.B * w.T * Cc * es + Cc * 16 + 2 * w.B * Cc * 3 * es
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del x, cs, q, k, v
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_launch": round(ms, 5),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": kernel_traffic("conv_prefill_8k")},
+            "steps": steps}
+
+
 def run_only(args, local_rank):
     import gated_deltanet_sequence_gdn_b200 as G
     torch.cuda.set_device(local_rank)
@@ -375,6 +409,8 @@ def run_only(args, local_rank):
         r = measure_decode(G, dev, stream, pk, args)
     elif args.only == "gdn2_b4_4k":
         r = measure_gdn2(G, dev, stream, pk, args)
+    elif args.only == "conv_prefill_8k":
+        r = measure_conv(G, dev, stream, pk, args)
     else:
         r = measure_prefill(G, args.only, dev, stream, pk, args)
     G.gdn_check_status(stream)
@@ -451,7 +487,7 @@ def main():
                     help="skip the decode / GDN-2 / long-prefill extras")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["prefill_8k", "decode_256", "gdn2_b4_4k", "prefill_128k",
-                                       "prefill_b8_16k"], default=None,
+                                       "prefill_b8_16k", "conv_prefill_8k"], default=None,
                     help="measure one secondary workload alone (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -18,6 +18,7 @@ import os
 import torch
 
 __all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_chunk_workspace_bytes", "gdn_recurrent_step",
+           "gdn_conv_prefill",
            "gdn2_chunk_fwd", "gdn2_chunk_workspace_bytes", "gdn_chunk_fwd_noalloc",
            "gdn_check_status", "GDNError", "LIB_PATH", "lib", "F32", "BF16",
            "QK_L2NORM", "GATES_PRECOMPUTED", "OUT_F32"]
@@ -48,6 +49,7 @@ lib.gdn_chunk_fwd_host.argtypes = [_vp] * 8 + [_i] * 7 + [_f, _i, _vp, _vp, _i, 
 lib.gdn_chunk_fwd_host_workspace_bytes.argtypes = [_i] * 9
 lib.gdn_chunk_fwd_host_workspace_bytes.restype = _sz
 lib.gdn_recurrent_step.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _vp]
+lib.gdn_conv_prefill.argtypes = [_vp] * 6 + [_i] * 7 + [_vp]
 lib.gdn_chunk_workspace_bytes.argtypes = [_i] * 7
 lib.gdn2_chunk_workspace_bytes.argtypes = [_i] * 6
 lib.gdn_chunk_workspace_bytes.restype = _sz
@@ -58,7 +60,7 @@ lib.gdn_status_string.restype = ctypes.c_char_p
 lib.gdn_version.argtypes = []
 for _fn in (lib.gdn_gate_prep, lib.gdn_chunk_fwd, lib.gdn_chunk_fwd_noalloc, lib.gdn_chunk_fwd_host,
             lib.gdn2_chunk_fwd,
-            lib.gdn_recurrent_step, lib.gdn_check_status, lib.gdn_version):
+            lib.gdn_recurrent_step, lib.gdn_conv_prefill, lib.gdn_check_status, lib.gdn_version):
     _fn.restype = _i
 
 
@@ -328,6 +330,31 @@ def gdn_recurrent_step(x, conv_w, conv_state, a, b, A_log, dt_bias, state, *, Hk
                                   _stream(stream)),
            "gdn_recurrent_step")
     return o
+
+
+def gdn_conv_prefill(x, conv_w, conv_state, *, Hk, Hv, dk, dv, q=None, k=None, v=None,
+                     stream=None):
+    """Causal conv1d (kernel 4) + SiLU over a prefill of the mixed stream
+    x [B, T, 2*Hk*dk + Hv*dv]; conv_state [B, Cc, 3] (or None: a zero window) is
+    read and then overwritten in place with the last three inputs.  Returns
+    (q [B,T,Hk,dk], k [B,T,Hk,dk], v [B,T,Hv,dv]), not normalised."""
+    B, T = x.shape[0], x.shape[1]
+    dt = x.dtype
+    Cc = 2 * Hk * dk + Hv * dv
+    _need(x, dt, (B, T, Cc), "x")
+    _need(conv_w, torch.float32, (Cc, 4), "conv_w")
+    if conv_state is not None:
+        _need(conv_state, dt, (B, Cc, 3), "conv_state")
+    q = torch.empty((B, T, Hk, dk), device=x.device, dtype=dt) if q is None else q
+    k = torch.empty((B, T, Hk, dk), device=x.device, dtype=dt) if k is None else k
+    v = torch.empty((B, T, Hv, dv), device=x.device, dtype=dt) if v is None else v
+    _need(q, dt, (B, T, Hk, dk), "q")
+    _need(k, dt, (B, T, Hk, dk), "k")
+    _need(v, dt, (B, T, Hv, dv), "v")
+    _check(lib.gdn_conv_prefill(_p(x), _p(conv_w), _p(conv_state), _p(q), _p(k), _p(v), B, T,
+                                Hk, Hv, dk, dv, _dtype_code(dt), _stream(stream)),
+           "gdn_conv_prefill")
+    return q, k, v
 
 
 def gdn_check_status(stream=None):

@@ -172,6 +172,20 @@ int gdn_recurrent_step(const void* x_qkv, const float* conv_w, void* conv_state,
                                          (flags & GDN_OUT_F32) != 0, (cudaStream_t)stream));
 }
 
+int gdn_conv_prefill(const void* x_qkv, const float* conv_w, void* conv_state, void* q, void* k,
+                     void* v, int B, int T, int Hk, int Hv, int dk, int dv, int dtype,
+                     gdn_stream_t stream) {
+  if (B < 0 || T < 0 || Hk <= 0 || Hv <= 0 || !ok_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  if (!ok_head_dim(dk) || !ok_head_dim(dv)) return GDN_ERR_UNSUPPORTED;
+  if (B == 0 || T == 0) return GDN_OK;
+  if ((T + 15) / 16 > 65535 || B > 65535) return GDN_ERR_UNSUPPORTED;
+  if (!ok_ptr(x_qkv) || !ok_ptr(conv_w) || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) ||
+      (conv_state != nullptr && !ok_elem(conv_state, elem_size(dtype))))
+    return GDN_ERR_INVALID_ARG;
+  return from_cuda(launch_conv_prefill(x_qkv, conv_w, conv_state, q, k, v, B, T, Hk, Hv, dk, dv,
+                                       dtype, (cudaStream_t)stream));
+}
+
 int gdn_check_status(gdn_stream_t stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDN_ERR_CUDA;
   int h = 0;

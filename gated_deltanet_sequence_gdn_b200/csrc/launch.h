@@ -28,6 +28,10 @@ cudaError_t launch_recurrent_step(const void* x, const float* conv_w, void* conv
                                   int Hk, int Hv, int dk, int dv, int dtype, float scale,
                                   bool out_f32, cudaStream_t s);
 
+cudaError_t launch_conv_prefill(const void* x, const float* conv_w, void* conv_state, void* q,
+                                void* k, void* v, int B, int T, int Hk, int Hv, int dk, int dv,
+                                int dtype, cudaStream_t s);
+
 // float32 CUDA-core chunk path (GDN and, with gdn2 = true, Gated DeltaNet-2).
 cudaError_t launch_chunk_simt(const ChunkArgs& a, bool gdn2, cudaStream_t s);
 

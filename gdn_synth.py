@@ -24,7 +24,7 @@ LN16 = math.log(16.0)
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str            # "gdn" | "decode" | "gdn2"
+    kind: str            # "gdn" | "decode" | "gdn2" | "conv"
     B: int
     T: int
     Hk: int
@@ -48,6 +48,9 @@ WORKLOADS = {
     "prefill_b8_16k": Workload("prefill_b8_16k", "gdn", 8, 16384, 16, 64, 128, torch.bfloat16, 1002),
     "decode_256": Workload("decode_256", "decode", 256, 1, 16, 64, 128, torch.bfloat16, 1003, steps=64),
     "gdn2_b4_4k": Workload("gdn2_b4_4k", "gdn2", 4, 4096, 16, 16, 128, torch.bfloat16, 1004),
+    # the prefill conv1d + SiLU over the mixed stream of the prefill_8k layer
+    "conv_prefill_8k": Workload("conv_prefill_8k", "conv", 1, 8192, 16, 64, 128, torch.bfloat16,
+                                1005),
 }
 
 
@@ -133,6 +136,20 @@ def decode_inputs(N, steps, Hk, Hv, d, dtype, seed, device="cpu", dv=None):
     }
 
 
+def conv_prefill_inputs(B, T, Hk, Hv, d, dtype, seed, device="cpu", dv=None):
+    """Inputs of one prefill conv call: x [B,T,Cc] pre-conv mixed [q|k|v] stream,
+    Cc = 2*Hk*d + Hv*dv, in ``dtype``; conv_w [Cc,4] fp32; conv_state [B,Cc,3]
+    ``dtype`` (the same distributions as the decode inputs)."""
+    dv = d if dv is None else dv
+    Cc = 2 * Hk * d + Hv * dv
+    g = _gen(seed, device)
+    return {
+        "x": _randn((B, T, Cc), g, device, dtype),
+        "conv_w": _uniform((Cc, 4), -0.5, 0.5, g, device),
+        "conv_state": _randn((B, Cc, 3), g, device, dtype),
+    }
+
+
 def workload_inputs(w: Workload, device="cpu"):
     if w.kind == "gdn":
         return gdn_inputs(w.B, w.T, w.Hk, w.Hv, w.d, w.dtype, w.seed, device, h0=w.h0)
@@ -140,4 +157,6 @@ def workload_inputs(w: Workload, device="cpu"):
         return gdn2_inputs(w.B, w.T, w.Hv, w.d, w.dtype, w.seed, device, h0=w.h0)
     if w.kind == "decode":
         return decode_inputs(w.B, w.steps, w.Hk, w.Hv, w.d, w.dtype, w.seed, device)
+    if w.kind == "conv":
+        return conv_prefill_inputs(w.B, w.T, w.Hk, w.Hv, w.d, w.dtype, w.seed, device)
     raise ValueError(w.kind)

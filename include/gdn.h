@@ -217,6 +217,36 @@ int gdn_recurrent_step(const void* x_qkv, const float* conv_w, void* conv_state,
                        int flags, gdn_stream_t stream);
 
 /*
+ * gdn_conv_prefill -- the causal depthwise conv1d (kernel 4) + SiLU over a
+ * whole prefill of the mixed [q | k | v] channel stream ("从 Full Attention 到
+ * Gated DeltaNet" section 10: x -> CausalConv1D -> SiLU -> q, k, v;
+ * "gated-deltanet-qwen3.5" section 因果卷积 and its architecture diagram, whose
+ * conv_states carry the window into the inference branch).  The same conv as
+ * gdn_recurrent_step, over T tokens at once: running it, then T decode steps'
+ * worth of inputs one at a time, gives the same window and outputs.
+ *   x_qkv      [B, T, Cc] dtype, Cc = 2*Hk*dk + Hv*dv, channel order q | k | v
+ *   conv_w     [Cc, 4] float32; tap 3 multiplies the newest input
+ *   conv_state [B, Cc, 3] dtype (index 2 newest) or NULL.  Non-NULL: read as the
+ *              three inputs before token 0, then overwritten with the last three
+ *              inputs (for T < 3 partly the old window, shifted).  NULL: a zero
+ *              window, and nothing is written.
+ *   q, k       [B, T, Hk, dk] dtype, written: SiLU(conv) of the q / k channels
+ *              (not normalised: gdn_chunk_fwd with GDN_QK_L2NORM applies the L2
+ *              norm in its prologue)
+ *   v          [B, T, Hv, dv] dtype, written
+ *   Ownership: every pointer is a device pointer owned by the caller; x_qkv,
+ *   conv_w, q, k and v 16-byte aligned, conv_state element aligned; q, k, v must
+ *   not overlap x_qkv or each other.  Arithmetic in float32, outputs rounded to
+ *   dtype once.  B = 0 or T = 0 enqueues nothing (the window is unchanged).
+ *   Returns GDN_ERR_INVALID_ARG (null or misaligned pointer, negative size, bad
+ *   dtype), GDN_ERR_UNSUPPORTED (dk or dv not 64 / 128, more than 65535 * 16
+ *   tokens or 65535 sequences), GDN_ERR_CUDA (launch failure).
+ */
+int gdn_conv_prefill(const void* x_qkv, const float* conv_w, void* conv_state,
+                     void* q, void* k, void* v, int B, int T, int Hk, int Hv,
+                     int dk, int dv, int dtype, gdn_stream_t stream);
+
+/*
  * gdn2_chunk_fwd -- chunkwise Gated DeltaNet-2 forward ("Gated DeltaNet-2",
  * 新更新公式 and 高效训练): channel-wise decay
  * D_t = diag(exp(-exp(A_log) (.) softplus(a_t + dt_bias))), erase gate

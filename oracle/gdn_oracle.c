@@ -223,6 +223,19 @@ int oracle_conv_step(const void* x, const void* conv_w, int in_f64, int N,
   return ORACLE_OK;
 }
 
+/* The conv step over a whole prefill, token after token (the window carried
+ * from one token to the next exactly as between decode steps):
+ * x [B, T, Cc], conv_state [B, Cc, 3] (float64) in/out, y [B, T, Cc] out. */
+int oracle_conv_prefill(const void* x, const void* conv_w, int in_f64, int B, int T,
+                        int Cc, double* conv_state, double* y) {
+  if (B < 0 || T < 0 || Cc <= 0) return ORACLE_EINVAL;
+  for (int b = 0; b < B; ++b)
+    for (int t = 0; t < T; ++t)
+      conv_silu_step(x, ((size_t)b * T + t) * Cc, conv_w, in_f64, Cc,
+                     conv_state + (size_t)b * Cc * 3, y + ((size_t)b * T + t) * Cc);
+  return ORACLE_OK;
+}
+
 /*
  * One decode step for the selected sequences: the conv step above over the
  * mixed [q | k | v] channel stream, then per value head the L2 norm, gates and

@@ -14,6 +14,8 @@ Each function cites the passage it follows (page title and section):
 * ``decode_step``  -- "gated-deltanet-qwen3.5" architecture diagram (decode
   updates conv_states / recurrent_states) and section 10 of the dingfen page
   (Linear -> CausalConv1D -> SiLU -> q, k, v).
+* ``conv_step`` / ``conv_prefill`` -- that conv alone, for one token or a whole
+  prefill ("gated-deltanet-qwen3.5" section 因果卷积: kernel 4, depthwise, causal).
 * ``gdn2_fwd``     -- "Gated DeltaNet-2" (zhichai), section 新更新公式.
 
 Parity: pinned by tests/test_oracle_pins.py (closed forms, special cases,
@@ -61,7 +63,9 @@ def _load():
             lib.oracle_gdn_decode_step.argtypes = [vp] * 6 + [ip] * 6 + [dp, ip, vp, vp, vp, vp, ip]
             lib.oracle_gdn2_fwd.argtypes = [vp] * 9 + [ip] * 6 + [dp, ip, ip, ip, vp, vp, vp, ip]
             lib.oracle_conv_step.argtypes = [vp, vp, ip, ip, ip, vp, vp]
+            lib.oracle_conv_prefill.argtypes = [vp, vp, ip, ip, ip, ip, vp, vp]
             for f in (lib.oracle_gdn_fwd, lib.oracle_gate_prep, lib.oracle_conv_step,
+                      lib.oracle_conv_prefill,
                       lib.oracle_gdn_decode_step, lib.oracle_gdn2_fwd):
                 f.restype = ctypes.c_int
             lib.oracle_max_threads.restype = ctypes.c_int
@@ -175,6 +179,24 @@ def conv_step(x, conv_w, conv_state):
     y = np.zeros((N, Cc))
     rc = _load().oracle_conv_step(_ptr(xa), _ptr(wa), int(f64), N, Cc, _ptr(conv_state), _ptr(y))
     _check(rc, "oracle_conv_step")
+    return y
+
+
+def conv_prefill(x, conv_w, conv_state):
+    """The conv step over a whole prefill, token after token.
+
+    x: [B, T, Cc]; conv_w: [Cc, 4]; conv_state: float64 [B, Cc, 3] updated IN
+    PLACE (it ends holding the last three inputs).  Returns y [B, T, Cc] float64.
+    """
+    B, T, Cc = x.shape
+    f64 = _is_f64(x, conv_w)
+    xa, wa = _arr(x, f64), _arr(conv_w, f64)
+    assert conv_state.dtype == np.float64 and conv_state.flags.c_contiguous
+    assert conv_state.shape == (B, Cc, 3)
+    y = np.zeros((B, T, Cc))
+    rc = _load().oracle_conv_prefill(_ptr(xa), _ptr(wa), int(f64), B, T, Cc, _ptr(conv_state),
+                                     _ptr(y))
+    _check(rc, "oracle_conv_prefill")
     return y
 
 

@@ -124,6 +124,24 @@ def test_gdn2_and_decode_reject_bad_arguments():
                            FAKE, FAKE, FAKE, None) == -1
 
 
+def test_conv_prefill_rejects_bad_arguments():
+    cp = G.lib.gdn_conv_prefill
+    # (x, conv_w, conv_state, q, k, v, B, T, Hk, Hv, dk, dv, dtype, stream)
+    assert cp(None, FAKE, None, FAKE, FAKE, FAKE, 1, 8, 2, 4, 128, 128, 1, None) == -1
+    assert cp(FAKE, None, None, FAKE, FAKE, FAKE, 1, 8, 2, 4, 128, 128, 1, None) == -1
+    assert cp(FAKE, FAKE, None, FAKE, None, FAKE, 1, 8, 2, 4, 128, 128, 1, None) == -1
+    assert cp(FAKE + 8, FAKE, None, FAKE, FAKE, FAKE, 1, 8, 2, 4, 128, 128, 1, None) == -1
+    assert cp(FAKE, FAKE, FAKE + 1, FAKE, FAKE, FAKE, 1, 8, 2, 4, 128, 128, 1, None) == -1
+    assert cp(FAKE, FAKE, None, FAKE, FAKE, FAKE, -1, 8, 2, 4, 128, 128, 1, None) == -1
+    assert cp(FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, 8, 2, 4, 128, 128, 7, None) == -1
+    assert cp(FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, 8, 2, 4, 96, 128, 1, None) == -2
+    assert cp(FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, 16 * 65535 + 1, 2, 4, 128, 128, 1,
+              None) == -2
+    # no tokens or no sequences: nothing enqueued, the window untouched
+    assert cp(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 0, 2, 4, 128, 128, 1, None) == 0
+    assert cp(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 2, 4, 128, 128, 1, None) == 0
+
+
 def test_empty_calls_are_no_ops():
     # zero tokens / zero sequences return before any launch (no state pointers)
     assert _chunk(T=0) == 0

@@ -47,6 +47,12 @@ MUTANTS = [
      "    double acc = ld(conv_w, in_f64, (size_t)c * 4 + 0) * cs[c * 3 + 0] +",
      "    double acc = ld(conv_w, in_f64, (size_t)c * 4 + 3) * cs[c * 3 + 0] +"),
     ("conv_no_shift", "    cs[c * 3 + 0] = cs[c * 3 + 1];\n", "\n"),
+    ("conv_prefill_shared_window",  # every sequence of the batch reads one window
+     "                     conv_state + (size_t)b * Cc * 3, y + ((size_t)b * T + t) * Cc);",
+     "                     conv_state, y + ((size_t)b * T + t) * Cc);"),
+    ("conv_prefill_time_major",  # x read as [T, B, Cc]
+     "      conv_silu_step(x, ((size_t)b * T + t) * Cc, conv_w, in_f64, Cc,",
+     "      conv_silu_step(x, ((size_t)t * B + b) * Cc, conv_w, in_f64, Cc,"),
     ("gdn2_decay_value_side",
      "        for (int j = 0; j < dv; ++j) S[(size_t)i * dv + j] *= dec[i];",
      "        for (int j = 0; j < dv; ++j) S[(size_t)i * dv + j] *= dec[j < dk ? j : 0];"),
@@ -75,7 +81,7 @@ def _run_pins_against(lib_path):
     real = O._load()
     mutant = ctypes.CDLL(lib_path)
     for fname in ("oracle_gdn_fwd", "oracle_gate_prep", "oracle_conv_step",
-                  "oracle_gdn_decode_step", "oracle_gdn2_fwd"):
+                  "oracle_conv_prefill", "oracle_gdn_decode_step", "oracle_gdn2_fwd"):
         getattr(mutant, fname).argtypes = getattr(real, fname).argtypes
         getattr(mutant, fname).restype = ctypes.c_int
     mutant.oracle_max_threads.restype = ctypes.c_int

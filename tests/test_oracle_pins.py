@@ -309,6 +309,47 @@ def test_conv_step_matches_library_conv1d():
     np.testing.assert_array_equal(cs, np.concatenate([cs0, xs.transpose(1, 2, 0)], 2)[:, :, -3:])
 
 
+@pytest.mark.parametrize("T", [1, 2, 3, 7])
+def test_conv_prefill_matches_library_conv1d(T):
+    """The conv over a whole prefill equals torch's grouped conv1d over the carried
+    window followed by the new inputs, then SiLU; the window it leaves is the last
+    three entries of that stream (for T < 3 partly the old window, shifted)."""
+    B, Cc = 2, 12
+    w = rng.uniform(-0.5, 0.5, size=(Cc, 4))
+    cs0 = _rand(B, Cc, 3)
+    x = _rand(B, T, Cc)
+    cs = cs0.copy()
+    y = O.conv_prefill(x, w, cs)
+    stream = torch.cat([torch.from_numpy(cs0), torch.from_numpy(x).permute(0, 2, 1)], dim=2)
+    ref = torch.nn.functional.silu(
+        torch.nn.functional.conv1d(stream, torch.from_numpy(w)[:, None, :], groups=Cc))
+    np.testing.assert_allclose(y, ref.permute(0, 2, 1).numpy(), rtol=1e-13, atol=1e-14)
+    np.testing.assert_array_equal(cs, stream.numpy()[:, :, -3:])
+
+
+def test_conv_prefill_streams():
+    """Two prefills with the window carried equal one prefill over both, and a zero
+    window at the start equals zero padding (causality: output t sees inputs <= t)."""
+    B, Cc, T1, T2 = 2, 8, 5, 9
+    w = rng.uniform(-0.5, 0.5, size=(Cc, 4))
+    x = _rand(B, T1 + T2, Cc)
+    cs = np.zeros((B, Cc, 3))
+    y = O.conv_prefill(x, w, cs)
+    cs_a = np.zeros((B, Cc, 3))
+    ya = O.conv_prefill(x[:, :T1], w, cs_a)
+    yb = O.conv_prefill(x[:, T1:], w, cs_a)
+    np.testing.assert_array_equal(np.concatenate([ya, yb], 1), y)
+    np.testing.assert_array_equal(cs_a, cs)
+    # causality: changing input t0 leaves the outputs before t0 unchanged and
+    # changes outputs t0 .. t0 + 3 only
+    x2 = x.copy()
+    x2[:, 6] += 1.0
+    y2 = O.conv_prefill(x2, w, np.zeros((B, Cc, 3)))
+    np.testing.assert_array_equal(y2[:, :6], y[:, :6])
+    np.testing.assert_array_equal(y2[:, 10:], y[:, 10:])
+    assert np.all(np.abs(y2[:, 6] - y[:, 6]) > 0)
+
+
 def test_decode_steps_equal_prefill_on_conv_stream():
     """A run of decode steps (conv fused) equals the conv step followed by the
     prefill oracle over the resulting q, k, v stream, with the state carried."""
