@@ -10,15 +10,19 @@
 // prologue (gdn_chunk_fwd with GDN_QK_L2NORM), which fuses it.
 //
 // HBM-bound: every input and every output element crosses HBM once.  A thread
-// takes 8 channels (16 bytes of bf16) of 16 consecutive tokens, loading them in
-// batches of 8 rows before using any; consecutive threads take consecutive
-// channel groups, so each warp reads and writes whole 512-byte runs of a token
-// row.  The three inputs before a token tile are re-read (from L2) by the tile's
-// threads.  The conv window in conv_state is read and rewritten only by the
+// takes 8 channels (16 bytes of bf16) of 16 consecutive tokens; consecutive
+// threads take consecutive channel groups, so each warp reads and writes whole
+// 512-byte runs of a token row.  A thread stages its input rows in shared memory
+// with asynchronous copies issued all at once (the three inputs before the tile
+// and its first 8 tokens, then the other 8), and works on the first 8 while the
+// rest arrive; it reads back only the rows it copied itself, so no barrier is
+// needed.  The three inputs before a token tile are re-read (from L2) by the
+// tile's threads.  The conv window in conv_state is read and rewritten only by the
 // threads of the first token tile, so an in-place update has no race between
 // CTAs.
 #include "common.cuh"
 #include "launch.h"
+#include "warp_mma.cuh"
 
 namespace gdn {
 namespace {
@@ -33,11 +37,9 @@ constexpr int kTT = 16;   // tokens per thread
 __device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.f + __expf(-x)); }
 
 // 8 channels of one token as loaded (16 bytes of bf16, 32 of fp32), and their
-// float32 values; rows of a batch are loaded before any is used, so that a
-// thread keeps a batch of 16-byte loads in flight.
+// float32 values.
 template <typename T> struct Raw8;
 template <> struct Raw8<__nv_bfloat16> {
-  static constexpr int kBatch = 8;
   uint4 u;
   __device__ __forceinline__ void load(const __nv_bfloat16* p) {
     u = *reinterpret_cast<const uint4*>(p);
@@ -53,7 +55,6 @@ template <> struct Raw8<__nv_bfloat16> {
   }
 };
 template <> struct Raw8<float> {
-  static constexpr int kBatch = 4;
   float4 a, b;
   __device__ __forceinline__ void load(const float* p) {
     a = reinterpret_cast<const float4*>(p)[0];
@@ -92,28 +93,52 @@ __device__ __forceinline__ void store8<float>(float* p, const float* f) {
 // x [B, T, Cc] with Cc = 2 QK + V (channel order q | k | v); conv_w [Cc, 4]
 // (tap 3 multiplies the newest input); conv_state [B, Cc, 3] (index 2 newest) or
 // null (a zero window, nothing written back); q, k [B, T, QK]; v [B, T, V].
+// Shared memory: rows r = 0 .. kTT + 2 (input t0 - 3 + r) of kCT threads x 8 channels.
+template <typename T>
+constexpr int conv_stage_bytes() { return (kTT + 3) * kCT * 8 * (int)sizeof(T); }
+
 template <typename T>
 __global__ void __launch_bounds__(kCT)
 conv_prefill_kernel(const T* __restrict__ x, const float* __restrict__ conv_w, T* conv_state,
                     T* __restrict__ q, T* __restrict__ k, T* __restrict__ v, int Tn, int Cc,
                     int QK, int V) {
+  extern __shared__ __align__(16) uint8_t stage[];
+  constexpr int EB = 8 * (int)sizeof(T);  // bytes of 8 channels
   const int cg = blockIdx.x * kCT + threadIdx.x;
-  if (cg >= Cc / 8) return;
+  if (cg >= Cc / 8) return;  // no barrier in this kernel
   const int c0 = 8 * cg, t0 = blockIdx.y * kTT, bb = blockIdx.z;
+  const int tn = min(kTT, Tn - t0);
+  const T* xb = x + (size_t)bb * Tn * Cc + c0;
+  uint8_t* my = stage + threadIdx.x * EB;  // row r of this thread at my + r * kCT * EB
+  {
+    const int r_end[2] = {3 + min(tn, 8), 3 + tn};
+    int r = t0 > 0 ? 0 : 3;
+#pragma unroll
+    for (int grp = 0; grp < 2; ++grp) {
+      for (; r < r_end[grp]; ++r) {
+        const T* src = xb + (size_t)(t0 - 3 + r) * Cc;
+#pragma unroll
+        for (int h = 0; h < EB / 16; ++h)
+          wm::cp16(my + (size_t)r * kCT * EB + 16 * h, src + h * (16 / (int)sizeof(T)), 16);
+      }
+      wm::cp_commit();
+    }
+  }
   float w[8][4];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const float4 t = *reinterpret_cast<const float4*>(conv_w + (size_t)(c0 + u) * 4);
     w[u][0] = t.x, w[u][1] = t.y, w[u][2] = t.z, w[u][3] = t.w;
   }
-  const T* xb = x + (size_t)bb * Tn * Cc + c0;
   T* cs = conv_state == nullptr ? nullptr : conv_state + ((size_t)bb * Cc + c0) * 3;
+  auto srow = [&](int r) { return reinterpret_cast<const T*>(my + (size_t)r * kCT * EB); };
   // the window before t0: inputs t0 - 3, t0 - 2, t0 - 1 (from the carried window at t0 = 0)
   float h0[8], h1[8], h2[8];
+  wm::cp_wait<1>();  // the first group: the window rows and tokens 0 .. 7
   if (t0 > 0) {
-    load8(xb + (size_t)(t0 - 3) * Cc, h0);
-    load8(xb + (size_t)(t0 - 2) * Cc, h1);
-    load8(xb + (size_t)(t0 - 1) * Cc, h2);
+    load8(srow(0), h0);
+    load8(srow(1), h1);
+    load8(srow(2), h2);
   } else {
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -128,29 +153,18 @@ conv_prefill_kernel(const T* __restrict__ x, const float* __restrict__ conv_w, T
   else if (c0 < 2 * QK) dst = k + (c0 - QK), ld = QK;
   else dst = v + (c0 - 2 * QK), ld = V;
   dst += ((size_t)bb * Tn + t0) * ld;
-  const int tn = min(kTT, Tn - t0);
-  constexpr int NB = Raw8<T>::kBatch;
 #pragma unroll 1
-  for (int ib = 0; ib < tn; ib += NB) {
-    Raw8<T> raw[NB];
+  for (int i = 0; i < tn; ++i) {
+    if (i == 8) wm::cp_wait<0>();  // the second group: tokens 8 .. 15
+    float xn[8], y[8];
+    load8(srow(3 + i), xn);
 #pragma unroll
-    for (int j = 0; j < NB; ++j)
-      if (ib + j < tn) raw[j].load(xb + (size_t)(t0 + ib + j) * Cc);
-#pragma unroll
-    for (int j = 0; j < NB; ++j) {
-      if (ib + j < tn) {
-        float xn[8], y[8];
-        raw[j].get(xn);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float acc =
-              w[u][0] * h0[u] + w[u][1] * h1[u] + w[u][2] * h2[u] + w[u][3] * xn[u];
-          y[u] = silu_fast(acc);
-          h0[u] = h1[u], h1[u] = h2[u], h2[u] = xn[u];
-        }
-        store8(dst + (size_t)(ib + j) * ld, y);
-      }
+    for (int u = 0; u < 8; ++u) {
+      const float acc = w[u][0] * h0[u] + w[u][1] * h1[u] + w[u][2] * h2[u] + w[u][3] * xn[u];
+      y[u] = silu_fast(acc);
+      h0[u] = h1[u], h1[u] = h2[u], h2[u] = xn[u];
     }
+    store8(dst + (size_t)i * ld, y);
   }
   // the window after the last token (inputs Tn - 3 .. Tn - 1; for Tn < 3 partly
   // the carried window), all read before any is written
@@ -187,11 +201,19 @@ cudaError_t launch_conv_prefill(const void* x, const float* conv_w, void* conv_s
   if (grid.y > 65535u || grid.z > 65535u) return cudaErrorInvalidValue;
   if (dtype == GDN_BF16) {
     using bf16 = __nv_bfloat16;
-    conv_prefill_kernel<bf16><<<grid, kCT, 0, s>>>(
+    constexpr int smem = conv_stage_bytes<bf16>();
+    cudaError_t e = cudaFuncSetAttribute(conv_prefill_kernel<bf16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    conv_prefill_kernel<bf16><<<grid, kCT, smem, s>>>(
         static_cast<const bf16*>(x), conv_w, static_cast<bf16*>(conv_state),
         static_cast<bf16*>(q), static_cast<bf16*>(k), static_cast<bf16*>(v), T, Cc, QK, V);
   } else {
-    conv_prefill_kernel<float><<<grid, kCT, 0, s>>>(
+    constexpr int smem = conv_stage_bytes<float>();
+    cudaError_t e = cudaFuncSetAttribute(conv_prefill_kernel<float>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    conv_prefill_kernel<float><<<grid, kCT, smem, s>>>(
         static_cast<const float*>(x), conv_w, static_cast<float*>(conv_state),
         static_cast<float*>(q), static_cast<float*>(k), static_cast<float*>(v), T, Cc, QK, V);
   }
