@@ -27,7 +27,7 @@
 namespace gdn {
 namespace {
 
-constexpr int kCT = 256;  // threads per CTA
+constexpr int kCT = 128;  // threads per CTA (five CTAs per SM: their load and SiLU phases stagger)
 constexpr int kTT = 16;   // tokens per thread
 
 // SiLU(x) = x / (1 + e^-x) with the hardware exp2 and reciprocal approximations
