@@ -34,6 +34,10 @@
  *  - Decode conv: torch-style causal cross-correlation over the window
  *    [cs0, cs1, cs2, x] with weight taps w[c][0..3]; cs2 is the newest cached
  *    input; SiLU(y) = y * sigmoid(y); no bias.
+ *  - Gated RMSNorm of the output ("gated-deltanet-qwen3.5" section 输出门控与
+ *    RMSNorm: RMSNormGated(core_attn_out, z), an RMSNorm and then the output
+ *    gate, SwiGLU-like): per token and value head, over the d_v channels,
+ *    y = o / sqrt(mean(o^2) + eps) * weight * SiLU(z).
  *
  * Parity: pinned (see tests/test_oracle_pins.py): linear-attention brute force,
  * delta-rule overwrite on orthonormal keys, per-step overwrite identity, pure
@@ -371,6 +375,27 @@ int oracle_gdn2_fwd(const void* q, const void* k, const void* v, const void* a,
     free(buf);
   }
   return err;
+}
+
+/* Gated RMSNorm of N rows of d_v channels: o, z [N, dv], weight [dv] (shared by
+ * every row), y [N, dv] out. */
+int oracle_rmsnorm_gated(const void* o, const void* z, const void* weight, int in_f64,
+                         int N, int dv, double eps, double* y) {
+  if (N < 0 || dv <= 0 || !(eps >= 0.0)) return ORACLE_EINVAL;
+  for (int n = 0; n < N; ++n) {
+    double ss = 0.0;
+    for (int j = 0; j < dv; ++j) {
+      const double v = ld(o, in_f64, (size_t)n * dv + j);
+      ss += v * v;
+    }
+    const double inv = 1.0 / sqrt(ss / dv + eps);
+    for (int j = 0; j < dv; ++j) {
+      const double zj = ld(z, in_f64, (size_t)n * dv + j);
+      y[(size_t)n * dv + j] =
+          ld(o, in_f64, (size_t)n * dv + j) * inv * ld(weight, in_f64, (size_t)j) * (zj * sigmoid(zj));
+    }
+  }
+  return ORACLE_OK;
 }
 
 int oracle_max_threads(void) {

@@ -16,6 +16,8 @@ Each function cites the passage it follows (page title and section):
   (Linear -> CausalConv1D -> SiLU -> q, k, v).
 * ``conv_step`` / ``conv_prefill`` -- that conv alone, for one token or a whole
   prefill ("gated-deltanet-qwen3.5" section 因果卷积: kernel 4, depthwise, causal).
+* ``rmsnorm_gated`` -- "gated-deltanet-qwen3.5" section 输出门控与 RMSNorm
+  (RMSNormGated(core_attn_out, z): the norm, then the SwiGLU-like z gate).
 * ``gdn2_fwd``     -- "Gated DeltaNet-2" (zhichai), section 新更新公式.
 
 Parity: pinned by tests/test_oracle_pins.py (closed forms, special cases,
@@ -64,8 +66,9 @@ def _load():
             lib.oracle_gdn2_fwd.argtypes = [vp] * 9 + [ip] * 6 + [dp, ip, ip, ip, vp, vp, vp, ip]
             lib.oracle_conv_step.argtypes = [vp, vp, ip, ip, ip, vp, vp]
             lib.oracle_conv_prefill.argtypes = [vp, vp, ip, ip, ip, ip, vp, vp]
+            lib.oracle_rmsnorm_gated.argtypes = [vp, vp, vp, ip, ip, ip, dp, vp]
             for f in (lib.oracle_gdn_fwd, lib.oracle_gate_prep, lib.oracle_conv_step,
-                      lib.oracle_conv_prefill,
+                      lib.oracle_conv_prefill, lib.oracle_rmsnorm_gated,
                       lib.oracle_gdn_decode_step, lib.oracle_gdn2_fwd):
                 f.restype = ctypes.c_int
             lib.oracle_max_threads.restype = ctypes.c_int
@@ -197,6 +200,24 @@ def conv_prefill(x, conv_w, conv_state):
     rc = _load().oracle_conv_prefill(_ptr(xa), _ptr(wa), int(f64), B, T, Cc, _ptr(conv_state),
                                      _ptr(y))
     _check(rc, "oracle_conv_prefill")
+    return y
+
+
+def rmsnorm_gated(o, z, weight, *, eps=1e-6):
+    """Gated RMSNorm of the core output: per row of the last axis (d_v),
+    y = o / sqrt(mean(o^2) + eps) * weight * SiLU(z).
+
+    o, z: [..., dv] (same shape); weight: [dv].  Returns y float64, o's shape.
+    """
+    f64 = _is_f64(o, z, weight)
+    oa, za, wa = _arr(o, f64), _arr(z, f64), _arr(weight, f64)
+    assert oa.shape == za.shape and wa.shape == (oa.shape[-1],)
+    dv = oa.shape[-1]
+    N = oa.size // dv
+    y = np.zeros(oa.shape)
+    rc = _load().oracle_rmsnorm_gated(_ptr(oa), _ptr(za), _ptr(wa), int(f64), N, dv, float(eps),
+                                      _ptr(y))
+    _check(rc, "oracle_rmsnorm_gated")
     return y
 
 

@@ -53,6 +53,17 @@ MUTANTS = [
     ("conv_prefill_time_major",  # x read as [T, B, Cc]
      "      conv_silu_step(x, ((size_t)b * T + t) * Cc, conv_w, in_f64, Cc,",
      "      conv_silu_step(x, ((size_t)t * B + b) * Cc, conv_w, in_f64, Cc,"),
+    ("rmsnorm_mean_as_sum",  # the sum of squares not divided by d_v
+     "    const double inv = 1.0 / sqrt(ss / dv + eps);",
+     "    const double inv = 1.0 / sqrt(ss + eps);"),
+    ("rmsnorm_eps_outside",
+     "    const double inv = 1.0 / sqrt(ss / dv + eps);",
+     "    const double inv = 1.0 / (sqrt(ss / dv) + eps);"),
+    ("rmsnorm_gate_sigmoid",  # sigmoid(z) in place of SiLU(z)
+     " * (zj * sigmoid(zj));", " * (sigmoid(zj));"),
+    ("rmsnorm_weight_dropped",
+     "ld(o, in_f64, (size_t)n * dv + j) * inv * ld(weight, in_f64, (size_t)j) * (zj * sigmoid(zj));",
+     "ld(o, in_f64, (size_t)n * dv + j) * inv * (zj * sigmoid(zj));"),
     ("gdn2_decay_value_side",
      "        for (int j = 0; j < dv; ++j) S[(size_t)i * dv + j] *= dec[i];",
      "        for (int j = 0; j < dv; ++j) S[(size_t)i * dv + j] *= dec[j < dk ? j : 0];"),
@@ -81,7 +92,8 @@ def _run_pins_against(lib_path):
     real = O._load()
     mutant = ctypes.CDLL(lib_path)
     for fname in ("oracle_gdn_fwd", "oracle_gate_prep", "oracle_conv_step",
-                  "oracle_conv_prefill", "oracle_gdn_decode_step", "oracle_gdn2_fwd"):
+                  "oracle_conv_prefill", "oracle_rmsnorm_gated", "oracle_gdn_decode_step",
+                  "oracle_gdn2_fwd"):
         getattr(mutant, fname).argtypes = getattr(real, fname).argtypes
         getattr(mutant, fname).restype = ctypes.c_int
     mutant.oracle_max_threads.restype = ctypes.c_int

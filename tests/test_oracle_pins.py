@@ -350,6 +350,40 @@ def test_conv_prefill_streams():
     assert np.all(np.abs(y2[:, 6] - y[:, 6]) > 0)
 
 
+def test_rmsnorm_gated_matches_library_rms_norm_and_silu():
+    """RMSNormGated(o, z) ("gated-deltanet-qwen3.5" 输出门控与 RMSNorm): torch's own
+    rms_norm over the d_v channels (with the weight), times SiLU(z), in float64."""
+    o, z = _rand(2, 5, 3, 16), _rand(2, 5, 3, 16)
+    w = rng.uniform(0.5, 1.5, size=16)
+    y = O.rmsnorm_gated(o, z, w, eps=1e-6)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(o), (16,), torch.from_numpy(w), 1e-6)
+    ref = ref * torch.nn.functional.silu(torch.from_numpy(z))
+    np.testing.assert_allclose(y, ref.numpy(), rtol=1e-13, atol=1e-15)
+
+
+def test_rmsnorm_gated_closed_forms():
+    """Closed forms: a constant row c gives c / sqrt(c^2 + eps) per channel (before the
+    weight and gate); z = 0 closes the gate; the norm sees only its own row; and
+    scaling o by lam with eps scaled by lam^2 leaves y unchanged."""
+    dv, c, eps = 8, -0.75, 1e-6
+    w = rng.uniform(0.5, 1.5, size=dv)
+    z = _rand(1, dv)
+    y = O.rmsnorm_gated(np.full((1, dv), c), z, w, eps=eps)
+    expect = c / math.sqrt(c * c + eps) * w * (z / (1 + np.exp(-z)))
+    np.testing.assert_allclose(y, expect, rtol=1e-14, atol=0)
+    o = _rand(4, dv)
+    assert not O.rmsnorm_gated(o, np.zeros((4, dv)), w).any()
+    o2 = o.copy()
+    o2[1] *= 1000.0  # another row's size does not move row 0
+    y1 = O.rmsnorm_gated(o, z.repeat(4, 0), w)
+    y2 = O.rmsnorm_gated(o2, z.repeat(4, 0), w)
+    np.testing.assert_array_equal(y1[0], y2[0])
+    lam = 37.0
+    np.testing.assert_allclose(O.rmsnorm_gated(lam * o, z.repeat(4, 0), w, eps=lam * lam * eps),
+                               O.rmsnorm_gated(o, z.repeat(4, 0), w, eps=eps), rtol=1e-13,
+                               atol=1e-15)
+
+
 def test_decode_steps_equal_prefill_on_conv_stream():
     """A run of decode steps (conv fused) equals the conv step followed by the
     prefill oracle over the resulting q, k, v stream, with the state carried."""
