@@ -377,6 +377,69 @@ int oracle_gdn2_fwd(const void* q, const void* k, const void* v, const void* a,
   return err;
 }
 
+/*
+ * KDA (Kimi Delta Attention) as the "Gated DeltaNet-2" page states its update
+ * (section 标量绑定的数学表达), computed literally:
+ *   S_t = (I - beta_t k_t k_t^T) D_t S_{t-1} + beta_t k_t v_t^T ;  o_t = S_t^T q_t
+ * with D_t = diag(exp(g_t)), g_t = -exp(A_log) * softplus(a_t + dt_bias) per key
+ * channel, and one scalar beta_t = sigmoid(b_t) per (token, head); the d_k x d_k
+ * erase projection P = I - beta k k^T is formed and applied to D S.
+ *   q,k [B,T,H,dk]; v [B,T,H,dv]; a [B,T,H,dk]; b [B,T,H]; A_log,dt_bias [H,dk];
+ *   h0 [B,H,dk,dv] or NULL.  Out: o [B*H][T][dv], ht [B*H][dk][dv] (either NULL).
+ */
+int oracle_kda_fwd(const void* q, const void* k, const void* v, const void* a,
+                   const void* b, const void* A_log, const void* dt_bias, const void* h0,
+                   int in_f64, int B, int T, int H, int dk, int dv, double scale, int l2norm,
+                   double* o, double* ht, int n_threads) {
+  if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0) return ORACLE_EINVAL;
+  int err = ORACLE_OK;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads > 0 ? n_threads : 1)
+  for (int bh = 0; bh < B * H; ++bh) {
+    const int bi = bh / H, h = bh % H;
+    double* S = (double*)calloc((size_t)dk * dv, sizeof(double));
+    double* DS = (double*)malloc(sizeof(double) * (size_t)dk * dv);
+    double* P = (double*)malloc(sizeof(double) * (size_t)dk * dk);
+    double* buf = (double*)malloc(sizeof(double) * (size_t)(3 * dk + 2 * dv));
+    if (!S || !DS || !P || !buf) {
+      free(S); free(DS); free(P); free(buf);
+#pragma omp atomic write
+      err = ORACLE_ENOMEM;
+      continue;
+    }
+    double *qt = buf, *kt = qt + dk, *dec = kt + dk, *vt = dec + dk, *ot = vt + dv;
+    if (h0)
+      for (size_t x = 0; x < (size_t)dk * dv; ++x)
+        S[x] = ld(h0, in_f64, (size_t)bh * dk * dv + x);
+    for (int t = 0; t < T; ++t) {
+      const size_t row = ((size_t)bi * T + t) * H + h;
+      load_vec(q, in_f64, row * dk, dk, l2norm, scale, qt);
+      load_vec(k, in_f64, row * dk, dk, l2norm, 1.0, kt);
+      load_vec(v, in_f64, row * dv, dv, 0, 1.0, vt);
+      for (int i = 0; i < dk; ++i)
+        dec[i] = exp(-exp(ld(A_log, in_f64, (size_t)h * dk + i)) *
+                     softplus(ld(a, in_f64, row * dk + i) + ld(dt_bias, in_f64, (size_t)h * dk + i)));
+      const double beta = sigmoid(ld(b, in_f64, row));
+      for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) DS[(size_t)i * dv + j] = dec[i] * S[(size_t)i * dv + j];
+      for (int i = 0; i < dk; ++i)
+        for (int l = 0; l < dk; ++l) P[(size_t)i * dk + l] = (i == l ? 1.0 : 0.0) - beta * kt[i] * kt[l];
+      for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) {
+          double acc = beta * kt[i] * vt[j];
+          for (int l = 0; l < dk; ++l) acc += P[(size_t)i * dk + l] * DS[(size_t)l * dv + j];
+          S[(size_t)i * dv + j] = acc;
+        }
+      for (int j = 0; j < dv; ++j) ot[j] = 0.0;
+      for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) ot[j] += S[(size_t)i * dv + j] * qt[i];
+      if (o) memcpy(o + ((size_t)bh * T + t) * dv, ot, sizeof(double) * dv);
+    }
+    if (ht) memcpy(ht + (size_t)bh * dk * dv, S, sizeof(double) * dk * dv);
+    free(S); free(DS); free(P); free(buf);
+  }
+  return err;
+}
+
 /* Gated RMSNorm of N rows of d_v channels: o, z [N, dv], weight [dv] (shared by
  * every row), y [N, dv] out. */
 int oracle_rmsnorm_gated(const void* o, const void* z, const void* weight, int in_f64,

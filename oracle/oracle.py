@@ -16,6 +16,8 @@ Each function cites the passage it follows (page title and section):
   (Linear -> CausalConv1D -> SiLU -> q, k, v).
 * ``conv_step`` / ``conv_prefill`` -- that conv alone, for one token or a whole
   prefill ("gated-deltanet-qwen3.5" section 因果卷积: kernel 4, depthwise, causal).
+* ``kda_fwd``      -- "Gated DeltaNet-2" (zhichai), section 标量绑定的数学表达 (the
+  KDA update with its erase projection written out) and 退化兼容性.
 * ``rmsnorm_gated`` -- "gated-deltanet-qwen3.5" section 输出门控与 RMSNorm
   (RMSNormGated(core_attn_out, z): the norm, then the SwiGLU-like z gate).
 * ``gdn2_fwd``     -- "Gated DeltaNet-2" (zhichai), section 新更新公式.
@@ -67,8 +69,9 @@ def _load():
             lib.oracle_conv_step.argtypes = [vp, vp, ip, ip, ip, vp, vp]
             lib.oracle_conv_prefill.argtypes = [vp, vp, ip, ip, ip, ip, vp, vp]
             lib.oracle_rmsnorm_gated.argtypes = [vp, vp, vp, ip, ip, ip, dp, vp]
+            lib.oracle_kda_fwd.argtypes = [vp] * 8 + [ip] * 6 + [dp, ip, vp, vp, ip]
             for f in (lib.oracle_gdn_fwd, lib.oracle_gate_prep, lib.oracle_conv_step,
-                      lib.oracle_conv_prefill, lib.oracle_rmsnorm_gated,
+                      lib.oracle_conv_prefill, lib.oracle_rmsnorm_gated, lib.oracle_kda_fwd,
                       lib.oracle_gdn_decode_step, lib.oracle_gdn2_fwd):
                 f.restype = ctypes.c_int
             lib.oracle_max_threads.restype = ctypes.c_int
@@ -201,6 +204,28 @@ def conv_prefill(x, conv_w, conv_state):
                                      _ptr(y))
     _check(rc, "oracle_conv_prefill")
     return y
+
+
+def kda_fwd(q, k, v, a, b, A_log, dt_bias, h0=None, *, scale=None, l2norm=True,
+            threads=None):
+    """Token-by-token KDA forward, the literal matrix form of its update.
+
+    q, k: [B,T,H,dk]; v: [B,T,H,dv]; a: [B,T,H,dk] (per-channel decay input);
+    b: [B,T,H] (beta logit); A_log, dt_bias: [H,dk]; h0: [B,H,dk,dv] or None.
+    Returns (o [B,T,H,dv], ht [B,H,dk,dv]) float64.
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    f64 = _is_f64(q, k, v, a, b, A_log, dt_bias, h0)
+    arrs = [_arr(x, f64) for x in (q, k, v, a, b, A_log, dt_bias, h0)]
+    scale = dk ** -0.5 if scale is None else scale
+    o = np.zeros((B * H, T, dv))
+    ht = np.zeros((B * H, dk, dv))
+    rc = _load().oracle_kda_fwd(*[_ptr(x) for x in arrs], int(f64), B, T, H, dk, dv,
+                                float(scale), int(l2norm), _ptr(o), _ptr(ht),
+                                int(threads or max_threads()))
+    _check(rc, "oracle_kda_fwd")
+    return o.reshape(B, H, T, dv).transpose(0, 2, 1, 3).copy(), ht.reshape(B, H, dk, dv)
 
 
 def rmsnorm_gated(o, z, weight, *, eps=1e-6):

@@ -53,6 +53,11 @@ MUTANTS = [
     ("conv_prefill_time_major",  # x read as [T, B, Cc]
      "      conv_silu_step(x, ((size_t)b * T + t) * Cc, conv_w, in_f64, Cc,",
      "      conv_silu_step(x, ((size_t)t * B + b) * Cc, conv_w, in_f64, Cc,"),
+    ("kda_decay_dropped",  # the projection applied to S instead of D S
+     "        for (int j = 0; j < dv; ++j) DS[(size_t)i * dv + j] = dec[i] * S[(size_t)i * dv + j];",
+     "        for (int j = 0; j < dv; ++j) DS[(size_t)i * dv + j] = S[(size_t)i * dv + j];"),
+    ("kda_write_unscaled", "          double acc = beta * kt[i] * vt[j];",
+     "          double acc = kt[i] * vt[j];"),
     ("rmsnorm_mean_as_sum",  # the sum of squares not divided by d_v
      "    const double inv = 1.0 / sqrt(ss / dv + eps);",
      "    const double inv = 1.0 / sqrt(ss + eps);"),
@@ -92,7 +97,8 @@ def _run_pins_against(lib_path):
     real = O._load()
     mutant = ctypes.CDLL(lib_path)
     for fname in ("oracle_gdn_fwd", "oracle_gate_prep", "oracle_conv_step",
-                  "oracle_conv_prefill", "oracle_rmsnorm_gated", "oracle_gdn_decode_step",
+                  "oracle_conv_prefill", "oracle_rmsnorm_gated", "oracle_kda_fwd",
+                  "oracle_gdn_decode_step",
                   "oracle_gdn2_fwd"):
         getattr(mutant, fname).argtypes = getattr(real, fname).argtypes
         getattr(mutant, fname).restype = ctypes.c_int

@@ -202,6 +202,40 @@ def test_gdn2_reduces_to_gdn():
     np.testing.assert_allclose(ht2, ht1, rtol=1e-12, atol=1e-13)
 
 
+def test_kda_is_gdn2_with_tied_gates():
+    """KDA's update S_t = (I - beta_t k k^T) D_t S + beta_t k v^T, computed with the
+    explicit erase projection, equals Gated DeltaNet-2 (read / correct form) with
+    b_t = beta_t 1 and w_t = beta_t 1 ("Gated DeltaNet-2", 退化兼容性), per-channel
+    decay kept."""
+    B, T, H, dk, dv = 2, 9, 2, 6, 5
+    q, k, v = _rand(B, T, H, dk), _rand(B, T, H, dk), _rand(B, T, H, dv)
+    a, b = _rand(B, T, H, dk), _rand(B, T, H)
+    A_log = rng.uniform(0, math.log(16), size=(H, dk))
+    dt_bias = rng.uniform(-4, -1, size=(H, dk))
+    h0 = 0.02 * _rand(B, H, dk, dv)
+    o1, ht1 = O.kda_fwd(q, k, v, a, b, A_log, dt_bias, h0)
+    o2, ht2 = O.gdn2_fwd(q, k, v, a, np.repeat(b[..., None], dk, -1),
+                         np.repeat(b[..., None], dv, -1), A_log, dt_bias, h0)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(ht1, ht2, rtol=1e-12, atol=1e-13)
+
+
+def test_kda_with_scalar_decay_is_gdn():
+    """With every channel of the decay equal (a, A_log, dt_bias constant over d_k),
+    KDA is Gated DeltaNet ("Gated DeltaNet-2", 退化兼容性, second case)."""
+    B, T, H, d = 1, 12, 3, 7
+    q, k, v = _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d)
+    a, b = _rand(B, T, H), _rand(B, T, H)
+    A_log = rng.uniform(0, math.log(16), size=H)
+    dt_bias = rng.uniform(-4, -1, size=H)
+    h0 = 0.02 * _rand(B, H, d, d)
+    rep = lambda x: np.repeat(x[..., None], d, axis=-1)
+    o1, ht1 = O.kda_fwd(q, k, v, rep(a), b, rep(A_log), rep(dt_bias), h0)
+    o2, ht2 = O.gdn_fwd(q, k, v, a, b, A_log, dt_bias, h0)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(ht1, ht2, rtol=1e-12, atol=1e-13)
+
+
 # --------------------------------------------------------------------------
 # Gates and normalisation: closed forms
 # --------------------------------------------------------------------------
