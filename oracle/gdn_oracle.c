@@ -22,7 +22,10 @@
  *  - "gated-deltanet-qwen3.5" (wanger-sjtu), architecture diagram: decode reads
  *    and updates conv_states and recurrent_states.
  *  - "Gated DeltaNet-2" (zhichai), section "新更新公式": S_bar = D S,
- *    r = S_bar^T e, S = S_bar + k (z - r)^T with e = b (.) k, z = w (.) v.
+ *    r = S_bar^T e, S = S_bar + k (z - r)^T with e = b (.) k, z = w (.) v;
+ *    section "标量绑定的数学表达": the KDA update (I - beta k k^T) D S + beta k v^T.
+ *  - "gated-deltanet-qwen3.5" (wanger-sjtu), section "输出门控与 RMSNorm":
+ *    RMSNormGated(core_attn_out, z).
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *  - L2 normalisation of q and k is x / sqrt(sum x^2 + 1e-6); q is then scaled
@@ -41,8 +44,10 @@
  *
  * Parity: pinned (see tests/test_oracle_pins.py): linear-attention brute force,
  * delta-rule overwrite on orthonormal keys, per-step overwrite identity, pure
- * decay closed form, matrix-form recurrence, GDN-2 -> GDN reduction, gate and
- * norm closed forms, conv against a library convolution.
+ * decay closed form, matrix-form recurrence, GDN-2 -> GDN reduction, KDA ->
+ * GDN-2 (tied gates) and -> GDN (scalar decay), gate and norm closed forms, the
+ * conv step and the prefill conv against a library convolution, the gated
+ * RMSNorm against a library rms_norm and its closed forms.
  */
 #include <math.h>
 #include <stddef.h>
