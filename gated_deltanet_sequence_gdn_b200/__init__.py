@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(_PKG, "libgdn.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m gated_deltanet_sequence_gdn_b200.build`"
+        f"{LIB_PATH} is missing: build it with `python gated_deltanet_sequence_gdn_b200/build.py`"
         " (nvcc, sm_100a). There is no fallback implementation.")
 
 lib = ctypes.CDLL(LIB_PATH)

@@ -1,6 +1,8 @@
 """Builds libgdn.so (all CUDA sources of the package, sm_100a) in the package dir.
 
-    python -m gated_deltanet_sequence_gdn_b200.build [--force] [--verbose]
+    python gated_deltanet_sequence_gdn_b200/build.py [--force] [--verbose]
+
+(run by path: importing the package needs the library this script builds)
 """
 from __future__ import annotations
 
