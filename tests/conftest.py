@@ -6,6 +6,20 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def pytest_sessionstart(session):
+    """A fresh checkout has no libgdn.so yet: build it (the tests load it through the
+    package, which refuses to import without it)."""
+    lib = os.path.join(ROOT, "gated_deltanet_sequence_gdn_b200", "libgdn.so")
+    if os.path.exists(lib):
+        return
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "gdn_b200_build", os.path.join(ROOT, "gated_deltanet_sequence_gdn_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size parity case (minutes)")
