@@ -237,6 +237,11 @@ def run_ours(args, rank, local_rank, world):
         extra["conv_prefill_8k"] = measure_conv(G, dev, stream, pk, args)
         extra["prefill_128k"] = measure_prefill(G, "prefill_128k", dev, stream, pk, args)
         extra["prefill_b8_16k"] = measure_prefill(G, "prefill_b8_16k", dev, stream, pk, args)
+        try:  # the newest secondary figure, last: its failure is reported here, not raised
+            extra["rmsnorm_gated_8k"] = measure_norm(G, dev, stream, pk, args)
+            torch.cuda.synchronize()
+        except Exception as e:  # noqa: BLE001
+            extra["rmsnorm_gated_8k"] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     launches = 2 * args.steps  # wy_prep_tc_kernel + state_scan_tc_kernel per step
     line = {
@@ -399,6 +404,32 @@ def measure_conv(G, dev, stream, pk, args):
             "steps": steps}
 
 
+def measure_norm(G, dev, stream, pk, args):
+    """gdn_rmsnorm_gated over the prefill_8k layer's core output (8192 tokens x 64
+    value heads x 128): HBM-bound, reported against the measured copy bandwidth.
+    Algorithmic bytes per launch: o and z read once, y written once, the weight."""
+    w = WORKLOADS["rmsnorm_gated_8k"]
+    x = workload_inputs(w, dev)
+    y = torch.empty_like(x["o"])
+
+    def step():
+        G.gdn_rmsnorm_gated(x["o"], x["z"], x["weight"], y=y, stream=stream)
+
+    steps = 20
+    total, per = time_steps(step, steps, 3, stream)
+    ms = sum(per) / len(per)
+    nbytes = 3 * x["o"].numel() * x["o"].element_size() + w.d * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del x, y
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_launch": round(ms, 5),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": kernel_traffic("rmsnorm_gated_8k")},
+            "steps": steps}
+
+
 def run_only(args, local_rank):
     import gated_deltanet_sequence_gdn_b200 as G
     torch.cuda.set_device(local_rank)
@@ -411,6 +442,8 @@ def run_only(args, local_rank):
         r = measure_gdn2(G, dev, stream, pk, args)
     elif args.only == "conv_prefill_8k":
         r = measure_conv(G, dev, stream, pk, args)
+    elif args.only == "rmsnorm_gated_8k":
+        r = measure_norm(G, dev, stream, pk, args)
     else:
         r = measure_prefill(G, args.only, dev, stream, pk, args)
     G.gdn_check_status(stream)
@@ -487,7 +520,8 @@ def main():
                     help="skip the decode / GDN-2 / long-prefill extras")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["prefill_8k", "decode_256", "gdn2_b4_4k", "prefill_128k",
-                                       "prefill_b8_16k", "conv_prefill_8k"], default=None,
+                                       "prefill_b8_16k", "conv_prefill_8k", "rmsnorm_gated_8k"],
+                    default=None,
                     help="measure one secondary workload alone (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -18,7 +18,7 @@ import os
 import torch
 
 __all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_chunk_workspace_bytes", "gdn_recurrent_step",
-           "gdn_conv_prefill",
+           "gdn_conv_prefill", "gdn_rmsnorm_gated",
            "gdn2_chunk_fwd", "gdn2_chunk_workspace_bytes", "gdn_chunk_fwd_noalloc",
            "gdn_check_status", "GDNError", "LIB_PATH", "lib", "F32", "BF16",
            "QK_L2NORM", "GATES_PRECOMPUTED", "OUT_F32"]
@@ -50,6 +50,7 @@ lib.gdn_chunk_fwd_host_workspace_bytes.argtypes = [_i] * 9
 lib.gdn_chunk_fwd_host_workspace_bytes.restype = _sz
 lib.gdn_recurrent_step.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _vp]
 lib.gdn_conv_prefill.argtypes = [_vp] * 6 + [_i] * 7 + [_vp]
+lib.gdn_rmsnorm_gated.argtypes = [_vp] * 4 + [ctypes.c_long, _i, _i, _f, _vp]
 lib.gdn_chunk_workspace_bytes.argtypes = [_i] * 7
 lib.gdn2_chunk_workspace_bytes.argtypes = [_i] * 6
 lib.gdn_chunk_workspace_bytes.restype = _sz
@@ -60,7 +61,8 @@ lib.gdn_status_string.restype = ctypes.c_char_p
 lib.gdn_version.argtypes = []
 for _fn in (lib.gdn_gate_prep, lib.gdn_chunk_fwd, lib.gdn_chunk_fwd_noalloc, lib.gdn_chunk_fwd_host,
             lib.gdn2_chunk_fwd,
-            lib.gdn_recurrent_step, lib.gdn_conv_prefill, lib.gdn_check_status, lib.gdn_version):
+            lib.gdn_recurrent_step, lib.gdn_conv_prefill, lib.gdn_rmsnorm_gated,
+            lib.gdn_check_status, lib.gdn_version):
     _fn.restype = _i
 
 
@@ -355,6 +357,23 @@ def gdn_conv_prefill(x, conv_w, conv_state, *, Hk, Hv, dk, dv, q=None, k=None, v
                                 Hk, Hv, dk, dv, _dtype_code(dt), _stream(stream)),
            "gdn_conv_prefill")
     return q, k, v
+
+
+def gdn_rmsnorm_gated(o, z, weight, *, eps=1e-6, y=None, stream=None):
+    """Gated RMSNorm of the core output over its last axis (d_v):
+    y = o / sqrt(mean(o^2) + eps) * weight * SiLU(z).  o, z [..., dv] (same shape
+    and dtype); weight [dv] float32.  y may be o or z (in place)."""
+    dt = o.dtype
+    dv = o.shape[-1]
+    _need(z, dt, tuple(o.shape), "z")
+    _need(weight, torch.float32, (dv,), "weight")
+    y = torch.empty_like(o) if y is None else y
+    _need(y, dt, tuple(o.shape), "y")
+    rows = o.numel() // dv if dv else 0
+    _check(lib.gdn_rmsnorm_gated(_p(o), _p(z), _p(weight), _p(y), rows, dv, _dtype_code(dt),
+                                 float(eps), _stream(stream)),
+           "gdn_rmsnorm_gated")
+    return y
 
 
 def gdn_check_status(stream=None):

@@ -186,6 +186,16 @@ int gdn_conv_prefill(const void* x_qkv, const float* conv_w, void* conv_state, v
                                        dtype, (cudaStream_t)stream));
 }
 
+int gdn_rmsnorm_gated(const void* o, const void* z, const float* weight, void* y, long rows,
+                      int dv, int dtype, float eps, gdn_stream_t stream) {
+  if (rows < 0 || !ok_dtype(dtype) || !(eps >= 0.f) || eps > 1.f) return GDN_ERR_INVALID_ARG;
+  if (!ok_head_dim(dv)) return GDN_ERR_UNSUPPORTED;
+  if (rows == 0) return GDN_OK;
+  if (!ok_ptr(o) || !ok_ptr(z) || !ok_ptr(y) || !ok_elem(weight, 4)) return GDN_ERR_INVALID_ARG;
+  return from_cuda(launch_rmsnorm_gated(o, z, weight, y, rows, dv, dtype, eps,
+                                        (cudaStream_t)stream));
+}
+
 int gdn_check_status(gdn_stream_t stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDN_ERR_CUDA;
   int h = 0;

@@ -32,6 +32,9 @@ cudaError_t launch_conv_prefill(const void* x, const float* conv_w, void* conv_s
                                 void* k, void* v, int B, int T, int Hk, int Hv, int dk, int dv,
                                 int dtype, cudaStream_t s);
 
+cudaError_t launch_rmsnorm_gated(const void* o, const void* z, const float* weight, void* y,
+                                 long rows, int dv, int dtype, float eps, cudaStream_t s);
+
 // float32 CUDA-core chunk path (GDN and, with gdn2 = true, Gated DeltaNet-2).
 cudaError_t launch_chunk_simt(const ChunkArgs& a, bool gdn2, cudaStream_t s);
 

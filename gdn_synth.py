@@ -24,7 +24,7 @@ LN16 = math.log(16.0)
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str            # "gdn" | "decode" | "gdn2" | "conv"
+    kind: str            # "gdn" | "decode" | "gdn2" | "conv" | "norm"
     B: int
     T: int
     Hk: int
@@ -51,6 +51,9 @@ WORKLOADS = {
     # the prefill conv1d + SiLU over the mixed stream of the prefill_8k layer
     "conv_prefill_8k": Workload("conv_prefill_8k", "conv", 1, 8192, 16, 64, 128, torch.bfloat16,
                                 1005),
+    # the gated RMSNorm of the prefill_8k layer's core output
+    "rmsnorm_gated_8k": Workload("rmsnorm_gated_8k", "norm", 1, 8192, 16, 64, 128,
+                                 torch.bfloat16, 1006),
 }
 
 
@@ -150,6 +153,17 @@ def conv_prefill_inputs(B, T, Hk, Hv, d, dtype, seed, device="cpu", dv=None):
     }
 
 
+def rmsnorm_inputs(B, T, Hv, dv, dtype, seed, device="cpu"):
+    """Inputs of one gated RMSNorm call: the core output o and the gate z
+    [B,T,Hv,dv] ~ N(0,1) in ``dtype``; weight [dv] ~ U(0.5, 1.5) fp32."""
+    g = _gen(seed, device)
+    return {
+        "o": _randn((B, T, Hv, dv), g, device, dtype),
+        "z": _randn((B, T, Hv, dv), g, device, dtype),
+        "weight": _uniform((dv,), 0.5, 1.5, g, device),
+    }
+
+
 def workload_inputs(w: Workload, device="cpu"):
     if w.kind == "gdn":
         return gdn_inputs(w.B, w.T, w.Hk, w.Hv, w.d, w.dtype, w.seed, device, h0=w.h0)
@@ -159,4 +173,6 @@ def workload_inputs(w: Workload, device="cpu"):
         return decode_inputs(w.B, w.steps, w.Hk, w.Hv, w.d, w.dtype, w.seed, device)
     if w.kind == "conv":
         return conv_prefill_inputs(w.B, w.T, w.Hk, w.Hv, w.d, w.dtype, w.seed, device)
+    if w.kind == "norm":
+        return rmsnorm_inputs(w.B, w.T, w.Hv, w.d, w.dtype, w.seed, device)
     raise ValueError(w.kind)

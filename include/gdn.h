@@ -247,6 +247,27 @@ int gdn_conv_prefill(const void* x_qkv, const float* conv_w, void* conv_state,
                      int dk, int dv, int dtype, gdn_stream_t stream);
 
 /*
+ * gdn_rmsnorm_gated -- the gated RMSNorm of the core output
+ * ("gated-deltanet-qwen3.5" section 输出门控与 RMSNorm: RMSNormGated(core_attn_out,
+ * z), an RMSNorm and then the SwiGLU-like z gate), per row of d_v channels:
+ *   y = o / sqrt(mean(o^2) + eps) * weight * SiLU(z)
+ *   o, z   [rows, dv] dtype: rows = B*T*Hv for the chunk path's o (layout
+ *          [B,T,Hv,dv]) or N*Hv for the decode step's o; z the matching slice of
+ *          the z projection
+ *   weight [dv] float32, shared by every row (and head)
+ *   y      [rows, dv] dtype, written; may be o or z (in place)
+ *   eps    added to mean(o^2) inside the root, 0 <= eps <= 1 (1e-6 by default in
+ *          the binding)
+ *   Ownership: device pointers owned by the caller; o, z, y 16-byte aligned,
+ *   weight float aligned.  Arithmetic in float32, y rounded to dtype once.
+ *   rows = 0 enqueues nothing.  Returns GDN_ERR_INVALID_ARG (null or misaligned
+ *   pointer, negative rows, bad dtype or eps), GDN_ERR_UNSUPPORTED (dv not 64 /
+ *   128), GDN_ERR_CUDA (launch failure).
+ */
+int gdn_rmsnorm_gated(const void* o, const void* z, const float* weight, void* y,
+                      long rows, int dv, int dtype, float eps, gdn_stream_t stream);
+
+/*
  * gdn2_chunk_fwd -- chunkwise Gated DeltaNet-2 forward ("Gated DeltaNet-2",
  * 新更新公式 and 高效训练): channel-wise decay
  * D_t = diag(exp(-exp(A_log) (.) softplus(a_t + dt_bias))), erase gate

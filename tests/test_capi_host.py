@@ -142,6 +142,20 @@ def test_conv_prefill_rejects_bad_arguments():
     assert cp(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 2, 4, 128, 128, 1, None) == 0
 
 
+def test_rmsnorm_gated_rejects_bad_arguments():
+    rn = G.lib.gdn_rmsnorm_gated
+    # (o, z, weight, y, rows, dv, dtype, eps, stream)
+    assert rn(None, FAKE, FAKE, FAKE, 8, 128, 1, 1e-6, None) == -1
+    assert rn(FAKE, FAKE, None, FAKE, 8, 128, 1, 1e-6, None) == -1
+    assert rn(FAKE, FAKE, FAKE, FAKE + 8, 8, 128, 1, 1e-6, None) == -1
+    assert rn(FAKE, FAKE, FAKE, FAKE, -1, 128, 1, 1e-6, None) == -1
+    assert rn(FAKE, FAKE, FAKE, FAKE, 8, 128, 5, 1e-6, None) == -1
+    assert rn(FAKE, FAKE, FAKE, FAKE, 8, 128, 1, -1.0, None) == -1
+    assert rn(FAKE, FAKE, FAKE, FAKE, 8, 128, 1, float("nan"), None) == -1
+    assert rn(FAKE, FAKE, FAKE, FAKE, 8, 96, 1, 1e-6, None) == -2
+    assert rn(FAKE, FAKE, FAKE, FAKE, 0, 128, 1, 1e-6, None) == 0
+
+
 def test_empty_calls_are_no_ops():
     # zero tokens / zero sequences return before any launch (no state pointers)
     assert _chunk(T=0) == 0
