@@ -112,6 +112,9 @@ static int validate_chunk(const ChunkArgs& c, bool gdn2) {
       !ok_elem(c.b, ges) || !ok_ptr(c.o))
     return GDN_ERR_INVALID_ARG;
   if (gdn2 && !ok_elem(c.w, ges)) return GDN_ERR_INVALID_ARG;
+  // the GDN-2 tensor-core prep copies its gate tiles in 16-byte pieces
+  if (gdn2 && chunk_mma_supported(c) && (!aligned16(c.a) || !aligned16(c.b) || !aligned16(c.w)))
+    return GDN_ERR_INVALID_ARG;
   if (!(c.flags & GDN_GATES_PRECOMPUTED) && (!ok_elem(c.A_log, 4) || !ok_elem(c.dt_bias, 4)))
     return GDN_ERR_INVALID_ARG;
   return GDN_OK;

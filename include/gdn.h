@@ -20,9 +20,11 @@
  *    dt_bias and conv weights are always float32; arithmetic is float32 with
  *    float32 accumulation.
  *  - Tensors moved in 16-byte pieces must be 16-byte aligned: q, k, v, o and
- *    q_out/k_out of the chunk and gate-prep calls, h0, ht, the decode state and
- *    conv_w.  The other pointers (gates a, b, w, A_log, dt_bias, g/beta outputs,
- *    the decode x, o and conv_state) need only their element alignment.  Head
+ *    q_out/k_out of the chunk and gate-prep calls, h0, ht, the decode state,
+ *    conv_w, and the per-channel gates a, b_logit, w_logit of gdn2_chunk_fwd on
+ *    its bf16 d = 128 path.  The other pointers (the GDN gates a, b, A_log,
+ *    dt_bias, g/beta outputs, the decode x, o and conv_state) need only their
+ *    element alignment.  Head
  *    dims dk, dv must be 64 or 128 (heads are tiled in 64-column blocks); Hv
  *    must be a multiple of Hk.
  *  - Return value: GDN_OK or a negative gdn_status.  Argument errors are

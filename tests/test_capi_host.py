@@ -111,6 +111,12 @@ def test_gdn2_and_decode_reject_bad_arguments():
                             128, 128, 1, 0.1, 1, FAKE, None, None, 0, None) == -1
     assert L.gdn2_chunk_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 64, 2,
                             100, 128, 1, 0.1, 1, FAKE, None, None, 0, None) == -2
+    # bf16, d = 128 (the tensor-core path) copies the gate tiles in 16-byte pieces:
+    # element-aligned but not 16-byte-aligned gates are refused there, not on the
+    # float32 path
+    for bad in ((FAKE + 2, FAKE, FAKE), (FAKE, FAKE + 2, FAKE), (FAKE, FAKE, FAKE + 2)):
+        assert L.gdn2_chunk_fwd(FAKE, FAKE, FAKE, *bad, FAKE, FAKE, None, 1, 64, 2, 128, 128, 1,
+                                0.1, 1, FAKE, None, FAKE, 1 << 30, None) == -1
     # decode: conv weights given but no conv state
     assert L.gdn_recurrent_step(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 4,
                                 128, 128, 1, 0.1, 0, None) == -1
