@@ -33,7 +33,7 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 import torch.distributed as dist  # noqa: E402
 
-from gdn_synth import WORKLOADS, workload_inputs  # noqa: E402
+from gdn_synth import WORKLOADS, kda_inputs, workload_inputs  # noqa: E402
 
 CHUNK_FLOP_PER_TOKEN_HEAD = 180_224  # dense GEMM FLOPs of the chunk form at C=64, d=128
 HEADLINE = "prefill_8k"
@@ -237,11 +237,13 @@ def run_ours(args, rank, local_rank, world):
         extra["conv_prefill_8k"] = measure_conv(G, dev, stream, pk, args)
         extra["prefill_128k"] = measure_prefill(G, "prefill_128k", dev, stream, pk, args)
         extra["prefill_b8_16k"] = measure_prefill(G, "prefill_b8_16k", dev, stream, pk, args)
-        try:  # the newest secondary figure, last: its failure is reported here, not raised
-            extra["rmsnorm_gated_8k"] = measure_norm(G, dev, stream, pk, args)
-            torch.cuda.synchronize()
-        except Exception as e:  # noqa: BLE001
-            extra["rmsnorm_gated_8k"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+        # the newest secondary figures, last: a failure is reported here, not raised
+        for name, fn in (("kda_b4_4k", measure_kda), ("rmsnorm_gated_8k", measure_norm)):
+            try:
+                extra[name] = fn(G, dev, stream, pk, args)
+                torch.cuda.synchronize()
+            except Exception as e:  # noqa: BLE001
+                extra[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     launches = 2 * args.steps  # wy_prep_tc_kernel + state_scan_tc_kernel per step
     line = {
@@ -404,6 +406,31 @@ def measure_conv(G, dev, stream, pk, args):
             "steps": steps}
 
 
+def measure_kda(G, dev, stream, pk, args):
+    """gdn_kda_chunk_fwd at the Gated DeltaNet-2 bench shape (B=4, T=4096, 16 heads,
+    d=128, bf16): the gate tiling plus the Gated DeltaNet-2 kernels."""
+    w = WORKLOADS["gdn2_b4_4k"]
+    x = kda_inputs(w.B, w.T, w.Hv, w.d, w.dtype, seed=1007, device=dev)
+    o = torch.empty((w.B, w.T, w.Hv, w.d), device=dev, dtype=w.dtype)
+    ht = torch.empty((w.B, w.Hv, w.d, w.d), device=dev, dtype=torch.float32)
+    n_ws = G.gdn_kda_chunk_workspace_bytes(w.B, w.T, w.Hv, w.d, w.d, w.dtype)
+    ws = torch.empty(n_ws, device=dev, dtype=torch.uint8)
+
+    def step():
+        G.gdn_kda_chunk_fwd(x["q"], x["k"], x["v"], x["a"], x["beta"], x["A_log"],
+                            x["dt_bias"], x["h0"], o=o, ht=ht, workspace=ws, stream=stream)
+
+    total, per = time_steps(step, 5, 2, stream)
+    ms = total / 5
+    flop = CHUNK_FLOP_PER_TOKEN_HEAD * w.T * w.Hv * w.B
+    ach = flop / (ms / 1e3) / 1e12
+    del x, o, ht, ws
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+            "achieved_tflops": round(ach, 2),
+            "frac_of_bf16_peak": round(ach / pk["bf16_tflops"], 4)}
+
+
 def measure_norm(G, dev, stream, pk, args):
     """gdn_rmsnorm_gated over the prefill_8k layer's core output (8192 tokens x 64
     value heads x 128): HBM-bound, reported against the measured copy bandwidth.
@@ -444,6 +471,8 @@ def run_only(args, local_rank):
         r = measure_conv(G, dev, stream, pk, args)
     elif args.only == "rmsnorm_gated_8k":
         r = measure_norm(G, dev, stream, pk, args)
+    elif args.only == "kda_b4_4k":
+        r = measure_kda(G, dev, stream, pk, args)
     else:
         r = measure_prefill(G, args.only, dev, stream, pk, args)
     G.gdn_check_status(stream)
@@ -520,7 +549,8 @@ def main():
                     help="skip the decode / GDN-2 / long-prefill extras")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["prefill_8k", "decode_256", "gdn2_b4_4k", "prefill_128k",
-                                       "prefill_b8_16k", "conv_prefill_8k", "rmsnorm_gated_8k"],
+                                       "prefill_b8_16k", "conv_prefill_8k", "rmsnorm_gated_8k",
+                                       "kda_b4_4k"],
                     default=None,
                     help="measure one secondary workload alone (profiling runs)")
     args = ap.parse_args()

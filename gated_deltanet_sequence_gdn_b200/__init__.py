@@ -18,7 +18,8 @@ import os
 import torch
 
 __all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_chunk_workspace_bytes", "gdn_recurrent_step",
-           "gdn_conv_prefill", "gdn_rmsnorm_gated",
+           "gdn_conv_prefill", "gdn_rmsnorm_gated", "gdn_kda_chunk_fwd",
+           "gdn_kda_chunk_workspace_bytes",
            "gdn2_chunk_fwd", "gdn2_chunk_workspace_bytes", "gdn_chunk_fwd_noalloc",
            "gdn_check_status", "GDNError", "LIB_PATH", "lib", "F32", "BF16",
            "QK_L2NORM", "GATES_PRECOMPUTED", "OUT_F32"]
@@ -51,6 +52,9 @@ lib.gdn_chunk_fwd_host_workspace_bytes.restype = _sz
 lib.gdn_recurrent_step.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _vp]
 lib.gdn_conv_prefill.argtypes = [_vp] * 6 + [_i] * 7 + [_vp]
 lib.gdn_rmsnorm_gated.argtypes = [_vp] * 4 + [ctypes.c_long, _i, _i, _f, _vp]
+lib.gdn_kda_chunk_fwd.argtypes = [_vp] * 8 + [_i] * 6 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
+lib.gdn_kda_chunk_workspace_bytes.argtypes = [_i] * 7
+lib.gdn_kda_chunk_workspace_bytes.restype = _sz
 lib.gdn_chunk_workspace_bytes.argtypes = [_i] * 7
 lib.gdn2_chunk_workspace_bytes.argtypes = [_i] * 6
 lib.gdn_chunk_workspace_bytes.restype = _sz
@@ -62,6 +66,7 @@ lib.gdn_version.argtypes = []
 for _fn in (lib.gdn_gate_prep, lib.gdn_chunk_fwd, lib.gdn_chunk_fwd_noalloc, lib.gdn_chunk_fwd_host,
             lib.gdn2_chunk_fwd,
             lib.gdn_recurrent_step, lib.gdn_conv_prefill, lib.gdn_rmsnorm_gated,
+            lib.gdn_kda_chunk_fwd,
             lib.gdn_check_status, lib.gdn_version):
     _fn.restype = _i
 
@@ -306,6 +311,48 @@ def gdn2_chunk_fwd(q, k, v, a, b_logit, w_logit, A_log=None, dt_bias=None, h0=No
                               float(scale), flags, _p(o), _p(ht), _p(workspace), ws_bytes,
                               _stream(stream)),
            "gdn2_chunk_fwd")
+    return o, ht
+
+
+def gdn_kda_chunk_workspace_bytes(B, T, H, dk, dv, dtype, gates_precomputed=False) -> int:
+    """Bytes of device workspace gdn_kda_chunk_fwd needs (the tiled gates included)."""
+    return int(lib.gdn_kda_chunk_workspace_bytes(B, T, H, dk, dv, _dtype_code(dtype),
+                                                 GATES_PRECOMPUTED if gates_precomputed else 0))
+
+
+def gdn_kda_chunk_fwd(q, k, v, a, beta, A_log=None, dt_bias=None, h0=None, *, scale=None,
+                      l2norm=True, gates_precomputed=False, out_f32=False, o=None, ht=None,
+                      want_ht=True, workspace=None, stream=None):
+    """Chunkwise KDA forward: Gated DeltaNet-2 with one beta per (token, head) for
+    the erase and the write.  q, k, a [B,T,H,dk]; v [B,T,H,dv]; beta [B,T,H] (the
+    logit, or beta in float32 with gates_precomputed, a then the per-channel
+    log-decay); A_log, dt_bias [H,dk] float32; h0 [B,H,dk,dv] or None."""
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    dt = q.dtype
+    scale = dk ** -0.5 if scale is None else scale
+    gdt = torch.float32 if gates_precomputed else dt
+    _need(k, dt, q.shape, "k")
+    _need(v, dt, (B, T, H, dv), "v")
+    _need(a, gdt, (B, T, H, dk), "a")
+    _need(beta, gdt, (B, T, H), "beta")
+    if h0 is not None:
+        _need(h0, torch.float32, (B, H, dk, dv), "h0")
+    odt = torch.float32 if out_f32 else dt
+    o = torch.empty((B, T, H, dv), device=q.device, dtype=odt) if o is None else o
+    _need(o, odt, (B, T, H, dv), "o")
+    if ht is None and want_ht:
+        ht = torch.empty((B, H, dk, dv), device=q.device, dtype=torch.float32)
+    flags = ((QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
+             | (OUT_F32 if out_f32 else 0))
+    ws_need = gdn_kda_chunk_workspace_bytes(B, T, H, dk, dv, dt, gates_precomputed)
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.gdn_kda_chunk_fwd(_p(q), _p(k), _p(v), _p(a), _p(beta), _p(A_log), _p(dt_bias),
+                                 _p(h0), B, T, H, dk, dv, _dtype_code(dt), float(scale), flags,
+                                 _p(o), _p(ht), _p(workspace), ws_bytes, _stream(stream)),
+           "gdn_kda_chunk_fwd")
     return o, ht
 
 

@@ -156,6 +156,55 @@ int gdn2_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
   return run_chunk(c, true, workspace, ws_bytes, (cudaStream_t)stream);
 }
 
+// KDA workspace: gdn2_chunk_fwd's, then the tiled erase gates [B*T*H][dk] and
+// the tiled write gates [B*T*H][dv], each rounded up to 256 bytes.
+static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+static bool kda_layout(int B, int T, int H, int dk, int dv, int dtype, int flags, size_t* ws2,
+                       size_t* tb, size_t* tw) {
+  if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0 || !ok_dtype(dtype)) return false;
+  const size_t ges = (flags & GDN_GATES_PRECOMPUTED) ? 4 : elem_size(dtype);
+  const size_t rows = (size_t)B * T * H;
+  *ws2 = up256(gdn2_chunk_workspace_bytes(B, T, H, dk, dv, dtype));
+  *tb = up256(rows * dk * ges);
+  *tw = up256(rows * dv * ges);
+  return true;
+}
+
+size_t gdn_kda_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype, int flags) {
+  size_t ws2, tb, tw;
+  if (!kda_layout(B, T, H, dk, dv, dtype, flags, &ws2, &tb, &tw)) return 0;
+  return ws2 + tb + tw;
+}
+
+int gdn_kda_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
+                      const void* beta, const float* A_log, const float* dt_bias,
+                      const float* h0, int B, int T, int H, int dk, int dv, int dtype,
+                      float scale, int flags, void* o, float* ht, void* workspace,
+                      size_t ws_bytes, gdn_stream_t stream) {
+  size_t ws2, tb, tw;
+  if (!kda_layout(B, T, H, dk, dv, dtype, flags, &ws2, &tb, &tw)) return GDN_ERR_INVALID_ARG;
+  uint8_t* W = static_cast<uint8_t*>(workspace);
+  const bool any = (long)B * T > 0;
+  // the gate tiles live in the workspace; the Gated DeltaNet-2 checks run on them
+  ChunkArgs c{q, k, v, a, any ? W + ws2 : nullptr, any ? W + ws2 + tb : nullptr, A_log, dt_bias,
+              h0, B, T, H, H, dk, dv, dtype, scale, flags, o, ht};
+  if (any) {
+    const size_t ges = (flags & GDN_GATES_PRECOMPUTED) ? 4 : elem_size(dtype);
+    if (!ok_elem(beta, ges)) return GDN_ERR_INVALID_ARG;
+    if (W == nullptr || !aligned16(W) || ws_bytes < ws2 + tb + tw) return GDN_ERR_WORKSPACE;
+  }
+  int st = validate_chunk(c, true);
+  if (st != GDN_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (any) {
+    const size_t ges = (flags & GDN_GATES_PRECOMPUTED) ? 4 : elem_size(dtype);
+    st = from_cuda(launch_tie_gates(beta, W + ws2, W + ws2 + tb, (size_t)B * T * H, dk, dv,
+                                    (int)ges, s));
+    if (st != GDN_OK) return st;
+  }
+  return run_chunk(c, true, any ? W : nullptr, ws2, s);
+}
+
 int gdn_recurrent_step(const void* x_qkv, const float* conv_w, void* conv_state, const void* a,
                        const void* b, const float* A_log, const float* dt_bias, float* state,
                        void* o, int N, int Hk, int Hv, int dk, int dv, int dtype, float scale,

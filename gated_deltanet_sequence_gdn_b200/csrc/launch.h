@@ -32,6 +32,11 @@ cudaError_t launch_conv_prefill(const void* x, const float* conv_w, void* conv_s
                                 void* k, void* v, int B, int T, int Hk, int Hv, int dk, int dv,
                                 int dtype, cudaStream_t s);
 
+// KDA on the Gated DeltaNet-2 path: beta [rows] tiled into b [rows][dk] and
+// w [rows][dv] (elements of elem_bytes bytes, copied bit for bit).
+cudaError_t launch_tie_gates(const void* beta, void* b, void* w, size_t rows, int dk, int dv,
+                             int elem_bytes, cudaStream_t s);
+
 cudaError_t launch_rmsnorm_gated(const void* o, const void* z, const float* weight, void* y,
                                  long rows, int dv, int dtype, float eps, cudaStream_t s);
 

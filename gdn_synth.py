@@ -153,6 +153,25 @@ def conv_prefill_inputs(B, T, Hk, Hv, d, dtype, seed, device="cpu", dv=None):
     }
 
 
+def kda_inputs(B, T, H, d, dtype, seed, device="cpu", h0=True, dv=None):
+    """Inputs of one KDA call: q, k [B,T,H,d]; v [B,T,H,dv]; a [B,T,H,d] (per-channel
+    decay input) and beta [B,T,H] (logit) in ``dtype``; A_log, dt_bias [H,d] fp32 as
+    for Gated DeltaNet-2; h0 [B,H,d,dv] fp32 (or None)."""
+    dv = d if dv is None else dv
+    g = _gen(seed, device)
+    out = {
+        "q": _randn((B, T, H, d), g, device, dtype),
+        "k": _randn((B, T, H, d), g, device, dtype),
+        "v": _randn((B, T, H, dv), g, device, dtype),
+        "a": _randn((B, T, H, d), g, device, dtype),
+        "beta": _randn((B, T, H), g, device, dtype),
+        "A_log": _uniform((H, d), 0.0, LN16, g, device),
+        "dt_bias": _uniform((H, d), -4.0, -1.0, g, device),
+    }
+    out["h0"] = _randn((B, H, d, dv), g, device, torch.float32, std=0.02) if h0 else None
+    return out
+
+
 def rmsnorm_inputs(B, T, Hv, dv, dtype, seed, device="cpu"):
     """Inputs of one gated RMSNorm call: the core output o and the gate z
     [B,T,Hv,dv] ~ N(0,1) in ``dtype``; weight [dv] ~ U(0.5, 1.5) fp32."""

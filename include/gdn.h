@@ -249,6 +249,33 @@ int gdn_conv_prefill(const void* x_qkv, const float* conv_w, void* conv_state,
                      int dk, int dv, int dtype, gdn_stream_t stream);
 
 /*
+ * gdn_kda_chunk_fwd -- KDA (Kimi Delta Attention): the channel-wise decay of
+ * Gated DeltaNet-2 with one scalar beta per (token, head) for both the erase
+ * and the write, S_t = (I - beta_t k_t k_t^T) D_t S_{t-1} + beta_t k_t v_t^T,
+ * o_t = S_t^T q_t ("Gated DeltaNet-2", sections 标量绑定的数学表达 and
+ * 退化兼容性: Gated DeltaNet-2 with b_t = beta_t 1 and w_t = beta_t 1).  It tiles
+ * beta into per-channel gate tiles in the workspace and runs gdn2_chunk_fwd's
+ * kernels on them, so the result is bit for bit that call's on tiled gates.
+ *   q, k, a [B,T,H,dk]; v [B,T,H,dv]; A_log, dt_bias [H,dk]; h0 / ht / o /
+ *   scale / flags as for gdn2_chunk_fwd.
+ *   beta [B,T,H]: the beta logit in dtype, or beta itself in float32 with
+ *     GDN_GATES_PRECOMPUTED (a then holds the per-channel log-decay in float32).
+ *   workspace / ws_bytes: device scratch owned by the caller, 16-byte aligned, at
+ *     least gdn_kda_chunk_workspace_bytes() bytes (the tiled gates and
+ *     gdn2_chunk_fwd's workspace) -> else GDN_ERR_WORKSPACE.
+ *   Returns as gdn2_chunk_fwd.  B = 0 or T = 0 copies h0 to ht (or zeros).
+ */
+int gdn_kda_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
+                      const void* beta, const float* A_log, const float* dt_bias,
+                      const float* h0, int B, int T, int H, int dk, int dv, int dtype,
+                      float scale, int flags, void* o, float* ht, void* workspace,
+                      size_t ws_bytes, gdn_stream_t stream);
+
+/* Device workspace bytes gdn_kda_chunk_fwd needs (0 for invalid sizes). */
+size_t gdn_kda_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype,
+                                     int flags);
+
+/*
  * gdn_rmsnorm_gated -- the gated RMSNorm of the core output
  * ("gated-deltanet-qwen3.5" section 输出门控与 RMSNorm: RMSNormGated(core_attn_out,
  * z), an RMSNorm and then the SwiGLU-like z gate), per row of d_v channels:

@@ -162,6 +162,33 @@ def test_rmsnorm_gated_rejects_bad_arguments():
     assert rn(FAKE, FAKE, FAKE, FAKE, 0, 128, 1, 1e-6, None) == 0
 
 
+def test_kda_workspace_and_arguments():
+    """KDA's workspace: gdn2_chunk_fwd's, then the tiled erase and write gates
+    (B*T*H rows of dk and dv gate elements), each rounded up to 256 bytes."""
+    L = G.lib
+    up = lambda x: (x + 255) // 256 * 256
+    B, T, H, d = 2, 100, 3, 128
+    for dtype, flags, ges in ((1, 0, 2), (1, 2, 4), (0, 0, 4)):
+        want = (up(L.gdn2_chunk_workspace_bytes(B, T, H, d, d, dtype)) + 2 * up(B * T * H * d * ges))
+        assert L.gdn_kda_chunk_workspace_bytes(B, T, H, d, d, dtype, flags) == want
+    assert L.gdn_kda_chunk_workspace_bytes(-1, T, H, d, d, 1, 0) == 0
+    n = L.gdn_kda_chunk_workspace_bytes(B, T, H, d, d, 1, 0)
+    kda = L.gdn_kda_chunk_fwd
+    # (q, k, v, a, beta, A_log, dt_bias, h0, B, T, H, dk, dv, dtype, scale, flags, o, ht,
+    #  ws, ws_bytes, stream)
+    assert kda(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, B, T, H, d, d, 1, 0.1, 1, FAKE,
+               None, FAKE, n, None) == -1
+    assert kda(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, B, T, H, d, d, 1, 0.1, 1, FAKE,
+               None, None, 0, None) == -5
+    assert kda(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, B, T, H, d, d, 1, 0.1, 1, FAKE,
+               None, FAKE, n - 1, None) == -5
+    assert kda(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, B, T, H, 96, d, 1, 0.1, 1, FAKE,
+               None, FAKE, 1 << 40, None) == -2
+    # no tokens: nothing to tile, no state to copy
+    assert kda(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, B, 0, H, d, d, 1, 0.1, 1, FAKE,
+               None, None, 0, None) == 0
+
+
 def test_empty_calls_are_no_ops():
     # zero tokens / zero sequences return before any launch (no state pointers)
     assert _chunk(T=0) == 0
