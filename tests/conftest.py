@@ -20,6 +20,15 @@ def pytest_sessionstart(session):
     mod.build()
 
 
+# The parity tests of the newest entry points run after all the others, so that a
+# run that stops at its first failure (-x) has already reported the rest.
+_RUN_LAST = ("test_kda_gpu.py", "test_rmsnorm_gated_gpu.py")
+
+
+def pytest_collection_modifyitems(session, config, items):
+    items.sort(key=lambda it: os.path.basename(str(it.fspath)) in _RUN_LAST)  # stable
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size parity case (minutes)")
