@@ -19,7 +19,7 @@ import torch
 
 __all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_chunk_workspace_bytes", "gdn_recurrent_step",
            "gdn_conv_prefill", "gdn_rmsnorm_gated", "gdn_kda_chunk_fwd",
-           "gdn_kda_chunk_workspace_bytes",
+           "gdn_kda_chunk_workspace_bytes", "gdn_chunk_fwd_varlen",
            "gdn2_chunk_fwd", "gdn2_chunk_workspace_bytes", "gdn_chunk_fwd_noalloc",
            "gdn_check_status", "GDNError", "LIB_PATH", "lib", "F32", "BF16",
            "QK_L2NORM", "GATES_PRECOMPUTED", "OUT_F32"]
@@ -52,6 +52,8 @@ lib.gdn_chunk_fwd_host_workspace_bytes.restype = _sz
 lib.gdn_recurrent_step.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _vp]
 lib.gdn_conv_prefill.argtypes = [_vp] * 6 + [_i] * 7 + [_vp]
 lib.gdn_rmsnorm_gated.argtypes = [_vp] * 4 + [ctypes.c_long, _i, _i, _f, _vp]
+lib.gdn_chunk_fwd_varlen.argtypes = ([_vp] * 8 + [ctypes.POINTER(ctypes.c_longlong)] + [_i] * 6
+                                     + [_f, _i, _vp, _vp, _vp, _sz, _vp])
 lib.gdn_kda_chunk_fwd.argtypes = [_vp] * 8 + [_i] * 6 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
 lib.gdn_kda_chunk_workspace_bytes.argtypes = [_i] * 7
 lib.gdn_kda_chunk_workspace_bytes.restype = _sz
@@ -66,7 +68,7 @@ lib.gdn_version.argtypes = []
 for _fn in (lib.gdn_gate_prep, lib.gdn_chunk_fwd, lib.gdn_chunk_fwd_noalloc, lib.gdn_chunk_fwd_host,
             lib.gdn2_chunk_fwd,
             lib.gdn_recurrent_step, lib.gdn_conv_prefill, lib.gdn_rmsnorm_gated,
-            lib.gdn_kda_chunk_fwd,
+            lib.gdn_kda_chunk_fwd, lib.gdn_chunk_fwd_varlen,
             lib.gdn_check_status, lib.gdn_version):
     _fn.restype = _i
 
@@ -311,6 +313,49 @@ def gdn2_chunk_fwd(q, k, v, a, b_logit, w_logit, A_log=None, dt_bias=None, h0=No
                               float(scale), flags, _p(o), _p(ht), _p(workspace), ws_bytes,
                               _stream(stream)),
            "gdn2_chunk_fwd")
+    return o, ht
+
+
+def gdn_chunk_fwd_varlen(q, k, v, a, b, A_log, dt_bias, h0, cu_seqlens, *, scale=None,
+                         l2norm=True, gates_precomputed=False, out_f32=False, o=None, ht=None,
+                         want_ht=True, workspace=None, stream=None):
+    """Chunkwise GDN prefill over a packed batch: q, k [T_total, Hk, dk]; v
+    [T_total, Hv, dv]; a, b [T_total, Hv]; cu_seqlens: N + 1 token offsets (a list
+    or a CPU int64 tensor, first 0); h0 [N, Hv, dk, dv] or None.  Returns
+    (o [T_total, Hv, dv], ht [N, Hv, dk, dv] or None)."""
+    cu = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    N = len(cu) - 1
+    Tt, Hk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    dt = q.dtype
+    scale = dk ** -0.5 if scale is None else scale
+    gdt = torch.float32 if gates_precomputed else dt
+    _need(k, dt, q.shape, "k")
+    _need(v, dt, (Tt, Hv, dv), "v")
+    _need(a, gdt, (Tt, Hv), "a")
+    _need(b, gdt, (Tt, Hv), "b")
+    if N < 0 or cu[0] != 0 or cu[-1] != Tt:
+        raise ValueError("cu_seqlens must start at 0 and end at the packed token count")
+    if h0 is not None:
+        _need(h0, torch.float32, (N, Hv, dk, dv), "h0")
+    odt = torch.float32 if out_f32 else dt
+    o = torch.empty((Tt, Hv, dv), device=q.device, dtype=odt) if o is None else o
+    _need(o, odt, (Tt, Hv, dv), "o")
+    if ht is None and want_ht:
+        ht = torch.empty((N, Hv, dk, dv), device=q.device, dtype=torch.float32)
+    flags = ((QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
+             | (OUT_F32 if out_f32 else 0))
+    longest = max([cu[i + 1] - cu[i] for i in range(N)] + [0])
+    ws_need = gdn_chunk_workspace_bytes(1, longest, Hk, Hv, dk, dv, dt) if longest else 0
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    cu_arr = (ctypes.c_longlong * len(cu))(*cu)
+    _check(lib.gdn_chunk_fwd_varlen(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(dt_bias),
+                                    _p(h0), cu_arr, N, Hk, Hv, dk, dv, _dtype_code(dt),
+                                    float(scale), flags, _p(o), _p(ht), _p(workspace), ws_bytes,
+                                    _stream(stream)),
+           "gdn_chunk_fwd_varlen")
     return o, ht
 
 

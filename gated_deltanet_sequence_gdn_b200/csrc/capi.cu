@@ -144,6 +144,64 @@ int gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* a, co
   return run_chunk(c, false, workspace, ws_bytes, (cudaStream_t)stream);
 }
 
+// Sequence i of a packed batch: the arguments of a one-sequence gdn_chunk_fwd call
+// on its token range [t0, t0 + Ti) and its own initial / final state.
+static ChunkArgs varlen_seq(const ChunkArgs& all, long long t0, int Ti, int i) {
+  const size_t es = elem_size(all.dtype);
+  const size_t ges = (all.flags & GDN_GATES_PRECOMPUTED) ? 4 : es;
+  const size_t oes = (all.flags & GDN_OUT_F32) ? 4 : es;
+  const size_t st = (size_t)all.Hv * all.dk * all.dv;
+  auto at = [](const void* p, size_t off) -> const void* {
+    return p ? static_cast<const uint8_t*>(p) + off : nullptr;
+  };
+  ChunkArgs c = all;
+  c.q = at(all.q, (size_t)t0 * all.Hk * all.dk * es);
+  c.k = at(all.k, (size_t)t0 * all.Hk * all.dk * es);
+  c.v = at(all.v, (size_t)t0 * all.Hv * all.dv * es);
+  c.a = at(all.a, (size_t)t0 * all.Hv * ges);
+  c.b = at(all.b, (size_t)t0 * all.Hv * ges);
+  c.o = all.o ? static_cast<uint8_t*>(all.o) + (size_t)t0 * all.Hv * all.dv * oes : nullptr;
+  c.h0 = all.h0 ? all.h0 + (size_t)i * st : nullptr;
+  c.ht = all.ht ? all.ht + (size_t)i * st : nullptr;
+  c.B = 1;
+  c.T = Ti;
+  return c;
+}
+
+int gdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, const void* a,
+                         const void* b, const float* A_log, const float* dt_bias,
+                         const float* h0, const long long* cu_seqlens, int N, int Hk, int Hv,
+                         int dk, int dv, int dtype, float scale, int flags, void* o, float* ht,
+                         void* workspace, size_t ws_bytes, gdn_stream_t stream) {
+  if (N < 0 || !ok_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  if (N == 0) return GDN_OK;
+  if (cu_seqlens == nullptr || cu_seqlens[0] != 0) return GDN_ERR_INVALID_ARG;
+  for (int i = 0; i < N; ++i) {
+    const long long Ti = cu_seqlens[i + 1] - cu_seqlens[i];
+    if (Ti < 0 || Ti > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
+  }
+  const ChunkArgs all{q, k, v, a, b, nullptr, A_log, dt_bias, h0, 1, 0, Hk, Hv, dk, dv,
+                      dtype, scale, flags, o, ht};
+  // every sequence is checked before anything is enqueued
+  for (int i = 0; i < N; ++i) {
+    const int Ti = (int)(cu_seqlens[i + 1] - cu_seqlens[i]);
+    const ChunkArgs c = varlen_seq(all, cu_seqlens[i], Ti, i);
+    const int st = validate_chunk(c, false);
+    if (st != GDN_OK) return st;
+    if (Ti > 0 && chunk_mma_supported(c) &&
+        (workspace == nullptr || !aligned16(workspace) ||
+         ws_bytes < chunk_mma_workspace_bytes(1, Ti, Hk, Hv)))
+      return GDN_ERR_WORKSPACE;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  for (int i = 0; i < N; ++i) {
+    const int Ti = (int)(cu_seqlens[i + 1] - cu_seqlens[i]);
+    const int st = run_chunk(varlen_seq(all, cu_seqlens[i], Ti, i), false, workspace, ws_bytes, s);
+    if (st != GDN_OK) return st;
+  }
+  return GDN_OK;
+}
+
 int gdn2_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
                    const void* b_logit, const void* w_logit, const float* A_log,
                    const float* dt_bias, const float* h0, int B, int T, int H, int dk, int dv,

@@ -249,6 +249,31 @@ int gdn_conv_prefill(const void* x_qkv, const float* conv_w, void* conv_state,
                      int dk, int dv, int dtype, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_fwd_varlen -- gdn_chunk_fwd over a packed batch of N sequences of
+ * different lengths: sequence i is tokens cu_seqlens[i] .. cu_seqlens[i+1] - 1
+ * of the packed arrays, with its own initial and final state, and its chunks
+ * start at its first token (the result of N one-sequence calls, run one after
+ * another on the stream).  The pages batch sequences by padding
+ * ("gated-deltanet-qwen3.5" architecture diagram, apply_mask_to_padding_states);
+ * packing is this library's way to batch without the padded tokens.
+ *   q, k [T_total, Hk, dk]; v, o [T_total, Hv, dv]; a, b [T_total, Hv]
+ *     (T_total = cu_seqlens[N]), dtypes, flags and scale as for gdn_chunk_fwd.
+ *   h0 / ht [N, Hv, dk, dv] float32 or NULL (ht may alias h0).
+ *   cu_seqlens: HOST array of N + 1 int64, cu_seqlens[0] = 0, non-decreasing;
+ *     read during the call only.  Empty sequences copy their h0 to ht.
+ *   workspace / ws_bytes: as for gdn_chunk_fwd, at least
+ *     gdn_chunk_workspace_bytes(1, longest sequence, ...) bytes; it is reused
+ *     by every sequence.
+ *   Every sequence is checked before anything is enqueued.  Returns as
+ *   gdn_chunk_fwd, and GDN_ERR_INVALID_ARG for a bad cu_seqlens.
+ */
+int gdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, const void* a,
+                         const void* b, const float* A_log, const float* dt_bias,
+                         const float* h0, const long long* cu_seqlens, int N, int Hk, int Hv,
+                         int dk, int dv, int dtype, float scale, int flags, void* o,
+                         float* ht, void* workspace, size_t ws_bytes, gdn_stream_t stream);
+
+/*
  * gdn_kda_chunk_fwd -- KDA (Kimi Delta Attention): the channel-wise decay of
  * Gated DeltaNet-2 with one scalar beta per (token, head) for both the erase
  * and the write, S_t = (I - beta_t k_t k_t^T) D_t S_{t-1} + beta_t k_t v_t^T,

@@ -189,6 +189,27 @@ def test_kda_workspace_and_arguments():
                None, None, 0, None) == 0
 
 
+def test_varlen_checks_cu_seqlens_before_anything():
+    import ctypes as C
+    vl = G.lib.gdn_chunk_fwd_varlen
+    arr = lambda *xs: (C.c_longlong * len(xs))(*xs)
+    # (q, k, v, a, b, A_log, dt_bias, h0, cu, N, Hk, Hv, dk, dv, dtype, scale, flags, o, ht,
+    #  ws, ws_bytes, stream)
+    args = lambda cu, N, **kw: [kw.get("q", FAKE), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, cu,
+                                N, 2, 4, 128, 128, 1, 0.1, 1, FAKE, None,
+                                kw.get("ws", FAKE), kw.get("ws_bytes", 1 << 40), None]
+    assert vl(*args(arr(0, 5), 0)) == 0                    # N = 0
+    assert vl(*args(None, 2)) == -1                        # no offsets
+    assert vl(*args(arr(1, 5, 9), 2)) == -1                # does not start at 0
+    assert vl(*args(arr(0, 9, 5), 2)) == -1                # decreasing
+    assert vl(*args(arr(0, 0, 0), 2)) == 0                 # empty sequences, no ht: nothing
+    assert vl(*args(arr(0, 64, 100), 2, ws=None, ws_bytes=0)) == -5
+    assert vl(*args(arr(0, 64, 100), 2, q=None)) == -1
+    # a sequence's workspace need is checked against the longest one
+    need = G.lib.gdn_chunk_workspace_bytes(1, 300, 2, 4, 128, 128, 1)
+    assert vl(*args(arr(0, 64, 364), 2, ws_bytes=need - 1)) == -5
+
+
 def test_empty_calls_are_no_ops():
     # zero tokens / zero sequences return before any launch (no state pointers)
     assert _chunk(T=0) == 0
