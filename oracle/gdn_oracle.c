@@ -382,6 +382,175 @@ int oracle_gdn2_fwd(const void* q, const void* k, const void* v, const void* a,
   return err;
 }
 
+/* Gradient of the L2 norm and scale of load_vec: x -> scale * x / sqrt(sum x^2 + eps)
+ * (or scale * x without the norm); gy is the gradient at the output, gx += the
+ * gradient at the input. */
+static void load_vec_bwd(const double* x, int n, int l2norm, double scale, const double* gy,
+                         double* gx) {
+  if (!l2norm) {
+    for (int i = 0; i < n; ++i) gx[i] += scale * gy[i];
+    return;
+  }
+  double ss = 0.0, xg = 0.0;
+  for (int i = 0; i < n; ++i) {
+    ss += x[i] * x[i];
+    xg += x[i] * gy[i];
+  }
+  const double nrm = sqrt(ss + 1e-6);
+  for (int i = 0; i < n; ++i) gx[i] += scale * (gy[i] / nrm - x[i] * xg / (nrm * nrm * nrm));
+}
+
+/*
+ * Backward of oracle_gdn_fwd (the next step after the forward pass): reverse-mode
+ * differentiation of the five-step token recurrence, token by token from the
+ * last, with the states of the forward pass stored.  For a cotangent do on o and
+ * dht on the final state, it returns the gradients of sum(o * do) + sum(ht * dht):
+ *   dq, dk [B,T,Hk,dk] (summed over the value heads of a key head), dv [B,T,Hv,dv],
+ *   da, db [B,T,Hv] (with gates_given: the gradients with respect to g and beta),
+ *   dA_log, ddt_bias [Hv] (summed over batch and tokens; untouched with
+ *   gates_given), dh0 [B,Hv,dk,dv].  dht may be NULL (zero).  Single-threaded:
+ *   it is meant for the small cases of the tests.
+ * Per token, with S the state before it:
+ *   S' = a S ; kv = S'^T k ; d = b (v - kv) ; S_t = S' + k d^T ; o = S_t^T q
+ * reversed: dS += q do^T, dq = S_t do ; dk = dS d, dd = dS^T k ; db = dd.(v - kv),
+ * dv = b dd, dkv = -b dd ; dS' = dS + k dkv^T, dk += S' dkv ; dS <- a dS',
+ * da = <dS', S>.
+ */
+int oracle_gdn_bwd(const double* q, const double* k, const double* v, const double* a,
+                   const double* b, const double* A_log, const double* dt_bias,
+                   const double* h0, const double* dout, const double* dht, int B, int T,
+                   int Hk, int Hv, int dk, int dv, double scale, int l2norm, int gates_given,
+                   double* dq, double* dkk, double* dvv, double* da, double* db,
+                   double* dA_log, double* ddt_bias, double* dh0) {
+  if (B < 0 || T < 0 || Hk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0 || Hv % Hk) return ORACLE_EINVAL;
+  const int group = Hv / Hk;
+  const size_t SZ = (size_t)dk * dv;
+  memset(dq, 0, sizeof(double) * (size_t)B * T * Hk * dk);
+  memset(dkk, 0, sizeof(double) * (size_t)B * T * Hk * dk);
+  if (!gates_given) {
+    memset(dA_log, 0, sizeof(double) * Hv);
+    memset(ddt_bias, 0, sizeof(double) * Hv);
+  }
+  double* Sp = (double*)malloc(sizeof(double) * SZ * ((size_t)T + 1));  /* states S_0 .. S_T */
+  double* St = (double*)malloc(sizeof(double) * SZ);                    /* S' of a token */
+  double* dS = (double*)malloc(sizeof(double) * SZ);
+  double* dSp = (double*)malloc(sizeof(double) * SZ);
+  double* w = (double*)malloc(sizeof(double) * (size_t)(4 * dk + 6 * dv + 4));
+  if (!Sp || !St || !dS || !dSp || !w) {
+    free(Sp); free(St); free(dS); free(dSp); free(w);
+    return ORACLE_ENOMEM;
+  }
+  double *qt = w, *kt = qt + dk, *gq = kt + dk, *gk = gq + dk;
+  double *vt = gk + dk, *kv = vt + dv, *dd = kv + dv, *dl = dd + dv, *ot = dl + dv, *dkv = ot + dv;
+  for (int bi = 0; bi < B; ++bi)
+    for (int hv = 0; hv < Hv; ++hv) {
+      const int hk = hv / group;
+      const size_t bh = (size_t)bi * Hv + hv;
+      for (size_t x = 0; x < SZ; ++x) Sp[x] = h0 ? h0[bh * SZ + x] : 0.0;
+      /* forward, keeping S_0 .. S_T */
+      for (int t = 0; t < T; ++t) {
+        const size_t row = (size_t)bi * T + t;
+        load_vec(q, 1, (row * Hk + hk) * dk, dk, l2norm, scale, qt);
+        load_vec(k, 1, (row * Hk + hk) * dk, dk, l2norm, 1.0, kt);
+        load_vec(v, 1, (row * Hv + hv) * dv, dv, 0, 1.0, vt);
+        double g, beta;
+        if (gates_given) {
+          g = a[row * Hv + hv];
+          beta = b[row * Hv + hv];
+        } else {
+          gdn_gates(a[row * Hv + hv], b[row * Hv + hv], A_log[hv], dt_bias[hv], &g, &beta);
+        }
+        memcpy(Sp + (size_t)(t + 1) * SZ, Sp + (size_t)t * SZ, sizeof(double) * SZ);
+        gdn_token_step(Sp + (size_t)(t + 1) * SZ, dk, dv, qt, kt, vt, exp(g), beta, kv, ot);
+      }
+      /* backward */
+      for (size_t x = 0; x < SZ; ++x) dS[x] = dht ? dht[bh * SZ + x] : 0.0;
+      for (int t = T - 1; t >= 0; --t) {
+        const size_t row = (size_t)bi * T + t;
+        const double* S0 = Sp + (size_t)t * SZ;   /* state before the token */
+        const double* S1 = Sp + (size_t)(t + 1) * SZ;
+        load_vec(q, 1, (row * Hk + hk) * dk, dk, l2norm, scale, qt);
+        load_vec(k, 1, (row * Hk + hk) * dk, dk, l2norm, 1.0, kt);
+        load_vec(v, 1, (row * Hv + hv) * dv, dv, 0, 1.0, vt);
+        double g, beta;
+        if (gates_given) {
+          g = a[row * Hv + hv];
+          beta = b[row * Hv + hv];
+        } else {
+          gdn_gates(a[row * Hv + hv], b[row * Hv + hv], A_log[hv], dt_bias[hv], &g, &beta);
+        }
+        const double alpha = exp(g);
+        const double* dO = dout + (row * Hv + hv) * dv;
+        /* recompute S', kv and delta of the token */
+        for (size_t x = 0; x < SZ; ++x) St[x] = alpha * S0[x];
+        for (int j = 0; j < dv; ++j) kv[j] = 0.0;
+        for (int i = 0; i < dk; ++i)
+          for (int j = 0; j < dv; ++j) kv[j] += St[(size_t)i * dv + j] * kt[i];
+        for (int j = 0; j < dv; ++j) dl[j] = beta * (vt[j] - kv[j]);
+        /* o = S_t^T q */
+        for (int i = 0; i < dk; ++i) {
+          double acc = 0.0;
+          for (int j = 0; j < dv; ++j) {
+            acc += S1[(size_t)i * dv + j] * dO[j];
+            dS[(size_t)i * dv + j] += qt[i] * dO[j];
+          }
+          gq[i] = acc;
+        }
+        /* S_t = S' + k delta^T */
+        for (int i = 0; i < dk; ++i) {
+          double acc = 0.0;
+          for (int j = 0; j < dv; ++j) acc += dS[(size_t)i * dv + j] * dl[j];
+          gk[i] = acc;
+        }
+        for (int j = 0; j < dv; ++j) {
+          double acc = 0.0;
+          for (int i = 0; i < dk; ++i) acc += dS[(size_t)i * dv + j] * kt[i];
+          dd[j] = acc;
+        }
+        /* delta = beta (v - kv) */
+        double dbeta = 0.0;
+        for (int j = 0; j < dv; ++j) {
+          dbeta += dd[j] * (vt[j] - kv[j]);
+          dvv[(row * Hv + hv) * dv + j] = beta * dd[j];
+          dkv[j] = -beta * dd[j];
+        }
+        /* kv = S'^T k */
+        for (int i = 0; i < dk; ++i) {
+          double acc = 0.0;
+          for (int j = 0; j < dv; ++j) {
+            dSp[(size_t)i * dv + j] = dS[(size_t)i * dv + j] + kt[i] * dkv[j];
+            acc += St[(size_t)i * dv + j] * dkv[j];
+          }
+          gk[i] += acc;
+        }
+        /* S' = alpha S */
+        double dalpha = 0.0;
+        for (size_t x = 0; x < SZ; ++x) {
+          dalpha += dSp[x] * S0[x];
+          dS[x] = alpha * dSp[x];
+        }
+        const double dg = dalpha * alpha;
+        if (gates_given) {
+          da[row * Hv + hv] = dg;
+          db[row * Hv + hv] = dbeta;
+        } else {
+          const double xg = a[row * Hv + hv] + dt_bias[hv];
+          const double dx = dg * (-exp(A_log[hv])) * sigmoid(xg);
+          da[row * Hv + hv] = dx;
+          ddt_bias[hv] += dx;
+          dA_log[hv] += dg * g;
+          db[row * Hv + hv] = dbeta * beta * (1.0 - beta);
+        }
+        /* the norms of q and k */
+        load_vec_bwd(q + (row * Hk + hk) * dk, dk, l2norm, scale, gq, dq + (row * Hk + hk) * dk);
+        load_vec_bwd(k + (row * Hk + hk) * dk, dk, l2norm, 1.0, gk, dkk + (row * Hk + hk) * dk);
+      }
+      if (dh0) memcpy(dh0 + bh * SZ, dS, sizeof(double) * SZ);
+    }
+  free(Sp); free(St); free(dS); free(dSp); free(w);
+  return ORACLE_OK;
+}
+
 /*
  * KDA (Kimi Delta Attention) as the "Gated DeltaNet-2" page states its update
  * (section 标量绑定的数学表达), computed literally:

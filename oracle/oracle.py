@@ -16,6 +16,8 @@ Each function cites the passage it follows (page title and section):
   (Linear -> CausalConv1D -> SiLU -> q, k, v).
 * ``conv_step`` / ``conv_prefill`` -- that conv alone, for one token or a whole
   prefill ("gated-deltanet-qwen3.5" section 因果卷积: kernel 4, depthwise, causal).
+* ``gdn_bwd``      -- the backward of ``gdn_fwd`` (the survey's last next row):
+  reverse-mode through the same five steps, pinned by finite differences.
 * ``kda_fwd``      -- "Gated DeltaNet-2" (zhichai), section 标量绑定的数学表达 (the
   KDA update with its erase projection written out) and 退化兼容性.
 * ``rmsnorm_gated`` -- "gated-deltanet-qwen3.5" section 输出门控与 RMSNorm
@@ -70,8 +72,10 @@ def _load():
             lib.oracle_conv_prefill.argtypes = [vp, vp, ip, ip, ip, ip, vp, vp]
             lib.oracle_rmsnorm_gated.argtypes = [vp, vp, vp, ip, ip, ip, dp, vp]
             lib.oracle_kda_fwd.argtypes = [vp] * 8 + [ip] * 6 + [dp, ip, vp, vp, ip]
+            lib.oracle_gdn_bwd.argtypes = [vp] * 10 + [ip] * 6 + [dp, ip, ip] + [vp] * 8
             for f in (lib.oracle_gdn_fwd, lib.oracle_gate_prep, lib.oracle_conv_step,
                       lib.oracle_conv_prefill, lib.oracle_rmsnorm_gated, lib.oracle_kda_fwd,
+                      lib.oracle_gdn_bwd,
                       lib.oracle_gdn_decode_step, lib.oracle_gdn2_fwd):
                 f.restype = ctypes.c_int
             lib.oracle_max_threads.restype = ctypes.c_int
@@ -204,6 +208,33 @@ def conv_prefill(x, conv_w, conv_state):
                                      _ptr(y))
     _check(rc, "oracle_conv_prefill")
     return y
+
+
+def gdn_bwd(q, k, v, a, b, A_log, dt_bias, h0, do, dht=None, *, scale=None, l2norm=True,
+            gates_given=False):
+    """Gradients of sum(o * do) + sum(ht * dht) for gdn_fwd's (o, ht), by reverse-mode
+    differentiation of the token recurrence (float64 throughout).
+
+    Shapes as for gdn_fwd; do [B,T,Hv,dv]; dht [B,Hv,dk,dv] or None.  Returns a dict
+    with dq, dk, dv, da, db, dA_log, ddt_bias, dh0 (with gates_given, da / db are the
+    gradients with respect to g and beta, and dA_log / ddt_bias are None).
+    """
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    f = lambda x: None if x is None else _arr(x, True)
+    arrs = [f(x) for x in (q, k, v, a, b, A_log, dt_bias, h0, do, dht)]
+    if scale is None:
+        scale = dk ** -0.5
+    out = {"dq": np.zeros((B, T, Hk, dk)), "dk": np.zeros((B, T, Hk, dk)),
+           "dv": np.zeros((B, T, Hv, dv)), "da": np.zeros((B, T, Hv)), "db": np.zeros((B, T, Hv)),
+           "dA_log": None if gates_given else np.zeros(Hv),
+           "ddt_bias": None if gates_given else np.zeros(Hv), "dh0": np.zeros((B, Hv, dk, dv))}
+    rc = _load().oracle_gdn_bwd(*[_ptr(x) for x in arrs], B, T, Hk, Hv, dk, dv, float(scale),
+                                int(l2norm), int(gates_given),
+                                *[_ptr(out[n]) for n in ("dq", "dk", "dv", "da", "db", "dA_log",
+                                                         "ddt_bias", "dh0")])
+    _check(rc, "oracle_gdn_bwd")
+    return out
 
 
 def kda_fwd(q, k, v, a, b, A_log, dt_bias, h0=None, *, scale=None, l2norm=True,

@@ -53,6 +53,15 @@ MUTANTS = [
     ("conv_prefill_time_major",  # x read as [T, B, Cc]
      "      conv_silu_step(x, ((size_t)b * T + t) * Cc, conv_w, in_f64, Cc,",
      "      conv_silu_step(x, ((size_t)t * B + b) * Cc, conv_w, in_f64, Cc,"),
+    ("bwd_read_term_dropped",  # dS' misses k dkv^T
+     "            dSp[(size_t)i * dv + j] = dS[(size_t)i * dv + j] + kt[i] * dkv[j];",
+     "            dSp[(size_t)i * dv + j] = dS[(size_t)i * dv + j];"),
+    ("bwd_decay_missing", "          dS[x] = alpha * dSp[x];", "          dS[x] = dSp[x];"),
+    ("bwd_dbeta_sign", "          dbeta += dd[j] * (vt[j] - kv[j]);",
+     "          dbeta += dd[j] * (kv[j] - vt[j]);"),
+    ("bwd_norm_projection_dropped",
+     "  for (int i = 0; i < n; ++i) gx[i] += scale * (gy[i] / nrm - x[i] * xg / (nrm * nrm * nrm));",
+     "  for (int i = 0; i < n; ++i) gx[i] += scale * (gy[i] / nrm);"),
     ("kda_decay_dropped",  # the projection applied to S instead of D S
      "        for (int j = 0; j < dv; ++j) DS[(size_t)i * dv + j] = dec[i] * S[(size_t)i * dv + j];",
      "        for (int j = 0; j < dv; ++j) DS[(size_t)i * dv + j] = S[(size_t)i * dv + j];"),
@@ -98,6 +107,7 @@ def _run_pins_against(lib_path):
     mutant = ctypes.CDLL(lib_path)
     for fname in ("oracle_gdn_fwd", "oracle_gate_prep", "oracle_conv_step",
                   "oracle_conv_prefill", "oracle_rmsnorm_gated", "oracle_kda_fwd",
+                  "oracle_gdn_bwd",
                   "oracle_gdn_decode_step",
                   "oracle_gdn2_fwd"):
         getattr(mutant, fname).argtypes = getattr(real, fname).argtypes

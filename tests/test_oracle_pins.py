@@ -236,6 +236,44 @@ def test_kda_with_scalar_decay_is_gdn():
     np.testing.assert_allclose(ht1, ht2, rtol=1e-12, atol=1e-13)
 
 
+@pytest.mark.parametrize("l2norm,gates_given", [(True, False), (False, True), (True, True)])
+def test_gdn_backward_matches_finite_differences(l2norm, gates_given):
+    """The backward of the token recurrence against central finite differences of
+    L = sum(o * R_o) + sum(ht * R_h), one random direction per input tensor, with
+    grouped heads (the q / k gradients sum over a key head's value heads)."""
+    B, T, Hk, Hv, d = 2, 5, 1, 2, 4
+    q, k, v = _rand(B, T, Hk, d), _rand(B, T, Hk, d), _rand(B, T, Hv, d)
+    if gates_given:
+        a, b = -rng.uniform(0.05, 1.0, size=(B, T, Hv)), rng.uniform(0.1, 0.9, size=(B, T, Hv))
+        A_log = dt_bias = None
+    else:
+        a, b = _rand(B, T, Hv), _rand(B, T, Hv)
+        A_log, dt_bias = rng.uniform(0, math.log(16), size=Hv), rng.uniform(-4, -1, size=Hv)
+    h0 = 0.3 * _rand(B, Hv, d, d)
+    Ro, Rh = _rand(B, T, Hv, d), _rand(B, Hv, d, d)
+    kw = dict(scale=0.7, l2norm=l2norm, gates_given=gates_given)
+    inputs = dict(q=q, k=k, v=v, a=a, b=b, A_log=A_log, dt_bias=dt_bias, h0=h0)
+
+    def loss(x):
+        o, ht = O.gdn_fwd(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                          x["h0"], **kw)
+        return float(np.sum(o * Ro) + np.sum(ht * Rh))
+
+    g = O.gdn_bwd(q, k, v, a, b, A_log, dt_bias, h0, Ro, Rh, **kw)
+    names = dict(q="dq", k="dk", v="dv", a="da", b="db", A_log="dA_log", dt_bias="ddt_bias",
+                 h0="dh0")
+    h = 1e-5
+    for n, x0 in inputs.items():
+        if x0 is None:
+            continue
+        u = _rand(*x0.shape)
+        xp, xm = dict(inputs), dict(inputs)
+        xp[n], xm[n] = x0 + h * u, x0 - h * u
+        fd = (loss(xp) - loss(xm)) / (2 * h)
+        an = float(np.sum(g[names[n]] * u))
+        assert abs(fd - an) <= 1e-7 * max(1.0, abs(fd)), (n, fd, an)
+
+
 # --------------------------------------------------------------------------
 # Gates and normalisation: closed forms
 # --------------------------------------------------------------------------
