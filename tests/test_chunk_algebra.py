@@ -107,6 +107,92 @@ def chunk_gdn2(q, k, v, g, b, w, S0, C, sub=16):
     return o, S
 
 
+def chunk_gdn_bwd(q, k, v, g, beta, S0, dO, dST, C):
+    """Backward of the scalar-decay chunk form above: the derivation a chunkwise
+    backward follows.  Chunks are taken from the last, the state gradient carried
+    from each chunk to the one before; a chunk's start state comes from the
+    forward chunk recurrence.  Per chunk, with K~ = diag(gamma_C / gamma) K,
+    U~ = U - W S0, O = diag(gamma) Q S0 + A_qk U~ and S1 = gamma_C S0 + K~^T U~,
+    the gradients run back through U = A diag(beta) V, W = A diag(beta gamma) K,
+    A = (I + L)^-1 (dL = -A^T dA A^T, kept strictly lower), the Gamma masks and
+    G = cumsum(g) (dg = reverse cumulative sum of dG).
+    Returns dq, dk, dv, dg, dbeta and the gradient of the initial state."""
+    T, dk = q.shape
+    starts, S = [], S0.copy()
+    for c0 in range(0, T, C):
+        starts.append(S.copy())
+        _, S = chunk_gdn(q[c0:c0 + C], k[c0:c0 + C], v[c0:c0 + C], g[c0:c0 + C],
+                         beta[c0:c0 + C], S, C)
+    dq, dk_, dv_ = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dg, dbeta = np.zeros(T), np.zeros(T)
+    dS = dST.copy()
+    for ci in reversed(range(len(starts))):
+        c0 = ci * C
+        c1 = min(c0 + C, T)
+        n = c1 - c0
+        Kc, Qc, Vc, bc, S = k[c0:c1], q[c0:c1], v[c0:c1], beta[c0:c1], starts[ci]
+        G = np.cumsum(g[c0:c1])
+        gam = np.exp(G)
+        gC = gam[-1]
+        low = np.tril(np.ones((n, n)))
+        Gam = np.exp(np.where(low > 0, G[:, None] - G[None, :], -np.inf))
+        KK, QK = Kc @ Kc.T, Qc @ Kc.T
+        M = KK * Gam
+        L = np.tril(bc[:, None] * M, -1)
+        A = forward_substitution_inverse(L)
+        Kb, Vb = (bc * gam)[:, None] * Kc, bc[:, None] * Vc
+        W, U = A @ Kb, A @ Vb
+        Aqk = np.tril(QK * Gam)
+        Ut = U - W @ S
+        ratio = gC / gam
+        Kt = ratio[:, None] * Kc
+        # S1 = gamma_C S0 + K~^T U~
+        dS0 = gC * dS
+        dgC = float(np.sum(dS * S))
+        dKt, dUt = Ut @ dS.T, Kt @ dS
+        # O = diag(gamma) Q S0 + A_qk U~
+        dOc = dO[c0:c1]
+        dgam = np.sum(dOc * (Qc @ S), axis=1)
+        dQ = gam[:, None] * (dOc @ S.T)
+        dS0 += (gam[:, None] * Qc).T @ dOc
+        dAqk = np.tril(dOc @ Ut.T)
+        dUt += Aqk.T @ dOc
+        # U~ = U - W S0
+        dU, dW = dUt, -dUt @ S.T
+        dS0 -= W.T @ dUt
+        # U = A Vb, W = A Kb
+        dA = dU @ Vb.T + dW @ Kb.T
+        dVb, dKb = A.T @ dU, A.T @ dW
+        dV = bc[:, None] * dVb
+        db = np.sum(dVb * Vc, axis=1)
+        dK = (bc * gam)[:, None] * dKb
+        dbg = np.sum(dKb * Kc, axis=1)
+        db += dbg * gam
+        dgam += dbg * bc
+        # A = (I + L)^-1, L = tril(diag(beta) (K K^T o Gamma), -1)
+        dL = np.tril(-A.T @ dA @ A.T, -1)
+        db += np.sum(dL * M, axis=1)
+        dM = bc[:, None] * dL
+        dKK, dGam = dM * Gam, dM * KK
+        dK += (dKK + dKK.T) @ Kc
+        # A_qk = tril(Q K^T o Gamma)
+        dQK = dAqk * Gam
+        dGam += dAqk * QK
+        dQ += dQK @ Kc
+        dK += dQK.T @ Qc
+        # K~ = diag(gamma_C / gamma) K
+        dK += ratio[:, None] * dKt
+        dratio = np.sum(dKt * Kc, axis=1)
+        # G: Gamma_rj = exp(G_r - G_j), gamma = exp(G), ratio = exp(G_C - G), gamma_C
+        tG = dGam * Gam
+        dG = tG.sum(1) - tG.sum(0) + dgam * gam - dratio * ratio
+        dG[-1] += float(np.sum(dratio * ratio)) + dgC * gC
+        dg[c0:c1] = np.cumsum(dG[::-1])[::-1]
+        dq[c0:c1], dk_[c0:c1], dv_[c0:c1], dbeta[c0:c1] = dQ, dK, dV, db
+        dS = dS0
+    return dq, dk_, dv_, dg, dbeta, dS
+
+
 def _gates(T, H, A_log, dt_bias, a, b):
     sp = np.log1p(np.exp(a + dt_bias))
     return -np.exp(A_log) * sp, 1 / (1 + np.exp(-b))
@@ -164,3 +250,26 @@ def test_scalar_gates_through_gdn2_chunk_form():
                         np.repeat(beta[:, None], dv, 1), S0, 64)
     np.testing.assert_allclose(o2, o1, rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(S2, S1, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("T", [1, 37, 64, 130])
+@pytest.mark.parametrize("C", [1, 16, 64])
+def test_chunk_gdn_backward_equals_token_backward(T, C):
+    """The chunkwise backward against the oracle's token-by-token backward (itself
+    pinned by finite differences), same gates and normalised keys."""
+    dk, dv = 16, 8
+    q, k, v = rng.standard_normal((T, dk)), rng.standard_normal((T, dk)), rng.standard_normal((T, dv))
+    q /= np.linalg.norm(q, axis=1, keepdims=True) * 4.0
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    g = -rng.uniform(0.0, 3.0, size=T)
+    beta = rng.uniform(0.0, 1.0, size=T)
+    S0 = 0.1 * rng.standard_normal((dk, dv))
+    dO, dST = rng.standard_normal((T, dv)), rng.standard_normal((dk, dv))
+    ref = O.gdn_bwd(q[None, :, None], k[None, :, None], v[None, :, None], g[None, :, None],
+                    beta[None, :, None], None, None, S0[None, None], dO[None, :, None],
+                    dST[None, None], scale=1.0, l2norm=False, gates_given=True)
+    dq, dk_, dv_, dg, dbeta, dS0 = chunk_gdn_bwd(q, k, v, g, beta, S0, dO, dST, C)
+    for got, want in ((dq, ref["dq"][0, :, 0]), (dk_, ref["dk"][0, :, 0]),
+                      (dv_, ref["dv"][0, :, 0]), (dg, ref["da"][0, :, 0]),
+                      (dbeta, ref["db"][0, :, 0]), (dS0, ref["dh0"][0, 0])):
+        np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-10)
