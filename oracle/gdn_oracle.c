@@ -552,6 +552,155 @@ int oracle_gdn_bwd(const double* q, const double* k, const double* v, const doub
 }
 
 /*
+ * Backward of oracle_gdn2_fwd ("Gated DeltaNet-2", section Gate-aware 反向传播:
+ * the per-channel gates stay inside the accumulations), reverse-mode token by
+ * token from the last, the forward states stored.  Per token, with S the state
+ * before it, d = exp(g) per key channel, e = b (.) k, z = w (.) v:
+ *   S_bar = diag(d) S ; r = S_bar^T e ; S_t = S_bar + k (z - r)^T ; o = S_t^T q
+ * reversed: dS += q do^T, dq = S_t do ; m = dS^T k, dk = dS (z - r), dz = m,
+ * dr = -m ; dS_bar = dS + e dr^T, de = S_bar dr ; db = de (.) k, dk += de (.) b ;
+ * dw = dz (.) v, dv = dz (.) w ; dS <- diag(d) dS_bar, dd_i = <dS_bar_i, S_i>.
+ * Gradients of sum(o * do) + sum(ht * dht): dq, dk [B,T,H,dk], dv [B,T,H,dv],
+ * da, db [B,T,H,dk], dw [B,T,H,dv] (with gates_given: with respect to g, b, w),
+ * dA_log, ddt_bias [H,dk] (summed over batch and tokens), dh0 [B,H,dk,dv].
+ */
+int oracle_gdn2_bwd(const double* q, const double* k, const double* v, const double* a,
+                    const double* b_logit, const double* w_logit, const double* A_log,
+                    const double* dt_bias, const double* h0, const double* dout,
+                    const double* dht, int B, int T, int H, int dk, int dv, double scale,
+                    int l2norm, int gates_given, double* dq, double* dkk, double* dvv,
+                    double* da, double* db, double* dw, double* dA_log, double* ddt_bias,
+                    double* dh0) {
+  if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0) return ORACLE_EINVAL;
+  const size_t SZ = (size_t)dk * dv;
+  memset(dq, 0, sizeof(double) * (size_t)B * T * H * dk);
+  memset(dkk, 0, sizeof(double) * (size_t)B * T * H * dk);
+  if (!gates_given) {
+    memset(dA_log, 0, sizeof(double) * (size_t)H * dk);
+    memset(ddt_bias, 0, sizeof(double) * (size_t)H * dk);
+  }
+  double* Sp = (double*)malloc(sizeof(double) * SZ * ((size_t)T + 1));
+  double* Sb = (double*)malloc(sizeof(double) * SZ);
+  double* dS = (double*)malloc(sizeof(double) * SZ);
+  double* wk = (double*)malloc(sizeof(double) * (size_t)(9 * dk + 7 * dv));
+  if (!Sp || !Sb || !dS || !wk) {
+    free(Sp); free(Sb); free(dS); free(wk);
+    return ORACLE_ENOMEM;
+  }
+  double *qt = wk, *kt = qt + dk, *gq = kt + dk, *gk = gq + dk, *dec = gk + dk, *gd = dec + dk;
+  double *bg = gd + dk, *et = bg + dk, *de = et + dk;
+  double *vt = de + dk, *wg = vt + dv, *zt = wg + dv, *rt = zt + dv, *ot = rt + dv, *m = ot + dv;
+  double* drr = m + dv;
+  for (int bi = 0; bi < B; ++bi)
+    for (int h = 0; h < H; ++h) {
+      const size_t bh = (size_t)bi * H + h;
+      for (size_t x = 0; x < SZ; ++x) Sp[x] = h0 ? h0[bh * SZ + x] : 0.0;
+      /* forward with the states kept: the same arithmetic as oracle_gdn2_fwd */
+      for (int pass = 0; pass < 2; ++pass) {
+        if (pass == 1)
+          for (size_t x = 0; x < SZ; ++x) dS[x] = dht ? dht[bh * SZ + x] : 0.0;
+        for (int tt = 0; tt < T; ++tt) {
+          const int t = pass == 0 ? tt : T - 1 - tt;
+          const size_t row = ((size_t)bi * T + t) * H + h;
+          load_vec(q, 1, row * dk, dk, l2norm, scale, qt);
+          load_vec(k, 1, row * dk, dk, l2norm, 1.0, kt);
+          load_vec(v, 1, row * dv, dv, 0, 1.0, vt);
+          for (int i = 0; i < dk; ++i) {
+            double gi;
+            if (gates_given) {
+              gi = a[row * dk + i];
+              bg[i] = b_logit[row * dk + i];
+            } else {
+              gi = -exp(A_log[(size_t)h * dk + i]) *
+                   softplus(a[row * dk + i] + dt_bias[(size_t)h * dk + i]);
+              bg[i] = sigmoid(b_logit[row * dk + i]);
+            }
+            gd[i] = gi;
+            dec[i] = exp(gi);
+            et[i] = bg[i] * kt[i];
+          }
+          for (int j = 0; j < dv; ++j) {
+            wg[j] = gates_given ? w_logit[row * dv + j] : sigmoid(w_logit[row * dv + j]);
+            zt[j] = wg[j] * vt[j];
+          }
+          const double* S0 = Sp + (size_t)t * SZ;
+          double* S1 = Sp + (size_t)(t + 1) * SZ;
+          for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j) Sb[(size_t)i * dv + j] = dec[i] * S0[(size_t)i * dv + j];
+          for (int j = 0; j < dv; ++j) rt[j] = 0.0;
+          for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j) rt[j] += Sb[(size_t)i * dv + j] * et[i];
+          if (pass == 0) {
+            for (int i = 0; i < dk; ++i)
+              for (int j = 0; j < dv; ++j)
+                S1[(size_t)i * dv + j] = Sb[(size_t)i * dv + j] + kt[i] * (zt[j] - rt[j]);
+            continue;
+          }
+          /* backward of the token */
+          const double* dO = dout + row * dv;
+          for (int i = 0; i < dk; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dv; ++j) {
+              acc += S1[(size_t)i * dv + j] * dO[j];
+              dS[(size_t)i * dv + j] += qt[i] * dO[j];
+            }
+            gq[i] = acc;
+          }
+          for (int j = 0; j < dv; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < dk; ++i) acc += dS[(size_t)i * dv + j] * kt[i];
+            m[j] = acc;
+            drr[j] = -acc;
+          }
+          for (int i = 0; i < dk; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dv; ++j) acc += dS[(size_t)i * dv + j] * (zt[j] - rt[j]);
+            gk[i] = acc;
+          }
+          for (int i = 0; i < dk; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dv; ++j) {
+              dS[(size_t)i * dv + j] += et[i] * drr[j];      /* dS_bar */
+              acc += Sb[(size_t)i * dv + j] * drr[j];
+            }
+            de[i] = acc;
+          }
+          for (int j = 0; j < dv; ++j) {
+            dvv[row * dv + j] = m[j] * wg[j];
+            const double dwj = m[j] * vt[j];
+            dw[row * dv + j] = gates_given ? dwj : dwj * wg[j] * (1.0 - wg[j]);
+          }
+          for (int i = 0; i < dk; ++i) {
+            const double dbi = de[i] * kt[i];
+            gk[i] += de[i] * bg[i];
+            db[row * dk + i] = gates_given ? dbi : dbi * bg[i] * (1.0 - bg[i]);
+            double ddi = 0.0;
+            for (int j = 0; j < dv; ++j) {
+              ddi += dS[(size_t)i * dv + j] * S0[(size_t)i * dv + j];
+              dS[(size_t)i * dv + j] *= dec[i];
+            }
+            const double dgi = ddi * dec[i];
+            if (gates_given) {
+              da[row * dk + i] = dgi;
+            } else {
+              const double xg = a[row * dk + i] + dt_bias[(size_t)h * dk + i];
+              const double dx = dgi * (-exp(A_log[(size_t)h * dk + i])) * sigmoid(xg);
+              da[row * dk + i] = dx;
+              ddt_bias[(size_t)h * dk + i] += dx;
+              dA_log[(size_t)h * dk + i] += dgi * gd[i];
+            }
+          }
+          load_vec_bwd(q + row * dk, dk, l2norm, scale, gq, dq + row * dk);
+          load_vec_bwd(k + row * dk, dk, l2norm, 1.0, gk, dkk + row * dk);
+        }
+      }
+      if (dh0) memcpy(dh0 + bh * SZ, dS, sizeof(double) * SZ);
+    }
+  free(Sp); free(Sb); free(dS); free(wk);
+  return ORACLE_OK;
+}
+
+/*
  * KDA (Kimi Delta Attention) as the "Gated DeltaNet-2" page states its update
  * (section 标量绑定的数学表达), computed literally:
  *   S_t = (I - beta_t k_t k_t^T) D_t S_{t-1} + beta_t k_t v_t^T ;  o_t = S_t^T q_t

@@ -16,8 +16,9 @@ Each function cites the passage it follows (page title and section):
   (Linear -> CausalConv1D -> SiLU -> q, k, v).
 * ``conv_step`` / ``conv_prefill`` -- that conv alone, for one token or a whole
   prefill ("gated-deltanet-qwen3.5" section 因果卷积: kernel 4, depthwise, causal).
-* ``gdn_bwd``      -- the backward of ``gdn_fwd`` (the survey's last next row):
-  reverse-mode through the same five steps, pinned by finite differences.
+* ``gdn_bwd`` / ``gdn2_bwd`` -- the backward of ``gdn_fwd`` / ``gdn2_fwd`` (the
+  survey's last next row; "Gated DeltaNet-2", Gate-aware 反向传播 for the second):
+  reverse-mode through the same steps, pinned by finite differences.
 * ``kda_fwd``      -- "Gated DeltaNet-2" (zhichai), section 标量绑定的数学表达 (the
   KDA update with its erase projection written out) and 退化兼容性.
 * ``rmsnorm_gated`` -- "gated-deltanet-qwen3.5" section 输出门控与 RMSNorm
@@ -73,9 +74,10 @@ def _load():
             lib.oracle_rmsnorm_gated.argtypes = [vp, vp, vp, ip, ip, ip, dp, vp]
             lib.oracle_kda_fwd.argtypes = [vp] * 8 + [ip] * 6 + [dp, ip, vp, vp, ip]
             lib.oracle_gdn_bwd.argtypes = [vp] * 10 + [ip] * 6 + [dp, ip, ip] + [vp] * 8
+            lib.oracle_gdn2_bwd.argtypes = [vp] * 11 + [ip] * 5 + [dp, ip, ip] + [vp] * 9
             for f in (lib.oracle_gdn_fwd, lib.oracle_gate_prep, lib.oracle_conv_step,
                       lib.oracle_conv_prefill, lib.oracle_rmsnorm_gated, lib.oracle_kda_fwd,
-                      lib.oracle_gdn_bwd,
+                      lib.oracle_gdn_bwd, lib.oracle_gdn2_bwd,
                       lib.oracle_gdn_decode_step, lib.oracle_gdn2_fwd):
                 f.restype = ctypes.c_int
             lib.oracle_max_threads.restype = ctypes.c_int
@@ -234,6 +236,33 @@ def gdn_bwd(q, k, v, a, b, A_log, dt_bias, h0, do, dht=None, *, scale=None, l2no
                                 *[_ptr(out[n]) for n in ("dq", "dk", "dv", "da", "db", "dA_log",
                                                          "ddt_bias", "dh0")])
     _check(rc, "oracle_gdn_bwd")
+    return out
+
+
+def gdn2_bwd(q, k, v, a, b_logit, w_logit, A_log, dt_bias, h0, do, dht=None, *, scale=None,
+             l2norm=True, gates_given=False):
+    """Gradients of sum(o * do) + sum(ht * dht) for gdn2_fwd's (o, ht) (float64).
+
+    Returns a dict with dq, dk, dv, da, db, dw, dA_log, ddt_bias, dh0 (with
+    gates_given: da, db, dw with respect to g, b, w; dA_log / ddt_bias None).
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    f = lambda x: None if x is None else _arr(x, True)
+    arrs = [f(x) for x in (q, k, v, a, b_logit, w_logit, A_log, dt_bias, h0, do, dht)]
+    if scale is None:
+        scale = dk ** -0.5
+    out = {"dq": np.zeros((B, T, H, dk)), "dk": np.zeros((B, T, H, dk)),
+           "dv": np.zeros((B, T, H, dv)), "da": np.zeros((B, T, H, dk)),
+           "db": np.zeros((B, T, H, dk)), "dw": np.zeros((B, T, H, dv)),
+           "dA_log": None if gates_given else np.zeros((H, dk)),
+           "ddt_bias": None if gates_given else np.zeros((H, dk)),
+           "dh0": np.zeros((B, H, dk, dv))}
+    rc = _load().oracle_gdn2_bwd(*[_ptr(x) for x in arrs], B, T, H, dk, dv, float(scale),
+                                 int(l2norm), int(gates_given),
+                                 *[_ptr(out[n]) for n in ("dq", "dk", "dv", "da", "db", "dw",
+                                                          "dA_log", "ddt_bias", "dh0")])
+    _check(rc, "oracle_gdn2_bwd")
     return out
 
 

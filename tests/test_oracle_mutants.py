@@ -62,6 +62,12 @@ MUTANTS = [
     ("bwd_norm_projection_dropped",
      "  for (int i = 0; i < n; ++i) gx[i] += scale * (gy[i] / nrm - x[i] * xg / (nrm * nrm * nrm));",
      "  for (int i = 0; i < n; ++i) gx[i] += scale * (gy[i] / nrm);"),
+    ("bwd2_erase_read_dropped",  # dS_bar misses e dr^T
+     "              dS[(size_t)i * dv + j] += et[i] * drr[j];      /* dS_bar */",
+     "              dS[(size_t)i * dv + j] += 0.0 * drr[j];      /* dS_bar */"),
+    ("bwd2_decay_missing", "              dS[(size_t)i * dv + j] *= dec[i];",
+     "              dS[(size_t)i * dv + j] *= 1.0;"),
+    ("bwd2_erase_gate_path_dropped", "            gk[i] += de[i] * bg[i];", "            gk[i] += 0.0;"),
     ("kda_decay_dropped",  # the projection applied to S instead of D S
      "        for (int j = 0; j < dv; ++j) DS[(size_t)i * dv + j] = dec[i] * S[(size_t)i * dv + j];",
      "        for (int j = 0; j < dv; ++j) DS[(size_t)i * dv + j] = S[(size_t)i * dv + j];"),
@@ -107,7 +113,7 @@ def _run_pins_against(lib_path):
     mutant = ctypes.CDLL(lib_path)
     for fname in ("oracle_gdn_fwd", "oracle_gate_prep", "oracle_conv_step",
                   "oracle_conv_prefill", "oracle_rmsnorm_gated", "oracle_kda_fwd",
-                  "oracle_gdn_bwd",
+                  "oracle_gdn_bwd", "oracle_gdn2_bwd",
                   "oracle_gdn_decode_step",
                   "oracle_gdn2_fwd"):
         getattr(mutant, fname).argtypes = getattr(real, fname).argtypes

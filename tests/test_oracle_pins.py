@@ -274,6 +274,47 @@ def test_gdn_backward_matches_finite_differences(l2norm, gates_given):
         assert abs(fd - an) <= 1e-7 * max(1.0, abs(fd)), (n, fd, an)
 
 
+@pytest.mark.parametrize("l2norm,gates_given", [(True, False), (False, True)])
+def test_gdn2_backward_matches_finite_differences(l2norm, gates_given):
+    """The Gated DeltaNet-2 backward (per-channel gates kept inside the
+    accumulations, "Gated DeltaNet-2" Gate-aware 反向传播) against central finite
+    differences along a random direction of every input."""
+    B, T, H, dk, dv = 2, 4, 2, 4, 3
+    q, k, v = _rand(B, T, H, dk), _rand(B, T, H, dk), _rand(B, T, H, dv)
+    if gates_given:
+        a = -rng.uniform(0.05, 1.0, size=(B, T, H, dk))
+        b = rng.uniform(0.1, 0.9, size=(B, T, H, dk))
+        w = rng.uniform(0.1, 0.9, size=(B, T, H, dv))
+        A_log = dt_bias = None
+    else:
+        a, b, w = _rand(B, T, H, dk), _rand(B, T, H, dk), _rand(B, T, H, dv)
+        A_log = rng.uniform(0, math.log(16), size=(H, dk))
+        dt_bias = rng.uniform(-4, -1, size=(H, dk))
+    h0 = 0.3 * _rand(B, H, dk, dv)
+    Ro, Rh = _rand(B, T, H, dv), _rand(B, H, dk, dv)
+    kw = dict(scale=0.7, l2norm=l2norm, gates_given=gates_given)
+    inputs = dict(q=q, k=k, v=v, a=a, b=b, w=w, A_log=A_log, dt_bias=dt_bias, h0=h0)
+
+    def loss(x):
+        o, ht = O.gdn2_fwd(x["q"], x["k"], x["v"], x["a"], x["b"], x["w"], x["A_log"],
+                           x["dt_bias"], x["h0"], **kw)
+        return float(np.sum(o * Ro) + np.sum(ht * Rh))
+
+    g = O.gdn2_bwd(q, k, v, a, b, w, A_log, dt_bias, h0, Ro, Rh, **kw)
+    names = dict(q="dq", k="dk", v="dv", a="da", b="db", w="dw", A_log="dA_log",
+                 dt_bias="ddt_bias", h0="dh0")
+    h = 1e-5
+    for n, x0 in inputs.items():
+        if x0 is None:
+            continue
+        u = _rand(*x0.shape)
+        xp, xm = dict(inputs), dict(inputs)
+        xp[n], xm[n] = x0 + h * u, x0 - h * u
+        fd = (loss(xp) - loss(xm)) / (2 * h)
+        an = float(np.sum(g[names[n]] * u))
+        assert abs(fd - an) <= 1e-7 * max(1.0, abs(fd)), (n, fd, an)
+
+
 # --------------------------------------------------------------------------
 # Gates and normalisation: closed forms
 # --------------------------------------------------------------------------
