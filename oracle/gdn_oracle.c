@@ -23,7 +23,9 @@
  *    and updates conv_states and recurrent_states.
  *  - "Gated DeltaNet-2" (zhichai), section "新更新公式": S_bar = D S,
  *    r = S_bar^T e, S = S_bar + k (z - r)^T with e = b (.) k, z = w (.) v;
- *    section "标量绑定的数学表达": the KDA update (I - beta k k^T) D S + beta k v^T.
+ *    section "标量绑定的数学表达": the KDA update (I - beta k k^T) D S + beta k v^T;
+ *    section "Gate-aware 反向传播": gradients with the channel gates inside the
+ *    accumulations.
  *  - "gated-deltanet-qwen3.5" (wanger-sjtu), section "输出门控与 RMSNorm":
  *    RMSNormGated(core_attn_out, z).
  *
@@ -47,7 +49,8 @@
  * decay closed form, matrix-form recurrence, GDN-2 -> GDN reduction, KDA ->
  * GDN-2 (tied gates) and -> GDN (scalar decay), gate and norm closed forms, the
  * conv step and the prefill conv against a library convolution, the gated
- * RMSNorm against a library rms_norm and its closed forms.
+ * RMSNorm against a library rms_norm and its closed forms, the GDN and GDN-2
+ * backward against central finite differences.
  */
 #include <math.h>
 #include <stddef.h>
