@@ -193,6 +193,88 @@ def chunk_gdn_bwd(q, k, v, g, beta, S0, dO, dST, C):
     return dq, dk_, dv_, dg, dbeta, dS
 
 
+def chunk_gdn2_bwd(q, k, v, g, b, w, S0, dO, dST, C):
+    """Backward of the channel-decay chunk form, written with the direct masked
+    contractions L_rj = sum_c E_rc K_jc Gamma_rjc (j < r) and
+    A_qk_rj = sum_c Q_rc K_jc Gamma_rjc (j <= r), Gamma_rjc = exp(G_rc - G_jc) (the
+    blocked form of the forward is the same numbers).  Per chunk, with
+    E-bar = gamma (.) E, Y = A E-bar, U = A Z, U~ = U - Y S0,
+    O = (gamma (.) Q) S0 + A_qk U~ and S1 = diag(gamma_C) S0 + K~^T U~,
+    dA = dU Z^T + dY E-bar^T ("Gated DeltaNet-2", Gate-aware 反向传播), then
+    dL = -A^T dA A^T (strictly lower), the masked contractions, the Gamma tensor and
+    the per-channel reverse cumulative sum for dg."""
+    T, dk = q.shape
+    starts, S = [], S0.copy()
+    for c0 in range(0, T, C):
+        starts.append(S.copy())
+        _, S = chunk_gdn2(q[c0:c0 + C], k[c0:c0 + C], v[c0:c0 + C], g[c0:c0 + C],
+                          b[c0:c0 + C], w[c0:c0 + C], S, C)
+    dq, dk_, dv_ = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dg, db, dw = np.zeros_like(g), np.zeros_like(b), np.zeros_like(w)
+    dS = dST.copy()
+    for ci in reversed(range(len(starts))):
+        c0 = ci * C
+        c1 = min(c0 + C, T)
+        n = c1 - c0
+        Kc, Qc, Vc, S = k[c0:c1], q[c0:c1], v[c0:c1], starts[ci]
+        bc, wc = b[c0:c1], w[c0:c1]
+        G = np.cumsum(g[c0:c1], axis=0)
+        gam = np.exp(G)
+        gC = gam[-1]
+        low = np.tril(np.ones((n, n)))
+        Gam = np.exp(np.where(low[:, :, None] > 0, G[:, None, :] - G[None, :, :], -np.inf))
+        E, Z = bc * Kc, wc * Vc
+        L = np.tril(np.einsum("rc,jc,rjc->rj", E, Kc, Gam), -1)
+        Aqk = np.tril(np.einsum("rc,jc,rjc->rj", Qc, Kc, Gam))
+        A = forward_substitution_inverse(L)
+        Eb = gam * E
+        Y, U = A @ Eb, A @ Z
+        Ut = U - Y @ S
+        ratio = gC[None, :] / gam
+        Kt = ratio * Kc
+        # S1 = diag(gamma_C) S0 + K~^T U~
+        dS0 = gC[:, None] * dS
+        dgC = np.sum(dS * S, axis=1)
+        dKt, dUt = Ut @ dS.T, Kt @ dS
+        # O = (gamma (.) Q) S0 + A_qk U~
+        dOc = dO[c0:c1]
+        dQg = dOc @ S.T
+        dQ = gam * dQg
+        dgam = Qc * dQg
+        dS0 += (gam * Qc).T @ dOc
+        dAqk = np.tril(dOc @ Ut.T)
+        dUt += Aqk.T @ dOc
+        # U~ = U - Y S0 ; U = A Z ; Y = A E-bar
+        dU, dY = dUt, -dUt @ S.T
+        dS0 -= Y.T @ dUt
+        dA = dU @ Z.T + dY @ Eb.T
+        dZ, dEb = A.T @ dU, A.T @ dY
+        dV = wc * dZ
+        dwc = Vc * dZ
+        dE = gam * dEb
+        dgam += E * dEb
+        dL = np.tril(-A.T @ dA @ A.T, -1)
+        # the masked contractions
+        dE += np.einsum("rj,jc,rjc->rc", dL, Kc, Gam)
+        dK = np.einsum("rj,rc,rjc->jc", dL, E, Gam) + np.einsum("rj,rc,rjc->jc", dAqk, Qc, Gam)
+        dQ += np.einsum("rj,jc,rjc->rc", dAqk, Kc, Gam)
+        tG = (np.einsum("rj,rc,jc->rjc", dL, E, Kc) + np.einsum("rj,rc,jc->rjc", dAqk, Qc, Kc)) * Gam
+        dG = tG.sum(1) - tG.sum(0)
+        # E = b (.) K
+        dbc = Kc * dE
+        dK += bc * dE
+        # K~ = (gamma_C / gamma) (.) K
+        dK += ratio * dKt
+        dratio = Kc * dKt
+        dG -= dratio * ratio
+        dG[-1] += np.sum(dratio * ratio, axis=0) + dgC * gC
+        dG += dgam * gam
+        dg[c0:c1] = np.cumsum(dG[::-1], axis=0)[::-1]
+        dq[c0:c1], dk_[c0:c1], dv_[c0:c1], db[c0:c1], dw[c0:c1] = dQ, dK, dV, dbc, dwc
+        dS = dS0
+    return dq, dk_, dv_, dg, db, dw, dS
+
+
 def _gates(T, H, A_log, dt_bias, a, b):
     sp = np.log1p(np.exp(a + dt_bias))
     return -np.exp(A_log) * sp, 1 / (1 + np.exp(-b))
@@ -273,3 +355,27 @@ def test_chunk_gdn_backward_equals_token_backward(T, C):
                       (dv_, ref["dv"][0, :, 0]), (dg, ref["da"][0, :, 0]),
                       (dbeta, ref["db"][0, :, 0]), (dS0, ref["dh0"][0, 0])):
         np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-10)
+
+
+@pytest.mark.parametrize("T", [1, 30, 64, 100])
+@pytest.mark.parametrize("C", [16, 64])
+def test_chunk_gdn2_backward_equals_token_backward(T, C):
+    """The channel-decay chunkwise backward against the oracle's token-by-token
+    Gated DeltaNet-2 backward (pinned by finite differences)."""
+    dk, dv = 16, 8
+    q, k, v = rng.standard_normal((T, dk)), rng.standard_normal((T, dk)), rng.standard_normal((T, dv))
+    q /= np.linalg.norm(q, axis=1, keepdims=True) * 4.0
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    g = -rng.uniform(0.0, 1.0, size=(T, dk))
+    b = rng.uniform(0.0, 1.0, size=(T, dk))
+    w = rng.uniform(0.0, 1.0, size=(T, dv))
+    S0 = 0.1 * rng.standard_normal((dk, dv))
+    dO, dST = rng.standard_normal((T, dv)), rng.standard_normal((dk, dv))
+    ref = O.gdn2_bwd(q[None, :, None], k[None, :, None], v[None, :, None], g[None, :, None],
+                     b[None, :, None], w[None, :, None], None, None, S0[None, None],
+                     dO[None, :, None], dST[None, None], scale=1.0, l2norm=False,
+                     gates_given=True)
+    got = chunk_gdn2_bwd(q, k, v, g, b, w, S0, dO, dST, C)
+    for x, name in zip(got, ("dq", "dk", "dv", "da", "db", "dw")):
+        np.testing.assert_allclose(x, ref[name][0, :, 0], rtol=1e-9, atol=1e-10)
+    np.testing.assert_allclose(got[6], ref["dh0"][0, 0], rtol=1e-9, atol=1e-10)
