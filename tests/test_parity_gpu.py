@@ -1,7 +1,6 @@
 """GPU parity: every entry point of libgdn.so, called through the C ABI, against
 the fp64 oracle on the same seeded inputs (max|err|/RMS per tensor, 1e-4 for
 float32 inputs, 2e-2 for bf16)."""
-import math
 
 import numpy as np
 import pytest

@@ -2,7 +2,6 @@
 ("gated-deltanet-qwen3.5" section 输出门控与 RMSNorm: RMSNormGated(core_attn_out,
 z)), called through the C ABI and compared with the fp64 oracle on the same
 seeded inputs (max|err|/RMS: 1e-4 for float32, 2e-2 for bf16)."""
-import numpy as np
 import pytest
 import torch
 
