@@ -2,16 +2,20 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Headline (`value`): GDN chunkwise prefill tokens/s on the Qwen3.5-shaped layer
-(B=1, T=8192, 16 key heads, 64 value heads, d=128, bf16 inputs, fp32 state);
-one step = one gdn_chunk_fwd call over that batch: two kernels, a chunk-parallel
-WY prep (gates, L2 norm, K K^T / Q K^T, (I+L)^-1, W, U, A_qk) and the scan over
-chunks (U - W S, output rows, state update).  The decode step
-(256 sequences, fused conv1d, state GB/s), the long-context prefill and the
-Gated DeltaNet-2 forward are measured in the same run and reported under
-"extra".  Multi-GPU runs are independent replicas (every (batch, head) scan is
-independent; no collective on the data path): weak scaling, time = max over
-ranks.  `--impl reference` times the fp64 CPU oracle on the host cores instead.
+Headline (`value`): GDN chunkwise prefill tokens/s on the long-context
+Qwen3.5-shaped layer (B=1, T=131072, 16 key heads, 64 value heads, d=128, bf16
+inputs, fp32 state), the largest configuration that runs on one GPU; one step =
+one gdn_chunk_fwd call over that batch: two kernels, a chunk-parallel WY prep
+(gates, L2 norm, K K^T / Q K^T, (I+L)^-1, W, U, A_qk) and the scan over chunks
+(U - W S, output rows, state update).  `e2e` is the same workload through the
+host entry point (gdn_chunk_fwd_host) with page-locked host inputs and outputs,
+every copy inside the timed region.  The 8K-token prefill, the batched 8 x 16K
+prefill, the decode step (256 sequences, fused conv1d, state GB/s), the Gated
+DeltaNet-2 and KDA forwards, the prefill conv and the gated RMSNorm are measured
+in the same run and reported under "extra".  Multi-GPU runs are independent
+replicas (every (batch, head) scan is independent; no collective on the data
+path): weak scaling, time = max over ranks.  `--impl reference` times the fp64
+CPU oracle on the host cores instead.
 """
 from __future__ import annotations
 
@@ -34,8 +38,12 @@ import torch.distributed as dist  # noqa: E402
 
 from gdn_synth import WORKLOADS, kda_inputs, workload_inputs  # noqa: E402
 
-CHUNK_FLOP_PER_TOKEN_HEAD = 180_224  # dense GEMM FLOPs of the chunk form at C=64, d=128
-HEADLINE = "prefill_8k"
+# dense GEMM FLOPs of the chunk form at C=64, d=128 per token and value head
+# (10 C d + 6 d^2); with the K K^T / Q K^T Gram formed once per key head and shared
+# by a GQA group of G = 4 value heads, the work the kernels need is 155,648
+CHUNK_FLOP_PER_TOKEN_HEAD = 180_224
+CHUNK_FLOP_PER_TOKEN_HEAD_GQA4 = 155_648
+HEADLINE = "prefill_128k"
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -189,6 +197,25 @@ def time_steps(fn, steps, warmup, stream, flush=None, sync_group=False):
     return start.elapsed_time(end), per
 
 
+def prefill_roofline(w, launch_ms, pk, profile):
+    """Roofline of one gdn_chunk_fwd call on workload w: the dense GEMM FLOPs of
+    the chunk form (and, beside them, the GQA-shared count) over the call's mean
+    CUDA-event time, against the measured bf16 burst peak."""
+    flop = CHUNK_FLOP_PER_TOKEN_HEAD * w.T * w.Hv * w.B
+    flop_gqa = CHUNK_FLOP_PER_TOKEN_HEAD_GQA4 * w.T * w.Hv * w.B
+    achieved = flop / (launch_ms / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 2),
+            "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(achieved / pk["bf16_tflops"], 4),
+            "traffic": kernel_traffic(profile),
+            "kernel": "gdn_chunk_fwd = wy_prep_tc_kernel + state_scan_tc_kernel (timed together)",
+            "flop_per_launch": flop,
+            "frac_gqa_shared_count": round(flop_gqa / (launch_ms / 1e3) / 1e12
+                                           / pk["bf16_tflops"], 4),
+            "flop_per_launch_gqa_shared": flop_gqa,
+            "peak_src": pk["src"] + " burst bf16"}
+
+
 def run_ours(args, rank, local_rank, world):
     import gated_deltanet_sequence_gdn_b200 as G
 
@@ -216,26 +243,27 @@ def run_ours(args, rank, local_rank, world):
     ms_step = max_over_ranks(total_ms, dev) / args.steps
     tokens = w.B * w.T
     value = job_rate(tokens, world, ms_step)
-    flop = CHUNK_FLOP_PER_TOKEN_HEAD * w.T * w.Hv * w.B
     launch_ms = sum(per) / len(per)
-    achieved = flop / (launch_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "achieved": round(achieved, 2),
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / pk["bf16_tflops"], 4),
-                "traffic": kernel_traffic("chunk_prefill_8k"),
-                "kernel": "gdn_chunk_fwd = wy_prep_tc_kernel + state_scan_tc_kernel (timed together)",
-                "flop_per_launch": flop, "peak_src": pk["src"] + " burst bf16"}
+    roofline = prefill_roofline(w, launch_ms, pk, "chunk_prefill_128k")
+    del ws, o, ht
+    torch.cuda.empty_cache()
 
     # ---- end to end through the public call, host buffers, copies inside the timed region
     e2e = measure_e2e(G, x, w, dev, stream, args, world)
+    x_cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        x_cpu = {n: (t.cpu() if t is not None else None) for n, t in x.items()}
+    del x
+    torch.cuda.empty_cache()
 
     extra = {}
     if not args.headline_only:
+        extra["prefill_8k"] = measure_prefill(G, "prefill_8k", dev, stream, pk, args)
+        extra["prefill_b8_16k"] = measure_prefill(G, "prefill_b8_16k", dev, stream, pk, args)
         extra["decode_256"] = measure_decode(G, dev, stream, pk, args)
         extra["gdn2_b4_4k"] = measure_gdn2(G, dev, stream, pk, args)
         extra["conv_prefill_8k"] = measure_conv(G, dev, stream, pk, args)
-        extra["prefill_128k"] = measure_prefill(G, "prefill_128k", dev, stream, pk, args)
-        extra["prefill_b8_16k"] = measure_prefill(G, "prefill_b8_16k", dev, stream, pk, args)
+        extra["gate_prep_8k"] = measure_gate_prep(G, dev, stream, pk, args)
         # the newest secondary figures, last: a failure is reported here, not raised
         for name, fn in (("kda_b4_4k", measure_kda), ("rmsnorm_gated_8k", measure_norm)):
             try:
@@ -252,12 +280,12 @@ def run_ours(args, rank, local_rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": HEADLINE, "B": w.B, "T": w.T, "Hk": w.Hk, "Hv": w.Hv,
                    "d": w.d, "chunk": 64, "state": "fp32", "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (q,k,v,o ~340 MB per step > 126 MB)"},
+                   "l2": "inputs larger than L2 (q,k,v,o ~5.4 GB per step > 126 MB)"},
         "roofline": roofline, "e2e": e2e, "clocks": clk, "gpu_launches": launches,
         "extra": extra,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, x)
+    if x_cpu is not None:
+        line["cpu_baseline"] = cpu_baseline(w, x_cpu)
     return line
 
 
@@ -282,7 +310,7 @@ def measure_e2e(G, x, w, dev, stream, args, world):
     def step():
         G.gdn_chunk_fwd_host(host["q"], host["k"], host["v"], host["a"], host["b"],
                              host["A_log"], host["dt_bias"], host["h0"], o=o_h, ht=ht_h,
-                             dev_workspace=dws, stream=stream)
+                             dev_workspace=dws, stream=stream, sync=False)
 
     steps = max(3, min(args.steps, 20))
     total_ms, _ = time_steps(step, steps, 2, stream, sync_group=world > 1)
@@ -305,15 +333,15 @@ def measure_prefill(G, name, dev, stream, pk, args):
         G.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
                         x["h0"], o=o, ht=ht, workspace=ws, stream=stream)
 
-    total, per = time_steps(step, 3, 1, stream)
-    ms = total / 3
-    flop = CHUNK_FLOP_PER_TOKEN_HEAD * w.T * w.Hv * w.B
-    ach = flop / (ms / 1e3) / 1e12
+    steps = 10 if w.T * w.B <= 16384 else 5
+    total, per = time_steps(step, steps, 3, stream)
+    ms = sum(per) / len(per)
+    rl = prefill_roofline(w, ms, pk, "chunk_" + name)
     del x, o, ht, ws
     torch.cuda.empty_cache()
     return {"tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
-            "B": w.B, "T": w.T, "achieved_tflops": round(ach, 2),
-            "frac_of_bf16_peak": round(ach / pk["bf16_tflops"], 4)}
+            "B": w.B, "T": w.T, "achieved_tflops": rl["achieved"],
+            "frac_of_bf16_peak": rl["frac"], "roofline": rl, "steps": steps}
 
 
 def measure_decode(G, dev, stream, pk, args):
@@ -405,6 +433,38 @@ def measure_conv(G, dev, stream, pk, args):
             "steps": steps}
 
 
+def measure_gate_prep(G, dev, stream, pk, args):
+    """gdn_gate_prep over the prefill_8k layer (q, k [1, 8192, 16, 128] bf16 and the
+    gate inputs of 64 value heads): HBM-bound.  Algorithmic bytes per launch: q, k
+    read and q_hat, k_hat written once (bf16), a, b read (bf16), g, beta written
+    (float32), A_log / dt_bias read."""
+    w = WORKLOADS["prefill_8k"]
+    x = workload_inputs(w, dev)
+    qo, ko = torch.empty_like(x["q"]), torch.empty_like(x["k"])
+    g = torch.empty((w.B, w.T, w.Hv), device=dev, dtype=torch.float32)
+    beta = torch.empty_like(g)
+
+    def step():
+        G.gdn_gate_prep(x["q"], x["k"], x["a"], x["b"], x["A_log"], x["dt_bias"], q_out=qo,
+                        k_out=ko, g_out=g, beta_out=beta, stream=stream)
+
+    steps = 20
+    total, per = time_steps(step, steps, 3, stream)
+    ms = sum(per) / len(per)
+    es = 2
+    nbytes = (2 * 2 * w.B * w.T * w.Hk * w.d * es + 2 * w.B * w.T * w.Hv * es
+              + 2 * w.B * w.T * w.Hv * 4 + 2 * w.Hv * 4)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del x, qo, ko, g, beta
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_launch": round(ms, 5),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": kernel_traffic("gate_prep_8k")},
+            "steps": steps}
+
+
 def measure_kda(G, dev, stream, pk, args):
     """gdn_kda_chunk_fwd at the Gated DeltaNet-2 bench shape (B=4, T=4096, 16 heads,
     d=128, bf16): the gate tiling plus the Gated DeltaNet-2 kernels."""
@@ -472,6 +532,8 @@ def run_only(args, local_rank):
         r = measure_norm(G, dev, stream, pk, args)
     elif args.only == "kda_b4_4k":
         r = measure_kda(G, dev, stream, pk, args)
+    elif args.only == "gate_prep_8k":
+        r = measure_gate_prep(G, dev, stream, pk, args)
     else:
         r = measure_prefill(G, args.only, dev, stream, pk, args)
     G.gdn_check_status(stream)
@@ -549,7 +611,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["prefill_8k", "decode_256", "gdn2_b4_4k", "prefill_128k",
                                        "prefill_b8_16k", "conv_prefill_8k", "rmsnorm_gated_8k",
-                                       "kda_b4_4k"],
+                                       "kda_b4_4k", "gate_prep_8k"],
                     default=None,
                     help="measure one secondary workload alone (profiling runs)")
     args = ap.parse_args()

@@ -21,7 +21,8 @@ __all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_chunk_workspace_bytes", "gdn_r
            "gdn_conv_prefill", "gdn_rmsnorm_gated", "gdn_kda_chunk_fwd",
            "gdn_kda_chunk_workspace_bytes", "gdn_chunk_fwd_varlen",
            "gdn2_chunk_fwd", "gdn2_chunk_workspace_bytes", "gdn_chunk_fwd_noalloc",
-           "gdn_check_status", "GDNError", "LIB_PATH", "lib", "F32", "BF16",
+           "gdn_check_status", "gdn_status", "gdn_test_set_wait_fault", "GDNError",
+           "LIB_PATH", "lib", "F32", "BF16",
            "QK_L2NORM", "GATES_PRECOMPUTED", "OUT_F32"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -62,6 +63,8 @@ lib.gdn2_chunk_workspace_bytes.argtypes = [_i] * 6
 lib.gdn_chunk_workspace_bytes.restype = _sz
 lib.gdn2_chunk_workspace_bytes.restype = _sz
 lib.gdn_check_status.argtypes = [_vp]
+lib.gdn_test_set_wait_fault.argtypes = [_i, ctypes.c_uint]
+lib.gdn_test_set_wait_fault.restype = _i
 lib.gdn_status_string.argtypes = [_i]
 lib.gdn_status_string.restype = ctypes.c_char_p
 lib.gdn_version.argtypes = []
@@ -233,14 +236,17 @@ def gdn_chunk_fwd_host_workspace_bytes(B, T, Hk, Hv, dk, dv, dtype, *, l2norm=Tr
 def gdn_chunk_fwd_host(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, scale=None,
                        l2norm=True, gates_precomputed=False, out_f32=False, o=None, ht=None,
                        want_ht=True, piece_tokens=0, dev_workspace=None, device=None,
-                       stream=None):
+                       stream=None, sync=True):
     """gdn_chunk_fwd for host (CPU) tensors: the library copies the sequence to the
     device piece by piece, overlapping the copies in, the compute and the copies
     out.  Arguments as gdn_chunk_fwd, all CPU tensors (pin_memory() for
     asynchronous copies); o / ht are CPU tensors (page-locked when allocated
     here).  dev_workspace: a uint8 CUDA tensor of at least
     gdn_chunk_fwd_host_workspace_bytes(...) bytes, allocated here when None.
-    Returns (o, ht) once the stream has completed."""
+    Returns (o, ht); with sync=True (the default) once the stream has completed, so
+    that they hold the results; with sync=False as soon as the work is enqueued (the
+    host buffers are written asynchronously until the stream completes, and a
+    dev_workspace allocated here must not be reused before then)."""
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     dt = q.dtype
@@ -270,6 +276,8 @@ def gdn_chunk_fwd_host(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, scal
                                   _ph(dt_bias), _ph(h0), B, T, Hk, Hv, dk, dv, _dtype_code(dt),
                                   float(scale), flags, _ph(o), _ph(ht), int(piece_tokens),
                                   _p(dev_workspace), ws_bytes, st), "gdn_chunk_fwd_host")
+    if sync:
+        (stream if stream is not None else torch.cuda.current_stream()).synchronize()
     return o, ht
 
 
@@ -469,5 +477,19 @@ def gdn_rmsnorm_gated(o, z, weight, *, eps=1e-6, y=None, stream=None):
 
 
 def gdn_check_status(stream=None):
-    """Synchronise the stream and raise if a bounded device wait expired."""
+    """Synchronise the stream and raise if a bounded device wait expired or an
+    fp16 operand left its range since the last check."""
     _check(lib.gdn_check_status(_stream(stream)), "gdn_check_status")
+
+
+def gdn_status(stream=None) -> int:
+    """Synchronise the stream, read and clear the device status word: the raw
+    gdn_check_status code (0 = GDN_OK, -4 = GDN_ERR_TIMEOUT, -6 = GDN_ERR_RANGE)."""
+    return int(lib.gdn_check_status(_stream(stream)))
+
+
+def gdn_test_set_wait_fault(site: int, spin_limit: int = 0):
+    """Test hook: make the tensor-core chunk kernels leave one bounded wait to
+    expire (site 1: the scan's first state hand-off, site 2: the prep's K / Q
+    tiles; 0: none), with spin_limit polls per wait (0 = the default)."""
+    _check(lib.gdn_test_set_wait_fault(int(site), int(spin_limit)), "gdn_test_set_wait_fault")

@@ -2,6 +2,9 @@
 // host-side argument validation, dispatch to the kernels, status reporting.
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -34,9 +37,13 @@ __global__ void copy_or_zero_kernel(const float* __restrict__ src, float* dst, s
 }  // namespace
 
 int* status_word() {
+  // one lookup per device; calls from several host threads may race to fill a slot,
+  // which the lock serialises
+  static std::mutex mu;
   static int* addr[64] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_gdn_status) != cudaSuccess) return nullptr;
@@ -44,6 +51,13 @@ int* status_word() {
   }
   return addr[dev];
 }
+
+namespace {
+std::atomic<int> g_fault_site{kFaultNone};
+std::atomic<unsigned> g_fault_spin{kWaitSpin};
+}  // namespace
+
+WaitFault wait_fault() { return WaitFault{g_fault_site.load(), g_fault_spin.load()}; }
 
 cudaError_t launch_copy_state(const float* h0, float* ht, size_t n, cudaStream_t s) {
   if (n == 0 || ht == nullptr || h0 == ht) return cudaSuccess;
@@ -313,8 +327,16 @@ int gdn_check_status(gdn_stream_t stream) {
   if (h != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_gdn_status, &zero, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
-    return (h & kStatusRange) ? GDN_ERR_RANGE : GDN_ERR_TIMEOUT;
+    // an expired wait is reported first: the outputs after it are not computed at all
+    return (h & ~kStatusRange) ? GDN_ERR_TIMEOUT : GDN_ERR_RANGE;
   }
+  return GDN_OK;
+}
+
+int gdn_test_set_wait_fault(int site, unsigned spin_limit) {
+  if (site < kFaultNone || site > kFaultPrepTiles) return GDN_ERR_INVALID_ARG;
+  g_fault_site.store(site);
+  g_fault_spin.store(spin_limit == 0 ? kWaitSpin : spin_limit);
   return GDN_OK;
 }
 

@@ -43,13 +43,17 @@ bool make_plan(int B, int T, int Hk, int Hv, int dk, int dv, int dtype, int flag
   const size_t es = dtype == GDN_F32 ? 4 : 2;
   const size_t ges = (flags & GDN_GATES_PRECOMPUTED) ? 4 : es;
   const size_t oes = (flags & GDN_OUT_F32) ? 4 : es;
-  int Tc = piece_tokens;
-  if (Tc <= 0) Tc = (T + 7) / 8;  // about eight pieces by default
+  // piece length in whole chunks, rounded in 64-bit arithmetic (a piece_tokens near
+  // INT_MAX must not wrap) and never longer than the sequence rounded up to a chunk
+  long long Tc = piece_tokens;
+  if (Tc <= 0) Tc = ((long long)T + 7) / 8;  // about eight pieces by default
+  const long long Tmax = (((long long)T + kC - 1) / kC) * kC;
+  if (Tmax > 0x7fffffc0LL) return false;
+  if (Tc > Tmax) Tc = Tmax;
   Tc = ((Tc + kC - 1) / kC) * kC;  // whole chunks
   if (Tc < kC) Tc = kC;
-  if (Tc > T) Tc = ((T + kC - 1) / kC) * kC;
-  p->Tc = Tc;
-  p->pieces = (T + Tc - 1) / Tc;
+  p->Tc = (int)Tc;
+  p->pieces = (int)(((long long)T + Tc - 1) / Tc);
   p->row_q = (size_t)Hk * dk * es;
   p->row_k = p->row_q;
   p->row_v = (size_t)Hv * dv * es;
@@ -60,11 +64,11 @@ bool make_plan(int B, int T, int Hk, int Hv, int dk, int dv, int dtype, int flag
   for (int s = 0; s < 2; ++s)
     for (int j = 0; j < 5; ++j) {
       p->in_off[s][j] = off;
-      off += up256((size_t)B * Tc * rows[j]);
+      off += up256((size_t)B * p->Tc * rows[j]);
     }
   for (int s = 0; s < 2; ++s) {
     p->o_off[s] = off;
-    off += up256((size_t)B * Tc * p->row_o);
+    off += up256((size_t)B * p->Tc * p->row_o);
   }
   p->state_off = off;
   off += up256((size_t)B * Hv * dk * dv * 4);
@@ -73,7 +77,7 @@ bool make_plan(int B, int T, int Hk, int Hv, int dk, int dv, int dtype, int flag
   p->dtb_off = off;
   off += up256((size_t)Hv * 4);
   p->ws_off = off;
-  p->ws_bytes = gdn_chunk_workspace_bytes(B, Tc, Hk, Hv, dk, dv, dtype);
+  p->ws_bytes = gdn_chunk_workspace_bytes(B, p->Tc, Hk, Hv, dk, dv, dtype);
   off += up256(p->ws_bytes);
   p->total = off;
   return true;

@@ -59,6 +59,17 @@ cudaError_t launch_scan_tc(const ChunkArgs& a, const void* workspace, int* statu
 // Device address of this device's status word (set up once per device).
 int* status_word();
 
+// Test hook behind gdn_test_set_wait_fault: a site at which one kernel leaves a
+// bounded wait to expire on purpose, and the poll limit of every bounded wait of
+// the tensor-core chunk kernels (kWaitSpin unless a test lowered it).
+constexpr unsigned kWaitSpin = 1u << 24;
+enum WaitFaultSite { kFaultNone = 0, kFaultScanState = 1, kFaultPrepTiles = 2 };
+struct WaitFault {
+  int site;
+  unsigned spin;
+};
+WaitFault wait_fault();
+
 cudaError_t launch_copy_state(const float* h0, float* ht, size_t n, cudaStream_t s);
 
 }  // namespace gdn

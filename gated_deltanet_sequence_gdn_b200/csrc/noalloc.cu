@@ -4,6 +4,8 @@
 // reserved only when this entry point is first used on a device.
 #include <stdint.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -16,9 +18,12 @@ static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 // Device address of this device's copy of the array (looked up once per device).
 void* static_scratch() {
+  // host threads calling at once on a fresh device would race to fill the slot
+  static std::mutex mu;
   static void* addr[64] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;

@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kPT, 2)
 wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict__ ga,
                   const void* __restrict__ gb, const float* __restrict__ A_log,
                   const float* __restrict__ dt_bias, int T, int Hk, int Hv, float scale, int l2,
-                  uint8_t* __restrict__ ws, WsLayout L, int* status) {
+                  uint8_t* __restrict__ ws, WsLayout L, int* status, int fault, uint32_t spin) {
   extern __shared__ __align__(1024) uint8_t sm_raw[];
   uint8_t* sm = sm_raw + ((1024u - (tc::smem_u32(sm_raw) & 1023u)) & 1023u);
   const uint32_t sb = tc::smem_u32(sm);
@@ -124,6 +124,9 @@ wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict_
   // thread 0's record of the copies and MMAs in flight (for the exit after an
   // expired wait)
   uint32_t v_issued[2] = {0, 0}, v_done[2] = {0, 0}, mma_issued = 0, mma_done = 0;
+  // (a test of the bounded waits withholds the K / Q tiles: every thread's first wait
+  // then expires and the CTA leaves through the drain below)
+  const bool kq_issued = fault != kFaultPrepTiles;
   bool kq_done = false;
 
   auto issue_v = [&](int h) {  // V tile of value head h into slot h % 2 (thread 0)
@@ -142,11 +145,13 @@ wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict_
     tc::prefetch_tmap(&maps.v);
     for (int i = 0; i < 4; ++i) tc::mbar_init(&bar[i], 1);
     tc::fence_mbar_init();
-    tc::mbar_arrive_expect_tx(&bar[0], 32768);
+    if (kq_issued) {
+      tc::mbar_arrive_expect_tx(&bar[0], 32768);
 #pragma unroll
-    for (int dh = 0; dh < 2; ++dh) {
-      tc::tma_load_4d(sm + S_KQ + dh * 16384, &maps.k, &bar[0], 64 * dh, hk, t0, b);
-      tc::tma_load_4d(sm + S_KQ + dh * 16384 + 8192, &maps.q, &bar[0], 64 * dh, hk, t0, b);
+      for (int dh = 0; dh < 2; ++dh) {
+        tc::tma_load_4d(sm + S_KQ + dh * 16384, &maps.k, &bar[0], 64 * dh, hk, t0, b);
+        tc::tma_load_4d(sm + S_KQ + dh * 16384 + 8192, &maps.q, &bar[0], 64 * dh, hk, t0, b);
+      }
     }
     issue_v(0);
     if (G > 1) issue_v(1);
@@ -162,7 +167,7 @@ wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict_
   // let the copies and MMAs in flight finish, free the tensor memory.
   auto drain_and_leave = [&]() {
     if (tid == 0) {
-      if (!kq_done) tc::mbar_wait(&bar[0], 0, nullptr, 0, 1u << 20);
+      if (kq_issued && !kq_done) tc::mbar_wait(&bar[0], 0, nullptr, 0, 1u << 20);
       for (int s = 0; s < 2; ++s)
         if (v_issued[s] > v_done[s]) tc::mbar_wait(&bar[1 + s], v_done[s] & 1, nullptr, 0, 1u << 20);
       if (mma_issued > mma_done) tc::mbar_wait(&bar[3], mma_done & 1, nullptr, 0, 1u << 20);
@@ -220,7 +225,7 @@ wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict_
 
   // 1. gates of the first heads while the tiles land
   gates_partial(0);
-  bool ok = tc::mbar_wait(&bar[0], 0, status, 121);
+  bool ok = tc::mbar_wait(&bar[0], 0, status, 121, spin);
   if (__syncthreads_or(!ok)) {
     drain_and_leave();
     return;
@@ -297,7 +302,7 @@ wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict_
     }
     tc::bulk_commit();
   }
-  ok = tc::mbar_wait(&bar[3], 0, status, 122);
+  ok = tc::mbar_wait(&bar[3], 0, status, 122, spin);
   if (__syncthreads_or(!ok)) {
     drain_and_leave();
     return;
@@ -377,7 +382,7 @@ wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict_
     invert_in_place(LX, Tm, tid, warp, g8, t4);
     bool vok = true;
     if (tid == 0) {
-      vok = tc::mbar_wait(&bar[1 + (h & 1)], (h >> 1) & 1, status, 123);
+      vok = tc::mbar_wait(&bar[1 + (h & 1)], (h >> 1) & 1, status, 123, spin);
       if (vok) ++v_done[h & 1];
       tc::bulk_wait_read_all();  // the staged A_qk tile is read (the lo operand goes there)
     }
@@ -429,7 +434,7 @@ wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict_
       tc::mma_commit(&bar[3]);
       ++mma_issued;
     }
-    ok = tc::mbar_wait(&bar[3], (uint32_t)(h + 1) & 1u, status, 124);
+    ok = tc::mbar_wait(&bar[3], (uint32_t)(h + 1) & 1u, status, 124, spin);
     if (__syncthreads_or(!ok)) {
       drain_and_leave();
       return;
@@ -517,8 +522,10 @@ cudaError_t launch_prep_tc(const ChunkArgs& a, void* ws, int* status, cudaStream
   auto prep = pre ? wy_prep_tc_kernel<true> : wy_prep_tc_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PT_SMEM);
   if (e != cudaSuccess) return e;
+  const WaitFault f = wait_fault();
   prep<<<dim3(Nc, a.B * a.Hk), kPT, PT_SMEM, s>>>(m, a.a, a.b, a.A_log, a.dt_bias, a.T, a.Hk,
-                                                  a.Hv, a.scale, l2, w, L, status);
+                                                  a.Hv, a.scale, l2, w, L, status, f.site,
+                                                  f.spin);
   return cudaGetLastError();
 }
 

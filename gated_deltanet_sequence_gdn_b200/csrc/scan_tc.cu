@@ -84,8 +84,9 @@ __device__ __forceinline__ void store_half_row_f16(uint8_t* tile, int r, int c0,
 
 // Bounded wait that also gives up as soon as another role of the CTA has given up.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status,
-                                              int where, volatile int* abort_flag) {
-  for (uint32_t i = 0; i < (1u << 24); ++i) {
+                                              int where, volatile int* abort_flag,
+                                              uint32_t spin) {
+  for (uint32_t i = 0; i < spin; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 255u && *abort_flag) return false;
   }
@@ -128,7 +129,7 @@ template <typename TO>
 __global__ void __launch_bounds__(kScanTcThreads, 1)
 state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __restrict__ ws,
                      WsLayout L, const float* h0, int T, int Hk, int Hv, TO* __restrict__ o,
-                     float* ht, int* status) {
+                     float* ht, int* status, int fault, uint32_t spin) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -163,10 +164,11 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      int issued = 0;  // stages armed so far
       for (int n = 0; n < Nc; ++n) {
         const int s = n & 1;
-        if (n >= 2 &&
-            !wait_or_abort(&bar[B_EMPTY0 + s], ((n >> 1) - 1) & 1, status, 101, abort_flag)) {
+        if (n >= 2 && !wait_or_abort(&bar[B_EMPTY0 + s], ((n >> 1) - 1) & 1, status, 101,
+                                     abort_flag, spin)) {
           *abort_flag = 1;
           break;
         }
@@ -185,9 +187,12 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
         tma_load_2d(st + ST_U + 0, &maps.u, full, c0, rw);
         tma_load_2d(st + ST_U + 8192, &maps.u, full, c0 + 32, rw);
         bulk_load(st + ST_SC, Sg + (size_t)n * kScal, kScal * 4, full);
+        issued = n + 1;
       }
-      // drain: every stage armed must have landed before the CTA may exit
-      for (int n = (Nc >= 2 ? Nc - 2 : 0); n < Nc; ++n)
+      // drain: every stage armed must have landed before the CTA may exit.  Stage n
+      // was armed only after stage n - 2 of the same slot had been consumed, so only
+      // the last two armed stages can still be in flight.
+      for (int n = (issued >= 2 ? issued - 2 : 0); n < issued; ++n)
         mbar_wait(&bar[B_FULL0 + (n & 1)], (n >> 1) & 1, nullptr, 0, 1u << 20);
     }
   } else if (warp == 1) {
@@ -200,8 +205,8 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       for (int n = 0; n < Nc; ++n) {
         const int s = n & 1;
         const uint32_t st = sbase + s * STAGE_BYTES;
-        if (!wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 102, abort_flag) ||
-            !wait_or_abort(&bar[B_S], n & 1, status, 103, abort_flag)) {
+        if (!wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 102, abort_flag, spin) ||
+            !wait_or_abort(&bar[B_S], n & 1, status, 103, abort_flag, spin)) {
           *abort_flag = 1;
           break;
         }
@@ -214,7 +219,7 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
         }
         mma_commit(&bar[B_QP]);
         ++qp_phases;
-        if (!wait_or_abort(&bar[B_UT], n & 1, status, 104, abort_flag)) {
+        if (!wait_or_abort(&bar[B_UT], n & 1, status, 104, abort_flag, spin)) {
           *abort_flag = 1;
           break;
         }
@@ -274,7 +279,9 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
     store_half_row_f16(sm + OFF_SB, row, 4 * half, S);
     fence_proxy_async_smem();
     named_barrier(1, kEpi);
-    if (e == 0) mbar_arrive(&bar[B_S]);
+    // (a test of the bounded waits withholds this first arrival: the MMA issue's
+    // wait for the state then expires and the CTA leaves through the abort path)
+    if (e == 0 && fault != kFaultScanState) mbar_arrive(&bar[B_S]);
 
     float OQ[32];
     for (int n = 0; n < Nc; ++n) {
@@ -282,8 +289,9 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       const uint8_t* st = sm + s * STAGE_BYTES;
       const float* sc = reinterpret_cast<const float*>(st + ST_SC);
       {  // every epilogue thread takes the same decision (no thread is left at a barrier)
-        const bool ok = wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 105, abort_flag) &&
-                        wait_or_abort(&bar[B_QP], n & 1, status, 106, abort_flag);
+        const bool ok =
+            wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 105, abort_flag, spin) &&
+            wait_or_abort(&bar[B_QP], n & 1, status, 106, abort_flag, spin) && !*abort_flag;
         if (named_barrier_or(1, kEpi, !ok)) {
           *abort_flag = 1;
           break;
@@ -335,7 +343,7 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
 
       // the state update first: it is what the next chunk waits for
       {
-        const bool ok = wait_or_abort(&bar[B_DS], n & 1, status, 107, abort_flag);
+        const bool ok = wait_or_abort(&bar[B_DS], n & 1, status, 107, abort_flag, spin);
         if (named_barrier_or(1, kEpi, !ok)) {
           *abort_flag = 1;
           break;
@@ -363,7 +371,7 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
 
       // then the output rows (lanes 0-63), overlapping the next chunk's products
       if (!p_rows) {
-        if (!wait_or_abort(&bar[B_OA], n & 1, status, 108, abort_flag)) continue;
+        if (!wait_or_abort(&bar[B_OA], n & 1, status, 108, abort_flag, spin)) continue;
         tc_fence_after();
         float OA[32];
         tmem_ld32(tl + TM_OA, OA);
@@ -412,8 +420,9 @@ cudaError_t launch_t(const ChunkArgs& a, const WsLayout& L, const uint8_t* ws, i
   cudaError_t e = cudaFuncSetAttribute(state_scan_tc_kernel<TO>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_TC_SMEM);
   if (e != cudaSuccess) return e;
+  const WaitFault f = wait_fault();
   state_scan_tc_kernel<TO><<<dim3(2, a.B * a.Hv), kScanTcThreads, SCAN_TC_SMEM, s>>>(
-      m, ws, L, a.h0, a.T, a.Hk, a.Hv, static_cast<TO*>(a.o), a.ht, status);
+      m, ws, L, a.h0, a.T, a.Hk, a.Hv, static_cast<TO*>(a.o), a.ht, status, f.site, f.spin);
   return cudaGetLastError();
 }
 

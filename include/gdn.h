@@ -7,6 +7,11 @@
  *    (allocated by any means: cudaMalloc, a PyTorch tensor, a pool).  The
  *    library never allocates, frees or synchronises; each call only enqueues
  *    kernels on `stream` and returns.  NULL stream = the legacy default stream.
+ *    Exceptions, each stated at its entry point: gdn_check_status synchronises
+ *    the stream by design; gdn_chunk_fwd_host takes HOST pointers, creates two
+ *    copy streams per device on its first call (kept until the process exits),
+ *    synchronises the stream when T = 0, and its copies to or from pageable
+ *    (not page-locked) host memory are synchronous.
  *  - Layouts are dense, row-major, token-major, with no padding:
  *      q, k        [B, T, Hk, dk]
  *      v, o        [B, T, Hv, dv]
@@ -183,6 +188,9 @@ int gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
  *   enqueued still completes on the stream), GDN_ERR_CUDA if a stream or event
  *   of the pipeline could not be made.  T = 0 copies h0 to ht (or zeros) after
  *   synchronising the stream.
+ *   Resources: the two copy streams of a device are created on its first call
+ *   and live until the process exits (they are reused by every later call);
+ *   the call itself allocates no memory.
  */
 int gdn_chunk_fwd_host(const void* q, const void* k, const void* v, const void* a,
                        const void* b, const float* A_log, const float* dt_bias,
@@ -351,13 +359,31 @@ size_t gdn2_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype
 
 /*
  * gdn_check_status -- waits for `stream`, then reads and clears the device
- * status word of the current device.  Returns GDN_OK, GDN_ERR_RANGE if an
- * intermediate of the tensor-core chunk path left the fp16 operand range since
- * the last check (inputs far outside the method's domain, e.g. keys of norm
- * >> 1 with GDN_QK_L2NORM off), GDN_ERR_TIMEOUT if a bounded wait in a kernel
- * expired, or GDN_ERR_CUDA.
+ * status word of the current device.  Returns GDN_OK, GDN_ERR_TIMEOUT if a
+ * bounded wait in a kernel expired since the last check (reported first when
+ * both happened), GDN_ERR_RANGE if an intermediate of the tensor-core chunk
+ * path left the fp16 operand range (inputs far outside the method's domain,
+ * e.g. keys of norm >> 1 with GDN_QK_L2NORM off, or values of magnitude
+ * ~1e6), or GDN_ERR_CUDA.  The word is shared by every call on the device, so a
+ * code belongs to some call since the previous check.
  */
 int gdn_check_status(gdn_stream_t stream);
+
+/*
+ * gdn_test_set_wait_fault -- test hook for the bounded device waits; the pages
+ * have no counterpart.  It makes the next tensor-core chunk calls leave one wait
+ * to expire on purpose, without anything left in flight on the GPU, so that a
+ * test can check that the kernel returns and gdn_check_status reports
+ * GDN_ERR_TIMEOUT:
+ *   site 0: no fault (the default);
+ *   site 1: the state scan withholds the first state hand-off to its MMA issue;
+ *   site 2: the WY prep withholds its K / Q tile loads.
+ *   spin_limit: polls before a wait gives up, for every bounded wait of those
+ *   kernels (0 = the default, 2^24).  The setting is process-wide and stays
+ *   until changed; the outputs of a faulted call are not valid.
+ * Returns GDN_OK, or GDN_ERR_INVALID_ARG for an unknown site.
+ */
+int gdn_test_set_wait_fault(int site, unsigned spin_limit);
 
 /* Human-readable name of a gdn_status value (static string). */
 const char* gdn_status_string(int status);

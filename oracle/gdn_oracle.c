@@ -29,7 +29,7 @@
  *  - "gated-deltanet-qwen3.5" (wanger-sjtu), section "输出门控与 RMSNorm":
  *    RMSNormGated(core_attn_out, z).
  *
- * Readings where the pages are silent (each also listed in the design notes):
+ * Readings where the pages are silent (this file's choices, stated here):
  *  - L2 normalisation of q and k is x / sqrt(sum x^2 + 1e-6); q is then scaled
  *    by `scale` (1/sqrt(d_k) by default).
  *  - Grouped heads: value head hv reads key/query head hv / (Hv/Hk).

@@ -17,8 +17,8 @@ Each function cites the passage it follows (page title and section):
 * ``conv_step`` / ``conv_prefill`` -- that conv alone, for one token or a whole
   prefill ("gated-deltanet-qwen3.5" section 因果卷积: kernel 4, depthwise, causal).
 * ``gdn_bwd`` / ``gdn2_bwd`` -- the backward of ``gdn_fwd`` / ``gdn2_fwd`` (the
-  survey's last next row; "Gated DeltaNet-2", Gate-aware 反向传播 for the second):
-  reverse-mode through the same steps, pinned by finite differences.
+  training direction of the method; "Gated DeltaNet-2", Gate-aware 反向传播 for the
+  second): reverse-mode through the same steps, pinned by finite differences.
 * ``kda_fwd``      -- "Gated DeltaNet-2" (zhichai), section 标量绑定的数学表达 (the
   KDA update with its erase projection written out) and 退化兼容性.
 * ``rmsnorm_gated`` -- "gated-deltanet-qwen3.5" section 输出门控与 RMSNorm

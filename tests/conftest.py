@@ -29,6 +29,31 @@ def pytest_collection_modifyitems(session, config, items):
     items.sort(key=lambda it: os.path.basename(str(it.fspath)) in _RUN_LAST)  # stable
 
 
+try:
+    import pytest
+    import torch
+    _CUDA = torch.cuda.is_available()
+except Exception:  # noqa: BLE001
+    _CUDA = False
+
+if _CUDA:
+    @pytest.fixture(autouse=True)
+    def _device_status_clean(request):
+        """Every GPU test starts and ends with a clean device status word: a set
+        GDN_ERR_RANGE or GDN_ERR_TIMEOUT bit left by any call of the test (the word is
+        sticky) fails the test that caused it.  Tests that provoke one on purpose
+        read it themselves, which clears it."""
+        if request.node.get_closest_marker("gpu") is None:
+            yield
+            return
+        import gated_deltanet_sequence_gdn_b200 as G
+        before = G.gdn_status()
+        assert before == 0, f"device status {before} left by an earlier test"
+        yield
+        after = G.gdn_status()
+        assert after == 0, f"device status {after} after the test (-4 timeout, -6 range)"
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size parity case (minutes)")

@@ -1,16 +1,28 @@
 """Shared helpers of the GPU parity tests: the error metric and tolerances.
 
-Metric (per output tensor): max |gpu - oracle| / RMS(oracle); bars 1e-4 for
-float32 inputs and 2e-2 for bf16 inputs (float32 accumulation and state).
+Metric (per output tensor), the one the bar is stated in: max |gpu - oracle| /
+RMS(oracle), with bars 1e-4 for float32 inputs and 2e-2 for bf16 inputs (float32
+accumulation and state), applied raw, with no allowance.
 
-Outputs stored in bf16 carry, on top of the computation's own error, the
-rounding of the final store: |rn(o) - o| <= u |o| with u = 2^-8 (bf16 keeps
-8 significant bits).  Since |o_bf16 - ref| <= |o - ref| + u (|ref| + |o - ref|),
-the error of the computation before that store is at least
-(|o_bf16 - ref| - u |ref|) / (1 + u) per element; that is the per-element
-error the bar is applied to for bf16 outputs.  Outputs written in float32
-(GDN_OUT_F32) get no allowance.  conv_state is a byte copy and is compared bit
-for bit.
+Where the bar is applied.  A bf16 store of an output rounds each element by up to
+2^-8 of its magnitude, so on outputs whose largest element is ~5-10 RMS the exact
+fp64 result, rounded to bf16, already scores 0.02-0.04 on this metric
+(tests/test_oracle_pins.py::test_bf16_store_alone_reaches_the_bar pins two such
+cases).  The bar therefore measures the computation, not the storage format: the
+chunk, decode, Gated DeltaNet-2, KDA and packed-batch parity tests read the
+float32 output of the same kernels (GDN_OUT_F32) and apply the bar to it raw,
+and separate tests check bit for bit that the bf16 output of a call is the
+round-to-nearest of that float32 output (`assert_bf16_store`), i.e. the bf16
+store adds its own rounding and nothing else.
+
+The standalone elementwise kernels with bf16 outputs only (the prefill conv, the
+gated RMSNorm, the gate prep's q / k) are held per element to one final rounding
+of the exact value: |y - ref| <= (2^-8 + 2^-16) |ref| + 2^-20 RMS(ref)
+(`rounding_ratio` <= 1), the bf16 half-ulp bound plus a margin for their float32
+arithmetic.  float32 outputs everywhere get the raw 1e-4 bar.
+
+`rel_err_store` is a diagnostic only, printed in some failure messages and never
+asserted: the error left after removing the bf16 store's own rounding.
 """
 import numpy as np
 import torch
@@ -19,21 +31,64 @@ TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
 U_BF16 = 2.0 ** -8
 
 
-def rel_err(x, ref) -> float:
-    bf16_out = hasattr(x, "dtype") and x.dtype == torch.bfloat16
+def _arrays(x, ref):
     if hasattr(x, "detach"):
         x = x.detach().float().cpu().double().numpy()
     x = np.asarray(x, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert x.shape == ref.shape, (x.shape, ref.shape)
     assert np.all(np.isfinite(x)), "non-finite values in the GPU result"
+    return x, ref
+
+
+def _ratio(err, ref) -> float:
+    if not err.size:
+        return 0.0
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    if rms == 0.0:
+        return float(np.max(err))
+    return float(np.max(err) / rms)
+
+
+def rel_err(x, ref) -> float:
+    """max |x - ref| / RMS(ref) over the whole tensor."""
+    x, ref = _arrays(x, ref)
+    return _ratio(np.abs(x - ref), ref)
+
+
+def rel_err_store(x, ref) -> float:
+    """Diagnostic: the error left after the bf16 store's own rounding allowance."""
+    bf16_out = hasattr(x, "dtype") and x.dtype == torch.bfloat16
+    x, ref = _arrays(x, ref)
     err = np.abs(x - ref)
     if bf16_out:
         err = np.maximum(err - U_BF16 * np.abs(ref), 0.0) / (1.0 + U_BF16)
+    return _ratio(err, ref)
+
+
+def rounding_ratio(y, ref) -> float:
+    """max over elements of |y - ref| / ((2^-8 + 2^-16) |ref| + 2^-20 RMS(ref)):
+    <= 1 when y is one bf16 rounding of ref up to float32 arithmetic error."""
+    y, ref = _arrays(y, ref)
+    if not y.size:
+        return 0.0
     rms = float(np.sqrt(np.mean(ref * ref)))
-    if rms == 0.0:
-        return float(np.max(err)) if err.size else 0.0
-    return float(np.max(err) / rms) if err.size else 0.0
+    bound = (U_BF16 + 2.0 ** -16) * np.abs(ref) + 2.0 ** -20 * rms
+    err = np.abs(y - ref)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.where(bound > 0, err / np.where(bound > 0, bound, 1.0), np.where(err > 0, np.inf, 0.0))
+    return float(np.max(r))
+
+
+def assert_bf16_store(o_bf16, o_f32):
+    """The bf16 output of a call equals, bit for bit, the round-to-nearest of the
+    float32 output of the same call with GDN_OUT_F32."""
+    assert o_bf16.dtype == torch.bfloat16 and o_f32.dtype == torch.float32
+    assert o_bf16.shape == o_f32.shape
+    want = o_f32.to(torch.bfloat16)
+    same = o_bf16.view(torch.int16) == want.view(torch.int16)
+    n_bad = int((~same).sum().item())
+    assert n_bad == 0, f"{n_bad} of {same.numel()} bf16 outputs differ from rn(float32 output)"
 
 
 def cpu(t):

@@ -10,7 +10,7 @@ import torch
 
 from gdn_synth import WORKLOADS, conv_prefill_inputs, gdn_inputs, workload_inputs
 from oracle import oracle as O
-from tests.parity import TOL, cpu, rel_err
+from tests.parity import cpu, rel_err, rounding_ratio
 
 pytestmark = pytest.mark.gpu
 
@@ -46,8 +46,11 @@ def test_conv_prefill_small(T, d, dtype, use_state):
     q, k, v = G.gdn_conv_prefill(x["x"], x["conv_w"], cs, Hk=Hk, Hv=Hv, dk=d, dv=d)
     y, r_cs = _oracle(x, use_state)
     rq, rk, rv = _split(y, Hk, Hv, d)
-    tol = TOL[dtype]
-    assert rel_err(q, rq) <= tol and rel_err(k, rk) <= tol and rel_err(v, rv) <= tol
+    if dtype == torch.bfloat16:  # one bf16 rounding of the exact conv + SiLU
+        assert rounding_ratio(q, rq) <= 1 and rounding_ratio(k, rk) <= 1
+        assert rounding_ratio(v, rv) <= 1
+    else:
+        assert rel_err(q, rq) <= 1e-4 and rel_err(k, rk) <= 1e-4 and rel_err(v, rv) <= 1e-4
     if use_state:
         np.testing.assert_array_equal(cpu(cs).double().numpy(), r_cs)
 
@@ -81,7 +84,7 @@ def test_conv_prefill_feeds_the_chunk_path():
     cs = x["conv_state"].clone()
     q, k, v = G.gdn_conv_prefill(x["x"], x["conv_w"], cs, Hk=Hk, Hv=Hv, dk=d, dv=d)
     o, ht = G.gdn_chunk_fwd(q, k, v, gates["a"], gates["b"], gates["A_log"], gates["dt_bias"],
-                            gates["h0"])
+                            gates["h0"], out_f32=True)
     y, _ = _oracle(x, True)
     y = torch.from_numpy(y).bfloat16().double().numpy()
     rq, rk, rv = _split(y, Hk, Hv, d)
@@ -119,7 +122,7 @@ def test_conv_prefill_full_size_sampled_tokens():
         ref.append(O.conv_step(xt, wcv, win)[0])
         got.append(torch.cat([qc[t].reshape(-1), kc[t].reshape(-1), vc[t].reshape(-1)]))
     got, ref = torch.stack(got), np.stack(ref)
-    assert rel_err(got, ref) <= 2e-2
-    assert rel_err(got[:, :QK], ref[:, :QK]) <= 2e-2
+    assert rounding_ratio(got, ref) <= 1
+    assert rounding_ratio(got[:, :QK], ref[:, :QK]) <= 1
     last = np.stack([row(w.T - 3), row(w.T - 2), row(w.T - 1)], 1)
     np.testing.assert_array_equal(cpu(cs)[0].double().numpy(), last)

@@ -544,3 +544,24 @@ def test_float32_inputs_match_float64_inputs():
     o64, h64 = O.gdn_fwd(*(x.astype(np.float64) for x in (q, k, v, a, b, A_log, dt_bias)))
     np.testing.assert_array_equal(o32, o64)
     np.testing.assert_array_equal(h32, h64)
+
+
+def test_bf16_store_alone_reaches_the_bar():
+    """Why the GPU parity bar is applied to float32 outputs: the exact fp64 result of
+    two small bf16 cases (a chunk prefill, T = 200 with grouped heads, and a prefill
+    conv), rounded to bf16 and nothing else, already scores about 0.02 on
+    max|err| / RMS(ref), the bar itself, because their largest elements are ~10 RMS
+    and a bf16 store rounds by up to 2^-8 of an element's magnitude."""
+    import torch
+    from gdn_synth import conv_prefill_inputs, gdn_inputs
+    x = gdn_inputs(1, 200, 2, 4, 128, torch.bfloat16, seed=7, device="cpu")
+    ro, _ = O.gdn_fwd(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"], x["h0"])
+    r16 = torch.from_numpy(ro).to(torch.bfloat16).double().numpy()
+    rms = np.sqrt(np.mean(ro ** 2))
+    assert np.abs(r16 - ro).max() / rms > 0.018
+    assert np.abs(r16 - ro).max() <= 2.0 ** -8 * np.abs(ro).max() * (1 + 1e-12)
+    x = conv_prefill_inputs(2, 17, 2, 4, 64, torch.bfloat16, seed=57, device="cpu")
+    cs = x["conv_state"].double().numpy().copy()
+    y = O.conv_prefill(x["x"], x["conv_w"], cs)
+    y16 = torch.from_numpy(y).to(torch.bfloat16).double().numpy()
+    assert np.abs(y16 - y).max() / np.sqrt(np.mean(y ** 2)) > 0.02

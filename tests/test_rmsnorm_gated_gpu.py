@@ -7,7 +7,7 @@ import torch
 
 from gdn_synth import WORKLOADS, rmsnorm_inputs, workload_inputs
 from oracle import oracle as O
-from tests.parity import TOL, cpu, rel_err
+from tests.parity import cpu, rel_err, rounding_ratio
 
 pytestmark = pytest.mark.gpu
 
@@ -15,6 +15,15 @@ if torch.cuda.is_available():
     import gated_deltanet_sequence_gdn_b200 as G
 
 DEV = "cuda"
+
+
+def _check(y, ref, dtype):
+    """float32: the raw 1e-4 bar; bf16 (the only output type): one final bf16
+    rounding of the exact value per element (tests/parity.py)."""
+    if dtype == torch.bfloat16:
+        assert rounding_ratio(y, ref) <= 1, rounding_ratio(y, ref)
+    else:
+        assert rel_err(y, ref) <= 1e-4, rel_err(y, ref)
 
 
 def _oracle(x, eps=1e-6):
@@ -29,7 +38,7 @@ def test_rmsnorm_gated_small(shape, dv, dtype):
     B, T, H = shape
     x = rmsnorm_inputs(B, T, H, dv, dtype, seed=60 + T, device=DEV)
     y = G.gdn_rmsnorm_gated(x["o"], x["z"], x["weight"])
-    assert rel_err(y, _oracle(x)) <= TOL[dtype]
+    _check(y, _oracle(x), dtype)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
@@ -40,7 +49,7 @@ def test_rmsnorm_gated_in_place_and_eps(dtype):
     ref = _oracle(x, eps=0.25)
     o = x["o"].clone()
     G.gdn_rmsnorm_gated(o, x["z"], x["weight"], eps=0.25, y=o)
-    assert rel_err(o, ref) <= TOL[dtype]
+    _check(o, ref, dtype)
     assert bool((o[0, 3] == 0).all())
 
 
@@ -49,4 +58,4 @@ def test_rmsnorm_gated_full_size():
     w = WORKLOADS["rmsnorm_gated_8k"]
     x = workload_inputs(w, DEV)
     y = G.gdn_rmsnorm_gated(x["o"], x["z"], x["weight"])
-    assert rel_err(y, _oracle(x)) <= 2e-2
+    _check(y, _oracle(x), torch.bfloat16)

@@ -30,7 +30,6 @@ def _lib():
     lib.probe_tmem_roundtrip.argtypes = [vp, vp]
     lib.probe_tma_load.argtypes = [vp, i, i, i, i, i, i, i, vp, vp]
     lib.probe_mma.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, vp]
-    lib.probe_skeleton.argtypes = [vp, vp, vp, vp, vp, vp, i, i, vp]
     return lib
 
 
@@ -128,125 +127,3 @@ def test_mma_layouts(lib, M, N, a_mn, b_mn, dcol):
     assert st.item() == 0
     ref = A.float() @ B.float()
     torch.testing.assert_close(D, ref, rtol=1e-5, atol=1e-4)
-
-
-def _swz(tile):
-    """bf16 [R][64] -> the 128-byte-swizzled byte image the kernels use
-    (16-byte chunk c of row r stored at chunk position c ^ (r % 8))."""
-    t = tile.contiguous().view(torch.int16).cpu().numpy().reshape(-1, 8, 8)
-    R = t.shape[0]
-    out = t.copy()
-    for r in range(R):
-        for p in range(8):
-            out[r, p] = t[r, p ^ (r % 8)]
-    return torch.from_numpy(out.reshape(-1)).view(torch.uint8)
-
-
-@pytest.mark.parametrize("tma_T,mode", [(0, 0), (1, 0), (64, 0), (1, 1), (1, 8), (1, 4), (1, 2),
-                                        (1, 15), (0, 16), (1, 31), (0, 32), (1, 32), (1, 63)])
-def test_mma_tmem_choreography(lib, tma_T, mode):
-    """Four commit/wait rounds on one barrier with interleaved MMAs of different
-    shapes, tile stores while the tensor cores run, at the chunk kernel's
-    shared-memory offsets (grid of two CTAs, 150 KB of shared memory).  With
-    tma_T > 0 the K, Q and V tiles are TMA loads of real [1, T, 1, 128] tensors
-    (rows past T zero-filled), as the chunk kernel issues them."""
-    g = torch.Generator().manual_seed(5)
-    bf = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16)
-    K, Q, V = bf(64, 128), bf(64, 128), bf(64, 64)
-    qd = kd = vd = None
-    if tma_T:
-        qd = bf(1, tma_T, 1, 128).cuda()
-        kd = bf(1, tma_T, 1, 128).cuda()
-        vd = bf(1, tma_T, 1, 128).cuda()
-        Q = torch.zeros(64, 128, dtype=torch.bfloat16); Q[:tma_T] = qd[0, :, 0].cpu()
-        K = torch.zeros(64, 128, dtype=torch.bfloat16); K[:tma_T] = kd[0, :, 0].cpu()
-        Vfull = torch.zeros(64, 128, dtype=torch.bfloat16); Vfull[:tma_T] = vd[0, :, 0].cpu()
-    Aqk, A1, A2, Wt, S = bf(64, 64), bf(64, 64), bf(64, 64), bf(64, 128), bf(128, 64)
-    Ut, Us = bf(64, 64), bf(64, 64)
-    img = torch.zeros(149056, dtype=torch.uint8)
-
-    def put(off, tile):
-        b = _swz(tile)
-        img[off:off + b.numel()] = b
-
-    put(0, K[:, :64]); put(8192, Q[:, :64]); put(16384, K[:, 64:]); put(24576, Q[:, 64:])
-    put(32768, V); put(40960, Aqk); put(49152, A1); put(57344, A2)
-    put(65536, Wt[:, :64]); put(73728, Wt[:, 64:]); put(81920, S)
-    put(98304, Ut); put(106496, Us)
-    tiles = img.cuda()
-    out = torch.full((2, 40960), float("nan"), device="cuda")
-    st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ptr = lambda t: None if t is None else _p(t)
-    sink = torch.zeros(1, device="cuda")
-    assert lib.probe_skeleton(_p(tiles), _p(out), _p(st), ptr(qd), ptr(kd), ptr(vd), tma_T, mode,
-                              _p(sink)) == 0
-    torch.cuda.synchronize()
-    assert st.item() == 0
-    f = lambda t: t.float()
-    for cta in range(2):
-        Vc = Vfull[:, 64 * cta:64 * cta + 64] if tma_T else V
-        refs = [(0, (torch.cat([K, Q]).float() @ f(K).T)), (8192, f(A1) @ f(K)),
-                (16384, f(A2) @ f(Vc)), (20480, f(Wt) @ f(S)), (24576, f(Q) @ f(S)),
-                (28672, f(Aqk) @ f(Ut)), (32768, f(K).T @ f(Us))]
-        for off, ref in refs:
-            got = out[cta, off:off + ref.numel()].view(ref.shape).cpu()
-            torch.testing.assert_close(got, ref, rtol=1e-5, atol=1e-3, msg=f"cta {cta} @ {off}")
-
-
-@pytest.mark.parametrize("T,stages", [(1, 0), (64, 0), (1, 1), (64, 1), (1, 2), (64, 2), (1, 3),
-                                      (64, 3)])
-def test_chunk_prologue_on_skeleton(lib, T, stages):
-    """The chunk kernel's own prologue code (gates from gate tensors, q norms,
-    KK / QK epilogue, forward substitution, A1 / A2) on the validated skeleton,
-    launched like the chunk kernel; then the W / U round on the computed tiles."""
-    lib.probe_prologue.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int, ctypes.c_float,
-                                                           ctypes.c_void_p, ctypes.c_void_p,
-                                                           ctypes.c_void_p, ctypes.c_int]
-    g = torch.Generator(device="cuda").manual_seed(T)
-    r = lambda *s, dt=torch.bfloat16: torch.randn(*s, device="cuda", generator=g).to(dt)
-    q, k, v = r(1, T, 1, 128), r(1, T, 1, 128), r(1, T, 1, 128)
-    a, b = r(1, T, 1), r(1, T, 1)
-    A_log = torch.rand(1, device="cuda", generator=g) * 2.7
-    dt_bias = -1 - 3 * torch.rand(1, device="cuda", generator=g)
-    h0 = r(1, 1, 128, 128, dt=torch.float32) * 0.02
-    o = torch.zeros(1, T, 1, 128, device="cuda", dtype=torch.bfloat16)
-    out = torch.full((2, 69632), float("nan"), device="cuda")
-    st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    rc = lib.probe_prologue(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(dt_bias), _p(h0), T,
-                            128 ** -0.5, _p(o), _p(out), _p(st), stages)
-    assert rc == 0, rc
-    torch.cuda.synchronize()
-    assert st.item() == 0
-    K = torch.zeros(64, 128); K[:T] = k[0, :, 0].float().cpu()
-    V = torch.zeros(64, 128); V[:T] = v[0, :, 0].float().cpu()
-    for cta in range(2):
-        A1 = out[cta, :4096].view(64, 64).cpu()
-        A2 = out[cta, 4096:8192].view(64, 64).cpu()
-        assert torch.isfinite(A1).all() and torch.isfinite(A2).all()
-        torch.testing.assert_close(out[cta, 8192:16384].view(64, 128).cpu(), A1 @ K,
-                                   rtol=1e-4, atol=1e-3)
-        torch.testing.assert_close(out[cta, 16384:20480].view(64, 64).cpu(),
-                                   A2 @ V[:, 64 * cta:64 * cta + 64], rtol=1e-4, atol=1e-3)
-        Sb = h0[0, 0, :, 64 * cta:64 * cta + 64].to(torch.bfloat16).float().cpu()
-        assert torch.equal(out[cta, 20480:28672].view(128, 64).cpu(), Sb)
-        if stages >= 1:
-            Wb = out[cta, 8192:16384].view(64, 128).cpu().to(torch.bfloat16).float()
-            Q = torch.zeros(64, 128); Q[:T] = q[0, :, 0].float().cpu()
-            torch.testing.assert_close(out[cta, 28672:32768].view(64, 64).cpu(), Wb @ Sb,
-                                       rtol=1e-3, atol=1e-3)
-            torch.testing.assert_close(out[cta, 32768:36864].view(64, 64).cpu(), Q @ Sb,
-                                       rtol=1e-3, atol=1e-3)
-        if stages >= 2:
-            Aqk = out[cta, 36864:40960].view(64, 64).cpu()
-            Ut = out[cta, 40960:45056].view(64, 64).cpu()
-            Us = out[cta, 45056:49152].view(64, 64).cpu()
-            torch.testing.assert_close(out[cta, 49152:53248].view(64, 64).cpu(), Aqk @ Ut,
-                                       rtol=1e-3, atol=1e-3)
-            Kb = K.to(torch.bfloat16).float()
-            torch.testing.assert_close(out[cta, 53248:61440].view(128, 64).cpu(), Kb.T @ Us,
-                                       rtol=1e-3, atol=1e-3)
-        if stages >= 3:
-            S_new = out[cta, 61440:69632].view(128, 64).cpu()
-            assert torch.isfinite(S_new).all()
-    if stages >= 3:
-        assert torch.isfinite(o.float()).all()

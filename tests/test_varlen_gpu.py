@@ -6,7 +6,7 @@ import torch
 
 from gdn_synth import gdn_inputs
 from oracle import oracle as O
-from tests.parity import TOL, cpu, rel_err
+from tests.parity import TOL, assert_bf16_store, cpu, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -26,13 +26,18 @@ def test_varlen_packed_batch(dtype, d):
     x = gdn_inputs(1, Tt, Hk, Hv, d, dtype, seed=90, device=DEV, h0=False)
     h0 = 0.02 * torch.randn(N, Hv, d, d, device=DEV)
     q, k, v, a, b = (x[n][0] for n in ("q", "k", "v", "a", "b"))
-    o, ht = G.gdn_chunk_fwd_varlen(q, k, v, a, b, x["A_log"], x["dt_bias"], h0, cu)
+    o, ht = G.gdn_chunk_fwd_varlen(q, k, v, a, b, x["A_log"], x["dt_bias"], h0, cu,
+                                   out_f32=True)
+    if dtype == torch.bfloat16:
+        o16, ht16 = G.gdn_chunk_fwd_varlen(q, k, v, a, b, x["A_log"], x["dt_bias"], h0, cu)
+        assert_bf16_store(o16, o)
+        assert torch.equal(ht16, ht)
     tol = TOL[dtype]
     for i in range(N):
         s0, s1 = cu[i], cu[i + 1]
         sl = lambda t: t[s0:s1][None]
         o1, h1 = G.gdn_chunk_fwd(sl(q), sl(k), sl(v), sl(a), sl(b), x["A_log"], x["dt_bias"],
-                                 h0[i:i + 1])
+                                 h0[i:i + 1], out_f32=True)
         assert torch.equal(o[s0:s1], o1[0]) and torch.equal(ht[i], h1[0])
         ro, rht = O.gdn_fwd(cpu(sl(q)), cpu(sl(k)), cpu(sl(v)), cpu(sl(a)), cpu(sl(b)),
                             cpu(x["A_log"]), cpu(x["dt_bias"]), cpu(h0[i:i + 1]))

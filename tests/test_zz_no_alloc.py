@@ -39,9 +39,13 @@ def test_noalloc_same_bits_as_workspace_path_and_oracle():
     assert torch.cuda.memory_stats()["allocation.all.allocated"] == n_alloc
     assert torch.cuda.memory_allocated() == used
     assert torch.equal(o, o_ref) and torch.equal(ht, ht_ref)
+    # parity on the float32 output of the same path (the bar of the test suite)
+    o32, ht32 = G.gdn_chunk_fwd_noalloc(*_args(x), out_f32=True)
+    assert torch.equal(ht32, ht)
     ro, rht = O.gdn_fwd(cpu(x["q"]), cpu(x["k"]), cpu(x["v"]), cpu(x["a"]), cpu(x["b"]),
                         cpu(x["A_log"]), cpu(x["dt_bias"]), cpu(x["h0"]))
-    assert rel_err(o, ro) <= TOL[torch.bfloat16] and rel_err(ht, rht) <= TOL[torch.bfloat16]
+    assert rel_err(o32, ro) <= TOL[torch.bfloat16] and rel_err(ht, rht) <= TOL[torch.bfloat16]
+    assert torch.equal(o32.to(torch.bfloat16), o)
 
 
 def test_noalloc_workspace_free_shapes_run_unchanged():
