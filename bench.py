@@ -264,6 +264,7 @@ def run_ours(args, rank, local_rank, world):
         extra["gdn2_b4_4k"] = measure_gdn2(G, dev, stream, pk, args)
         extra["conv_prefill_8k"] = measure_conv(G, dev, stream, pk, args)
         extra["gate_prep_8k"] = measure_gate_prep(G, dev, stream, pk, args)
+        extra["prefill_8k_gated_norm"] = measure_prefill_gated_norm(G, dev, stream, pk, args)
         # the newest secondary figures, last: a failure is reported here, not raised
         for name, fn in (("kda_b4_4k", measure_kda), ("rmsnorm_gated_8k", measure_norm)):
             try:
@@ -465,6 +466,42 @@ def measure_gate_prep(G, dev, stream, pk, args):
             "steps": steps}
 
 
+def measure_prefill_gated_norm(G, dev, stream, pk, args):
+    """prefill_8k through gdn_chunk_fwd_gated_norm (the gated RMSNorm of the output
+    stage fused into the scan's output store), beside gdn_chunk_fwd followed by the
+    standalone gdn_rmsnorm_gated: the same result, one HBM pass over o and the
+    norm's own kernel fewer."""
+    w = WORKLOADS["prefill_8k"]
+    x = workload_inputs(w, dev)
+    g = torch.Generator(device="cpu").manual_seed(1008)
+    z = torch.randn((w.B, w.T, w.Hv, w.d), generator=g).to(w.dtype).to(dev)
+    nw = (0.5 + torch.rand(w.d, generator=g)).to(dev)
+    o = torch.empty((w.B, w.T, w.Hv, w.d), device=dev, dtype=w.dtype)
+    y = torch.empty_like(o)
+    ht = torch.empty((w.B, w.Hv, w.d, w.d), device=dev, dtype=torch.float32)
+    ws = chunk_workspace(G, w, dev)
+
+    def fused():
+        G.gdn_chunk_fwd_gated_norm(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"],
+                                   x["dt_bias"], x["h0"], z, nw, o=o, ht=ht, workspace=ws,
+                                   stream=stream)
+
+    def composed():
+        G.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                        x["h0"], o=o, ht=ht, workspace=ws, stream=stream)
+        G.gdn_rmsnorm_gated(o, z, nw, y=y, stream=stream)
+
+    _, per_f = time_steps(fused, 10, 3, stream)
+    _, per_c = time_steps(composed, 10, 3, stream)
+    ms_f, ms_c = sum(per_f) / len(per_f), sum(per_c) / len(per_c)
+    rl = prefill_roofline(w, ms_f, pk, "chunk_prefill_8k_gated_norm")
+    del x, z, o, y, ht, ws
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(w.B * w.T / (ms_f / 1e3), 1), "ms_per_step": round(ms_f, 4),
+            "ms_per_step_unfused": round(ms_c, 4), "frac_of_bf16_peak": rl["frac"],
+            "roofline": rl}
+
+
 def measure_kda(G, dev, stream, pk, args):
     """gdn_kda_chunk_fwd at the Gated DeltaNet-2 bench shape (B=4, T=4096, 16 heads,
     d=128, bf16): the gate tiling plus the Gated DeltaNet-2 kernels."""
@@ -534,6 +571,8 @@ def run_only(args, local_rank):
         r = measure_kda(G, dev, stream, pk, args)
     elif args.only == "gate_prep_8k":
         r = measure_gate_prep(G, dev, stream, pk, args)
+    elif args.only == "prefill_8k_gated_norm":
+        r = measure_prefill_gated_norm(G, dev, stream, pk, args)
     else:
         r = measure_prefill(G, args.only, dev, stream, pk, args)
     G.gdn_check_status(stream)
@@ -611,7 +650,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["prefill_8k", "decode_256", "gdn2_b4_4k", "prefill_128k",
                                        "prefill_b8_16k", "conv_prefill_8k", "rmsnorm_gated_8k",
-                                       "kda_b4_4k", "gate_prep_8k"],
+                                       "kda_b4_4k", "gate_prep_8k", "prefill_8k_gated_norm"],
                     default=None,
                     help="measure one secondary workload alone (profiling runs)")
     args = ap.parse_args()

@@ -21,6 +21,7 @@ __all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_chunk_workspace_bytes", "gdn_r
            "gdn_conv_prefill", "gdn_rmsnorm_gated", "gdn_kda_chunk_fwd",
            "gdn_kda_chunk_workspace_bytes", "gdn_chunk_fwd_varlen",
            "gdn2_chunk_fwd", "gdn2_chunk_workspace_bytes", "gdn_chunk_fwd_noalloc",
+           "gdn_chunk_fwd_gated_norm", "gdn_recurrent_step_gated_norm",
            "gdn_check_status", "gdn_status", "gdn_test_set_wait_fault", "GDNError",
            "LIB_PATH", "lib", "F32", "BF16",
            "QK_L2NORM", "GATES_PRECOMPUTED", "OUT_F32"]
@@ -62,6 +63,9 @@ lib.gdn_chunk_workspace_bytes.argtypes = [_i] * 7
 lib.gdn2_chunk_workspace_bytes.argtypes = [_i] * 6
 lib.gdn_chunk_workspace_bytes.restype = _sz
 lib.gdn2_chunk_workspace_bytes.restype = _sz
+lib.gdn_chunk_fwd_gated_norm.argtypes = [_vp] * 10 + [_f] + [_i] * 7 + [_f, _i, _vp, _vp, _vp,
+                                                                       _sz, _vp]
+lib.gdn_recurrent_step_gated_norm.argtypes = [_vp] * 10 + [_f, _vp] + [_i] * 6 + [_f, _i, _vp]
 lib.gdn_check_status.argtypes = [_vp]
 lib.gdn_test_set_wait_fault.argtypes = [_i, ctypes.c_uint]
 lib.gdn_test_set_wait_fault.restype = _i
@@ -69,6 +73,7 @@ lib.gdn_status_string.argtypes = [_i]
 lib.gdn_status_string.restype = ctypes.c_char_p
 lib.gdn_version.argtypes = []
 for _fn in (lib.gdn_gate_prep, lib.gdn_chunk_fwd, lib.gdn_chunk_fwd_noalloc, lib.gdn_chunk_fwd_host,
+            lib.gdn_chunk_fwd_gated_norm, lib.gdn_recurrent_step_gated_norm,
             lib.gdn2_chunk_fwd,
             lib.gdn_recurrent_step, lib.gdn_conv_prefill, lib.gdn_rmsnorm_gated,
             lib.gdn_kda_chunk_fwd, lib.gdn_chunk_fwd_varlen,
@@ -190,6 +195,45 @@ def gdn_chunk_fwd(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, scale=Non
     _check(lib.gdn_chunk_fwd(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(dt_bias), _p(h0),
                              B, T, Hk, Hv, dk, dv, _dtype_code(dt), float(scale), flags, _p(o),
                              _p(ht), _p(workspace), ws_bytes, _stream(stream)), "gdn_chunk_fwd")
+    return o, ht
+
+
+def gdn_chunk_fwd_gated_norm(q, k, v, a, b, A_log, dt_bias, h0, z, norm_weight, *, eps=1e-6,
+                             scale=None, l2norm=True, gates_precomputed=False, out_f32=False,
+                             o=None, ht=None, want_ht=True, workspace=None, stream=None):
+    """gdn_chunk_fwd with the gated RMSNorm of the output stage applied to o:
+    o = core / sqrt(mean(core^2) + eps) * norm_weight * SiLU(z) per (token, value
+    head); z [B,T,Hv,dv] in the input dtype, norm_weight [dv] float32.  Fused into
+    the scan's output store on the bf16 d = 128 path.  Returns (o, ht)."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dt = q.dtype
+    scale = dk ** -0.5 if scale is None else scale
+    _need(k, dt, q.shape, "k")
+    _need(v, dt, (B, T, Hv, dv), "v")
+    gdt = torch.float32 if gates_precomputed else dt
+    _need(a, gdt, (B, T, Hv), "a")
+    _need(b, gdt, (B, T, Hv), "b")
+    _need(z, dt, (B, T, Hv, dv), "z")
+    _need(norm_weight, torch.float32, (dv,), "norm_weight")
+    if h0 is not None:
+        _need(h0, torch.float32, (B, Hv, dk, dv), "h0")
+    odt = torch.float32 if out_f32 else dt
+    o = torch.empty((B, T, Hv, dv), device=q.device, dtype=odt) if o is None else o
+    _need(o, odt, (B, T, Hv, dv), "o")
+    if ht is None and want_ht:
+        ht = torch.empty((B, Hv, dk, dv), device=q.device, dtype=torch.float32)
+    flags = ((QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
+             | (OUT_F32 if out_f32 else 0))
+    ws_need = gdn_chunk_workspace_bytes(B, T, Hk, Hv, dk, dv, dt)
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.gdn_chunk_fwd_gated_norm(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log),
+                                        _p(dt_bias), _p(h0), _p(z), _p(norm_weight),
+                                        float(eps), B, T, Hk, Hv, dk, dv, _dtype_code(dt),
+                                        float(scale), flags, _p(o), _p(ht), _p(workspace),
+                                        ws_bytes, _stream(stream)), "gdn_chunk_fwd_gated_norm")
     return o, ht
 
 
@@ -431,6 +475,35 @@ def gdn_recurrent_step(x, conv_w, conv_state, a, b, A_log, dt_bias, state, *, Hk
                                   _dtype_code(dt), float(scale), OUT_F32 if out_f32 else 0,
                                   _stream(stream)),
            "gdn_recurrent_step")
+    return o
+
+
+def gdn_recurrent_step_gated_norm(x, conv_w, conv_state, a, b, A_log, dt_bias, state, z,
+                                  norm_weight, *, Hk, Hv, dk, dv, eps=1e-6, scale=None,
+                                  out_f32=False, o=None, stream=None):
+    """gdn_recurrent_step with the gated RMSNorm of the output stage fused into the
+    store of o; z [N, Hv, dv] in the input dtype, norm_weight [dv] float32."""
+    N = x.shape[0]
+    dt = x.dtype
+    scale = dk ** -0.5 if scale is None else scale
+    _need(x, dt, (N, 2 * Hk * dk + Hv * dv), "x")
+    _need(a, dt, (N, Hv), "a")
+    _need(b, dt, (N, Hv), "b")
+    _need(state, torch.float32, (N, Hv, dk, dv), "state")
+    _need(z, dt, (N, Hv, dv), "z")
+    _need(norm_weight, torch.float32, (dv,), "norm_weight")
+    if conv_w is not None:
+        _need(conv_w, torch.float32, (x.shape[1], 4), "conv_w")
+        _need(conv_state, dt, (N, x.shape[1], 3), "conv_state")
+    odt = torch.float32 if out_f32 else dt
+    o = torch.empty((N, Hv, dv), device=x.device, dtype=odt) if o is None else o
+    _need(o, odt, (N, Hv, dv), "o")
+    _check(lib.gdn_recurrent_step_gated_norm(_p(x), _p(conv_w), _p(conv_state), _p(a), _p(b),
+                                             _p(A_log), _p(dt_bias), _p(state), _p(z),
+                                             _p(norm_weight), float(eps), _p(o), N, Hk, Hv, dk,
+                                             dv, _dtype_code(dt), float(scale),
+                                             OUT_F32 if out_f32 else 0, _stream(stream)),
+           "gdn_recurrent_step_gated_norm")
     return o
 
 

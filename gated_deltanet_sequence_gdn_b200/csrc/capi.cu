@@ -158,6 +158,36 @@ int gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* a, co
   return run_chunk(c, false, workspace, ws_bytes, (cudaStream_t)stream);
 }
 
+int gdn_chunk_fwd_gated_norm(const void* q, const void* k, const void* v, const void* a,
+                             const void* b, const float* A_log, const float* dt_bias,
+                             const float* h0, const void* z, const float* norm_weight, float eps,
+                             int B, int T, int Hk, int Hv, int dk, int dv, int dtype, float scale,
+                             int flags, void* o, float* ht, void* workspace, size_t ws_bytes,
+                             gdn_stream_t stream) {
+  ChunkArgs c{q, k, v, a, b, nullptr, A_log, dt_bias, h0, B, T, Hk, Hv, dk, dv, dtype,
+              scale, flags, o, ht};
+  int st = validate_chunk(c, false);
+  if (st != GDN_OK) return st;
+  if (!(eps >= 0.f) || eps > 1.f) return GDN_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((long)B * T == 0) return run_chunk(c, false, workspace, ws_bytes, s);
+  if (!ok_ptr(z) || !ok_elem(norm_weight, 4)) return GDN_ERR_INVALID_ARG;
+  if (chunk_mma_supported(c)) {  // fused into the scan's output rows
+    c.norm_z = z;
+    c.norm_w = norm_weight;
+    c.norm_eps = eps;
+    return run_chunk(c, false, workspace, ws_bytes, s);
+  }
+  // the float32 / d = 64 path: the forward, then the gated RMSNorm over o in place
+  st = run_chunk(c, false, workspace, ws_bytes, s);
+  if (st != GDN_OK) return st;
+  const long rows = (long)B * T * Hv;
+  if (dtype == GDN_BF16 && (flags & GDN_OUT_F32))  // float32 cores, bf16 gate
+    return from_cuda(launch_rmsnorm_gated_f32_bf16z(static_cast<float*>(o), z, norm_weight,
+                                                    static_cast<float*>(o), rows, dv, eps, s));
+  return from_cuda(launch_rmsnorm_gated(o, z, norm_weight, o, rows, dv, dtype, eps, s));
+}
+
 // Sequence i of a packed batch: the arguments of a one-sequence gdn_chunk_fwd call
 // on its token range [t0, t0 + Ti) and its own initial / final state.
 static ChunkArgs varlen_seq(const ChunkArgs& all, long long t0, int Ti, int i) {
@@ -293,7 +323,34 @@ int gdn_recurrent_step(const void* x_qkv, const float* conv_w, void* conv_state,
   if (conv_w != nullptr && !ok_elem(conv_state, es)) return GDN_ERR_INVALID_ARG;
   return from_cuda(launch_recurrent_step(x_qkv, conv_w, conv_state, a, b, A_log, dt_bias,
                                          state, o, N, Hk, Hv, dk, dv, dtype, scale,
-                                         (flags & GDN_OUT_F32) != 0, (cudaStream_t)stream));
+                                         (flags & GDN_OUT_F32) != 0, DecodeNorm{},
+                                         (cudaStream_t)stream));
+}
+
+int gdn_recurrent_step_gated_norm(const void* x_qkv, const float* conv_w, void* conv_state,
+                                  const void* a, const void* b, const float* A_log,
+                                  const float* dt_bias, float* state, const void* z,
+                                  const float* norm_weight, float eps, void* o, int N, int Hk,
+                                  int Hv, int dk, int dv, int dtype, float scale, int flags,
+                                  gdn_stream_t stream) {
+  if (N < 0 || Hk <= 0 || Hv <= 0 || !ok_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  if (flags & ~GDN_OUT_F32) return GDN_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || eps > 1.f) return GDN_ERR_INVALID_ARG;
+  if (!ok_head_dim(dk) || !ok_head_dim(dv) || Hv % Hk != 0) return GDN_ERR_UNSUPPORTED;
+  if (N == 0) return GDN_OK;
+  const size_t es = elem_size(dtype);
+  if (!ok_elem(x_qkv, es) || !ok_elem(a, es) || !ok_elem(b, es) || !ok_elem(A_log, 4) ||
+      !ok_elem(dt_bias, 4) || !ok_ptr(state) || !ok_elem(o, (flags & GDN_OUT_F32) ? 4 : es) ||
+      !ok_opt(conv_w) || !ok_elem(z, es) || !ok_elem(norm_weight, 4))
+    return GDN_ERR_INVALID_ARG;
+  if (conv_w != nullptr && !ok_elem(conv_state, es)) return GDN_ERR_INVALID_ARG;
+  DecodeNorm nm;
+  nm.z = z;
+  nm.w = norm_weight;
+  nm.eps = eps;
+  return from_cuda(launch_recurrent_step(x_qkv, conv_w, conv_state, a, b, A_log, dt_bias,
+                                         state, o, N, Hk, Hv, dk, dv, dtype, scale,
+                                         (flags & GDN_OUT_F32) != 0, nm, (cudaStream_t)stream));
 }
 
 int gdn_conv_prefill(const void* x_qkv, const float* conv_w, void* conv_state, void* q, void* k,

@@ -12,6 +12,11 @@
 // group's query/key conv channels are shared by its Hv/Hk value heads, so the
 // CTA that owns them is the only one that shifts their conv window (no race
 // between CTAs on the in-place conv state).
+//
+// With NORM each output row leaves through the gated RMSNorm of the pages' output
+// stage ("gated-deltanet-qwen3.5", 输出门控与 RMSNorm): y = o / sqrt(mean(o^2) + eps)
+// * w * SiLU(z) over the dv columns of the (sequence, value head); the CTA holds
+// the whole row, so the mean is a block reduction.
 #include "common.cuh"
 #include "launch.h"
 
@@ -20,13 +25,14 @@ namespace {
 
 constexpr int kThreads = 256;
 
-template <typename T, typename TO, int DK, int DV>
+template <typename T, typename TO, int DK, int DV, bool NORM>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_step_kernel(const T* __restrict__ x, const float* __restrict__ conv_w,
                    T* __restrict__ conv_state, const T* __restrict__ a,
                    const T* __restrict__ b, const float* __restrict__ A_log,
                    const float* __restrict__ dt_bias, float* __restrict__ state,
-                   TO* __restrict__ o, int Hk, int Hv, float scale) {
+                   TO* __restrict__ o, int Hk, int Hv, float scale, const T* __restrict__ nz,
+                   const float* __restrict__ nw, float neps) {
   constexpr int TPR = DV / 4;               // threads per state row (float4 each)
   constexpr int RPP = kThreads / TPR;       // rows covered per pass
   constexpr int PASSES = DK / RPP;          // rows per thread
@@ -44,6 +50,7 @@ decode_step_kernel(const T* __restrict__ x, const float* __restrict__ conv_w,
   float* red = vv + G * DV;         // [RPP][DV] partial sums
   float* gates = red + RPP * DV;    // [G][2] alpha, beta
   __shared__ float norm_ss[2];
+  __shared__ float row_ss[DV / 32];
 
   // ---- 1. conv1d + SiLU over the group's channels, window shifted in place
   const int n_ch = 2 * DK + G * DV;
@@ -139,12 +146,26 @@ decode_step_kernel(const T* __restrict__ x, const float* __restrict__ conv_w,
     __syncthreads();  // everyone has read `red`
     reinterpret_cast<float4*>(red + rsub * DV)[col4] = oo;
     __syncthreads();
+    float acc = 0.f;
     if (tid < DV) {
-      float acc = 0.f;
 #pragma unroll 4
       for (int r = 0; r < RPP; ++r) acc += red[r * DV + tid];
-      o[((size_t)n * Hv + hv) * DV + tid] = from_f32<TO>(acc);
     }
+    if (NORM) {  // sum of squares of the row over its DV columns (warps 0 .. DV/32-1)
+      if (tid < DV) {
+        const float ss = warp_sum(acc * acc);
+        if ((tid & 31) == 0) row_ss[tid >> 5] = ss;
+      }
+      __syncthreads();
+      if (tid < DV) {
+        float ss = 0.f;
+#pragma unroll
+        for (int w = 0; w < DV / 32; ++w) ss += row_ss[w];
+        const float zz = to_f32(nz[((size_t)n * Hv + hv) * DV + tid]);
+        acc *= rsqrtf(ss * (1.f / DV) + neps) * nw[tid] * (zz * sigmoid_f(zz));
+      }
+    }
+    if (tid < DV) o[((size_t)n * Hv + hv) * DV + tid] = from_f32<TO>(acc);
     __syncthreads();
   }
 }
@@ -152,11 +173,13 @@ decode_step_kernel(const T* __restrict__ x, const float* __restrict__ conv_w,
 template <typename T, typename TO, int DK, int DV>
 cudaError_t launch_t(const void* x, const float* conv_w, void* conv_state, const void* a,
                      const void* b, const float* A_log, const float* dt_bias, float* state,
-                     void* o, int N, int Hk, int Hv, float scale, cudaStream_t s) {
+                     void* o, int N, int Hk, int Hv, float scale, const DecodeNorm& nm,
+                     cudaStream_t s) {
   const int G = Hv / Hk;
   constexpr int RPP = kThreads / (DV / 4);
   const size_t smem = sizeof(float) * (2 * DK + G * DV + RPP * DV + 2 * G);
-  auto kern = decode_step_kernel<T, TO, DK, DV>;
+  auto kern = nm.z ? decode_step_kernel<T, TO, DK, DV, true>
+                   : decode_step_kernel<T, TO, DK, DV, false>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -164,7 +187,7 @@ cudaError_t launch_t(const void* x, const float* conv_w, void* conv_state, const
   }
   kern<<<(unsigned)(N * Hk), kThreads, smem, s>>>(
       (const T*)x, conv_w, (T*)conv_state, (const T*)a, (const T*)b, A_log, dt_bias, state,
-      (TO*)o, Hk, Hv, scale);
+      (TO*)o, Hk, Hv, scale, static_cast<const T*>(nm.z), nm.w, nm.eps);
   return cudaGetLastError();
 }
 
@@ -172,11 +195,11 @@ template <typename T, typename TO>
 cudaError_t launch_dt(int dk, int dv, const void* x, const float* conv_w, void* conv_state,
                       const void* a, const void* b, const float* A_log, const float* dt_bias,
                       float* state, void* o, int N, int Hk, int Hv, float scale,
-                      cudaStream_t s) {
+                      const DecodeNorm& nm, cudaStream_t s) {
 #define GDN_DEC(DK_, DV_)                                                               \
   if (dk == DK_ && dv == DV_)                                                           \
     return launch_t<T, TO, DK_, DV_>(x, conv_w, conv_state, a, b, A_log, dt_bias, state, o, \
-                                 N, Hk, Hv, scale, s);
+                                 N, Hk, Hv, scale, nm, s);
   GDN_DEC(64, 64) GDN_DEC(64, 128) GDN_DEC(128, 64) GDN_DEC(128, 128)
 #undef GDN_DEC
   return cudaErrorInvalidValue;
@@ -188,16 +211,16 @@ cudaError_t launch_recurrent_step(const void* x, const float* conv_w, void* conv
                                   const void* a, const void* b, const float* A_log,
                                   const float* dt_bias, float* state, void* o, int N,
                                   int Hk, int Hv, int dk, int dv, int dtype, float scale,
-                                  bool out_f32, cudaStream_t s) {
+                                  bool out_f32, const DecodeNorm& nm, cudaStream_t s) {
   if (N == 0) return cudaSuccess;
   if (dtype == GDN_BF16)
     return out_f32 ? launch_dt<__nv_bfloat16, float>(dk, dv, x, conv_w, conv_state, a, b, A_log,
-                                                     dt_bias, state, o, N, Hk, Hv, scale, s)
+                                                     dt_bias, state, o, N, Hk, Hv, scale, nm, s)
                    : launch_dt<__nv_bfloat16, __nv_bfloat16>(dk, dv, x, conv_w, conv_state, a,
                                                              b, A_log, dt_bias, state, o, N, Hk,
-                                                             Hv, scale, s);
+                                                             Hv, scale, nm, s);
   return launch_dt<float, float>(dk, dv, x, conv_w, conv_state, a, b, A_log, dt_bias, state, o,
-                                 N, Hk, Hv, scale, s);
+                                 N, Hk, Hv, scale, nm, s);
 }
 
 }  // namespace gdn

@@ -6,8 +6,9 @@
 // this library's reading of the pages.
 //
 // HBM-bound: one read of q, k, a, b and one write of the outputs.  One CTA per
-// group of token rows; one warp per (row, head) vector of q or k, each lane
-// moving 16-byte pieces; the gates are spread over the CTA's threads.
+// group of token rows; a group of lanes per (row, head) vector of q or k, each
+// lane moving 16-byte pieces, several vectors in flight per lane; the gates are
+// spread over the CTA's threads.
 #include "common.cuh"
 #include "launch.h"
 
@@ -47,7 +48,16 @@ template <> __device__ __forceinline__ uint4 pack<__nv_bfloat16>(const float* f)
   return v;
 }
 
-// rows_per_cta token rows per CTA; d in {64, 128}.
+// Sum over the `width` lanes of an aligned lane group (width a power of 2 <= 32).
+__device__ __forceinline__ float group_sum(float v, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// rows_per_cta token rows per CTA; d in {64, 128}.  A q / k vector of one (row,
+// head) is d / E lanes of 16 bytes (a lane group); a warp holds 32 / (d / E) such
+// groups, and each group takes kU vectors per pass, all loads issued before the
+// first reduction, so that every lane has kU 16-byte loads in flight.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 gate_prep_kernel(const T* q, const T* k,
@@ -58,37 +68,54 @@ gate_prep_kernel(const T* q, const T* k,
                  float* __restrict__ beta_out) {
   using V = typename Vec16<T>::type;
   constexpr int E = Vec16<T>::n;
+  constexpr int kU = 4;
   const long row0 = (long)blockIdx.x * rows_per_cta;
   const long row1 = min(rows, row0 + rows_per_cta);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int vecs_per_head = d / E;            // 8..32 pieces of 16 bytes
-  const int per_lane = (vecs_per_head + 31) / 32;  // 1
-  // q / k vectors: item = (row, head, which)
+  const int width = d / E;                 // lanes per vector: 8, 16 or 32
+  const int groups = 32 / width;           // vectors per warp and pass step
+  const int gl = lane % width, grp = lane / width;
+  // vectors: item = (row, head, which), q and k of a head adjacent
   const long n_items = (row1 - row0) * Hk * 2;
-  for (long it = warp; it < n_items; it += kThreads / 32) {
-    const long r = row0 + it / (2 * Hk);
-    const int rem = (int)(it % (2 * Hk));
-    const int h = rem >> 1;
-    const bool is_q = (rem & 1) == 0;
-    const size_t off = ((size_t)r * Hk + h) * d;
-    const V* src = reinterpret_cast<const V*>((is_q ? q : k) + off);
-    V* dst = reinterpret_cast<V*>((is_q ? q_out : k_out) + off);
-    float f[E];
-    float ss = 0.f;
-    V vin{};
-    (void)per_lane;
-    if (lane < vecs_per_head) {
-      vin = src[lane];
-      unpack<T>(vin, f);
+  const long step = (long)(kThreads / 32) * groups;
+  // the loop bound is the same for every lane of the warp (the shuffles below take
+  // all 32 lanes); a group past the end just has nothing to load
+  for (long wbase = (long)warp * groups; wbase < n_items; wbase += step * kU) {
+    const long base = wbase + grp;
+    V vin[kU];
+    bool have[kU];
 #pragma unroll
-      for (int i = 0; i < E; ++i) ss += f[i] * f[i];
+    for (int u = 0; u < kU; ++u) {
+      const long it = base + u * step;
+      have[u] = it < n_items;
+      if (have[u]) {
+        const long r = row0 + it / (2 * Hk);
+        const int rem = (int)(it % (2 * Hk));
+        const size_t off = ((size_t)r * Hk + (rem >> 1)) * d;
+        vin[u] = reinterpret_cast<const V*>(((rem & 1) == 0 ? q : k) + off)[gl];
+      }
     }
-    ss = warp_sum(ss);
-    const float mul = rsqrtf(ss + 1e-6f) * (is_q ? scale : 1.f);
-    if (lane < vecs_per_head) {
 #pragma unroll
-      for (int i = 0; i < E; ++i) f[i] *= mul;
-      dst[lane] = pack<T>(f);
+    for (int u = 0; u < kU; ++u) {
+      const long it = base + u * step;
+      float f[E];
+      float ss = 0.f;
+      if (have[u]) {
+        unpack<T>(vin[u], f);
+#pragma unroll
+        for (int i = 0; i < E; ++i) ss += f[i] * f[i];
+      }
+      ss = group_sum(ss, width);  // every lane takes part (no divergent shuffles)
+      if (have[u]) {
+        const long r = row0 + it / (2 * Hk);
+        const int rem = (int)(it % (2 * Hk));
+        const bool is_q = (rem & 1) == 0;
+        const size_t off = ((size_t)r * Hk + (rem >> 1)) * d;
+        const float mul = rsqrtf(ss + 1e-6f) * (is_q ? scale : 1.f);
+#pragma unroll
+        for (int i = 0; i < E; ++i) f[i] *= mul;
+        reinterpret_cast<V*>((is_q ? q_out : k_out) + off)[gl] = pack<T>(f);
+      }
     }
   }
   // gates: item = (row, value head)
@@ -111,7 +138,7 @@ cudaError_t launch_gate_prep(const void* q, const void* k, int dtype, const void
                              cudaStream_t s) {
   const long rows = (long)B * T;
   if (rows == 0) return cudaSuccess;
-  const int rows_per_cta = 4;
+  const int rows_per_cta = 8;
   const long grid = (rows + rows_per_cta - 1) / rows_per_cta;
   if (dtype == GDN_BF16) {
     gate_prep_kernel<__nv_bfloat16><<<(unsigned)grid, kThreads, 0, s>>>(

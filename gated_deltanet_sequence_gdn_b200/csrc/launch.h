@@ -14,6 +14,8 @@ struct ChunkArgs {
   float scale;
   int flags;
   void* o; float* ht;
+  // gated RMSNorm of the output rows (o = RMSNormGated(core, z)); norm_z == NULL: none
+  const void* norm_z = nullptr; const float* norm_w = nullptr; float norm_eps = 0.f;
 };
 
 cudaError_t launch_gate_prep(const void* q, const void* k, int dtype, const void* a,
@@ -22,11 +24,18 @@ cudaError_t launch_gate_prep(const void* q, const void* k, int dtype, const void
                              void* q_out, void* k_out, float* g_out, float* beta_out,
                              cudaStream_t s);
 
+// Gated RMSNorm of the decode step's output rows; z == NULL: none.
+struct DecodeNorm {
+  const void* z = nullptr;  // [N, Hv, dv], the input dtype
+  const float* w = nullptr; // [dv]
+  float eps = 0.f;
+};
+
 cudaError_t launch_recurrent_step(const void* x, const float* conv_w, void* conv_state,
                                   const void* a, const void* b, const float* A_log,
                                   const float* dt_bias, float* state, void* o, int N,
                                   int Hk, int Hv, int dk, int dv, int dtype, float scale,
-                                  bool out_f32, cudaStream_t s);
+                                  bool out_f32, const DecodeNorm& nm, cudaStream_t s);
 
 cudaError_t launch_conv_prefill(const void* x, const float* conv_w, void* conv_state, void* q,
                                 void* k, void* v, int B, int T, int Hk, int Hv, int dk, int dv,
@@ -39,6 +48,10 @@ cudaError_t launch_tie_gates(const void* beta, void* b, void* w, size_t rows, in
 
 cudaError_t launch_rmsnorm_gated(const void* o, const void* z, const float* weight, void* y,
                                  long rows, int dv, int dtype, float eps, cudaStream_t s);
+// The same with float32 o / y and a bf16 gate z.
+cudaError_t launch_rmsnorm_gated_f32_bf16z(const float* o, const void* z, const float* weight,
+                                           float* y, long rows, int dv, float eps,
+                                           cudaStream_t s);
 
 // float32 CUDA-core chunk path (GDN and, with gdn2 = true, Gated DeltaNet-2).
 cudaError_t launch_chunk_simt(const ChunkArgs& a, bool gdn2, cudaStream_t s);

@@ -29,9 +29,11 @@ __device__ __forceinline__ void store_per(T* p, const float* f) {
   for (int i = 0; i < PER; ++i) p[i] = from_f32<T>(f[i]);
 }
 
-template <typename T, int DV>
+// o and y of type T, the gate z of type TZ (float32 cores gated by bf16 z on the
+// float32-output path of gdn_chunk_fwd_gated_norm).
+template <typename T, typename TZ, int DV>
 __global__ void __launch_bounds__(kRT)
-rmsnorm_gated_kernel(const T* o, const T* z, const float* __restrict__ weight, T* y, long rows,
+rmsnorm_gated_kernel(const T* o, const TZ* z, const float* __restrict__ weight, T* y, long rows,
                      float eps) {
   constexpr int PER = DV / 32;
   const int lane = threadIdx.x & 31;
@@ -40,7 +42,7 @@ rmsnorm_gated_kernel(const T* o, const T* z, const float* __restrict__ weight, T
   const size_t off = (size_t)row * DV + lane * PER;
   float ov[PER], zv[PER], wv[PER];
   load_per<T, PER>(o + off, ov);
-  load_per<T, PER>(z + off, zv);
+  load_per<TZ, PER>(z + off, zv);
 #pragma unroll
   for (int i = 0; i < PER; ++i) wv[i] = weight[lane * PER + i];
   float ss = 0.f;
@@ -57,12 +59,12 @@ rmsnorm_gated_kernel(const T* o, const T* z, const float* __restrict__ weight, T
   store_per<T, PER>(y + off, yv);
 }
 
-template <typename T, int DV>
+template <typename T, typename TZ, int DV>
 cudaError_t launch_typed(const void* o, const void* z, const float* w, void* y, long rows,
                          float eps, cudaStream_t s) {
   const long blocks = (rows + kRT / 32 - 1) / (kRT / 32);
-  rmsnorm_gated_kernel<T, DV><<<(unsigned)blocks, kRT, 0, s>>>(
-      static_cast<const T*>(o), static_cast<const T*>(z), w, static_cast<T*>(y), rows, eps);
+  rmsnorm_gated_kernel<T, TZ, DV><<<(unsigned)blocks, kRT, 0, s>>>(
+      static_cast<const T*>(o), static_cast<const TZ*>(z), w, static_cast<T*>(y), rows, eps);
   return cudaGetLastError();
 }
 
@@ -74,10 +76,20 @@ cudaError_t launch_rmsnorm_gated(const void* o, const void* z, const float* weig
   if ((rows + kRT / 32 - 1) / (kRT / 32) > 0x7fffffffL) return cudaErrorInvalidValue;
   using bf16 = __nv_bfloat16;
   if (dtype == GDN_BF16)
-    return dv == 128 ? launch_typed<bf16, 128>(o, z, weight, y, rows, eps, s)
-                     : launch_typed<bf16, 64>(o, z, weight, y, rows, eps, s);
-  return dv == 128 ? launch_typed<float, 128>(o, z, weight, y, rows, eps, s)
-                   : launch_typed<float, 64>(o, z, weight, y, rows, eps, s);
+    return dv == 128 ? launch_typed<bf16, bf16, 128>(o, z, weight, y, rows, eps, s)
+                     : launch_typed<bf16, bf16, 64>(o, z, weight, y, rows, eps, s);
+  return dv == 128 ? launch_typed<float, float, 128>(o, z, weight, y, rows, eps, s)
+                   : launch_typed<float, float, 64>(o, z, weight, y, rows, eps, s);
+}
+
+cudaError_t launch_rmsnorm_gated_f32_bf16z(const float* o, const void* z, const float* weight,
+                                           float* y, long rows, int dv, float eps,
+                                           cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if ((rows + kRT / 32 - 1) / (kRT / 32) > 0x7fffffffL) return cudaErrorInvalidValue;
+  using bf16 = __nv_bfloat16;
+  return dv == 128 ? launch_typed<float, bf16, 128>(o, z, weight, y, rows, eps, s)
+                   : launch_typed<float, bf16, 64>(o, z, weight, y, rows, eps, s);
 }
 
 }  // namespace gdn

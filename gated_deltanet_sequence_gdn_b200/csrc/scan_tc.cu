@@ -21,6 +21,18 @@
 // Hand-offs go through mbarriers; every wait is bounded and an expired wait ends
 // the kernel through the status word (GDN_ERR_TIMEOUT) after its copies and
 // tensor-core work in flight have drained.
+//
+// With NORM the output rows leave through the gated RMSNorm of the pages'
+// output stage, y = o / sqrt(mean(o^2) + eps) * w * SiLU(z) over the d_v columns
+// of each (token, value head) ("gated-deltanet-qwen3.5", 输出门控与 RMSNorm).
+// A row's columns are split over the two column-half CTAs of a head, which then
+// run as a cluster of two: each sends the sums of squares of its 64 columns of
+// the chunk's rows to the other through distributed shared memory (st.async into
+// the peer's buffer, counted as transaction bytes on the peer's mbarrier, so no
+// release fence waits on this thread's output stores).  The rows of chunk n wait
+// in shared memory, with their gate z copied in behind them, and are normalised
+// and stored during chunk n + 1, so the peer's sums have a whole chunk step to
+// arrive and the two CTAs' chains do not wait on each other.
 #include "chunk_layout.cuh"
 #include "common.cuh"
 #include "launch.h"
@@ -48,16 +60,26 @@ constexpr uint32_t OFF_SB = 2 * STAGE_BYTES;  // state (scaled) fp16, MN-major B
 constexpr uint32_t OFF_UT = OFF_SB + 16384;   // U~ fp16 [64][64]
 constexpr uint32_t OFF_US = OFF_UT + 8192;    // U~s fp16 [64][64]
 constexpr uint32_t OFF_RED = OFF_US + 8192;   // CTA max reduction (8 floats)
-constexpr uint32_t OFF_BAR = OFF_RED + 64;    // mbarriers + TMEM address
+constexpr uint32_t OFF_NRM = OFF_RED + 64;    // NORM: row sums of squares [64][2], and the
+                                              // peer's [2 chunk parities][64]
+constexpr uint32_t OFF_BAR = OFF_NRM + 1024;  // mbarriers + TMEM address
 constexpr uint32_t SCAN_TC_SMEM = OFF_BAR + 128 + 1024;
+// NORM only: the previous chunk's output rows before the norm, [64 rows][64] fp32,
+// and their gate z, [64 rows][64] bf16 (copied in one chunk ahead)
+constexpr uint32_t OFF_OBUF = OFF_BAR + 128;
+constexpr uint32_t OFF_ZBUF = OFF_OBUF + 64 * 64 * 4;
+constexpr uint32_t SCAN_TC_SMEM_NORM = SCAN_TC_SMEM + 64 * 64 * 4 + 64 * 64 * 2;
 static_assert(ST_SC + kScal * 4 <= STAGE_BYTES, "stage layout");
-static_assert(SCAN_TC_SMEM <= 227 * 1024, "shared memory of the tcgen05 scan");
+static_assert(SCAN_TC_SMEM_NORM <= 227 * 1024, "shared memory of the tcgen05 scan");
 
 // TMEM columns of the accumulators (M = 128, N = 64 each)
 constexpr uint32_t TM_QP = 0, TM_OA = 64, TM_DS = 128, TM_COLS = 256;
 
 // barrier indices
-enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_QP, B_UT, B_DS, B_OA, B_S, B_COUNT };
+enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_QP, B_UT, B_DS, B_OA, B_S,
+       B_PX0, B_PX1,  // NORM: the peer's row sums of squares of a chunk have arrived
+       B_COUNT };
+static_assert(B_COUNT * 8 + 8 <= 128, "barrier area");
 
 // Byte offset of 16-byte chunk c16 of row r in a 128-byte swizzled tile.
 __device__ __forceinline__ uint32_t swz(int r, int c16) {
@@ -94,6 +116,25 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, in
   *abort_flag = 1;
   return false;
 }
+// The same with acquire at cluster scope (for a barrier a peer CTA arrives on).
+__device__ __forceinline__ bool wait_cluster_or_abort(uint64_t* bar, uint32_t parity, int* status,
+                                                      int where, volatile int* abort_flag,
+                                                      uint32_t spin) {
+  for (uint32_t i = 0; i < spin; ++i) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((i & 255u) == 255u && *abort_flag) return false;
+  }
+  report_timeout(status, where);
+  *abort_flag = 1;
+  return false;
+}
+
+// Parameters of the gated RMSNorm applied to the output rows (NORM).
+struct NormArgs {
+  const __nv_bfloat16* z;  // [B, T, Hv, dv]
+  const float* w;          // [dv]
+  float eps;
+};
 
 // 32 output values of one row with 16-byte stores.
 template <typename TO>
@@ -121,15 +162,37 @@ __device__ __forceinline__ void store_row<bf16>(bf16* dst, const float* v) {
   }
 }
 
+// 8 output values with one 16-byte store (bf16) or two (float32).
+template <typename TO>
+__device__ __forceinline__ void store8(TO* dst, const float* v);
+template <>
+__device__ __forceinline__ void store8<float>(float* dst, const float* v) {
+  *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+template <>
+__device__ __forceinline__ void store8<bf16>(bf16* dst, const float* v) {
+  uint4 p;
+  __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
+  __nv_bfloat162 h1 = __floats2bfloat162_rn(v[2], v[3]);
+  __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]);
+  __nv_bfloat162 h3 = __floats2bfloat162_rn(v[6], v[7]);
+  p.x = *reinterpret_cast<uint32_t*>(&h0);
+  p.y = *reinterpret_cast<uint32_t*>(&h1);
+  p.z = *reinterpret_cast<uint32_t*>(&h2);
+  p.w = *reinterpret_cast<uint32_t*>(&h3);
+  *reinterpret_cast<uint4*>(dst) = p;
+}
+
 struct ScanMaps {
   CUtensorMap q, w, k, a, u;
 };
 
-template <typename TO>
+template <typename TO, bool NORM>
 __global__ void __launch_bounds__(kScanTcThreads, 1)
 state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __restrict__ ws,
                      WsLayout L, const float* h0, int T, int Hk, int Hv, TO* __restrict__ o,
-                     float* ht, int* status, int fault, uint32_t spin) {
+                     float* ht, int* status, int fault, uint32_t spin, NormArgs na) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -147,9 +210,14 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
 
   if (warp == 1) tmem_alloc(tmem_slot, TM_COLS);
   if (tid == 0) {
-    for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], (i == B_EMPTY0 || i == B_EMPTY1) ? 2 : 1);
+    for (int i = 0; i < B_COUNT; ++i)
+      mbar_init(&bar[i], (i == B_EMPTY0 || i == B_EMPTY1) ? 2 : 1);
     *abort_flag = 0;
     fence_mbar_init();
+    if (NORM) {  // each chunk's 64 peer sums arrive as 256 transaction bytes
+      mbar_arrive_expect_tx(&bar[B_PX0], 64 * 4);
+      mbar_arrive_expect_tx(&bar[B_PX1], 64 * 4);
+    }
     prefetch_tmap(&maps.q);
     prefetch_tmap(&maps.w);
     prefetch_tmap(&maps.k);
@@ -160,6 +228,8 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the peer's barriers are initialised before anything arrives on them
+  if (NORM) cluster_sync();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -284,6 +354,54 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
     if (e == 0 && fault != kFaultScanState) mbar_arrive(&bar[B_S]);
 
     float OQ[32];
+    // NORM: sums of squares of the rows, this CTA's and the peer's; the pending rows
+    float* ssq = reinterpret_cast<float*>(sm + OFF_NRM);  // [64][2]
+    float* xin = ssq + 128;                               // [2 chunk parities][64], from the peer
+    float* obuf = reinterpret_cast<float*>(sm + OFF_OBUF);
+    bf16* zbuf = reinterpret_cast<bf16*>(sm + OFF_ZBUF);
+    const uint32_t peer = NORM ? cluster_rank() ^ 1u : 0u;
+    float pend_part = 0.f;  // this CTA's sum of squares of the pending row
+    // Normalise and store the pending rows of chunk m (row threads, uniformly):
+    // y = o / sqrt(mean(o^2) + eps) * w * SiLU(z), the mean over both halves.
+    auto norm_finish = [&](int m, int r, int hf, int cbase, float part) -> bool {
+      const int slot = m & 1;
+      const bool got = wait_cluster_or_abort(&bar[B_PX0 + slot], (m >> 1) & 1, status, 109,
+                                             abort_flag, spin);
+      if (named_barrier_or(2, 128, !got)) return false;
+      const float rinv = rsqrtf((part + xin[64 * slot + r]) * (1.f / kD) + na.eps);
+      // the slot takes chunk m + 2 next; the peer sends it only after this CTA's sums
+      // of chunk m + 1, which follow this read (barrier 2 between)
+      if (r == 0 && hf == 0 && m + 2 < Nc) mbar_arrive_expect_tx(&bar[B_PX0 + slot], 64 * 4);
+      const int tm = m * kC + r;
+      asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's copy of z
+      if (tm < T) {
+        const float* ob = obuf + r * 64 + cbase;
+        const bf16* zr = zbuf + r * 64 + cbase;
+        const float* wr = na.w + c0 + cbase;
+        TO* dst = o + (((size_t)b * T + tm) * Hv + hv) * kD + c0 + cbase;
+#pragma unroll
+        for (int c8 = 0; c8 < 32; c8 += 8) {
+          float y[8];
+          const uint4 zz = *reinterpret_cast<const uint4*>(zr + c8);
+          const float4 wa = *reinterpret_cast<const float4*>(wr + c8);
+          const float4 wb = *reinterpret_cast<const float4*>(wr + c8 + 4);
+          const float4 oa = *reinterpret_cast<const float4*>(ob + c8);
+          const float4 obb = *reinterpret_cast<const float4*>(ob + c8 + 4);
+          const uint32_t zw[4] = {zz.x, zz.y, zz.z, zz.w};
+          const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+          const float ov[8] = {oa.x, oa.y, oa.z, oa.w, obb.x, obb.y, obb.z, obb.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 zf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zw[j]));
+            y[2 * j] = ov[2 * j] * rinv * wv[2 * j] * __fdividef(zf.x, 1.f + __expf(-zf.x));
+            y[2 * j + 1] =
+                ov[2 * j + 1] * rinv * wv[2 * j + 1] * __fdividef(zf.y, 1.f + __expf(-zf.y));
+          }
+          store8<TO>(dst + c8, y);
+        }
+      }
+      return true;
+    };
     for (int n = 0; n < Nc; ++n) {
       const int s = n & 1;
       const uint8_t* st = sm + s * STAGE_BYTES;
@@ -371,20 +489,56 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
 
       // then the output rows (lanes 0-63), overlapping the next chunk's products
       if (!p_rows) {
-        if (!wait_or_abort(&bar[B_OA], n & 1, status, 108, abort_flag, spin)) continue;
+        bool ok = wait_or_abort(&bar[B_OA], n & 1, status, 108, abort_flag, spin);
+        if (NORM) ok = !named_barrier_or(2, 128, !ok);  // the 128 row threads decide as one
+        if (!ok) continue;
         tc_fence_after();
         float OA[32];
         tmem_ld32(tl + TM_OA, OA);
         tc_fence_before();
         const int t = n * kC + row;
-        if (t < T) {
-          TO* dst = o + (((size_t)b * T + t) * Hv + hv) * kD + c0 + cb;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) OA[c] = (fo * OQ[c] + OA[c]) * inv_sigma;
+        for (int c = 0; c < 32; ++c) OA[c] = (fo * OQ[c] + OA[c]) * inv_sigma;
+        if (NORM) {
+          // the previous chunk's rows: the peer's sums arrived during this chunk step
+          if (n > 0 && !norm_finish(n - 1, row, half, cb, pend_part)) continue;
+          // this chunk's rows: sums of squares of the CTA's 64 columns to the peer, the
+          // rows themselves to shared memory until the next chunk
+          float ss = 0.f;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ss = fmaf(OA[c], OA[c], ss);
+          ssq[2 * row + half] = ss;
+          named_barrier(2, 128);
+          pend_part = ssq[2 * row] + ssq[2 * row + 1];
+          if (half == 0) {
+            const int slot = n & 1;
+            st_async_peer_f32(map_peer(xin + 64 * slot + row, peer), pend_part,
+                              map_peer(&bar[B_PX0 + slot], peer));
+          }
+          float* ob = obuf + row * 64 + cb;
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(ob + c) = make_float4(OA[c], OA[c + 1], OA[c + 2], OA[c + 3]);
+          // the gate of these rows, copied in while the next chunk runs
+          if (t < T) {
+            const bf16* zsrc = na.z + (((size_t)b * T + t) * Hv + hv) * kD + c0 + cb;
+            const uint32_t zdst = smem_u32(zbuf + row * 64 + cb);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(zdst + 16 * j),
+                           "l"(zsrc + 8 * j)
+                           : "memory");
+            asm volatile("cp.async.commit_group;" ::: "memory");
+          }
+        } else if (t < T) {
+          TO* dst = o + (((size_t)b * T + t) * Hv + hv) * kD + c0 + cb;
           store_row<TO>(dst, OA);
         }
       }
     }
+    // the last chunk's rows (NORM); every row thread calls this (the abort decision
+    // is taken inside by a vote of the 128)
+    if (NORM && !p_rows && Nc > 0) norm_finish(Nc - 1, row, half, cb, pend_part);
     if (!(range <= kF16Max)) report_range(status);
     if (ht != nullptr && !*abort_flag) {
       float* dst = ht + ((size_t)head * kD + row) * kD + c0 + cb;
@@ -401,12 +555,14 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
     tc_fence_after();
     tmem_dealloc(tmem, TM_COLS);
   }
+  // no CTA of the pair leaves while the other may still store into its shared memory
+  if (NORM) cluster_sync();
 }
 
 // ---------------------------------------------------------------- host side
-template <typename TO>
+template <typename TO, bool NORM>
 cudaError_t launch_t(const ChunkArgs& a, const WsLayout& L, const uint8_t* ws, int* status,
-                     cudaStream_t s) {
+                     const NormArgs& na, cudaStream_t s) {
   if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
   const uint64_t Tp = (uint64_t)((a.T + kC - 1) / kC) * kC;
   const uint64_t rv = (uint64_t)a.B * a.Hv * Tp, rk = (uint64_t)a.B * a.Hk * Tp;
@@ -417,12 +573,28 @@ cudaError_t launch_t(const ChunkArgs& a, const WsLayout& L, const uint8_t* ws, i
       !make_map_rows(&m.a, ws + L.a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kC, rv) ||
       !make_map_rows(&m.u, ws + L.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kD, rv))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(state_scan_tc_kernel<TO>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_TC_SMEM);
+  auto kern = state_scan_tc_kernel<TO, NORM>;
+  const uint32_t smem = NORM ? SCAN_TC_SMEM_NORM : SCAN_TC_SMEM;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const WaitFault f = wait_fault();
-  state_scan_tc_kernel<TO><<<dim3(2, a.B * a.Hv), kScanTcThreads, SCAN_TC_SMEM, s>>>(
-      m, ws, L, a.h0, a.T, a.Hk, a.Hv, static_cast<TO*>(a.o), a.ht, status, f.site, f.spin);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, a.B * a.Hv);
+  cfg.blockDim = dim3(kScanTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (NORM) {  // the two column halves of a head form a cluster
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  e = cudaLaunchKernelEx(&cfg, kern, m, ws, L, a.h0, a.T, a.Hk, a.Hv, static_cast<TO*>(a.o),
+                         a.ht, status, f.site, f.spin, na);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -431,8 +603,13 @@ cudaError_t launch_t(const ChunkArgs& a, const WsLayout& L, const uint8_t* ws, i
 cudaError_t launch_scan_tc(const ChunkArgs& a, const void* ws, int* status, cudaStream_t s) {
   const WsLayout L = ws_layout(a.B, a.T, a.Hk, a.Hv);
   const uint8_t* w = static_cast<const uint8_t*>(ws);
-  if (a.flags & GDN_OUT_F32) return launch_t<float>(a, L, w, status, s);
-  return launch_t<bf16>(a, L, w, status, s);
+  const NormArgs na{static_cast<const bf16*>(a.norm_z), a.norm_w, a.norm_eps};
+  const bool norm = a.norm_z != nullptr;
+  if (a.flags & GDN_OUT_F32)
+    return norm ? launch_t<float, true>(a, L, w, status, na, s)
+                : launch_t<float, false>(a, L, w, status, na, s);
+  return norm ? launch_t<bf16, true>(a, L, w, status, na, s)
+              : launch_t<bf16, false>(a, L, w, status, na, s);
 }
 
 }  // namespace gdn

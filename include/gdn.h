@@ -136,6 +136,30 @@ int gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* a,
                   int dtype, float scale, int flags, void* o, float* ht,
                   void* workspace, size_t ws_bytes, gdn_stream_t stream);
 
+/*
+ * gdn_chunk_fwd_gated_norm -- gdn_chunk_fwd whose output rows leave through the
+ * gated RMSNorm of the layer's output stage ("gated-deltanet-qwen3.5", section
+ * 输出门控与 RMSNorm: RMSNormGated(core_attn_out, z); "Qwen3.5" module skeleton,
+ * self.norm(core_attn_out, z)), per (token, value head) over the dv columns:
+ *   o = core / sqrt(mean(core^2) + eps) * norm_weight * SiLU(z),
+ * core being the output gdn_chunk_fwd writes.  On the bf16 dk = dv = 128 path the
+ * norm is applied in the scan's output epilogue before the single store of o (the
+ * two column-half CTAs of a head run as a cluster and exchange the rows' sums of
+ * squares through distributed shared memory), so core never reaches memory; the
+ * float32 / d = 64 path runs the forward and then gdn_rmsnorm_gated on o in place.
+ *   z           [B,T,Hv,dv] dtype, read; 16-byte aligned
+ *   norm_weight [dv] float32, read (shared by every head)
+ *   eps         0 <= eps <= 1 (1e-6 in the binding)
+ *   everything else as gdn_chunk_fwd (same workspace size).
+ * Returns as gdn_chunk_fwd.
+ */
+int gdn_chunk_fwd_gated_norm(const void* q, const void* k, const void* v, const void* a,
+                             const void* b, const float* A_log, const float* dt_bias,
+                             const float* h0, const void* z, const float* norm_weight,
+                             float eps, int B, int T, int Hk, int Hv, int dk, int dv,
+                             int dtype, float scale, int flags, void* o, float* ht,
+                             void* workspace, size_t ws_bytes, gdn_stream_t stream);
+
 /* Workspace bytes gdn_chunk_fwd needs for these sizes: for the tensor-core
  * path (bf16, dk = dv = 128) B*Hv*(Tp*896 + (Tp/64)*1040) + B*Hk*Tp*512 with
  * Tp = T rounded up to a multiple of 64 (per padded token and value head: a W
@@ -225,6 +249,22 @@ int gdn_recurrent_step(const void* x_qkv, const float* conv_w, void* conv_state,
                        const float* dt_bias, float* state, void* o, int N,
                        int Hk, int Hv, int dk, int dv, int dtype, float scale,
                        int flags, gdn_stream_t stream);
+
+/*
+ * gdn_recurrent_step_gated_norm -- gdn_recurrent_step with the gated RMSNorm of
+ * the output stage ("gated-deltanet-qwen3.5", 输出门控与 RMSNorm) fused into the
+ * store of o: o = core / sqrt(mean(core^2) + eps) * norm_weight * SiLU(z) per
+ * (sequence, value head) over dv (the CTA that forms a row holds all of it).
+ *   z           [N, Hv, dv] dtype, read (element aligned)
+ *   norm_weight [dv] float32; eps in [0, 1]
+ *   everything else as gdn_recurrent_step.
+ */
+int gdn_recurrent_step_gated_norm(const void* x_qkv, const float* conv_w, void* conv_state,
+                                  const void* a, const void* b, const float* A_log,
+                                  const float* dt_bias, float* state, const void* z,
+                                  const float* norm_weight, float eps, void* o, int N,
+                                  int Hk, int Hv, int dk, int dv, int dtype, float scale,
+                                  int flags, gdn_stream_t stream);
 
 /*
  * gdn_conv_prefill -- the causal depthwise conv1d (kernel 4) + SiLU over a

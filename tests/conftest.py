@@ -22,11 +22,17 @@ def pytest_sessionstart(session):
 
 # The parity tests of the newest entry points run after all the others, so that a
 # run that stops at its first failure (-x) has already reported the rest.
-_RUN_LAST = ("test_kda_gpu.py", "test_rmsnorm_gated_gpu.py", "test_varlen_gpu.py")
+_RUN_LAST = ("test_kda_gpu.py", "test_rmsnorm_gated_gpu.py", "test_varlen_gpu.py",
+             "test_gated_norm_fused_gpu.py")
 
 
 def pytest_collection_modifyitems(session, config, items):
-    items.sort(key=lambda it: os.path.basename(str(it.fspath)) in _RUN_LAST)  # stable
+    def rank(it):
+        name = os.path.basename(str(it.fspath))
+        if name == "test_zz_no_alloc.py":  # the no-allocation entry point's test: always last
+            return 2
+        return 1 if name in _RUN_LAST else 0
+    items.sort(key=rank)  # stable
 
 
 try:
