@@ -29,10 +29,11 @@
 // run as a cluster of two: each sends the sums of squares of its 64 columns of
 // the chunk's rows to the other through distributed shared memory (st.async into
 // the peer's buffer, counted as transaction bytes on the peer's mbarrier, so no
-// release fence waits on this thread's output stores).  The rows of chunk n wait
-// in shared memory, with their gate z copied in behind them, and are normalised
-// and stored during chunk n + 1, so the peer's sums have a whole chunk step to
-// arrive and the two CTAs' chains do not wait on each other.
+// release fence waits on output stores).  The output-row threads (TMEM lanes
+// 0-63) leave the chunk's rows in shared memory, with their gate z copied in
+// behind them; during the next chunk step the P-row threads, which run on the
+// other two SM sub-partitions and are idle after the state update, normalise and
+// store them.  The peer's sums have a whole chunk step to arrive.
 #include "chunk_layout.cuh"
 #include "common.cuh"
 #include "launch.h"
@@ -60,15 +61,20 @@ constexpr uint32_t OFF_SB = 2 * STAGE_BYTES;  // state (scaled) fp16, MN-major B
 constexpr uint32_t OFF_UT = OFF_SB + 16384;   // U~ fp16 [64][64]
 constexpr uint32_t OFF_US = OFF_UT + 8192;    // U~s fp16 [64][64]
 constexpr uint32_t OFF_RED = OFF_US + 8192;   // CTA max reduction (8 floats)
-constexpr uint32_t OFF_NRM = OFF_RED + 64;    // NORM: row sums of squares [64][2], and the
-                                              // peer's [2 chunk parities][64]
-constexpr uint32_t OFF_BAR = OFF_NRM + 1024;  // mbarriers + TMEM address
+constexpr uint32_t OFF_NRM = OFF_RED + 64;    // NORM: row sums of squares [2 chunks][64][2],
+                                              // and the peer's [4 chunks][64]
+constexpr uint32_t OFF_BAR = OFF_NRM + 2048;  // mbarriers + TMEM address
 constexpr uint32_t SCAN_TC_SMEM = OFF_BAR + 128 + 1024;
 // NORM only: the previous chunk's output rows before the norm, [64 rows][64] fp32,
-// and their gate z, [64 rows][64] bf16 (copied in one chunk ahead)
+// and their gate z, [64 rows][64] bf16 (copied in one chunk ahead).  A warp's lanes
+// own consecutive rows, so the rows are padded by 16 bytes: the 16-byte accesses of
+// eight lanes then fall in distinct banks.
+constexpr int kOS = 64 + 4;  // row stride of the row buffer (floats)
+constexpr int kZS = 64 + 8;  // row stride of the gate buffer (bf16)
 constexpr uint32_t OFF_OBUF = OFF_BAR + 128;
-constexpr uint32_t OFF_ZBUF = OFF_OBUF + 64 * 64 * 4;
-constexpr uint32_t SCAN_TC_SMEM_NORM = SCAN_TC_SMEM + 64 * 64 * 4 + 64 * 64 * 2;
+constexpr uint32_t OFF_ZBUF = OFF_OBUF + 64 * kOS * 4;
+constexpr uint32_t OFF_WBUF = OFF_ZBUF + 64 * kZS * 2;  // the CTA's 64 norm weights
+constexpr uint32_t SCAN_TC_SMEM_NORM = SCAN_TC_SMEM + 64 * kOS * 4 + 64 * kZS * 2 + 64 * 4;
 static_assert(ST_SC + kScal * 4 <= STAGE_BYTES, "stage layout");
 static_assert(SCAN_TC_SMEM_NORM <= 227 * 1024, "shared memory of the tcgen05 scan");
 
@@ -77,7 +83,7 @@ constexpr uint32_t TM_QP = 0, TM_OA = 64, TM_DS = 128, TM_COLS = 256;
 
 // barrier indices
 enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_QP, B_UT, B_DS, B_OA, B_S,
-       B_PX0, B_PX1,  // NORM: the peer's row sums of squares of a chunk have arrived
+       B_PX0, B_PX1, B_PX2, B_PX3,  // NORM: the peer's row sums of a chunk have arrived
        B_COUNT };
 static_assert(B_COUNT * 8 + 8 <= 128, "barrier area");
 
@@ -110,18 +116,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, in
                                               uint32_t spin) {
   for (uint32_t i = 0; i < spin; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 255u && *abort_flag) return false;
-  }
-  report_timeout(status, where);
-  *abort_flag = 1;
-  return false;
-}
-// The same with acquire at cluster scope (for a barrier a peer CTA arrives on).
-__device__ __forceinline__ bool wait_cluster_or_abort(uint64_t* bar, uint32_t parity, int* status,
-                                                      int where, volatile int* abort_flag,
-                                                      uint32_t spin) {
-  for (uint32_t i = 0; i < spin; ++i) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((i & 255u) == 255u && *abort_flag) return false;
   }
   report_timeout(status, where);
@@ -214,10 +208,8 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       mbar_init(&bar[i], (i == B_EMPTY0 || i == B_EMPTY1) ? 2 : 1);
     *abort_flag = 0;
     fence_mbar_init();
-    if (NORM) {  // each chunk's 64 peer sums arrive as 256 transaction bytes
-      mbar_arrive_expect_tx(&bar[B_PX0], 64 * 4);
-      mbar_arrive_expect_tx(&bar[B_PX1], 64 * 4);
-    }
+    if (NORM)  // each chunk's 64 peer sums arrive as 256 transaction bytes
+      for (int i = 0; i < 4; ++i) mbar_arrive_expect_tx(&bar[B_PX0 + i], 64 * 4);
     prefetch_tmap(&maps.q);
     prefetch_tmap(&maps.w);
     prefetch_tmap(&maps.k);
@@ -354,33 +346,45 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
     if (e == 0 && fault != kFaultScanState) mbar_arrive(&bar[B_S]);
 
     float OQ[32];
-    // NORM: sums of squares of the rows, this CTA's and the peer's; the pending rows
-    float* ssq = reinterpret_cast<float*>(sm + OFF_NRM);  // [64][2]
-    float* xin = ssq + 128;                               // [2 chunk parities][64], from the peer
+    // NORM: the rows' sums of squares, this CTA's [2 chunks][64][2] and the peer's
+    // [4 chunks][64]; the rows of the previous chunk and their gate z
+    float* ssq = reinterpret_cast<float*>(sm + OFF_NRM);
+    float* xin = ssq + 256;
     float* obuf = reinterpret_cast<float*>(sm + OFF_OBUF);
     bf16* zbuf = reinterpret_cast<bf16*>(sm + OFF_ZBUF);
+    float* wbuf = reinterpret_cast<float*>(sm + OFF_WBUF);
+    // the weights once, in shared memory: read from global memory inside the row
+    // loop, each load would wait behind the row's own output stores (may alias)
+    if (NORM && e < 64) wbuf[e] = na.w[c0 + e];  // first read after a barrier 1
     const uint32_t peer = NORM ? cluster_rank() ^ 1u : 0u;
-    float pend_part = 0.f;  // this CTA's sum of squares of the pending row
-    // Normalise and store the pending rows of chunk m (row threads, uniformly):
-    // y = o / sqrt(mean(o^2) + eps) * w * SiLU(z), the mean over both halves.
-    auto norm_finish = [&](int m, int r, int hf, int cbase, float part) -> bool {
-      const int slot = m & 1;
-      const bool got = wait_cluster_or_abort(&bar[B_PX0 + slot], (m >> 1) & 1, status, 109,
-                                             abort_flag, spin);
-      if (named_barrier_or(2, 128, !got)) return false;
-      const float rinv = rsqrtf((part + xin[64 * slot + r]) * (1.f / kD) + na.eps);
-      // the slot takes chunk m + 2 next; the peer sends it only after this CTA's sums
-      // of chunk m + 1, which follow this read (barrier 2 between)
-      if (r == 0 && hf == 0 && m + 2 < Nc) mbar_arrive_expect_tx(&bar[B_PX0 + slot], 64 * 4);
+    // Normalise and store row r of chunk m, columns cbase .. cbase + ncols - 1:
+    // y = o / sqrt(mean(o^2) + eps) * w * SiLU(z), the mean over both CTAs' halves.
+    // A row's 32 columns of a thread pair go 8 to the output-row thread (TMEM lanes
+    // 0-63, barrier 2 among them), which also has the chunk's own rows to take, and
+    // 24 to its P-row partner (barrier 3), so the norm's exponentials and divisions
+    // spread over all four SM sub-partitions; each group calls this uniformly.  The
+    // peer's sums arrive by st.async, whose transaction bytes complete the barrier
+    // phase: a CTA-scope wait sees them.
+    auto norm_rows = [&](int m, int r, int hf, int cbase, int ncols, int gbar) -> bool {
+      const int slot = m & 3;
+      const bool got =
+          wait_or_abort(&bar[B_PX0 + slot], (m >> 2) & 1, status, 109, abort_flag, spin);
+      if (named_barrier_or(gbar, 128, !got)) return false;
+      const float* sq = ssq + 128 * (m & 1);
+      const float rinv =
+          rsqrtf((sq[2 * r] + sq[2 * r + 1] + xin[64 * slot + r]) * (1.f / kD) + na.eps);
+      // the slot takes chunk m + 4 next: the peer sends that only after it has the
+      // sums of chunk m + 2 from this CTA, which leave after both groups' reads
+      if (gbar == 3 && r == 0 && hf == 0 && m + 4 < Nc)
+        mbar_arrive_expect_tx(&bar[B_PX0 + slot], 64 * 4);
       const int tm = m * kC + r;
-      asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's copy of z
       if (tm < T) {
-        const float* ob = obuf + r * 64 + cbase;
-        const bf16* zr = zbuf + r * 64 + cbase;
-        const float* wr = na.w + c0 + cbase;
+        const float* ob = obuf + r * kOS + cbase;
+        const bf16* zr = zbuf + r * kZS + cbase;
+        const float* wr = wbuf + cbase;
         TO* dst = o + (((size_t)b * T + tm) * Hv + hv) * kD + c0 + cbase;
 #pragma unroll
-        for (int c8 = 0; c8 < 32; c8 += 8) {
+        for (int c8 = 0; c8 < ncols; c8 += 8) {
           float y[8];
           const uint4 zz = *reinterpret_cast<const uint4*>(zr + c8);
           const float4 wa = *reinterpret_cast<const float4*>(wr + c8);
@@ -458,6 +462,9 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       tc_fence_before();
       named_barrier(1, kEpi);
       if (e == 0) mbar_arrive(&bar[B_UT]);
+      // NORM: the gate of the previous chunk's rows has landed before the barrier
+      // below, after which the P-row threads read it
+      if (NORM && !p_rows) asm volatile("cp.async.wait_all;" ::: "memory");
 
       // the state update first: it is what the next chunk waits for
       {
@@ -486,6 +493,13 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
         mbar_arrive(&bar[B_S]);
         mbar_arrive(&bar[B_EMPTY0 + s]);  // U and the factors of the stage are read
       }
+      // NORM: the P-row threads normalise and store their part of the previous
+      // chunk's output rows, then release the row buffer to the output-row threads
+      // (barrier 4: 128 arrive here, 128 wait before overwriting it)
+      if (NORM && p_rows && n > 0) {
+        if (!norm_rows(n - 1, row - 64, half, cb + 8, 24, 3)) *abort_flag = 1;
+        named_barrier_arrive(4, 256);
+      }
 
       // then the output rows (lanes 0-63), overlapping the next chunk's products
       if (!p_rows) {
@@ -500,29 +514,32 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
 #pragma unroll
         for (int c = 0; c < 32; ++c) OA[c] = (fo * OQ[c] + OA[c]) * inv_sigma;
         if (NORM) {
-          // the previous chunk's rows: the peer's sums arrived during this chunk step
-          if (n > 0 && !norm_finish(n - 1, row, half, cb, pend_part)) continue;
-          // this chunk's rows: sums of squares of the CTA's 64 columns to the peer, the
-          // rows themselves to shared memory until the next chunk
+          // this chunk's rows: the sums of squares of the CTA's 64 columns to the
+          // peer, the rows themselves to shared memory for the P-row threads
           float ss = 0.f;
 #pragma unroll
           for (int c = 0; c < 32; ++c) ss = fmaf(OA[c], OA[c], ss);
-          ssq[2 * row + half] = ss;
+          float* sq = ssq + 128 * (n & 1);
+          sq[2 * row + half] = ss;
           named_barrier(2, 128);
-          pend_part = ssq[2 * row] + ssq[2 * row + 1];
           if (half == 0) {
-            const int slot = n & 1;
-            st_async_peer_f32(map_peer(xin + 64 * slot + row, peer), pend_part,
+            const int slot = n & 3;
+            st_async_peer_f32(map_peer(xin + 64 * slot + row, peer), sq[2 * row] + sq[2 * row + 1],
                               map_peer(&bar[B_PX0 + slot], peer));
           }
-          float* ob = obuf + row * 64 + cb;
+          if (n > 0) {
+            // the rest of the previous chunk's rows, then wait for the P rows
+            if (!norm_rows(n - 1, row, half, cb, 8, 2)) *abort_flag = 1;
+            named_barrier(4, 256);
+          }
+          float* ob = obuf + row * kOS + cb;
 #pragma unroll
           for (int c = 0; c < 32; c += 4)
             *reinterpret_cast<float4*>(ob + c) = make_float4(OA[c], OA[c + 1], OA[c + 2], OA[c + 3]);
           // the gate of these rows, copied in while the next chunk runs
           if (t < T) {
             const bf16* zsrc = na.z + (((size_t)b * T + t) * Hv + hv) * kD + c0 + cb;
-            const uint32_t zdst = smem_u32(zbuf + row * 64 + cb);
+            const uint32_t zdst = smem_u32(zbuf + row * kZS + cb);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(zdst + 16 * j),
@@ -536,9 +553,19 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
         }
       }
     }
-    // the last chunk's rows (NORM); every row thread calls this (the abort decision
-    // is taken inside by a vote of the 128)
-    if (NORM && !p_rows && Nc > 0) norm_finish(Nc - 1, row, half, cb, pend_part);
+    // NORM: the last chunk's rows, by the P-row threads once the output-row threads'
+    // buffers and gate copies are complete (every epilogue thread gets here: the
+    // loop's exits are uniform)
+    if (NORM && Nc > 0) {
+      if (!p_rows) asm volatile("cp.async.wait_all;" ::: "memory");
+      const bool aborted = named_barrier_or(1, kEpi, *abort_flag != 0);  // one answer for all
+      if (!aborted) {
+        if (p_rows)
+          norm_rows(Nc - 1, row - 64, half, cb + 8, 24, 3);
+        else
+          norm_rows(Nc - 1, row, half, cb, 8, 2);
+      }
+    }
     if (!(range <= kF16Max)) report_range(status);
     if (ht != nullptr && !*abort_flag) {
       float* dst = ht + ((size_t)head * kD + row) * kD + c0 + cb;

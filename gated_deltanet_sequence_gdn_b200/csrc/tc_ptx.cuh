@@ -77,18 +77,6 @@ __device__ __forceinline__ void st_async_peer_f32(uint32_t addr, float v, uint32
                "r"(__float_as_uint(v)), "r"(bar_addr)
                : "memory");
 }
-// try_wait with acquire at cluster scope (sees the stores a peer released).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
 // Barrier over every thread of every CTA of the cluster.
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
@@ -157,6 +145,12 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // Barrier among `count` threads (a multiple of 32) on hardware barrier `id` (1..15).
 __device__ __forceinline__ void named_barrier(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Arrive on named barrier `id` of `count` threads without waiting (the waiting side
+// uses named_barrier); this thread's earlier memory accesses are performed relative
+// to the threads that wait.
+__device__ __forceinline__ void named_barrier_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 // Barrier among `count` threads on barrier `id` that also returns whether any of
 // them passed pred != 0 (the same answer in every thread).
