@@ -403,9 +403,10 @@ size_t gdn2_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype
  * bounded wait in a kernel expired since the last check (reported first when
  * both happened), GDN_ERR_RANGE if an intermediate of the tensor-core chunk
  * path left the fp16 operand range (inputs far outside the method's domain,
- * e.g. keys of norm >> 1 with GDN_QK_L2NORM off, or values of magnitude
- * ~1e6), or GDN_ERR_CUDA.  The word is shared by every call on the device, so a
- * code belongs to some call since the previous check.
+ * e.g. queries or keys of norm >> 1 with GDN_QK_L2NORM off; large values alone
+ * do not trigger it, the scan's power-of-2 range scale absorbs them), or
+ * GDN_ERR_CUDA.  The word is shared by every call on the device, so a code
+ * belongs to some call since the previous check.
  */
 int gdn_check_status(gdn_stream_t stream);
 
