@@ -266,7 +266,8 @@ def run_ours(args, rank, local_rank, world):
         extra["gate_prep_8k"] = measure_gate_prep(G, dev, stream, pk, args)
         extra["prefill_8k_gated_norm"] = measure_prefill_gated_norm(G, dev, stream, pk, args)
         # the newest secondary figures, last: a failure is reported here, not raised
-        for name, fn in (("kda_b4_4k", measure_kda), ("rmsnorm_gated_8k", measure_norm)):
+        for name, fn in (("kda_b4_4k", measure_kda), ("rmsnorm_gated_8k", measure_norm),
+                         ("bwd_8k", measure_bwd)):
             try:
                 extra[name] = fn(G, dev, stream, pk, args)
                 torch.cuda.synchronize()
@@ -466,6 +467,46 @@ def measure_gate_prep(G, dev, stream, pk, args):
             "steps": steps}
 
 
+# Dense products of one gdn_chunk_bwd call per 64-token chunk and value head at
+# d = 128, in multiply-adds: the chunk prep (K K^T, Q K^T, W, U: 4 C^2 d), the
+# forward state scan (W S0, K~^T U~: 2 C d^2), the reverse scan (K~ dS, (gamma Q)^T
+# dO, W^T dU~: 3 C d^2, A_qk^T dO: C^2 d) and the per-chunk gradients (dQ, dW, dK~,
+# Q S0: 4 C d^2; dA_qk, dA twice, dVb, dKb, dKK K twice, dQK K, dQK^T Q: 9 C^2 d;
+# dA A^T, A^T (.): 2 C^3) -> 2 (9 C d^2 + 14 C^2 d + 2 C^3) / C FLOP per token.
+BWD_FLOP_PER_TOKEN_HEAD = 2 * (9 * 64 * 128 * 128 + 14 * 64 * 64 * 128 + 2 * 64 ** 3) // 64
+
+
+def measure_bwd(G, dev, stream, pk, args):
+    """gdn_chunk_bwd on the prefill_8k layer (the backward of one gdn_chunk_fwd call,
+    output gradients ~ N(0,1)); float32 arithmetic on the CUDA cores, so its
+    roofline is the fp32 FMA rate: 148 SMs x 128 lanes x 2 FLOP x the SM clock."""
+    from gdn_synth import bwd_cotangents
+    w = WORKLOADS["prefill_8k"]
+    x = workload_inputs(w, dev)
+    ct = bwd_cotangents(w.B, w.T, w.Hv, w.d, w.d, w.dtype, 1501, dev)
+    ws = torch.empty(G.gdn_chunk_bwd_workspace_bytes(w.B, w.T, w.Hk, w.Hv, w.d, w.d),
+                     device=dev, dtype=torch.uint8)
+
+    def step():
+        G.gdn_chunk_bwd(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                        x["h0"], ct["do"], ct["dht"], workspace=ws, stream=stream)
+
+    steps = 3
+    total, per = time_steps(step, steps, 3, stream)
+    ms = sum(per) / len(per)
+    flop = BWD_FLOP_PER_TOKEN_HEAD * w.B * w.T * w.Hv
+    tf = flop / (ms / 1e3) / 1e12
+    peak = 148 * 128 * 2 * 1965e6 / 1e12  # clocks.max.sm of this part: 1965 MHz
+    del x, ct, ws
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_call": round(ms, 4),
+            "roofline": {"bound": "alu", "achieved": round(tf, 2), "peak": round(peak, 1),
+                         "unit": "TFLOP/s", "frac": round(tf / peak, 4),
+                         "flop_per_call": flop,
+                         "peak_src": "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock"},
+            "steps": steps}
+
+
 def measure_prefill_gated_norm(G, dev, stream, pk, args):
     """prefill_8k through gdn_chunk_fwd_gated_norm (the gated RMSNorm of the output
     stage fused into the scan's output store), beside gdn_chunk_fwd followed by the
@@ -573,6 +614,8 @@ def run_only(args, local_rank):
         r = measure_gate_prep(G, dev, stream, pk, args)
     elif args.only == "prefill_8k_gated_norm":
         r = measure_prefill_gated_norm(G, dev, stream, pk, args)
+    elif args.only == "bwd_8k":
+        r = measure_bwd(G, dev, stream, pk, args)
     else:
         r = measure_prefill(G, args.only, dev, stream, pk, args)
     G.gdn_check_status(stream)
@@ -650,7 +693,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["prefill_8k", "decode_256", "gdn2_b4_4k", "prefill_128k",
                                        "prefill_b8_16k", "conv_prefill_8k", "rmsnorm_gated_8k",
-                                       "kda_b4_4k", "gate_prep_8k", "prefill_8k_gated_norm"],
+                                       "kda_b4_4k", "gate_prep_8k", "prefill_8k_gated_norm",
+                                       "bwd_8k"],
                     default=None,
                     help="measure one secondary workload alone (profiling runs)")
     args = ap.parse_args()

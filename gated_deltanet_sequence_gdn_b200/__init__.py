@@ -22,6 +22,7 @@ __all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_chunk_workspace_bytes", "gdn_r
            "gdn_kda_chunk_workspace_bytes", "gdn_chunk_fwd_varlen",
            "gdn2_chunk_fwd", "gdn2_chunk_workspace_bytes", "gdn_chunk_fwd_noalloc",
            "gdn_chunk_fwd_gated_norm", "gdn_recurrent_step_gated_norm",
+           "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes",
            "gdn_check_status", "gdn_status", "gdn_test_set_wait_fault", "GDNError",
            "LIB_PATH", "lib", "F32", "BF16",
            "QK_L2NORM", "GATES_PRECOMPUTED", "OUT_F32"]
@@ -66,6 +67,9 @@ lib.gdn2_chunk_workspace_bytes.restype = _sz
 lib.gdn_chunk_fwd_gated_norm.argtypes = [_vp] * 10 + [_f] + [_i] * 7 + [_f, _i, _vp, _vp, _vp,
                                                                        _sz, _vp]
 lib.gdn_recurrent_step_gated_norm.argtypes = [_vp] * 10 + [_f, _vp] + [_i] * 6 + [_f, _i, _vp]
+lib.gdn_chunk_bwd.argtypes = [_vp] * 10 + [_i] * 7 + [_f, _i] + [_vp] * 9 + [_sz, _vp]
+lib.gdn_chunk_bwd_workspace_bytes.argtypes = [_i] * 6
+lib.gdn_chunk_bwd_workspace_bytes.restype = _sz
 lib.gdn_check_status.argtypes = [_vp]
 lib.gdn_test_set_wait_fault.argtypes = [_i, ctypes.c_uint]
 lib.gdn_test_set_wait_fault.restype = _i
@@ -235,6 +239,52 @@ def gdn_chunk_fwd_gated_norm(q, k, v, a, b, A_log, dt_bias, h0, z, norm_weight, 
                                         float(scale), flags, _p(o), _p(ht), _p(workspace),
                                         ws_bytes, _stream(stream)), "gdn_chunk_fwd_gated_norm")
     return o, ht
+
+
+def gdn_chunk_bwd_workspace_bytes(B, T, Hk, Hv, dk, dv):
+    return lib.gdn_chunk_bwd_workspace_bytes(B, T, Hk, Hv, dk, dv)
+
+
+def gdn_chunk_bwd(q, k, v, a, b, A_log, dt_bias, h0, do, dht=None, *, scale=None, l2norm=True,
+                  gates_precomputed=False, want_dh0=True, workspace=None, stream=None):
+    """Gradients of sum(o * do) + sum(ht * dht) for gdn_chunk_fwd's (o, ht) on the same
+    inputs (see include/gdn.h).  Returns a dict of float32 tensors dq, dk [B,T,Hk,dk],
+    dv [B,T,Hv,dv], da, db [B,T,Hv] (with gates_precomputed: with respect to g and
+    beta), dA_log, ddt_bias [Hv] (None with gates_precomputed) and dh0 [B,Hv,dk,dv]
+    (None unless want_dh0)."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dt = q.dtype
+    scale = dk ** -0.5 if scale is None else scale
+    _need(k, dt, q.shape, "k")
+    _need(v, dt, (B, T, Hv, dv), "v")
+    _need(do, dt, (B, T, Hv, dv), "do")
+    gdt = torch.float32 if gates_precomputed else dt
+    _need(a, gdt, (B, T, Hv), "a")
+    _need(b, gdt, (B, T, Hv), "b")
+    if h0 is not None:
+        _need(h0, torch.float32, (B, Hv, dk, dv), "h0")
+    if dht is not None:
+        _need(dht, torch.float32, (B, Hv, dk, dv), "dht")
+    f32 = dict(device=q.device, dtype=torch.float32)
+    out = {"dq": torch.empty((B, T, Hk, dk), **f32), "dk": torch.empty((B, T, Hk, dk), **f32),
+           "dv": torch.empty((B, T, Hv, dv), **f32), "da": torch.empty((B, T, Hv), **f32),
+           "db": torch.empty((B, T, Hv), **f32),
+           "dA_log": None if gates_precomputed else torch.empty((Hv,), **f32),
+           "ddt_bias": None if gates_precomputed else torch.empty((Hv,), **f32),
+           "dh0": torch.empty((B, Hv, dk, dv), **f32) if want_dh0 else None}
+    flags = (QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
+    ws_need = gdn_chunk_bwd_workspace_bytes(B, T, Hk, Hv, dk, dv)
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.gdn_chunk_bwd(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(dt_bias), _p(h0),
+                             _p(do), _p(dht), B, T, Hk, Hv, dk, dv, _dtype_code(dt),
+                             float(scale), flags, _p(out["dq"]), _p(out["dk"]), _p(out["dv"]),
+                             _p(out["da"]), _p(out["db"]), _p(out["dA_log"]),
+                             _p(out["ddt_bias"]), _p(out["dh0"]), _p(workspace), ws_bytes,
+                             _stream(stream)), "gdn_chunk_bwd")
+    return out
 
 
 def gdn_chunk_fwd_noalloc(q, k, v, a, b, A_log=None, dt_bias=None, h0=None, *, scale=None,

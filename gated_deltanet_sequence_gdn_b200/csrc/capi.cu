@@ -188,6 +188,52 @@ int gdn_chunk_fwd_gated_norm(const void* q, const void* k, const void* v, const 
   return from_cuda(launch_rmsnorm_gated(o, z, norm_weight, o, rows, dv, dtype, eps, s));
 }
 
+size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv) {
+  if (B <= 0 || T <= 0 || Hk <= 0 || Hv <= 0 || dk != dv || !ok_head_dim(dk)) return 0;
+  return bwd_workspace_bytes(B, T, Hk, Hv, dk);
+}
+
+int gdn_chunk_bwd(const void* q, const void* k, const void* v, const void* a, const void* b,
+                  const float* A_log, const float* dt_bias, const float* h0, const void* dout,
+                  const float* dht, int B, int T, int Hk, int Hv, int dk, int dv, int dtype,
+                  float scale, int flags, float* dq, float* dk_out, float* dv_out, float* da,
+                  float* db, float* dA_log, float* ddt_bias, float* dh0, void* workspace,
+                  size_t ws_bytes, gdn_stream_t stream) {
+  if (B < 0 || T < 0 || Hk <= 0 || Hv <= 0 || !ok_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  if (flags & ~(GDN_QK_L2NORM | GDN_GATES_PRECOMPUTED)) return GDN_ERR_INVALID_ARG;
+  if (dk != dv || !ok_head_dim(dk) || Hv % Hk != 0) return GDN_ERR_UNSUPPORTED;
+  if (!ok_opt(h0) || !ok_opt(dht) || !ok_opt(dh0)) return GDN_ERR_INVALID_ARG;
+  const bool pre = (flags & GDN_GATES_PRECOMPUTED) != 0;
+  if (!pre && (!ok_elem(A_log, 4) || !ok_elem(dt_bias, 4) || !ok_elem(dA_log, 4) ||
+               !ok_elem(ddt_bias, 4)))
+    return GDN_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((long)B * T == 0) {  // no tokens: dh0 = dht, and nothing flows to the gates' parameters
+    if (dh0) {
+      const cudaError_t e = launch_copy_state(dht, dh0, (size_t)B * Hv * dk * dv, s);
+      if (e != cudaSuccess) return from_cuda(e);
+    }
+    if (!pre) {
+      cudaError_t e = cudaMemsetAsync(dA_log, 0, sizeof(float) * Hv, s);
+      if (e == cudaSuccess) e = cudaMemsetAsync(ddt_bias, 0, sizeof(float) * Hv, s);
+      return from_cuda(e);
+    }
+    return GDN_OK;
+  }
+  const size_t ges = pre ? 4 : elem_size(dtype);
+  if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_elem(a, ges) || !ok_elem(b, ges) ||
+      !ok_ptr(dout) || !ok_ptr(dq) || !ok_ptr(dk_out) || !ok_ptr(dv_out) || !ok_elem(da, 4) ||
+      !ok_elem(db, 4))
+    return GDN_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned16(workspace) ||
+      ws_bytes < gdn_chunk_bwd_workspace_bytes(B, T, Hk, Hv, dk, dv))
+    return GDN_ERR_WORKSPACE;
+  BwdArgs args{q,    k,     v,     a,  b,      A_log,  dt_bias, h0,     dout,
+               dht,  B,     T,     Hk, Hv,     dk,     dtype,   scale,  flags,
+               dq,   dk_out, dv_out, da, db,   dA_log, ddt_bias, dh0};
+  return from_cuda(launch_chunk_bwd(args, workspace, s));
+}
+
 // Sequence i of a packed batch: the arguments of a one-sequence gdn_chunk_fwd call
 // on its token range [t0, t0 + Ti) and its own initial / final state.
 static ChunkArgs varlen_seq(const ChunkArgs& all, long long t0, int Ti, int i) {

@@ -85,4 +85,20 @@ WaitFault wait_fault();
 
 cudaError_t launch_copy_state(const float* h0, float* ht, size_t n, cudaStream_t s);
 
+// Arguments of the chunk backward (gdn_chunk_bwd); D = dk = dv.
+struct BwdArgs {
+  const void *q, *k, *v, *a, *b;
+  const float *A_log, *dt_bias, *h0;
+  const void* dout;
+  const float* dht;
+  int B, T, Hk, Hv, D, dtype;
+  float scale;
+  int flags;
+  float *dq, *dk, *dv, *da, *db, *dA_log, *ddt_bias, *dh0;
+};
+// Workspace bytes of the backward for these sizes (fp32 intermediates).
+size_t bwd_workspace_bytes(int B, int T, int Hk, int Hv, int D);
+// The backward on the CUDA cores (T >= 1; the caller handles T = 0).
+cudaError_t launch_chunk_bwd(const BwdArgs& a, void* workspace, cudaStream_t s);
+
 }  // namespace gdn

@@ -183,6 +183,14 @@ def rmsnorm_inputs(B, T, Hv, dv, dtype, seed, device="cpu"):
     }
 
 
+def bwd_cotangents(B, T, Hv, dv, dk, dtype, seed, device="cpu", dht=True):
+    """Gradients at the outputs of one GDN call, for its backward: do [B,T,Hv,dv]
+    ~ N(0,1) in ``dtype``; dht [B,Hv,dk,dv] ~ N(0,1) fp32 (or None)."""
+    g = _gen(seed, device)
+    return {"do": _randn((B, T, Hv, dv), g, device, dtype),
+            "dht": _randn((B, Hv, dk, dv), g, device, torch.float32) if dht else None}
+
+
 def workload_inputs(w: Workload, device="cpu"):
     if w.kind == "gdn":
         return gdn_inputs(w.B, w.T, w.Hk, w.Hv, w.d, w.dtype, w.seed, device, h0=w.h0)

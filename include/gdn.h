@@ -297,6 +297,48 @@ int gdn_conv_prefill(const void* x_qkv, const float* conv_w, void* conv_state,
                      int dk, int dv, int dtype, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_bwd -- the backward of gdn_chunk_fwd: the gradients of
+ * sum(o * dout) + sum(ht * dht) for the forward's o and final state ht, by
+ * reverse-mode differentiation of the WY chunk form ("Gated DeltaNet-2",
+ * sections 高效训练：WY 算法依然成立 and Gate-aware 反向传播, with the scalar
+ * decay of GDN; "Qwen3.5" (rainlin-net), GDN详解, for the gates and norms).  It
+ * recomputes the forward's per-chunk factors and every chunk's start state,
+ * carries the state gradient from the last chunk to the first, forms the
+ * per-chunk gradients, then applies the chain rule through the L2 norms of q, k
+ * and through the gates.  fp32 arithmetic on the CUDA cores for both input
+ * types.
+ *   q, k [B,T,Hk,dk], v [B,T,Hv,dv], a, b [B,T,Hv], A_log, dt_bias, h0, flags
+ *     (GDN_QK_L2NORM, GDN_GATES_PRECOMPUTED) and scale: as given to
+ *     gdn_chunk_fwd, read.  dk = dv = 64 or 128 (else GDN_ERR_UNSUPPORTED).
+ *   dout [B,T,Hv,dv] dtype, read: the gradient at o.
+ *   dht [B,Hv,dk,dv] float32, read; NULL = zero gradient at the final state.
+ *   dq, dk_out [B,T,Hk,dk] float32, written (summed over the value heads of
+ *     each key head); dv_out [B,T,Hv,dv] float32, written.
+ *   da, db [B,T,Hv] float32, written: the gradients with respect to the gate
+ *     logits a and b, or with GDN_GATES_PRECOMPUTED with respect to g and beta.
+ *   dA_log, ddt_bias [Hv] float32, written (summed over batch and tokens);
+ *     unused (may be NULL) with GDN_GATES_PRECOMPUTED.
+ *   dh0 [B,Hv,dk,dv] float32, written; NULL = not stored.
+ *   workspace / ws_bytes: device scratch owned by the caller, 16-byte aligned, at
+ *     least gdn_chunk_bwd_workspace_bytes() bytes, overwritten; too small or
+ *     misaligned -> GDN_ERR_WORKSPACE, nothing launched.
+ *   T = 0 writes dh0 = dht (or zeros) and zero dA_log, ddt_bias.
+ * Errors as for gdn_chunk_fwd; asynchronous on `stream`.
+ */
+int gdn_chunk_bwd(const void* q, const void* k, const void* v, const void* a,
+                  const void* b, const float* A_log, const float* dt_bias,
+                  const float* h0, const void* dout, const float* dht, int B, int T,
+                  int Hk, int Hv, int dk, int dv, int dtype, float scale, int flags,
+                  float* dq, float* dk_out, float* dv_out, float* da, float* db,
+                  float* dA_log, float* ddt_bias, float* dh0, void* workspace,
+                  size_t ws_bytes, gdn_stream_t stream);
+
+/* Workspace bytes gdn_chunk_bwd needs: fp32 intermediates, about
+ * B*T*(Hv*(12*dv*4 + (2*dk*dv*4 + 8*64*64*4)/64) + Hk*2*dk*4) bytes (5.5 GB at
+ * B=1, T=8192, Hk=16, Hv=64, d=128); 0 for T = 0, B = 0 or unsupported sizes. */
+size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv);
+
+/*
  * gdn_chunk_fwd_varlen -- gdn_chunk_fwd over a packed batch of N sequences of
  * different lengths: sequence i is tokens cu_seqlens[i] .. cu_seqlens[i+1] - 1
  * of the packed arrays, with its own initial and final state, and its chunks

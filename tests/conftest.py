@@ -23,7 +23,7 @@ def pytest_sessionstart(session):
 # The parity tests of the newest entry points run after all the others, so that a
 # run that stops at its first failure (-x) has already reported the rest.
 _RUN_LAST = ("test_kda_gpu.py", "test_rmsnorm_gated_gpu.py", "test_varlen_gpu.py",
-             "test_gated_norm_fused_gpu.py")
+             "test_gated_norm_fused_gpu.py", "test_bwd_gpu.py")
 
 
 def pytest_collection_modifyitems(session, config, items):

@@ -256,3 +256,33 @@ def test_host_pipeline_rejects_bad_arguments():
     assert f(*bad) == 0                                      # B = 0: nothing to do
     bad = list(args); bad[20] = FAKE; bad[21] = 1024
     assert f(*bad) == -5                                     # scratch too small
+
+
+def _bwd(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, a=FAKE, b=FAKE, A_log=FAKE, dt_bias=FAKE, h0=None,
+                do=FAKE, dht=None, B=1, T=64, Hk=2, Hv=4, dk=128, dv=128, dtype=1, scale=0.1,
+                flags=1, dq=FAKE, dk_out=FAKE, dv_out=FAKE, da=FAKE, db=FAKE, dA_log=FAKE,
+                ddt_bias=FAKE, dh0=None, ws=None, ws_bytes=0)
+    args.update(kw)
+    names = ("q", "k", "v", "a", "b", "A_log", "dt_bias", "h0", "do", "dht", "B", "T", "Hk",
+             "Hv", "dk", "dv", "dtype", "scale", "flags", "dq", "dk_out", "dv_out", "da",
+             "db", "dA_log", "ddt_bias", "dh0", "ws", "ws_bytes")
+    return G.lib.gdn_chunk_bwd(*[args[n] for n in names], None)
+
+
+def test_backward_arguments_checked_before_any_launch():
+    """gdn_chunk_bwd refuses bad arguments and a short workspace on the host."""
+    assert _bwd(dk=128, dv=64) == -2          # GDN_ERR_UNSUPPORTED: dk != dv
+    assert _bwd(dk=96, dv=96) == -2           # head size outside {64, 128}
+    assert _bwd(Hk=3, Hv=4) == -2             # Hv % Hk != 0
+    assert _bwd(flags=4) == -1                # GDN_OUT_F32 has no meaning here
+    assert _bwd(dtype=7) == -1
+    assert _bwd(A_log=None) == -1             # gates from logits need A_log ...
+    assert _bwd(dA_log=None) == -1            # ... and somewhere for its gradient
+    assert _bwd(dq=FAKE + 4) == -1            # misaligned output
+    assert _bwd() == -5                       # no workspace
+    need = G.lib.gdn_chunk_bwd_workspace_bytes(1, 64, 2, 4, 128, 128)
+    assert need > 0
+    assert _bwd(ws=FAKE, ws_bytes=need - 1) == -5
+    assert G.lib.gdn_chunk_bwd_workspace_bytes(1, 0, 2, 4, 128, 128) == 0
+    assert G.lib.gdn_chunk_bwd_workspace_bytes(1, 64, 2, 4, 128, 64) == 0
