@@ -78,24 +78,25 @@ enum { kScNone = 0, kScBeta = 1, kScBetaGamma = 2, kScGamma = 3 };
 enum { kMaskNone = 0, kMaskLower = 1, kMaskStrict = 2 };
 
 struct BmmArgs {
-  Opnd x, y;          // out[64 x N] = alpha op(x)[64 x K] diag(ks) op(y)[K x N]
+  Opnd x, y;          // out[M x N] = alpha op(x)[M x K] diag(ks) op(y)[K x N]
   float* out;
-  int out_kind;       // kTV (N = D) or kCC (N = 64)
-  int N, K;
+  int out_kind;       // kTV (M = 64, N = D), kCC (M = N = 64) or kDD (M = N = D)
+  int M, N, K;
   float alpha;
-  int kscale, rscale, cscale, mask;  // kscale needs K = 64, cscale N = 64
+  int kscale, rscale, cscale, mask;  // kscale needs K = 64, rscale M = 64, cscale N = 64
   int accumulate;
   const float2* gb;   // (G, beta) per [B*Hv][Tp]
 };
 
 // Batched product, one 64 x 64 output tile per CTA (blockIdx.x: (h, c),
-// blockIdx.y: column tile); 256 threads with 4 x 4 outputs each; K in steps of 32
-// through shared memory.
-__global__ void __launch_bounds__(256) bmm_kernel(BmmArgs P, Dims d) {
+// blockIdx.y: column tile, blockIdx.z: row tile); 256 threads with 4 x 4 outputs
+// each; K in steps of 32 through shared memory.
+template <bool XT, bool YT>
+__global__ void __launch_bounds__(256, 3) bmm_kernel(BmmArgs P, Dims d) {
   __shared__ __align__(16) float Xs[32][68];
   __shared__ __align__(16) float Ys[32][68];
   __shared__ float sv[3][kC];
-  const int z = blockIdx.x, n0 = blockIdx.y * 64, tid = threadIdx.x;
+  const int z = blockIdx.x, n0 = blockIdx.y * 64, m0 = blockIdx.z * 64, tid = threadIdx.x;
   const int h = z / d.Nc, c = z % d.Nc;
   const float* X = P.x.p + opnd_off(P.x.kind, z, d);
   const float* Y = P.y.p + opnd_off(P.y.kind, z, d);
@@ -120,23 +121,13 @@ __global__ void __launch_bounds__(256) bmm_kernel(BmmArgs P, Dims d) {
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
   for (int k0 = 0; k0 < P.K; k0 += 32) {
     __syncthreads();
-    for (int i = tid; i < 2048; i += 256) {
-      int m, k;
-      if (!P.x.t) {
-        m = i >> 5, k = i & 31;
-        Xs[k][m] = X[(size_t)m * ldx + k0 + k];
-      } else {
-        k = i >> 6, m = i & 63;
-        Xs[k][m] = X[(size_t)(k0 + k) * ldx + m];
-      }
-      int n;
-      if (!P.y.t) {
-        k = i >> 6, n = i & 63;
-        Ys[k][n] = Y[(size_t)(k0 + k) * ldy + n0 + n];
-      } else {
-        n = i >> 5, k = i & 31;
-        Ys[k][n] = Y[(size_t)(n0 + n) * ldy + k0 + k];
-      }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = tid + 256 * u;
+      if (!XT) Xs[i & 31][i >> 5] = X[(size_t)(m0 + (i >> 5)) * ldx + k0 + (i & 31)];
+      else Xs[i >> 6][i & 63] = X[(size_t)(k0 + (i >> 6)) * ldx + m0 + (i & 63)];
+      if (!YT) Ys[i >> 6][i & 63] = Y[(size_t)(k0 + (i >> 6)) * ldy + n0 + (i & 63)];
+      else Ys[i & 31][i >> 5] = Y[(size_t)(n0 + (i >> 5)) * ldy + k0 + (i & 31)];
     }
     __syncthreads();
 #pragma unroll 8
@@ -152,8 +143,9 @@ __global__ void __launch_bounds__(256) bmm_kernel(BmmArgs P, Dims d) {
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
   }
-  float* out = P.out + (P.out_kind == kCC ? (size_t)z * kC * kC
-                                          : ((size_t)h * d.Tp + (size_t)c * kC) * d.D);
+  float* out = P.out + (P.out_kind == kCC   ? (size_t)z * kC * kC
+                        : P.out_kind == kDD ? (size_t)z * d.D * d.D + (size_t)m0 * d.D
+                                            : ((size_t)h * d.Tp + (size_t)c * kC) * d.D);
   const int ldo = P.out_kind == kCC ? kC : d.D;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -161,7 +153,7 @@ __global__ void __launch_bounds__(256) bmm_kernel(BmmArgs P, Dims d) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int col = n0 + 4 * tn + j;
-      float v = P.alpha * acc[i][j] * sv[1][r];
+      float v = P.alpha * acc[i][j] * (P.rscale != kScNone ? sv[1][r] : 1.f);
       if (P.cscale != kScNone) v *= sv[2][col];
       if ((P.mask == kMaskLower && col > r) || (P.mask == kMaskStrict && col >= r)) v = 0.f;
       float* o = out + (size_t)r * ldo + col;
@@ -297,6 +289,31 @@ __global__ void __launch_bounds__(64) tri_inverse_kernel(float* Lb) {
 }
 
 // ------------------------------------------------------------------ the scans
+// 16-byte asynchronous copies of a [64][D] fp32 tile into shared rows of D + 4.
+template <int D>
+__device__ __forceinline__ void tile_async(float* dst, const float* src, int tid) {
+#pragma unroll
+  for (int u = 0; u < kC * D / 4 / 256; ++u) {
+    const int i = tid + 256 * u, r = i / (D / 4), q4 = i % (D / 4);
+    const uint32_t sa = (uint32_t)__cvta_generic_to_shared(dst + r * (D + 4) + 4 * q4);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa),
+                 "l"(src + (size_t)r * D + 4 * q4)
+                 : "memory");
+  }
+}
+__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void async_wait_prev() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
+// Shared memory of the scans: W and K tiles twice (the next chunk's land while
+// the current one is used), the state (or its gradient) slice and a 64 x kNS
+// row block.
+template <int D>
+constexpr size_t scan_smem_bytes() {
+  return (size_t)(4 * kC * (D + 4) + D * (kNS + 4) + kC * (kNS + 4) + kC) * 4;
+}
+
 // Forward: S0 of every chunk (the state before it, slice of kNS columns) and
 // U~ = U - W S0 (in place over U).  One CTA per (slice, h); 256 threads.
 template <int D>
@@ -304,28 +321,33 @@ __global__ void __launch_bounds__(256) fwd_state_scan_kernel(const float* Wm, fl
                                                              const float* KN, const float2* GB,
                                                              const float* h0, float* S0, Dims d) {
   extern __shared__ __align__(16) float sm[];
-  float* Ws = sm;                       // [64][D + 4]
-  float* Ks = Ws + kC * (D + 4);        // [64][D + 4]
-  float* S = Ks + kC * (D + 4);         // [D][kNS + 4]
-  float* Us = S + D * (kNS + 4);        // [64][kNS + 4]
-  float* ratio = Us + kC * (kNS + 4);   // [64]
+  float* Wb = sm;                          // [2][64][D + 4]
+  float* Kb = Wb + 2 * kC * (D + 4);       // [2][64][D + 4]
+  float* S = Kb + 2 * kC * (D + 4);        // [D][kNS + 4]
+  float* Us = S + D * (kNS + 4);           // [64][kNS + 4]
+  float* ratio = Us + kC * (kNS + 4);      // [64]
   const int n0 = blockIdx.x * kNS, h = blockIdx.y, tid = threadIdx.x;
   const int b = h / d.Hv, hv = h % d.Hv, kh = b * d.Hk + hv / (d.Hv / d.Hk);
   for (int i = tid; i < D * kNS; i += 256) {
     const int k = i / kNS, n = i % kNS;
     S[k * (kNS + 4) + n] = h0 ? h0[((size_t)h * D + k) * D + n0 + n] : 0.f;
   }
+  auto rowv = [&](int c) { return ((size_t)h * d.Tp + (size_t)c * kC) * D; };
+  auto rowk = [&](int c) { return ((size_t)kh * d.Tp + (size_t)c * kC) * D; };
+  tile_async<D>(Wb, Wm + rowv(0), tid);
+  tile_async<D>(Kb, KN + rowk(0), tid);
+  async_commit();
   const int tm = tid >> 4, tn = tid & 15;
   for (int c = 0; c < d.Nc; ++c) {
-    const size_t z = (size_t)h * d.Nc + c;
-    const size_t rv = ((size_t)h * d.Tp + (size_t)c * kC) * D;
-    const size_t rk = ((size_t)kh * d.Tp + (size_t)c * kC) * D;
-    __syncthreads();  // the previous chunk is done with Ws, Ks, Us and S
-    for (int i = tid; i < kC * D; i += 256) {
-      const int r = i / D, k = i % D;
-      Ws[r * (D + 4) + k] = Wm[rv + i];
-      Ks[r * (D + 4) + k] = KN[rk + i];
+    const size_t z = (size_t)h * d.Nc + c, rv = rowv(c);
+    const float* Ws = Wb + (c & 1) * kC * (D + 4);
+    const float* Ks = Kb + (c & 1) * kC * (D + 4);
+    if (c + 1 < d.Nc) {  // the next chunk's tiles, into the other buffers
+      tile_async<D>(Wb + ((c + 1) & 1) * kC * (D + 4), Wm + rowv(c + 1), tid);
+      tile_async<D>(Kb + ((c + 1) & 1) * kC * (D + 4), KN + rowk(c + 1), tid);
     }
+    async_commit();
+    async_wait_prev();  // this chunk's tiles have landed (this thread's copies)
     if (tid < kC) {
       const float G = GB[(size_t)h * d.Tp + (size_t)c * kC + tid].x;
       const float GC = GB[(size_t)h * d.Tp + (size_t)c * kC + kC - 1].x;
@@ -335,7 +357,7 @@ __global__ void __launch_bounds__(256) fwd_state_scan_kernel(const float* Wm, fl
       const int k = i / kNS, n = i % kNS;
       S0[z * D * D + (size_t)k * D + n0 + n] = S[k * (kNS + 4) + n];
     }
-    __syncthreads();
+    __syncthreads();  // every thread's copies, S and ratio are visible
     // U~ = U - W S0: rows 4 tm .. 4 tm + 3, columns 4 tn .. 4 tn + 3
     {
       float acc[4][4];
@@ -357,18 +379,16 @@ __global__ void __launch_bounds__(256) fwd_state_scan_kernel(const float* Wm, fl
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = 4 * tm + i;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int n = 4 * tn + j;
-          const float u = Um[rv + (size_t)r * D + n0 + n] - acc[i][j];
-          Um[rv + (size_t)r * D + n0 + n] = u;
-          Us[r * (kNS + 4) + n] = u;
-        }
+        const float4 u4 = *reinterpret_cast<const float4*>(&Um[rv + (size_t)r * D + n0 + 4 * tn]);
+        const float4 o4 = make_float4(u4.x - acc[i][0], u4.y - acc[i][1], u4.z - acc[i][2],
+                                      u4.w - acc[i][3]);
+        *reinterpret_cast<float4*>(&Um[rv + (size_t)r * D + n0 + 4 * tn]) = o4;
+        *reinterpret_cast<float4*>(&Us[r * (kNS + 4) + 4 * tn]) = o4;
       }
     }
     __syncthreads();
-    // S <- gamma_C S + K~^T U~: rows (d_k) 8 tm' .. + 7 with tm' = tid / 16 over D / 8
-    // groups, columns 4 tn .. + 3
+    // S <- gamma_C S + K~^T U~: rows (d_k) k0 .. k0 + 7 with k0 = 8 tm (+ 128),
+    // columns 4 tn .. + 3
     {
       const float gC = expf(GB[(size_t)h * d.Tp + (size_t)c * kC + kC - 1].x);
       for (int k0 = 8 * tm; k0 < D; k0 += 128) {
@@ -380,13 +400,16 @@ __global__ void __launch_bounds__(256) fwd_state_scan_kernel(const float* Wm, fl
         for (int r = 0; r < kC; ++r) {
           const float4 u4 = *reinterpret_cast<const float4*>(&Us[r * (kNS + 4) + 4 * tn]);
           const float rr = ratio[r];
+          const float4 ka = *reinterpret_cast<const float4*>(&Ks[r * (D + 4) + k0]);
+          const float4 kb = *reinterpret_cast<const float4*>(&Ks[r * (D + 4) + k0 + 4]);
+          const float kv[8] = {ka.x * rr, ka.y * rr, ka.z * rr, ka.w * rr,
+                               kb.x * rr, kb.y * rr, kb.z * rr, kb.w * rr};
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float kv = Ks[r * (D + 4) + k0 + i] * rr;
-            acc[i][0] = fmaf(kv, u4.x, acc[i][0]);
-            acc[i][1] = fmaf(kv, u4.y, acc[i][1]);
-            acc[i][2] = fmaf(kv, u4.z, acc[i][2]);
-            acc[i][3] = fmaf(kv, u4.w, acc[i][3]);
+            acc[i][0] = fmaf(kv[i], u4.x, acc[i][0]);
+            acc[i][1] = fmaf(kv[i], u4.y, acc[i][1]);
+            acc[i][2] = fmaf(kv[i], u4.z, acc[i][2]);
+            acc[i][3] = fmaf(kv[i], u4.w, acc[i][3]);
           }
         }
 #pragma unroll
@@ -398,60 +421,59 @@ __global__ void __launch_bounds__(256) fwd_state_scan_kernel(const float* Wm, fl
           }
       }
     }
+    __syncthreads();  // the buffers of this chunk are free for the chunk after next
   }
 }
 
 // Reverse: dS1 of every chunk (the state gradient after it) and dU~; the final dS
-// is dh0.  One CTA per (slice, h); 256 threads.
+// is dh0.  The terms that do not depend on dS come precomputed: P1 = A_qk^T dO in
+// dUt (replaced by dU~ in place) and P2 = (diag(gamma) Q)^T dO per chunk.  One
+// CTA per (slice, h); 256 threads.
 template <int D>
-__global__ void __launch_bounds__(256) rev_state_scan_kernel(
-    const float* Wm, const float* KN, const float* QN, const float* Aq, const float* dO32,
-    const float2* GB, const float* dht, float* dS1, float* dUt, float* dh0, Dims d) {
+__global__ void __launch_bounds__(256) rev_state_scan_kernel(const float* Wm, const float* KN,
+                                                             const float* P2, const float2* GB,
+                                                             const float* dht, float* dS1,
+                                                             float* dUt, float* dh0, Dims d) {
   extern __shared__ __align__(16) float sm[];
-  float* Ws = sm;                          // [64][D + 4]
-  float* Ks = Ws + kC * (D + 4);           // [64][D + 4]
-  float* Qs = Ks + kC * (D + 4);           // [64][D + 4]
-  float* As = Qs + kC * (D + 4);           // [64][65]  A_qk
-  float* dS = As + kC * (kC + 1);          // [D][kNS + 4]
-  float* dOs = dS + D * (kNS + 4);         // [64][kNS + 4]
-  float* dUs = dOs + kC * (kNS + 4);       // [64][kNS + 4]
+  float* Wb = sm;                          // [2][64][D + 4]
+  float* Kb = Wb + 2 * kC * (D + 4);       // [2][64][D + 4]
+  float* dS = Kb + 2 * kC * (D + 4);       // [D][kNS + 4]
+  float* dUs = dS + D * (kNS + 4);         // [64][kNS + 4]
   float* ratio = dUs + kC * (kNS + 4);     // [64]
-  float* gam = ratio + kC;                 // [64]
   const int n0 = blockIdx.x * kNS, h = blockIdx.y, tid = threadIdx.x;
   const int b = h / d.Hv, hv = h % d.Hv, kh = b * d.Hk + hv / (d.Hv / d.Hk);
   for (int i = tid; i < D * kNS; i += 256) {
     const int k = i / kNS, n = i % kNS;
     dS[k * (kNS + 4) + n] = dht ? dht[((size_t)h * D + k) * D + n0 + n] : 0.f;
   }
+  auto rowv = [&](int c) { return ((size_t)h * d.Tp + (size_t)c * kC) * D; };
+  auto rowk = [&](int c) { return ((size_t)kh * d.Tp + (size_t)c * kC) * D; };
+  const int last = d.Nc - 1;
+  tile_async<D>(Wb + (last & 1) * kC * (D + 4), Wm + rowv(last), tid);
+  tile_async<D>(Kb + (last & 1) * kC * (D + 4), KN + rowk(last), tid);
+  async_commit();
   const int tm = tid >> 4, tn = tid & 15;
-  for (int c = d.Nc - 1; c >= 0; --c) {
-    const size_t z = (size_t)h * d.Nc + c;
-    const size_t rv = ((size_t)h * d.Tp + (size_t)c * kC) * D;
-    const size_t rk = ((size_t)kh * d.Tp + (size_t)c * kC) * D;
-    __syncthreads();
-    for (int i = tid; i < kC * D; i += 256) {
-      const int r = i / D, k = i % D;
-      Ws[r * (D + 4) + k] = Wm[rv + i];
-      Ks[r * (D + 4) + k] = KN[rk + i];
-      Qs[r * (D + 4) + k] = QN[rk + i];
+  for (int c = last; c >= 0; --c) {
+    const size_t z = (size_t)h * d.Nc + c, rv = rowv(c);
+    const float* Ws = Wb + (c & 1) * kC * (D + 4);
+    const float* Ks = Kb + (c & 1) * kC * (D + 4);
+    if (c > 0) {  // the previous chunk's tiles, into the other buffers
+      tile_async<D>(Wb + ((c - 1) & 1) * kC * (D + 4), Wm + rowv(c - 1), tid);
+      tile_async<D>(Kb + ((c - 1) & 1) * kC * (D + 4), KN + rowk(c - 1), tid);
     }
-    for (int i = tid; i < kC * kC; i += 256) As[(i >> 6) * (kC + 1) + (i & 63)] = Aq[z * kC * kC + i];
-    for (int i = tid; i < kC * kNS; i += 256) {
-      const int r = i / kNS, n = i % kNS;
-      dOs[r * (kNS + 4) + n] = dO32[rv + (size_t)r * D + n0 + n];
-    }
+    async_commit();
+    async_wait_prev();
     if (tid < kC) {
       const float G = GB[(size_t)h * d.Tp + (size_t)c * kC + tid].x;
       const float GC = GB[(size_t)h * d.Tp + (size_t)c * kC + kC - 1].x;
       ratio[tid] = expf(GC - G);
-      gam[tid] = expf(G);
     }
     for (int i = tid; i < D * kNS; i += 256) {
       const int k = i / kNS, n = i % kNS;
       dS1[z * D * D + (size_t)k * D + n0 + n] = dS[k * (kNS + 4) + n];
     }
     __syncthreads();
-    // dU~ = K~ dS1 + A_qk^T dO
+    // dU~ = K~ dS1 + P1
     {
       float acc[4][4];
 #pragma unroll
@@ -471,33 +493,18 @@ __global__ void __launch_bounds__(256) rev_state_scan_kernel(
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float rr = ratio[4 * tm + i];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] *= rr;
-      }
-      for (int j = 0; j < kC; ++j) {
-        const float4 o4 = *reinterpret_cast<const float4*>(&dOs[j * (kNS + 4) + 4 * tn]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float a = As[j * (kC + 1) + 4 * tm + i];  // A_qk[j][r], r = 4 tm + i
-          acc[i][0] = fmaf(a, o4.x, acc[i][0]);
-          acc[i][1] = fmaf(a, o4.y, acc[i][1]);
-          acc[i][2] = fmaf(a, o4.z, acc[i][2]);
-          acc[i][3] = fmaf(a, o4.w, acc[i][3]);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
         const int r = 4 * tm + i;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          dUs[r * (kNS + 4) + 4 * tn + j] = acc[i][j];
-          dUt[rv + (size_t)r * D + n0 + 4 * tn + j] = acc[i][j];
-        }
+        const float rr = ratio[r];
+        float* g = &dUt[rv + (size_t)r * D + n0 + 4 * tn];
+        const float4 p4 = *reinterpret_cast<const float4*>(g);
+        const float4 o4 = make_float4(fmaf(rr, acc[i][0], p4.x), fmaf(rr, acc[i][1], p4.y),
+                                      fmaf(rr, acc[i][2], p4.z), fmaf(rr, acc[i][3], p4.w));
+        *reinterpret_cast<float4*>(g) = o4;
+        *reinterpret_cast<float4*>(&dUs[r * (kNS + 4) + 4 * tn]) = o4;
       }
     }
     __syncthreads();
-    // dS <- gamma_C dS + (diag(gamma) Q)^T dO - W^T dU~
+    // dS <- gamma_C dS + P2 - W^T dU~
     {
       const float gC = expf(GB[(size_t)h * d.Tp + (size_t)c * kC + kC - 1].x);
       for (int k0 = 8 * tm; k0 < D; k0 += 128) {
@@ -507,30 +514,33 @@ __global__ void __launch_bounds__(256) rev_state_scan_kernel(
 #pragma unroll
           for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
         for (int r = 0; r < kC; ++r) {
-          const float4 o4 = *reinterpret_cast<const float4*>(&dOs[r * (kNS + 4) + 4 * tn]);
           const float4 u4 = *reinterpret_cast<const float4*>(&dUs[r * (kNS + 4) + 4 * tn]);
-          const float gr = gam[r];
+          const float4 wa = *reinterpret_cast<const float4*>(&Ws[r * (D + 4) + k0]);
+          const float4 wb = *reinterpret_cast<const float4*>(&Ws[r * (D + 4) + k0 + 4]);
+          const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float qv = Qs[r * (D + 4) + k0 + i] * gr;
-            const float wv = Ws[r * (D + 4) + k0 + i];
-            acc[i][0] = fmaf(qv, o4.x, fmaf(-wv, u4.x, acc[i][0]));
-            acc[i][1] = fmaf(qv, o4.y, fmaf(-wv, u4.y, acc[i][1]));
-            acc[i][2] = fmaf(qv, o4.z, fmaf(-wv, u4.z, acc[i][2]));
-            acc[i][3] = fmaf(qv, o4.w, fmaf(-wv, u4.w, acc[i][3]));
+            acc[i][0] = fmaf(wv[i], u4.x, acc[i][0]);
+            acc[i][1] = fmaf(wv[i], u4.y, acc[i][1]);
+            acc[i][2] = fmaf(wv[i], u4.z, acc[i][2]);
+            acc[i][3] = fmaf(wv[i], u4.w, acc[i][3]);
           }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 8; ++i) {
+          const float4 p4 =
+              *reinterpret_cast<const float4*>(&P2[z * D * D + (size_t)(k0 + i) * D + n0 + 4 * tn]);
+          const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             float* s = &dS[(k0 + i) * (kNS + 4) + 4 * tn + j];
-            *s = fmaf(gC, *s, acc[i][j]);
+            *s = fmaf(gC, *s, pv[j] - acc[i][j]);
           }
+        }
       }
     }
+    __syncthreads();
   }
-  __syncthreads();
   if (dh0)
     for (int i = tid; i < D * kNS; i += 256) {
       const int k = i / kNS, n = i % kNS;
@@ -539,26 +549,25 @@ __global__ void __launch_bounds__(256) rev_state_scan_kernel(
 }
 
 // ------------------------------------------------------------------ chunk-local
-// Per-row sums over the D columns of two token-row operands: out[r] = sum_d
-// X[r][d] Y[r][d], for the 64 rows of (h, c).  4 threads per row.
-__device__ __forceinline__ float row_dot(const float* X, const float* Y, int r, int part, int D) {
-  float s = 0.f;
-  for (int i = part; i < D; i += 4) s = fmaf(X[(size_t)r * D + i], Y[(size_t)r * D + i], s);
-  s += __shfl_xor_sync(0xffffffffu, s, 1);
-  s += __shfl_xor_sync(0xffffffffu, s, 2);
-  return s;
-}
-
 // Per chunk scalars and rows (float4 per row of (h, c)): x = dgam, y = dbeta,
 // z = dG collected from the Gamma masks, w unused.  dgam starts as
 // rowsum(dO o Q S0); dgC = <dS1, S0> per chunk.
+// The row kernels below take one warp per token row (8 rows per warp), the lanes
+// over the row's D columns, so every access is a coalesced row segment.
 __global__ void __launch_bounds__(256) dgam_kernel(const float* dO32, const float* QS,
                                                    float4* VB, Dims d) {
-  const int z = blockIdx.x, h = z / d.Nc, c = z % d.Nc, tid = threadIdx.x;
+  const int z = blockIdx.x, h = z / d.Nc, c = z % d.Nc;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t rv = ((size_t)h * d.Tp + (size_t)c * kC) * d.D;
-  const int r = tid >> 2, part = tid & 3;
-  const float s = row_dot(dO32 + rv, QS + rv, r, part, d.D);
-  if (part == 0) VB[(size_t)z * kC + r] = make_float4(s, 0.f, 0.f, 0.f);
+  for (int r = warp; r < kC; r += 8) {
+    float s = 0.f;
+    for (int i = lane; i < d.D; i += 32) {
+      const size_t e = rv + (size_t)r * d.D + i;
+      s = fmaf(dO32[e], QS[e], s);
+    }
+    s = warp_sum(s);
+    if (lane == 0) VB[(size_t)z * kC + r] = make_float4(s, 0.f, 0.f, 0.f);
+  }
 }
 
 __global__ void __launch_bounds__(256) dgc_kernel(const float* dS1, const float* S0, float* SC,
@@ -585,26 +594,31 @@ __global__ void __launch_bounds__(256) vb_kernel(const float* dVb, const float* 
                                                  const float* V32, const float* KN,
                                                  const float2* GB, float* dK, float4* VB,
                                                  float* dv_out, Dims d) {
-  const int z = blockIdx.x, h = z / d.Nc, c = z % d.Nc, tid = threadIdx.x;
+  const int z = blockIdx.x, h = z / d.Nc, c = z % d.Nc;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = h / d.Hv, hv = h % d.Hv, kh = b * d.Hk + hv / (d.Hv / d.Hk);
   const size_t rv = ((size_t)h * d.Tp + (size_t)c * kC) * d.D;
   const size_t rk = ((size_t)kh * d.Tp + (size_t)c * kC) * d.D;
-  const int r = tid >> 2, part = tid & 3;
-  const float2 gb = GB[(size_t)h * d.Tp + (size_t)c * kC + r];
-  const float be = gb.y, gm = expf(gb.x);
-  const float s1 = row_dot(dVb + rv, V32 + rv, r, part, d.D);
-  const float s2 = row_dot(dKb + rv, KN + rk, r, part, d.D);
-  const int t = c * kC + r;
-  for (int i = part; i < d.D; i += 4) {
-    const size_t e = rv + (size_t)r * d.D + i;
-    dK[e] = be * gm * dKb[e];
-    if (t < d.T) dv_out[(((size_t)b * d.T + t) * d.Hv + hv) * d.D + i] = be * dVb[e];
-  }
-  if (part == 0) {
-    float4 v = VB[(size_t)z * kC + r];
-    v.x += be * s2;
-    v.y = s1 + gm * s2;
-    VB[(size_t)z * kC + r] = v;
+  for (int r = warp; r < kC; r += 8) {
+    const float2 gb = GB[(size_t)h * d.Tp + (size_t)c * kC + r];
+    const float be = gb.y, gm = expf(gb.x);
+    const int t = c * kC + r;
+    float s1 = 0.f, s2 = 0.f;
+    for (int i = lane; i < d.D; i += 32) {
+      const size_t e = rv + (size_t)r * d.D + i;
+      const float vb = dVb[e], kb = dKb[e];
+      s1 = fmaf(vb, V32[e], s1);
+      s2 = fmaf(kb, KN[rk + (size_t)r * d.D + i], s2);
+      dK[e] = be * gm * kb;
+      if (t < d.T) dv_out[(((size_t)b * d.T + t) * d.Hv + hv) * d.D + i] = be * vb;
+    }
+    s1 = warp_sum(s1), s2 = warp_sum(s2);
+    if (lane == 0) {
+      float4 v = VB[(size_t)z * kC + r];
+      v.x += be * s2;
+      v.y = s1 + gm * s2;
+      VB[(size_t)z * kC + r] = v;
+    }
   }
 }
 
@@ -660,22 +674,27 @@ __global__ void __launch_bounds__(256) dg_kernel(const float* dKt, const float* 
                                                  Dims d) {
   __shared__ float dG[kC], rrat[kC];
   const int z = blockIdx.x, h = z / d.Nc, c = z % d.Nc, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int b = h / d.Hv, hv = h % d.Hv, kh = b * d.Hk + hv / (d.Hv / d.Hk);
   const size_t rv = ((size_t)h * d.Tp + (size_t)c * kC) * d.D;
   const size_t rk = ((size_t)kh * d.Tp + (size_t)c * kC) * d.D;
-  const int r = tid >> 2, part = tid & 3;
   const float GC = GB[(size_t)h * d.Tp + (size_t)c * kC + kC - 1].x;
-  const float G = GB[(size_t)h * d.Tp + (size_t)c * kC + r].x;
-  const float ratio = expf(GC - G), gm = expf(G);
-  const float dratio = row_dot(dKt + rv, KN + rk, r, part, d.D);
-  for (int i = part; i < d.D; i += 4) {
-    const size_t e = rv + (size_t)r * d.D + i;
-    dK[e] = fmaf(ratio, dKt[e], dK[e]);
-  }
-  if (part == 0) {
-    const float4 v = VB[(size_t)z * kC + r];
-    dG[r] = v.z + v.x * gm - dratio * ratio;
-    rrat[r] = dratio * ratio;
+  for (int r = warp; r < kC; r += 8) {
+    const float G = GB[(size_t)h * d.Tp + (size_t)c * kC + r].x;
+    const float ratio = expf(GC - G), gm = expf(G);
+    float dratio = 0.f;
+    for (int i = lane; i < d.D; i += 32) {
+      const size_t e = rv + (size_t)r * d.D + i;
+      const float kt = dKt[e];
+      dratio = fmaf(kt, KN[rk + (size_t)r * d.D + i], dratio);
+      dK[e] = fmaf(ratio, kt, dK[e]);
+    }
+    dratio = warp_sum(dratio);
+    if (lane == 0) {
+      const float4 v = VB[(size_t)z * kC + r];
+      dG[r] = v.z + v.x * gm - dratio * ratio;
+      rrat[r] = dratio * ratio;
+    }
   }
   __syncthreads();
   if (tid < 32) {  // the last row's gamma_C terms, then the reverse cumulative sum
@@ -796,7 +815,7 @@ __global__ void __launch_bounds__(256) reduce_gates_kernel(const float2* R, floa
 // ------------------------------------------------------------------ host side
 struct BwdLayout {
   size_t QN, KN, V32, dO32, Wm, Um, dUt, dQ, dW, dKt, QS, dVb, dKb, dK;  // token rows
-  size_t S0, dS1;                                                          // D x D per chunk
+  size_t S0, dS1, P2;                                                      // D x D per chunk
   size_t KK, QK, Am, Aq, dAqk, dA, T1, dL;                                 // 64 x 64 per chunk
   size_t GB, DG, VB, SC, R;
   size_t total;
@@ -817,7 +836,7 @@ BwdLayout bwd_layout(int B, int T, int Hk, int Hv, int D) {
   L.V32 = take(tv), L.dO32 = take(tv), L.Wm = take(tv), L.Um = take(tv), L.dUt = take(tv);
   L.dQ = take(tv), L.dW = take(tv), L.dKt = take(tv), L.QS = take(tv), L.dVb = take(tv);
   L.dKb = take(tv), L.dK = take(tv);
-  L.S0 = take(dd), L.dS1 = take(dd);
+  L.S0 = take(dd), L.dS1 = take(dd), L.P2 = take(dd);
   L.KK = take(cc), L.QK = take(cc), L.Am = take(cc), L.Aq = take(cc), L.dAqk = take(cc);
   L.dA = take(cc), L.T1 = take(cc), L.dL = take(cc);
   L.GB = take((size_t)B * Hv * Tp * 8), L.DG = take((size_t)B * Hv * Tp * 8);
@@ -869,9 +888,13 @@ static cudaError_t run_bwd(const BwdArgs& a, uint8_t* ws, cudaStream_t s) {
   }
   auto bmm = [&](Opnd x, Opnd y, size_t out, int out_kind, int K, float alpha, int ks, int rs,
                  int cs, int mask, int accumulate) -> cudaError_t {
-    BmmArgs P{x, y, F(out), out_kind, out_kind == kCC ? kC : a.D, K, alpha, ks, rs, cs, mask,
-              accumulate, GB};
-    bmm_kernel<<<dim3(Z, P.N / 64), 256, 0, s>>>(P, d);
+    const int M = out_kind == kDD ? a.D : kC, N = out_kind == kCC ? kC : a.D;
+    BmmArgs P{x, y, F(out), out_kind, M, N, K, alpha, ks, rs, cs, mask, accumulate, GB};
+    const dim3 grid(Z, N / 64, M / 64);
+    if (x.t && y.t) bmm_kernel<true, true><<<grid, 256, 0, s>>>(P, d);
+    else if (x.t) bmm_kernel<true, false><<<grid, 256, 0, s>>>(P, d);
+    else if (y.t) bmm_kernel<false, true><<<grid, 256, 0, s>>>(P, d);
+    else bmm_kernel<false, false><<<grid, 256, 0, s>>>(P, d);
     return cudaGetLastError();
   };
   const float* QN = F(L.QN);
@@ -888,42 +911,40 @@ static cudaError_t run_bwd(const BwdArgs& a, uint8_t* ws, cudaStream_t s) {
     return e;
   if ((e = bmm(O(L.Am, kCC, 0), O(L.V32, kTV, 0), L.Um, kTV, kC, 1.f, kScBeta, 0, 0, 0, 0)))
     return e;
-  // the two scans
+  // the two scans; the reverse one takes its dS-independent terms precomputed:
+  // P1 = A_qk^T dO (into dUt) and P2 = (diag(gamma) Q)^T dO
+  if ((e = bmm(O(L.Aq, kCC, 1), O(L.dO32, kTV, 0), L.dUt, kTV, kC, 1.f, 0, 0, 0, 0, 0)))
+    return e;
+  if ((e = bmm(Opnd{QN, kTK, 1}, O(L.dO32, kTV, 0), L.P2, kDD, kC, 1.f, kScGamma, 0, 0, 0, 0)))
+    return e;
   {
-    const size_t smf = a.D == 128 ? (size_t)(2 * kC * (128 + 4) + 128 * (kNS + 4) +
-                                             kC * (kNS + 4) + kC) * 4
-                                  : (size_t)(2 * kC * (64 + 4) + 64 * (kNS + 4) +
-                                             kC * (kNS + 4) + kC) * 4;
-    const size_t smr = a.D == 128 ? (size_t)(3 * kC * (128 + 4) + kC * (kC + 1) +
-                                             128 * (kNS + 4) + 2 * kC * (kNS + 4) + 2 * kC) * 4
-                                  : (size_t)(3 * kC * (64 + 4) + kC * (kC + 1) +
-                                             64 * (kNS + 4) + 2 * kC * (kNS + 4) + 2 * kC) * 4;
     const dim3 grid(a.D / kNS, a.B * a.Hv);
     if (a.D == 128) {
+      constexpr size_t sm = scan_smem_bytes<128>();
       e = cudaFuncSetAttribute(fwd_state_scan_kernel<128>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf);
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
       if (e) return e;
-      fwd_state_scan_kernel<128><<<grid, 256, smf, s>>>(F(L.Wm), F(L.Um), KN, GB, a.h0,
-                                                          F(L.S0), d);
+      fwd_state_scan_kernel<128><<<grid, 256, sm, s>>>(F(L.Wm), F(L.Um), KN, GB, a.h0, F(L.S0),
+                                                         d);
       GDN_BWD_CHECK();
       e = cudaFuncSetAttribute(rev_state_scan_kernel<128>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
       if (e) return e;
-      rev_state_scan_kernel<128><<<grid, 256, smr, s>>>(F(L.Wm), KN, QN, F(L.Aq), F(L.dO32), GB,
-                                                          a.dht, F(L.dS1), F(L.dUt), a.dh0, d);
+      rev_state_scan_kernel<128><<<grid, 256, sm, s>>>(F(L.Wm), KN, F(L.P2), GB, a.dht, F(L.dS1),
+                                                         F(L.dUt), a.dh0, d);
       GDN_BWD_CHECK();
     } else {
+      constexpr size_t sm = scan_smem_bytes<64>();
       e = cudaFuncSetAttribute(fwd_state_scan_kernel<64>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf);
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
       if (e) return e;
-      fwd_state_scan_kernel<64><<<grid, 256, smf, s>>>(F(L.Wm), F(L.Um), KN, GB, a.h0,
-                                                         F(L.S0), d);
+      fwd_state_scan_kernel<64><<<grid, 256, sm, s>>>(F(L.Wm), F(L.Um), KN, GB, a.h0, F(L.S0), d);
       GDN_BWD_CHECK();
       e = cudaFuncSetAttribute(rev_state_scan_kernel<64>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
       if (e) return e;
-      rev_state_scan_kernel<64><<<grid, 256, smr, s>>>(F(L.Wm), KN, QN, F(L.Aq), F(L.dO32), GB,
-                                                         a.dht, F(L.dS1), F(L.dUt), a.dh0, d);
+      rev_state_scan_kernel<64><<<grid, 256, sm, s>>>(F(L.Wm), KN, F(L.P2), GB, a.dht, F(L.dS1),
+                                                        F(L.dUt), a.dh0, d);
       GDN_BWD_CHECK();
     }
   }
