@@ -20,6 +20,7 @@ import torch
 __all__ = ["gdn_gate_prep", "gdn_chunk_fwd", "gdn_chunk_workspace_bytes", "gdn_recurrent_step",
            "gdn_conv_prefill", "gdn_rmsnorm_gated", "gdn_kda_chunk_fwd",
            "gdn_kda_chunk_workspace_bytes", "gdn_chunk_fwd_varlen",
+           "gdn_chunk_varlen_workspace_bytes",
            "gdn2_chunk_fwd", "gdn2_chunk_workspace_bytes", "gdn_chunk_fwd_noalloc",
            "gdn_chunk_fwd_gated_norm", "gdn_recurrent_step_gated_norm",
            "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes",
@@ -57,6 +58,8 @@ lib.gdn_conv_prefill.argtypes = [_vp] * 6 + [_i] * 7 + [_vp]
 lib.gdn_rmsnorm_gated.argtypes = [_vp] * 4 + [ctypes.c_long, _i, _i, _f, _vp]
 lib.gdn_chunk_fwd_varlen.argtypes = ([_vp] * 8 + [ctypes.POINTER(ctypes.c_longlong)] + [_i] * 6
                                      + [_f, _i, _vp, _vp, _vp, _sz, _vp])
+lib.gdn_chunk_varlen_workspace_bytes.argtypes = [ctypes.POINTER(ctypes.c_longlong)] + [_i] * 6
+lib.gdn_chunk_varlen_workspace_bytes.restype = _sz
 lib.gdn_kda_chunk_fwd.argtypes = [_vp] * 8 + [_i] * 6 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
 lib.gdn_kda_chunk_workspace_bytes.argtypes = [_i] * 7
 lib.gdn_kda_chunk_workspace_bytes.restype = _sz
@@ -418,6 +421,17 @@ def gdn2_chunk_fwd(q, k, v, a, b_logit, w_logit, A_log=None, dt_bias=None, h0=No
     return o, ht
 
 
+def gdn_chunk_varlen_workspace_bytes(cu_seqlens, Hk, Hv, dk, dv, dtype) -> int:
+    """Device workspace bytes gdn_chunk_fwd_varlen needs for these N + 1 token
+    offsets (0 when the call needs none)."""
+    cu = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    if len(cu) < 2:
+        return 0
+    arr = (ctypes.c_longlong * len(cu))(*cu)
+    return int(lib.gdn_chunk_varlen_workspace_bytes(arr, len(cu) - 1, Hk, Hv, dk, dv,
+                                                    _dtype_code(dtype)))
+
+
 def gdn_chunk_fwd_varlen(q, k, v, a, b, A_log, dt_bias, h0, cu_seqlens, *, scale=None,
                          l2norm=True, gates_precomputed=False, out_f32=False, o=None, ht=None,
                          want_ht=True, workspace=None, stream=None):
@@ -447,12 +461,11 @@ def gdn_chunk_fwd_varlen(q, k, v, a, b, A_log, dt_bias, h0, cu_seqlens, *, scale
         ht = torch.empty((N, Hv, dk, dv), device=q.device, dtype=torch.float32)
     flags = ((QK_L2NORM if l2norm else 0) | (GATES_PRECOMPUTED if gates_precomputed else 0)
              | (OUT_F32 if out_f32 else 0))
-    longest = max([cu[i + 1] - cu[i] for i in range(N)] + [0])
-    ws_need = gdn_chunk_workspace_bytes(1, longest, Hk, Hv, dk, dv, dt) if longest else 0
+    cu_arr = (ctypes.c_longlong * len(cu))(*cu)
+    ws_need = gdn_chunk_varlen_workspace_bytes(cu, Hk, Hv, dk, dv, dt)
     if workspace is None and ws_need > 0:
         workspace = torch.empty(ws_need, device=q.device, dtype=torch.uint8)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    cu_arr = (ctypes.c_longlong * len(cu))(*cu)
     _check(lib.gdn_chunk_fwd_varlen(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(dt_bias),
                                     _p(h0), cu_arr, N, Hk, Hv, dk, dv, _dtype_code(dt),
                                     float(scale), flags, _p(o), _p(ht), _p(workspace), ws_bytes,

@@ -3,8 +3,11 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <memory>
 #include <mutex>
+#include <new>
 
+#include "chunk_layout.cuh"
 #include "common.cuh"
 #include "launch.h"
 
@@ -258,6 +261,44 @@ static ChunkArgs varlen_seq(const ChunkArgs& all, long long t0, int Ti, int i) {
   return c;
 }
 
+// Sequences per launch pair of a packed batch: at most kVarlenMaxSeqs, and few
+// enough that the scan's grid (2, sequences x Hv) stays within 65535 rows.
+static int varlen_group(int Hv) { return Hv > 0 && 65535 / Hv < kVarlenMaxSeqs ? 65535 / Hv : kVarlenMaxSeqs; }
+
+// Chunks of the packed batch's sequences i0 .. i1 - 1 (each starts a new chunk).
+static long long varlen_chunks(const long long* cu, int i0, int i1) {
+  long long nv = 0;
+  for (int i = i0; i < i1; ++i) nv += (cu[i + 1] - cu[i] + kC - 1) / kC;
+  return nv;
+}
+
+// cu_seqlens starts at 0, does not decrease, and the packed token count fits an int.
+static bool varlen_offsets_ok(const long long* cu, int N) {
+  if (cu == nullptr || cu[0] != 0) return false;
+  for (int i = 0; i < N; ++i)
+    if (cu[i + 1] < cu[i]) return false;
+  return cu[N] <= 0x7fffffffLL;
+}
+
+size_t gdn_chunk_varlen_workspace_bytes(const long long* cu_seqlens, int N, int Hk, int Hv,
+                                        int dk, int dv, int dtype) {
+  if (N <= 0 || Hk <= 0 || Hv <= 0 || !ok_dtype(dtype) || !varlen_offsets_ok(cu_seqlens, N))
+    return 0;
+  ChunkArgs probe{};
+  probe.B = 1, probe.T = 1, probe.Hk = Hk, probe.Hv = Hv, probe.dk = dk, probe.dv = dv;
+  probe.dtype = dtype;
+  if (!chunk_mma_supported(probe)) return 0;  // the CUDA-core path needs none
+  const int G = varlen_group(Hv);
+  size_t need = 0;
+  for (int i0 = 0; i0 < N; i0 += G) {
+    const long long nv = varlen_chunks(cu_seqlens, i0, i0 + G < N ? i0 + G : N);
+    if (nv > 0x7fffffffLL / kC) return 0;
+    const size_t b = varlen_ws_bytes((int)nv, Hk, Hv);
+    need = b > need ? b : need;
+  }
+  return need;
+}
+
 int gdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, const void* a,
                          const void* b, const float* A_log, const float* dt_bias,
                          const float* h0, const long long* cu_seqlens, int N, int Hk, int Hv,
@@ -265,29 +306,60 @@ int gdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, const void
                          void* workspace, size_t ws_bytes, gdn_stream_t stream) {
   if (N < 0 || !ok_dtype(dtype)) return GDN_ERR_INVALID_ARG;
   if (N == 0) return GDN_OK;
-  if (cu_seqlens == nullptr || cu_seqlens[0] != 0) return GDN_ERR_INVALID_ARG;
-  for (int i = 0; i < N; ++i) {
-    const long long Ti = cu_seqlens[i + 1] - cu_seqlens[i];
-    if (Ti < 0 || Ti > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
-  }
+  if (!varlen_offsets_ok(cu_seqlens, N)) return GDN_ERR_INVALID_ARG;
   const ChunkArgs all{q, k, v, a, b, nullptr, A_log, dt_bias, h0, 1, 0, Hk, Hv, dk, dv,
                       dtype, scale, flags, o, ht};
   // every sequence is checked before anything is enqueued
   for (int i = 0; i < N; ++i) {
     const int Ti = (int)(cu_seqlens[i + 1] - cu_seqlens[i]);
-    const ChunkArgs c = varlen_seq(all, cu_seqlens[i], Ti, i);
-    const int st = validate_chunk(c, false);
+    const int st = validate_chunk(varlen_seq(all, cu_seqlens[i], Ti, i), false);
     if (st != GDN_OK) return st;
-    if (Ti > 0 && chunk_mma_supported(c) &&
-        (workspace == nullptr || !aligned16(workspace) ||
-         ws_bytes < chunk_mma_workspace_bytes(1, Ti, Hk, Hv)))
-      return GDN_ERR_WORKSPACE;
   }
   cudaStream_t s = (cudaStream_t)stream;
-  for (int i = 0; i < N; ++i) {
-    const int Ti = (int)(cu_seqlens[i + 1] - cu_seqlens[i]);
-    const int st = run_chunk(varlen_seq(all, cu_seqlens[i], Ti, i), false, workspace, ws_bytes, s);
-    if (st != GDN_OK) return st;
+  ChunkArgs probe = all;
+  probe.T = 1;
+  if (!chunk_mma_supported(probe)) {  // the CUDA-core path: one call per sequence
+    for (int i = 0; i < N; ++i) {
+      const int Ti = (int)(cu_seqlens[i + 1] - cu_seqlens[i]);
+      const int st = run_chunk(varlen_seq(all, cu_seqlens[i], Ti, i), false, nullptr, 0, s);
+      if (st != GDN_OK) return st;
+    }
+    return GDN_OK;
+  }
+  // the tensor-core path: one prep and one scan launch per group of sequences
+  const size_t need = gdn_chunk_varlen_workspace_bytes(cu_seqlens, N, Hk, Hv, dk, dv, dtype);
+  if (need == 0 || workspace == nullptr || !aligned16(workspace) || ws_bytes < need)
+    return GDN_ERR_WORKSPACE;
+  const size_t st_elems = (size_t)Hv * dk * dv;
+  const int G = varlen_group(Hv);
+  std::unique_ptr<VarlenTab> tp(new (std::nothrow) VarlenTab);  // 16 KB, host memory
+  if (!tp) return GDN_ERR_CUDA;
+  VarlenTab& tab = *tp;
+  for (int i0 = 0; i0 < N; i0 += G) {
+    const int i1 = i0 + G < N ? i0 + G : N;
+    tab.n = i1 - i0;
+    int nv = 0;
+    for (int i = i0; i < i1; ++i) {
+      const int Ti = (int)(cu_seqlens[i + 1] - cu_seqlens[i]);
+      tab.seq[i - i0] = make_int4(nv, Ti, (int)cu_seqlens[i], 0);
+      nv += (Ti + kC - 1) / kC;
+    }
+    ChunkArgs g = all;
+    g.B = i1 - i0;
+    g.T = (int)cu_seqlens[N];
+    g.h0 = h0 ? h0 + (size_t)i0 * st_elems : nullptr;
+    g.ht = ht ? ht + (size_t)i0 * st_elems : nullptr;
+    cudaError_t e;
+    if (nv == 0) {  // only empty sequences: their states are copied
+      e = launch_copy_state(g.h0, g.ht, (size_t)g.B * st_elems, s);
+    } else {
+      uint8_t* tabp = static_cast<uint8_t*>(workspace) + varlen_tab_offset(nv, Hk, Hv);
+      e = launch_varlen_table(tab, tabp, s);
+      g.vtab = tabp;
+      g.vNv = nv;
+      if (e == cudaSuccess) e = launch_chunk_mma(g, false, workspace, s);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
   }
   return GDN_OK;
 }

@@ -35,6 +35,25 @@ inline WsLayout ws_layout(int B, int T, int Hk, int Hv) {
   return L;
 }
 
+// Packed batches of sequences of different lengths (gdn_chunk_fwd_varlen) run
+// as one prep and one scan launch over a table with one entry per sequence:
+// (first chunk in the packed chunk numbering, length, first token, 0).  The
+// chunks of all sequences are numbered one after another (each sequence's first
+// chunk starts at its first token), and the workspace is that of one batch row
+// of Nv * 64 tokens (Nv chunks in all), followed by the table.  A launch pair
+// takes at most kVarlenMaxSeqs sequences.
+constexpr int kVarlenMaxSeqs = 1024;
+struct VarlenTab {
+  int n;
+  int4 seq[kVarlenMaxSeqs];
+};
+inline size_t varlen_tab_offset(int Nv, int Hk, int Hv) {
+  return (ws_layout(1, Nv * kC, Hk, Hv).total + 255) & ~size_t(255);
+}
+inline size_t varlen_ws_bytes(int Nv, int Hk, int Hv) {
+  return varlen_tab_offset(Nv, Hk, Hv) + sizeof(int4) * kVarlenMaxSeqs;
+}
+
 // Two consecutive output values in the output type.
 template <typename TO>
 __device__ __forceinline__ void store2(TO* p, float x, float y);

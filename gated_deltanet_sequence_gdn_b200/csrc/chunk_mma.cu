@@ -37,6 +37,8 @@
 #include "common.cuh"
 #include "launch.h"
 #include "chunk_layout.cuh"
+#include "tc_ptx.cuh"
+#include "tmap.cuh"
 #include "warp_mma.cuh"
 #include "wy_common.cuh"
 
@@ -84,18 +86,38 @@ constexpr int Q2_X = Q2_L + kC * LDX * 4;      // A staging (f32), then the inve
 constexpr int Q2_OP = Q2_X + kC * LDX * 4;     // raw gate tiles, decays d, fp16 operands, E-bar
 constexpr int Q2_OPB = 192 * LDT * 2;
 constexpr int Q2_VEC = Q2_OP + Q2_OPB;         // rk, sq [64], carry [3][128], misc [64]
-constexpr int Q2_BYTES = Q2_VEC + 576 * 4;
+constexpr int Q2_BAR = Q2_VEC + 576 * 4;       // 2 mbarriers (tile loads, products) + TMEM address
+constexpr int Q2_BYTES = Q2_BAR + 32 + 1024;   // + slack for the 1024-byte alignment of the base
+// The products W^T = E-bar^T X^T and U^T = Z^T X^T on the tcgen05 tensor cores
+// (M = 128 channels d, N = 64 tokens t, K = 64 tokens t'), accumulators in TMEM:
+// E-bar and Z (bf16 hi, lo) as MN-major A operands, [2 d-halves][64 t'][128 B]
+// with the 128-byte swizzle (in the operand scratch and the Z tiles' space), X as
+// bf16 hi + lo K-major B operands, [64 t][128 B] swizzled (in the A staging's
+// space, free once the inverse is done).
+constexpr int Q2_XH = Q2_X;                    // X hi, then X lo at + 8192
+constexpr uint32_t Q2_TM_W = 0, Q2_TM_U = 64, Q2_TM_COLS = 128;
+static_assert(Q2_ZH % 1024 == 0 && Q2_ZL % 1024 == 0 && Q2_X % 1024 == 0 && Q2_OP % 1024 == 0,
+              "swizzled operand tiles need 1024-byte alignment");
+static_assert(2 * 8192 <= kC * LDX * 4, "X hi + lo fit the A staging's space");
+
+// Byte offset of the 16-byte unit u (0..7) of row t in a [64 rows][128 B] swizzled box.
+__device__ __forceinline__ int box16(int t, int u) { return (t << 7) + ((u ^ (t & 7)) << 4); }
+
+// TMA maps of the tile loads: raw k, q, v rows and the three gate tiles, each a
+// box of 64 time steps of one head, landing as padded rows (LDT bf16 or LDG f32).
+struct Prep2Maps {
+  CUtensorMap k, q, v, ga, gb, gw;
+};
 static_assert(Q2_BYTES <= 227 * 1024, "shared memory of the GDN-2 prep kernel");
 static_assert(kC * LDG * 4 <= Q2_OPB, "a float32 [64][LDG] tile (raw w, the decays) fits the operand scratch");
 
 template <bool PRE>
 __global__ void __launch_bounds__(kThreads, 1)
-wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
-                const void* __restrict__ ga, const void* __restrict__ gb,
-                const void* __restrict__ gw, const float* __restrict__ A_log,
+wy_prep2_kernel(const __grid_constant__ Prep2Maps maps, const float* __restrict__ A_log,
                 const float* __restrict__ dt_bias, int T, int H, float scale, int l2,
-                uint8_t* __restrict__ ws, WsLayout L, int* status) {
-  extern __shared__ __align__(16) uint8_t sm[];
+                uint8_t* __restrict__ ws, WsLayout L, int* status, uint32_t spin) {
+  extern __shared__ __align__(1024) uint8_t sm_raw[];
+  uint8_t* sm = sm_raw + ((1024u - (tc::smem_u32(sm_raw) & 1023u)) & 1023u);
   bf16* Kt = reinterpret_cast<bf16*>(sm + Q2_KT);
   bf16* Qt = reinterpret_cast<bf16*>(sm + Q2_QT);
   bf16* Zh = reinterpret_cast<bf16*>(sm + Q2_ZH);
@@ -109,6 +131,9 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   float* sq = rk + 64;
   float* carry = sq + 64;     // [3][128] prefix sums of the first three quarters
   float* misc = carry + 384;  // [8..23] per-warp max |U|
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Q2_BAR);  // tile loads, products
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Q2_BAR + 16);
+  const uint32_t sb = tc::smem_u32(sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
@@ -118,32 +143,41 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   const int t0 = n * kC, nv = min(kC, T - t0);
   float range = 0.f;
 
-  // 1. raw q, k, v tiles and the gate tiles (rows past the end of the sequence are zeros)
-  for (int i = tid; i < 3 * kC * 16; i += kThreads) {
-    const int which = i >> 10, r = (i >> 4) & 63, c16 = i & 15;
-    const bool ok = r < nv;
-    const size_t off = ok ? ((((size_t)b * T + t0 + r) * H + h) * kD + c16 * 8) : 0;
-    bf16* dst = (which == 0 ? Kt : (which == 1 ? Qt : Zh)) + r * LDT + c16 * 8;
-    cp16(dst, (which == 0 ? k : (which == 1 ? q : v)) + off, ok ? 16 : 0);
-    if (!PRE) {  // a, b, w logits in bf16
-      const bf16* src = reinterpret_cast<const bf16*>(which == 0 ? ga : (which == 1 ? gb : gw));
-      cp16(reinterpret_cast<bf16*>(op + which * kC * LDT * 2) + r * LDT + c16 * 8, src + off,
-           ok ? 16 : 0);
+  // 1. raw q, k, v tiles and the gate tiles by TMA, as padded rows (time steps past
+  //    the end of the sequence and the pad columns read as zeros)
+  if (tid == 0) {
+    tc::mbar_init(&bar[0], 1);
+    tc::mbar_init(&bar[1], 1);
+    tc::fence_mbar_init();
+    constexpr uint32_t kRow16 = kC * LDT * 2, kRow32 = kC * LDG * 4;
+    tc::mbar_arrive_expect_tx(&bar[0], 3 * kRow16 + 3 * (PRE ? kRow32 : kRow16));
+    tc::tma_load_4d(Kt, &maps.k, &bar[0], 0, h, t0, b);
+    tc::tma_load_4d(Qt, &maps.q, &bar[0], 0, h, t0, b);
+    tc::tma_load_4d(Zh, &maps.v, &bar[0], 0, h, t0, b);
+    if (PRE) {  // g, b, w values in float32
+      tc::tma_load_4d(Gm, &maps.ga, &bar[0], 0, h, t0, b);
+      tc::tma_load_4d(Em, &maps.gb, &bar[0], 0, h, t0, b);
+      tc::tma_load_4d(op, &maps.gw, &bar[0], 0, h, t0, b);
+    } else {  // a, b, w logits in bf16
+      tc::tma_load_4d(op, &maps.ga, &bar[0], 0, h, t0, b);
+      tc::tma_load_4d(op + kRow16, &maps.gb, &bar[0], 0, h, t0, b);
+      tc::tma_load_4d(op + 2 * kRow16, &maps.gw, &bar[0], 0, h, t0, b);
     }
   }
-  if (PRE) {  // g, b, w values in float32
-    for (int i = tid; i < 3 * kC * 32; i += kThreads) {
-      const int which = i / (kC * 32), r = (i >> 5) & 63, c32 = i & 31;
-      const bool ok = r < nv;
-      const size_t off = ok ? ((((size_t)b * T + t0 + r) * H + h) * kD + c32 * 4) : 0;
-      const float* src = reinterpret_cast<const float*>(which == 0 ? ga : (which == 1 ? gb : gw));
-      float* dst = (which == 0 ? Gm : (which == 1 ? Em : reinterpret_cast<float*>(op))) + r * LDG;
-      cp16(dst + c32 * 4, src + off, ok ? 16 : 0);
-    }
-  }
-  cp_commit();
-  cp_wait<0>();
+  if (warp == 0) tc::tmem_alloc(tmem_slot, Q2_TM_COLS);
+  tc::tc_fence_before();
   __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  {
+    const bool ok = tc::mbar_wait(&bar[0], 0, status, 131, spin);
+    if (__syncthreads_or(!ok)) {  // leave once the copies in flight have landed
+      if (tid == 0) tc::mbar_wait(&bar[0], 0, nullptr, 0, 1u << 20);
+      __syncthreads();
+      if (warp == 0) tc::tmem_dealloc(tmem, Q2_TM_COLS);
+      return;
+    }
+  }
 
   // 2. L2 norms: rk = 1 / |k|, sq = scale / |q| (four threads per row)
   {
@@ -428,74 +462,110 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   invert_in_place(Lm, Xm, tid, warp, g8, t4);
   float* Xi = Lm;  // X
 
-  // 7. E-bar = exp(G) (.) e in bf16 (the B operand of W), in the operand scratch
-  bf16* Eb = reinterpret_cast<bf16*>(op);
-  for (int i = tid; i < kC * 16; i += kThreads) {
-    const int r = i >> 4, c8 = (i & 15) * 8;
-    uint4 o;
-    uint32_t* po = reinterpret_cast<uint32_t*>(&o);
+  // 7. W^T = E-bar^T X^T and U^T = Z^T X^T on the tcgen05 tensor cores.  First
+  //    E-bar = exp(G) (.) e in bf16 (MN-major A operand, in the operand scratch) and
+  //    X as bf16 hi + lo (K-major B operands, in the A staging's space)
+  {
+    uint8_t* eb = op;
+    for (int i = tid; i < kC * 16; i += kThreads) {
+      const int r = i >> 4, c8 = (i & 15) * 8;
+      uint4 o;
+      uint32_t* po = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-    for (int h4 = 0; h4 < 2; ++h4) {
-      const float4 g4 = *reinterpret_cast<const float4*>(Gm + r * LDG + c8 + 4 * h4);
-      const float4 e4 = *reinterpret_cast<const float4*>(Em + r * LDG + c8 + 4 * h4);
-      po[2 * h4] = pack2(__expf(g4.x) * e4.x, __expf(g4.y) * e4.y);
-      po[2 * h4 + 1] = pack2(__expf(g4.z) * e4.z, __expf(g4.w) * e4.w);
+      for (int h4 = 0; h4 < 2; ++h4) {
+        const float4 g4 = *reinterpret_cast<const float4*>(Gm + r * LDG + c8 + 4 * h4);
+        const float4 e4 = *reinterpret_cast<const float4*>(Em + r * LDG + c8 + 4 * h4);
+        po[2 * h4] = pack2(__expf(g4.x) * e4.x, __expf(g4.y) * e4.y);
+        po[2 * h4 + 1] = pack2(__expf(g4.z) * e4.z, __expf(g4.w) * e4.w);
+      }
+      *reinterpret_cast<uint4*>(eb + (c8 >> 6) * 8192 + box16(r, (c8 & 63) >> 3)) = o;
     }
-    *reinterpret_cast<uint4*>(Eb + r * LDT + c8) = o;
+    uint8_t* xh = sm + Q2_XH;
+    for (int i = tid; i < kC * 8; i += kThreads) {
+      const int t = i >> 3, ch = i & 7;
+      const float* xr = Xi + t * LDX + 8 * ch;
+      const float4 a0 = *reinterpret_cast<const float4*>(xr);
+      const float4 a1 = *reinterpret_cast<const float4*>(xr + 4);
+      uint32_t ph[4], pl[4];
+      split2(a0.x, a0.y, ph[0], pl[0]);
+      split2(a0.z, a0.w, ph[1], pl[1]);
+      split2(a1.x, a1.y, ph[2], pl[2]);
+      split2(a1.z, a1.w, ph[3], pl[3]);
+      const int off = box16(t, ch);
+      *reinterpret_cast<uint4*>(xh + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+      *reinterpret_cast<uint4*>(xh + 8192 + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+    }
   }
-  __syncthreads();
-
-  //    W = X E-bar (fp16 out) and U = X Z (fp32 out, X and Z both as hi + lo);
-  //    warp -> rows 16 (warp % 4), cols 32 (warp / 4)
-  const int mt = warp & 3, nb = 32 * (warp >> 2);
-  const int ra = 16 * mt + g8;
-  float umax = 0.f;
-#pragma unroll 1
-  for (int which = 0; which < 2; ++which) {
-    float acc[4][4] = {};
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      uint32_t ah[4], al[4];
-      frag_a_split(Xi, LDX, 16 * mt, 16 * ks, g8, t4, ah, al);
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        const int bo = (16 * ks + lrow_a(lane)) * LDT + nb + 16 * np + lcol_a(lane);
-        uint32_t bh[4];
-        ldsm_x4_t(bh, (which ? Zh : Eb) + bo);
-        mma_bf16(acc[2 * np], ah, bh[0], bh[1]);
-        mma_bf16(acc[2 * np + 1], ah, bh[2], bh[3]);
-        if (which) {
-          uint32_t bl[4];
-          ldsm_x4_t(bl, Zl + bo);
-          mma_bf16(acc[2 * np], ah, bl[0], bl[1]);
-          mma_bf16(acc[2 * np + 1], ah, bl[2], bl[3]);
-          mma_bf16(acc[2 * np], al, bh[0], bh[1]);
-          mma_bf16(acc[2 * np + 1], al, bh[2], bh[3]);
-        }
-      }
+  __syncthreads();  // e is read: its space takes the Z operand tiles
+  //    Z = w (.) v, hi and lo (padded rows) -> MN-major operand tiles in e's space
+  {
+    const bf16* zl_rows = reinterpret_cast<const bf16*>(sm + Q2_ZL);
+    uint8_t* zt = sm + Q2_E;
+    for (int i = tid; i < 2 * kC * 16; i += kThreads) {
+      const int part = i >> 10, r = (i >> 4) & 63, c8 = (i & 15) * 8;
+      const uint4 u = *reinterpret_cast<const uint4*>((part ? zl_rows : Zh) + r * LDT + c8);
+      *reinterpret_cast<uint4*>(zt + part * 16384 + (c8 >> 6) * 8192 + box16(r, (c8 & 63) >> 3)) =
+          u;
     }
-    if (which == 0) {
-      __half* dw = reinterpret_cast<__half*>(ws + L.w) + (head * Tp + t0) * kD;
+  }
+  tc::fence_proxy_async_smem();  // generic-proxy writes -> the MMA's reads
+  tc::tc_fence_before();
+  __syncthreads();
+  if (tid == 0) {  // W: X hi / lo against E-bar; U: the three hi / lo pairs but lo.lo
+    tc::tc_fence_after();
+    const uint32_t id = tc::idesc_bf16(128, 64, true, false);
+    const uint32_t eb = sb + Q2_OP, zh = sb + Q2_E, zl = zh + 16384;
+    const uint32_t xh = sb + Q2_XH, xl = xh + 8192;
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        const int c = nb + 8 * nt + 2 * t4;
-        range = fmaxf(range, fmaxf(fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][1])),
-                                   fmaxf(fabsf(acc[nt][2]), fabsf(acc[nt][3]))));
-        *reinterpret_cast<uint32_t*>(dw + (size_t)ra * kD + c) = pack2h(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<uint32_t*>(dw + (size_t)(ra + 8) * kD + c) =
-            pack2h(acc[nt][2], acc[nt][3]);
+    for (int k16 = 0; k16 < 4; ++k16) {
+      const uint64_t dxh = tc::sw128_desc(xh + k16 * 32, 16, 1024);
+      const uint64_t dxl = tc::sw128_desc(xl + k16 * 32, 16, 1024);
+      const uint64_t de = tc::sw128_desc(eb + k16 * 2048, 8192, 1024);
+      const uint64_t dzh = tc::sw128_desc(zh + k16 * 2048, 8192, 1024);
+      const uint64_t dzl = tc::sw128_desc(zl + k16 * 2048, 8192, 1024);
+      tc::mma_bf16(tmem + Q2_TM_W, de, dxh, id, k16 > 0);
+      tc::mma_bf16(tmem + Q2_TM_W, de, dxl, id, 1u);
+      tc::mma_bf16(tmem + Q2_TM_U, dzh, dxh, id, k16 > 0);
+      tc::mma_bf16(tmem + Q2_TM_U, dzh, dxl, id, 1u);
+      tc::mma_bf16(tmem + Q2_TM_U, dzl, dxh, id, 1u);
+    }
+    tc::mma_commit(&bar[1]);
+  }
+  {
+    const bool ok = tc::mbar_wait(&bar[1], 0, status, 132, spin);
+    if (__syncthreads_or(!ok)) {  // leave once the products in flight are done
+      if (tid == 0) tc::mbar_wait(&bar[1], 0, nullptr, 0, 1u << 20);
+      tc::tc_fence_before();
+      __syncthreads();
+      if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, Q2_TM_COLS);
       }
-    } else {
-      float* du = reinterpret_cast<float*>(ws + L.u) + (head * Tp + t0) * kD;
+      return;
+    }
+  }
+  tc::tc_fence_after();
+  //    W (fp16) and U (fp32) to the workspace: lane = channel d; warp w takes the 16
+  //    tokens 16 (w / 4) .. + 15 of its lane quarter w % 4, so the 32 lanes of a
+  //    warp store 32 consecutive channels of one row
+  float umax = 0.f;
+  {
+    const int q4 = warp & 3, tb = 16 * (warp >> 2), d = 32 * q4 + lane;
+    const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)tb;
+    __half* dw = reinterpret_cast<__half*>(ws + L.w) + (head * Tp + t0 + tb) * kD + d;
+    float* du = reinterpret_cast<float*>(ws + L.u) + (head * Tp + t0 + tb) * kD + d;
+    float v[16];
+    tc::tmem_ld16(tq + Q2_TM_W, v);
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        const int c = nb + 8 * nt + 2 * t4;
-        umax = fmaxf(umax, fmaxf(fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][1])),
-                                 fmaxf(fabsf(acc[nt][2]), fabsf(acc[nt][3]))));
-        *reinterpret_cast<float2*>(du + (size_t)ra * kD + c) = make_float2(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<float2*>(du + (size_t)(ra + 8) * kD + c) =
-            make_float2(acc[nt][2], acc[nt][3]);
-      }
+    for (int j = 0; j < 16; ++j) {
+      range = fmaxf(range, fabsf(v[j]));
+      dw[(size_t)j * kD] = __float2half_rn(v[j]);
+    }
+    tc::tmem_ld16(tq + Q2_TM_U, v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      umax = fmaxf(umax, fabsf(v[j]));
+      du[(size_t)j * kD] = v[j];
     }
   }
   if (!(range <= kF16Max)) report_range(status);
@@ -552,6 +622,12 @@ wy_prep2_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
       sc[kScMaxU + tid] = tid == 0 ? m : 0.f;
     }
   }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, Q2_TM_COLS);
+  }
 }
 
 template <typename TO>
@@ -564,13 +640,23 @@ cudaError_t launch_t(const ChunkArgs& a, bool gdn2, uint8_t* ws, const WsLayout&
   if (status == nullptr) return cudaErrorUnknown;
   cudaError_t e;
   if (gdn2) {
+    if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
+    Prep2Maps m;
+    const CUtensorMapDataType g_dt =
+        pre ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int g_es = pre ? 4 : 2, g_box = pre ? LDG : LDT;
+    if (!make_map_bthd_rows(&m.k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.B, a.T, a.Hv, LDT) ||
+        !make_map_bthd_rows(&m.q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.B, a.T, a.Hv, LDT) ||
+        !make_map_bthd_rows(&m.v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.B, a.T, a.Hv, LDT) ||
+        !make_map_bthd_rows(&m.ga, a.a, g_dt, g_es, a.B, a.T, a.Hv, g_box) ||
+        !make_map_bthd_rows(&m.gb, a.b, g_dt, g_es, a.B, a.T, a.Hv, g_box) ||
+        !make_map_bthd_rows(&m.gw, a.w, g_dt, g_es, a.B, a.T, a.Hv, g_box))
+      return cudaErrorInvalidValue;
     auto prep = pre ? wy_prep2_kernel<true> : wy_prep2_kernel<false>;
     e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, Q2_BYTES);
     if (e != cudaSuccess) return e;
     prep<<<dim3(1, Nc, a.B * a.Hv), kThreads, Q2_BYTES, s>>>(
-        static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
-        static_cast<const bf16*>(a.v), a.a, a.b, a.w, a.A_log, a.dt_bias, a.T, a.Hv, a.scale, l2,
-        ws, L, status);
+        m, a.A_log, a.dt_bias, a.T, a.Hv, a.scale, l2, ws, L, status, wait_fault().spin);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   } else {

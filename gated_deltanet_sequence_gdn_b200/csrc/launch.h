@@ -16,6 +16,9 @@ struct ChunkArgs {
   void* o; float* ht;
   // gated RMSNorm of the output rows (o = RMSNormGated(core, z)); norm_z == NULL: none
   const void* norm_z = nullptr; const float* norm_w = nullptr; float norm_eps = 0.f;
+  // packed batch (bf16 tensor-core path only): B sequences of the device table
+  // vtab (chunk_layout.cuh) over T packed tokens, vNv chunks in all; NULL: dense
+  const void* vtab = nullptr; int vNv = 0;
 };
 
 cudaError_t launch_gate_prep(const void* q, const void* k, int dtype, const void* a,
@@ -84,6 +87,9 @@ struct WaitFault {
 WaitFault wait_fault();
 
 cudaError_t launch_copy_state(const float* h0, float* ht, size_t n, cudaStream_t s);
+// Copy a packed batch's sequence table (passed by value) to device memory.
+struct VarlenTab;
+cudaError_t launch_varlen_table(const VarlenTab& tab, void* dst, cudaStream_t s);
 
 // Arguments of the chunk backward (gdn_chunk_bwd); D = dk = dv.
 struct BwdArgs {

@@ -89,7 +89,8 @@ __global__ void __launch_bounds__(kPT, 2)
 wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict__ ga,
                   const void* __restrict__ gb, const float* __restrict__ A_log,
                   const float* __restrict__ dt_bias, int T, int Hk, int Hv, float scale, int l2,
-                  uint8_t* __restrict__ ws, WsLayout L, int* status, int fault, uint32_t spin) {
+                  uint8_t* __restrict__ ws, WsLayout L, int* status, int fault, uint32_t spin,
+                  const int4* __restrict__ vtab, int nseq) {
   extern __shared__ __align__(1024) uint8_t sm_raw[];
   uint8_t* sm = sm_raw + ((1024u - (tc::smem_u32(sm_raw) & 1023u)) & 1023u);
   const uint32_t sb = tc::smem_u32(sm);
@@ -116,7 +117,22 @@ wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict_
   const int G = Hv / Hk;
   const int n = blockIdx.x, Nc = gridDim.x, Tp = Nc * kC;
   const int b = blockIdx.y / Hk, hk = blockIdx.y % Hk;
-  const int t0 = n * kC, nv = min(kC, T - t0);
+  // first time step and valid rows of the chunk; the workspace rows of the chunk
+  // start at row n * 64 of its head
+  int t0 = n * kC, nv = min(kC, T - t0);
+  if (vtab != nullptr) {  // packed batch: the sequence whose chunks include chunk n
+    int lo = 0, hi = nseq - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (vtab[mid].x <= n) lo = mid;
+      else hi = mid - 1;
+    }
+    const int4 e = vtab[lo];
+    const int j = n - e.x;
+    t0 = e.z + j * kC;
+    nv = min(kC, e.y - j * kC);
+  }
+  const int wrow = n * kC;
   const int q4 = warp & 3, hc = warp >> 2;  // TMEM lane quarter, column half
   const int r = 32 * q4 + lane;             // accumulator lane of this thread
   float range = 0.f;                        // largest magnitude converted to fp16
@@ -294,7 +310,7 @@ wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict_
   tc::fence_proxy_async_smem();
   __syncthreads();
   if (tid == 0) {
-    const int row = blockIdx.y * Tp + t0;
+    const int row = blockIdx.y * Tp + wrow;
 #pragma unroll
     for (int dh = 0; dh < 2; ++dh) {
       tc::tma_store_2d(&maps.kh, sm + S_R + dh * 8192, 64 * dh, row);
@@ -312,7 +328,7 @@ wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict_
 
   for (int h = 0; h < G; ++h) {
     const size_t head = (size_t)b * Hv + hk * G + h;
-    const int row0 = (int)(head * Tp) + t0;  // first workspace row of this chunk and head
+    const int row0 = (int)(head * Tp) + wrow;  // first workspace row of this chunk and head
     if (h > 0 && (h & 3) == 0) {             // gates of the next four heads
       __syncthreads();
       gates_partial(h);
@@ -505,14 +521,17 @@ wy_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const void* __restrict_
 }  // namespace
 
 cudaError_t launch_prep_tc(const ChunkArgs& a, void* ws, int* status, cudaStream_t s) {
-  const WsLayout L = ws_layout(a.B, a.T, a.Hk, a.Hv);
-  const int Nc = (a.T + kC - 1) / kC;
+  // a packed batch (a.vtab) is one batch row of a.T tokens cut into a.vNv chunks
+  const bool packed = a.vtab != nullptr;
+  const int B = packed ? 1 : a.B;
+  const int Nc = packed ? a.vNv : (a.T + kC - 1) / kC;
+  const WsLayout L = ws_layout(B, Nc * kC, a.Hk, a.Hv);
   const uint64_t Tp = (uint64_t)Nc * kC;
-  const uint64_t rv = (uint64_t)a.B * a.Hv * Tp, rk = (uint64_t)a.B * a.Hk * Tp;
+  const uint64_t rv = (uint64_t)B * a.Hv * Tp, rk = (uint64_t)B * a.Hk * Tp;
   uint8_t* w = static_cast<uint8_t*>(ws);
   PrepMaps m;
-  if (!make_map_bthd(&m.q, a.q, a.B, a.T, a.Hk) || !make_map_bthd(&m.k, a.k, a.B, a.T, a.Hk) ||
-      !make_map_bthd(&m.v, a.v, a.B, a.T, a.Hv) ||
+  if (!make_map_bthd(&m.q, a.q, B, a.T, a.Hk) || !make_map_bthd(&m.k, a.k, B, a.T, a.Hk) ||
+      !make_map_bthd(&m.v, a.v, B, a.T, a.Hv) ||
       !make_map_rows(&m.qh, w + L.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rk) ||
       !make_map_rows(&m.kh, w + L.kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rk) ||
       !make_map_rows(&m.a, w + L.a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kC, rv))
@@ -523,9 +542,9 @@ cudaError_t launch_prep_tc(const ChunkArgs& a, void* ws, int* status, cudaStream
   cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PT_SMEM);
   if (e != cudaSuccess) return e;
   const WaitFault f = wait_fault();
-  prep<<<dim3(Nc, a.B * a.Hk), kPT, PT_SMEM, s>>>(m, a.a, a.b, a.A_log, a.dt_bias, a.T, a.Hk,
-                                                  a.Hv, a.scale, l2, w, L, status, f.site,
-                                                  f.spin);
+  prep<<<dim3(Nc, B * a.Hk), kPT, PT_SMEM, s>>>(m, a.a, a.b, a.A_log, a.dt_bias, a.T, a.Hk,
+                                                a.Hv, a.scale, l2, w, L, status, f.site, f.spin,
+                                                static_cast<const int4*>(a.vtab), a.B);
   return cudaGetLastError();
 }
 

@@ -10,16 +10,21 @@
 // scan Q / K rows; fp32 U; per-chunk factors), see chunk_mma.cu for the algebra,
 // the precision design and the range scale sigma.
 //
-// Warp roles (320 threads):
+// Warp roles (288 threads):
 //   warp 0      TMA producer: every tile of chunk n into stage n % 2 (10 bulk copies)
-//   warp 1      TMEM allocation and the tcgen05.mma issue (one thread)
-//   warps 2-9   epilogue, two warps per TMEM lane quarter (warps w and w + 4 take
+//               (the whole warp also allocates and releases the TMEM)
+//   warps 1-8   epilogue, two warps per TMEM lane quarter (warps w and w + 4 take
 //               columns 0-31 and 32-63): 32 columns of one state row (d_k row =
 //               TMEM lane) per thread in fp32 registers; TMEM loads of the
 //               accumulators, U~ / U~s / the state written back to shared memory
-//               as fp16 operands, o stored.
-// Hand-offs go through mbarriers; every wait is bounded and an expired wait ends
-// the kernel through the status word (GDN_ERR_TIMEOUT) after its copies and
+//               as fp16 operands, o stored.  One epilogue thread also issues the
+//               tcgen05.mma products, each right after the epilogue barrier at
+//               which its operands are complete: per chunk the chain is
+//               [Q; W] S -> U~ (epilogue) -> DS -> state (epilogue) -> next chunk,
+//               with O_a issued behind DS and run while the state is updated.
+// The tensor cores report completion through mbarriers (tcgen05.commit), the TMA
+// producer through transaction counts; every wait is bounded and an expired wait
+// ends the kernel through the status word (GDN_ERR_TIMEOUT) after its copies and
 // tensor-core work in flight have drained.
 //
 // With NORM the output rows leave through the gated RMSNorm of the pages'
@@ -46,7 +51,7 @@ namespace {
 using namespace tc;
 using bf16 = __nv_bfloat16;
 
-constexpr int kScanTcThreads = 320;
+constexpr int kScanTcThreads = 288;
 constexpr int kEpi = 256;  // epilogue threads
 // shared memory map (offsets from a 1024-byte aligned base); 128-byte swizzled
 // fp16 tiles are stored as 64-column halves of [64 rows][128 bytes]
@@ -78,11 +83,14 @@ constexpr uint32_t SCAN_TC_SMEM_NORM = SCAN_TC_SMEM + 64 * kOS * 4 + 64 * kZS * 
 static_assert(ST_SC + kScal * 4 <= STAGE_BYTES, "stage layout");
 static_assert(SCAN_TC_SMEM_NORM <= 227 * 1024, "shared memory of the tcgen05 scan");
 
-// TMEM columns of the accumulators (M = 128, N = 64 each)
-constexpr uint32_t TM_QP = 0, TM_OA = 64, TM_DS = 128, TM_COLS = 256;
+// TMEM columns of the accumulators (M = 128, N = 64 each); [O_q; P] alternates
+// between two buffers by chunk parity, so that the output rows read O_q of chunk n
+// while the products of chunk n + 1 run
+constexpr uint32_t TM_QP0 = 0, TM_OA = 64, TM_DS = 128, TM_QP1 = 192, TM_COLS = 256;
+__device__ __forceinline__ uint32_t tm_qp(int n) { return (n & 1) ? TM_QP1 : TM_QP0; }
 
 // barrier indices
-enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_QP, B_UT, B_DS, B_OA, B_S,
+enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_QP, B_DS, B_OA,
        B_PX0, B_PX1, B_PX2, B_PX3,  // NORM: the peer's row sums of a chunk have arrived
        B_COUNT };
 static_assert(B_COUNT * 8 + 8 <= 128, "barrier area");
@@ -186,7 +194,8 @@ template <typename TO, bool NORM>
 __global__ void __launch_bounds__(kScanTcThreads, 1)
 state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __restrict__ ws,
                      WsLayout L, const float* h0, int T, int Hk, int Hv, TO* __restrict__ o,
-                     float* ht, int* status, int fault, uint32_t spin, NormArgs na) {
+                     float* ht, int* status, int fault, uint32_t spin, NormArgs na,
+                     const int4* __restrict__ vtab, int Nv) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -197,12 +206,27 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c0 = 64 * blockIdx.x;
   const int head = blockIdx.y, b = head / Hv, hv = head % Hv, hk = hv / (Hv / Hk);
-  const int Nc = (T + kC - 1) / kC, Tp = Nc * kC;
-  const int khead = b * Hk + hk;
-  const float* Sg = reinterpret_cast<const float*>(ws + L.scal) + (size_t)head * Nc * kScal;
+  // this CTA's sequence: Ts time steps from token tok0 of the o / z rows, Nc chunks
+  // from chunk cb of its workspace head wsh (a dense batch row b: b T, all of T,
+  // chunk 0 of head (b, hv); a packed batch: sequence b of the table, whose chunks
+  // follow those of the sequences before it in one batch row of Nv chunks)
+  int Ts = T, Nc = (T + kC - 1) / kC, cb = 0, wsh = head, khead = b * Hk + hk;
+  size_t tok0 = (size_t)b * T;
+  if (vtab != nullptr) {
+    const int4 e = vtab[b];
+    cb = e.x;
+    Ts = e.y;
+    Nc = (Ts + kC - 1) / kC;
+    tok0 = (size_t)e.z;
+    wsh = hv;
+    khead = hk;
+  }
+  const int Tp = (vtab != nullptr ? Nv : Nc) * kC;  // workspace rows per head
+  const float* Sg =
+      reinterpret_cast<const float*>(ws + L.scal) + ((size_t)wsh * (Tp / kC) + cb) * kScal;
   const uint32_t sbase = smem_u32(sm);
 
-  if (warp == 1) tmem_alloc(tmem_slot, TM_COLS);
+  if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
   if (tid == 0) {
     for (int i = 0; i < B_COUNT; ++i)
       mbar_init(&bar[i], (i == B_EMPTY0 || i == B_EMPTY1) ? 2 : 1);
@@ -238,7 +262,7 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
         uint8_t* st = sm + s * STAGE_BYTES;
         uint64_t* full = &bar[B_FULL0 + s];
         mbar_arrive_expect_tx(full, TX_BYTES);
-        const int rq = khead * Tp + n * kC, rw = head * Tp + n * kC;
+        const int rq = khead * Tp + (cb + n) * kC, rw = wsh * Tp + (cb + n) * kC;
         tma_load_2d(st + ST_QW + 0, &maps.q, full, 0, rq);
         tma_load_2d(st + ST_QW + 16384, &maps.q, full, 64, rq);
         tma_load_2d(st + ST_QW + 8192, &maps.w, full, 0, rw);
@@ -257,57 +281,11 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       for (int n = (issued >= 2 ? issued - 2 : 0); n < issued; ++n)
         mbar_wait(&bar[B_FULL0 + (n & 1)], (n >> 1) & 1, nullptr, 0, 1u << 20);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      const uint32_t id_qw = idesc_f16(128, 64, false, true);
-      const uint32_t id_a = idesc_f16(128, 64, false, true);
-      const uint32_t id_k = idesc_f16(128, 64, true, true);
-      uint32_t qp_phases = 0;  // phases of B_QP completed by our commits
-      for (int n = 0; n < Nc; ++n) {
-        const int s = n & 1;
-        const uint32_t st = sbase + s * STAGE_BYTES;
-        if (!wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 102, abort_flag, spin) ||
-            !wait_or_abort(&bar[B_S], n & 1, status, 103, abort_flag, spin)) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        // [O_q; P] = [Q; W] S   (K = d_k = 128: two 64-column halves of 4 steps)
-        for (int k16 = 0; k16 < 8; ++k16) {
-          const uint32_t aoff = (uint32_t)(k16 >> 2) * 16384u + (uint32_t)(k16 & 3) * 32u;
-          mma_bf16(tmem + TM_QP, sw128_desc(st + ST_QW + aoff, 16, 1024),
-                   sw128_desc(sbase + OFF_SB + k16 * 2048, 8192, 1024), id_qw, k16 > 0);
-        }
-        mma_commit(&bar[B_QP]);
-        ++qp_phases;
-        if (!wait_or_abort(&bar[B_UT], n & 1, status, 104, abort_flag, spin)) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        // DS = K^T U~s first (the state update waits for it), then O_a = A_qk U~
-        // (K = 64 tokens: 4 steps each)
-        for (int k16 = 0; k16 < 4; ++k16)
-          mma_bf16(tmem + TM_DS, sw128_desc(st + ST_K + k16 * 2048, 8192, 1024),
-                   sw128_desc(sbase + OFF_US + k16 * 2048, 8192, 1024), id_k, k16 > 0);
-        mma_commit(&bar[B_DS]);
-        for (int k16 = 0; k16 < 4; ++k16)
-          mma_bf16(tmem + TM_OA, sw128_desc(st + ST_A + k16 * 32, 16, 1024),
-                   sw128_desc(sbase + OFF_UT + k16 * 2048, 8192, 1024), id_a, k16 > 0);
-        mma_commit(&bar[B_OA]);
-        mma_commit(&bar[B_EMPTY0 + s]);  // the stage's operands have been read
-      }
-      // drain: nothing of ours may still run on the tensor cores at teardown (the
-      // commit below completes phase qp_phases of B_QP once all our MMAs are done)
-      mma_commit(&bar[B_QP]);
-      mbar_wait(&bar[B_QP], qp_phases & 1, nullptr, 0, 1u << 20);
-    }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = tid - 64;                       // 0..255
+    const int e = tid - 32;                       // 0..255
     const int row = 32 * (warp & 3) + lane;       // TMEM lane = d_k row of the state
-    const int half = (warp - 2) >> 2;             // columns 32 half .. 32 half + 31
+    const int half = (warp - 1) >> 2;             // columns 32 half .. 32 half + 31
     const int cb = 32 * half;
     const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)cb;
     const bool p_rows = row >= 64;                // lanes 64-127: rows of P (token row - 64)
@@ -325,7 +303,7 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
     for (int n = e; n < Nc; n += kEpi) mx = fmaxf(mx, Sg[(size_t)n * kScal + kScMaxU]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    if (lane == 0) red[warp - 2] = mx;
+    if (lane == 0) red[warp - 1] = mx;
     named_barrier(1, kEpi);
     mx = red[0];
 #pragma unroll
@@ -338,14 +316,49 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       S[c] *= sigma;
       range = fmaxf(range, fabsf(S[c]));
     }
+    // One epilogue thread issues every product of the CTA (completion through
+    // tcgen05.commit on an mbarrier; a commit covers all earlier products of the
+    // thread).  It is lane 0 of a P-row warp: an issue that waits for the tensor
+    // pipe then only holds up a warp that waits for those products anyway.
+    const bool issuer = tid == 64;
+    const uint32_t id_qw = idesc_f16(128, 64, false, true);
+    const uint32_t id_a = idesc_f16(128, 64, false, true);
+    const uint32_t id_k = idesc_f16(128, 64, true, true);
+    uint32_t qp_phases = 0;  // commits to B_QP so far (issuer)
+    // [O_q; P] = [Q; W] S of chunk m (K = d_k = 128: two 64-column halves of 4
+    // steps), once its stage has landed; the state is in shared memory
+    auto issue_qw = [&](int m) -> bool {
+      const uint32_t st = sbase + (m & 1) * STAGE_BYTES;
+      if (!wait_or_abort(&bar[B_FULL0 + (m & 1)], (m >> 1) & 1, status, 102, abort_flag, spin))
+        return false;
+      tc_fence_after();
+      for (int k16 = 0; k16 < 8; ++k16) {
+        const uint32_t aoff = (uint32_t)(k16 >> 2) * 16384u + (uint32_t)(k16 & 3) * 32u;
+        mma_bf16(tmem + tm_qp(m), sw128_desc(st + ST_QW + aoff, 16, 1024),
+                 sw128_desc(sbase + OFF_SB + k16 * 2048, 8192, 1024), id_qw, k16 > 0);
+      }
+      mma_commit(&bar[B_QP]);
+      ++qp_phases;
+      return true;
+    };
+    // O_a = A_qk U~ of chunk m (K = 64 tokens), then the stage's operands are read
+    auto issue_oa = [&](int m) {
+      const uint32_t st = sbase + (m & 1) * STAGE_BYTES;
+      for (int k16 = 0; k16 < 4; ++k16)
+        mma_bf16(tmem + TM_OA, sw128_desc(st + ST_A + k16 * 32, 16, 1024),
+                 sw128_desc(sbase + OFF_UT + k16 * 2048, 8192, 1024), id_a,
+                 k16 > 0);
+      mma_commit(&bar[B_OA]);
+      mma_commit(&bar[B_EMPTY0 + (m & 1)]);
+    };
+
     store_half_row_f16(sm + OFF_SB, row, 4 * half, S);
     fence_proxy_async_smem();
     named_barrier(1, kEpi);
-    // (a test of the bounded waits withholds this first arrival: the MMA issue's
-    // wait for the state then expires and the CTA leaves through the abort path)
-    if (e == 0 && fault != kFaultScanState) mbar_arrive(&bar[B_S]);
+    // (a test of the bounded waits withholds these first products: every epilogue
+    // thread's wait for them then expires and the CTA leaves through the abort path)
+    if (issuer && fault != kFaultScanState && Nc > 0 && !issue_qw(0)) *abort_flag = 1;
 
-    float OQ[32];
     // NORM: the rows' sums of squares, this CTA's [2 chunks][64][2] and the peer's
     // [4 chunks][64]; the rows of the previous chunk and their gate z
     float* ssq = reinterpret_cast<float*>(sm + OFF_NRM);
@@ -378,11 +391,11 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       if (gbar == 3 && r == 0 && hf == 0 && m + 4 < Nc)
         mbar_arrive_expect_tx(&bar[B_PX0 + slot], 64 * 4);
       const int tm = m * kC + r;
-      if (tm < T) {
+      if (tm < Ts) {
         const float* ob = obuf + r * kOS + cbase;
         const bf16* zr = zbuf + r * kZS + cbase;
         const float* wr = wbuf + cbase;
-        TO* dst = o + (((size_t)b * T + tm) * Hv + hv) * kD + c0 + cbase;
+        TO* dst = o + ((tok0 + tm) * Hv + hv) * kD + c0 + cbase;
 #pragma unroll
         for (int c8 = 0; c8 < ncols; c8 += 8) {
           float y[8];
@@ -410,15 +423,10 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       const int s = n & 1;
       const uint8_t* st = sm + s * STAGE_BYTES;
       const float* sc = reinterpret_cast<const float*>(st + ST_SC);
-      {  // every epilogue thread takes the same decision (no thread is left at a barrier)
-        const bool ok =
-            wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 105, abort_flag, spin) &&
-            wait_or_abort(&bar[B_QP], n & 1, status, 106, abort_flag, spin) && !*abort_flag;
-        if (named_barrier_or(1, kEpi, !ok)) {
-          *abort_flag = 1;
-          break;
-        }
-      }
+      // an expired wait is decided on at the next barrier, by a vote of all epilogue
+      // threads (no thread is left at a barrier; what is computed meanwhile is dropped)
+      bool ok = wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 105, abort_flag, spin) &&
+                wait_or_abort(&bar[B_QP], n & 1, status, 106, abort_flag, spin);
       tc_fence_after();
       float fo = 0.f;
       if (p_rows) {
@@ -427,7 +435,7 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
         const int r = row - 64;
         const float fs = sc[kC + r];
         float P[32];
-        tmem_ld32(tl + TM_QP, P);
+        tmem_ld32(tl + tm_qp(n), P);
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {  // U box `half` holds columns cb .. cb + 31
           const float4 u = *reinterpret_cast<const float4*>(st + ST_U + half * 8192 + swz(r, ch));
@@ -455,25 +463,31 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
 #pragma unroll
         for (int c = 0; c < 32; ++c) range = fmaxf(range, fabsf(P[c]));
       } else {
-        tmem_ld32(tl + TM_QP, OQ);  // O_q of token row, this thread's 32 columns
-        fo = sc[row];
+        fo = sc[row];  // (O_q of the row is read with O_a, in the output step)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_barrier(1, kEpi);
-      if (e == 0) mbar_arrive(&bar[B_UT]);
+      if (named_barrier_or(1, kEpi, !ok || *abort_flag)) {
+        *abort_flag = 1;
+        break;
+      }
+      // DS = K^T U~s (K = 64 tokens) first: the state update waits for it; then
+      // O_a, which runs while the state is updated
+      if (issuer) {
+        tc_fence_after();
+        const uint32_t stb = sbase + s * STAGE_BYTES;
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_bf16(tmem + TM_DS, sw128_desc(stb + ST_K + k16 * 2048, 8192, 1024),
+                   sw128_desc(sbase + OFF_US + k16 * 2048, 8192, 1024), id_k, k16 > 0);
+        mma_commit(&bar[B_DS]);
+        issue_oa(n);
+      }
       // NORM: the gate of the previous chunk's rows has landed before the barrier
       // below, after which the P-row threads read it
       if (NORM && !p_rows) asm volatile("cp.async.wait_all;" ::: "memory");
 
       // the state update first: it is what the next chunk waits for
-      {
-        const bool ok = wait_or_abort(&bar[B_DS], n & 1, status, 107, abort_flag, spin);
-        if (named_barrier_or(1, kEpi, !ok)) {
-          *abort_flag = 1;
-          break;
-        }
-      }
+      ok = wait_or_abort(&bar[B_DS], n & 1, status, 107, abort_flag, spin);
       tc_fence_after();
       {
         float D[32];
@@ -488,9 +502,14 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       store_half_row_f16(sm + OFF_SB, row, 4 * half, S);
       fence_proxy_async_smem();
       tc_fence_before();
-      named_barrier(1, kEpi);
-      if (e == 0) {
-        mbar_arrive(&bar[B_S]);
+      if (named_barrier_or(1, kEpi, !ok || *abort_flag)) {
+        *abort_flag = 1;
+        break;
+      }
+      // the next chunk's [Q; W] S
+      if (issuer) {
+        tc_fence_after();
+        if (n + 1 < Nc && !issue_qw(n + 1)) *abort_flag = 1;
         mbar_arrive(&bar[B_EMPTY0 + s]);  // U and the factors of the stage are read
       }
       // NORM: the P-row threads normalise and store their part of the previous
@@ -503,11 +522,12 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
 
       // then the output rows (lanes 0-63), overlapping the next chunk's products
       if (!p_rows) {
-        bool ok = wait_or_abort(&bar[B_OA], n & 1, status, 108, abort_flag, spin);
-        if (NORM) ok = !named_barrier_or(2, 128, !ok);  // the 128 row threads decide as one
-        if (!ok) continue;
+        bool oa_ok = wait_or_abort(&bar[B_OA], n & 1, status, 108, abort_flag, spin);
+        if (NORM) oa_ok = !named_barrier_or(2, 128, !oa_ok);  // the 128 row threads decide as one
+        if (!oa_ok) continue;
         tc_fence_after();
-        float OA[32];
+        float OQ[32], OA[32];
+        tmem_ld32(tl + tm_qp(n), OQ);  // O_q of token row, this thread's 32 columns
         tmem_ld32(tl + TM_OA, OA);
         tc_fence_before();
         const int t = n * kC + row;
@@ -537,8 +557,8 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
           for (int c = 0; c < 32; c += 4)
             *reinterpret_cast<float4*>(ob + c) = make_float4(OA[c], OA[c + 1], OA[c + 2], OA[c + 3]);
           // the gate of these rows, copied in while the next chunk runs
-          if (t < T) {
-            const bf16* zsrc = na.z + (((size_t)b * T + t) * Hv + hv) * kD + c0 + cb;
+          if (t < Ts) {
+            const bf16* zsrc = na.z + ((tok0 + t) * Hv + hv) * kD + c0 + cb;
             const uint32_t zdst = smem_u32(zbuf + row * kZS + cb);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -547,11 +567,15 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
                            : "memory");
             asm volatile("cp.async.commit_group;" ::: "memory");
           }
-        } else if (t < T) {
-          TO* dst = o + (((size_t)b * T + t) * Hv + hv) * kD + c0 + cb;
+        } else if (t < Ts) {
+          TO* dst = o + ((tok0 + t) * Hv + hv) * kD + c0 + cb;
           store_row<TO>(dst, OA);
         }
       }
+    }
+    if (issuer) {  // nothing of ours may still run on the tensor cores at teardown
+      mma_commit(&bar[B_QP]);
+      mbar_wait(&bar[B_QP], qp_phases & 1, nullptr, 0, 1u << 20);
     }
     // NORM: the last chunk's rows, by the P-row threads once the output-row threads'
     // buffers and gate copies are complete (every epilogue thread gets here: the
@@ -578,7 +602,7 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, TM_COLS);
   }
@@ -591,8 +615,11 @@ template <typename TO, bool NORM>
 cudaError_t launch_t(const ChunkArgs& a, const WsLayout& L, const uint8_t* ws, int* status,
                      const NormArgs& na, cudaStream_t s) {
   if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
-  const uint64_t Tp = (uint64_t)((a.T + kC - 1) / kC) * kC;
-  const uint64_t rv = (uint64_t)a.B * a.Hv * Tp, rk = (uint64_t)a.B * a.Hk * Tp;
+  // a packed batch (a.vtab): a.B sequences in one batch row of a.vNv chunks
+  const bool packed = a.vtab != nullptr;
+  const uint64_t Tp = packed ? (uint64_t)a.vNv * kC : (uint64_t)((a.T + kC - 1) / kC) * kC;
+  const uint64_t rows_b = packed ? 1 : (uint64_t)a.B;
+  const uint64_t rv = rows_b * a.Hv * Tp, rk = rows_b * a.Hk * Tp;
   ScanMaps m;
   if (!make_map_rows(&m.q, ws + L.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rk) ||
       !make_map_rows(&m.w, ws + L.w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, rv) ||
@@ -620,15 +647,26 @@ cudaError_t launch_t(const ChunkArgs& a, const WsLayout& L, const uint8_t* ws, i
     cfg.numAttrs = 1;
   }
   e = cudaLaunchKernelEx(&cfg, kern, m, ws, L, a.h0, a.T, a.Hk, a.Hv, static_cast<TO*>(a.o),
-                         a.ht, status, f.site, f.spin, na);
+                         a.ht, status, f.site, f.spin, na, static_cast<const int4*>(a.vtab),
+                         a.vNv);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
+__global__ void varlen_table_kernel(const __grid_constant__ VarlenTab tab, int4* dst) {
+  for (int i = threadIdx.x; i < tab.n; i += blockDim.x) dst[i] = tab.seq[i];
+}
+
 }  // namespace
 
+cudaError_t launch_varlen_table(const VarlenTab& tab, void* dst, cudaStream_t s) {
+  varlen_table_kernel<<<1, 256, 0, s>>>(tab, static_cast<int4*>(dst));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_scan_tc(const ChunkArgs& a, const void* ws, int* status, cudaStream_t s) {
-  const WsLayout L = ws_layout(a.B, a.T, a.Hk, a.Hv);
+  const WsLayout L = a.vtab != nullptr ? ws_layout(1, a.vNv * kC, a.Hk, a.Hv)
+                                       : ws_layout(a.B, a.T, a.Hk, a.Hv);
   const uint8_t* w = static_cast<const uint8_t*>(ws);
   const NormArgs na{static_cast<const bf16*>(a.norm_z), a.norm_w, a.norm_eps};
   const bool norm = a.norm_z != nullptr;

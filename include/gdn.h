@@ -342,18 +342,26 @@ size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int d
  * gdn_chunk_fwd_varlen -- gdn_chunk_fwd over a packed batch of N sequences of
  * different lengths: sequence i is tokens cu_seqlens[i] .. cu_seqlens[i+1] - 1
  * of the packed arrays, with its own initial and final state, and its chunks
- * start at its first token (the result of N one-sequence calls, run one after
- * another on the stream).  The pages batch sequences by padding
- * ("gated-deltanet-qwen3.5" architecture diagram, apply_mask_to_padding_states);
- * packing is this library's way to batch without the padded tokens.
+ * start at its first token (the result of N one-sequence calls).  The pages
+ * batch sequences by padding ("gated-deltanet-qwen3.5" architecture diagram,
+ * apply_mask_to_padding_states); packing is this library's way to batch without
+ * the padded tokens.
  *   q, k [T_total, Hk, dk]; v, o [T_total, Hv, dv]; a, b [T_total, Hv]
- *     (T_total = cu_seqlens[N]), dtypes, flags and scale as for gdn_chunk_fwd.
+ *     (T_total = cu_seqlens[N] < 2^31), dtypes, flags and scale as for
+ *     gdn_chunk_fwd.
  *   h0 / ht [N, Hv, dk, dv] float32 or NULL (ht may alias h0).
  *   cu_seqlens: HOST array of N + 1 int64, cu_seqlens[0] = 0, non-decreasing;
  *     read during the call only.  Empty sequences copy their h0 to ht.
- *   workspace / ws_bytes: as for gdn_chunk_fwd, at least
- *     gdn_chunk_workspace_bytes(1, longest sequence, ...) bytes; it is reused
- *     by every sequence.
+ *   workspace / ws_bytes: device scratch owned by the caller, 16-byte aligned, at
+ *     least gdn_chunk_varlen_workspace_bytes(cu_seqlens, ...) bytes (0: none
+ *     needed) -> else GDN_ERR_WORKSPACE, nothing launched.
+ *   The bf16 dk = dv = 128 path runs the whole batch as one prep and one state
+ *   scan launch (per group of up to 1024 sequences, and of at most 65535 / Hv):
+ *   the chunks of all sequences are numbered one after another, the prep takes
+ *   every chunk of every sequence in one grid, and the scan one CTA pair per
+ *   (sequence, value head).  A small kernel first copies the group's sequence
+ *   table (passed by value) into the workspace.  The float32 and d = 64 path
+ *   runs one call per sequence.
  *   Every sequence is checked before anything is enqueued.  Returns as
  *   gdn_chunk_fwd, and GDN_ERR_INVALID_ARG for a bad cu_seqlens.
  */
@@ -362,6 +370,12 @@ int gdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, const void
                          const float* h0, const long long* cu_seqlens, int N, int Hk, int Hv,
                          int dk, int dv, int dtype, float scale, int flags, void* o,
                          float* ht, void* workspace, size_t ws_bytes, gdn_stream_t stream);
+
+/* Device workspace bytes gdn_chunk_fwd_varlen needs for this packed batch (its
+ * host cu_seqlens, N + 1 entries); 0 for the float32 / d = 64 path, which needs
+ * none, and for invalid arguments. */
+size_t gdn_chunk_varlen_workspace_bytes(const long long* cu_seqlens, int N, int Hk, int Hv,
+                                        int dk, int dv, int dtype);
 
 /*
  * gdn_kda_chunk_fwd -- KDA (Kimi Delta Attention): the channel-wise decay of

@@ -205,9 +205,16 @@ def test_varlen_checks_cu_seqlens_before_anything():
     assert vl(*args(arr(0, 0, 0), 2)) == 0                 # empty sequences, no ht: nothing
     assert vl(*args(arr(0, 64, 100), 2, ws=None, ws_bytes=0)) == -5
     assert vl(*args(arr(0, 64, 100), 2, q=None)) == -1
-    # a sequence's workspace need is checked against the longest one
-    need = G.lib.gdn_chunk_workspace_bytes(1, 300, 2, 4, 128, 128, 1)
+    # the workspace holds every chunk of the packed batch and its sequence table
+    wsb = G.lib.gdn_chunk_varlen_workspace_bytes
+    need = wsb(arr(0, 64, 364), 2, 2, 4, 128, 128, 1)
+    assert need >= G.lib.gdn_chunk_workspace_bytes(1, 6 * 64, 2, 4, 128, 128, 1)
     assert vl(*args(arr(0, 64, 364), 2, ws_bytes=need - 1)) == -5
+    assert wsb(arr(0, 64, 364), 2, 2, 4, 64, 64, 1) == 0      # the CUDA-core path: none
+    assert wsb(arr(0, 64, 364), 2, 2, 4, 128, 128, 0) == 0    # float32: none
+    assert wsb(arr(0, 9, 5), 2, 2, 4, 128, 128, 1) == 0       # decreasing offsets
+    # empty sequences take no chunk: only the table's space
+    assert wsb(arr(0, 0, 0), 2, 2, 4, 128, 128, 1) == wsb(arr(0, 0), 1, 2, 4, 128, 128, 1) > 0
 
 
 def test_empty_calls_are_no_ops():
