@@ -10,18 +10,21 @@
 // scan Q / K rows; fp32 U; per-chunk factors), see chunk_mma.cu for the algebra,
 // the precision design and the range scale sigma.
 //
-// Warp roles (288 threads):
+// Warp roles (320 threads):
 //   warp 0      TMA producer: every tile of chunk n into stage n % 2 (10 bulk copies)
 //               (the whole warp also allocates and releases the TMEM)
-//   warps 1-8   epilogue, two warps per TMEM lane quarter (warps w and w + 4 take
+//   warp 1      tcgen05.mma issue (lane 0)
+//   warps 2-9   epilogue, two warps per TMEM lane quarter (warps w and w + 4 take
 //               columns 0-31 and 32-63): 32 columns of one state row (d_k row =
 //               TMEM lane) per thread in fp32 registers; TMEM loads of the
 //               accumulators, U~ / U~s / the state written back to shared memory
-//               as fp16 operands, o stored.  One epilogue thread also issues the
-//               tcgen05.mma products, each right after the epilogue barrier at
-//               which its operands are complete: per chunk the chain is
-//               [Q; W] S -> U~ (epilogue) -> DS -> state (epilogue) -> next chunk,
-//               with O_a issued behind DS and run while the state is updated.
+//               as fp16 operands, o stored.
+// Per chunk the chain is [Q; W] S -> U~ (epilogue) -> DS -> state (epilogue) ->
+// next chunk, with O_a issued behind DS and run while the state is updated.  The
+// epilogue hands its operands to the MMA warp through a hardware named barrier
+// that the MMA warp waits on (and that carries the vote on giving up), so the
+// issue follows the last epilogue store without an mbarrier round trip, and no
+// epilogue warp waits while the tensor pipe accepts the products.
 // The tensor cores report completion through mbarriers (tcgen05.commit), the TMA
 // producer through transaction counts; every wait is bounded and an expired wait
 // ends the kernel through the status word (GDN_ERR_TIMEOUT) after its copies and
@@ -51,8 +54,11 @@ namespace {
 using namespace tc;
 using bf16 = __nv_bfloat16;
 
-constexpr int kScanTcThreads = 288;
+constexpr int kScanTcThreads = 320;
 constexpr int kEpi = 256;  // epilogue threads
+// hand-off barrier between the epilogue and the MMA warp (hardware named barrier:
+// the 256 epilogue threads and the 32 threads of the MMA warp)
+constexpr int kHand = 5, kHandCount = kEpi + 32;
 // shared memory map (offsets from a 1024-byte aligned base); 128-byte swizzled
 // fp16 tiles are stored as 64-column halves of [64 rows][128 bytes]
 constexpr uint32_t ST_QW = 0;        // [Q; W] K-major: half h at h * 16384 (Q rows, then W rows)
@@ -281,11 +287,68 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       for (int n = (issued >= 2 ? issued - 2 : 0); n < issued; ++n)
         mbar_wait(&bar[B_FULL0 + (n & 1)], (n >> 1) & 1, nullptr, 0, 1u << 20);
     }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    // The whole warp takes part in the epilogue's hand-off barriers, which also
+    // carry the vote on giving up; lane 0 issues the products right after each
+    // (completion through tcgen05.commit on an mbarrier; a commit covers all
+    // earlier products of the thread).
+    const uint32_t id_qw = idesc_f16(128, 64, false, true);
+    const uint32_t id_a = idesc_f16(128, 64, false, true);
+    const uint32_t id_k = idesc_f16(128, 64, true, true);
+    uint32_t qp_phases = 0;  // commits to B_QP so far (lane 0)
+    bool quit = named_barrier_or(kHand, kHandCount, false);  // the initial state is stored
+    for (int n = 0; n < Nc && !quit; ++n) {
+      const int s = n & 1;
+      const uint32_t st = sbase + s * STAGE_BYTES;
+      bool ok = true;
+      // [O_q; P] = [Q; W] S (K = d_k = 128: two 64-column halves of 4 steps), once
+      // the stage has landed.  (A test of the bounded waits withholds the first
+      // products: the epilogue's wait for them then expires and the CTA leaves
+      // through the abort path.)
+      if (lane == 0 && !(n == 0 && fault == kFaultScanState)) {
+        ok = wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 102, abort_flag, spin);
+        if (ok) {
+          tc_fence_after();
+          for (int k16 = 0; k16 < 8; ++k16) {
+            const uint32_t aoff = (uint32_t)(k16 >> 2) * 16384u + (uint32_t)(k16 & 3) * 32u;
+            mma_bf16(tmem + tm_qp(n), sw128_desc(st + ST_QW + aoff, 16, 1024),
+                     sw128_desc(sbase + OFF_SB + k16 * 2048, 8192, 1024), id_qw, k16 > 0);
+          }
+          mma_commit(&bar[B_QP]);
+          ++qp_phases;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (named_barrier_or(kHand, kHandCount, !ok)) break;  // U~ and U~s are stored
+      // DS = K^T U~s (K = 64 tokens) first: the state update waits for it; then
+      // O_a = A_qk U~, which runs while the state is updated
+      if (lane == 0) {
+        tc_fence_after();
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_bf16(tmem + TM_DS, sw128_desc(st + ST_K + k16 * 2048, 8192, 1024),
+                   sw128_desc(sbase + OFF_US + k16 * 2048, 8192, 1024), id_k, k16 > 0);
+        mma_commit(&bar[B_DS]);
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_bf16(tmem + TM_OA, sw128_desc(st + ST_A + k16 * 32, 16, 1024),
+                   sw128_desc(sbase + OFF_UT + k16 * 2048, 8192, 1024), id_a, k16 > 0);
+        mma_commit(&bar[B_OA]);
+        mma_commit(&bar[B_EMPTY0 + s]);  // the stage's operands have been read
+      }
+      __syncwarp();
+      quit = named_barrier_or(kHand, kHandCount, false);  // the new state is stored
+    }
+    // drain: nothing of ours may still run on the tensor cores at teardown
+    if (lane == 0) {
+      mma_commit(&bar[B_QP]);
+      mbar_wait(&bar[B_QP], qp_phases & 1, nullptr, 0, 1u << 20);
+    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = tid - 32;                       // 0..255
+    const int e = tid - 64;                       // 0..255
     const int row = 32 * (warp & 3) + lane;       // TMEM lane = d_k row of the state
-    const int half = (warp - 1) >> 2;             // columns 32 half .. 32 half + 31
+    const int half = (warp - 2) >> 2;             // columns 32 half .. 32 half + 31
     const int cb = 32 * half;
     const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)cb;
     const bool p_rows = row >= 64;                // lanes 64-127: rows of P (token row - 64)
@@ -303,7 +366,7 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
     for (int n = e; n < Nc; n += kEpi) mx = fmaxf(mx, Sg[(size_t)n * kScal + kScMaxU]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    if (lane == 0) red[warp - 1] = mx;
+    if (lane == 0) red[warp - 2] = mx;
     named_barrier(1, kEpi);
     mx = red[0];
 #pragma unroll
@@ -316,48 +379,9 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       S[c] *= sigma;
       range = fmaxf(range, fabsf(S[c]));
     }
-    // One epilogue thread issues every product of the CTA (completion through
-    // tcgen05.commit on an mbarrier; a commit covers all earlier products of the
-    // thread).  It is lane 0 of a P-row warp: an issue that waits for the tensor
-    // pipe then only holds up a warp that waits for those products anyway.
-    const bool issuer = tid == 64;
-    const uint32_t id_qw = idesc_f16(128, 64, false, true);
-    const uint32_t id_a = idesc_f16(128, 64, false, true);
-    const uint32_t id_k = idesc_f16(128, 64, true, true);
-    uint32_t qp_phases = 0;  // commits to B_QP so far (issuer)
-    // [O_q; P] = [Q; W] S of chunk m (K = d_k = 128: two 64-column halves of 4
-    // steps), once its stage has landed; the state is in shared memory
-    auto issue_qw = [&](int m) -> bool {
-      const uint32_t st = sbase + (m & 1) * STAGE_BYTES;
-      if (!wait_or_abort(&bar[B_FULL0 + (m & 1)], (m >> 1) & 1, status, 102, abort_flag, spin))
-        return false;
-      tc_fence_after();
-      for (int k16 = 0; k16 < 8; ++k16) {
-        const uint32_t aoff = (uint32_t)(k16 >> 2) * 16384u + (uint32_t)(k16 & 3) * 32u;
-        mma_bf16(tmem + tm_qp(m), sw128_desc(st + ST_QW + aoff, 16, 1024),
-                 sw128_desc(sbase + OFF_SB + k16 * 2048, 8192, 1024), id_qw, k16 > 0);
-      }
-      mma_commit(&bar[B_QP]);
-      ++qp_phases;
-      return true;
-    };
-    // O_a = A_qk U~ of chunk m (K = 64 tokens), then the stage's operands are read
-    auto issue_oa = [&](int m) {
-      const uint32_t st = sbase + (m & 1) * STAGE_BYTES;
-      for (int k16 = 0; k16 < 4; ++k16)
-        mma_bf16(tmem + TM_OA, sw128_desc(st + ST_A + k16 * 32, 16, 1024),
-                 sw128_desc(sbase + OFF_UT + k16 * 2048, 8192, 1024), id_a,
-                 k16 > 0);
-      mma_commit(&bar[B_OA]);
-      mma_commit(&bar[B_EMPTY0 + (m & 1)]);
-    };
-
     store_half_row_f16(sm + OFF_SB, row, 4 * half, S);
     fence_proxy_async_smem();
-    named_barrier(1, kEpi);
-    // (a test of the bounded waits withholds these first products: every epilogue
-    // thread's wait for them then expires and the CTA leaves through the abort path)
-    if (issuer && fault != kFaultScanState && Nc > 0 && !issue_qw(0)) *abort_flag = 1;
+    named_barrier_or(kHand, kHandCount, false);  // to the MMA warp: the state is stored
 
     // NORM: the rows' sums of squares, this CTA's [2 chunks][64][2] and the peer's
     // [4 chunks][64]; the rows of the previous chunk and their gate z
@@ -467,20 +491,9 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      if (named_barrier_or(1, kEpi, !ok || *abort_flag)) {
+      if (named_barrier_or(kHand, kHandCount, !ok || *abort_flag)) {  // to the MMA warp
         *abort_flag = 1;
         break;
-      }
-      // DS = K^T U~s (K = 64 tokens) first: the state update waits for it; then
-      // O_a, which runs while the state is updated
-      if (issuer) {
-        tc_fence_after();
-        const uint32_t stb = sbase + s * STAGE_BYTES;
-        for (int k16 = 0; k16 < 4; ++k16)
-          mma_bf16(tmem + TM_DS, sw128_desc(stb + ST_K + k16 * 2048, 8192, 1024),
-                   sw128_desc(sbase + OFF_US + k16 * 2048, 8192, 1024), id_k, k16 > 0);
-        mma_commit(&bar[B_DS]);
-        issue_oa(n);
       }
       // NORM: the gate of the previous chunk's rows has landed before the barrier
       // below, after which the P-row threads read it
@@ -502,16 +515,11 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       store_half_row_f16(sm + OFF_SB, row, 4 * half, S);
       fence_proxy_async_smem();
       tc_fence_before();
-      if (named_barrier_or(1, kEpi, !ok || *abort_flag)) {
+      if (named_barrier_or(kHand, kHandCount, !ok || *abort_flag)) {  // to the MMA warp
         *abort_flag = 1;
         break;
       }
-      // the next chunk's [Q; W] S
-      if (issuer) {
-        tc_fence_after();
-        if (n + 1 < Nc && !issue_qw(n + 1)) *abort_flag = 1;
-        mbar_arrive(&bar[B_EMPTY0 + s]);  // U and the factors of the stage are read
-      }
+      if (e == 0) mbar_arrive(&bar[B_EMPTY0 + s]);  // U and the factors of the stage are read
       // NORM: the P-row threads normalise and store their part of the previous
       // chunk's output rows, then release the row buffer to the output-row threads
       // (barrier 4: 128 arrive here, 128 wait before overwriting it)
@@ -572,10 +580,6 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
           store_row<TO>(dst, OA);
         }
       }
-    }
-    if (issuer) {  // nothing of ours may still run on the tensor cores at teardown
-      mma_commit(&bar[B_QP]);
-      mbar_wait(&bar[B_QP], qp_phases & 1, nullptr, 0, 1u << 20);
     }
     // NORM: the last chunk's rows, by the P-row threads once the output-row threads'
     // buffers and gate copies are complete (every epilogue thread gets here: the
