@@ -314,6 +314,7 @@ def measure_e2e(G, x, w, dev, stream, args, world):
                              host["A_log"], host["dt_bias"], host["h0"], o=o_h, ht=ht_h,
                              dev_workspace=dws, stream=stream, sync=False)
 
+    piece = max(64, (((w.T + 7) // 8 + 63) // 64) * 64)
     steps = max(3, min(args.steps, 20))
     total_ms, _ = time_steps(step, steps, 2, stream, sync_group=world > 1)
     ms_step = max_over_ranks(total_ms, dev) / steps
@@ -321,7 +322,8 @@ def measure_e2e(G, x, w, dev, stream, args, world):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms_step, 4), "steps": steps,
             "path": "pinned host -> gdn_chunk_fwd_host (C ABI; copies in, kernels and copies "
-                    "out pipelined over pieces of 1024 tokens) -> pinned host"}
+                    f"out pipelined over pieces of {piece} tokens, the default T/8 in whole "
+                    "chunks) -> pinned host"}
 
 
 def measure_prefill(G, name, dev, stream, pk, args):
