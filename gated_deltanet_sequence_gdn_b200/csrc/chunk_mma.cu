@@ -4,7 +4,10 @@
 //  the prep, parallel over the whole sequence:
 //    GDN   : wy_prep_tc_kernel (prep_tc.cu, tcgen05), one CTA per (chunk, key
 //            head) serving the value heads of its GQA group;
-//    GDN-2 : wy_prep2_kernel (this file), one CTA per (chunk, value head).
+//    GDN-2 : wy_prep2_kernel (this file), one CTA per (chunk, value head): TMA
+//            tile loads, the element-wise diagonal blocks and the 16-row
+//            off-diagonal blocks (warp-level mma.sync, below tcgen05's minimum
+//            M of 64), and W, U as tcgen05 products with TMEM accumulators.
 //    Both form the in-chunk prefix sums G_r of the log-decays, the strictly
 //    lower L = diag(beta) (K^ K^^T o Gamma), X = (I + L)^-1 by blocked forward
 //    substitution in fp32, W = X diag(beta gamma) K^, U = X diag(beta) V and
@@ -20,8 +23,8 @@
 // Gamma_rj = exp(G_r - G_j) only for j <= r, so every exponent is <= 0.
 //
 // Precision: fp32 accumulation and state.  The prep's products take bf16
-// operands (the inputs are bf16; X diag(beta) is carried as bf16 hi + lo, one
-// mma per part, and U is stored in fp32).  The scan's products take fp16
+// operands (the inputs are bf16; X (diag(beta)) is carried as bf16 hi + lo, one
+// product per part, and U is stored in fp32).  The scan's products take fp16
 // operands (11 significant bits): W, A_qk, the state, U~ and U~ diag(fs), and
 // the raw Q / K rows.  fp16 has a narrow range, so every fp16 operand is kept in
 // range by an exact power-of-2 scale folded into a factor applied in fp32:
