@@ -11,7 +11,8 @@
 // the precision design and the range scale sigma.
 //
 // Warp roles (320 threads):
-//   warp 0      TMA producer: every tile of chunk n into stage n % 2 (10 bulk copies)
+//   warp 0      TMA producer: every tile of chunk n into stage n % 2 (10 bulk copies,
+//               the [Q; W] tiles and the rest on separate barriers)
 //               (the whole warp also allocates and releases the TMEM)
 //   warp 1      tcgen05.mma issue (lane 0)
 //   warps 2-9   epilogue, two warps per TMEM lane quarter (warps w and w + 4 take
@@ -67,7 +68,10 @@ constexpr uint32_t ST_A = 49152;     // A_qk [64][64]
 constexpr uint32_t ST_U = 57344;     // U (fp32) columns c0 .. c0 + 63: two [64][32] boxes
 constexpr uint32_t ST_SC = 73728;    // per-chunk factors (kScal floats)
 constexpr uint32_t STAGE_BYTES = 75776;
-constexpr uint32_t TX_BYTES = 32768 + 16384 + 8192 + 16384 + kScal * 4;
+// A stage fills in two parts with their own barriers: [Q; W], read by the first
+// products only, and the rest (K, A_qk, U, factors)
+constexpr uint32_t TXQ_BYTES = 32768;
+constexpr uint32_t TX_BYTES = 16384 + 8192 + 16384 + kScal * 4;
 constexpr uint32_t OFF_SB = 2 * STAGE_BYTES;  // state (scaled) fp16, MN-major B: [128][64]
 constexpr uint32_t OFF_UT = OFF_SB + 16384;   // U~ fp16 [64][64]
 constexpr uint32_t OFF_US = OFF_UT + 8192;    // U~s fp16 [64][64]
@@ -98,6 +102,7 @@ __device__ __forceinline__ uint32_t tm_qp(int n) { return (n & 1) ? TM_QP1 : TM_
 // barrier indices
 enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_QP, B_DS, B_OA,
        B_PX0, B_PX1, B_PX2, B_PX3,  // NORM: the peer's row sums of a chunk have arrived
+       B_FULLQ0, B_FULLQ1, B_EMPTYQ0, B_EMPTYQ1,  // the [Q; W] part of a stage
        B_COUNT };
 static_assert(B_COUNT * 8 + 8 <= 128, "barrier area");
 
@@ -256,23 +261,35 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int issued = 0;  // stages armed so far
+      // The [Q; W] part of chunk n's stage is loaded as soon as the first products
+      // of chunk n - 2 have read it, the rest once all of chunk n - 2 is done, so
+      // the tiles needed first have about two chunk steps to land.
+      int issued_q = 0, issued = 0;  // parts armed so far
       for (int n = 0; n < Nc; ++n) {
         const int s = n & 1;
-        if (n >= 2 && !wait_or_abort(&bar[B_EMPTY0 + s], ((n >> 1) - 1) & 1, status, 101,
+        if (n >= 2 && !wait_or_abort(&bar[B_EMPTYQ0 + s], ((n >> 1) - 1) & 1, status, 103,
                                      abort_flag, spin)) {
           *abort_flag = 1;
           break;
         }
         if (*abort_flag) break;
         uint8_t* st = sm + s * STAGE_BYTES;
+        const int rq = khead * Tp + (cb + n) * kC, rw = wsh * Tp + (cb + n) * kC;
+        uint64_t* fullq = &bar[B_FULLQ0 + s];
+        mbar_arrive_expect_tx(fullq, TXQ_BYTES);
+        tma_load_2d(st + ST_QW + 0, &maps.q, fullq, 0, rq);
+        tma_load_2d(st + ST_QW + 16384, &maps.q, fullq, 64, rq);
+        tma_load_2d(st + ST_QW + 8192, &maps.w, fullq, 0, rw);
+        tma_load_2d(st + ST_QW + 24576, &maps.w, fullq, 64, rw);
+        issued_q = n + 1;
+        if (n >= 2 && !wait_or_abort(&bar[B_EMPTY0 + s], ((n >> 1) - 1) & 1, status, 101,
+                                     abort_flag, spin)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
         uint64_t* full = &bar[B_FULL0 + s];
         mbar_arrive_expect_tx(full, TX_BYTES);
-        const int rq = khead * Tp + (cb + n) * kC, rw = wsh * Tp + (cb + n) * kC;
-        tma_load_2d(st + ST_QW + 0, &maps.q, full, 0, rq);
-        tma_load_2d(st + ST_QW + 16384, &maps.q, full, 64, rq);
-        tma_load_2d(st + ST_QW + 8192, &maps.w, full, 0, rw);
-        tma_load_2d(st + ST_QW + 24576, &maps.w, full, 64, rw);
         tma_load_2d(st + ST_K + 0, &maps.k, full, 0, rq);
         tma_load_2d(st + ST_K + 8192, &maps.k, full, 64, rq);
         tma_load_2d(st + ST_A, &maps.a, full, 0, rw);
@@ -281,9 +298,11 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
         bulk_load(st + ST_SC, Sg + (size_t)n * kScal, kScal * 4, full);
         issued = n + 1;
       }
-      // drain: every stage armed must have landed before the CTA may exit.  Stage n
-      // was armed only after stage n - 2 of the same slot had been consumed, so only
-      // the last two armed stages can still be in flight.
+      // drain: every part armed must have landed before the CTA may exit.  A part
+      // of chunk n was armed only after the same part of chunk n - 2 had been
+      // consumed, so only the last two armed of each kind can still be in flight.
+      for (int n = (issued_q >= 2 ? issued_q - 2 : 0); n < issued_q; ++n)
+        mbar_wait(&bar[B_FULLQ0 + (n & 1)], (n >> 1) & 1, nullptr, 0, 1u << 20);
       for (int n = (issued >= 2 ? issued - 2 : 0); n < issued; ++n)
         mbar_wait(&bar[B_FULL0 + (n & 1)], (n >> 1) & 1, nullptr, 0, 1u << 20);
     }
@@ -303,11 +322,11 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       const uint32_t st = sbase + s * STAGE_BYTES;
       bool ok = true;
       // [O_q; P] = [Q; W] S (K = d_k = 128: two 64-column halves of 4 steps), once
-      // the stage has landed.  (A test of the bounded waits withholds the first
-      // products: the epilogue's wait for them then expires and the CTA leaves
-      // through the abort path.)
+      // the stage's [Q; W] part has landed.  (A test of the bounded waits withholds
+      // the first products: the epilogue's wait for them then expires and the CTA
+      // leaves through the abort path.)
       if (lane == 0 && !(n == 0 && fault == kFaultScanState)) {
-        ok = wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 102, abort_flag, spin);
+        ok = wait_or_abort(&bar[B_FULLQ0 + s], (n >> 1) & 1, status, 102, abort_flag, spin);
         if (ok) {
           tc_fence_after();
           for (int k16 = 0; k16 < 8; ++k16) {
@@ -316,9 +335,14 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
                      sw128_desc(sbase + OFF_SB + k16 * 2048, 8192, 1024), id_qw, k16 > 0);
           }
           mma_commit(&bar[B_QP]);
+          mma_commit(&bar[B_EMPTYQ0 + s]);  // the stage's [Q; W] part has been read
           ++qp_phases;
         }
       }
+      // the rest of the stage (K and A_qk for the next products), waited for while
+      // the epilogue forms U~, which needs the same part
+      if (lane == 0)
+        ok = ok && wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 104, abort_flag, spin);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (named_barrier_or(kHand, kHandCount, !ok)) break;  // U~ and U~s are stored
       // DS = K^T U~s (K = 64 tokens) first: the state update waits for it; then
@@ -449,24 +473,35 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
       const float* sc = reinterpret_cast<const float*>(st + ST_SC);
       // an expired wait is decided on at the next barrier, by a vote of all epilogue
       // threads (no thread is left at a barrier; what is computed meanwhile is dropped)
-      bool ok = wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 105, abort_flag, spin) &&
-                wait_or_abort(&bar[B_QP], n & 1, status, 106, abort_flag, spin);
+      bool ok = wait_or_abort(&bar[B_FULL0 + s], (n >> 1) & 1, status, 105, abort_flag, spin);
+      // what does not depend on the products is read before waiting for them: the
+      // P-row threads' U row (sigma U) and factor, the output-row threads' factor
+      float P[32], fs = 0.f, fo = 0.f;
+      if (p_rows) {
+        const int r = row - 64;
+        fs = sc[kC + r];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {  // U box `half` holds columns cb .. cb + 31
+          const float4 u = *reinterpret_cast<const float4*>(st + ST_U + half * 8192 + swz(r, ch));
+          P[4 * ch + 0] = sigma * u.x;
+          P[4 * ch + 1] = sigma * u.y;
+          P[4 * ch + 2] = sigma * u.z;
+          P[4 * ch + 3] = sigma * u.w;
+        }
+      } else {
+        fo = sc[row];  // (O_q of the row is read with O_a, in the output step)
+      }
+      ok = ok && wait_or_abort(&bar[B_QP], n & 1, status, 106, abort_flag, spin);
       tc_fence_after();
-      float fo = 0.f;
       if (p_rows) {
         // U~ = sigma U - P and U~s = U~ fs for token r and this thread's 32 columns,
         // written as fp16 operand rows
         const int r = row - 64;
-        const float fs = sc[kC + r];
-        float P[32];
-        tmem_ld32(tl + tm_qp(n), P);
+        {
+          float Pm[32];
+          tmem_ld32(tl + tm_qp(n), Pm);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {  // U box `half` holds columns cb .. cb + 31
-          const float4 u = *reinterpret_cast<const float4*>(st + ST_U + half * 8192 + swz(r, ch));
-          P[4 * ch + 0] = fmaf(sigma, u.x, -P[4 * ch + 0]);
-          P[4 * ch + 1] = fmaf(sigma, u.y, -P[4 * ch + 1]);
-          P[4 * ch + 2] = fmaf(sigma, u.z, -P[4 * ch + 2]);
-          P[4 * ch + 3] = fmaf(sigma, u.w, -P[4 * ch + 3]);
+          for (int c = 0; c < 32; ++c) P[c] -= Pm[c];
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -484,10 +519,6 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
           *reinterpret_cast<uint4*>(sm + OFF_UT + off) = pu;
           *reinterpret_cast<uint4*>(sm + OFF_US + off) = ps;
         }
-#pragma unroll
-        for (int c = 0; c < 32; ++c) range = fmaxf(range, fabsf(P[c]));
-      } else {
-        fo = sc[row];  // (O_q of the row is read with O_a, in the output step)
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -495,22 +526,24 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
         *abort_flag = 1;
         break;
       }
+      // the fp16 range of U~, taken while the MMA warp issues the products
+      if (p_rows) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) range = fmaxf(range, fabsf(P[c]));
+      }
       // NORM: the gate of the previous chunk's rows has landed before the barrier
       // below, after which the P-row threads read it
       if (NORM && !p_rows) asm volatile("cp.async.wait_all;" ::: "memory");
 
       // the state update first: it is what the next chunk waits for
+      const float gc = sc[kScGC + row];
       ok = wait_or_abort(&bar[B_DS], n & 1, status, 107, abort_flag, spin);
       tc_fence_after();
       {
         float D[32];
         tmem_ld32(tl + TM_DS, D);
-        const float gc = sc[kScGC + row];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          S[c] = fmaf(gc, S[c], D[c]);
-          range = fmaxf(range, fabsf(S[c]));
-        }
+        for (int c = 0; c < 32; ++c) S[c] = fmaf(gc, S[c], D[c]);
       }
       store_half_row_f16(sm + OFF_SB, row, 4 * half, S);
       fence_proxy_async_smem();
@@ -519,6 +552,8 @@ state_scan_tc_kernel(const __grid_constant__ ScanMaps maps, const uint8_t* __res
         *abort_flag = 1;
         break;
       }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) range = fmaxf(range, fabsf(S[c]));
       if (e == 0) mbar_arrive(&bar[B_EMPTY0 + s]);  // U and the factors of the stage are read
       // NORM: the P-row threads normalise and store their part of the previous
       // chunk's output rows, then release the row buffer to the output-row threads
