@@ -473,7 +473,8 @@ int gdn_check_status(gdn_stream_t stream);
  * test can check that the kernel returns and gdn_check_status reports
  * GDN_ERR_TIMEOUT:
  *   site 0: no fault (the default);
- *   site 1: the state scan withholds the first state hand-off to its MMA issue;
+ *   site 1: the state scan issues no first products, so its epilogue's wait for
+ *           them expires;
  *   site 2: the WY prep withholds its K / Q tile loads.
  *   spin_limit: polls before a wait gives up, for every bounded wait of those
  *   kernels (0 = the default, 2^24).  The setting is process-wide and stays
